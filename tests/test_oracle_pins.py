@@ -1,0 +1,289 @@
+"""Pins of the fp64 oracle to things other than itself.
+
+Each test checks the oracle against a closed form, a library routine, a
+special case with a textbook answer, an invariant, or an independent brute
+force; the pages ("STILL: Selecting Tokens for Intra-Layer Hybrid Attention to
+Linearize LLMs": [p1] jsqmd.com "Self-Saliency Score", "NP-Map",
+"Chunk-Wise"; [p4] atlas.scime.ai "Approach") print no worked example.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.special as sps
+import torch
+
+from oracle import brute
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rand(rng, *shape, scale=1.0):
+    return rng.standard_normal(shape) * scale
+
+
+def _problem(rng, B=1, H=2, Hkv=1, N=40, d=8, D=6, spread=1.5):
+    q = _rand(rng, B, H, N, d) * np.exp(rng.normal(0, 0.5, (B, H, N, 1))) * spread
+    k = _rand(rng, B, Hkv, N, d) * np.exp(rng.normal(0, 0.5, (B, Hkv, N, 1))) * spread
+    v = _rand(rng, B, Hkv, N, d)
+    wq = _rand(rng, H, d, D, scale=1 / math.sqrt(d))
+    wk = _rand(rng, Hkv, d, D, scale=1 / math.sqrt(d))
+    return q, k, v, wq, wk
+
+
+# ---------------------------------------------------------------- saliency
+
+@pytest.mark.parametrize("w", [1, 4, 8, 64])
+def test_saliency_equals_closed_form(oracle_mod, w):
+    """KL(p'||p) summed term by term equals -ln(1-p_ii) = softplus(s_ii - LSE_{j!=i} s_ij)."""
+    rng = np.random.default_rng(1)
+    q, k, *_ = _problem(rng, H=3, Hkv=1, N=70, d=16)
+    dims = oracle_mod.Dims(B=1, H=3, Hkv=1, N=70, d=16, D=4, w=w, C=w, k=0 if w == 0 else 1)
+    sigma, r = oracle_mod.saliency(dims, q, k)
+    tau = 1 / math.sqrt(16)
+    for h in range(3):
+        for i in range(70):
+            lo = max(0, i - w + 1)
+            s = tau * (k[0, 0, lo:i + 1] @ q[0, h, i])
+            if len(s) == 1:
+                assert sigma[0, h, i] == math.inf
+                continue
+            closed = np.logaddexp(0.0, s[-1] - sps.logsumexp(s[:-1]))
+            assert sigma[0, h, i] == pytest.approx(closed, rel=1e-11, abs=1e-13)
+    assert np.allclose(r[0, 0], sigma[0].mean(0))
+
+
+def test_saliency_zero_query(oracle_mod):
+    """q = 0: every logit is 0, so p_ii = 1/n and sigma = ln(n/(n-1)) with n the band size."""
+    rng = np.random.default_rng(2)
+    N, w = 50, 16
+    k = _rand(rng, 1, 1, N, 8)
+    q = np.zeros((1, 1, N, 8))
+    sigma, _ = oracle_mod.saliency(oracle_mod.Dims(1, 1, 1, N, 8, 4, w, 16, 2), q, k)
+    for i in range(N):
+        n = min(w, i + 1)
+        want = math.inf if n == 1 else math.log(n / (n - 1))
+        assert sigma[0, 0, i] == pytest.approx(want, rel=1e-13)
+
+
+def test_saliency_gqa_identical_heads(oracle_mod):
+    """G identical query heads: the group score equals the single-head score."""
+    rng = np.random.default_rng(3)
+    q1, k, *_ = _problem(rng, H=1, Hkv=1, N=45, d=8)
+    q4 = np.repeat(q1, 4, axis=1)
+    s1, r1 = oracle_mod.saliency(oracle_mod.Dims(1, 1, 1, 45, 8, 4, 8, 8, 2), q1, k)
+    s4, r4 = oracle_mod.saliency(oracle_mod.Dims(1, 4, 1, 45, 8, 4, 8, 8, 2), q4, k)
+    np.testing.assert_allclose(r4, r1, rtol=1e-14)
+    np.testing.assert_allclose(r1[0, 0], s1[0, 0], rtol=0)
+
+
+def test_saliency_golden(oracle_mod):
+    """Hand-derived values (tests/golden/saliency_hand.json)."""
+    with open(os.path.join(GOLDEN, "saliency_hand.json")) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        q = np.array(c["q"], dtype=np.float64)[None, None, :, :]
+        k = np.array(c["k"], dtype=np.float64)[None, None, :, :]
+        N, d = q.shape[2], q.shape[3]
+        dims = oracle_mod.Dims(1, 1, 1, N, d, 2, c["w"], c["w"], 1, scale=c["scale"])
+        sigma, _ = oracle_mod.saliency(dims, q, k)
+        for i, want in enumerate(c["sigma"]):
+            want = math.inf if want == "inf" else want
+            assert sigma[0, 0, i] == pytest.approx(want, rel=1e-9), (c["name"], i)
+
+
+# ---------------------------------------------------------------- top-k
+
+def test_topk_matches_sort(oracle_mod):
+    """Top-k = first k of a sort by (score desc, index asc), reported ascending; ties and +inf."""
+    rng = np.random.default_rng(4)
+    B, Hkv, C, T, kk = 2, 3, 16, 5, 5
+    N = C * T + 7
+    r = rng.integers(0, 6, size=(B, Hkv, N)).astype(np.float64)   # many ties
+    r[0, 0, 3] = math.inf
+    r[1, 2, 20] = math.inf
+    r[1, 2, 21] = math.inf
+    idx = oracle_mod.topk(oracle_mod.Dims(B, 2 * Hkv, Hkv, N, 8, 8, C, C, kk), r)
+    for b in range(B):
+        for g in range(Hkv):
+            for c in range(T):
+                mem = list(range(c * C, (c + 1) * C))
+                want = sorted(sorted(mem, key=lambda j: (-r[b, g, j], j))[:kk])
+                assert list(idx[b, g, c]) == want
+
+
+def test_topk_permutation(oracle_mod):
+    """Distinct scores: permuting the scores inside a chunk permutes the kept set."""
+    rng = np.random.default_rng(5)
+    C, kk = 32, 7
+    r = rng.standard_normal((1, 1, C))
+    perm = rng.permutation(C)
+    d = oracle_mod.Dims(1, 1, 1, C, 8, 8, C, C, kk)
+    a = set(oracle_mod.topk(d, r)[0, 0, 0])
+    bset = set(oracle_mod.topk(d, r[:, :, perm])[0, 0, 0])
+    assert {int(perm[j]) for j in bset} == {int(j) for j in a}
+
+
+# ---------------------------------------------------------------- NP-Map
+
+def test_npmap_norm_and_direction(oracle_mod):
+    """||phi(x)|| = ||x||; direction = softmax(xW) normalised (scipy); W = 0 gives ||x|| 1/sqrt(D); phi(0) = 0."""
+    rng = np.random.default_rng(6)
+    x = _rand(rng, 33, 16) * np.exp(rng.normal(0, 1, (33, 1)))
+    W = _rand(rng, 16, 24, scale=0.5)
+    phi = oracle_mod.npmap(x, W)
+    np.testing.assert_allclose(np.linalg.norm(phi, axis=1), np.linalg.norm(x, axis=1), rtol=1e-13)
+    f = sps.softmax(x @ W, axis=1)
+    np.testing.assert_allclose(phi / np.linalg.norm(phi, axis=1, keepdims=True),
+                               f / np.linalg.norm(f, axis=1, keepdims=True), rtol=1e-12)
+    phi0 = oracle_mod.npmap(x, np.zeros((16, 24)))
+    np.testing.assert_allclose(phi0, np.linalg.norm(x, axis=1, keepdims=True) / math.sqrt(24) * np.ones((1, 24)),
+                               rtol=1e-13)
+    assert np.all(oracle_mod.npmap(np.zeros((2, 16)), W) == 0)
+
+
+# ---------------------------------------------------------------- routing + merge limits
+
+@pytest.mark.parametrize("B,H,Hkv,N,C,m", [(1, 2, 1, 50, 8, 1), (2, 4, 2, 37, 6, 2), (1, 3, 3, 64, 16, 1)])
+def test_all_kept_is_causal_softmax(oracle_mod, B, H, Hkv, N, C, m):
+    """k = C: every decided chunk is kept whole, so the layer is exact causal softmax attention (torch SDPA)."""
+    rng = np.random.default_rng(7)
+    q, k, v, wq, wk = _problem(rng, B, H, Hkv, N, 8, 6)
+    out = oracle_mod.prefill(oracle_mod.Dims(B, H, Hkv, N, 8, 6, m * C, C, C), q, k, v, wq, wk)
+    G = H // Hkv
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q), torch.from_numpy(np.repeat(k, G, axis=1)), torch.from_numpy(np.repeat(v, G, axis=1)),
+        is_causal=True).numpy()
+    np.testing.assert_allclose(out["o"], ref, rtol=1e-10, atol=1e-12)
+
+
+def test_no_window_is_linear_attention_closed_form(oracle_mod):
+    """w = 0, k = 0, W = 0: <phi(q),phi(k)> = ||q|| ||k||, so o_i = sum_{j<=i} ||k_j|| v_j / sum_{j<=i} ||k_j||."""
+    rng = np.random.default_rng(8)
+    B, H, Hkv, N, d, D = 1, 2, 1, 45, 8, 6
+    q, k, v, _, _ = _problem(rng, B, H, Hkv, N, d, D)
+    out = oracle_mod.prefill(oracle_mod.Dims(B, H, Hkv, N, d, D, 0, 8, 0), q, k, v,
+                             np.zeros((H, d, D)), np.zeros((Hkv, d, D)))
+    nk = np.linalg.norm(k[0, 0], axis=1)
+    want = np.cumsum(nk[:, None] * v[0, 0], axis=0) / np.cumsum(nk)[:, None]
+    for h in range(H):
+        np.testing.assert_allclose(out["o"][0, h], want, rtol=1e-12)
+
+
+def test_no_window_equals_recurrence(oracle_mod):
+    """w = 0, k = 0: the layer equals the token-by-token linear recurrence S_i = S_{i-1} + phi(k_i) v_i^T."""
+    rng = np.random.default_rng(9)
+    B, H, Hkv, N, d, D = 1, 2, 2, 41, 8, 6
+    q, k, v, wq, wk = _problem(rng, B, H, Hkv, N, d, D)
+    out = oracle_mod.prefill(oracle_mod.Dims(B, H, Hkv, N, d, D, 0, 8, 0), q, k, v, wq, wk)
+    for h in range(H):
+        pq = oracle_mod.npmap(q[0, h], wq[h])
+        pk = oracle_mod.npmap(k[0, h], wk[h])
+        S = np.zeros((D, d))
+        z = np.zeros(D)
+        for i in range(N):
+            S += np.outer(pk[i], v[0, h, i])
+            z += pk[i]
+            np.testing.assert_allclose(out["o"][0, h, i], (pq[i] @ S) / (pq[i] @ z), rtol=1e-11)
+
+
+@pytest.mark.parametrize("m,kk", [(1, 0), (1, 3), (2, 3), (1, 8)])
+def test_zero_query_routing_sets(oracle_mod, m, kk):
+    """q = 0: logits are 0 and phi(q) = 0, so o_i is the plain mean of v over Soft(i); the scores are
+    ln(n/(n-1)), so each chunk keeps its first k tokens.  Soft(i) = window [(t-m)C, i] plus the first k
+    tokens of every chunk c <= t-m-1 (chunk-granular delay)."""
+    rng = np.random.default_rng(10)
+    C, N, d = 8, 61, 8
+    k = _rand(rng, 1, 1, N, d)
+    v = _rand(rng, 1, 1, N, d)
+    q = np.zeros((1, 1, N, d))
+    out = oracle_mod.prefill(oracle_mod.Dims(1, 1, 1, N, d, 4, m * C, C, kk), q, k, v,
+                             _rand(rng, 1, d, 4), _rand(rng, 1, d, 4))
+    for i in range(N):
+        t = i // C
+        soft = set(range(max(0, (t - m) * C), i + 1))
+        for c in range(0, t - m):
+            soft |= set(range(c * C, c * C + kk))
+        want = v[0, 0, sorted(soft)].mean(0)
+        np.testing.assert_allclose(out["o"][0, 0, i], want, rtol=1e-12, atol=1e-14)
+
+
+def test_linear_state_closed_form(oracle_mod):
+    """W = 0: phi(k) = ||k|| 1/sqrt(D), so S_t = 1/sqrt(D) * sum over unkept decided tokens of ||k_j|| v_j."""
+    rng = np.random.default_rng(11)
+    C, N, d, D, kk, m = 8, 48, 8, 5, 3, 1
+    q, k, v, _, _ = _problem(rng, 1, 1, 1, N, d, D)
+    dims = oracle_mod.Dims(1, 1, 1, N, d, D, m * C, C, kk)
+    idx = oracle_mod.prefill(dims, q, k, v, np.zeros((1, d, D)), np.zeros((1, d, D)))["idx"]
+    for t in range(N // C + 1):
+        S, z = oracle_mod.linear_state(dims, k, v, np.zeros((1, d, D)), idx, 0, 0, t)
+        lin = [j for c in range(0, min(t - m, N // C)) for j in range(c * C, (c + 1) * C) if j not in idx[0, 0, c]]
+        nk = np.linalg.norm(k[0, 0, lin], axis=1) if lin else np.zeros(0)
+        wantS = np.outer(np.ones(D), (nk[:, None] * v[0, 0, lin]).sum(0)) / math.sqrt(D)
+        np.testing.assert_allclose(S, wantS, rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(z, np.full(D, nk.sum() / math.sqrt(D)), rtol=1e-12, atol=1e-14)
+
+
+# ---------------------------------------------------------------- brute force
+
+@pytest.mark.parametrize("B,H,Hkv,N,d,D,w,C,kk", [
+    (1, 2, 1, 24, 4, 3, 4, 4, 1),
+    (2, 4, 2, 29, 8, 5, 8, 4, 2),    # GQA, ragged tail, m = 2
+    (1, 1, 1, 33, 6, 4, 8, 8, 8),    # k = C
+    (1, 2, 2, 20, 4, 4, 0, 4, 0),    # no window: pure linear
+    (1, 3, 1, 40, 4, 6, 8, 8, 0),    # k = 0: chunked SWA + linear
+    (1, 2, 1, 6, 4, 3, 8, 8, 2),     # N < C
+])
+def test_brute_force_agrees(oracle_mod, B, H, Hkv, N, d, D, w, C, kk):
+    rng = np.random.default_rng(12)
+    q, k, v, wq, wk = _problem(rng, B, H, Hkv, N, d, D)
+    out = oracle_mod.prefill(oracle_mod.Dims(B, H, Hkv, N, d, D, w, C, kk), q, k, v, wq, wk)
+    o, r, sel = brute.layer(q, k, v, wq, wk, w, C, kk)
+    np.testing.assert_allclose(out["o"], o, rtol=1e-11, atol=1e-13)
+    if w > 0:
+        np.testing.assert_allclose(out["r"], r, rtol=1e-11, atol=1e-14)
+    for (b, g, c), lst in sel.items():
+        assert list(out["idx"][b, g, c]) == lst
+
+
+def test_injected_selection(oracle_mod):
+    rng = np.random.default_rng(13)
+    B, H, Hkv, N, d, D, w, C, kk = 1, 2, 1, 32, 4, 3, 8, 8, 3
+    q, k, v, wq, wk = _problem(rng, B, H, Hkv, N, d, D)
+    idx = np.stack([np.sort(rng.choice(np.arange(c * C, (c + 1) * C), kk, replace=False)) for c in range(N // C)])
+    idx = idx[None, None]
+    out = oracle_mod.prefill(oracle_mod.Dims(B, H, Hkv, N, d, D, w, C, kk), q, k, v, wq, wk, idx_in=idx)
+    o, _, _ = brute.layer(q, k, v, wq, wk, w, C, kk, idx_in=idx)
+    np.testing.assert_allclose(out["o"], o, rtol=1e-11)
+
+
+def test_rows_subset(oracle_mod):
+    rng = np.random.default_rng(14)
+    dims = oracle_mod.Dims(2, 4, 2, 40, 8, 5, 8, 8, 2)
+    q, k, v, wq, wk = _problem(rng, 2, 4, 2, 40, 8, 5)
+    full = oracle_mod.prefill(dims, q, k, v, wq, wk)["o"]
+    rows = np.array([[0, 0, 0], [1, 3, 39], [0, 2, 17], [1, 1, 8]])
+    part = oracle_mod.prefill(dims, q, k, v, wq, wk, rows=rows)["o"]
+    for b, h, i in rows:
+        np.testing.assert_array_equal(part[b, h, i], full[b, h, i])
+
+
+# ---------------------------------------------------------------- decode
+
+@pytest.mark.parametrize("w,C,kk,Hkv", [(8, 8, 2, 1), (16, 8, 3, 2), (0, 8, 0, 1), (8, 8, 8, 1), (8, 8, 0, 2)])
+def test_decode_state_machine_equals_prefill(oracle_mod, w, C, kk, Hkv):
+    """Feeding tokens one at a time through the chunk-delayed state machine gives the prefill's rows."""
+    rng = np.random.default_rng(15)
+    B, H, N, d, D = 2, 2 * Hkv, 53, 8, 5
+    q, k, v, wq, wk = _problem(rng, B, H, Hkv, N, d, D)
+    dims = oracle_mod.Dims(B, H, Hkv, N, d, D, w, C, kk)
+    full = oracle_mod.prefill(dims, q, k, v, wq, wk)
+    dec = oracle_mod.Decoder(dims, wq, wk)
+    for p in range(N):
+        o, r = dec.step(q[:, :, p], k[:, :, p], v[:, :, p])
+        np.testing.assert_allclose(o, full["o"][:, :, p], rtol=1e-11, atol=1e-13)
+        if w > 0:
+            np.testing.assert_allclose(r, full["r"][:, :, p], rtol=1e-12, atol=1e-14)
+    assert dec.pos == N
