@@ -1,0 +1,368 @@
+#!/usr/bin/env python
+"""Prefill throughput of the STILL hybrid-attention layer on B200, through the C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+One step = one still_hybrid_prefill over one batch of synthetic input: saliency,
+per-chunk top-k + gather, NP-Map of the keys, linear state, softmax/linear
+merge (every step of the layer).  Prints ONE JSON line (rank 0).
+
+* value: tokens/s of the whole job (B*N tokens per step per GPU), inputs resident
+  in HBM, L2 flushed (a 512 MiB write) before every step outside the timed
+  events; per-step CUDA events on the launching stream, max over ranks.
+* e2e: the same metric through the same call with pinned HOST buffers, the
+  host->device copies of q, k, v, Wq, Wk and the device->host copy of o inside
+  the timed region.
+* roofline: the merge kernel (dominant), algorithmic FLOPs per launch over its
+  event-timed duration, against the measured bf16 dense peak.
+* cpu_baseline: the fp64 oracle on the host cores, on a bounded sample of the
+  same workload (one (batch, KV-group) slice, a stride of its query rows),
+  scaled to the whole layer.
+* --impl reference: that oracle arm alone, as the line's value.
+Multi-GPU: independent replicas (the layer has no cross-GPU exchange), weak scaling.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from linear_attention_still_b200.synth import WORKLOADS, make_inputs  # noqa: E402
+
+DEFAULT_WORKLOAD = "llama32_1b_layer_n16k"
+METRIC = "STILL hybrid-attn prefill tokens/s per layer at 16K/64K; % of roofline"
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=100)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    p.add_argument("--cpu-seconds", type=float, default=15.0, help="target oracle time of the CPU baseline")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--e2e-steps", type=int, default=10)
+    return p.parse_args()
+
+
+# ----------------------------------------------------------------------------- algorithmic counts
+
+def soft_sizes(shape, N=None):
+    """|Soft(i)| for every query position i (same for every (b, h))."""
+    import numpy as np
+    N = shape.N if N is None else N
+    i = np.arange(N, dtype=np.int64)
+    if shape.w == 0:
+        return np.zeros(N, dtype=np.int64)
+    m = shape.w // shape.C
+    t = i // shape.C
+    lo = np.maximum(0, (t - m) * shape.C)
+    return (i - lo + 1) + shape.k * np.maximum(0, t - m)
+
+
+def merge_flops(shape):
+    """Algorithmic FLOPs of the merge kernel per launch: 4d per (query-head, softmax key) for QK^T and
+    PV, plus 2dD for phi(q) = NP-Map GEMV and 2dD + 2D for phi(q)^T S and phi(q)^T z per query-head."""
+    rows = shape.B * shape.H
+    return rows * (4 * shape.d * int(soft_sizes(shape).sum()) + shape.N * (4 * shape.d * shape.D + 2 * shape.D))
+
+
+def layer_flops(shape):
+    """Algorithmic FLOPs of one whole step (all kernels)."""
+    import numpy as np
+    N, d, D = shape.N, shape.d, shape.D
+    band = np.minimum(np.arange(N) + 1, shape.w) if shape.w > 0 else np.zeros(N)
+    sal = shape.B * shape.H * 2 * d * float(band.sum()) if shape.k > 0 else 0.0
+    phik = shape.B * shape.Hkv * N * 2 * d * D
+    lin = shape.B * shape.Hkv * N * 2 * D * d
+    return merge_flops(shape) + sal + phik + lin
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ["index", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, gpu_id: str | None):
+        self.rows = []
+        self.proc = None
+        self.gpu_id = gpu_id
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={','.join(self.FIELDS)}", "--format=csv,noheader,nounits", "-lms", "100"]
+        if self.gpu_id:
+            cmd += ["-i", self.gpu_id]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) == len(self.FIELDS):
+                self.rows.append(parts)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=5)
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[j] for r in self.rows for j in range(4) if r[5 + j].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(self.rows),
+                "power_w_max": max((float(r[3]) for r in self.rows if r[3].replace(".", "").isdigit()),
+                                   default=None)}
+
+
+# ----------------------------------------------------------------------------- CPU baseline (oracle)
+
+def oracle_sample(shape, seconds: float, nthreads: int | None = None):
+    """Time the fp64 oracle on one (batch 0, KV group 0) slice: its saliency + top-k over all N tokens, and
+    the outputs of every `stride`-th query row of its G heads; scale to the whole layer.  Returns
+    (tokens/s, seconds measured, description, threads)."""
+    import numpy as np
+
+    import oracle
+    oracle.build()
+    nth = nthreads or len(os.sched_getaffinity(0))
+    sl = shape.replace(B=1, H=shape.G, Hkv=1)
+    inp = make_inputs(shape.replace(decode_steps=0), batches=[0])
+    q = inp.q[:, :shape.G]
+    k, v = inp.k[:, :1], inp.v[:, :1]
+    wq, wk = inp.wq[:shape.G], inp.wk[:1]
+    d = oracle.Dims.of(sl)
+    t0 = time.perf_counter()
+    idx = None
+    if shape.w > 0 and shape.k > 0 and shape.T > 0:
+        _, r = oracle.saliency(d, q, k, nthreads=nth)
+        idx = oracle.topk(d, r)
+    t_sel = time.perf_counter() - t0
+    # calibrate the row stride on a coarse sample, then size the sample to the time budget
+    stride = max(1, shape.N // 64)
+    rows = np.array([(0, h, i) for h in range(shape.G) for i in range(0, shape.N, stride)], dtype=np.int32)
+    t0 = time.perf_counter()
+    oracle.prefill(d, q, k, v, wq, wk, idx_in=idx, rows=rows, nthreads=nth)
+    t_cal = time.perf_counter() - t0
+    budget = max(seconds - t_sel, 0.5)
+    new_stride = max(1, int(math.ceil(stride * t_cal / budget)))
+    if new_stride < stride:
+        stride = new_stride
+        rows = np.array([(0, h, i) for h in range(shape.G) for i in range(0, shape.N, stride)], dtype=np.int32)
+        t0 = time.perf_counter()
+        oracle.prefill(d, q, k, v, wq, wk, idx_in=idx, rows=rows, nthreads=nth)
+        t_cal = time.perf_counter() - t0
+    frac = len(rows) / (shape.G * shape.N)
+    t_slice = t_sel + t_cal / frac
+    t_layer = t_slice * shape.B * shape.Hkv
+    desc = (f"oracle fp64 on batch 0 / KV group 0 ({shape.G} heads): saliency + top-k over all {shape.N} tokens "
+            f"({t_sel:.2f} s) and every {stride}-th query row ({len(rows)} rows, {t_cal:.2f} s), scaled by "
+            f"1/{frac:.4g} rows and x{shape.B * shape.Hkv} slices")
+    return shape.B * shape.N / t_layer, t_sel + t_cal, desc, nth
+
+
+# ----------------------------------------------------------------------------- main arms
+
+def dist_setup(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def run_reference(args):
+    rank, world, _ = dist_setup(args)
+    if rank != 0:
+        return
+    shape = WORKLOADS[args.workload]
+    per_step = max(2.0, 150.0 / max(1, args.steps + args.warmup))
+    vals = []
+    desc, nth = "", 1
+    for i in range(args.warmup + args.steps):
+        v, t, desc, nth = oracle_sample(shape, per_step)
+        if i >= args.warmup:
+            vals.append(v)
+    value = statistics.median(vals) if vals else None
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(shape, args),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": nth, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_of(shape, args):
+    return {"workload": args.workload, "B": shape.B, "H": shape.H, "Hkv": shape.Hkv, "N": shape.N, "d": shape.d,
+            "D": shape.D, "w": shape.w, "C": shape.C, "k": shape.k, "global_batch": shape.B * args.gpus,
+            "seq_len": shape.N, "parallelism": f"replicas{args.gpus}", "l2": "flushed before every step"}
+
+
+def run_ours(args):
+    import numpy as np
+    import torch
+
+    rank, world, local = dist_setup(args)
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    from linear_attention_still_b200 import still
+
+    shape = WORKLOADS[args.workload]
+    tdt = torch.bfloat16 if shape.dtype == "bf16" else torch.float32
+    inp = make_inputs(shape.replace(seed=rank))
+    host = {n: torch.from_numpy(np.ascontiguousarray(getattr(inp, n)[:, :, :shape.N] if n in "qkv" else
+                                                     getattr(inp, n))).to(tdt)
+            for n in ("q", "k", "v", "wq", "wk")}
+    del inp
+    devt = {n: t.cuda() for n, t in host.items()}
+    o = torch.empty_like(devt["q"])
+    dims = still.dims_of(shape)
+    ws = torch.empty(still.still_prefill_workspace_bytes(dims), dtype=torch.uint8, device="cuda")
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(t):
+        still.still_hybrid_prefill(dims, t["q"], t["k"], t["v"], t["wq"], t["wk"], o, workspace=ws)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step(devt)
+    torch.cuda.synchronize()
+    if still.still_get_device_status() != 0:
+        raise RuntimeError("device-side check failed during warm-up")
+
+    gpu_id = None
+    try:
+        gpu_id = f"GPU-{torch.cuda.get_device_properties(local).uuid}"
+    except Exception:
+        gpu_id = None
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+    n0 = still.still_launch_count()
+    still.still_timing_read()
+    still.still_timing_enable(True)
+    for s_, e_ in evs:
+        flush.zero_()
+        s_.record(stream)
+        step(devt)
+        e_.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    still.still_timing_enable(False)
+    launches = still.still_launch_count() - n0
+    clocks = sampler.stop()
+    kern = still.still_timing_read()
+    total_ms = sum(s_.elapsed_time(e_) for s_, e_ in evs)
+    if world > 1:
+        t = torch.tensor([total_ms], device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    tokens = shape.B * shape.N
+    value = world * tokens * args.steps / (total_ms / 1e3)
+
+    # end to end through the same call with pinned host buffers
+    pinned = {n: t.pin_memory() for n, t in host.items()}
+    o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in pinned.values())
+    d2h = o_host.numel() * o_host.element_size()
+    e_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+             for _ in range(args.e2e_steps)]
+    for s_, e_ in e_evs:
+        flush.zero_()
+        s_.record(stream)
+        for n in devt:
+            devt[n].copy_(pinned[n], non_blocking=True)
+        step(devt)
+        o_host.copy_(o, non_blocking=True)
+        e_.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = sum(s_.elapsed_time(e_) for s_, e_ in e_evs)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * tokens * args.e2e_steps / (e2e_ms / 1e3)
+    status = still.still_get_device_status()
+
+    peaks = {}
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peaks = json.load(f)
+    except OSError:
+        pass
+    merge_ms, merge_n = kern["merge"]
+    achieved = merge_flops(shape) / (merge_ms / merge_n / 1e3) / 1e12 if merge_n else None
+    peak = peaks.get("bf16_tflops", 1590.0) if shape.dtype == "bf16" else None
+    roofline = {
+        "kernel": "merge", "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+        "frac": (achieved / peak) if (achieved and peak) else None,
+        "peak_source": "measured bf16_tflops" if "bf16_tflops" in peaks else "fallback 1.59 PFLOP/s",
+        "traffic": None, "flops_per_launch": merge_flops(shape), "launch_ms": merge_ms / merge_n if merge_n else None,
+    }
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": shape.dtype, "data": "synthetic", "config": config_of(shape, args),
+        "roofline": roofline,
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches, "clocks": clocks,
+        "kernel_ms_per_step": {k_: v_[0] / args.steps for k_, v_ in kern.items()},
+        "layer_tflops": layer_flops(shape) / (ms_per_step / 1e3) / 1e12, "device_status": status,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, t, desc, nth = oracle_sample(shape, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": nth, "kind": "oracle", "sample": desc}
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

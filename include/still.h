@@ -1,0 +1,206 @@
+/*
+ * still.h -- C ABI of libstill.so, the B200 (sm_100a) implementation of the
+ * STILL intra-layer hybrid attention layer.
+ *
+ * Method: "STILL: Selecting Tokens for Intra-Layer Hybrid Attention to
+ * Linearize LLMs".  Passages cited below:
+ *   [p1] jsqmd.com news article -- introduction (two branches in one layer:
+ *        selected tokens go to softmax attention, the rest to linear
+ *        attention), "Self-Saliency Score", "Norm-Preserved Feature Map
+ *        (NP-Map)", "Chunk-Wise parallel + delayed selection";
+ *   [p4] atlas.scime.ai summary -- "Approach".
+ *
+ * Conventions (all entry points):
+ *  - Every tensor argument is a caller-owned DEVICE pointer in the row-major
+ *    layout stated at the call, 16-byte aligned.  The library never allocates
+ *    device memory; scratch space is passed in by the caller.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream).  Every call is asynchronous on that stream.
+ *  - Argument errors are detected on the host before anything is launched and
+ *    returned as a still_status; nothing is launched then.  Errors found by a
+ *    kernel (an injected index outside its chunk, a decode position that does
+ *    not match the state, a bounded wait that ran out) are recorded in a
+ *    per-device error word and reported by still_get_device_status().
+ *  - Shapes: B batch, H query heads, Hkv key/value heads (H % Hkv == 0, query
+ *    head h reads KV head h / (H/Hkv)), N tokens, head dim d, NP-Map feature
+ *    width D, window w, chunk C, k tokens kept per full chunk.  The window is
+ *    a whole number of chunks, w = m*C with m >= 1, or w = 0 (no window: pure
+ *    linear attention, then k must be 0).  0 <= k <= C.  N is arbitrary; a
+ *    trailing partial chunk is never selected from.
+ *  - dtype applies to q, k, v, o, Wq, Wk; scores, features and linear states
+ *    are always fp32.
+ */
+#ifndef STILL_H
+#define STILL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define STILL_API __attribute__((visibility("default")))
+#else
+#define STILL_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    STILL_OK = 0,
+    STILL_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad shape, constraint violated */
+    STILL_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. d > 256) */
+    STILL_ERR_WORKSPACE = 3,    /* workspace or state buffer too small */
+    STILL_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
+    STILL_ERR_DEVICE_CHECK = 5, /* a kernel found bad data (see still_get_device_status) */
+    STILL_ERR_TIMEOUT = 6       /* a kernel's bounded wait ran out */
+} still_status;
+
+typedef enum { STILL_F32 = 0, STILL_BF16 = 1 } still_dtype;
+
+typedef struct {
+    int B, H, Hkv, N, d, D, w, C, k;
+    float scale;       /* logit scale tau; 0 selects 1/sqrt(d) */
+    still_dtype dtype;
+} still_dims;
+
+/* Text of a status code (static storage). */
+STILL_API const char *still_status_string(int status);
+
+/*
+ * Self-Saliency Score ([p1] "Self-Saliency Score"; [p4] "Approach").
+ * For query head h and token i, with band B(i) = [max(0, i-w+1), i] and
+ * logits s_ij = tau <q_hi, k_gj>:
+ *     sigma_hi = KL(p' || p) = -ln(1 - p_ii) = softplus(s_ii - LSE_{j in B(i), j != i} s_ij)
+ * (p: band softmax with the diagonal, p': without it); +inf when the band
+ * holds only i.  Group score r_gi = mean of sigma over the G query heads of g.
+ *   q    [B,H,N,d]   dtype
+ *   k    [B,Hkv,N,d] dtype
+ *   r_kv [B,Hkv,N]   fp32 out
+ *   r_q  [B,H,N]     fp32 out, may be NULL (per-query-head sigma)
+ * Requires w >= 1.
+ */
+STILL_API still_status still_saliency(const still_dims *dims, const void *q, const void *k, float *r_kv, float *r_q,
+                            void *stream);
+
+/*
+ * Per-chunk top-k ([p1] "Chunk-Wise": scores per chunk, kept tokens chosen in
+ * one batch; [p4] "Approach": top-scoring tokens go to softmax attention).
+ * For every full chunk c < T = floor(N/C) of every (b, g): the k positions
+ * with the largest r, ties broken by the lower position, written in
+ * ascending order.  Bit-exact given r.
+ *   r_kv [B,Hkv,N]    fp32 in
+ *   idx  [B,Hkv,T,k]  int32 out (absolute token positions)
+ */
+STILL_API still_status still_select_topk(const still_dims *dims, const float *r_kv, int32_t *idx, void *stream);
+
+/*
+ * NP-Map feature map ([p1] "Norm-Preserved Feature Map"; [p4] "Approach"):
+ *     phi(x) = ||x||_2 * f(x W) / ||f(x W)||_2,   f = softmax over the D features
+ * with one bias-free d->D map per head.
+ *   x   [B,Hx,N,d] dtype
+ *   W   [Hx,d,D]   dtype
+ *   phi [B,Hx,N,D] fp32 out
+ */
+STILL_API still_status still_npmap(int B, int Hx, int N, int d, int D, still_dtype dtype, const void *x, const void *W,
+                         float *phi, void *stream);
+
+/* Bytes of scratch still_hybrid_prefill needs for `dims` (256-byte aligned pointer). */
+STILL_API size_t still_prefill_workspace_bytes(const still_dims *dims);
+
+/* Byte offsets of the intermediate results inside the prefill workspace, for inspection. */
+typedef struct {
+    size_t r;      /* fp32  [B,Hkv,N]          group saliency scores          */
+    size_t idx;    /* int32 [B,Hkv,T,k]        kept positions per chunk        */
+    size_t khat;   /* dtype [B,Hkv,T*k,d]      kept keys, chunk order          */
+    size_t vhat;   /* dtype [B,Hkv,T*k,d]      kept values                     */
+    size_t S;      /* fp32  [B,Hkv,T+1,D,d]    linear state seen by chunk t    */
+    size_t z;      /* fp32  [B,Hkv,T+1,D]      linear normaliser seen by chunk t */
+    size_t phik;   /* fp32  [B,Hkv,N,D]        NP-Map features of the keys     */
+    size_t total;
+} still_ws_layout;
+
+STILL_API still_status still_prefill_workspace_layout(const still_dims *dims, still_ws_layout *out);
+
+/*
+ * Hybrid-attention forward of one layer (prefill), all five steps ([p1]
+ * introduction and "Chunk-Wise"; [p4] "Approach"):
+ *   1. group saliency r (skipped if idx_in is given or k == 0);
+ *   2. per-chunk top-k -> idx, and the kept K/V rows gathered into a compact
+ *      chunk-ordered cache;
+ *   3. softmax branch of query i in chunk t = floor(i/C), m = w/C:
+ *      Soft(i) = [max(0,(t-m)C), i]  U  kept rows of chunks c <= t-m-1;
+ *   4. linear branch over the other tokens of the chunks c <= t-m-1, with NP-Map
+ *      features: S_t = sum phi(k_j) v_j^T, z_t = sum phi(k_j);
+ *   5. one shared normaliser:
+ *      o_i = (sum_Soft e^{s_ij} v_j + phi(q_i)^T S_t) / (sum_Soft e^{s_ij} + phi(q_i)^T z_t).
+ *   w = 0: no softmax branch; every j <= i is linear.
+ *   q [B,H,N,d], k/v [B,Hkv,N,d], Wq [H,d,D], Wk [Hkv,d,D], o [B,H,N,d]  (dtype)
+ *   idx_in     [B,Hkv,T,k] int32 or NULL: use this selection instead of computing it
+ *              (each index must lie in its chunk; violations set the device error word
+ *              and the row is ignored)
+ *   workspace  device scratch of workspace_bytes >= still_prefill_workspace_bytes(dims)
+ *   state      NULL, or a decode state made by still_decode_init with capacity
+ *              state_capacity >= N: it is left holding the layer's cache after N tokens
+ *              (positioned at N), ready for still_decode_step.
+ */
+STILL_API still_status still_hybrid_prefill(const still_dims *dims, const void *q, const void *k, const void *v, const void *Wq,
+                                  const void *Wk, void *o, const int32_t *idx_in, void *workspace,
+                                  size_t workspace_bytes, void *state, int state_capacity, void *stream);
+
+/*
+ * Chunk-granular delayed decode ([p1] "Chunk-Wise": during decoding the
+ * selection is delayed at chunk granularity).  The state is one caller-owned
+ * device buffer holding, per (b, g): the kept K/V cache, the linear state
+ * S [D,d] and z [D], the window ring (K/V and scores of chunks t-m..t) and
+ * the position.  dims->N is ignored; `capacity` is the largest number of
+ * tokens the state can hold.
+ */
+STILL_API size_t still_decode_state_bytes(const still_dims *dims, int capacity);
+
+/* Empty state at position 0. */
+STILL_API still_status still_decode_init(const still_dims *dims, int capacity, void *state, void *stream);
+
+/*
+ * One token per sequence at position `pos` (must equal the state's position;
+ * 0 <= pos < capacity): scores it, attends over window + kept cache + linear
+ * state exactly as the prefill does for row pos, and, if pos closes chunk t
+ * (pos % C == C-1) and t-m >= 0, selects chunk t-m, appends its kept rows and
+ * folds the others into S, z.
+ *   q_t [B,H,d], k_t/v_t [B,Hkv,d], o_t [B,H,d] (dtype); Wq, Wk as for prefill.
+ */
+STILL_API still_status still_decode_step(const still_dims *dims, void *state, int capacity, int pos, const void *Wq,
+                               const void *Wk, const void *q_t, const void *k_t, const void *v_t, void *o_t,
+                               void *stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the current device's error
+ * word: STILL_OK, STILL_ERR_DEVICE_CHECK or STILL_ERR_TIMEOUT (or
+ * STILL_ERR_CUDA if the synchronisation itself failed).
+ */
+STILL_API still_status still_get_device_status(void *stream);
+
+/* Number of kernels this library has launched in this process (all devices). */
+STILL_API uint64_t still_launch_count(void);
+
+/*
+ * Per-kernel timing for benchmarks (no counterpart in the method; host-side
+ * instrumentation).  While enabled, every kernel launched by
+ * still_hybrid_prefill is bracketed by a pair of CUDA events recorded on the
+ * caller's stream (at most STILL_TIMING_MAX_LAUNCHES launches are kept; later
+ * ones are not timed).  still_timing_read synchronises those events and, for
+ * each kernel class c < n, writes the summed milliseconds to ms[c] and the
+ * number of timed launches to launches[c], then forgets them.  Classes:
+ * 0 saliency, 1 top-k + gather, 2 NP-Map, 3 linear state, 4 softmax/linear
+ * merge, 5 decode-state export.  Single-threaded use only.
+ */
+#define STILL_TIMING_MAX_LAUNCHES 4096
+#define STILL_TIMING_CLASSES 6
+STILL_API still_status still_timing_enable(int on);
+STILL_API still_status still_timing_read(double *ms, int *launches, int n);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STILL_H */

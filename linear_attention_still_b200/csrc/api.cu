@@ -1,0 +1,366 @@
+// api.cu -- the C ABI of libstill.so (declared in include/still.h): argument validation on the
+// host, workspace and state layout, and the launch sequence of each entry point.
+#include <atomic>
+#include <cmath>
+#include <mutex>
+
+#include "common.cuh"
+#include "still.h"
+#include "still_internal.h"
+
+namespace still {
+cudaError_t launch_gather(const Dims &s, const int32_t *idx, const void *k, const void *v, void *khat, void *vhat,
+                          unsigned *err, cudaStream_t st);
+bool tc_merge_supported(const Dims &s);
+cudaError_t launch_merge_tc(const Dims &s, const void *q, const void *k, const void *v, const void *Wq,
+                            const void *khat, const void *vhat, const float *S, const float *z, void *o,
+                            unsigned *err, cudaStream_t st);
+bool tc_saliency_supported(const Dims &s);
+cudaError_t launch_saliency_tc(const Dims &s, const void *q, const void *k, float *r_kv, float *r_q, unsigned *err,
+                               cudaStream_t st);
+}  // namespace still
+
+using namespace still;
+
+__device__ unsigned g_still_device_error;  // one per device (module globals are per context)
+
+namespace {
+
+std::atomic<uint64_t> g_launches{0};
+std::mutex g_err_mu;
+unsigned *g_err_ptr[128] = {nullptr};
+
+unsigned *device_error_word() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return nullptr;
+    std::lock_guard<std::mutex> lk(g_err_mu);
+    if (!g_err_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_still_device_error) != cudaSuccess) return nullptr;
+        g_err_ptr[dev] = static_cast<unsigned *>(p);
+    }
+    return g_err_ptr[dev];
+}
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+still_status check_dims(const still_dims *in, Dims *out, bool need_N = true) {
+    if (!in) return STILL_ERR_INVALID_ARG;
+    const still_dims &d = *in;
+    if (d.B < 0 || d.H < 1 || d.Hkv < 1 || (need_N && d.N < 0) || d.C < 1 || d.k < 0 || d.w < 0)
+        return STILL_ERR_INVALID_ARG;
+    if (d.H % d.Hkv != 0 || d.k > d.C || d.w % d.C != 0) return STILL_ERR_INVALID_ARG;
+    if (d.w == 0 && d.k != 0) return STILL_ERR_INVALID_ARG;
+    if (d.dtype != STILL_F32 && d.dtype != STILL_BF16) return STILL_ERR_INVALID_ARG;
+    if (d.d < 8 || d.d % 8 != 0 || d.D < 8 || d.D % 8 != 0) return STILL_ERR_INVALID_ARG;
+    if (!std::isfinite(d.scale) || d.scale < 0.f) return STILL_ERR_INVALID_ARG;
+    if (d.d > 256 || d.D > 256 || d.H / d.Hkv > 32 || d.C > 16384) return STILL_ERR_UNSUPPORTED;
+    if ((long long)d.B * d.H > 65535 || (need_N && d.N > (1 << 26))) return STILL_ERR_UNSUPPORTED;
+    Dims s{};
+    s.B = d.B;
+    s.H = d.H;
+    s.Hkv = d.Hkv;
+    s.N = need_N ? d.N : 0;
+    s.d = d.d;
+    s.D = d.D;
+    s.w = d.w;
+    s.C = d.C;
+    s.k = d.k;
+    s.scale = d.scale == 0.f ? 1.0f / std::sqrt((float)d.d) : d.scale;
+    s.bf16 = d.dtype == STILL_BF16;
+    *out = s;
+    return STILL_OK;
+}
+
+still_ws_layout ws_layout(const Dims &s) {
+    still_ws_layout L{};
+    const size_t es = s.bf16 ? 2 : 4, BK = (size_t)s.B * s.Hkv, T = (size_t)s.T();
+    size_t off = 0;
+    L.r = off;
+    off = al256(off + BK * s.N * 4);
+    L.idx = off;
+    off = al256(off + BK * T * s.k * 4);
+    L.khat = off;
+    off = al256(off + BK * T * s.k * s.d * es);
+    L.vhat = off;
+    off = al256(off + BK * T * s.k * s.d * es);
+    L.S = off;
+    off = al256(off + BK * (T + 1) * s.D * s.d * 4);
+    L.z = off;
+    off = al256(off + BK * (T + 1) * s.D * 4);
+    L.phik = off;
+    off = al256(off + BK * s.N * s.D * 4);
+    L.total = off;
+    return L;
+}
+
+inline still_status cuda_status(cudaError_t e) { return e == cudaSuccess ? STILL_OK : STILL_ERR_CUDA; }
+
+#define STILL_LAUNCH(expr)                                   \
+    do {                                                     \
+        cudaError_t e_ = (expr);                             \
+        if (e_ != cudaSuccess) return STILL_ERR_CUDA;        \
+        g_launches.fetch_add(1, std::memory_order_relaxed);  \
+    } while (0)
+
+// ---- optional per-kernel event timing (still_timing_enable / still_timing_read)
+struct TimedLaunch {
+    cudaEvent_t a, b;
+    int cls;
+};
+bool g_timing = false;
+TimedLaunch g_timed[STILL_TIMING_MAX_LAUNCHES];
+int g_ntimed = 0;
+cudaEvent_t g_ev_pool[2 * STILL_TIMING_MAX_LAUNCHES];
+int g_ev_made = 0;
+
+struct TimingScope {
+    int slot = -1;
+    cudaStream_t st;
+    TimingScope(int cls, cudaStream_t s) : st(s) {
+        if (!g_timing || g_ntimed >= STILL_TIMING_MAX_LAUNCHES) return;
+        const int i = g_ntimed;
+        for (int e = 0; e < 2; ++e)
+            if (g_ev_made <= 2 * i + e) {
+                if (cudaEventCreate(&g_ev_pool[2 * i + e]) != cudaSuccess) return;
+                ++g_ev_made;
+            }
+        g_timed[i] = {g_ev_pool[2 * i], g_ev_pool[2 * i + 1], cls};
+        if (cudaEventRecord(g_timed[i].a, st) != cudaSuccess) return;
+        slot = i;
+        ++g_ntimed;
+    }
+    ~TimingScope() {
+        if (slot >= 0) cudaEventRecord(g_timed[slot].b, st);
+    }
+};
+
+}  // namespace
+
+extern "C" {
+
+const char *still_status_string(int status) {
+    switch (status) {
+        case STILL_OK: return "ok";
+        case STILL_ERR_INVALID_ARG: return "invalid argument";
+        case STILL_ERR_UNSUPPORTED: return "unsupported shape or type";
+        case STILL_ERR_WORKSPACE: return "workspace or state buffer too small";
+        case STILL_ERR_CUDA: return "CUDA error";
+        case STILL_ERR_DEVICE_CHECK: return "device-side check failed";
+        case STILL_ERR_TIMEOUT: return "device-side wait timed out";
+        default: return "unknown status";
+    }
+}
+
+uint64_t still_launch_count(void) { return g_launches.load(); }
+
+still_status still_saliency(const still_dims *dims, const void *q, const void *k, float *r_kv, float *r_q,
+                            void *stream) {
+    Dims s;
+    still_status st = check_dims(dims, &s);
+    if (st) return st;
+    if (s.w < 1) return STILL_ERR_INVALID_ARG;
+    if ((long long)s.B * s.N == 0) return STILL_OK;
+    if (!q || !k || !r_kv || !aligned16(q) || !aligned16(k) || !aligned16(r_kv)) return STILL_ERR_INVALID_ARG;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (tc_saliency_supported(s)) {
+        unsigned *err = device_error_word();
+        STILL_LAUNCH(launch_saliency_tc(s, q, k, r_kv, r_q, err, cs));
+    } else {
+        STILL_LAUNCH(launch_saliency_generic(s, q, k, r_kv, r_q, cs));
+    }
+    return STILL_OK;
+}
+
+still_status still_select_topk(const still_dims *dims, const float *r_kv, int32_t *idx, void *stream) {
+    Dims s;
+    still_status st = check_dims(dims, &s);
+    if (st) return st;
+    if ((long long)s.B * s.T() * s.k == 0) return STILL_OK;
+    if (!r_kv || !idx || !aligned16(r_kv) || !aligned16(idx)) return STILL_ERR_INVALID_ARG;
+    STILL_LAUNCH(launch_topk_gather(s, r_kv, idx, nullptr, nullptr, nullptr, nullptr, static_cast<cudaStream_t>(stream)));
+    return STILL_OK;
+}
+
+still_status still_npmap(int B, int Hx, int N, int d, int D, still_dtype dtype, const void *x, const void *W,
+                         float *phi, void *stream) {
+    if (B < 0 || Hx < 1 || N < 0 || d < 8 || d % 8 || D < 8 || D % 8) return STILL_ERR_INVALID_ARG;
+    if (dtype != STILL_F32 && dtype != STILL_BF16) return STILL_ERR_INVALID_ARG;
+    if (d > 256 || D > 256) return STILL_ERR_UNSUPPORTED;
+    const long long rows = (long long)B * Hx * N;
+    if (rows == 0) return STILL_OK;
+    if (rows > (1ll << 31) - 4) return STILL_ERR_UNSUPPORTED;
+    if (!x || !W || !phi || !aligned16(x) || !aligned16(W) || !aligned16(phi)) return STILL_ERR_INVALID_ARG;
+    STILL_LAUNCH(launch_npmap((int)rows, Hx, N, d, D, dtype == STILL_BF16, x, W, phi, static_cast<cudaStream_t>(stream)));
+    return STILL_OK;
+}
+
+size_t still_prefill_workspace_bytes(const still_dims *dims) {
+    Dims s;
+    if (check_dims(dims, &s)) return 0;
+    return ws_layout(s).total;
+}
+
+still_status still_prefill_workspace_layout(const still_dims *dims, still_ws_layout *out) {
+    Dims s;
+    still_status st = check_dims(dims, &s);
+    if (st) return st;
+    if (!out) return STILL_ERR_INVALID_ARG;
+    *out = ws_layout(s);
+    return STILL_OK;
+}
+
+size_t still_decode_state_bytes(const still_dims *dims, int capacity) {
+    Dims s;
+    if (check_dims(dims, &s, false) || capacity < 0) return 0;
+    return decode_layout(s, capacity).total;
+}
+
+still_status still_decode_init(const still_dims *dims, int capacity, void *state, void *stream) {
+    Dims s;
+    still_status st = check_dims(dims, &s, false);
+    if (st) return st;
+    if (capacity < 0 || capacity > (1 << 26)) return STILL_ERR_INVALID_ARG;
+    if (!state || !aligned16(state)) return STILL_ERR_INVALID_ARG;
+    DecodeLayout L = decode_layout(s, capacity);
+    STILL_LAUNCH(launch_decode_init(s, static_cast<unsigned char *>(state), L, capacity,
+                                    static_cast<cudaStream_t>(stream)));
+    return STILL_OK;
+}
+
+still_status still_hybrid_prefill(const still_dims *dims, const void *q, const void *k, const void *v, const void *Wq,
+                                  const void *Wk, void *o, const int32_t *idx_in, void *workspace,
+                                  size_t workspace_bytes, void *state, int state_capacity, void *stream) {
+    Dims s;
+    still_status st = check_dims(dims, &s);
+    if (st) return st;
+    if (state && (state_capacity < s.N || !aligned16(state))) return STILL_ERR_INVALID_ARG;
+    if ((long long)s.B * s.N == 0) return STILL_OK;
+    const void *ptrs[] = {q, k, v, Wq, Wk, o, workspace};
+    for (const void *p : ptrs)
+        if (!p || !aligned16(p)) return STILL_ERR_INVALID_ARG;
+    if (idx_in && !aligned16(idx_in)) return STILL_ERR_INVALID_ARG;
+    const still_ws_layout W = ws_layout(s);
+    if (workspace_bytes < W.total) return STILL_ERR_WORKSPACE;
+    if (((uintptr_t)workspace & 255u) != 0) return STILL_ERR_INVALID_ARG;
+
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    unsigned char *ws = static_cast<unsigned char *>(workspace);
+    unsigned *err = device_error_word();
+    float *r = reinterpret_cast<float *>(ws + W.r);
+    int32_t *idx = reinterpret_cast<int32_t *>(ws + W.idx);
+    void *khat = ws + W.khat, *vhat = ws + W.vhat;
+    float *S = reinterpret_cast<float *>(ws + W.S), *z = reinterpret_cast<float *>(ws + W.z);
+    float *phik = reinterpret_cast<float *>(ws + W.phik);
+    const bool select = s.w > 0 && s.k > 0 && s.T() > 0;
+    const bool need_r = s.w > 0 && s.k > 0 && (!idx_in || state);
+
+    // 1. Self-Saliency Score per KV group
+    if (need_r) {
+        TimingScope ts(0, cs);
+        if (tc_saliency_supported(s)) STILL_LAUNCH(launch_saliency_tc(s, q, k, r, nullptr, err, cs));
+        else STILL_LAUNCH(launch_saliency_generic(s, q, k, r, nullptr, cs));
+    }
+    // 2. per-chunk top-k and gather of the kept rows
+    const int32_t *idx_used = idx;
+    if (select) {
+        TimingScope ts(1, cs);
+        if (idx_in) {
+            idx_used = idx_in;
+            STILL_LAUNCH(launch_gather(s, idx_in, k, v, khat, vhat, err, cs));
+        } else {
+            STILL_LAUNCH(launch_topk_gather(s, r, idx, k, v, khat, vhat, cs));
+        }
+    }
+    // 3./4. NP-Map of the keys and the linear state seen by every query chunk
+    {
+        TimingScope ts(2, cs);
+        STILL_LAUNCH(launch_npmap(s.B * s.Hkv * s.N, s.Hkv, s.N, s.d, s.D, s.bf16, k, Wk, phik, cs));
+    }
+    {
+        TimingScope ts(3, cs);
+        STILL_LAUNCH(launch_linear_state(s, phik, v, idx_used, S, z, err, cs));
+        g_launches.fetch_add(s.T() - s.m() > 0 ? 1 : 0);  // the delta kernel (the prefix was counted)
+    }
+    // 5. softmax branch + linear branch + merge
+    {
+    TimingScope ts(4, cs);
+    if (tc_merge_supported(s)) STILL_LAUNCH(launch_merge_tc(s, q, k, v, Wq, khat, vhat, S, z, o, err, cs));
+    else STILL_LAUNCH(launch_merge_generic(s, q, k, v, Wq, khat, vhat, S, z, phik, o, cs));
+    }
+    // hand-off to decode
+    if (state) {
+        DecodeLayout L = decode_layout(s, state_capacity);
+        TimingScope ts(5, cs);
+        STILL_LAUNCH(launch_state_export(s, static_cast<unsigned char *>(state), L, k, v, need_r ? r : nullptr, khat,
+                                         vhat, S, z, cs));
+    }
+    return STILL_OK;
+}
+
+still_status still_decode_step(const still_dims *dims, void *state, int capacity, int pos, const void *Wq,
+                               const void *Wk, const void *q_t, const void *k_t, const void *v_t, void *o_t,
+                               void *stream) {
+    Dims s;
+    still_status st = check_dims(dims, &s, false);
+    if (st) return st;
+    if (capacity < 1 || pos < 0 || pos >= capacity) return STILL_ERR_INVALID_ARG;
+    if (s.B == 0) return STILL_OK;
+    const void *ptrs[] = {state, Wq, Wk, q_t, k_t, v_t, o_t};
+    for (const void *p : ptrs)
+        if (!p || !aligned16(p)) return STILL_ERR_INVALID_ARG;
+    s.N = capacity;
+    DecodeLayout L = decode_layout(s, capacity);
+    int launches = 0;
+    cudaError_t e = launch_decode_step(s, static_cast<unsigned char *>(state), L, pos, Wq, Wk, q_t, k_t, v_t, o_t,
+                                       device_error_word(), static_cast<cudaStream_t>(stream), &launches);
+    g_launches.fetch_add(launches);
+    return cuda_status(e);
+}
+
+still_status still_timing_enable(int on) {
+    g_timing = on != 0;
+    return STILL_OK;
+}
+
+still_status still_timing_read(double *ms, int *launches, int n) {
+    if (n < 0 || (n > 0 && (!ms || !launches))) return STILL_ERR_INVALID_ARG;
+    for (int c = 0; c < n; ++c) {
+        ms[c] = 0.0;
+        launches[c] = 0;
+    }
+    still_status st = STILL_OK;
+    for (int i = 0; i < g_ntimed; ++i) {
+        float t = 0.f;
+        if (cudaEventSynchronize(g_timed[i].b) != cudaSuccess ||
+            cudaEventElapsedTime(&t, g_timed[i].a, g_timed[i].b) != cudaSuccess) {
+            st = STILL_ERR_CUDA;
+            continue;
+        }
+        const int c = g_timed[i].cls;
+        if (c < n) {
+            ms[c] += t;
+            launches[c] += 1;
+        }
+    }
+    g_ntimed = 0;
+    return st;
+}
+
+still_status still_get_device_status(void *stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return STILL_ERR_CUDA;
+    unsigned *p = device_error_word();
+    if (!p) return STILL_ERR_CUDA;
+    unsigned v = 0;
+    if (cudaMemcpy(&v, p, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return STILL_ERR_CUDA;
+    if (v) {
+        unsigned zero = 0;
+        if (cudaMemcpy(p, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return STILL_ERR_CUDA;
+    }
+    if (v & DEV_ERR_TIMEOUT) return STILL_ERR_TIMEOUT;
+    if (v) return STILL_ERR_DEVICE_CHECK;
+    return STILL_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,487 @@
+// kernels_decode.cu -- chunk-granular delayed decode ([p1] jsqmd.com "Chunk-Wise": during
+// decoding the token selection is delayed at chunk granularity) and the prefill -> decode
+// state hand-off, for "STILL: Selecting Tokens for Intra-Layer Hybrid Attention to Linearize LLMs".
+//
+// State per (b, g): kept K/V cache (chunk order), linear state S [D,d] / z [D], and a ring of
+// m+1 chunk slots holding K/V rows and scores of the chunks t-m..t still inside the window.
+// One step at position p (chunk t = p / C):
+//   append  -> ring row of p;
+//   attn    -> split-K online softmax over [kept rows 0..k(t-m)) ++ window [max(0,(t-m)C), p],
+//              plus the band statistics of the new token's Self-Saliency Score;
+//   combine -> merges the splits, adds phi(q)^T S and phi(q)^T z under one normaliser, writes o,
+//              and stores the group score of p in the ring;
+//   close   -> only when p ends chunk t and c = t-m >= 0: top-k of chunk c on the stored scores,
+//              append its kept rows, fold the others into S and z.
+#include "common.cuh"
+#include "rowops.cuh"
+#include "still_internal.h"
+#include "topk.cuh"
+
+namespace still {
+
+static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+DecodeLayout decode_layout(const Dims &s, int capacity) {
+    DecodeLayout L{};
+    const size_t es = s.bf16 ? 2 : 4, BK = (size_t)s.B * s.Hkv;
+    L.cap_chunks = capacity / s.C;
+    L.ring_rows = (s.w > 0 ? s.m() + 1 : 1) * s.C;
+    L.nsplit_max = kDecodeMaxSplits;
+    size_t off = 0;
+    L.header = off;
+    off += 256;
+    L.khat = off;
+    off = align256(off + BK * L.cap_chunks * s.k * s.d * es);
+    L.vhat = off;
+    off = align256(off + BK * L.cap_chunks * s.k * s.d * es);
+    L.S = off;
+    off = align256(off + BK * s.D * s.d * 4);
+    L.z = off;
+    off = align256(off + BK * s.D * 4);
+    L.ring_k = off;
+    off = align256(off + BK * L.ring_rows * s.d * es);
+    L.ring_v = off;
+    off = align256(off + BK * L.ring_rows * s.d * es);
+    L.ring_r = off;
+    off = align256(off + BK * L.ring_rows * 4);
+    L.part = off;
+    off = align256(off + (size_t)s.B * s.H * kDecodeMaxSplits * (s.d + 2) * 4);
+    L.band = off;
+    off = align256(off + (size_t)s.B * s.H * kDecodeMaxSplits * 3 * 4);
+    L.total = off;
+    return L;
+}
+
+namespace {
+
+struct StepGeom {
+    int pos, t, lo, nk, n, nsplit, per;
+};
+
+__device__ __forceinline__ int ring_row(const Dims &s, int j) {
+    const int slot = s.w > 0 ? (j / s.C) % (s.m() + 1) : 0;
+    return slot * s.C + j % s.C;
+}
+
+template <typename T>
+__global__ void decode_append_kernel(Dims s, DecodeLayout L, unsigned char *state, int pos, const T *__restrict__ k_t,
+                                     const T *__restrict__ v_t, unsigned *err) {
+    const int bg = blockIdx.x;
+    if (bg == 0 && threadIdx.x == 0) {
+        const DecodeHeader *hd = reinterpret_cast<const DecodeHeader *>(state + L.header);
+        if (hd->pos != pos) report(err, DEV_ERR_POSITION);
+    }
+    T *rk = reinterpret_cast<T *>(state + L.ring_k) + ((size_t)bg * L.ring_rows + ring_row(s, pos)) * s.d;
+    T *rv = reinterpret_cast<T *>(state + L.ring_v) + ((size_t)bg * L.ring_rows + ring_row(s, pos)) * s.d;
+    for (int x = threadIdx.x; x < s.d; x += blockDim.x) {
+        rk[x] = k_t[(size_t)bg * s.d + x];
+        rv[x] = v_t[(size_t)bg * s.d + x];
+    }
+}
+
+// Row of key number li of the softmax list [kept 0..nk) ++ window [lo, pos].
+template <typename T>
+__device__ __forceinline__ const T *list_row(const Dims &s, const DecodeLayout &L, const unsigned char *state, int bg,
+                                             const StepGeom &gm, int li, bool value) {
+    if (li < gm.nk) {
+        const T *base = reinterpret_cast<const T *>(state + (value ? L.vhat : L.khat));
+        return base + ((size_t)bg * L.cap_chunks * s.k + li) * s.d;
+    }
+    const int j = gm.lo + (li - gm.nk);
+    const T *base = reinterpret_cast<const T *>(state + (value ? L.ring_v : L.ring_k));
+    return base + ((size_t)bg * L.ring_rows + ring_row(s, j)) * s.d;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(128) decode_attn_kernel(Dims s, DecodeLayout L, unsigned char *state, StepGeom gm,
+                                                          const T *__restrict__ q_t) {
+    __shared__ __align__(16) float qs[4][kMaxD];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bg = blockIdx.x, split = blockIdx.y, b = bg / s.Hkv, g = bg % s.Hkv, G = s.G();
+    const int l0 = split * gm.per, l1 = min(gm.n, l0 + gm.per);
+    const int band_lo = max(0, gm.pos - s.w + 1);  // band keys [band_lo, pos-1], diagonal pos
+    float *part = reinterpret_cast<float *>(state + L.part);
+    float *band = reinterpret_cast<float *>(state + L.band);
+    for (int hh = warp; hh < G; hh += 4) {
+        const int h = g * G + hh;
+        for (int x = lane; x < s.d; x += 32) qs[warp][x] = to_f(q_t[((size_t)b * s.H + h) * s.d + x]);
+        __syncwarp();
+        float acc[kMaxD / 32];
+#pragma unroll
+        for (int u = 0; u < kMaxD / 32; ++u) acc[u] = 0.f;
+        float M = -INFINITY, Ls = 0.f, bm = -INFINITY, bl = 0.f, sdiag = -INFINITY;
+        for (int base = l0; base < l1; base += 32) {
+            const int li = base + lane;
+            float l = -INFINITY;
+            if (li < l1) {
+                l = s.scale * dot_row(qs[warp], list_row<T>(s, L, state, bg, gm, li, false), s.d);
+                if (li >= gm.nk) {
+                    const int j = gm.lo + (li - gm.nk);
+                    if (j == gm.pos) sdiag = l;
+                    else if (j >= band_lo) {
+                        if (l > bm) {
+                            bl = bl * expf(bm - l) + 1.f;
+                            bm = l;
+                        } else {
+                            bl += expf(l - bm);
+                        }
+                    }
+                }
+            }
+            float gmx = warp_max(l);
+            float nm = fmaxf(M, gmx);
+            float so = (M == -INFINITY) ? 0.f : expf(M - nm);
+            float p = li < l1 ? expf(l - nm) : 0.f;
+            Ls = Ls * so + warp_sum(p);
+#pragma unroll
+            for (int u = 0; u < kMaxD / 32; ++u) acc[u] *= so;
+            const int cnt = min(32, l1 - base);
+            for (int jj = 0; jj < cnt; ++jj) {
+                float pj = __shfl_sync(0xffffffffu, p, jj);
+                const T *vr = list_row<T>(s, L, state, bg, gm, base + jj, true);
+#pragma unroll
+                for (int u = 0; u < kMaxD / 32; ++u) {
+                    int x = lane + 32 * u;
+                    if (x < s.d) acc[u] = fmaf(pj, to_f(vr[x]), acc[u]);
+                }
+            }
+            M = nm;
+        }
+        // combine the lanes' band statistics
+        float BM = warp_max(bm);
+        float BL = warp_sum(bm == -INFINITY ? 0.f : bl * expf(bm - BM));
+        float SD = warp_max(sdiag);
+        const size_t pi = ((size_t)b * s.H + h) * kDecodeMaxSplits + split;
+        float *pp = part + pi * (s.d + 2);
+        if (lane == 0) {
+            pp[0] = M;
+            pp[1] = Ls;
+            band[pi * 3 + 0] = BM;
+            band[pi * 3 + 1] = BL;
+            band[pi * 3 + 2] = SD;
+        }
+#pragma unroll
+        for (int u = 0; u < kMaxD / 32; ++u) {
+            int x = lane + 32 * u;
+            if (x < s.d) pp[2 + x] = acc[u];
+        }
+        __syncwarp();
+    }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(128) decode_combine_kernel(Dims s, DecodeLayout L, unsigned char *state, StepGeom gm,
+                                                             const T *__restrict__ q_t, const T *__restrict__ Wq,
+                                                             const T *__restrict__ Wk, T *__restrict__ o_t) {
+    __shared__ __align__(16) float qs[4][kMaxD];
+    __shared__ __align__(16) float ps[4][kMaxDf];
+    __shared__ __align__(16) float ks[4][kMaxD];
+    __shared__ __align__(16) float pk[4][kMaxDf];
+    __shared__ float sig[32];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bg = blockIdx.x, b = bg / s.Hkv, g = bg % s.Hkv, G = s.G(), d = s.d, D = s.D;
+    const float *part = reinterpret_cast<const float *>(state + L.part);
+    const float *band = reinterpret_cast<const float *>(state + L.band);
+    const float *S = reinterpret_cast<const float *>(state + L.S) + (size_t)bg * D * d;
+    const float *z = reinterpret_cast<const float *>(state + L.z) + (size_t)bg * D;
+    for (int hh = warp; hh < G; hh += 4) {
+        const int h = g * G + hh;
+        float M = -INFINITY, Ls = 0.f, BM = -INFINITY, BL = 0.f, SD = -INFINITY;
+        for (int sp = 0; sp < gm.nsplit; ++sp) {
+            const size_t pi = ((size_t)b * s.H + h) * kDecodeMaxSplits + sp;
+            M = fmaxf(M, part[pi * (d + 2)]);
+            BM = fmaxf(BM, band[pi * 3]);
+            SD = fmaxf(SD, band[pi * 3 + 2]);
+        }
+        float acc[kMaxD / 32];
+#pragma unroll
+        for (int u = 0; u < kMaxD / 32; ++u) acc[u] = 0.f;
+        for (int sp = 0; sp < gm.nsplit; ++sp) {
+            const size_t pi = ((size_t)b * s.H + h) * kDecodeMaxSplits + sp;
+            const float *pp = part + pi * (d + 2);
+            const float ms = pp[0];
+            const float f = ms == -INFINITY ? 0.f : expf(ms - M);
+            Ls += pp[1] * f;
+#pragma unroll
+            for (int u = 0; u < kMaxD / 32; ++u) {
+                int x = lane + 32 * u;
+                if (x < d) acc[u] = fmaf(pp[2 + x], f, acc[u]);
+            }
+            const float bms = band[pi * 3];
+            if (bms != -INFINITY) BL += band[pi * 3 + 1] * expf(bms - BM);
+        }
+        // saliency of the new token for this head
+        float sigma = 0.f;
+        if (s.w > 0) {
+            const int band_lo = max(0, gm.pos - s.w + 1);
+            sigma = (band_lo == gm.pos) ? INFINITY : softplus_f(SD - (BM + logf(BL)));
+        }
+        if (lane == 0) sig[hh] = sigma;
+        // linear branch
+        for (int x = lane; x < d; x += 32) qs[warp][x] = to_f(q_t[((size_t)b * s.H + h) * d + x]);
+        __syncwarp();
+        npmap_row_warp<T>(qs[warp], Wq + (size_t)h * d * D, d, D, ps[warp], lane);
+        __syncwarp();
+        float lin[kMaxD / 32];
+#pragma unroll
+        for (int u = 0; u < kMaxD / 32; ++u) lin[u] = 0.f;
+        float lden = 0.f;
+        for (int a = 0; a < D; ++a) {
+            const float pa = ps[warp][a];
+            lden = fmaf(pa, z[a], lden);
+#pragma unroll
+            for (int u = 0; u < kMaxD / 32; ++u) {
+                int x = lane + 32 * u;
+                if (x < d) lin[u] = fmaf(pa, S[(size_t)a * d + x], lin[u]);
+            }
+        }
+        if (s.w == 0) {
+            // open chunk [tC, pos] is linear too; features computed on the fly
+            const T *rk = reinterpret_cast<const T *>(state + L.ring_k) + (size_t)bg * L.ring_rows * d;
+            const T *rv = reinterpret_cast<const T *>(state + L.ring_v) + (size_t)bg * L.ring_rows * d;
+            for (int j = gm.t * s.C; j <= gm.pos; ++j) {
+                const int rr = j % s.C;
+                for (int x = lane; x < d; x += 32) ks[warp][x] = to_f(rk[(size_t)rr * d + x]);
+                __syncwarp();
+                npmap_row_warp<T>(ks[warp], Wk + (size_t)g * d * D, d, D, pk[warp], lane);
+                __syncwarp();
+                float wpart = 0.f;
+                for (int a = lane; a < D; a += 32) wpart = fmaf(ps[warp][a], pk[warp][a], wpart);
+                const float wj = warp_sum(wpart);
+                lden += wj;
+#pragma unroll
+                for (int u = 0; u < kMaxD / 32; ++u) {
+                    int x = lane + 32 * u;
+                    if (x < d) lin[u] = fmaf(wj, to_f(rv[(size_t)rr * d + x]), lin[u]);
+                }
+                __syncwarp();
+            }
+        }
+        float Ms = M;
+        if (lden > 0.f) Ms = fmaxf(M, logf(lden));
+        const float a_soft = (M == -INFINITY) ? 0.f : expf(M - Ms);
+        const float a_lin = (Ms == -INFINITY) ? 0.f : expf(-Ms);
+        const float den = Ls * a_soft + lden * a_lin;
+        const float inv = den > 0.f ? 1.f / den : 0.f;
+        T *orow = o_t + ((size_t)b * s.H + h) * d;
+#pragma unroll
+        for (int u = 0; u < kMaxD / 32; ++u) {
+            int x = lane + 32 * u;
+            if (x < d) orow[x] = from_f<T>((acc[u] * a_soft + lin[u] * a_lin) * inv);
+        }
+        __syncwarp();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float acc = 0.f;
+        for (int hh = 0; hh < G; ++hh) acc += sig[hh];
+        float *rr = reinterpret_cast<float *>(state + L.ring_r);
+        rr[(size_t)bg * L.ring_rows + ring_row(s, gm.pos)] = s.w > 0 ? acc / (float)G : 0.f;
+        if (bg == 0) reinterpret_cast<DecodeHeader *>(state + L.header)->pos = gm.pos + 1;
+    }
+}
+
+// Decide chunk c = t-m of (b, g): top-k on its stored scores, append kept rows, fold the rest.
+// grid (B*Hkv, passes): each pass owns kFoldEnt*512 entries of S; pass 0 also appends the kept rows.
+constexpr int kFoldTok = 16;   // rows featurised per step (one per warp)
+constexpr int kFoldEnt = 32;   // S entries per thread per pass
+constexpr int kFoldThreads = 512;
+
+template <typename T>
+__global__ void __launch_bounds__(kFoldThreads) decode_close_kernel(Dims s, DecodeLayout L, unsigned char *state,
+                                                                    int c, const T *__restrict__ Wk, int P, int Pk) {
+    extern __shared__ unsigned long long csm[];
+    unsigned long long *keys = csm;                                     // P
+    uint32_t *pos = reinterpret_cast<uint32_t *>(keys + P);             // Pk
+    unsigned char *kept = reinterpret_cast<unsigned char *>(pos + Pk);  // C (rounded to 16)
+    float *xs = reinterpret_cast<float *>(kept + ((s.C + 15) & ~15));   // [kFoldTok][d]
+    float *ph = xs + kFoldTok * s.d;                                    // [kFoldTok][D]
+    float *vs = ph + kFoldTok * s.D;                                    // [kFoldTok][d]
+    const int bg = blockIdx.x, g = bg % s.Hkv, d = s.d, D = s.D;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int slot = s.w > 0 ? c % (s.m() + 1) : 0;
+    const float *rc = reinterpret_cast<const float *>(state + L.ring_r) + (size_t)bg * L.ring_rows + slot * s.C;
+    const T *rk = reinterpret_cast<const T *>(state + L.ring_k) + ((size_t)bg * L.ring_rows + slot * s.C) * d;
+    const T *rv = reinterpret_cast<const T *>(state + L.ring_v) + ((size_t)bg * L.ring_rows + slot * s.C) * d;
+    for (int j = threadIdx.x; j < s.C; j += blockDim.x) kept[j] = 0;
+    __syncthreads();
+    if (s.k > 0) {
+        block_topk(rc, s.C, s.k, keys, pos, P, Pk);  // syncs internally
+        if (blockIdx.y == 0) {
+            T *kh = reinterpret_cast<T *>(state + L.khat) + ((size_t)bg * L.cap_chunks * s.k + (size_t)c * s.k) * d;
+            T *vh = reinterpret_cast<T *>(state + L.vhat) + ((size_t)bg * L.cap_chunks * s.k + (size_t)c * s.k) * d;
+            for (int t = threadIdx.x; t < s.k * d; t += blockDim.x) {
+                const int rr = t / d, x = t % d;
+                kh[(size_t)rr * d + x] = rk[(size_t)pos[rr] * d + x];
+                vh[(size_t)rr * d + x] = rv[(size_t)pos[rr] * d + x];
+            }
+        }
+        for (int t = threadIdx.x; t < s.k; t += blockDim.x) kept[pos[t]] = 1;
+    }
+    __syncthreads();
+    // fold: S += sum_{unkept j} phi(k_j) v_j^T, z += sum phi(k_j)
+    const int Dd = D * d;
+    const int ebase = blockIdx.y * kFoldThreads * kFoldEnt;
+    float acc[kFoldEnt];
+#pragma unroll
+    for (int u = 0; u < kFoldEnt; ++u) acc[u] = 0.f;
+    float zacc = 0.f;
+    for (int jb = 0; jb < s.C; jb += kFoldTok) {
+        const int j = jb + warp;
+        if (warp < kFoldTok) {
+            float *xr = xs + warp * d;
+            for (int x = lane; x < d; x += 32) xr[x] = j < s.C ? to_f(rk[(size_t)j * d + x]) : 0.f;
+            for (int x = lane; x < d; x += 32) vs[warp * d + x] = j < s.C ? to_f(rv[(size_t)j * d + x]) : 0.f;
+            __syncwarp();
+            if (j < s.C && !kept[j]) {
+                npmap_row_warp<T>(xr, Wk + (size_t)g * d * D, d, D, ph + warp * D, lane);
+            } else {
+                for (int a = lane; a < D; a += 32) ph[warp * D + a] = 0.f;
+            }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int u = 0; u < kFoldEnt; ++u) {
+            const int e = ebase + threadIdx.x + u * kFoldThreads;
+            if (e < Dd) {
+                const int a = e / d, x = e % d;
+                float sa = acc[u];
+                for (int rr = 0; rr < kFoldTok; ++rr) sa = fmaf(ph[rr * D + a], vs[rr * d + x], sa);
+                acc[u] = sa;
+            }
+        }
+        if (blockIdx.y == 0 && threadIdx.x < D)
+            for (int rr = 0; rr < kFoldTok; ++rr) zacc += ph[rr * D + threadIdx.x];
+        __syncthreads();
+    }
+    float *S = reinterpret_cast<float *>(state + L.S) + (size_t)bg * Dd;
+    float *z = reinterpret_cast<float *>(state + L.z) + (size_t)bg * D;
+#pragma unroll
+    for (int u = 0; u < kFoldEnt; ++u) {
+        const int e = ebase + threadIdx.x + u * kFoldThreads;
+        if (e < Dd) S[e] += acc[u];
+    }
+    if (blockIdx.y == 0 && threadIdx.x < D) z[threadIdx.x] += zacc;
+}
+
+// Prefill -> decode hand-off: after N tokens the state holds chunks c <= T-m-1 decided (kept rows
+// and S_T, z_T), and the ring holds positions [max(0,(T-m)C), N) (w = 0: [TC, N)).
+template <typename T>
+__global__ void state_export_kernel(Dims s, DecodeLayout L, unsigned char *state, const T *__restrict__ k,
+                                    const T *__restrict__ v, const float *__restrict__ r, const T *__restrict__ khat,
+                                    const T *__restrict__ vhat, const float *__restrict__ Sw,
+                                    const float *__restrict__ zw) {
+    const int bg = blockIdx.x, d = s.d, D = s.D, T_ = s.T(), m = s.m();
+    const int lo = s.w > 0 ? max(0, (T_ - m) * s.C) : T_ * s.C;
+    for (int t = threadIdx.x; t < (s.N - lo) * d; t += blockDim.x) {
+        const int j = lo + t / d, x = t % d;
+        const size_t dst = ((size_t)bg * L.ring_rows + ring_row(s, j)) * d + x;
+        reinterpret_cast<T *>(state + L.ring_k)[dst] = k[((size_t)bg * s.N + j) * d + x];
+        reinterpret_cast<T *>(state + L.ring_v)[dst] = v[((size_t)bg * s.N + j) * d + x];
+    }
+    for (int j = lo + threadIdx.x; j < s.N; j += blockDim.x)
+        reinterpret_cast<float *>(state + L.ring_r)[(size_t)bg * L.ring_rows + ring_row(s, j)] =
+            r ? r[(size_t)bg * s.N + j] : 0.f;
+    const int nkept = s.w > 0 ? s.k * max(0, T_ - m) : 0;
+    for (int t = threadIdx.x; t < nkept * d; t += blockDim.x) {
+        const size_t src = (size_t)bg * T_ * s.k * d + t;
+        const size_t dst = (size_t)bg * L.cap_chunks * s.k * d + t;
+        reinterpret_cast<T *>(state + L.khat)[dst] = khat[src];
+        reinterpret_cast<T *>(state + L.vhat)[dst] = vhat[src];
+    }
+    const float *Ss = Sw + ((size_t)bg * (T_ + 1) + T_) * D * d;
+    const float *zs = zw + ((size_t)bg * (T_ + 1) + T_) * D;
+    for (int t = threadIdx.x; t < D * d; t += blockDim.x)
+        reinterpret_cast<float *>(state + L.S)[(size_t)bg * D * d + t] = Ss[t];
+    for (int t = threadIdx.x; t < D; t += blockDim.x)
+        reinterpret_cast<float *>(state + L.z)[(size_t)bg * D + t] = zs[t];
+    if (bg == 0 && threadIdx.x == 0) {
+        DecodeHeader *hd = reinterpret_cast<DecodeHeader *>(state + L.header);
+        hd->pos = s.N;
+    }
+}
+
+__global__ void decode_header_kernel(unsigned char *state, DecodeLayout L, int capacity) {
+    DecodeHeader *hd = reinterpret_cast<DecodeHeader *>(state + L.header);
+    hd->pos = 0;
+    hd->capacity = capacity;
+    hd->magic = kDecodeMagic;
+}
+
+}  // namespace
+
+cudaError_t launch_decode_init(const Dims &s, unsigned char *state, const DecodeLayout &L, int capacity,
+                               cudaStream_t st) {
+    cudaError_t e = cudaMemsetAsync(state + L.S, 0, L.ring_k - L.S, st);  // S and z
+    if (e != cudaSuccess) return e;
+    decode_header_kernel<<<1, 1, 0, st>>>(state, L, capacity);
+    return cudaGetLastError();
+}
+
+template <typename T>
+static cudaError_t decode_step_t(const Dims &s, unsigned char *state, const DecodeLayout &L, int pos, const void *Wq,
+                                 const void *Wk, const void *q_t, const void *k_t, const void *v_t, void *o_t,
+                                 unsigned *err, cudaStream_t st, int *launches) {
+    StepGeom gm{};
+    gm.pos = pos;
+    gm.t = pos / s.C;
+    const int m = s.m();
+    if (s.w > 0) {
+        gm.lo = max(0, (gm.t - m) * s.C);
+        gm.nk = s.k * max(0, gm.t - m);
+        gm.n = gm.nk + (pos - gm.lo + 1);
+    } else {
+        gm.lo = pos + 1;
+        gm.nk = 0;
+        gm.n = 0;
+    }
+    gm.nsplit = gm.n == 0 ? 0 : min(kDecodeMaxSplits, (gm.n + 255) / 256);
+    gm.per = gm.nsplit ? (gm.n + gm.nsplit - 1) / gm.nsplit : 0;
+    const int BK = s.B * s.Hkv;
+    decode_append_kernel<T><<<BK, 128, 0, st>>>(s, L, state, pos, (const T *)k_t, (const T *)v_t, err);
+    ++*launches;
+    if (gm.nsplit) {
+        decode_attn_kernel<T><<<dim3(BK, gm.nsplit), 128, 0, st>>>(s, L, state, gm, (const T *)q_t);
+        ++*launches;
+    }
+    decode_combine_kernel<T><<<BK, 128, 0, st>>>(s, L, state, gm, (const T *)q_t, (const T *)Wq, (const T *)Wk,
+                                                 (T *)o_t);
+    ++*launches;
+    if (pos % s.C == s.C - 1 && gm.t - m >= 0) {
+        const int P = pow2_ceil(s.C), Pk = pow2_ceil(s.k > 0 ? s.k : 1);
+        size_t smem = (size_t)P * 8 + (size_t)Pk * 4 + ((s.C + 15) & ~15) + (size_t)kFoldTok * (2 * s.d + s.D) * 4;
+        cudaError_t e =
+            cudaFuncSetAttribute(decode_close_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        const int passes = (s.D * s.d + kFoldThreads * kFoldEnt - 1) / (kFoldThreads * kFoldEnt);
+        decode_close_kernel<T><<<dim3(BK, passes), kFoldThreads, smem, st>>>(s, L, state, gm.t - m, (const T *)Wk, P,
+                                                                             Pk);
+        ++*launches;
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decode_step(const Dims &s, unsigned char *state, const DecodeLayout &L, int pos, const void *Wq,
+                               const void *Wk, const void *q_t, const void *k_t, const void *v_t, void *o_t,
+                               unsigned *err, cudaStream_t st, int *launches) {
+    if (s.bf16)
+        return decode_step_t<__nv_bfloat16>(s, state, L, pos, Wq, Wk, q_t, k_t, v_t, o_t, err, st, launches);
+    return decode_step_t<float>(s, state, L, pos, Wq, Wk, q_t, k_t, v_t, o_t, err, st, launches);
+}
+
+cudaError_t launch_state_export(const Dims &s, unsigned char *state, const DecodeLayout &L, const void *k,
+                                const void *v, const float *r, const void *khat, const void *vhat, const float *S,
+                                const float *z, cudaStream_t st) {
+    const int BK = s.B * s.Hkv;
+    if (BK == 0) return cudaSuccess;
+    typedef __nv_bfloat16 bf;
+    if (s.bf16)
+        state_export_kernel<bf><<<BK, 256, 0, st>>>(s, L, state, (const bf *)k, (const bf *)v, r, (const bf *)khat,
+                                                    (const bf *)vhat, S, z);
+    else
+        state_export_kernel<float><<<BK, 256, 0, st>>>(s, L, state, (const float *)k, (const float *)v, r,
+                                                       (const float *)khat, (const float *)vhat, S, z);
+    return cudaGetLastError();
+}
+
+}  // namespace still

@@ -1,0 +1,61 @@
+// still_internal.h -- launcher interface between the C-ABI layer (api.cu) and
+// the kernel translation units.  Not installed; C++ only.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace still {
+
+struct Dims {
+    int B, H, Hkv, N, d, D, w, C, k;
+    float scale;  // resolved (never 0)
+    int bf16;     // 1: q/k/v/o/W are bf16, 0: fp32
+    __host__ __device__ int G() const { return H / Hkv; }
+    __host__ __device__ int T() const { return N / C; }
+    __host__ __device__ int m() const { return w / C; }
+};
+
+// Decode state buffer layout (byte offsets from the state base pointer).
+struct DecodeLayout {
+    size_t header, khat, vhat, S, z, ring_k, ring_v, ring_r, part, band, total;
+    int cap_chunks;  // capacity / C
+    int ring_rows;   // (m+1)*C, or C when w == 0
+    int nsplit_max;
+};
+
+struct DecodeHeader {
+    long long pos;
+    int capacity;
+    int magic;
+};
+constexpr int kDecodeMagic = 0x5711D ^ 0x1234;
+constexpr int kDecodeMaxSplits = 64;
+
+DecodeLayout decode_layout(const Dims &s, int capacity);
+
+// ---- generic kernels (fp32 or bf16 storage, fp32 arithmetic) ----
+cudaError_t launch_saliency_generic(const Dims &s, const void *q, const void *k, float *r_kv, float *r_q,
+                                    cudaStream_t st);
+cudaError_t launch_topk_gather(const Dims &s, const float *r, int32_t *idx, const void *k, const void *v, void *khat,
+                               void *vhat, cudaStream_t st);
+cudaError_t launch_npmap(int rows, int Hx, int N, int d, int D, int bf16, const void *x, const void *W, float *phi,
+                         cudaStream_t st);
+cudaError_t launch_linear_state(const Dims &s, const float *phik, const void *v, const int32_t *idx, float *S,
+                                float *z, unsigned *err, cudaStream_t st);
+cudaError_t launch_merge_generic(const Dims &s, const void *q, const void *k, const void *v, const void *Wq,
+                                 const void *khat, const void *vhat, const float *S, const float *z,
+                                 const float *phik, void *o, cudaStream_t st);
+
+// ---- decode ----
+cudaError_t launch_decode_step(const Dims &s, unsigned char *state, const DecodeLayout &L, int pos, const void *Wq,
+                               const void *Wk, const void *q_t, const void *k_t, const void *v_t, void *o_t,
+                               unsigned *err, cudaStream_t st, int *launches);
+cudaError_t launch_state_export(const Dims &s, unsigned char *state, const DecodeLayout &L, const void *k,
+                                const void *v, const float *r, const void *khat, const void *vhat, const float *S,
+                                const float *z, cudaStream_t st);
+cudaError_t launch_decode_init(const Dims &s, unsigned char *state, const DecodeLayout &L, int capacity,
+                               cudaStream_t st);
+
+}  // namespace still

@@ -1,0 +1,185 @@
+"""Python binding of libstill.so (include/still.h): argument marshalling only.
+
+Each function has the name of its C entry point and takes device tensors (or
+raw device addresses as ints); it passes their addresses, the sizes and the
+current CUDA stream to the library and raises StillError on a non-OK status.
+Every step of the computation runs in the library's kernels; there is no
+fallback.  If libstill.so is missing, importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes as ct
+import math
+import os
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libstill.so")
+
+STILL_F32, STILL_BF16 = 0, 1
+STATUS = {0: "STILL_OK", 1: "STILL_ERR_INVALID_ARG", 2: "STILL_ERR_UNSUPPORTED", 3: "STILL_ERR_WORKSPACE",
+          4: "STILL_ERR_CUDA", 5: "STILL_ERR_DEVICE_CHECK", 6: "STILL_ERR_TIMEOUT"}
+
+EXPORTS = ("still_status_string", "still_saliency", "still_select_topk", "still_npmap",
+           "still_prefill_workspace_bytes", "still_prefill_workspace_layout", "still_hybrid_prefill",
+           "still_decode_state_bytes", "still_decode_init", "still_decode_step", "still_get_device_status",
+           "still_launch_count", "still_timing_enable", "still_timing_read")
+
+
+class StillError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} -> {STATUS.get(status, status)} ({status_string(status)})")
+
+
+class still_dims(ct.Structure):
+    _fields_ = [(n, ct.c_int) for n in ("B", "H", "Hkv", "N", "d", "D", "w", "C", "k")] + \
+               [("scale", ct.c_float), ("dtype", ct.c_int)]
+
+
+class still_ws_layout(ct.Structure):
+    _fields_ = [(n, ct.c_size_t) for n in ("r", "idx", "khat", "vhat", "S", "z", "phik", "total")]
+
+
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(f"libstill.so is not built ({_LIB_PATH}); run linear_attention_still_b200._build")
+
+_lib = ct.CDLL(_LIB_PATH)
+_P = ct.c_void_p
+_D = ct.POINTER(still_dims)
+_SIG = {
+    "still_status_string": ([ct.c_int], ct.c_char_p),
+    "still_saliency": ([_D, _P, _P, _P, _P, _P], ct.c_int),
+    "still_select_topk": ([_D, _P, _P, _P], ct.c_int),
+    "still_npmap": ([ct.c_int, ct.c_int, ct.c_int, ct.c_int, ct.c_int, ct.c_int, _P, _P, _P, _P], ct.c_int),
+    "still_prefill_workspace_bytes": ([_D], ct.c_size_t),
+    "still_prefill_workspace_layout": ([_D, ct.POINTER(still_ws_layout)], ct.c_int),
+    "still_hybrid_prefill": ([_D, _P, _P, _P, _P, _P, _P, _P, _P, ct.c_size_t, _P, ct.c_int, _P], ct.c_int),
+    "still_decode_state_bytes": ([_D, ct.c_int], ct.c_size_t),
+    "still_decode_init": ([_D, ct.c_int, _P, _P], ct.c_int),
+    "still_decode_step": ([_D, _P, ct.c_int, ct.c_int, _P, _P, _P, _P, _P, _P, _P], ct.c_int),
+    "still_get_device_status": ([_P], ct.c_int),
+    "still_launch_count": ([], ct.c_uint64),
+    "still_timing_enable": ([ct.c_int], ct.c_int),
+    "still_timing_read": ([ct.POINTER(ct.c_double), ct.POINTER(ct.c_int), ct.c_int], ct.c_int),
+}
+for _name, (_args, _res) in _SIG.items():
+    _f = getattr(_lib, _name)
+    _f.argtypes = _args
+    _f.restype = _res
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def make_dims(B, H, Hkv, N, d, D, w, C, k, dtype="bf16", scale=0.0) -> still_dims:
+    dt = {"bf16": STILL_BF16, "f32": STILL_F32}[dtype] if isinstance(dtype, str) else int(dtype)
+    return still_dims(B, H, Hkv, N, d, D, w, C, k, float(scale), dt)
+
+
+def dims_of(shape, N: int | None = None) -> still_dims:
+    """still_dims of a synth.Shape (N overridable)."""
+    return make_dims(shape.B, shape.H, shape.Hkv, shape.N if N is None else N, shape.d, shape.D, shape.w,
+                     shape.C, shape.k, shape.dtype)
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _ok(fn: str, st: int):
+    if st != 0:
+        raise StillError(fn, st)
+
+
+def status_string(status: int) -> str:
+    return _lib.still_status_string(int(status)).decode()
+
+
+def still_saliency(dims, q, k, r_kv, r_q=None, stream=None):
+    _ok("still_saliency", _lib.still_saliency(ct.byref(dims), _ptr(q), _ptr(k), _ptr(r_kv), _ptr(r_q),
+                                              _stream(stream)))
+
+
+def still_select_topk(dims, r_kv, idx, stream=None):
+    _ok("still_select_topk", _lib.still_select_topk(ct.byref(dims), _ptr(r_kv), _ptr(idx), _stream(stream)))
+
+
+def still_npmap(B, Hx, N, d, D, dtype, x, W, phi, stream=None):
+    dt = {"bf16": STILL_BF16, "f32": STILL_F32}[dtype] if isinstance(dtype, str) else int(dtype)
+    _ok("still_npmap", _lib.still_npmap(B, Hx, N, d, D, dt, _ptr(x), _ptr(W), _ptr(phi), _stream(stream)))
+
+
+def still_prefill_workspace_bytes(dims) -> int:
+    return int(_lib.still_prefill_workspace_bytes(ct.byref(dims)))
+
+
+def still_prefill_workspace_layout(dims) -> dict:
+    out = still_ws_layout()
+    _ok("still_prefill_workspace_layout", _lib.still_prefill_workspace_layout(ct.byref(dims), ct.byref(out)))
+    return {n: int(getattr(out, n)) for n, _ in still_ws_layout._fields_}
+
+
+def still_hybrid_prefill(dims, q, k, v, wq, wk, o, idx_in=None, workspace=None, workspace_bytes=None, state=None,
+                         state_capacity=0, stream=None):
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _ok("still_hybrid_prefill",
+        _lib.still_hybrid_prefill(ct.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(wq), _ptr(wk), _ptr(o),
+                                  _ptr(idx_in), _ptr(workspace), int(workspace_bytes), _ptr(state),
+                                  int(state_capacity), _stream(stream)))
+
+
+def still_decode_state_bytes(dims, capacity: int) -> int:
+    return int(_lib.still_decode_state_bytes(ct.byref(dims), int(capacity)))
+
+
+def still_decode_init(dims, capacity, state, stream=None):
+    _ok("still_decode_init", _lib.still_decode_init(ct.byref(dims), int(capacity), _ptr(state), _stream(stream)))
+
+
+def still_decode_step(dims, state, capacity, pos, wq, wk, q_t, k_t, v_t, o_t, stream=None):
+    _ok("still_decode_step",
+        _lib.still_decode_step(ct.byref(dims), _ptr(state), int(capacity), int(pos), _ptr(wq), _ptr(wk), _ptr(q_t),
+                               _ptr(k_t), _ptr(v_t), _ptr(o_t), _stream(stream)))
+
+
+def still_get_device_status(stream=None) -> int:
+    """Synchronises the stream; returns the (cleared) device status code."""
+    return int(_lib.still_get_device_status(_stream(stream)))
+
+
+def still_launch_count() -> int:
+    return int(_lib.still_launch_count())
+
+
+TIMING_CLASSES = ("saliency", "topk_gather", "npmap", "linear_state", "merge", "state_export")
+
+
+def still_timing_enable(on: bool = True):
+    _ok("still_timing_enable", _lib.still_timing_enable(1 if on else 0))
+
+
+def still_timing_read() -> dict:
+    """{class: (milliseconds, launches)} of the kernels timed since the last read."""
+    n = len(TIMING_CLASSES)
+    ms = (ct.c_double * n)()
+    cnt = (ct.c_int * n)()
+    _ok("still_timing_read", _lib.still_timing_read(ms, cnt, n))
+    return {name: (ms[i], cnt[i]) for i, name in enumerate(TIMING_CLASSES)}
+
+
+def default_scale(d: int) -> float:
+    return 1.0 / math.sqrt(d)

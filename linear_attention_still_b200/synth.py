@@ -14,8 +14,10 @@ to Linearize LLMs, "Efficiency" results: Llama-3.2-1B / Llama-3.1-8B layers at
   drawn without replacement from [1, N) per batch item; their Q, K and V rows
   are scaled by 4 in every head;
 * the NP-Map weights Wq [H, d, D] and Wk [Hkv, d, D] are N(0, 1/d);
-* everything is drawn in fp32 from numpy's PCG64 in the fixed order
-  Q, K, V, lambda_q, lambda_k, lambda_v, heavy positions, Wq, Wk, then rounded
+* everything is drawn in fp32 from numpy PCG64 streams: SeedSequence(seed)
+  spawns B+1 children; child 0 draws Wq then Wk, child 1+b draws batch item
+  b's Q, K, V, lambda_q, lambda_k, lambda_v and heavy positions in that order
+  (so one batch item can be regenerated alone); then everything is rounded
   to the workload dtype (bf16 by round-to-nearest-even).
 """
 from __future__ import annotations
@@ -25,7 +27,7 @@ import math
 
 import numpy as np
 
-__all__ = ["Shape", "WORKLOADS", "Inputs", "make_inputs", "round_to_bf16", "bf16_bits_to_f32"]
+__all__ = ["Shape", "WORKLOADS", "Inputs", "make_inputs", "round_to_bf16", "round_to_bf16_", "bf16_bits_to_f32"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -81,11 +83,20 @@ def round_to_bf16(x: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
 
     Returns (values as fp32, raw bf16 bit patterns as uint16).  Inputs are
     finite by construction."""
-    x = np.ascontiguousarray(x, dtype=np.float32)
+    vals = np.array(x, dtype=np.float32, copy=True)
+    round_to_bf16_(vals)
+    return vals, (vals.view(np.uint32) >> 16).astype(np.uint16)
+
+
+def round_to_bf16_(x: np.ndarray) -> np.ndarray:
+    """In-place variant: x (contiguous fp32) is replaced by its bf16-rounded values."""
     u = x.view(np.uint32)
-    bias = ((u >> 16) & 1) + np.uint32(0x7FFF)
-    bits = ((u + bias) >> 16).astype(np.uint16)
-    return bf16_bits_to_f32(bits), bits
+    tmp = u >> 16
+    tmp &= 1
+    tmp += np.uint32(0x7FFF)
+    u += tmp
+    u &= np.uint32(0xFFFF0000)
+    return x
 
 
 def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
@@ -108,36 +119,46 @@ class Inputs:
         return round_to_bf16(getattr(self, name))[1]
 
 
-def make_inputs(shape: Shape, seed: int | None = None) -> Inputs:
-    """Draw the inputs for `shape` (Ntot = N + decode_steps tokens)."""
+def make_inputs(shape: Shape, seed: int | None = None, batches=None) -> Inputs:
+    """Draw the inputs for `shape` (Ntot = N + decode_steps tokens).
+
+    batches: optional list of batch indices to draw (others are skipped); the
+    returned arrays then hold only those items, in the given order."""
     s = shape
     seed = s.seed if seed is None else seed
     ntot = s.N + s.decode_steps
-    rng = np.random.Generator(np.random.PCG64(seed))
+    bsel = list(range(s.B)) if batches is None else [int(b) for b in batches]
     f32 = np.float32
-    q = rng.standard_normal((s.B, s.H, ntot, s.d), dtype=f32)
-    k = rng.standard_normal((s.B, s.Hkv, ntot, s.d), dtype=f32)
-    v = rng.standard_normal((s.B, s.Hkv, ntot, s.d), dtype=f32)
-    lq = rng.lognormal(0.0, 0.5, size=(s.B, s.H, ntot)).astype(f32)
-    lk = rng.lognormal(0.0, 0.5, size=(s.B, s.Hkv, ntot)).astype(f32)
-    lv = rng.lognormal(0.0, 0.5, size=(s.B, s.Hkv, ntot)).astype(f32)
+    children = np.random.SeedSequence(seed).spawn(s.B + 1)
+    wrng = np.random.Generator(np.random.PCG64(children[0]))
+    wq = wrng.standard_normal((s.H, s.d, s.D), dtype=f32) * f32(1.0 / math.sqrt(s.d))
+    wk = wrng.standard_normal((s.Hkv, s.d, s.D), dtype=f32) * f32(1.0 / math.sqrt(s.d))
+    nb = len(bsel)
+    q = np.empty((nb, s.H, ntot, s.d), dtype=f32)
+    k = np.empty((nb, s.Hkv, ntot, s.d), dtype=f32)
+    v = np.empty((nb, s.Hkv, ntot, s.d), dtype=f32)
     nh = min(s.n_heavy, max(ntot - 1, 0))
-    heavy = np.stack([rng.choice(np.arange(1, ntot), size=nh, replace=False) for _ in range(s.B)]) \
-        if nh > 0 else np.zeros((s.B, 0), dtype=np.int64)
-    wq = rng.standard_normal((s.H, s.d, s.D), dtype=f32) * f32(1.0 / math.sqrt(s.d))
-    wk = rng.standard_normal((s.Hkv, s.d, s.D), dtype=f32) * f32(1.0 / math.sqrt(s.d))
-
-    q *= lq[..., None]
-    k *= lk[..., None]
-    v *= lv[..., None]
-    for b in range(s.B):
-        pos = heavy[b]
-        q[b, :, pos, :] *= f32(4.0)
-        k[b, :, pos, :] *= f32(4.0)
-        v[b, :, pos, :] *= f32(4.0)
-
+    heavy = np.zeros((nb, nh), dtype=np.int64)
+    for n, b in enumerate(bsel):
+        rng = np.random.Generator(np.random.PCG64(children[1 + b]))
+        rng.standard_normal((s.H, ntot, s.d), dtype=f32, out=q[n])
+        rng.standard_normal((s.Hkv, ntot, s.d), dtype=f32, out=k[n])
+        rng.standard_normal((s.Hkv, ntot, s.d), dtype=f32, out=v[n])
+        lq = rng.lognormal(0.0, 0.5, size=(s.H, ntot)).astype(f32)
+        lk = rng.lognormal(0.0, 0.5, size=(s.Hkv, ntot)).astype(f32)
+        lv = rng.lognormal(0.0, 0.5, size=(s.Hkv, ntot)).astype(f32)
+        if nh > 0:
+            heavy[n] = rng.choice(np.arange(1, ntot), size=nh, replace=False)
+        q[n] *= lq[..., None]
+        k[n] *= lk[..., None]
+        v[n] *= lv[..., None]
+        pos = heavy[n]
+        q[n][:, pos, :] *= f32(4.0)
+        k[n][:, pos, :] *= f32(4.0)
+        v[n][:, pos, :] *= f32(4.0)
     if s.dtype == "bf16":
-        q, k, v, wq, wk = (round_to_bf16(a)[0] for a in (q, k, v, wq, wk))
+        for a in (q, k, v, wq, wk):
+            round_to_bf16_(a)
     elif s.dtype != "f32":
         raise ValueError(f"unknown dtype {s.dtype}")
-    return Inputs(s, q, k, v, wq, wk, heavy.astype(np.int64))
+    return Inputs(s, q, k, v, wq, wk, heavy)

@@ -1,0 +1,111 @@
+"""CPU checks of the C-ABI library: it loads, exports every entry point include/still.h declares,
+and rejects bad arguments on the host before launching anything (no GPU needed)."""
+import ctypes as ct
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from linear_attention_still_b200 import _build
+    _build.build()
+    from linear_attention_still_b200 import still
+    return still
+
+
+def _declared():
+    names = []
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", f)).read()
+            names += re.findall(r"STILL_API\s+[\w\s\*]+?\b(still_\w+)\s*\(", txt)
+    return sorted(set(names))
+
+
+def test_exports_every_declared_symbol(lib):
+    declared = _declared()
+    assert len(declared) >= 12
+    so = ct.CDLL(lib.library_path())
+    for name in declared:
+        assert hasattr(so, name), name
+    assert set(declared) == set(lib.EXPORTS)
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        assert lib.status_string(code)
+    assert lib.status_string(99) == "unknown status"
+
+
+def _dims(lib, **kw):
+    base = dict(B=1, H=4, Hkv=2, N=300, d=64, D=64, w=128, C=64, k=8, dtype="bf16")
+    base.update(kw)
+    return lib.make_dims(**base)
+
+
+FAKE = 1 << 20  # an aligned address that is never dereferenced: validation fails first
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(w=100), 1),          # window not a whole number of chunks
+    (dict(w=0, k=4), 1),       # no window but tokens kept
+    (dict(k=65), 1),           # k > C
+    (dict(H=6, Hkv=4), 1),     # H % Hkv
+    (dict(d=12), 1),           # head dim not a multiple of 8
+    (dict(D=0), 1),
+    (dict(d=512), 2),          # beyond the supported head dim
+    (dict(H=64, Hkv=1), 2),    # group larger than 32
+    (dict(N=-1), 1),
+    (dict(dtype=7), 1),
+])
+def test_prefill_rejects_bad_dims(lib, kw, code):
+    d = _dims(lib, **kw)
+    assert lib._lib.still_hybrid_prefill(ct.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 40,
+                                         None, 0, None) == code
+    assert lib.still_prefill_workspace_bytes(d) == 0
+
+
+def test_prefill_rejects_bad_pointers_and_workspace(lib):
+    d = _dims(lib)
+    need = lib.still_prefill_workspace_bytes(d)
+    assert need > 0
+    L = lib.still_prefill_workspace_layout(d)
+    assert L["total"] == need and L["r"] == 0
+    assert all(L[a] < L[b] for a, b in zip(("r", "idx", "khat", "vhat", "S", "z", "phik"),
+                                             ("idx", "khat", "vhat", "S", "z", "phik", "total")))
+    f = lib._lib.still_hybrid_prefill
+    assert f(ct.byref(d), None, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, need, None, 0, None) == 1
+    assert f(ct.byref(d), FAKE + 4, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, need, None, 0, None) == 1
+    assert f(ct.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, need - 1, None, 0, None) == 3
+    assert f(ct.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, need, FAKE, 299, None) == 1
+    assert f(None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, need, None, 0, None) == 1
+
+
+def test_step_entry_points_reject(lib):
+    d = _dims(lib, w=0, k=0)
+    assert lib._lib.still_saliency(ct.byref(d), FAKE, FAKE, FAKE, None, None) == 1  # needs a window
+    d = _dims(lib)
+    assert lib._lib.still_saliency(ct.byref(d), None, FAKE, FAKE, None, None) == 1
+    assert lib._lib.still_select_topk(ct.byref(d), FAKE + 8, FAKE, None) == 1
+    assert lib._lib.still_npmap(1, 2, 10, 12, 64, 1, FAKE, FAKE, FAKE, None) == 1
+    assert lib._lib.still_npmap(1, 2, 10, 64, 512, 1, FAKE, FAKE, FAKE, None) == 2
+
+
+def test_decode_rejects(lib):
+    d = _dims(lib)
+    assert lib.still_decode_state_bytes(d, 4096) > 0
+    f = lib._lib.still_decode_step
+    assert f(ct.byref(d), FAKE, 100, 100, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 1   # pos == capacity
+    assert f(ct.byref(d), FAKE, 100, -1, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 1
+    assert f(ct.byref(d), None, 100, 0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 1
+    assert lib._lib.still_decode_init(ct.byref(d), -1, FAKE, None) == 1
+
+
+def test_decode_state_size_grows_with_capacity(lib):
+    d = _dims(lib)
+    a, b = lib.still_decode_state_bytes(d, 1024), lib.still_decode_state_bytes(d, 8192)
+    assert b > a > 0

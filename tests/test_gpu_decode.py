@@ -1,0 +1,88 @@
+"""GPU parity of the chunk-granular delayed decode: prefill(N0) -> T decode steps reproduces rows
+N0..N0+T-1 of the oracle's prefill of N0+T tokens, including the steps that close a chunk."""
+import numpy as np
+import pytest
+import torch
+
+from linear_attention_still_b200.synth import WORKLOADS, Shape, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+from tests._gpu import OUT_TOL, dev, gpu_prefill, odims, row_rel_err  # noqa: E402
+
+CASES = {
+    # name: (shape with N = prefill length, decode steps)
+    "f32_b1_h2": (WORKLOADS["still_f32_b1_h2_n512"].replace(N=300), 100),
+    "bf16_gqa": (Shape(B=2, H=8, Hkv=2, N=520, d=64, D=64, w=128, C=128, k=16), 260),
+    "bf16_d128_two_chunk_window": (Shape(B=1, H=4, Hkv=1, N=390, d=128, D=128, w=256, C=128, k=24), 140),
+    "f32_no_window": (Shape(B=1, H=2, Hkv=1, N=100, d=64, D=32, w=0, C=64, k=0, dtype="f32"), 60),
+    "bf16_keep_none": (Shape(B=1, H=4, Hkv=2, N=250, d=64, D=64, w=128, C=128, k=0), 20),
+    "bf16_from_empty": (Shape(B=1, H=4, Hkv=2, N=0, d=64, D=64, w=128, C=128, k=16), 300),
+}
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from linear_attention_still_b200 import _build
+    _build.build()
+    from linear_attention_still_b200 import still
+    return still
+
+
+def run_decode(lib, shape, T, inp):
+    N0 = shape.N
+    cap = N0 + T
+    d = lib.dims_of(shape, N=N0)
+    state = torch.zeros(lib.still_decode_state_bytes(d, cap), dtype=torch.uint8, device="cuda")
+    lib.still_decode_init(d, cap, state)
+    if N0 > 0:
+        out = gpu_prefill(shape, inp, N=N0, state=state, capacity=cap)
+        assert out["status"] == 0
+    q, k, v = (dev(getattr(inp, n), shape) for n in ("q", "k", "v"))
+    wq, wk = dev(inp.wq, shape), dev(inp.wk, shape)
+    outs = []
+    o_t = torch.empty(shape.B, shape.H, shape.d, dtype=q.dtype, device="cuda")
+    for p in range(N0, cap):
+        lib.still_decode_step(d, state, cap, p, wq, wk, q[:, :, p].contiguous(), k[:, :, p].contiguous(),
+                              v[:, :, p].contiguous(), o_t)
+        outs.append(o_t.float().cpu().numpy().copy())
+    assert lib.still_get_device_status() == 0
+    return np.stack(outs, axis=2), state  # [B,H,T,d]
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_decode_matches_prefill_rows(lib, oracle_mod, name):
+    shape, T = CASES[name]
+    full = shape.replace(N=shape.N + T)
+    inp = make_inputs(shape.replace(decode_steps=T))
+    got, _ = run_decode(lib, shape, T, inp)
+    gp = gpu_prefill(full, inp)
+    idx = gp["idx"] if full.k > 0 and full.T > 0 else None
+    ref = oracle_mod.prefill(odims(full), inp.q, inp.k, inp.v, inp.wq, inp.wk, idx_in=idx)["o"]
+    tol = OUT_TOL[shape.dtype]
+    assert row_rel_err(got, ref[:, :, shape.N:]) <= tol
+    assert row_rel_err(got, gp["o"][:, :, shape.N:]) <= tol
+
+
+def test_decode_from_empty_matches_oracle_state_machine(lib, oracle_mod):
+    shape, T = Shape(B=1, H=2, Hkv=1, N=0, d=64, D=64, w=64, C=64, k=8, dtype="f32"), 200
+    inp = make_inputs(shape.replace(decode_steps=T))
+    got, _ = run_decode(lib, shape, T, inp)
+    dec = oracle_mod.Decoder(odims(shape.replace(N=T)), inp.wq, inp.wk)
+    for p in range(T):
+        o, _ = dec.step(inp.q[:, :, p], inp.k[:, :, p], inp.v[:, :, p])
+        assert row_rel_err(got[:, :, p], o) <= OUT_TOL["f32"], p
+
+
+def test_decode_position_mismatch_is_reported(lib):
+    shape = Shape(B=1, H=2, Hkv=1, N=0, d=64, D=64, w=64, C=64, k=8)
+    d = lib.dims_of(shape)
+    cap = 64
+    state = torch.zeros(lib.still_decode_state_bytes(d, cap), dtype=torch.uint8, device="cuda")
+    lib.still_decode_init(d, cap, state)
+    x = torch.zeros(shape.B, shape.H, shape.d, dtype=torch.bfloat16, device="cuda")
+    kv = torch.zeros(shape.B, shape.Hkv, shape.d, dtype=torch.bfloat16, device="cuda")
+    w = torch.zeros(shape.H, shape.d, shape.D, dtype=torch.bfloat16, device="cuda")
+    o = torch.empty_like(x)
+    lib.still_decode_step(d, state, cap, 3, w, w[:1], x, kv, kv, o)  # state is at 0
+    assert lib.still_get_device_status() == 5
