@@ -16,8 +16,8 @@ merge (every step of the layer).  Prints ONE JSON line (rank 0).
 * roofline: the merge kernel (dominant), algorithmic FLOPs per launch over its
   event-timed duration, against the measured bf16 dense peak.
 * cpu_baseline: the fp64 oracle on the host cores, on a bounded sample of the
-  same workload (one (batch, KV-group) slice, a stride of its query rows),
-  scaled to the whole layer.
+  same workload (whole (batch, KV-group) slices, every query row or a stride
+  of them, about 15 s of CPU work), scaled to the whole layer.
 * --impl reference: that oracle arm alone, as the line's value.
 Multi-GPU: independent replicas (the layer has no cross-GPU exchange), weak scaling.
 """
@@ -142,47 +142,58 @@ class ClockSampler:
 # ----------------------------------------------------------------------------- CPU baseline (oracle)
 
 def oracle_sample(shape, seconds: float, nthreads: int | None = None):
-    """Time the fp64 oracle on one (batch 0, KV group 0) slice: its saliency + top-k over all N tokens, and
-    the outputs of every `stride`-th query row of its G heads; scale to the whole layer.  Returns
-    (tokens/s, seconds measured, description, threads)."""
+    """Time the fp64 oracle on whole (batch, KV group) slices -- saliency + top-k over all N tokens, then
+    the outputs of every `stride`-th query row of the group's G heads -- slice after slice until about
+    `seconds` have been spent (stride 1 when a slice is cheap enough), and scale to the whole layer.
+    Returns (tokens/s, seconds measured, description, threads)."""
     import numpy as np
 
     import oracle
     oracle.build()
     nth = nthreads or len(os.sched_getaffinity(0))
     sl = shape.replace(B=1, H=shape.G, Hkv=1)
-    inp = make_inputs(shape.replace(decode_steps=0), batches=[0])
-    q = inp.q[:, :shape.G]
-    k, v = inp.k[:, :1], inp.v[:, :1]
-    wq, wk = inp.wq[:shape.G], inp.wk[:1]
     d = oracle.Dims.of(sl)
-    t0 = time.perf_counter()
-    idx = None
-    if shape.w > 0 and shape.k > 0 and shape.T > 0:
-        _, r = oracle.saliency(d, q, k, nthreads=nth)
-        idx = oracle.topk(d, r)
-    t_sel = time.perf_counter() - t0
-    # calibrate the row stride on a coarse sample, then size the sample to the time budget
-    stride = max(1, shape.N // 64)
-    rows = np.array([(0, h, i) for h in range(shape.G) for i in range(0, shape.N, stride)], dtype=np.int32)
-    t0 = time.perf_counter()
-    oracle.prefill(d, q, k, v, wq, wk, idx_in=idx, rows=rows, nthreads=nth)
-    t_cal = time.perf_counter() - t0
-    budget = max(seconds - t_sel, 0.5)
-    new_stride = max(1, int(math.ceil(stride * t_cal / budget)))
-    if new_stride < stride:
-        stride = new_stride
-        rows = np.array([(0, h, i) for h in range(shape.G) for i in range(0, shape.N, stride)], dtype=np.int32)
+    slices = [(b, g) for b in range(shape.B) for g in range(shape.Hkv)]
+    stride = None
+    t_total, rows_done, done, t_sel_sum = 0.0, 0, 0, 0.0
+    cur_b, inp = None, None
+    for b, g in slices:
+        if b != cur_b:
+            inp = make_inputs(shape.replace(decode_steps=0), batches=[b])
+            cur_b = b
+        q = np.ascontiguousarray(inp.q[:, g * shape.G:(g + 1) * shape.G])
+        k, v = inp.k[:, g:g + 1], inp.v[:, g:g + 1]
+        wq, wk = inp.wq[g * shape.G:(g + 1) * shape.G], inp.wk[g:g + 1]
         t0 = time.perf_counter()
+        idx = None
+        if shape.w > 0 and shape.k > 0 and shape.T > 0:
+            _, r = oracle.saliency(d, q, k, nthreads=nth)
+            idx = oracle.topk(d, r)
+        t_sel = time.perf_counter() - t0
+        if stride is None:  # calibrate on a coarse sample of the first slice
+            cal = max(1, shape.N // 64)
+            rows = np.array([(0, h, i) for h in range(shape.G) for i in range(0, shape.N, cal)], dtype=np.int32)
+            t1 = time.perf_counter()
+            oracle.prefill(d, q, k, v, wq, wk, idx_in=idx, rows=rows, nthreads=nth)
+            per_row = (time.perf_counter() - t1) / len(rows)
+            full = per_row * shape.G * shape.N
+            stride = max(1, int(math.ceil(full / max(seconds - t_sel, 0.5))))
+        rows = np.array([(0, h, i) for h in range(shape.G) for i in range(0, shape.N, stride)], dtype=np.int32)
+        t1 = time.perf_counter()
         oracle.prefill(d, q, k, v, wq, wk, idx_in=idx, rows=rows, nthreads=nth)
-        t_cal = time.perf_counter() - t0
-    frac = len(rows) / (shape.G * shape.N)
-    t_slice = t_sel + t_cal / frac
-    t_layer = t_slice * shape.B * shape.Hkv
-    desc = (f"oracle fp64 on batch 0 / KV group 0 ({shape.G} heads): saliency + top-k over all {shape.N} tokens "
-            f"({t_sel:.2f} s) and every {stride}-th query row ({len(rows)} rows, {t_cal:.2f} s), scaled by "
-            f"1/{frac:.4g} rows and x{shape.B * shape.Hkv} slices")
-    return shape.B * shape.N / t_layer, t_sel + t_cal, desc, nth
+        t_rows = time.perf_counter() - t1
+        frac = len(rows) / (shape.G * shape.N)
+        t_total += t_sel + t_rows / frac
+        t_sel_sum += t_sel + t_rows
+        rows_done += len(rows)
+        done += 1
+        if t_sel_sum >= seconds:
+            break
+    t_layer = t_total / done * len(slices)
+    desc = (f"oracle fp64, {done} of {len(slices)} (batch, KV group) slices of {shape.G} heads: saliency + top-k "
+            f"over all {shape.N} tokens and every {stride}-th query row ({rows_done} rows); "
+            f"{t_sel_sum:.1f} s measured, scaled to all rows and slices")
+    return shape.B * shape.N / t_layer, t_sel_sum, desc, nth
 
 
 # ----------------------------------------------------------------------------- main arms

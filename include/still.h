@@ -117,6 +117,8 @@ typedef struct {
     size_t S;      /* fp32  [B,Hkv,T+1,D,d]    linear state seen by chunk t    */
     size_t z;      /* fp32  [B,Hkv,T+1,D]      linear normaliser seen by chunk t */
     size_t phik;   /* fp32  [B,Hkv,N,D]        NP-Map features of the keys     */
+    size_t wqt;    /* bf16  [H,D,d]            Wq transposed (bf16 tensor-core path) */
+    size_t st;     /* bf16  [B,Hkv,T+1,d,D]    S_t transposed (bf16 tensor-core path) */
     size_t total;
 } still_ws_layout;
 
@@ -194,6 +196,15 @@ STILL_API uint64_t still_launch_count(void);
  * 0 saliency, 1 top-k + gather, 2 NP-Map, 3 linear state, 4 softmax/linear
  * merge, 5 decode-state export.  Single-threaded use only.
  */
+/*
+ * Diagnostics (no counterpart in the method): when `words` is non-NULL, the
+ * tensor-core merge kernel records 16 progress words per CTA there (producer,
+ * MMA issuer and each softmax warp: last step reached; 0xBAD.. on a bounded
+ * wait that gave up; 0xD0E / 0xF1F at exit).  Pass host-mapped (pinned)
+ * memory to read it while a kernel runs.  NULL (the default) disables it.
+ */
+STILL_API void still_debug_set_trace(unsigned *words);
+
 #define STILL_TIMING_MAX_LAUNCHES 4096
 #define STILL_TIMING_CLASSES 6
 STILL_API still_status still_timing_enable(int on);

@@ -12,10 +12,12 @@ namespace still {
 cudaError_t launch_gather(const Dims &s, const int32_t *idx, const void *k, const void *v, void *khat, void *vhat,
                           unsigned *err, cudaStream_t st);
 bool tc_merge_supported(const Dims &s);
-cudaError_t launch_merge_tc(const Dims &s, const void *q, const void *k, const void *v, const void *Wq,
-                            const void *khat, const void *vhat, const float *S, const float *z, void *o,
+cudaError_t launch_wq_transpose(const Dims &s, const void *wq, void *wqt, cudaStream_t st);
+cudaError_t launch_merge_tc(const Dims &s, const void *q, const void *k, const void *v, const void *wqt,
+                            const void *khat, const void *vhat, const void *st_t, const float *z, void *o,
                             unsigned *err, cudaStream_t st);
 bool tc_saliency_supported(const Dims &s);
+void set_debug_trace_words(unsigned *p);
 cudaError_t launch_saliency_tc(const Dims &s, const void *q, const void *k, float *r_kv, float *r_q, unsigned *err,
                                cudaStream_t st);
 }  // namespace still
@@ -91,6 +93,11 @@ still_ws_layout ws_layout(const Dims &s) {
     off = al256(off + BK * (T + 1) * s.D * 4);
     L.phik = off;
     off = al256(off + BK * s.N * s.D * 4);
+    const bool tc = s.bf16 != 0;  // transposed bf16 operands of the tensor-core merge
+    L.wqt = off;
+    off = al256(off + (tc ? (size_t)s.H * s.D * s.d * 2 : 0));
+    L.st = off;
+    off = al256(off + (tc ? BK * (T + 1) * s.D * s.d * 2 : 0));
     L.total = off;
     return L;
 }
@@ -253,6 +260,8 @@ still_status still_hybrid_prefill(const still_dims *dims, const void *q, const v
     void *khat = ws + W.khat, *vhat = ws + W.vhat;
     float *S = reinterpret_cast<float *>(ws + W.S), *z = reinterpret_cast<float *>(ws + W.z);
     float *phik = reinterpret_cast<float *>(ws + W.phik);
+    void *wqt = ws + W.wqt, *st_t = ws + W.st;
+    const bool use_tc = tc_merge_supported(s);
     const bool select = s.w > 0 && s.k > 0 && s.T() > 0;
     const bool need_r = s.w > 0 && s.k > 0 && (!idx_in || state);
 
@@ -280,13 +289,16 @@ still_status still_hybrid_prefill(const still_dims *dims, const void *q, const v
     }
     {
         TimingScope ts(3, cs);
-        STILL_LAUNCH(launch_linear_state(s, phik, v, idx_used, S, z, err, cs));
+        STILL_LAUNCH(launch_linear_state(s, phik, v, idx_used, S, z, use_tc ? st_t : nullptr, err, cs));
         g_launches.fetch_add(s.T() - s.m() > 0 ? 1 : 0);  // the delta kernel (the prefix was counted)
     }
     // 5. softmax branch + linear branch + merge
     {
     TimingScope ts(4, cs);
-    if (tc_merge_supported(s)) STILL_LAUNCH(launch_merge_tc(s, q, k, v, Wq, khat, vhat, S, z, o, err, cs));
+    if (use_tc) {
+        STILL_LAUNCH(launch_wq_transpose(s, Wq, wqt, cs));
+        STILL_LAUNCH(launch_merge_tc(s, q, k, v, wqt, khat, vhat, st_t, z, o, err, cs));
+    }
     else STILL_LAUNCH(launch_merge_generic(s, q, k, v, Wq, khat, vhat, S, z, phik, o, cs));
     }
     // hand-off to decode
@@ -318,6 +330,8 @@ still_status still_decode_step(const still_dims *dims, void *state, int capacity
     g_launches.fetch_add(launches);
     return cuda_status(e);
 }
+
+void still_debug_set_trace(unsigned *words) { set_debug_trace_words(words); }
 
 still_status still_timing_enable(int on) {
     g_timing = on != 0;

@@ -215,7 +215,9 @@ __global__ void __launch_bounds__(256) linear_delta_kernel(Dims s, const float *
 }
 
 // Inclusive prefix over slots 0..T: slots 0..m are zero (no chunk has been decided for them).
-__global__ void linear_prefix_kernel(Dims s, float *__restrict__ S, float *__restrict__ z) {
+// st_t (optional): a bf16 copy of every S_t, transposed to [d, D] (K-major operand of phi(q) S_t).
+__global__ void linear_prefix_kernel(Dims s, float *__restrict__ S, float *__restrict__ z,
+                                     __nv_bfloat16 *__restrict__ st_t) {
     const int T_ = s.T(), m = s.m();
     const int Dd = s.D * s.d, per = Dd + s.D;
     const size_t gid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -228,6 +230,10 @@ __global__ void linear_prefix_kernel(Dims s, float *__restrict__ S, float *__res
         float *p = e < Dd ? &S[(bg * (T_ + 1) + t) * Dd + e] : &z[(bg * (T_ + 1) + t) * s.D + (e - Dd)];
         if (t >= m + 1) run += *p;
         *p = run;
+        if (st_t && e < Dd) {
+            const int a = e / s.d, x = e % s.d;
+            st_t[((bg * (T_ + 1) + t) * s.d + x) * s.D + a] = __float2bfloat16_rn(run);
+        }
     }
 }
 
@@ -416,7 +422,7 @@ cudaError_t launch_npmap(int rows, int Hx, int N, int d, int D, int bf16, const 
 }
 
 cudaError_t launch_linear_state(const Dims &s, const float *phik, const void *v, const int32_t *idx, float *S,
-                                float *z, unsigned *err, cudaStream_t st) {
+                                float *z, void *st_t, unsigned *err, cudaStream_t st) {
     const int T_ = s.T(), m = s.m();
     const int nc = T_ - m;  // chunks c <= T-m-1 are seen by some query chunk
     if (s.B * s.Hkv == 0) return cudaSuccess;
@@ -441,7 +447,8 @@ cudaError_t launch_linear_state(const Dims &s, const float *phik, const void *v,
         if (e != cudaSuccess) return e;
     }
     const size_t total = (size_t)s.B * s.Hkv * ((size_t)s.D * s.d + s.D);
-    linear_prefix_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(s, S, z);
+    linear_prefix_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(s, S, z,
+                                                                         static_cast<__nv_bfloat16 *>(st_t));
     return cudaGetLastError();
 }
 

@@ -1,15 +1,628 @@
-// kernels_tc.cu -- tcgen05 / TMEM / TMA kernels for sm_100a (bf16): the hybrid merge and the
-// banded saliency.  (Filled in below as they land; until then the generic kernels serve.)
+// kernels_tc.cu -- tcgen05 / TMEM / TMA kernels for sm_100a (bf16 storage, fp32 accumulation):
+// the hybrid merge of "STILL: Selecting Tokens for Intra-Layer Hybrid Attention to Linearize LLMs"
+// ([p1] jsqmd.com introduction: kept tokens -> softmax attention, the rest -> linear attention, in
+// the same layer; "NP-Map": one shared distribution for both branches; [p4] atlas.scime.ai
+// "Approach").
+//
+// One CTA = one (batch b, KV group g) x HP query heads of that group x 128 consecutive queries of
+// one chunk t (C is a multiple of 128).  The HP heads see the same keys, so every K/V tile is loaded
+// once per CTA.  Per query row i (TMEM lane = row):
+//   prologue:  Y = Q Wq^T (tensor cores) -> phi(q) = ||q|| e/||e||, e = exp(Y - max Y)
+//              O := phi(q) S_t^T (tensor cores), l := phi(q) . z_t (fp32), running max := 0
+//              (or -inf, l := 0 when the linear branch is empty) -- the linear branch enters the
+//              online softmax as a pre-accumulated term under the shared normaliser;
+//   main loop: key tiles of 128: the kept rows of chunks c <= t-m-1 (compact cache, ragged last
+//              tile masked), then the window [max(0,(t-m)C), i0+127] (diagonal tile masked
+//              causally); S = Q K^T into TMEM, softmax rows in registers, P (bf16) written back
+//              into TMEM over S, O += P V with P as the TMEM operand;
+//   epilogue:  o = O / l.
+// Warp roles: 4*HP softmax warps (warpgroup x owns head tile x), one TMA producer warp, one MMA
+// warp (also allocates TMEM).  Every mbarrier wait is bounded; on a timeout the CTA records
+// DEV_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
+#include <cuda.h>
+
 #include "common.cuh"
 #include "still_internal.h"
+#include "tc_ptx.cuh"
 
 namespace still {
 
-bool tc_merge_supported(const Dims &) { return false; }
-cudaError_t launch_merge_tc(const Dims &, const void *, const void *, const void *, const void *, const void *,
-                            const void *, const float *, const float *, void *, unsigned *, cudaStream_t) {
+using namespace tc;
+
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int DH, int DF, int HP>
+struct MergeCfg {
+    static constexpr int BM = 128;                     // query rows per head tile
+    static constexpr int BN = 128;                     // keys per tile
+    static constexpr int REG = 128 * 128;              // one 128-row x 64-col bf16 region (16 KB)
+    static constexpr int TILE_BYTES = 128 * DH * 2;    // 128 x DH bf16 = DH/64 regions
+    static constexpr int Q_BYTES = HP * TILE_BYTES;
+    static constexpr int NS = DH == 128 ? 2 : 4;       // K/V pipeline stages
+    static constexpr int STAGE_BYTES = 2 * TILE_BYTES; // K + V
+    static constexpr int WQ_BYTES = DF * DH * 2;       // one Wq^T [DF rows x DH]
+    static constexpr int ST_BYTES = DH * DF * 2;       // S_t^T [DH rows x DF]
+    static_assert(HP * WQ_BYTES + ST_BYTES <= NS * STAGE_BYTES, "prologue tiles must fit the stage area");
+    static constexpr int NUM_BARS = 4 + 3 * NS + 5 * HP;      // see the slot map in the kernel
+    static constexpr int TMEM_SLOT_OFF = 8 * NUM_BARS;          // u32 TMEM base address
+    static constexpr int ABORT_OFF = TMEM_SLOT_OFF + 8;         // int abort flag
+    static constexpr int BAR_BYTES = 256;
+    static_assert(ABORT_OFF + 8 <= BAR_BYTES, "barrier area overflow");
+    static constexpr int SMEM = Q_BYTES + NS * STAGE_BYTES + BAR_BYTES + 1024;
+    static constexpr int THREADS = 128 * HP + 64;
+    static constexpr int PRODUCER_WARP = 4 * HP;
+    static constexpr int MMA_WARP = 4 * HP + 1;
+    static constexpr int TMEM_COLS = 512;
+    __host__ __device__ static constexpr int s_col(int x) { return x * 128; }
+    __host__ __device__ static constexpr int o_col(int x) { return 128 * HP + x * DH; }
+    static_assert(128 * HP + HP * DH <= TMEM_COLS, "TMEM budget");
+};
+
+struct MergeParams {
+    int B, H, Hkv, N, C, k, w, G, T;
+    float scale_log2;      // tau * log2(e)
+    const float *z;        // [B*Hkv*(T+1), DF] fp32
+    __nv_bfloat16 *o;      // [B,H,N,DH]
+    unsigned *err;
+    int n_qtiles;          // ceil(N/128)
+    int pairs;             // G / HP
+    unsigned *trace;       // optional progress words (16 per CTA), see still_debug_set_trace
+};
+
+// Progress word of this CTA (diagnostics only; a no-op unless a trace buffer is set).
+__device__ __forceinline__ void trace_word(unsigned *trace, int slot, unsigned v) {
+    if (trace) {
+        *reinterpret_cast<volatile unsigned *>(trace + blockIdx.x * 16 + slot) = v;
+        __threadfence_system();
+    }
+}
+
+// tcgen05.ld/st are warp-collective: every decision that guards them is made warp-uniform.
+__device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
+
+// K-major SW128 descriptor of k-step kk (16 elements) of a tile whose rows are split into 64-col
+// regions of `region_bytes` each.
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, int kk, uint32_t region_bytes) {
+    return sw128_desc(base + (kk >> 2) * region_bytes + (kk & 3) * 32, 16, 1024);
+}
+
+template <int DH, int DF, int HP>
+__global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
+    merge_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+                    const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_kh,
+                    const __grid_constant__ CUtensorMap map_vh, const __grid_constant__ CUtensorMap map_wq,
+                    const __grid_constant__ CUtensorMap map_st, const MergeParams p) {
+    using Cfg = MergeCfg<DH, DF, HP>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t sQ = sbase;                         // HP tiles
+    const uint32_t sStage = sbase + Cfg::Q_BYTES;      // NS x (K tile, V tile); prologue Wq^T / S^T alias it
+    uint8_t *bar_area = smem + Cfg::Q_BYTES + Cfg::NS * Cfg::STAGE_BYTES;
+    const uint32_t sBar = smem_u32(bar_area);
+    // barrier slots (8 bytes each)
+    auto BAR = [&](int i) { return sBar + 8u * i; };
+    const int B_QFULL = 0, B_WFULL = 1, B_PRO = 2, B_DRAIN = 3;
+    const int B_KFULL = 4, B_VFULL = 4 + Cfg::NS, B_KVEMPTY = 4 + 2 * Cfg::NS;
+    const int B_Y = 4 + 3 * Cfg::NS, B_PHI = B_Y + HP, B_S = B_PHI + HP, B_P = B_S + HP, B_O = B_P + HP;
+    static_assert(Cfg::NUM_BARS == 4 + 3 * Cfg::NS + 5 * HP, "slot map");
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_area + Cfg::TMEM_SLOT_OFF);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bar_area + Cfg::ABORT_OFF);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // ---- CTA -> (b, g, head pair, query tile); heavier (later) query tiles first
+    const int per_qt = p.B * p.Hkv * p.pairs;
+    const int qt = p.n_qtiles - 1 - (int)(blockIdx.x / per_qt);
+    const int rem = blockIdx.x % per_qt;
+    const int pair = rem % p.pairs;
+    const int bg = rem / p.pairs;
+    const int b = bg / p.Hkv, g = bg % p.Hkv;
+    const int i0 = qt * Cfg::BM;
+    const int t = i0 / p.C;
+    const int m = p.w / p.C;
+    const int nk = p.k * max(0, t - m);                  // kept rows seen by this chunk
+    const int lo = max(0, (t - m) * p.C);                // window start
+    const int n_pre = (nk + Cfg::BN - 1) / Cfg::BN;
+    const int n_tiles = n_pre + (i0 - lo) / Cfg::BN + 1;
+    const int tslot = bg * (p.T + 1) + t;                // linear state slot
+
+    if (threadIdx.x == 0) {
+        mbar_init(BAR(B_QFULL), 1);
+        mbar_init(BAR(B_WFULL), 1);
+        mbar_init(BAR(B_PRO), 1);
+        mbar_init(BAR(B_DRAIN), 1);
+        for (int s = 0; s < Cfg::NS; ++s) {
+            mbar_init(BAR(B_KFULL + s), 1);
+            mbar_init(BAR(B_VFULL + s), 1);
+            mbar_init(BAR(B_KVEMPTY + s), 1);
+        }
+        for (int x = 0; x < HP; ++x) {
+            mbar_init(BAR(B_Y + x), 1);
+            mbar_init(BAR(B_PHI + x), 128);
+            mbar_init(BAR(B_S + x), 1);
+            mbar_init(BAR(B_P + x), 128);
+            mbar_init(BAR(B_O + x), 1);
+        }
+        *abort_flag = 0;
+        mbar_fence_init();
+    }
+    if (warp == Cfg::MMA_WARP) {
+        tmem_alloc(smem_u32(tmem_slot), Cfg::TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (warp == Cfg::PRODUCER_WARP && lane == 0) {
+        tma_prefetch_desc(&map_q);
+        tma_prefetch_desc(&map_k);
+        tma_prefetch_desc(&map_v);
+        tma_prefetch_desc(&map_kh);
+        tma_prefetch_desc(&map_vh);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == Cfg::PRODUCER_WARP) {
+        // ================================================================ TMA producer
+        if (lane == 0) {
+            bool ok = true;
+            int issued = 0;
+            mbar_arrive_expect_tx(BAR(B_QFULL), Cfg::Q_BYTES);
+            for (int x = 0; x < HP; ++x) {
+                const int h = g * p.G + pair * HP + x;
+                for (int rr = 0; rr < DH / 64; ++rr)
+                    tma_load_3d(sQ + x * Cfg::TILE_BYTES + rr * Cfg::REG, &map_q, BAR(B_QFULL), rr * 64, i0,
+                                b * p.H + h);
+            }
+            mbar_arrive_expect_tx(BAR(B_WFULL), HP * Cfg::WQ_BYTES + Cfg::ST_BYTES);
+            for (int x = 0; x < HP; ++x) {
+                const int h = g * p.G + pair * HP + x;
+                for (int rr = 0; rr < DH / 64; ++rr)
+                    tma_load_3d(sStage + x * Cfg::WQ_BYTES + rr * (DF * 128), &map_wq, BAR(B_WFULL), rr * 64, 0, h);
+            }
+            for (int rr = 0; rr < DF / 64; ++rr)
+                tma_load_3d(sStage + HP * Cfg::WQ_BYTES + rr * (DH * 128), &map_st, BAR(B_WFULL), rr * 64, 0,
+                            tslot);
+            trace_word(p.trace, 0, 1);
+            ok = mbar_wait(BAR(B_PRO), 0, abort_flag);  // prologue operands consumed
+            trace_word(p.trace, 0, ok ? 2 : 0xBAD2);
+            for (int j = 0; ok && j < n_tiles; ++j) {
+                const int s = j % Cfg::NS;
+                if (j >= Cfg::NS) {
+                    ok = mbar_wait(BAR(B_KVEMPTY + s), ((j / Cfg::NS) - 1) & 1, abort_flag);
+                    if (!ok) break;
+                }
+                const uint32_t sK = sStage + s * Cfg::STAGE_BYTES, sV = sK + Cfg::TILE_BYTES;
+                const CUtensorMap *mk = j < n_pre ? &map_kh : &map_k;
+                const CUtensorMap *mv = j < n_pre ? &map_vh : &map_v;
+                const int row = j < n_pre ? j * Cfg::BN : lo + (j - n_pre) * Cfg::BN;
+                mbar_arrive_expect_tx(BAR(B_KFULL + s), Cfg::TILE_BYTES);
+                for (int rr = 0; rr < DH / 64; ++rr)
+                    tma_load_3d(sK + rr * Cfg::REG, mk, BAR(B_KFULL + s), rr * 64, row, bg);
+                mbar_arrive_expect_tx(BAR(B_VFULL + s), Cfg::TILE_BYTES);
+                for (int rr = 0; rr < DH / 64; ++rr)
+                    tma_load_3d(sV + rr * Cfg::REG, mv, BAR(B_VFULL + s), rr * 64, row, bg);
+                issued = j + 1;
+                trace_word(p.trace, 0, 0x100 + j);
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                report(p.err, DEV_ERR_TIMEOUT);
+                // drain this CTA's copies still in flight
+                mbar_wait_drain(BAR(B_QFULL), 0, 100000000ull);
+                mbar_wait_drain(BAR(B_WFULL), 0, 100000000ull);
+                for (int j = max(0, issued - Cfg::NS); j < issued; ++j) {
+                    mbar_wait_drain(BAR(B_KFULL + j % Cfg::NS), (j / Cfg::NS) & 1, 100000000ull);
+                    mbar_wait_drain(BAR(B_VFULL + j % Cfg::NS), (j / Cfg::NS) & 1, 100000000ull);
+                }
+            }
+        }
+    } else if (warp == Cfg::MMA_WARP) {
+        // ================================================================ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t ID_Y = idesc_bf16(128, DF, 0, 0);
+            constexpr uint32_t ID_LIN = idesc_bf16(128, DH, 0, 0);
+            constexpr uint32_t ID_S = idesc_bf16(128, 128, 0, 0);
+            constexpr uint32_t ID_PV = idesc_bf16(128, DH, 0, 1);
+            bool ok = mbar_wait(BAR(B_QFULL), 0, abort_flag) && mbar_wait(BAR(B_WFULL), 0, abort_flag);
+            trace_word(p.trace, 1, ok ? 1 : 0xBAD1);
+            if (ok) {
+                tc_fence_after();
+                for (int x = 0; x < HP; ++x) {
+                    const uint32_t aq = sQ + x * Cfg::TILE_BYTES, bw = sStage + x * Cfg::WQ_BYTES;
+                    for (int kk = 0; kk < DH / 16; ++kk)
+                        mma_ss(tmem + Cfg::s_col(x), kmajor_desc(aq, kk, Cfg::REG), kmajor_desc(bw, kk, DF * 128),
+                               ID_Y, kk > 0);
+                    mma_commit(BAR(B_Y + x));
+                }
+                for (int x = 0; x < HP && ok; ++x) {
+                    ok = mbar_wait(BAR(B_PHI + x), 0, abort_flag);
+                    trace_word(p.trace, 1, ok ? 3 + x : 0xBAD3);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t bs = sStage + HP * Cfg::WQ_BYTES;
+                    for (int kk = 0; kk < DF / 16; ++kk)
+                        mma_ts(tmem + Cfg::o_col(x), tmem + Cfg::s_col(x) + kk * 8, kmajor_desc(bs, kk, DH * 128),
+                               ID_LIN, kk > 0);
+                }
+                if (ok) mma_commit(BAR(B_PRO));
+                trace_word(p.trace, 1, 5);
+            }
+            // first score tiles
+            if (ok) ok = mbar_wait(BAR(B_KFULL + 0), 0, abort_flag);
+            if (ok) {
+                tc_fence_after();
+                for (int x = 0; x < HP; ++x) {
+                    for (int kk = 0; kk < DH / 16; ++kk)
+                        mma_ss(tmem + Cfg::s_col(x), kmajor_desc(sQ + x * Cfg::TILE_BYTES, kk, Cfg::REG),
+                               kmajor_desc(sStage, kk, Cfg::REG), ID_S, kk > 0);
+                    mma_commit(BAR(B_S + x));
+                }
+            }
+            for (int j = 0; ok && j < n_tiles; ++j) {
+                const int s = j % Cfg::NS;
+                const uint32_t sV = sStage + s * Cfg::STAGE_BYTES + Cfg::TILE_BYTES;
+                for (int x = 0; x < HP && ok; ++x) {
+                    if (x == 0) ok = mbar_wait(BAR(B_VFULL + s), (j / Cfg::NS) & 1, abort_flag);
+                    if (ok) ok = mbar_wait(BAR(B_P + x), j & 1, abort_flag);
+                    trace_word(p.trace, 1, (ok ? 0x1000u : 0xB000u) + 0x10u * j + x);
+                    if (!ok) break;
+                    tc_fence_after();
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_ts(tmem + Cfg::o_col(x), tmem + Cfg::s_col(x) + kk * 8,
+                               sw128_desc(sV + kk * 2048, Cfg::REG, 1024), ID_PV, 1);
+                    mma_commit(BAR(B_O + x));
+                    if (j + 1 < n_tiles) {
+                        const int s1 = (j + 1) % Cfg::NS;
+                        if (x == 0) ok = mbar_wait(BAR(B_KFULL + s1), ((j + 1) / Cfg::NS) & 1, abort_flag);
+                        if (!ok) break;
+                        tc_fence_after();
+                        const uint32_t sK1 = sStage + s1 * Cfg::STAGE_BYTES;
+                        for (int kk = 0; kk < DH / 16; ++kk)
+                            mma_ss(tmem + Cfg::s_col(x), kmajor_desc(sQ + x * Cfg::TILE_BYTES, kk, Cfg::REG),
+                                   kmajor_desc(sK1, kk, Cfg::REG), ID_S, kk > 0);
+                        mma_commit(BAR(B_S + x));
+                    }
+                }
+                if (ok) mma_commit(BAR(B_KVEMPTY + s));
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                report(p.err, DEV_ERR_TIMEOUT);
+            }
+            // drain every MMA this thread issued before TMEM is released
+            mma_commit(BAR(B_DRAIN));
+            mbar_wait_drain(BAR(B_DRAIN), 0, 100000000ull);
+        }
+    } else {
+        // ================================================================ softmax warpgroups
+        const int x = warp >> 2;                       // head tile
+        const int r = (warp & 3) * 32 + lane;          // row in the tile = TMEM lane
+        const int i = i0 + r;
+        const int h = g * p.G + pair * HP + x;
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        const uint32_t tS = tmem + lane_off + Cfg::s_col(x);
+        const uint32_t tO = tmem + lane_off + Cfg::o_col(x);
+        bool ok = true;
+
+        // ---- prologue: phi(q) from Y = Q Wq^T
+        float m_run, l_run;
+        {
+            ok = warp_all(mbar_wait(BAR(B_QFULL), 0, abort_flag) && mbar_wait(BAR(B_Y + x), 0, abort_flag));
+            if (lane == 0) trace_word(p.trace, 2 + warp, ok ? 1 : 0xBAD1);
+            float y[DF];
+            if (ok) {
+                tc_fence_after();
+#pragma unroll
+                for (int c = 0; c < DF / 32; ++c) {
+                    uint32_t u[32];
+                    tmem_ld32(tS + c * 32, u);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) y[c * 32 + e] = __uint_as_float(u[e]);
+                }
+            }
+            // ||q||^2 from the swizzled Q tile in shared memory
+            float qq = 0.f;
+            const uint8_t *qrow = smem + x * Cfg::TILE_BYTES + r * 128;
+#pragma unroll
+            for (int rr = 0; rr < DH / 64; ++rr) {
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    const uint4 u = *reinterpret_cast<const uint4 *>(qrow + rr * Cfg::REG + ((ch ^ (r & 7)) << 4));
+                    const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = __bfloat1622float2(h2[e]);
+                        qq = fmaf(f.x, f.x, qq);
+                        qq = fmaf(f.y, f.y, qq);
+                    }
+                }
+            }
+            float ymax = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < DF; ++c) ymax = fmaxf(ymax, y[c]);
+            float ee = 0.f;
+#pragma unroll
+            for (int c = 0; c < DF; ++c) {
+                y[c] = ex2((y[c] - ymax) * kLog2e);
+                ee = fmaf(y[c], y[c], ee);
+            }
+            const float f = sqrtf(qq) * rsqrtf(ee);
+            const float *zt = p.z + (size_t)tslot * DF;
+            float bden = 0.f;
+#pragma unroll
+            for (int c = 0; c < DF; ++c) {
+                y[c] *= f;
+                bden = fmaf(y[c], __ldg(zt + c), bden);
+            }
+            if (ok) {
+#pragma unroll
+                for (int c = 0; c < DF / 64; ++c) {
+                    uint32_t u[32];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) u[e] = pack_bf16x2(y[c * 64 + 2 * e], y[c * 64 + 2 * e + 1]);
+                    tmem_st32(tS + c * 32, u);
+                }
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            mbar_arrive(BAR(B_PHI + x));
+            if (lane == 0) trace_word(p.trace, 2 + warp, 2);
+            if (bden > 0.f) {
+                m_run = 0.f;
+                l_run = bden;
+            } else {
+                m_run = -INFINITY;
+                l_run = 0.f;
+            }
+        }
+
+        // ---- main loop over key tiles
+        for (int j = 0; ok && j < n_tiles; ++j) {
+            ok = warp_all(mbar_wait(BAR(B_S + x), j & 1, abort_flag));
+            if (lane == 0) trace_word(p.trace, 2 + warp, (ok ? 0x100u : 0xB00u) + 0x10u * j + 1);
+            if (!ok) break;
+            tc_fence_after();
+            float sv[128];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t u[32];
+                tmem_ld32(tS + c * 32, u);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) sv[c * 32 + e] = __uint_as_float(u[e]);
+            }
+            tmem_wait_ld();
+            // masks: ragged last tile of the kept prefix, causal diagonal tile
+            int limit = 128;
+            if (j < n_pre) limit = min(128, nk - j * Cfg::BN);
+            else if (j == n_tiles - 1) limit = r + 1;  // keys i0 .. i0+r
+#pragma unroll
+            for (int c = 0; c < 128; ++c)
+                if (c >= limit) sv[c] = -INFINITY;
+            float mx0 = sv[0], mx1 = sv[1], mx2 = sv[2], mx3 = sv[3];
+#pragma unroll
+            for (int c = 4; c < 128; c += 4) {
+                mx0 = fmaxf(mx0, sv[c]);
+                mx1 = fmaxf(mx1, sv[c + 1]);
+                mx2 = fmaxf(mx2, sv[c + 2]);
+                mx3 = fmaxf(mx3, sv[c + 3]);
+            }
+            const float mnew = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * p.scale_log2;
+            // Lazy rescale: a row moves its reference max only when the max grows by more than 2^8.
+            // The O rescale uses warp-collective tcgen05.ld/st, so the warp takes it together when
+            // any of its rows needs it (rows that do not keep alpha = 1).
+            const bool need = mnew > m_run + 8.0f;
+            const float alpha = need ? ex2(m_run - mnew) : 1.f;
+            const bool touch_o = need && m_run != -INFINITY;  // O is still zero while m_run = -inf
+            if (__any_sync(0xffffffffu, touch_o)) {
+                ok = warp_all(j == 0 ? mbar_wait(BAR(B_PRO), 0, abort_flag)
+                                     : mbar_wait(BAR(B_O + x), (j - 1) & 1, abort_flag));
+                if (!ok) break;
+                tc_fence_after();
+                const float f = touch_o ? alpha : 1.f;
+#pragma unroll
+                for (int c = 0; c < DH / 32; ++c) {
+                    uint32_t u[32];
+                    tmem_ld32(tO + c * 32, u);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * f);
+                    tmem_st32(tO + c * 32, u);
+                }
+                tmem_wait_st();
+            }
+            if (need) {
+                l_run *= alpha;
+                m_run = mnew;
+            }
+            const float neg = -m_run;
+            float ls0 = 0.f, ls1 = 0.f;
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                uint32_t u[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const float p0 = ex2(fmaf(sv[c * 64 + 2 * e], p.scale_log2, neg));
+                    const float p1 = ex2(fmaf(sv[c * 64 + 2 * e + 1], p.scale_log2, neg));
+                    ls0 += p0;
+                    ls1 += p1;
+                    u[e] = pack_bf16x2(p0, p1);
+                }
+                tmem_st32(tS + c * 32, u);
+            }
+            l_run += ls0 + ls1;
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(BAR(B_P + x));
+            if (lane == 0) trace_word(p.trace, 2 + warp, 0x100u + 0x10u * j + 2);
+        }
+        // ---- epilogue: o = O / l
+        ok = warp_all(ok && mbar_wait(BAR(B_O + x), (n_tiles - 1) & 1, abort_flag));
+        if (lane == 0) trace_word(p.trace, 2 + warp, ok ? 0xE00 : 0xBADE);
+        if (ok) {
+            tc_fence_after();
+            const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+            __nv_bfloat16 *orow = p.o + (((size_t)b * p.H + h) * p.N + i) * DH;
+#pragma unroll
+            for (int c = 0; c < DH / 32; ++c) {
+                uint32_t u[32];
+                tmem_ld32(tO + c * 32, u);
+                tmem_wait_ld();
+                if (i < p.N) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
+#pragma unroll
+                    for (int v4 = 0; v4 < 4; ++v4) {
+                        uint4 w;
+                        w.x = pack_bf16x2(__uint_as_float(u[8 * v4 + 0]) * inv, __uint_as_float(u[8 * v4 + 1]) * inv);
+                        w.y = pack_bf16x2(__uint_as_float(u[8 * v4 + 2]) * inv, __uint_as_float(u[8 * v4 + 3]) * inv);
+                        w.z = pack_bf16x2(__uint_as_float(u[8 * v4 + 4]) * inv, __uint_as_float(u[8 * v4 + 5]) * inv);
+                        w.w = pack_bf16x2(__uint_as_float(u[8 * v4 + 6]) * inv, __uint_as_float(u[8 * v4 + 7]) * inv);
+                        dst[v4] = w;
+                    }
+                }
+            }
+        }
+        if (!ok) {
+            *abort_flag = 1;
+            report(p.err, DEV_ERR_TIMEOUT);
+        }
+    }
+
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (threadIdx.x == 0) trace_word(p.trace, 14, 0xD0E);
+    if (warp == Cfg::MMA_WARP) tmem_dealloc(tmem, Cfg::TMEM_COLS);
+    if (threadIdx.x == 0) trace_word(p.trace, 15, 0xF1F);
+}
+
+// ------------------------------------------------------------------ small helper kernels
+// Wq [H, d, D] -> Wq^T [H, D, d] (bf16), the K-major operand of Y = Q Wq.
+__global__ void transpose_wq_kernel(const __nv_bfloat16 *__restrict__ wq, __nv_bfloat16 *__restrict__ wqt, int H,
+                                    int d, int D) {
+    const size_t n = (size_t)H * d * D;
+    for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < n; e += (size_t)gridDim.x * blockDim.x) {
+        const int h = (int)(e / ((size_t)d * D));
+        const int rem = (int)(e % ((size_t)d * D));
+        const int c = rem / d, a = rem % d;  // output [h][c][a]
+        wqt[e] = wq[((size_t)h * d + a) * D + c];
+    }
+}
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+// bf16 tensor [d2][d1][d0] (d0 innermost), box {64, box1, 1}, 128-byte swizzle, zero fill out of range.
+bool make_map(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box1) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn || ((uintptr_t)base & 15)) return false;
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+    cuuint32_t box[3] = {64, box1, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+unsigned *debug_trace_words();
+namespace {
+
+template <int DH, int DF, int HP>
+cudaError_t launch_merge_cfg(const Dims &s, const void *q, const void *k, const void *v, const void *wqt,
+                             const void *khat, const void *vhat, const void *st_t, const float *z, void *o,
+                             unsigned *err, cudaStream_t st) {
+    using Cfg = MergeCfg<DH, DF, HP>;
+    const int T = s.T();
+    CUtensorMap mq, mk, mv, mkh, mvh, mw, ms;
+    const uint64_t khrows = (uint64_t)T * s.k > 0 ? (uint64_t)T * s.k : 1;
+    bool ok = make_map(&mq, q, DH, s.N, (uint64_t)s.B * s.H, 128) && make_map(&mk, k, DH, s.N, (uint64_t)s.B * s.Hkv, 128) &&
+              make_map(&mv, v, DH, s.N, (uint64_t)s.B * s.Hkv, 128) &&
+              make_map(&mkh, khat, DH, khrows, (uint64_t)s.B * s.Hkv, 128) &&
+              make_map(&mvh, vhat, DH, khrows, (uint64_t)s.B * s.Hkv, 128) &&
+              make_map(&mw, wqt, DH, DF, s.H, DF) &&
+              make_map(&ms, st_t, DF, DH, (uint64_t)s.B * s.Hkv * (T + 1), DH);
+    if (!ok) return cudaErrorInvalidValue;
+    MergeParams prm;
+    prm.B = s.B;
+    prm.H = s.H;
+    prm.Hkv = s.Hkv;
+    prm.N = s.N;
+    prm.C = s.C;
+    prm.k = s.k;
+    prm.w = s.w;
+    prm.G = s.G();
+    prm.T = T;
+    prm.scale_log2 = s.scale * kLog2e;
+    prm.z = z;
+    prm.o = static_cast<__nv_bfloat16 *>(o);
+    prm.err = err;
+    prm.n_qtiles = (s.N + 127) / 128;
+    prm.pairs = s.G() / HP;
+    prm.trace = debug_trace_words();
+    auto kern = merge_tc_kernel<DH, DF, HP>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)prm.n_qtiles * s.B * s.Hkv * prm.pairs;
+    kern<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(mq, mk, mv, mkh, mvh, mw, ms, prm);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+static unsigned *g_debug_trace = nullptr;
+unsigned *debug_trace_words() { return g_debug_trace; }
+void set_debug_trace_words(unsigned *p) { g_debug_trace = p; }
+
+bool tc_merge_supported(const Dims &s) {
+    return s.bf16 && s.w > 0 && (s.d == 64 || s.d == 128) && (s.D == 64 || s.D == 128) && s.C % 128 == 0 &&
+           s.N > 0 && encode_fn() != nullptr;
+}
+
+cudaError_t launch_wq_transpose(const Dims &s, const void *wq, void *wqt, cudaStream_t st) {
+    const size_t n = (size_t)s.H * s.d * s.D;
+    const unsigned blocks = (unsigned)std::min<size_t>((n + 255) / 256, 4096);
+    transpose_wq_kernel<<<blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(wq),
+                                                 static_cast<__nv_bfloat16 *>(wqt), s.H, s.d, s.D);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_merge_tc(const Dims &s, const void *q, const void *k, const void *v, const void *wqt,
+                            const void *khat, const void *vhat, const void *st_t, const float *z, void *o,
+                            unsigned *err, cudaStream_t st) {
+    const bool pair = s.G() % 2 == 0;
+#define STILL_MERGE_CASE(DH, DF)                                                                            \
+    if (s.d == DH && s.D == DF)                                                                             \
+        return pair ? launch_merge_cfg<DH, DF, 2>(s, q, k, v, wqt, khat, vhat, st_t, z, o, err, st)        \
+                    : launch_merge_cfg<DH, DF, 1>(s, q, k, v, wqt, khat, vhat, st_t, z, o, err, st);
+    STILL_MERGE_CASE(64, 64)
+    STILL_MERGE_CASE(128, 128)
+    STILL_MERGE_CASE(64, 128)
+    STILL_MERGE_CASE(128, 64)
+#undef STILL_MERGE_CASE
     return cudaErrorNotSupported;
 }
+
 bool tc_saliency_supported(const Dims &) { return false; }
 cudaError_t launch_saliency_tc(const Dims &, const void *, const void *, float *, float *, unsigned *, cudaStream_t) {
     return cudaErrorNotSupported;

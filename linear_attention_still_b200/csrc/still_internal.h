@@ -43,7 +43,7 @@ cudaError_t launch_topk_gather(const Dims &s, const float *r, int32_t *idx, cons
 cudaError_t launch_npmap(int rows, int Hx, int N, int d, int D, int bf16, const void *x, const void *W, float *phi,
                          cudaStream_t st);
 cudaError_t launch_linear_state(const Dims &s, const float *phik, const void *v, const int32_t *idx, float *S,
-                                float *z, unsigned *err, cudaStream_t st);
+                                float *z, void *st_t, unsigned *err, cudaStream_t st);
 cudaError_t launch_merge_generic(const Dims &s, const void *q, const void *k, const void *v, const void *Wq,
                                  const void *khat, const void *vhat, const float *S, const float *z,
                                  const float *phik, void *o, cudaStream_t st);

@@ -21,7 +21,7 @@ STATUS = {0: "STILL_OK", 1: "STILL_ERR_INVALID_ARG", 2: "STILL_ERR_UNSUPPORTED",
 EXPORTS = ("still_status_string", "still_saliency", "still_select_topk", "still_npmap",
            "still_prefill_workspace_bytes", "still_prefill_workspace_layout", "still_hybrid_prefill",
            "still_decode_state_bytes", "still_decode_init", "still_decode_step", "still_get_device_status",
-           "still_launch_count", "still_timing_enable", "still_timing_read")
+           "still_launch_count", "still_timing_enable", "still_timing_read", "still_debug_set_trace")
 
 
 class StillError(RuntimeError):
@@ -36,7 +36,7 @@ class still_dims(ct.Structure):
 
 
 class still_ws_layout(ct.Structure):
-    _fields_ = [(n, ct.c_size_t) for n in ("r", "idx", "khat", "vhat", "S", "z", "phik", "total")]
+    _fields_ = [(n, ct.c_size_t) for n in ("r", "idx", "khat", "vhat", "S", "z", "phik", "wqt", "st", "total")]
 
 
 if not os.path.exists(_LIB_PATH):
@@ -59,6 +59,7 @@ _SIG = {
     "still_get_device_status": ([_P], ct.c_int),
     "still_launch_count": ([], ct.c_uint64),
     "still_timing_enable": ([ct.c_int], ct.c_int),
+    "still_debug_set_trace": ([_P], None),
     "still_timing_read": ([ct.POINTER(ct.c_double), ct.POINTER(ct.c_int), ct.c_int], ct.c_int),
 }
 for _name, (_args, _res) in _SIG.items():
@@ -163,6 +164,11 @@ def still_get_device_status(stream=None) -> int:
 
 def still_launch_count() -> int:
     return int(_lib.still_launch_count())
+
+
+def still_debug_set_trace(words=None):
+    """Diagnostics: progress words of the tensor-core kernels go to `words` (pinned tensor or None)."""
+    _lib.still_debug_set_trace(_ptr(words))
 
 
 TIMING_CLASSES = ("saliency", "topk_gather", "npmap", "linear_state", "merge", "state_export")
