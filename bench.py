@@ -45,7 +45,7 @@ METRIC = "STILL hybrid-attn prefill tokens/s per layer at 16K/64K; % of roofline
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=100)
+    p.add_argument("--steps", type=int, default=300)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
@@ -101,7 +101,7 @@ class ClockSampler:
         self.gpu_id = gpu_id
 
     def start(self):
-        cmd = ["nvidia-smi", f"--query-gpu={','.join(self.FIELDS)}", "--format=csv,noheader,nounits", "-lms", "100"]
+        cmd = ["nvidia-smi", f"--query-gpu={','.join(self.FIELDS)}", "--format=csv,noheader,nounits", "-lms", "20"]
         if self.gpu_id:
             cmd += ["-i", self.gpu_id]
         try:

@@ -78,7 +78,9 @@ STILL_API const char *still_status_string(int status);
  *   k    [B,Hkv,N,d] dtype
  *   r_kv [B,Hkv,N]   fp32 out
  *   r_q  [B,H,N]     fp32 out, may be NULL (per-query-head sigma)
- * Requires w >= 1.
+ * Requires w >= 1.  bf16 with d in {64, 128} and w a multiple of 128 runs on
+ * the tensor cores when r_q is given or G <= 2 (r_q doubles as the per-head
+ * buffer); otherwise the SIMT kernel computes the same scores.
  */
 STILL_API still_status still_saliency(const still_dims *dims, const void *q, const void *k, float *r_kv, float *r_q,
                             void *stream);
@@ -117,6 +119,7 @@ typedef struct {
     size_t S;      /* fp32  [B,Hkv,T+1,D,d]    linear state seen by chunk t    */
     size_t z;      /* fp32  [B,Hkv,T+1,D]      linear normaliser seen by chunk t */
     size_t phik;   /* fp32  [B,Hkv,N,D]        NP-Map features of the keys     */
+    size_t sig;    /* fp32  [B,H,N]            per-query-head saliency (bf16 tensor-core path) */
     size_t wqt;    /* bf16  [H,D,d]            Wq transposed (bf16 tensor-core path) */
     size_t st;     /* bf16  [B,Hkv,T+1,d,D]    S_t transposed (bf16 tensor-core path) */
     size_t total;

@@ -93,7 +93,9 @@ still_ws_layout ws_layout(const Dims &s) {
     off = al256(off + BK * (T + 1) * s.D * 4);
     L.phik = off;
     off = al256(off + BK * s.N * s.D * 4);
-    const bool tc = s.bf16 != 0;  // transposed bf16 operands of the tensor-core merge
+    const bool tc = s.bf16 != 0;  // per-head scores and transposed bf16 operands of the tensor-core path
+    L.sig = off;
+    off = al256(off + (tc ? (size_t)s.B * s.H * s.N * 4 : 0));
     L.wqt = off;
     off = al256(off + (tc ? (size_t)s.H * s.D * s.d * 2 : 0));
     L.st = off;
@@ -171,7 +173,7 @@ still_status still_saliency(const still_dims *dims, const void *q, const void *k
     if ((long long)s.B * s.N == 0) return STILL_OK;
     if (!q || !k || !r_kv || !aligned16(q) || !aligned16(k) || !aligned16(r_kv)) return STILL_ERR_INVALID_ARG;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    if (tc_saliency_supported(s)) {
+    if (tc_saliency_supported(s) && (r_q || s.G() <= 2)) {
         unsigned *err = device_error_word();
         STILL_LAUNCH(launch_saliency_tc(s, q, k, r_kv, r_q, err, cs));
     } else {
@@ -268,7 +270,8 @@ still_status still_hybrid_prefill(const still_dims *dims, const void *q, const v
     // 1. Self-Saliency Score per KV group
     if (need_r) {
         TimingScope ts(0, cs);
-        if (tc_saliency_supported(s)) STILL_LAUNCH(launch_saliency_tc(s, q, k, r, nullptr, err, cs));
+        if (tc_saliency_supported(s))
+            STILL_LAUNCH(launch_saliency_tc(s, q, k, r, reinterpret_cast<float *>(ws + W.sig), err, cs));
         else STILL_LAUNCH(launch_saliency_generic(s, q, k, r, nullptr, cs));
     }
     // 2. per-chunk top-k and gather of the kept rows

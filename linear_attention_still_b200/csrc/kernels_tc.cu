@@ -501,6 +501,253 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
     if (threadIdx.x == 0) trace_word(p.trace, 15, 0xF1F);
 }
 
+// ------------------------------------------------------------------ banded saliency
+// Self-Saliency Score ([p1] "Self-Saliency Score"; [p4] "Approach"): for query row i of head h,
+// sigma = softplus(s_ii - LSE_{j in [i-w+1, i-1]} s_ij) = -ln(1 - p_ii), +inf for an empty band.
+// One CTA = (b, g, HP heads, 128 queries).  Key tiles cover [max(0, i0-w), i0+127] (w is a multiple
+// of 128): the first tile of a full window masks c <= r (key i0-w+c is below row r's band), the
+// diagonal tile masks c >= r and takes c == r as s_ii.  S = Q K^T in TMEM, double-buffered per head so
+// the next tile's MMA overlaps this tile's exponentials; per row an online log-sum-exp in registers.
+// Writes sigma per query head; the group mean is taken by mean_heads_kernel.
+template <int DH, int HP>
+struct SalCfg {
+    static constexpr int REG = 128 * 128;
+    static constexpr int TILE_BYTES = 128 * DH * 2;
+    static constexpr int Q_BYTES = HP * TILE_BYTES;
+    static constexpr int NS = DH == 128 ? 4 : 6;
+    static constexpr int NUM_BARS = 2 + 2 * NS + 4 * HP;
+    static constexpr int TMEM_SLOT_OFF = 8 * NUM_BARS;
+    static constexpr int ABORT_OFF = TMEM_SLOT_OFF + 8;
+    static constexpr int BAR_BYTES = 256;
+    static_assert(ABORT_OFF + 8 <= BAR_BYTES, "barrier area overflow");
+    static constexpr int SIG_BYTES = HP * 128 * 4;  // per-row sigma of each head (group mean)
+    static constexpr int SMEM = Q_BYTES + NS * TILE_BYTES + BAR_BYTES + SIG_BYTES + 1024;
+    static constexpr int THREADS = 128 * HP + 64;
+    static constexpr int PRODUCER_WARP = 4 * HP;
+    static constexpr int MMA_WARP = 4 * HP + 1;
+    static constexpr int TMEM_COLS = HP == 2 ? 512 : 256;
+    __host__ __device__ static constexpr int s_col(int x, int buf) { return (x * 2 + buf) * 128; }
+};
+
+struct SalParams {
+    int B, H, Hkv, N, w, G, pairs, n_qtiles;
+    float scale_log2;
+    float *sigma;      // [B,H,N] or nullptr
+    float *r_kv;       // [B,Hkv,N], written here when the CTA holds the whole group (pairs == 1)
+    unsigned *err;
+};
+
+template <int DH, int HP>
+__global__ void __launch_bounds__(SalCfg<DH, HP>::THREADS, 1)
+    saliency_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+                       const SalParams p) {
+    using Cfg = SalCfg<DH, HP>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t sQ = sbase, sK = sbase + Cfg::Q_BYTES;
+    uint8_t *bar_area = smem + Cfg::Q_BYTES + Cfg::NS * Cfg::TILE_BYTES;
+    const uint32_t sBar = smem_u32(bar_area);
+    auto BAR = [&](int i) { return sBar + 8u * i; };
+    const int B_QFULL = 0, B_DRAIN = 1, B_KFULL = 2, B_KEMPTY = 2 + Cfg::NS;
+    const int B_SFULL = 2 + 2 * Cfg::NS, B_SEMPTY = B_SFULL + 2 * HP;  // [x*2 + buf]
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_area + Cfg::TMEM_SLOT_OFF);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bar_area + Cfg::ABORT_OFF);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    const int per_qt = p.B * p.Hkv * p.pairs;
+    const int qt = p.n_qtiles - 1 - (int)(blockIdx.x / per_qt);
+    const int rem = blockIdx.x % per_qt;
+    const int pair = rem % p.pairs;
+    const int bg = rem / p.pairs;
+    const int b = bg / p.Hkv, g = bg % p.Hkv;
+    const int i0 = qt * 128;
+    const int kbase = max(0, i0 - p.w);
+    const int n_tiles = (i0 - kbase) / 128 + 1;
+    const bool low_mask_first = i0 >= p.w;  // first tile starts at i0 - w
+
+    if (threadIdx.x == 0) {
+        mbar_init(BAR(B_QFULL), 1);
+        mbar_init(BAR(B_DRAIN), 1);
+        for (int s = 0; s < Cfg::NS; ++s) {
+            mbar_init(BAR(B_KFULL + s), 1);
+            mbar_init(BAR(B_KEMPTY + s), 1);
+        }
+        for (int e = 0; e < 2 * HP; ++e) {
+            mbar_init(BAR(B_SFULL + e), 1);
+            mbar_init(BAR(B_SEMPTY + e), 128);
+        }
+        *abort_flag = 0;
+        mbar_fence_init();
+    }
+    if (warp == Cfg::MMA_WARP) {
+        tmem_alloc(smem_u32(tmem_slot), Cfg::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == Cfg::PRODUCER_WARP) {
+        if (lane == 0) {
+            bool ok = true;
+            int issued = 0;
+            mbar_arrive_expect_tx(BAR(B_QFULL), Cfg::Q_BYTES);
+            for (int x = 0; x < HP; ++x) {
+                const int h = g * p.G + pair * HP + x;
+                for (int rr = 0; rr < DH / 64; ++rr)
+                    tma_load_3d(sQ + x * Cfg::TILE_BYTES + rr * Cfg::REG, &map_q, BAR(B_QFULL), rr * 64, i0,
+                                b * p.H + h);
+            }
+            for (int j = 0; j < n_tiles; ++j) {
+                const int s = j % Cfg::NS;
+                if (j >= Cfg::NS) {
+                    ok = mbar_wait(BAR(B_KEMPTY + s), ((j / Cfg::NS) - 1) & 1, abort_flag);
+                    if (!ok) break;
+                }
+                mbar_arrive_expect_tx(BAR(B_KFULL + s), Cfg::TILE_BYTES);
+                for (int rr = 0; rr < DH / 64; ++rr)
+                    tma_load_3d(sK + s * Cfg::TILE_BYTES + rr * Cfg::REG, &map_k, BAR(B_KFULL + s), rr * 64,
+                                kbase + j * 128, bg);
+                issued = j + 1;
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                report(p.err, DEV_ERR_TIMEOUT);
+                mbar_wait_drain(BAR(B_QFULL), 0, 100000000ull);
+                for (int j = max(0, issued - Cfg::NS); j < issued; ++j)
+                    mbar_wait_drain(BAR(B_KFULL + j % Cfg::NS), (j / Cfg::NS) & 1, 100000000ull);
+            }
+        }
+    } else if (warp == Cfg::MMA_WARP) {
+        if (lane == 0) {
+            constexpr uint32_t ID_S = idesc_bf16(128, 128, 0, 0);
+            bool ok = mbar_wait(BAR(B_QFULL), 0, abort_flag);
+            for (int j = 0; ok && j < n_tiles; ++j) {
+                const int s = j % Cfg::NS, buf = j & 1;
+                ok = mbar_wait(BAR(B_KFULL + s), (j / Cfg::NS) & 1, abort_flag);
+                for (int x = 0; x < HP && ok; ++x) {
+                    if (j >= 2) ok = mbar_wait(BAR(B_SEMPTY + 2 * x + buf), ((j >> 1) - 1) & 1, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+                    for (int kk = 0; kk < DH / 16; ++kk)
+                        mma_ss(tmem + Cfg::s_col(x, buf), kmajor_desc(sQ + x * Cfg::TILE_BYTES, kk, Cfg::REG),
+                               kmajor_desc(sK + s * Cfg::TILE_BYTES, kk, Cfg::REG), ID_S, kk > 0);
+                    mma_commit(BAR(B_SFULL + 2 * x + buf));
+                }
+                if (ok) mma_commit(BAR(B_KEMPTY + s));
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                report(p.err, DEV_ERR_TIMEOUT);
+            }
+            mma_commit(BAR(B_DRAIN));
+            mbar_wait_drain(BAR(B_DRAIN), 0, 100000000ull);
+        }
+    } else {
+        const int x = warp >> 2;
+        const int r = (warp & 3) * 32 + lane;
+        const int i = i0 + r;
+        const int h = g * p.G + pair * HP + x;
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        float m2 = -INFINITY, l = 0.f, sdiag = 0.f;
+        bool ok = true;
+        for (int j = 0; j < n_tiles; ++j) {
+            const int buf = j & 1;
+            ok = warp_all(mbar_wait(BAR(B_SFULL + 2 * x + buf), (j >> 1) & 1, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            float sv[128];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t u[32];
+                tmem_ld32(tmem + lane_off + Cfg::s_col(x, buf) + c * 32, u);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) sv[c * 32 + e] = __uint_as_float(u[e]);
+            }
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(BAR(B_SEMPTY + 2 * x + buf));  // the buffer can take tile j+2
+            // band [lo_c, hi_c): keys kbase + j*128 + c
+            int lo_c = 0, hi_c = 128;
+            if (j == 0 && low_mask_first) lo_c = r + 1;
+            if (j == n_tiles - 1) {
+                hi_c = r;
+#pragma unroll
+                for (int c = 0; c < 128; ++c)
+                    if (c == r) sdiag = sv[c];  // unrolled select keeps sv in registers
+            }
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 128; ++c) {
+                const bool in = c >= lo_c && c < hi_c;
+                sv[c] = in ? sv[c] * p.scale_log2 : -INFINITY;
+                mx = fmaxf(mx, sv[c]);
+            }
+            if (mx > m2) {
+                l *= ex2(m2 - mx);
+                m2 = mx;
+            }
+            if (m2 != -INFINITY) {
+                float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+                for (int c = 0; c < 128; c += 4) {
+                    a0 += ex2(sv[c] - m2);
+                    a1 += ex2(sv[c + 1] - m2);
+                    a2 += ex2(sv[c + 2] - m2);
+                    a3 += ex2(sv[c + 3] - m2);
+                }
+                l += (a0 + a1) + (a2 + a3);
+            }
+        }
+        // ln-domain: LSE = (m2 + log2 l) ln 2, s_ii = sdiag * tau
+        float sigma = INFINITY;
+        if (m2 != -INFINITY) {
+            const float lse = (m2 + __log2f(l)) * 0.6931471805599453f;
+            sigma = softplus_f(sdiag * (p.scale_log2 * 0.6931471805599453f) - lse);
+        }
+        if (!ok) {
+            *abort_flag = 1;
+            report(p.err, DEV_ERR_TIMEOUT);
+        }
+        if (ok && p.sigma && i < p.N) p.sigma[((size_t)b * p.H + h) * p.N + i] = sigma;
+        if (p.pairs == 1) {
+            // the CTA holds every head of the group: mean over heads, in head order
+            float *ssig = reinterpret_cast<float *>(bar_area + Cfg::BAR_BYTES);
+            ssig[x * 128 + r] = sigma;
+            asm volatile("bar.sync 1, %0;" ::"r"(128 * HP) : "memory");
+            if (ok && x == 0 && i < p.N) {
+                float acc = 0.f;
+#pragma unroll
+                for (int xx = 0; xx < HP; ++xx) acc += ssig[xx * 128 + r];
+                p.r_kv[(size_t)bg * p.N + i] = acc / (float)HP;
+            }
+        }
+    }
+
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == Cfg::MMA_WARP) tmem_dealloc(tmem, Cfg::TMEM_COLS);
+}
+
+// r[b,g,i] = mean over the G heads of g of sigma[b,h,i], summed in head order.
+__global__ void mean_heads_kernel(const float *__restrict__ sigma, float *__restrict__ r, int B, int H, int Hkv,
+                                  int N) {
+    const int G = H / Hkv;
+    const size_t total = (size_t)B * Hkv * N;
+    for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < total; e += (size_t)gridDim.x * blockDim.x) {
+        const size_t bg = e / N;
+        const int i = (int)(e % N);
+        const size_t b = bg / Hkv, g = bg % Hkv;
+        float acc = 0.f;
+        for (int hh = 0; hh < G; ++hh) acc += sigma[((b * H) + g * G + hh) * N + i];
+        r[e] = acc / (float)G;
+    }
+}
+
 // ------------------------------------------------------------------ small helper kernels
 // Wq [H, d, D] -> Wq^T [H, D, d] (bf16), the K-major operand of Y = Q Wq.
 __global__ void transpose_wq_kernel(const __nv_bfloat16 *__restrict__ wq, __nv_bfloat16 *__restrict__ wqt, int H,
@@ -623,9 +870,57 @@ cudaError_t launch_merge_tc(const Dims &s, const void *q, const void *k, const v
     return cudaErrorNotSupported;
 }
 
-bool tc_saliency_supported(const Dims &) { return false; }
-cudaError_t launch_saliency_tc(const Dims &, const void *, const void *, float *, float *, unsigned *, cudaStream_t) {
-    return cudaErrorNotSupported;
+bool tc_saliency_supported(const Dims &s) {
+    return s.bf16 && s.w > 0 && (s.d == 64 || s.d == 128) && s.w % 128 == 0 && s.N > 0 && encode_fn() != nullptr;
+}
+
+template <int DH, int HP>
+static cudaError_t launch_saliency_cfg(const Dims &s, const void *q, const void *k, float *r_kv, float *sigma,
+                                       unsigned *err, cudaStream_t st) {
+    using Cfg = SalCfg<DH, HP>;
+    CUtensorMap mq, mk;
+    if (!make_map(&mq, q, DH, s.N, (uint64_t)s.B * s.H, 128) || !make_map(&mk, k, DH, s.N, (uint64_t)s.B * s.Hkv, 128))
+        return cudaErrorInvalidValue;
+    SalParams prm;
+    prm.B = s.B;
+    prm.H = s.H;
+    prm.Hkv = s.Hkv;
+    prm.N = s.N;
+    prm.w = s.w;
+    prm.G = s.G();
+    prm.pairs = s.G() / HP;
+    prm.n_qtiles = (s.N + 127) / 128;
+    prm.scale_log2 = s.scale * kLog2e;
+    prm.sigma = sigma;
+    prm.r_kv = r_kv;
+    prm.err = err;
+    auto kern = saliency_tc_kernel<DH, HP>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)prm.n_qtiles * s.B * s.Hkv * prm.pairs;
+    kern<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(mq, mk, prm);
+    return cudaGetLastError();
+}
+
+// r_kv: [B,Hkv,N]; sigma: [B,H,N] per-head scores (may be nullptr only when G <= 2, where one CTA
+// holds the whole group and writes the mean itself).
+cudaError_t launch_saliency_tc(const Dims &s, const void *q, const void *k, float *r_kv, float *sigma, unsigned *err,
+                               cudaStream_t st) {
+    const bool pair = s.G() % 2 == 0;
+    if (!sigma && s.G() > 2) return cudaErrorInvalidValue;
+    cudaError_t e;
+    if (s.d == 64)
+        e = pair ? launch_saliency_cfg<64, 2>(s, q, k, r_kv, sigma, err, st)
+                 : launch_saliency_cfg<64, 1>(s, q, k, r_kv, sigma, err, st);
+    else
+        e = pair ? launch_saliency_cfg<128, 2>(s, q, k, r_kv, sigma, err, st)
+                 : launch_saliency_cfg<128, 1>(s, q, k, r_kv, sigma, err, st);
+    if (e != cudaSuccess) return e;
+    if (s.G() <= 2) return cudaSuccess;  // the kernel wrote the group mean
+    const size_t total = (size_t)s.B * s.Hkv * s.N;
+    const unsigned blocks = (unsigned)std::min<size_t>((total + 255) / 256, 8192);
+    mean_heads_kernel<<<blocks, 256, 0, st>>>(sigma, r_kv, s.B, s.H, s.Hkv, s.N);
+    return cudaGetLastError();
 }
 
 }  // namespace still
