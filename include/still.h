@@ -121,6 +121,7 @@ typedef struct {
     size_t phik;   /* fp32  [B,Hkv,N,D]        NP-Map features of the keys     */
     size_t sig;    /* fp32  [B,H,N]            per-query-head saliency (bf16 tensor-core path) */
     size_t wqt;    /* bf16  [H,D,d]            Wq transposed (bf16 tensor-core path) */
+    size_t wkt;    /* bf16  [Hkv,D,d]          Wk transposed (bf16 tensor-core path) */
     size_t st;     /* bf16  [B,Hkv,T+1,d,D]    S_t transposed (bf16 tensor-core path) */
     size_t total;
 } still_ws_layout;

@@ -12,7 +12,10 @@ namespace still {
 cudaError_t launch_gather(const Dims &s, const int32_t *idx, const void *k, const void *v, void *khat, void *vhat,
                           unsigned *err, cudaStream_t st);
 bool tc_merge_supported(const Dims &s);
-cudaError_t launch_wq_transpose(const Dims &s, const void *wq, void *wqt, cudaStream_t st);
+cudaError_t launch_w_transpose(int Hx, int d, int D, const void *w, void *wt, cudaStream_t st);
+bool tc_linear_supported(const Dims &s);
+cudaError_t launch_linear_tc(const Dims &s, const void *k, const void *v, const void *wkt, const int32_t *idx,
+                             float *S, float *z, unsigned *err, cudaStream_t st);
 cudaError_t launch_merge_tc(const Dims &s, const void *q, const void *k, const void *v, const void *wqt,
                             const void *khat, const void *vhat, const void *st_t, const float *z, void *o,
                             unsigned *err, cudaStream_t st);
@@ -98,6 +101,8 @@ still_ws_layout ws_layout(const Dims &s) {
     off = al256(off + (tc ? (size_t)s.B * s.H * s.N * 4 : 0));
     L.wqt = off;
     off = al256(off + (tc ? (size_t)s.H * s.D * s.d * 2 : 0));
+    L.wkt = off;
+    off = al256(off + (tc ? (size_t)s.Hkv * s.D * s.d * 2 : 0));
     L.st = off;
     off = al256(off + (tc ? BK * (T + 1) * s.D * s.d * 2 : 0));
     L.total = off;
@@ -262,8 +267,9 @@ still_status still_hybrid_prefill(const still_dims *dims, const void *q, const v
     void *khat = ws + W.khat, *vhat = ws + W.vhat;
     float *S = reinterpret_cast<float *>(ws + W.S), *z = reinterpret_cast<float *>(ws + W.z);
     float *phik = reinterpret_cast<float *>(ws + W.phik);
-    void *wqt = ws + W.wqt, *st_t = ws + W.st;
+    void *wqt = ws + W.wqt, *st_t = ws + W.st, *wkt = ws + W.wkt;
     const bool use_tc = tc_merge_supported(s);
+    const bool use_tc_lin = use_tc && tc_linear_supported(s);
     const bool select = s.w > 0 && s.k > 0 && s.T() > 0;
     const bool need_r = s.w > 0 && s.k > 0 && (!idx_in || state);
 
@@ -286,11 +292,17 @@ still_status still_hybrid_prefill(const still_dims *dims, const void *q, const v
         }
     }
     // 3./4. NP-Map of the keys and the linear state seen by every query chunk
-    {
-        TimingScope ts(2, cs);
-        STILL_LAUNCH(launch_npmap(s.B * s.Hkv * s.N, s.Hkv, s.N, s.d, s.D, s.bf16, k, Wk, phik, cs));
-    }
-    {
+    if (use_tc_lin) {
+        // NP-Map of the keys fused into the tensor-core linear-state kernel
+        TimingScope ts(3, cs);
+        STILL_LAUNCH(launch_w_transpose(s.Hkv, s.d, s.D, Wk, wkt, cs));
+        STILL_LAUNCH(launch_linear_tc(s, k, v, wkt, idx_used, S, z, err, cs));
+        STILL_LAUNCH(launch_linear_prefix(s, S, z, use_tc ? st_t : nullptr, cs));
+    } else {
+        {
+            TimingScope ts(2, cs);
+            STILL_LAUNCH(launch_npmap(s.B * s.Hkv * s.N, s.Hkv, s.N, s.d, s.D, s.bf16, k, Wk, phik, cs));
+        }
         TimingScope ts(3, cs);
         STILL_LAUNCH(launch_linear_state(s, phik, v, idx_used, S, z, use_tc ? st_t : nullptr, err, cs));
         g_launches.fetch_add(s.T() - s.m() > 0 ? 1 : 0);  // the delta kernel (the prefix was counted)
@@ -299,7 +311,7 @@ still_status still_hybrid_prefill(const still_dims *dims, const void *q, const v
     {
     TimingScope ts(4, cs);
     if (use_tc) {
-        STILL_LAUNCH(launch_wq_transpose(s, Wq, wqt, cs));
+        STILL_LAUNCH(launch_w_transpose(s.H, s.d, s.D, Wq, wqt, cs));
         STILL_LAUNCH(launch_merge_tc(s, q, k, v, wqt, khat, vhat, st_t, z, o, err, cs));
     }
     else STILL_LAUNCH(launch_merge_generic(s, q, k, v, Wq, khat, vhat, S, z, phik, o, cs));

@@ -446,7 +446,12 @@ cudaError_t launch_linear_state(const Dims &s, const float *phik, const void *v,
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
+    return launch_linear_prefix(s, S, z, st_t, st);
+}
+
+cudaError_t launch_linear_prefix(const Dims &s, float *S, float *z, void *st_t, cudaStream_t st) {
     const size_t total = (size_t)s.B * s.Hkv * ((size_t)s.D * s.d + s.D);
+    if (total == 0) return cudaSuccess;
     linear_prefix_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(s, S, z,
                                                                          static_cast<__nv_bfloat16 *>(st_t));
     return cudaGetLastError();

@@ -748,6 +748,282 @@ __global__ void mean_heads_kernel(const float *__restrict__ sigma, float *__rest
     }
 }
 
+// ------------------------------------------------------------------ linear state (NP-Map fused)
+// Linear branch state ([p1] introduction: the unselected tokens are aggregated linearly; "NP-Map":
+// phi(x) = ||x|| f(x Wk) / ||f(x Wk)||): for each (b, g) and each chunk c <= T-m-1 that some query
+// chunk sees, Delta S_c = sum over the unkept tokens j of c of phi(k_j) v_j^T [D, d] and
+// Delta z_c = sum phi(k_j), written to slot c+m+1 of S / z (the prefix kernel then sums the slots).
+// One CTA per (b, g, c); per 128-token subtile: Y = K Wk^T (tcgen05, TMEM, double-buffered) ->
+// four warps turn their token's row into phi (zero for kept tokens) and store it bf16 into shared
+// memory in the 128-byte-swizzled layout -> Delta S += Phi^T V and Delta z += Phi^T 1 (tcgen05,
+// Phi^T and V as MN-major operands, fp32 accumulators in TMEM).  The feature dimension is padded
+// to 128 rows of the MMA (D = 64 leaves the upper half zero).
+template <int DH, int DF>
+struct LinCfg {
+    static constexpr int REG = 128 * 128;                 // 128 rows x 64 bf16
+    static constexpr int TILE_BYTES = 128 * DH * 2;       // 128 tokens x DH
+    static constexpr int NS = 2;
+    static constexpr int STAGE_BYTES = 2 * TILE_BYTES;    // K + V
+    static constexpr int WK_BYTES = DF * DH * 2;          // Wk^T [DF rows x DH]
+    static constexpr int PHI_BYTES = 2 * REG;             // [128 tokens x 128 features] (2 regions)
+    static constexpr int ONES_BYTES = 2 * 16 * 128;       // [16 rows x 128 tokens] of ones (2 regions)
+    static constexpr int NUM_BARS = 9 + 3 * NS;
+    static constexpr int TMEM_SLOT_OFF = 8 * NUM_BARS;
+    static constexpr int ABORT_OFF = TMEM_SLOT_OFF + 8;
+    static constexpr int BAR_BYTES = 256;
+    static_assert(ABORT_OFF + 8 <= BAR_BYTES, "barrier area overflow");
+    static constexpr int SMEM = WK_BYTES + NS * STAGE_BYTES + PHI_BYTES + ONES_BYTES + BAR_BYTES + 1024;
+    static constexpr int THREADS = 128 + 64;
+    static constexpr int PRODUCER_WARP = 4, MMA_WARP = 5;
+    static constexpr int Y_COL = 0, S_COL = 256, Z_COL = 384, TMEM_COLS = 512;
+};
+
+struct LinParams {
+    int B, Hkv, N, C, k, m, T;
+    const int32_t *idx;   // [B,Hkv,T,k] kept positions
+    float *S;             // [B,Hkv,T+1,D,d]
+    float *z;             // [B,Hkv,T+1,D]
+    unsigned *err;
+};
+
+template <int DH, int DF>
+__global__ void __launch_bounds__(LinCfg<DH, DF>::THREADS, 1)
+    linear_state_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
+                           const __grid_constant__ CUtensorMap map_wk, const LinParams p) {
+    using Cfg = LinCfg<DH, DF>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t sWk = sbase;
+    const uint32_t sStage = sWk + Cfg::WK_BYTES;
+    const uint32_t sPhi = sStage + Cfg::NS * Cfg::STAGE_BYTES;
+    const uint32_t sOnes = sPhi + Cfg::PHI_BYTES;
+    uint8_t *phi_ptr = smem + (sPhi - sbase);
+    uint8_t *bar_area = smem + (sOnes - sbase) + Cfg::ONES_BYTES;
+    const uint32_t sBar = smem_u32(bar_area);
+    auto BAR = [&](int i) { return sBar + 8u * i; };
+    // slots: 0 WK full, 1 drain, 2/3 Y full [buf], 4/5 Y empty [buf], 6 Phi full, 7 Phi empty,
+    //        8.. K full[s], 8+NS.. V full[s], 8+2NS.. KV empty[s], 8+3NS done
+    const int B_WK = 0, B_DRAIN = 1, B_YFULL = 2, B_YEMPTY = 4, B_PFULL = 6, B_PEMPTY = 7, B_KFULL = 8,
+              B_VFULL = 8 + Cfg::NS, B_KVEMPTY = 8 + 2 * Cfg::NS, B_DONE = 8 + 3 * Cfg::NS;
+    static_assert(8 + 3 * Cfg::NS + 1 == Cfg::NUM_BARS, "slot map");
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_area + Cfg::TMEM_SLOT_OFF);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bar_area + Cfg::ABORT_OFF);
+    __shared__ unsigned char kept[1024];  // per-subtile scratch is enough: C <= 1024 checked on the host
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nc = p.T - p.m;
+    const int c = blockIdx.x % nc;
+    const int bg = blockIdx.x / nc;
+    const int g = bg % p.Hkv;
+    const int nsub = p.C / 128;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < Cfg::NUM_BARS; ++i) mbar_init(BAR(i), (i == B_PFULL || i == B_YEMPTY || i == B_YEMPTY + 1) ? 128 : 1);
+        *abort_flag = 0;
+        mbar_fence_init();
+    }
+    for (int j = threadIdx.x; j < p.C; j += blockDim.x) kept[j] = 0;
+    // constant tile of ones (any layout: every element is 1) and zero Phi (the padded features stay 0)
+    for (int e = threadIdx.x; e < Cfg::ONES_BYTES / 4; e += blockDim.x)
+        reinterpret_cast<uint32_t *>(smem + (sOnes - sbase))[e] = 0x3F803F80u;
+    for (int e = threadIdx.x; e < Cfg::PHI_BYTES / 16; e += blockDim.x)
+        reinterpret_cast<uint4 *>(phi_ptr)[e] = make_uint4(0, 0, 0, 0);
+    if (warp == Cfg::MMA_WARP) {
+        tmem_alloc(smem_u32(tmem_slot), Cfg::TMEM_COLS);
+        tmem_relinquish();
+    }
+    __syncthreads();
+    for (int n = threadIdx.x; n < p.k; n += blockDim.x) {
+        const int j = p.idx[((size_t)bg * p.T + c) * p.k + n] - c * p.C;
+        if (j >= 0 && j < p.C) kept[j] = 1;
+        else report(p.err, DEV_ERR_INDEX);
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // ones / zero Phi -> tensor core
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == Cfg::PRODUCER_WARP) {
+        if (lane == 0) {
+            bool ok = true;
+            int issued = 0;
+            mbar_arrive_expect_tx(BAR(B_WK), Cfg::WK_BYTES);
+            for (int rr = 0; rr < DH / 64; ++rr) tma_load_3d(sWk + rr * (DF * 128), &map_wk, BAR(B_WK), rr * 64, 0, g);
+            for (int u = 0; u < nsub; ++u) {
+                const int s = u % Cfg::NS;
+                if (u >= Cfg::NS) {
+                    ok = mbar_wait(BAR(B_KVEMPTY + s), ((u / Cfg::NS) - 1) & 1, abort_flag);
+                    if (!ok) break;
+                }
+                const uint32_t sK = sStage + s * Cfg::STAGE_BYTES, sV = sK + Cfg::TILE_BYTES;
+                const int row = c * p.C + u * 128;
+                mbar_arrive_expect_tx(BAR(B_KFULL + s), Cfg::TILE_BYTES);
+                for (int rr = 0; rr < DH / 64; ++rr) tma_load_3d(sK + rr * Cfg::REG, &map_k, BAR(B_KFULL + s), rr * 64, row, bg);
+                mbar_arrive_expect_tx(BAR(B_VFULL + s), Cfg::TILE_BYTES);
+                for (int rr = 0; rr < DH / 64; ++rr) tma_load_3d(sV + rr * Cfg::REG, &map_v, BAR(B_VFULL + s), rr * 64, row, bg);
+                issued = u + 1;
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                report(p.err, DEV_ERR_TIMEOUT);
+                mbar_wait_drain(BAR(B_WK), 0, 100000000ull);
+                for (int u = max(0, issued - Cfg::NS); u < issued; ++u) {
+                    mbar_wait_drain(BAR(B_KFULL + u % Cfg::NS), (u / Cfg::NS) & 1, 100000000ull);
+                    mbar_wait_drain(BAR(B_VFULL + u % Cfg::NS), (u / Cfg::NS) & 1, 100000000ull);
+                }
+            }
+        }
+    } else if (warp == Cfg::MMA_WARP) {
+        if (lane == 0) {
+            constexpr uint32_t ID_Y = idesc_bf16(128, DF, 0, 0);
+            constexpr uint32_t ID_S = idesc_bf16(128, DH, 1, 1);   // A = Phi^T (MN-major), B = V (MN-major)
+            constexpr uint32_t ID_Z = idesc_bf16(128, 16, 1, 0);   // B = ones (K-major)
+            bool ok = mbar_wait(BAR(B_WK), 0, abort_flag);
+            // Y for subtile u goes to buffer u&1; the next Y is issued as soon as its K tile is in
+            auto issue_y = [&](int u) -> bool {
+                const int s = u % Cfg::NS, yb = u & 1;
+                if (!mbar_wait(BAR(B_KFULL + s), (u / Cfg::NS) & 1, abort_flag)) return false;
+                if (u >= 2 && !mbar_wait(BAR(B_YEMPTY + yb), ((u >> 1) - 1) & 1, abort_flag)) return false;
+                tc_fence_after();
+                const uint32_t sK = sStage + s * Cfg::STAGE_BYTES;
+                for (int kk = 0; kk < DH / 16; ++kk)
+                    mma_ss(tmem + Cfg::Y_COL + yb * 128, kmajor_desc(sK, kk, Cfg::REG), kmajor_desc(sWk, kk, DF * 128),
+                           ID_Y, kk > 0);
+                mma_commit(BAR(B_YFULL + yb));
+                return true;
+            };
+            if (ok) ok = issue_y(0);
+            for (int u = 0; ok && u < nsub; ++u) {
+                const int s = u % Cfg::NS;
+                if (u + 1 < nsub) ok = issue_y(u + 1);
+                if (ok) ok = mbar_wait(BAR(B_VFULL + s), (u / Cfg::NS) & 1, abort_flag);
+                if (ok) ok = mbar_wait(BAR(B_PFULL), u & 1, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t sV = sStage + s * Cfg::STAGE_BYTES + Cfg::TILE_BYTES;
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint64_t adesc = sw128_desc(sPhi + kk * 2048, Cfg::REG, 1024);
+                    mma_ss(tmem + Cfg::S_COL, adesc, sw128_desc(sV + kk * 2048, Cfg::REG, 1024), ID_S,
+                           (u > 0 || kk > 0) ? 1u : 0u);
+                    mma_ss(tmem + Cfg::Z_COL, adesc, kmajor_desc(sOnes, kk, 16 * 128), ID_Z, (u > 0 || kk > 0) ? 1u : 0u);
+                }
+                mma_commit(BAR(B_PEMPTY));
+                mma_commit(BAR(B_KVEMPTY + s));
+            }
+            if (ok) mma_commit(BAR(B_DONE));
+            if (!ok) {
+                *abort_flag = 1;
+                report(p.err, DEV_ERR_TIMEOUT);
+            }
+            mma_commit(BAR(B_DRAIN));
+            mbar_wait_drain(BAR(B_DRAIN), 0, 100000000ull);
+        }
+    } else {
+        // epilogue warps: row r = token of the subtile (featurise), then row r = feature (write out)
+        const int r = warp * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        bool ok = true;
+        for (int u = 0; u < nsub; ++u) {
+            const int s = u % Cfg::NS, yb = u & 1;
+            ok = warp_all(mbar_wait(BAR(B_YFULL + yb), (u >> 1) & 1, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            float y[DF];
+#pragma unroll
+            for (int cc = 0; cc < DF / 32; ++cc) {
+                uint32_t uu[32];
+                tmem_ld32(tmem + lane_off + Cfg::Y_COL + yb * 128 + cc * 32, uu);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) y[cc * 32 + e] = __uint_as_float(uu[e]);
+            }
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(BAR(B_YEMPTY + yb));
+            // ||k||^2 from the swizzled K tile (still resident: released only after this subtile's MMAs)
+            float kk2 = 0.f;
+            const uint8_t *krow = smem + (sStage - sbase) + s * Cfg::STAGE_BYTES + r * 128;
+#pragma unroll
+            for (int rr = 0; rr < DH / 64; ++rr) {
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    const uint4 v4 = *reinterpret_cast<const uint4 *>(krow + rr * Cfg::REG + ((ch ^ (r & 7)) << 4));
+                    const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&v4);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = __bfloat1622float2(h2[e]);
+                        kk2 = fmaf(f.x, f.x, kk2);
+                        kk2 = fmaf(f.y, f.y, kk2);
+                    }
+                }
+            }
+            float ymax = -INFINITY;
+#pragma unroll
+            for (int a = 0; a < DF; ++a) ymax = fmaxf(ymax, y[a]);
+            float ee = 0.f;
+#pragma unroll
+            for (int a = 0; a < DF; ++a) {
+                y[a] = ex2((y[a] - ymax) * kLog2e);
+                ee = fmaf(y[a], y[a], ee);
+            }
+            const float f = kept[u * 128 + r] ? 0.f : sqrtf(kk2) * rsqrtf(ee);
+            // Phi buffer free again (previous subtile's MMAs done)?
+            if (u > 0) {
+                ok = warp_all(mbar_wait(BAR(B_PEMPTY), (u - 1) & 1, abort_flag));
+                if (!ok) break;
+            }
+#pragma unroll
+            for (int rr = 0; rr < DF / 64; ++rr) {
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    uint4 w;
+                    const int a0 = rr * 64 + ch * 8;
+                    w.x = pack_bf16x2(y[a0 + 0] * f, y[a0 + 1] * f);
+                    w.y = pack_bf16x2(y[a0 + 2] * f, y[a0 + 3] * f);
+                    w.z = pack_bf16x2(y[a0 + 4] * f, y[a0 + 5] * f);
+                    w.w = pack_bf16x2(y[a0 + 6] * f, y[a0 + 7] * f);
+                    *reinterpret_cast<uint4 *>(phi_ptr + rr * Cfg::REG + r * 128 + ((ch ^ (r & 7)) << 4)) = w;
+                }
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            mbar_arrive(BAR(B_PFULL));
+        }
+        if (ok) ok = warp_all(mbar_wait(BAR(B_DONE), 0, abort_flag));
+        if (ok) {
+            tc_fence_after();
+            // lane = feature a; columns = x (S) and column 0 (z)
+            const size_t slot = (size_t)bg * (p.T + 1) + c + p.m + 1;
+            float *Srow = p.S + (slot * DF + r) * DH;
+#pragma unroll
+            for (int cc = 0; cc < DH / 32; ++cc) {
+                uint32_t uu[32];
+                tmem_ld32(tmem + lane_off + Cfg::S_COL + cc * 32, uu);
+                tmem_wait_ld();
+                if (r < DF) {
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4)
+                        *reinterpret_cast<float4 *>(Srow + cc * 32 + e) =
+                            make_float4(__uint_as_float(uu[e]), __uint_as_float(uu[e + 1]), __uint_as_float(uu[e + 2]),
+                                        __uint_as_float(uu[e + 3]));
+                }
+            }
+            uint32_t zz[32];
+            tmem_ld32(tmem + lane_off + Cfg::Z_COL, zz);
+            tmem_wait_ld();
+            if (r < DF) p.z[slot * DF + r] = __uint_as_float(zz[0]);
+        }
+        if (!ok) {
+            *abort_flag = 1;
+            report(p.err, DEV_ERR_TIMEOUT);
+        }
+    }
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == Cfg::MMA_WARP) tmem_dealloc(tmem, Cfg::TMEM_COLS);
+}
+
 // ------------------------------------------------------------------ small helper kernels
 // Wq [H, d, D] -> Wq^T [H, D, d] (bf16), the K-major operand of Y = Q Wq.
 __global__ void transpose_wq_kernel(const __nv_bfloat16 *__restrict__ wq, __nv_bfloat16 *__restrict__ wqt, int H,
@@ -846,12 +1122,60 @@ bool tc_merge_supported(const Dims &s) {
            s.N > 0 && encode_fn() != nullptr;
 }
 
-cudaError_t launch_wq_transpose(const Dims &s, const void *wq, void *wqt, cudaStream_t st) {
-    const size_t n = (size_t)s.H * s.d * s.D;
+// W [Hx, d, D] -> W^T [Hx, D, d] (bf16).
+cudaError_t launch_w_transpose(int Hx, int d, int D, const void *w, void *wt, cudaStream_t st) {
+    const size_t n = (size_t)Hx * d * D;
     const unsigned blocks = (unsigned)std::min<size_t>((n + 255) / 256, 4096);
-    transpose_wq_kernel<<<blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(wq),
-                                                 static_cast<__nv_bfloat16 *>(wqt), s.H, s.d, s.D);
+    transpose_wq_kernel<<<blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(w), static_cast<__nv_bfloat16 *>(wt),
+                                                 Hx, d, D);
     return cudaGetLastError();
+}
+
+bool tc_linear_supported(const Dims &s) {
+    return s.bf16 && s.w > 0 && (s.d == 64 || s.d == 128) && (s.D == 64 || s.D == 128) && s.C % 128 == 0 &&
+           s.C <= 1024 && encode_fn() != nullptr;
+}
+
+template <int DH, int DF>
+static cudaError_t launch_linear_cfg(const Dims &s, const void *k, const void *v, const void *wkt,
+                                     const int32_t *idx, float *S, float *z, unsigned *err, cudaStream_t st) {
+    using Cfg = LinCfg<DH, DF>;
+    const int nc = s.T() - s.m();
+    if (nc <= 0 || s.B * s.Hkv == 0) return cudaSuccess;
+    CUtensorMap mk, mv, mw;
+    if (!make_map(&mk, k, DH, s.N, (uint64_t)s.B * s.Hkv, 128) || !make_map(&mv, v, DH, s.N, (uint64_t)s.B * s.Hkv, 128) ||
+        !make_map(&mw, wkt, DH, DF, s.Hkv, DF))
+        return cudaErrorInvalidValue;
+    LinParams prm;
+    prm.B = s.B;
+    prm.Hkv = s.Hkv;
+    prm.N = s.N;
+    prm.C = s.C;
+    prm.k = s.k;
+    prm.m = s.m();
+    prm.T = s.T();
+    prm.idx = idx;
+    prm.S = S;
+    prm.z = z;
+    prm.err = err;
+    auto kern = linear_state_tc_kernel<DH, DF>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+    if (e != cudaSuccess) return e;
+    kern<<<(unsigned)(s.B * s.Hkv * nc), Cfg::THREADS, Cfg::SMEM, st>>>(mk, mv, mw, prm);
+    return cudaGetLastError();
+}
+
+// Delta S / Delta z of every chunk into slot c+m+1 (the prefix kernel finishes S_t, z_t).
+cudaError_t launch_linear_tc(const Dims &s, const void *k, const void *v, const void *wkt, const int32_t *idx,
+                             float *S, float *z, unsigned *err, cudaStream_t st) {
+#define STILL_LIN_CASE(DH, DF) \
+    if (s.d == DH && s.D == DF) return launch_linear_cfg<DH, DF>(s, k, v, wkt, idx, S, z, err, st);
+    STILL_LIN_CASE(64, 64)
+    STILL_LIN_CASE(128, 128)
+    STILL_LIN_CASE(64, 128)
+    STILL_LIN_CASE(128, 64)
+#undef STILL_LIN_CASE
+    return cudaErrorNotSupported;
 }
 
 cudaError_t launch_merge_tc(const Dims &s, const void *q, const void *k, const void *v, const void *wqt,

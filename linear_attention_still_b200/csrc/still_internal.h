@@ -44,6 +44,7 @@ cudaError_t launch_npmap(int rows, int Hx, int N, int d, int D, int bf16, const 
                          cudaStream_t st);
 cudaError_t launch_linear_state(const Dims &s, const float *phik, const void *v, const int32_t *idx, float *S,
                                 float *z, void *st_t, unsigned *err, cudaStream_t st);
+cudaError_t launch_linear_prefix(const Dims &s, float *S, float *z, void *st_t, cudaStream_t st);
 cudaError_t launch_merge_generic(const Dims &s, const void *q, const void *k, const void *v, const void *Wq,
                                  const void *khat, const void *vhat, const float *S, const float *z,
                                  const float *phik, void *o, cudaStream_t st);

@@ -36,7 +36,7 @@ class still_dims(ct.Structure):
 
 
 class still_ws_layout(ct.Structure):
-    _fields_ = [(n, ct.c_size_t) for n in ("r", "idx", "khat", "vhat", "S", "z", "phik", "sig", "wqt", "st", "total")]
+    _fields_ = [(n, ct.c_size_t) for n in ("r", "idx", "khat", "vhat", "S", "z", "phik", "sig", "wqt", "wkt", "st", "total")]
 
 
 if not os.path.exists(_LIB_PATH):

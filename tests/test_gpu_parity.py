@@ -98,17 +98,29 @@ def test_npmap_entry_point(lib, oracle_mod, dtype, d, D):
             assert row_rel_err(got[b, h], ref) <= 1e-5
 
 
-def test_linear_state_parity(lib, oracle_mod):
-    shape = CASES["bf16_gqa_ragged"]
+# The linear state is an intermediate: fp32 features on the SIMT path; on the bf16 tensor-core path
+# phi(k) enters the Phi^T V product rounded to bf16 (relative 2^-9 per element).
+STATE_TOL = {"f32": 1e-4, "bf16": 5e-3}
+
+
+@pytest.mark.parametrize("name", ["bf16_gqa_ragged", "bf16_d128_two_chunk_window", "f32_gqa_d128_D64",
+                                  "bf16_d128_g8"])
+def test_linear_state_parity(lib, oracle_mod, name):
+    shape = CASES[name]
     inp = make_inputs(shape)
     out = gpu_prefill(shape, inp)
     d = odims(shape)
-    for b, g, t in [(0, 0, 0), (0, 1, 2), (1, 0, 3), (1, 1, shape.T)]:
+    T = shape.T
+    for b, g, t in {(0, 0, 0), (0, shape.Hkv - 1, min(2, T)), (shape.B - 1, 0, min(3, T)),
+                    (shape.B - 1, shape.Hkv - 1, T)}:
         S, z = oracle_mod.linear_state(d, inp.k, inp.v, inp.wk, out["idx"], b, g, t)
         gs, gz = out["S"][b, g, t], out["z"][b, g, t]
-        scale = max(np.abs(S).max(), 1e-30)
-        assert np.abs(gs - S).max() / scale <= 1e-4
-        assert np.abs(gz - z).max() / max(np.abs(z).max(), 1e-30) <= 1e-4
+        tol = STATE_TOL[shape.dtype]
+        if np.abs(S).max() == 0:
+            assert np.abs(gs).max() == 0 and np.abs(gz).max() == 0
+            continue
+        assert np.abs(gs - S).max() / np.abs(S).max() <= tol, (b, g, t)
+        assert np.abs(gz - z).max() / np.abs(z).max() <= tol, (b, g, t)
 
 
 def test_injected_selection(lib, oracle_mod):
