@@ -235,6 +235,22 @@ def config_of(shape, args):
             "seq_len": shape.N, "parallelism": f"replicas{args.gpus}", "l2": "flushed before every step"}
 
 
+def max_over_ranks(value_ms: float, world: int, device=None) -> float:
+    """Max of a per-rank time over all ranks (identity on one rank)."""
+    if world <= 1:
+        return value_ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value_ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank: int, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
+    return world * tokens_per_rank * steps / (max_ms / 1e3)
+
+
 def run_ours(args):
     import numpy as np
     import torch
@@ -299,14 +315,10 @@ def run_ours(args):
     launches = still.still_launch_count() - n0
     clocks = sampler.stop()
     kern = still.still_timing_read()
-    total_ms = sum(s_.elapsed_time(e_) for s_, e_ in evs)
-    if world > 1:
-        t = torch.tensor([total_ms], device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(s_.elapsed_time(e_) for s_, e_ in evs), world, "cuda")
     ms_per_step = total_ms / args.steps
     tokens = shape.B * shape.N
-    value = world * tokens * args.steps / (total_ms / 1e3)
+    value = job_throughput(tokens, args.steps, world, total_ms)
 
     # end to end through the same call with pinned host buffers
     pinned = {n: t.pin_memory() for n, t in host.items()}
@@ -324,12 +336,8 @@ def run_ours(args):
         o_host.copy_(o, non_blocking=True)
         e_.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = sum(s_.elapsed_time(e_) for s_, e_ in e_evs)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * tokens * args.e2e_steps / (e2e_ms / 1e3)
+    e2e_ms = max_over_ranks(sum(s_.elapsed_time(e_) for s_, e_ in e_evs), world, "cuda")
+    e2e_value = job_throughput(tokens, args.e2e_steps, world, e2e_ms)
     status = still.still_get_device_status()
 
     peaks = {}

@@ -109,3 +109,18 @@ def test_decode_state_size_grows_with_capacity(lib):
     d = _dims(lib)
     a, b = lib.still_decode_state_bytes(d, 1024), lib.still_decode_state_bytes(d, 8192)
     assert b > a > 0
+
+
+def test_binding_fails_loudly_without_the_library(tmp_path):
+    """No fallback: a package copy without libstill.so refuses to import its binding."""
+    import shutil
+    import subprocess
+    import sys
+    pkg = os.path.join(ROOT, "linear_attention_still_b200")
+    dst = tmp_path / "linear_attention_still_b200"
+    dst.mkdir()
+    for f in ("__init__.py", "still.py", "synth.py"):
+        shutil.copy(os.path.join(pkg, f), dst / f)
+    r = subprocess.run([sys.executable, "-c", "import linear_attention_still_b200.still"], cwd=tmp_path,
+                       capture_output=True, text=True)
+    assert r.returncode != 0 and "libstill.so is not built" in r.stderr

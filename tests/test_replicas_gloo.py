@@ -1,0 +1,48 @@
+"""The multi-GPU benchmark path is independent replicas: each rank times its own batch and the job
+value uses the slowest rank.  Checked with two gloo ranks on CPU (no GPU needed)."""
+import os
+import socket
+
+import pytest
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    import bench
+    my_ms = [120.0, 150.0][rank]
+    worst = bench.max_over_ranks(my_ms, world)
+    value = bench.job_throughput(16384, 10, world, worst)
+    dist.barrier()
+    dist.destroy_process_group()
+    q.put((rank, worst, value))
+
+
+def test_two_replicas_take_the_slowest_rank():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, worst, value in res:
+        assert worst == 150.0
+        assert value == pytest.approx(2 * 16384 * 10 / 0.150)
+
+
+def test_single_rank_is_identity():
+    import bench
+    assert bench.max_over_ranks(3.5, 1) == 3.5
+    assert bench.job_throughput(100, 4, 1, 2.0) == pytest.approx(200000.0)
