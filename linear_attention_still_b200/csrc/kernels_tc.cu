@@ -45,19 +45,29 @@ struct MergeCfg {
     static constexpr int WQ_BYTES = DF * DH * 2;       // one Wq^T [DF rows x DH]
     static constexpr int ST_BYTES = DH * DF * 2;       // S_t^T [DH rows x DF]
     static_assert(HP * WQ_BYTES + ST_BYTES <= NS * STAGE_BYTES, "prologue tiles must fit the stage area");
-    static constexpr int NUM_BARS = 4 + 3 * NS + 5 * HP;      // see the slot map in the kernel
+    static constexpr int NUM_BARS = 4 + 3 * NS + 6 * HP + 2;  // see the slot map in the kernel
     static constexpr int TMEM_SLOT_OFF = 8 * NUM_BARS;          // u32 TMEM base address
     static constexpr int ABORT_OFF = TMEM_SLOT_OFF + 8;         // int abort flag
     static constexpr int BAR_BYTES = 256;
     static_assert(ABORT_OFF + 8 <= BAR_BYTES, "barrier area overflow");
     static constexpr int SMEM = Q_BYTES + NS * STAGE_BYTES + BAR_BYTES + 1024;
-    static constexpr int THREADS = 128 * HP + 64;
+    // Two heads: three full warpgroups (softmax 0, softmax 1, producer + MMA + 2 idle warps) so the
+    // register budget can be moved from the third warpgroup to the softmax ones (setmaxnreg).
+    static constexpr int THREADS = HP == 2 ? 384 : 128 * HP + 64;
     static constexpr int PRODUCER_WARP = 4 * HP;
     static constexpr int MMA_WARP = 4 * HP + 1;
+    // launch budget 384 x 168 = 64512 registers = 2 x 128 x 208 (softmax) + 128 x 88 (the rest)
+    static constexpr int REG_SOFTMAX = 208, REG_OTHER = 88;
+    static_assert(HP != 2 || 2 * 128 * REG_SOFTMAX + 128 * REG_OTHER <= THREADS * 168, "register split");
     static constexpr int TMEM_COLS = 512;
+    // d = 64: P (bf16, 64 columns) gets its own TMEM columns, so the next tile's S = Q K^T can be
+    // issued as soon as the softmax has read S (it then overlaps the exponentials).  d = 128: the
+    // budget is full (2 x S + 2 x O = 512 columns) and P is written over S.
+    static constexpr bool PSEP = DH == 64;
     __host__ __device__ static constexpr int s_col(int x) { return x * 128; }
-    __host__ __device__ static constexpr int o_col(int x) { return 128 * HP + x * DH; }
-    static_assert(128 * HP + HP * DH <= TMEM_COLS, "TMEM budget");
+    __host__ __device__ static constexpr int p_col(int x) { return PSEP ? 128 * HP + x * 64 : x * 128; }
+    __host__ __device__ static constexpr int o_col(int x) { return 128 * HP + (PSEP ? 64 * HP : 0) + x * DH; }
+    static_assert(128 * HP + (PSEP ? 64 * HP : 0) + HP * DH <= TMEM_COLS, "TMEM budget");
 };
 
 struct MergeParams {
@@ -71,12 +81,20 @@ struct MergeParams {
     unsigned *trace;       // optional progress words (16 per CTA), see still_debug_set_trace
 };
 
+// Phase timeline of one CTA (diagnostics only): words [16*gridDim.x + (role*64 + j)*8 + phase] hold
+// the SM clock() when `role` (0/1 softmax warpgroup, 2 MMA issuer, 3 producer) reached `phase` of
+// key tile j, recorded for blockIdx.x == trace[16*gridDim.x + 2048] only.
+__device__ __forceinline__ void trace_time(unsigned *trace, int role, int j, int phase) {
+    if (trace && j < 64) {
+        const unsigned target = trace[16 * gridDim.x + 2048];
+        if (blockIdx.x == target)
+            trace[16 * gridDim.x + (role * 64 + j) * 8 + phase] = (unsigned)clock();
+    }
+}
+
 // Progress word of this CTA (diagnostics only; a no-op unless a trace buffer is set).
 __device__ __forceinline__ void trace_word(unsigned *trace, int slot, unsigned v) {
-    if (trace) {
-        *reinterpret_cast<volatile unsigned *>(trace + blockIdx.x * 16 + slot) = v;
-        __threadfence_system();
-    }
+    if (trace) *reinterpret_cast<volatile unsigned *>(trace + blockIdx.x * 16 + slot) = v;
 }
 
 // tcgen05.ld/st are warp-collective: every decision that guards them is made warp-uniform.
@@ -107,7 +125,9 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
     const int B_QFULL = 0, B_WFULL = 1, B_PRO = 2, B_DRAIN = 3;
     const int B_KFULL = 4, B_VFULL = 4 + Cfg::NS, B_KVEMPTY = 4 + 2 * Cfg::NS;
     const int B_Y = 4 + 3 * Cfg::NS, B_PHI = B_Y + HP, B_S = B_PHI + HP, B_P = B_S + HP, B_O = B_P + HP;
-    static_assert(Cfg::NUM_BARS == 4 + 3 * Cfg::NS + 5 * HP, "slot map");
+    const int B_TURN = B_O + HP;  // [2]: exponential-phase turn of softmax warpgroup 0 / 1
+    const int B_SFREE = B_TURN + 2;  // [HP]: the softmax has read S (separate-P schedule)
+    static_assert(Cfg::NUM_BARS == 4 + 3 * Cfg::NS + 6 * HP + 2, "slot map");
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_area + Cfg::TMEM_SLOT_OFF);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(bar_area + Cfg::ABORT_OFF);
 
@@ -146,6 +166,9 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
             mbar_init(BAR(B_P + x), 128);
             mbar_init(BAR(B_O + x), 1);
         }
+        mbar_init(BAR(B_TURN + 0), 128);
+        mbar_init(BAR(B_TURN + 1), 128);
+        for (int x = 0; x < HP; ++x) mbar_init(BAR(B_SFREE + x), 128);
         *abort_flag = 0;
         mbar_fence_init();
     }
@@ -164,7 +187,10 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-
+    // Register budget changes sit at the top of each warpgroup's branch, so every role's code is
+    // dominated by its own setmaxnreg.
+    if (warp >= 4 * HP) {
+    if (HP == 2) setmaxnreg_dec<Cfg::REG_OTHER>();
     if (warp == Cfg::PRODUCER_WARP) {
         // ================================================================ TMA producer
         if (lane == 0) {
@@ -207,6 +233,7 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
                     tma_load_3d(sV + rr * Cfg::REG, mv, BAR(B_VFULL + s), rr * 64, row, bg);
                 issued = j + 1;
                 trace_word(p.trace, 0, 0x100 + j);
+                trace_time(p.trace, 3, j, 0);
             }
             if (!ok) {
                 *abort_flag = 1;
@@ -251,41 +278,60 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
                 if (ok) mma_commit(BAR(B_PRO));
                 trace_word(p.trace, 1, 5);
             }
+            // Descriptors are built once per operand tile and advanced per 16-element k-step by a
+            // constant added to the start-address field (addresses stay below 256 KB, so no carry).
+            // K-major k-step kk: region kk/4, 32 bytes per step inside the 128-byte row.
+            auto kstep = [](int kk) -> uint64_t { return (uint64_t)((((kk >> 2) * Cfg::REG) + ((kk & 3) * 32)) >> 4); };
+            uint64_t dq[HP];
+#pragma unroll
+            for (int x = 0; x < HP; ++x) dq[x] = sw128_desc(sQ + x * Cfg::TILE_BYTES, 16, 1024);
+            auto issue_s = [&](int x, uint32_t sK) {
+                const uint64_t dk = sw128_desc(sK, 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < DH / 16; ++kk)
+                    mma_ss(tmem + Cfg::s_col(x), dq[x] + kstep(kk), dk + kstep(kk), ID_S, kk > 0);
+                mma_commit(BAR(B_S + x));
+            };
             // first score tiles
             if (ok) ok = mbar_wait(BAR(B_KFULL + 0), 0, abort_flag);
             if (ok) {
                 tc_fence_after();
-                for (int x = 0; x < HP; ++x) {
-                    for (int kk = 0; kk < DH / 16; ++kk)
-                        mma_ss(tmem + Cfg::s_col(x), kmajor_desc(sQ + x * Cfg::TILE_BYTES, kk, Cfg::REG),
-                               kmajor_desc(sStage, kk, Cfg::REG), ID_S, kk > 0);
-                    mma_commit(BAR(B_S + x));
-                }
+                for (int x = 0; x < HP; ++x) issue_s(x, sStage);
             }
             for (int j = 0; ok && j < n_tiles; ++j) {
                 const int s = j % Cfg::NS;
-                const uint32_t sV = sStage + s * Cfg::STAGE_BYTES + Cfg::TILE_BYTES;
+                const uint64_t dv = sw128_desc(sStage + s * Cfg::STAGE_BYTES + Cfg::TILE_BYTES, Cfg::REG, 1024);
+                const int s1 = (j + 1) % Cfg::NS;
+                const uint32_t sK1 = sStage + s1 * Cfg::STAGE_BYTES;
                 for (int x = 0; x < HP && ok; ++x) {
+                    if (Cfg::PSEP) {
+                        // next scores first: they only need the softmax to have read S_x(j)
+                        if (j + 1 < n_tiles) {
+                            if (x == 0) ok = mbar_wait(BAR(B_KFULL + s1), ((j + 1) / Cfg::NS) & 1, abort_flag);
+                            if (ok) ok = mbar_wait(BAR(B_SFREE + x), j & 1, abort_flag);
+                            if (!ok) break;
+                            tc_fence_after();
+                            issue_s(x, sK1);
+                        }
+                    }
                     if (x == 0) ok = mbar_wait(BAR(B_VFULL + s), (j / Cfg::NS) & 1, abort_flag);
+                    if (x == 0) trace_time(p.trace, 2, j, 4);
                     if (ok) ok = mbar_wait(BAR(B_P + x), j & 1, abort_flag);
-                    trace_word(p.trace, 1, (ok ? 0x1000u : 0xB000u) + 0x10u * j + x);
+                    trace_time(p.trace, 2, j, 2 * x);
                     if (!ok) break;
                     tc_fence_after();
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_ts(tmem + Cfg::o_col(x), tmem + Cfg::s_col(x) + kk * 8,
-                               sw128_desc(sV + kk * 2048, Cfg::REG, 1024), ID_PV, 1);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)  // V k-step: 16 keys = 16 rows of 128 bytes
+                        mma_ts(tmem + Cfg::o_col(x), tmem + Cfg::p_col(x) + kk * 8, dv + (uint64_t)(kk * 128), ID_PV, 1);
                     mma_commit(BAR(B_O + x));
-                    if (j + 1 < n_tiles) {
-                        const int s1 = (j + 1) % Cfg::NS;
+                    if (!Cfg::PSEP && j + 1 < n_tiles) {
+                        // P_x(j) lives over S_x: the next scores wait for PV_x(j) (in-order issue)
                         if (x == 0) ok = mbar_wait(BAR(B_KFULL + s1), ((j + 1) / Cfg::NS) & 1, abort_flag);
                         if (!ok) break;
                         tc_fence_after();
-                        const uint32_t sK1 = sStage + s1 * Cfg::STAGE_BYTES;
-                        for (int kk = 0; kk < DH / 16; ++kk)
-                            mma_ss(tmem + Cfg::s_col(x), kmajor_desc(sQ + x * Cfg::TILE_BYTES, kk, Cfg::REG),
-                                   kmajor_desc(sK1, kk, Cfg::REG), ID_S, kk > 0);
-                        mma_commit(BAR(B_S + x));
+                        issue_s(x, sK1);
                     }
+                    trace_time(p.trace, 2, j, 2 * x + 1);
                 }
                 if (ok) mma_commit(BAR(B_KVEMPTY + s));
             }
@@ -297,7 +343,9 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
             mma_commit(BAR(B_DRAIN));
             mbar_wait_drain(BAR(B_DRAIN), 0, 100000000ull);
         }
+    }
     } else {
+        if (HP == 2) setmaxnreg_inc<Cfg::REG_SOFTMAX>();
         // ================================================================ softmax warpgroups
         const int x = warp >> 2;                       // head tile
         const int r = (warp & 3) * 32 + lane;          // row in the tile = TMEM lane
@@ -306,6 +354,7 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t tS = tmem + lane_off + Cfg::s_col(x);
         const uint32_t tO = tmem + lane_off + Cfg::o_col(x);
+        const uint32_t tP = tmem + lane_off + Cfg::p_col(x);
         bool ok = true;
 
         // ---- prologue: phi(q) from Y = Q Wq^T
@@ -386,6 +435,7 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
             ok = warp_all(mbar_wait(BAR(B_S + x), j & 1, abort_flag));
             if (lane == 0) trace_word(p.trace, 2 + warp, (ok ? 0x100u : 0xB00u) + 0x10u * j + 1);
             if (!ok) break;
+            if (threadIdx.x % 128 == 0) trace_time(p.trace, x, j, 0);
             tc_fence_after();
             float sv[128];
 #pragma unroll
@@ -396,13 +446,20 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
                 for (int e = 0; e < 32; ++e) sv[c * 32 + e] = __uint_as_float(u[e]);
             }
             tmem_wait_ld();
-            // masks: ragged last tile of the kept prefix, causal diagonal tile
-            int limit = 128;
-            if (j < n_pre) limit = min(128, nk - j * Cfg::BN);
-            else if (j == n_tiles - 1) limit = r + 1;  // keys i0 .. i0+r
+            if (Cfg::PSEP) {
+                tc_fence_before();
+                mbar_arrive(BAR(B_SFREE + x));  // S_x may now take the next tile's scores
+            }
+            // masks, only on the tiles that need them (warp-uniform test): the ragged last tile of the
+            // kept prefix and the causal diagonal tile
+            const bool diag = j == n_tiles - 1;
+            const bool ragged = j < n_pre && nk - j * Cfg::BN < Cfg::BN;
+            if (diag || ragged) {
+                const int limit = diag ? r + 1 : nk - j * Cfg::BN;
 #pragma unroll
-            for (int c = 0; c < 128; ++c)
-                if (c >= limit) sv[c] = -INFINITY;
+                for (int c = 0; c < 128; ++c)
+                    if (c >= limit) sv[c] = -INFINITY;
+            }
             float mx0 = sv[0], mx1 = sv[1], mx2 = sv[2], mx3 = sv[3];
 #pragma unroll
             for (int c = 4; c < 128; c += 4) {
@@ -412,12 +469,19 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
                 mx3 = fmaxf(mx3, sv[c + 3]);
             }
             const float mnew = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * p.scale_log2;
+            if (threadIdx.x % 128 == 0) trace_time(p.trace, x, j, 1);
             // Lazy rescale: a row moves its reference max only when the max grows by more than 2^8.
             // The O rescale uses warp-collective tcgen05.ld/st, so the warp takes it together when
             // any of its rows needs it (rows that do not keep alpha = 1).
             const bool need = mnew > m_run + 8.0f;
             const float alpha = need ? ex2(m_run - mnew) : 1.f;
             const bool touch_o = need && m_run != -INFINITY;  // O is still zero while m_run = -inf
+            if (Cfg::PSEP && j > 0) {
+                // PV_x(j-1) must be done: it still reads P_x, and O is about to be rescaled
+                ok = warp_all(mbar_wait(BAR(B_O + x), (j - 1) & 1, abort_flag));
+                if (!ok) break;
+                tc_fence_after();
+            }
             if (__any_sync(0xffffffffu, touch_o)) {
                 ok = warp_all(j == 0 ? mbar_wait(BAR(B_PRO), 0, abort_flag)
                                      : mbar_wait(BAR(B_O + x), (j - 1) & 1, abort_flag));
@@ -439,25 +503,36 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
                 l_run *= alpha;
                 m_run = mnew;
             }
+            // Two heads per CTA: the warpgroups take turns on the exponential units, so one
+            // warpgroup's exponentials overlap the other head's MMAs instead of contending with them.
+            if (HP == 2 && (x == 1 || j > 0)) {
+                ok = warp_all(mbar_wait(BAR(B_TURN + x), (x == 1 ? j : j - 1) & 1, abort_flag));
+                if (!ok) break;
+            }
+            if (threadIdx.x % 128 == 0) trace_time(p.trace, x, j, 2);
             const float neg = -m_run;
             float ls0 = 0.f, ls1 = 0.f;
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                uint32_t u[32];
+            for (int c = 0; c < 4; ++c) {
+                uint32_t u[16];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const float p0 = ex2(fmaf(sv[c * 64 + 2 * e], p.scale_log2, neg));
-                    const float p1 = ex2(fmaf(sv[c * 64 + 2 * e + 1], p.scale_log2, neg));
+                for (int e = 0; e < 16; ++e) {
+                    const float p0 = ex2(fmaf(sv[c * 32 + 2 * e], p.scale_log2, neg));
+                    const float p1 = ex2(fmaf(sv[c * 32 + 2 * e + 1], p.scale_log2, neg));
                     ls0 += p0;
                     ls1 += p1;
                     u[e] = pack_bf16x2(p0, p1);
                 }
-                tmem_st32(tS + c * 32, u);
+                tmem_st16(tP + c * 16, u);
             }
+            if (HP == 2) mbar_arrive(BAR(B_TURN + (x ^ 1)));
+            if (threadIdx.x % 128 == 0) trace_time(p.trace, x, j, 3);
             l_run += ls0 + ls1;
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(BAR(B_P + x));
+            if (threadIdx.x % 128 == 0) trace_time(p.trace, x, j, 4);
+            else if (lane == 0) trace_time(p.trace, x, j, 4 + (warp & 3));  // warps 1..3 of the group
             if (lane == 0) trace_word(p.trace, 2 + warp, 0x100u + 0x10u * j + 2);
         }
         // ---- epilogue: o = O / l
@@ -631,6 +706,7 @@ __global__ void __launch_bounds__(SalCfg<DH, HP>::THREADS, 1)
                     if (j >= 2) ok = mbar_wait(BAR(B_SEMPTY + 2 * x + buf), ((j >> 1) - 1) & 1, abort_flag);
                     if (!ok) break;
                     tc_fence_after();
+                    #pragma unroll 1
                     for (int kk = 0; kk < DH / 16; ++kk)
                         mma_ss(tmem + Cfg::s_col(x, buf), kmajor_desc(sQ + x * Cfg::TILE_BYTES, kk, Cfg::REG),
                                kmajor_desc(sK + s * Cfg::TILE_BYTES, kk, Cfg::REG), ID_S, kk > 0);
@@ -887,6 +963,7 @@ __global__ void __launch_bounds__(LinCfg<DH, DF>::THREADS, 1)
                 if (u >= 2 && !mbar_wait(BAR(B_YEMPTY + yb), ((u >> 1) - 1) & 1, abort_flag)) return false;
                 tc_fence_after();
                 const uint32_t sK = sStage + s * Cfg::STAGE_BYTES;
+                #pragma unroll 1
                 for (int kk = 0; kk < DH / 16; ++kk)
                     mma_ss(tmem + Cfg::Y_COL + yb * 128, kmajor_desc(sK, kk, Cfg::REG), kmajor_desc(sWk, kk, DF * 128),
                            ID_Y, kk > 0);
@@ -902,6 +979,7 @@ __global__ void __launch_bounds__(LinCfg<DH, DF>::THREADS, 1)
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t sV = sStage + s * Cfg::STAGE_BYTES + Cfg::TILE_BYTES;
+                #pragma unroll 1
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint64_t adesc = sw128_desc(sPhi + kk * 2048, Cfg::REG, 1024);
                     mma_ss(tmem + Cfg::S_COL, adesc, sw128_desc(sV + kk * 2048, Cfg::REG, 1024), ID_S,
