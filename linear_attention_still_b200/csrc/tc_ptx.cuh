@@ -213,6 +213,39 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+// ---------------------------------------------------------------- packed fp32 pairs (sm_100a)
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// 2^x for a pair, on the FMA pipe (offloads the MUFU unit).  Cody-Waite split x = j + f with
+// j = rint(x) (magic-number rounding, 1.5 * 2^23), f in [-1/2, 1/2]; 2^f by a degree-3 polynomial
+// whose coefficients were fitted here for minimax relative error on [-1/2, 1/2] (Lawson's
+// iteratively reweighted least squares; max relative error 7.7e-5); 2^j is added to the exponent
+// field.  x is clamped at -125 so the biased exponent stays >= 1 (p >= 2^-1/2 has exponent >= 126):
+// the result is then ~2^-125, below every weight that matters, and never wraps into the sign bit.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+    constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+    x.x = fmaxf(x.x, -125.f);
+    x.y = fmaxf(x.y, -125.f);
+    const float2 t = fadd2(x, make_float2(kMagic, kMagic));
+    const float2 j = fadd2(t, make_float2(-kMagic, -kMagic));
+    const float2 f = ffma2(j, make_float2(-1.f, -1.f), x);
+    float2 p = ffma2(make_float2(0.05522262305021286f, 0.05522262305021286f), f,
+                     make_float2(0.24261526763439178f, 0.24261526763439178f));
+    p = ffma2(p, f, make_float2(0.6932516098022461f, 0.6932516098022461f));
+    p = ffma2(p, f, make_float2(0.9999275803565979f, 0.9999275803565979f));
+    float2 r;
+    r.x = __int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23));
+    r.y = __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23));
+    return r;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&h);
