@@ -214,7 +214,10 @@ def run_reference(args):
     vals = []
     desc, nth = "", 1
     for i in range(args.warmup + args.steps):
-        v, t, desc, nth = oracle_sample(shape, per_step)
+        if shape.decode_steps > 0:
+            v, t, desc, nth = oracle_decode_sample(shape, per_step)
+        else:
+            v, t, desc, nth = oracle_sample(shape, per_step)
         if i >= args.warmup:
             vals.append(v)
     value = statistics.median(vals) if vals else None
@@ -346,14 +349,18 @@ def run_ours(args):
             peaks = json.load(f)
     except OSError:
         pass
-    merge_ms, merge_n = kern["merge"]
+    # the merge runs as one kernel (SIMT path) or as two tensor-core phases (window part with the fused
+    # saliency, then the kept prefix + linear branch); achieved = algorithmic FLOPs of one step's merge
+    # over the summed device time of its launches
+    merge_ms = kern["merge"][0] + kern["merge_prefix"][0]
+    merge_n = args.steps if merge_ms > 0 else 0
     achieved = merge_flops(shape) / (merge_ms / merge_n / 1e3) / 1e12 if merge_n else None
     peak = peaks.get("bf16_tflops", 1590.0) if shape.dtype == "bf16" else None
     roofline = {
-        "kernel": "merge", "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+        "kernel": "merge (window phase + kept-prefix phase)", "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
         "frac": (achieved / peak) if (achieved and peak) else None,
         "peak_source": "measured bf16_tflops" if "bf16_tflops" in peaks else "fallback 1.59 PFLOP/s",
-        "traffic": None, "flops_per_launch": merge_flops(shape), "launch_ms": merge_ms / merge_n if merge_n else None,
+        "traffic": None, "flops_per_step": merge_flops(shape), "ms_per_step": merge_ms / merge_n if merge_n else None,
     }
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -375,10 +382,187 @@ def run_ours(args):
         print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------- decode workload
+
+def decode_step_bytes(shape, pos: int) -> int:
+    """Algorithmic HBM bytes of one decode step at position pos (one token for each of the B
+    sequences): per (b, g) the kept rows and the window rows of K and V, S [D,d] and z [D] in fp32;
+    per (b, h) q and o."""
+    es = 2 if shape.dtype == "bf16" else 4
+    m, t = shape.w // shape.C, pos // shape.C
+    lo = max(0, (t - m) * shape.C)
+    rows = shape.k * max(0, t - m) + (pos - lo + 1)
+    per_bg = rows * 2 * shape.d * es + shape.D * shape.d * 4 + shape.D * 4
+    return shape.B * shape.Hkv * per_bg + shape.B * shape.H * 2 * shape.d * es
+
+
+def oracle_decode_sample(shape, seconds: float):
+    """fp64 oracle cost of decode rows: one (batch 0, KV group 0) slice of N + steps tokens, the output
+    rows of a sample of decode positions (the oracle evaluates the same definition as the prefill
+    row), scaled to tokens/s of one sequence over all KV groups."""
+    import numpy as np
+
+    import oracle
+    oracle.build()
+    nth = len(os.sched_getaffinity(0))
+    full = shape.replace(B=1, H=shape.G, Hkv=1, N=shape.N + shape.decode_steps, decode_steps=0)
+    inp = make_inputs(shape.replace(B=1, H=shape.G, Hkv=1))
+    d = oracle.Dims.of(full)
+    _, r = oracle.saliency(d, inp.q, inp.k, nthreads=nth)
+    idx = oracle.topk(d, r)
+    positions = [shape.N + s_ for s_ in range(0, shape.decode_steps, max(1, shape.decode_steps // 8))]
+    rows = np.array([(0, h, p_) for p_ in positions for h in range(shape.G)], dtype=np.int32)
+    t0 = time.perf_counter()
+    oracle.prefill(d, inp.q, inp.k, inp.v, inp.wq, inp.wk, idx_in=idx, rows=rows, nthreads=nth)
+    t_rows = time.perf_counter() - t0
+    per_token = t_rows / len(positions) * shape.Hkv  # one token of one sequence, every KV group
+    desc = (f"oracle fp64: rows of {len(positions)} decode positions x {shape.G} heads of one KV group at "
+            f"context {shape.N} ({t_rows:.2f} s), scaled to all {shape.Hkv} KV groups")
+    return 1.0 / per_token, t_rows, desc, nth
+
+
+def run_decode(args):
+    import numpy as np
+    import torch
+
+    rank, world, local = dist_setup(args)
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    from linear_attention_still_b200 import still
+    shape = WORKLOADS[args.workload]
+    N, steps, B = shape.N, shape.decode_steps, shape.B
+    tdt = torch.bfloat16 if shape.dtype == "bf16" else torch.float32
+    e2e_steps = min(args.e2e_steps, 20)
+    K = min(args.steps, steps - args.warmup - e2e_steps)
+    cap = N + steps
+    dims = still.dims_of(shape)
+    q = torch.empty(B, shape.H, N, shape.d, dtype=tdt, device="cuda")
+    k = torch.empty(B, shape.Hkv, N, shape.d, dtype=tdt, device="cuda")
+    v = torch.empty_like(k)
+    qd = torch.empty(steps, B, shape.H, shape.d, dtype=tdt)   # decode tokens, host
+    kd = torch.empty(steps, B, shape.Hkv, shape.d, dtype=tdt)
+    vd = torch.empty_like(kd)
+    wq = wk = None
+    for b in range(B):  # one batch item at a time keeps the host footprint bounded
+        inp = make_inputs(shape.replace(seed=shape.seed + rank), batches=[b])
+        q[b].copy_(torch.from_numpy(inp.q[0, :, :N]).to(tdt))
+        k[b].copy_(torch.from_numpy(inp.k[0, :, :N]).to(tdt))
+        v[b].copy_(torch.from_numpy(inp.v[0, :, :N]).to(tdt))
+        qd[:, b] = torch.from_numpy(np.ascontiguousarray(inp.q[0, :, N:].transpose(1, 0, 2))).to(tdt)
+        kd[:, b] = torch.from_numpy(np.ascontiguousarray(inp.k[0, :, N:].transpose(1, 0, 2))).to(tdt)
+        vd[:, b] = torch.from_numpy(np.ascontiguousarray(inp.v[0, :, N:].transpose(1, 0, 2))).to(tdt)
+        wq, wk = torch.from_numpy(inp.wq).to(tdt).cuda(), torch.from_numpy(inp.wk).to(tdt).cuda()
+        del inp
+    state = torch.empty(still.still_decode_state_bytes(dims, cap), dtype=torch.uint8, device="cuda")
+    still.still_decode_init(dims, cap, state)
+    o = torch.empty_like(q)
+    ws = torch.empty(still.still_prefill_workspace_bytes(dims), dtype=torch.uint8, device="cuda")
+    still.still_hybrid_prefill(dims, q, k, v, wq, wk, o, workspace=ws, state=state, state_capacity=cap)
+    del ws, o, q, k, v
+    torch.cuda.synchronize()
+    qdd, kdd, vdd = qd.cuda(), kd.cuda(), vd.cuda()
+    o_t = torch.empty(B, shape.H, shape.d, dtype=tdt, device="cuda")
+    stream = torch.cuda.current_stream()
+    pos = N
+    for _ in range(args.warmup):
+        still.still_decode_step(dims, state, cap, pos, wq, wk, qdd[pos - N], kdd[pos - N], vdd[pos - N], o_t)
+        pos += 1
+    torch.cuda.synchronize()
+    if still.still_get_device_status() != 0:
+        raise RuntimeError("device-side check failed during warm-up")
+    gpu_id = None
+    try:
+        gpu_id = f"GPU-{torch.cuda.get_device_properties(local).uuid}"
+    except Exception:
+        pass
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+    n0 = still.still_launch_count()
+    first = pos
+    for s_, e_ in evs:
+        s_.record(stream)
+        still.still_decode_step(dims, state, cap, pos, wq, wk, qdd[pos - N], kdd[pos - N], vdd[pos - N], o_t)
+        e_.record(stream)
+        pos += 1
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop()
+    launches = still.still_launch_count() - n0
+    times = [s_.elapsed_time(e_) for s_, e_ in evs]
+    total_ms = max_over_ranks(sum(times), world, "cuda")
+    ms_per_step = total_ms / K
+    value = job_throughput(B, K, world, total_ms)
+    nbytes = sum(decode_step_bytes(shape, p_) for p_ in range(first, first + K))
+    peaks = {}
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peaks = json.load(f)
+    except OSError:
+        pass
+    peak = peaks.get("hbm_gbs", 6650.0)
+    achieved = nbytes / (sum(times) / 1e3) / 1e9
+    close_steps = [j for j, p_ in enumerate(range(first, first + K)) if p_ % shape.C == shape.C - 1]
+    # end to end: pinned host token -> device, step, o_t -> host
+    pins = [t_.pin_memory() for t_ in (qd, kd, vd)]
+    o_host = torch.empty(o_t.shape, dtype=tdt).pin_memory()
+    qb, kb, vb = (torch.empty_like(t_[0], device="cuda") for t_ in (qd, kd, vd))
+    e_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(e2e_steps)]
+    for s_, e_ in e_evs:
+        s_.record(stream)
+        qb.copy_(pins[0][pos - N], non_blocking=True)
+        kb.copy_(pins[1][pos - N], non_blocking=True)
+        vb.copy_(pins[2][pos - N], non_blocking=True)
+        still.still_decode_step(dims, state, cap, pos, wq, wk, qb, kb, vb, o_t)
+        o_host.copy_(o_t, non_blocking=True)
+        e_.record(stream)
+        pos += 1
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(sum(s_.elapsed_time(e_) for s_, e_ in e_evs), world, "cuda")
+    status = still.still_get_device_status()
+    line = {
+        "metric": "STILL chunk-delayed decode tokens/s per layer (one token per sequence per step)",
+        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": shape.dtype, "data": "synthetic",
+        "config": dict(config_of(shape, args), decode_steps_timed=K, first_position=first,
+                       chunk_close_steps_timed=len(close_steps),
+                       l2="decode state (kept cache + window) larger than L2"),
+        "roofline": {"kernel": "decode step (all kernels)", "bound": "hbm", "achieved": achieved, "peak": peak,
+                     "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                     "bytes_per_step": nbytes / K,
+                     "peak_source": "measured hbm_gbs" if "hbm_gbs" in peaks else "fallback 6.65 TB/s"},
+        "e2e": {"value": job_throughput(B, e2e_steps, world, e2e_ms), "unit": "tokens/s",
+                "h2d_bytes_per_step": (qb.numel() + kb.numel() + vb.numel()) * qb.element_size(),
+                "d2h_bytes_per_step": o_host.numel() * o_host.element_size()},
+        "gpu_launches": launches, "clocks": clocks,
+        "step_ms": {"median": float(np.median(times)), "max": float(max(times)),
+                    "chunk_close": [times[j] for j in close_steps]},
+        "device_status": status,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v_, t_, desc, nth = oracle_decode_sample(shape, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": v_, "unit": "tokens/s", "cores": nth, "kind": "oracle", "sample": desc}
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif WORKLOADS[args.workload].decode_steps > 0:
+        run_decode(args)
     else:
         run_ours(args)
 

@@ -120,6 +120,8 @@ typedef struct {
     size_t z;      /* fp32  [B,Hkv,T+1,D]      linear normaliser seen by chunk t */
     size_t phik;   /* fp32  [B,Hkv,N,D]        NP-Map features of the keys     */
     size_t sig;    /* fp32  [B,H,N]            per-query-head saliency (bf16 tensor-core path) */
+    size_t lse;    /* fp32  [B,H,N]            log2-sum-exp of each row's window part (same path) */
+    size_t fix;    /* u32 count + int32 [B*H*N] rows whose band score is recomputed (same path) */
     size_t wqt;    /* bf16  [H,D,d]            Wq transposed (bf16 tensor-core path) */
     size_t wkt;    /* bf16  [Hkv,D,d]          Wk transposed (bf16 tensor-core path) */
     size_t st;     /* bf16  [B,Hkv,T+1,d,D]    S_t transposed (bf16 tensor-core path) */
@@ -197,8 +199,10 @@ STILL_API uint64_t still_launch_count(void);
  * ones are not timed).  still_timing_read synchronises those events and, for
  * each kernel class c < n, writes the summed milliseconds to ms[c] and the
  * number of timed launches to launches[c], then forgets them.  Classes:
- * 0 saliency, 1 top-k + gather, 2 NP-Map, 3 linear state, 4 softmax/linear
- * merge, 5 decode-state export.  Single-threaded use only.
+ * 0 saliency (group mean on the tensor-core path), 1 top-k + gather, 2 NP-Map,
+ * 3 linear state, 4 softmax/linear merge (tensor-core path: window part with
+ * the fused saliency), 5 decode-state export, 6 tensor-core merge of the kept
+ * prefix and the linear branch.  Single-threaded use only.
  */
 /*
  * Diagnostics (no counterpart in the method): when `words` is non-NULL, the
@@ -210,7 +214,7 @@ STILL_API uint64_t still_launch_count(void);
 STILL_API void still_debug_set_trace(unsigned *words);
 
 #define STILL_TIMING_MAX_LAUNCHES 4096
-#define STILL_TIMING_CLASSES 6
+#define STILL_TIMING_CLASSES 7
 STILL_API still_status still_timing_enable(int on);
 STILL_API still_status still_timing_read(double *ms, int *launches, int n);
 

@@ -16,9 +16,10 @@ cudaError_t launch_w_transpose(int Hx, int d, int D, const void *w, void *wt, cu
 bool tc_linear_supported(const Dims &s);
 cudaError_t launch_linear_tc(const Dims &s, const void *k, const void *v, const void *wkt, const int32_t *idx,
                              float *S, float *z, unsigned *err, cudaStream_t st);
-cudaError_t launch_merge_tc(const Dims &s, const void *q, const void *k, const void *v, const void *wqt,
-                            const void *khat, const void *vhat, const void *st_t, const float *z, void *o,
-                            unsigned *err, cudaStream_t st);
+cudaError_t launch_merge_tc(int mode, const Dims &s, const MergeOperands &a, unsigned *err, cudaStream_t st);
+cudaError_t launch_mean_heads(const Dims &s, const float *sigma, float *r, cudaStream_t st);
+cudaError_t launch_saliency_fixup(const Dims &s, const void *q, const void *k, const int *list, const unsigned *count,
+                                  float *sigma, cudaStream_t st);
 bool tc_saliency_supported(const Dims &s);
 void set_debug_trace_words(unsigned *p);
 cudaError_t launch_saliency_tc(const Dims &s, const void *q, const void *k, float *r_kv, float *r_q, unsigned *err,
@@ -94,11 +95,16 @@ still_ws_layout ws_layout(const Dims &s) {
     off = al256(off + BK * (T + 1) * s.D * s.d * 4);
     L.z = off;
     off = al256(off + BK * (T + 1) * s.D * 4);
-    L.phik = off;
-    off = al256(off + BK * s.N * s.D * 4);
+    L.phik = off;  // phi(K) only on the SIMT path (the tensor-core linear state featurises in place)
+    const bool fused_lin = s.bf16 && tc_merge_supported(s) && tc_linear_supported(s);
+    off = al256(off + (fused_lin ? 0 : BK * s.N * s.D * 4));
     const bool tc = s.bf16 != 0;  // per-head scores and transposed bf16 operands of the tensor-core path
     L.sig = off;
     off = al256(off + (tc ? (size_t)s.B * s.H * s.N * 4 : 0));
+    L.lse = off;
+    off = al256(off + (tc ? (size_t)s.B * s.H * s.N * 4 : 0));
+    L.fix = off;  // u32 count, then up to B*H*N row indices
+    off = al256(off + (tc ? 256 + (size_t)s.B * s.H * s.N * 4 : 0));
     L.wqt = off;
     off = al256(off + (tc ? (size_t)s.H * s.D * s.d * 2 : 0));
     L.wkt = off;
@@ -273,12 +279,27 @@ still_status still_hybrid_prefill(const still_dims *dims, const void *q, const v
     const bool select = s.w > 0 && s.k > 0 && s.T() > 0;
     const bool need_r = s.w > 0 && s.k > 0 && (!idx_in || state);
 
-    // 1. Self-Saliency Score per KV group
+    float *sig = reinterpret_cast<float *>(ws + W.sig), *lse = reinterpret_cast<float *>(ws + W.lse);
+    unsigned *fix_count = reinterpret_cast<unsigned *>(ws + W.fix);
+    int *fix_list = reinterpret_cast<int *>(ws + W.fix + 256);
+    MergeOperands mo{q, k, v, wqt, khat, vhat, st_t, z, o, lse, sig, fix_list, fix_count};
+    if (use_tc) {
+        // 1a. window part of the softmax branch and, from the same exponentials, the Self-Saliency
+        //     Score of every query head (tensor cores)
+        TimingScope ts(4, cs);
+        if (cudaMemsetAsync(fix_count, 0, sizeof(unsigned), cs) != cudaSuccess) return STILL_ERR_CUDA;
+        STILL_LAUNCH(launch_w_transpose(s.H, s.d, s.D, Wq, wqt, cs));
+        STILL_LAUNCH(launch_merge_tc(0, s, mo, err, cs));
+    }
+    // 1b. Self-Saliency Score per KV group
     if (need_r) {
         TimingScope ts(0, cs);
-        if (tc_saliency_supported(s))
-            STILL_LAUNCH(launch_saliency_tc(s, q, k, r, reinterpret_cast<float *>(ws + W.sig), err, cs));
-        else STILL_LAUNCH(launch_saliency_generic(s, q, k, r, nullptr, cs));
+        if (use_tc) {
+            STILL_LAUNCH(launch_saliency_fixup(s, q, k, fix_list, fix_count, sig, cs));
+            STILL_LAUNCH(launch_mean_heads(s, sig, r, cs));
+        } else {
+            STILL_LAUNCH(launch_saliency_generic(s, q, k, r, nullptr, cs));
+        }
     }
     // 2. per-chunk top-k and gather of the kept rows
     const int32_t *idx_used = idx;
@@ -307,14 +328,13 @@ still_status still_hybrid_prefill(const still_dims *dims, const void *q, const v
         STILL_LAUNCH(launch_linear_state(s, phik, v, idx_used, S, z, use_tc ? st_t : nullptr, err, cs));
         g_launches.fetch_add(s.T() - s.m() > 0 ? 1 : 0);  // the delta kernel (the prefix was counted)
     }
-    // 5. softmax branch + linear branch + merge
-    {
-    TimingScope ts(4, cs);
+    // 5. kept-prefix part of the softmax branch + linear branch, merged with the window part
     if (use_tc) {
-        STILL_LAUNCH(launch_w_transpose(s.H, s.d, s.D, Wq, wqt, cs));
-        STILL_LAUNCH(launch_merge_tc(s, q, k, v, wqt, khat, vhat, st_t, z, o, err, cs));
-    }
-    else STILL_LAUNCH(launch_merge_generic(s, q, k, v, Wq, khat, vhat, S, z, phik, o, cs));
+        TimingScope ts(6, cs);
+        STILL_LAUNCH(launch_merge_tc(1, s, mo, err, cs));
+    } else {
+        TimingScope ts(4, cs);
+        STILL_LAUNCH(launch_merge_generic(s, q, k, v, Wq, khat, vhat, S, z, phik, o, cs));
     }
     // hand-off to decode
     if (state) {

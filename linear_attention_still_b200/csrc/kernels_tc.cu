@@ -22,6 +22,7 @@
 #include <cuda.h>
 
 #include "common.cuh"
+#include "rowops.cuh"
 #include "still_internal.h"
 #include "tc_ptx.cuh"
 
@@ -74,9 +75,14 @@ struct MergeParams {
     int B, H, Hkv, N, C, k, w, G, T;
     float scale_log2;      // tau * log2(e)
     const float *z;        // [B*Hkv*(T+1), DF] fp32
-    __nv_bfloat16 *o;      // [B,H,N,DH]
+    __nv_bfloat16 *o;      // [B,H,N,DH]: window part (normalised) after LOCAL, final output after PREFIX
+    float *lse;            // [B,H,N]: log2-sum-exp of the window part (LOCAL writes, PREFIX reads)
+    float *sigma;          // [B,H,N]: Self-Saliency Score per query head (LOCAL writes)
+    int *fix_list;         // rows whose band sum underflowed against the window max (recomputed later)
+    unsigned *fix_count;
     unsigned *err;
     int n_qtiles;          // ceil(N/128)
+    int qt_first;          // first query tile of this launch (PREFIX: chunks t > m only)
     int pairs;             // G / HP
     unsigned *trace;       // optional progress words (16 per CTA), see still_debug_set_trace
 };
@@ -97,6 +103,44 @@ __device__ __forceinline__ void trace_word(unsigned *trace, int slot, unsigned v
     if (trace) *reinterpret_cast<volatile unsigned *>(trace + blockIdx.x * 16 + slot) = v;
 }
 
+constexpr float kLn2 = 0.6931471805599453f;
+
+// Exponentials of one 128-key row tile: p_c = 2^(s_c tau log2e - m), summed (ls0 + ls1) and written
+// as bf16 P to TMEM (four tcgen05.st of 16 columns).  BAND additionally sums p_c over the columns
+// [bc_lo, bc_hi) into bsum (the Self-Saliency band of this row inside the tile).
+template <int EXPV, bool BAND>
+__device__ __forceinline__ void exp_tile(const float (&sv)[128], float scale_log2, float m_run, uint32_t tP,
+                                         float &ls0, float &ls1, float &bsum, int bc_lo, int bc_hi) {
+    const float2 sc2 = make_float2(scale_log2, scale_log2);
+    const float2 neg2 = make_float2(-m_run, -m_run);
+    float2 ls = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        uint32_t u[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const int c0 = c * 32 + 2 * e;
+            const float2 xx = ffma2(make_float2(sv[c0], sv[c0 + 1]), sc2, neg2);
+            float2 pp;
+            if (EXPV == 2 && c == 3) {
+                pp = exp2_poly2(xx);  // FMA pipe
+            } else {
+                pp.x = ex2(xx.x);      // MUFU
+                pp.y = ex2(xx.y);
+            }
+            ls = fadd2(ls, pp);
+            if (BAND) {
+                if (c0 >= bc_lo && c0 < bc_hi) bsum += pp.x;
+                if (c0 + 1 >= bc_lo && c0 + 1 < bc_hi) bsum += pp.y;
+            }
+            u[e] = pack_bf16x2(pp.x, pp.y);
+        }
+        tmem_st16(tP + c * 16, u);
+    }
+    ls0 = ls.x;
+    ls1 = ls.y;
+}
+
 // tcgen05.ld/st are warp-collective: every decision that guards them is made warp-uniform.
 __device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
 
@@ -110,7 +154,17 @@ __device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, int kk, uint32_t 
 // 2 packed with the last 32-key chunk of each row on the FMA-pipe exp2.  Measured on B200 (1B 16K /
 // 8B B4 16K layers, merge ms): 0.502/3.276, 0.493/3.146, 0.497/3.209 -> variant 1 is built.
 constexpr int kMergeExpVariant = 1;
-template <int DH, int DF, int HP, int EXPV>
+// MODE kMergeLocal: keys = the window [max(0,(t-m)C), i]; also the Self-Saliency Score of every row
+//   ([p1] "Self-Saliency Score"): the band keys [i-w+1, i-1] are window keys, so the band's
+//   log-sum-exp is accumulated from the same exponentials (masked adds on the two partial tiles),
+//   and the diagonal logit is read from the diagonal tile.  Writes o_A = window part / its sum,
+//   lse_A (log2 units) and sigma.
+// MODE kMergePrefix: keys = the kept rows of the decided chunks; the prologue folds the linear
+//   branch and the window part into the accumulator under one shared normaliser:
+//   M = max(lse_A, log2 b), O = O_lin 2^-M + o_A 2^(lse_A - M), l = 2^(lse_A - M) + b 2^-M.
+constexpr int kMergeLocal = 0, kMergePrefix = 1;
+
+template <int DH, int DF, int HP, int EXPV, int MODE>
 __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
     merge_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_kh,
@@ -139,7 +193,7 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
 
     // ---- CTA -> (b, g, head pair, query tile); heavier (later) query tiles first
     const int per_qt = p.B * p.Hkv * p.pairs;
-    const int qt = p.n_qtiles - 1 - (int)(blockIdx.x / per_qt);
+    const int qt = p.n_qtiles - 1 - (int)(blockIdx.x / per_qt);  // >= qt_first by the grid size
     const int rem = blockIdx.x % per_qt;
     const int pair = rem % p.pairs;
     const int bg = rem / p.pairs;
@@ -149,8 +203,9 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
     const int m = p.w / p.C;
     const int nk = p.k * max(0, t - m);                  // kept rows seen by this chunk
     const int lo = max(0, (t - m) * p.C);                // window start
-    const int n_pre = (nk + Cfg::BN - 1) / Cfg::BN;
-    const int n_tiles = n_pre + (i0 - lo) / Cfg::BN + 1;
+    constexpr bool LOCAL = MODE == kMergeLocal;
+    const int n_pre = LOCAL ? 0 : (nk + Cfg::BN - 1) / Cfg::BN;
+    const int n_tiles = LOCAL ? (i0 - lo) / Cfg::BN + 1 : n_pre;
     const int tslot = bg * (p.T + 1) + t;                // linear state slot
 
     if (threadIdx.x == 0) {
@@ -207,18 +262,21 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
                     tma_load_3d(sQ + x * Cfg::TILE_BYTES + rr * Cfg::REG, &map_q, BAR(B_QFULL), rr * 64, i0,
                                 b * p.H + h);
             }
-            mbar_arrive_expect_tx(BAR(B_WFULL), HP * Cfg::WQ_BYTES + Cfg::ST_BYTES);
-            for (int x = 0; x < HP; ++x) {
-                const int h = g * p.G + pair * HP + x;
-                for (int rr = 0; rr < DH / 64; ++rr)
-                    tma_load_3d(sStage + x * Cfg::WQ_BYTES + rr * (DF * 128), &map_wq, BAR(B_WFULL), rr * 64, 0, h);
+            if (!LOCAL) {
+                mbar_arrive_expect_tx(BAR(B_WFULL), HP * Cfg::WQ_BYTES + Cfg::ST_BYTES);
+                for (int x = 0; x < HP; ++x) {
+                    const int h = g * p.G + pair * HP + x;
+                    for (int rr = 0; rr < DH / 64; ++rr)
+                        tma_load_3d(sStage + x * Cfg::WQ_BYTES + rr * (DF * 128), &map_wq, BAR(B_WFULL), rr * 64, 0,
+                                    h);
+                }
+                for (int rr = 0; rr < DF / 64; ++rr)
+                    tma_load_3d(sStage + HP * Cfg::WQ_BYTES + rr * (DH * 128), &map_st, BAR(B_WFULL), rr * 64, 0,
+                                tslot);
+                trace_word(p.trace, 0, 1);
+                ok = mbar_wait(BAR(B_PRO), 0, abort_flag);  // prologue operands consumed
+                trace_word(p.trace, 0, ok ? 2 : 0xBAD2);
             }
-            for (int rr = 0; rr < DF / 64; ++rr)
-                tma_load_3d(sStage + HP * Cfg::WQ_BYTES + rr * (DH * 128), &map_st, BAR(B_WFULL), rr * 64, 0,
-                            tslot);
-            trace_word(p.trace, 0, 1);
-            ok = mbar_wait(BAR(B_PRO), 0, abort_flag);  // prologue operands consumed
-            trace_word(p.trace, 0, ok ? 2 : 0xBAD2);
             for (int j = 0; ok && j < n_tiles; ++j) {
                 const int s = j % Cfg::NS;
                 if (j >= Cfg::NS) {
@@ -226,9 +284,9 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
                     if (!ok) break;
                 }
                 const uint32_t sK = sStage + s * Cfg::STAGE_BYTES, sV = sK + Cfg::TILE_BYTES;
-                const CUtensorMap *mk = j < n_pre ? &map_kh : &map_k;
-                const CUtensorMap *mv = j < n_pre ? &map_vh : &map_v;
-                const int row = j < n_pre ? j * Cfg::BN : lo + (j - n_pre) * Cfg::BN;
+                const CUtensorMap *mk = LOCAL ? &map_k : &map_kh;
+                const CUtensorMap *mv = LOCAL ? &map_v : &map_vh;
+                const int row = LOCAL ? lo + j * Cfg::BN : j * Cfg::BN;
                 mbar_arrive_expect_tx(BAR(B_KFULL + s), Cfg::TILE_BYTES);
                 for (int rr = 0; rr < DH / 64; ++rr)
                     tma_load_3d(sK + rr * Cfg::REG, mk, BAR(B_KFULL + s), rr * 64, row, bg);
@@ -244,7 +302,7 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
                 report(p.err, DEV_ERR_TIMEOUT);
                 // drain this CTA's copies still in flight
                 mbar_wait_drain(BAR(B_QFULL), 0, 100000000ull);
-                mbar_wait_drain(BAR(B_WFULL), 0, 100000000ull);
+                if (!LOCAL) mbar_wait_drain(BAR(B_WFULL), 0, 100000000ull);
                 for (int j = max(0, issued - Cfg::NS); j < issued; ++j) {
                     mbar_wait_drain(BAR(B_KFULL + j % Cfg::NS), (j / Cfg::NS) & 1, 100000000ull);
                     mbar_wait_drain(BAR(B_VFULL + j % Cfg::NS), (j / Cfg::NS) & 1, 100000000ull);
@@ -258,9 +316,9 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
             constexpr uint32_t ID_LIN = idesc_bf16(128, DH, 0, 0);
             constexpr uint32_t ID_S = idesc_bf16(128, 128, 0, 0);
             constexpr uint32_t ID_PV = idesc_bf16(128, DH, 0, 1);
-            bool ok = mbar_wait(BAR(B_QFULL), 0, abort_flag) && mbar_wait(BAR(B_WFULL), 0, abort_flag);
+            bool ok = mbar_wait(BAR(B_QFULL), 0, abort_flag) && (LOCAL || mbar_wait(BAR(B_WFULL), 0, abort_flag));
             trace_word(p.trace, 1, ok ? 1 : 0xBAD1);
-            if (ok) {
+            if (ok && !LOCAL) {
                 tc_fence_after();
                 for (int x = 0; x < HP; ++x) {
                     const uint32_t aq = sQ + x * Cfg::TILE_BYTES, bw = sStage + x * Cfg::WQ_BYTES;
@@ -297,8 +355,8 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
                 mma_commit(BAR(B_S + x));
             };
             // first score tiles
-            if (ok) ok = mbar_wait(BAR(B_KFULL + 0), 0, abort_flag);
-            if (ok) {
+            if (ok && n_tiles > 0) ok = mbar_wait(BAR(B_KFULL + 0), 0, abort_flag);
+            if (ok && n_tiles > 0) {
                 tc_fence_after();
                 for (int x = 0; x < HP; ++x) issue_s(x, sStage);
             }
@@ -326,7 +384,8 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)  // V k-step: 16 keys = 16 rows of 128 bytes
-                        mma_ts(tmem + Cfg::o_col(x), tmem + Cfg::p_col(x) + kk * 8, dv + (uint64_t)(kk * 128), ID_PV, 1);
+                        mma_ts(tmem + Cfg::o_col(x), tmem + Cfg::p_col(x) + kk * 8, dv + (uint64_t)(kk * 128), ID_PV,
+                               (LOCAL && j == 0 && kk == 0) ? 0u : 1u);  // LOCAL: the first PV starts O
                     mma_commit(BAR(B_O + x));
                     if (!Cfg::PSEP && j + 1 < n_tiles) {
                         // P_x(j) lives over S_x: the next scores wait for PV_x(j) (in-order issue)
@@ -361,9 +420,12 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
         const uint32_t tP = tmem + lane_off + Cfg::p_col(x);
         bool ok = true;
 
-        // ---- prologue: phi(q) from Y = Q Wq^T
-        float m_run, l_run;
-        {
+        const size_t row = ((size_t)b * p.H + h) * p.N + i;  // this thread's query row
+        float m_run = -INFINITY, l_run = 0.f;
+        float bs = 0.f, sdiag = 0.f;  // LOCAL: band sum (same reference as l) and raw diagonal score
+
+        if constexpr (!LOCAL) {
+            // ---- prologue: phi(q) from Y = Q Wq^T
             ok = warp_all(mbar_wait(BAR(B_QFULL), 0, abort_flag) && mbar_wait(BAR(B_Y + x), 0, abort_flag));
             if (lane == 0) trace_word(p.trace, 2 + warp, ok ? 1 : 0xBAD1);
             float y[DF];
@@ -425,12 +487,37 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
             tc_fence_before();
             mbar_arrive(BAR(B_PHI + x));
             if (lane == 0) trace_word(p.trace, 2 + warp, 2);
-            if (bden > 0.f) {
-                m_run = 0.f;
-                l_run = bden;
-            } else {
-                m_run = -INFINITY;
-                l_run = 0.f;
+            // ---- fold the window part (o_A, lse_A) into O = phi(q) S_t^T under one normaliser
+            ok = warp_all(ok && mbar_wait(BAR(B_PRO), 0, abort_flag));
+            if (ok) {
+                tc_fence_after();
+                const bool valid = i < p.N;
+                const float lse_a = valid ? p.lse[row] : 0.f;
+                const float M = bden > 0.f ? fmaxf(lse_a, __log2f(bden)) : lse_a;
+                const float wa = ex2(lse_a - M), wb = ex2(-M);
+                const uint4 *orow = reinterpret_cast<const uint4 *>(p.o + row * DH);
+#pragma unroll
+                for (int c = 0; c < DH / 32; ++c) {
+                    uint32_t u[32];
+                    tmem_ld32(tO + c * 32, u);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int v4 = 0; v4 < 4; ++v4) {
+                        const uint4 w = valid ? orow[c * 4 + v4] : make_uint4(0, 0, 0, 0);
+                        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&ww[e]));
+                            const int q0 = 8 * v4 + 2 * e;
+                            u[q0] = __float_as_uint(fmaf(__uint_as_float(u[q0]), wb, a.x * wa));
+                            u[q0 + 1] = __float_as_uint(fmaf(__uint_as_float(u[q0 + 1]), wb, a.y * wa));
+                        }
+                    }
+                    tmem_st32(tO + c * 32, u);
+                }
+                tmem_wait_st();
+                m_run = M;
+                l_run = wa + bden * wb;
             }
         }
 
@@ -454,10 +541,15 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
                 tc_fence_before();
                 mbar_arrive(BAR(B_SFREE + x));  // S_x may now take the next tile's scores
             }
-            // masks, only on the tiles that need them (warp-uniform test): the ragged last tile of the
-            // kept prefix and the causal diagonal tile
-            const bool diag = j == n_tiles - 1;
-            const bool ragged = j < n_pre && nk - j * Cfg::BN < Cfg::BN;
+            // masks, only on the tiles that need them (warp-uniform test): LOCAL the causal diagonal
+            // tile, PREFIX the ragged last tile of the kept rows
+            const bool diag = LOCAL && j == n_tiles - 1;
+            const bool ragged = !LOCAL && nk - j * Cfg::BN < Cfg::BN;
+            if (diag) {
+#pragma unroll
+                for (int c = 0; c < 128; ++c)
+                    if (c == r) sdiag = sv[c];  // unrolled select keeps sv in registers
+            }
             if (diag || ragged) {
                 const int limit = diag ? r + 1 : nk - j * Cfg::BN;
 #pragma unroll
@@ -479,7 +571,7 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
             // any of its rows needs it (rows that do not keep alpha = 1).
             const bool need = mnew > m_run + 8.0f;
             const float alpha = need ? ex2(m_run - mnew) : 1.f;
-            const bool touch_o = need && m_run != -INFINITY;  // O is still zero while m_run = -inf
+            const bool touch_o = need && m_run != -INFINITY;  // O holds nothing yet while m_run = -inf
             if (Cfg::PSEP && j > 0) {
                 // PV_x(j-1) must be done: it still reads P_x, and O is about to be rescaled
                 ok = warp_all(mbar_wait(BAR(B_O + x), (j - 1) & 1, abort_flag));
@@ -487,7 +579,7 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
                 tc_fence_after();
             }
             if (__any_sync(0xffffffffu, touch_o)) {
-                ok = warp_all(j == 0 ? mbar_wait(BAR(B_PRO), 0, abort_flag)
+                ok = warp_all(j == 0 ? (LOCAL || mbar_wait(BAR(B_PRO), 0, abort_flag))
                                      : mbar_wait(BAR(B_O + x), (j - 1) & 1, abort_flag));
                 if (!ok) break;
                 tc_fence_after();
@@ -505,6 +597,7 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
             }
             if (need) {
                 l_run *= alpha;
+                bs *= alpha;
                 m_run = mnew;
             }
             // Two heads per CTA: the warpgroups take turns on the exponential units, so one
@@ -514,50 +607,27 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
                 if (!ok) break;
             }
             if (threadIdx.x % 128 == 0) trace_time(p.trace, x, j, 2);
-            float ls0 = 0.f, ls1 = 0.f;
-            if constexpr (EXPV == 0) {
-                const float neg = -m_run;
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t u[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const float p0 = ex2(fmaf(sv[c * 32 + 2 * e], p.scale_log2, neg));
-                        const float p1 = ex2(fmaf(sv[c * 32 + 2 * e + 1], p.scale_log2, neg));
-                        ls0 += p0;
-                        ls1 += p1;
-                        u[e] = pack_bf16x2(p0, p1);
-                    }
-                    tmem_st16(tP + c * 16, u);
-                }
+            // LOCAL band tiles: keys kstart + c; the band of row r is [i-w+1, i-1]
+            int btype = 0;  // 0 none, 1 whole tile, 2 columns c > r, 3 columns c < r
+            if (LOCAL) {
+                const int kstart = lo + j * Cfg::BN;
+                if (diag) btype = 3;
+                else if (i0 >= p.w && kstart == i0 - p.w) btype = 2;
+                else if (i0 >= p.w && kstart < i0 - p.w) btype = 0;
+                else btype = 1;
+            }
+            float ls0, ls1, bsum = 0.f;
+            if (btype >= 2) {
+                const int bc_lo = btype == 2 ? r + 1 : 0, bc_hi = btype == 2 ? 128 : r;
+                exp_tile<EXPV, true>(sv, p.scale_log2, m_run, tP, ls0, ls1, bsum, bc_lo, bc_hi);
             } else {
-                const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
-                const float2 neg2 = make_float2(-m_run, -m_run);
-                float2 ls = make_float2(0.f, 0.f);
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t u[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const float2 xx = ffma2(make_float2(sv[c * 32 + 2 * e], sv[c * 32 + 2 * e + 1]), sc2, neg2);
-                        float2 pp;
-                        if (EXPV == 2 && c == 3) {
-                            pp = exp2_poly2(xx);  // FMA pipe
-                        } else {
-                            pp.x = ex2(xx.x);      // MUFU
-                            pp.y = ex2(xx.y);
-                        }
-                        ls = fadd2(ls, pp);
-                        u[e] = pack_bf16x2(pp.x, pp.y);
-                    }
-                    tmem_st16(tP + c * 16, u);
-                }
-                ls0 = ls.x;
-                ls1 = ls.y;
+                exp_tile<EXPV, false>(sv, p.scale_log2, m_run, tP, ls0, ls1, bsum, 0, 0);
             }
             if (HP == 2) mbar_arrive(BAR(B_TURN + (x ^ 1)));
             if (threadIdx.x % 128 == 0) trace_time(p.trace, x, j, 3);
             l_run += ls0 + ls1;
+            if (btype == 1) bs += ls0 + ls1;
+            else if (btype >= 2) bs += bsum;
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(BAR(B_P + x));
@@ -566,12 +636,12 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
             if (lane == 0) trace_word(p.trace, 2 + warp, 0x100u + 0x10u * j + 2);
         }
         // ---- epilogue: o = O / l
-        ok = warp_all(ok && mbar_wait(BAR(B_O + x), (n_tiles - 1) & 1, abort_flag));
+        ok = warp_all(ok && (n_tiles > 0 ? mbar_wait(BAR(B_O + x), (n_tiles - 1) & 1, abort_flag) : true));
         if (lane == 0) trace_word(p.trace, 2 + warp, ok ? 0xE00 : 0xBADE);
         if (ok) {
             tc_fence_after();
             const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-            __nv_bfloat16 *orow = p.o + (((size_t)b * p.H + h) * p.N + i) * DH;
+            __nv_bfloat16 *orow = p.o + row * DH;
 #pragma unroll
             for (int c = 0; c < DH / 32; ++c) {
                 uint32_t u[32];
@@ -589,6 +659,23 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
                         dst[v4] = w;
                     }
                 }
+            }
+            if (LOCAL && i < p.N) {
+                p.lse[row] = m_run + __log2f(l_run);
+                // sigma = softplus(s_ii - LSE_{band}) in natural units; +inf for an empty band (i = 0)
+                float sig = INFINITY;
+                if (i > 0) {
+                    if (bs > 0x1p-90f) {
+                        const float lse_band = (m_run + __log2f(bs)) * kLn2;
+                        sig = softplus_f(sdiag * (p.scale_log2 * kLn2) - lse_band);
+                    } else {
+                        // every band key sits > 90 binary orders below the window maximum: the shared
+                        // reference has underflowed the band sum; the row is rescored with its own max
+                        p.fix_list[atomicAdd(p.fix_count, 1u)] = (int)row;
+                        sig = 0.f;
+                    }
+                }
+                p.sigma[row] = sig;
             }
         }
         if (!ok) {
@@ -661,7 +748,7 @@ __global__ void __launch_bounds__(SalCfg<DH, HP>::THREADS, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     const int per_qt = p.B * p.Hkv * p.pairs;
-    const int qt = p.n_qtiles - 1 - (int)(blockIdx.x / per_qt);
+    const int qt = p.n_qtiles - 1 - (int)(blockIdx.x / per_qt);  // >= qt_first by the grid size
     const int rem = blockIdx.x % per_qt;
     const int pair = rem % p.pairs;
     const int bg = rem / p.pairs;
@@ -1180,19 +1267,22 @@ unsigned *debug_trace_words();
 namespace {
 
 template <int DH, int DF, int HP>
-cudaError_t launch_merge_cfg(const Dims &s, const void *q, const void *k, const void *v, const void *wqt,
-                             const void *khat, const void *vhat, const void *st_t, const float *z, void *o,
-                             unsigned *err, cudaStream_t st) {
+cudaError_t launch_merge_cfg(int mode, const Dims &s, const MergeOperands &a, unsigned *err, cudaStream_t st) {
     using Cfg = MergeCfg<DH, DF, HP>;
     const int T = s.T();
+    const int n_qtiles = (s.N + 127) / 128;
+    // PREFIX: only the query chunks t > m see a kept prefix or a linear state
+    const int qt_first = mode == kMergeLocal ? 0 : std::min(n_qtiles, (s.m() + 1) * s.C / 128);
+    if (qt_first >= n_qtiles) return cudaSuccess;
     CUtensorMap mq, mk, mv, mkh, mvh, mw, ms;
     const uint64_t khrows = (uint64_t)T * s.k > 0 ? (uint64_t)T * s.k : 1;
-    bool ok = make_map(&mq, q, DH, s.N, (uint64_t)s.B * s.H, 128) && make_map(&mk, k, DH, s.N, (uint64_t)s.B * s.Hkv, 128) &&
-              make_map(&mv, v, DH, s.N, (uint64_t)s.B * s.Hkv, 128) &&
-              make_map(&mkh, khat, DH, khrows, (uint64_t)s.B * s.Hkv, 128) &&
-              make_map(&mvh, vhat, DH, khrows, (uint64_t)s.B * s.Hkv, 128) &&
-              make_map(&mw, wqt, DH, DF, s.H, DF) &&
-              make_map(&ms, st_t, DF, DH, (uint64_t)s.B * s.Hkv * (T + 1), DH);
+    bool ok = make_map(&mq, a.q, DH, s.N, (uint64_t)s.B * s.H, 128) &&
+              make_map(&mk, a.k, DH, s.N, (uint64_t)s.B * s.Hkv, 128) &&
+              make_map(&mv, a.v, DH, s.N, (uint64_t)s.B * s.Hkv, 128) &&
+              make_map(&mkh, a.khat, DH, khrows, (uint64_t)s.B * s.Hkv, 128) &&
+              make_map(&mvh, a.vhat, DH, khrows, (uint64_t)s.B * s.Hkv, 128) &&
+              make_map(&mw, a.wqt, DH, DF, s.H, DF) &&
+              make_map(&ms, a.st_t, DF, DH, (uint64_t)s.B * s.Hkv * (T + 1), DH);
     if (!ok) return cudaErrorInvalidValue;
     MergeParams prm;
     prm.B = s.B;
@@ -1205,16 +1295,22 @@ cudaError_t launch_merge_cfg(const Dims &s, const void *q, const void *k, const 
     prm.G = s.G();
     prm.T = T;
     prm.scale_log2 = s.scale * kLog2e;
-    prm.z = z;
-    prm.o = static_cast<__nv_bfloat16 *>(o);
+    prm.z = a.z;
+    prm.o = static_cast<__nv_bfloat16 *>(a.o);
+    prm.lse = a.lse;
+    prm.sigma = a.sigma;
+    prm.fix_list = a.fix_list;
+    prm.fix_count = a.fix_count;
     prm.err = err;
-    prm.n_qtiles = (s.N + 127) / 128;
+    prm.n_qtiles = n_qtiles;
+    prm.qt_first = qt_first;
     prm.pairs = s.G() / HP;
     prm.trace = debug_trace_words();
-    auto kern = merge_tc_kernel<DH, DF, HP, kMergeExpVariant>;
+    auto kern = mode == kMergeLocal ? merge_tc_kernel<DH, DF, HP, kMergeExpVariant, kMergeLocal>
+                                    : merge_tc_kernel<DH, DF, HP, kMergeExpVariant, kMergePrefix>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
     if (e != cudaSuccess) return e;
-    const unsigned grid = (unsigned)prm.n_qtiles * s.B * s.Hkv * prm.pairs;
+    const unsigned grid = (unsigned)(n_qtiles - qt_first) * s.B * s.Hkv * prm.pairs;
     kern<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(mq, mk, mv, mkh, mvh, mw, ms, prm);
     return cudaGetLastError();
 }
@@ -1286,14 +1382,13 @@ cudaError_t launch_linear_tc(const Dims &s, const void *k, const void *v, const 
     return cudaErrorNotSupported;
 }
 
-cudaError_t launch_merge_tc(const Dims &s, const void *q, const void *k, const void *v, const void *wqt,
-                            const void *khat, const void *vhat, const void *st_t, const float *z, void *o,
-                            unsigned *err, cudaStream_t st) {
+// mode 0: window part + Self-Saliency Score (writes o_A, lse_A, sigma); mode 1: kept prefix + linear
+// branch folded with the window part (writes o).
+cudaError_t launch_merge_tc(int mode, const Dims &s, const MergeOperands &a, unsigned *err, cudaStream_t st) {
     const bool pair = s.G() % 2 == 0;
-#define STILL_MERGE_CASE(DH, DF)                                                                            \
-    if (s.d == DH && s.D == DF)                                                                             \
-        return pair ? launch_merge_cfg<DH, DF, 2>(s, q, k, v, wqt, khat, vhat, st_t, z, o, err, st)        \
-                    : launch_merge_cfg<DH, DF, 1>(s, q, k, v, wqt, khat, vhat, st_t, z, o, err, st);
+#define STILL_MERGE_CASE(DH, DF)                                                                     \
+    if (s.d == DH && s.D == DF)                                                                      \
+        return pair ? launch_merge_cfg<DH, DF, 2>(mode, s, a, err, st) : launch_merge_cfg<DH, DF, 1>(mode, s, a, err, st);
     STILL_MERGE_CASE(64, 64)
     STILL_MERGE_CASE(128, 128)
     STILL_MERGE_CASE(64, 128)
@@ -1331,6 +1426,62 @@ static cudaError_t launch_saliency_cfg(const Dims &s, const void *q, const void 
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)prm.n_qtiles * s.B * s.Hkv * prm.pairs;
     kern<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(mq, mk, prm);
+    return cudaGetLastError();
+}
+
+// Self-Saliency Score of the rows listed by the window kernel, recomputed with the band's own maximum
+// (one warp per row, lanes split the band keys; same definition as the window kernel:
+// sigma = softplus(s_ii - LSE_{j in [i-w+1, i-1]} s_ij)).
+__global__ void __launch_bounds__(128) saliency_fixup_kernel(const __nv_bfloat16 *__restrict__ q,
+                                                             const __nv_bfloat16 *__restrict__ k,
+                                                             const int *__restrict__ list,
+                                                             const unsigned *__restrict__ count, float *sigma, int H,
+                                                             int Hkv, int N, int d, int w, float scale) {
+    __shared__ __align__(16) float qs[4][256];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const unsigned n = *count;
+    for (unsigned e = blockIdx.x * 4 + warp; e < n; e += gridDim.x * 4) {
+        const size_t row = (size_t)list[e];
+        const int i = (int)(row % N);
+        const size_t bh = row / N;
+        const int h = (int)(bh % H), b = (int)(bh / H), g = h / (H / Hkv);
+        const __nv_bfloat16 *kg = k + ((size_t)b * Hkv + g) * N * d;
+        for (int x = lane; x < d; x += 32) qs[warp][x] = __bfloat162float(q[row * d + x]);
+        __syncwarp();
+        const int lo = max(0, i - w + 1);
+        float mx = -INFINITY, sm = 0.f;
+        for (int j = lo + lane; j < i; j += 32) {
+            const float l = scale * dot_row(qs[warp], kg + (size_t)j * d, d);
+            if (l > mx) {
+                sm = sm * expf(mx - l) + 1.f;
+                mx = l;
+            } else {
+                sm += expf(l - mx);
+            }
+        }
+        const float M = warp_max(mx);
+        const float Z = warp_sum(mx == -INFINITY ? 0.f : sm * expf(mx - M));
+        float dp = 0.f;
+        for (int x = lane; x < d; x += 32) dp = fmaf(qs[warp][x], __bfloat162float(kg[(size_t)i * d + x]), dp);
+        const float sii = scale * warp_sum(dp);
+        if (lane == 0) sigma[row] = (i == lo) ? INFINITY : softplus_f(sii - (M + logf(Z)));
+        __syncwarp();
+    }
+}
+
+cudaError_t launch_saliency_fixup(const Dims &s, const void *q, const void *k, const int *list, const unsigned *count,
+                                  float *sigma, cudaStream_t st) {
+    saliency_fixup_kernel<<<148, 128, 0, st>>>(static_cast<const __nv_bfloat16 *>(q),
+                                                static_cast<const __nv_bfloat16 *>(k), list, count, sigma, s.H,
+                                                s.Hkv, s.N, s.d, s.w, s.scale);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_mean_heads(const Dims &s, const float *sigma, float *r, cudaStream_t st) {
+    const size_t total = (size_t)s.B * s.Hkv * s.N;
+    if (total == 0) return cudaSuccess;
+    const unsigned blocks = (unsigned)std::min<size_t>((total + 255) / 256, 8192);
+    mean_heads_kernel<<<blocks, 256, 0, st>>>(sigma, r, s.B, s.H, s.Hkv, s.N);
     return cudaGetLastError();
 }
 

@@ -35,6 +35,16 @@ constexpr int kDecodeMaxSplits = 64;
 
 DecodeLayout decode_layout(const Dims &s, int capacity);
 
+// Operands of the tensor-core merge phases (device pointers).
+struct MergeOperands {
+    const void *q, *k, *v, *wqt, *khat, *vhat, *st_t;
+    const float *z;
+    void *o;
+    float *lse, *sigma;
+    int *fix_list;
+    unsigned *fix_count;
+};
+
 // ---- generic kernels (fp32 or bf16 storage, fp32 arithmetic) ----
 cudaError_t launch_saliency_generic(const Dims &s, const void *q, const void *k, float *r_kv, float *r_q,
                                     cudaStream_t st);

@@ -36,7 +36,7 @@ class still_dims(ct.Structure):
 
 
 class still_ws_layout(ct.Structure):
-    _fields_ = [(n, ct.c_size_t) for n in ("r", "idx", "khat", "vhat", "S", "z", "phik", "sig", "wqt", "wkt", "st", "total")]
+    _fields_ = [(n, ct.c_size_t) for n in ("r", "idx", "khat", "vhat", "S", "z", "phik", "sig", "lse", "fix", "wqt", "wkt", "st", "total")]
 
 
 if not os.path.exists(_LIB_PATH):
@@ -171,7 +171,7 @@ def still_debug_set_trace(words=None):
     _lib.still_debug_set_trace(_ptr(words))
 
 
-TIMING_CLASSES = ("saliency", "topk_gather", "npmap", "linear_state", "merge", "state_export")
+TIMING_CLASSES = ("saliency", "topk_gather", "npmap", "linear_state", "merge", "state_export", "merge_prefix")
 
 
 def still_timing_enable(on: bool = True):
