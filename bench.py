@@ -473,6 +473,28 @@ def run_decode(args):
     torch.cuda.synchronize()
     if still.still_get_device_status() != 0:
         raise RuntimeError("device-side check failed during warm-up")
+    # end to end: pinned host token -> device, step, o_t -> host
+    pins = [t_.pin_memory() for t_ in (qd, kd, vd)]
+    o_host = torch.empty(o_t.shape, dtype=tdt).pin_memory()
+    qb, kb, vb = (torch.empty_like(t_[0], device="cuda") for t_ in (qd, kd, vd))
+    e_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(e2e_steps)]
+    for s_, e_ in e_evs:
+        s_.record(stream)
+        qb.copy_(pins[0][pos - N], non_blocking=True)
+        kb.copy_(pins[1][pos - N], non_blocking=True)
+        vb.copy_(pins[2][pos - N], non_blocking=True)
+        still.still_decode_step(dims, state, cap, pos, wq, wk, qb, kb, vb, o_t)
+        o_host.copy_(o_t, non_blocking=True)
+        e_.record(stream)
+        pos += 1
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(sum(s_.elapsed_time(e_) for s_, e_ in e_evs), world, "cuda")
+    # untimed steps up to the timed region, which ends at the last position: it holds the step that
+    # closes a chunk (position C-1 mod C) along with ordinary ones
+    while pos < cap - K:
+        still.still_decode_step(dims, state, cap, pos, wq, wk, qdd[pos - N], kdd[pos - N], vdd[pos - N], o_t)
+        pos += 1
+    torch.cuda.synchronize()
     gpu_id = None
     try:
         gpu_id = f"GPU-{torch.cuda.get_device_properties(local).uuid}"
@@ -510,22 +532,6 @@ def run_decode(args):
     peak = peaks.get("hbm_gbs", 6650.0)
     achieved = nbytes / (sum(times) / 1e3) / 1e9
     close_steps = [j for j, p_ in enumerate(range(first, first + K)) if p_ % shape.C == shape.C - 1]
-    # end to end: pinned host token -> device, step, o_t -> host
-    pins = [t_.pin_memory() for t_ in (qd, kd, vd)]
-    o_host = torch.empty(o_t.shape, dtype=tdt).pin_memory()
-    qb, kb, vb = (torch.empty_like(t_[0], device="cuda") for t_ in (qd, kd, vd))
-    e_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(e2e_steps)]
-    for s_, e_ in e_evs:
-        s_.record(stream)
-        qb.copy_(pins[0][pos - N], non_blocking=True)
-        kb.copy_(pins[1][pos - N], non_blocking=True)
-        vb.copy_(pins[2][pos - N], non_blocking=True)
-        still.still_decode_step(dims, state, cap, pos, wq, wk, qb, kb, vb, o_t)
-        o_host.copy_(o_t, non_blocking=True)
-        e_.record(stream)
-        pos += 1
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(sum(s_.elapsed_time(e_) for s_, e_ in e_evs), world, "cuda")
     status = still.still_get_device_status()
     line = {
         "metric": "STILL chunk-delayed decode tokens/s per layer (one token per sequence per step)",
@@ -544,7 +550,11 @@ def run_decode(args):
                 "d2h_bytes_per_step": o_host.numel() * o_host.element_size()},
         "gpu_launches": launches, "clocks": clocks,
         "step_ms": {"median": float(np.median(times)), "max": float(max(times)),
-                    "chunk_close": [times[j] for j in close_steps]},
+                    "chunk_close": [times[j] for j in close_steps],
+                    # one chunk's worth of steps: C-1 ordinary steps and the one that closes the chunk
+                    "chunk_cycle_mean": (float(np.median([t_ for j, t_ in enumerate(times) if j not in close_steps]))
+                                         * (shape.C - 1) + max([times[j] for j in close_steps], default=0.0))
+                    / shape.C if close_steps else None},
         "device_status": status,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

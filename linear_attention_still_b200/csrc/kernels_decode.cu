@@ -169,6 +169,227 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(Dims s, DecodeLayout L
     }
 }
 
+// One lane's DPL consecutive elements of a K or V row, held in the storage type until used.
+template <typename T, int DPL>
+struct RowSlice;
+template <>
+struct RowSlice<__nv_bfloat16, 4> {
+    uint2 u;
+    __device__ __forceinline__ void load(const __nv_bfloat16 *row, int lane) {
+        u = __ldg(reinterpret_cast<const uint2 *>(row) + lane);
+    }
+    __device__ __forceinline__ void get(float (&f)[4]) const {
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+        const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+        f[0] = a.x; f[1] = a.y; f[2] = c.x; f[3] = c.y;
+    }
+};
+template <>
+struct RowSlice<__nv_bfloat16, 2> {
+    unsigned u;
+    __device__ __forceinline__ void load(const __nv_bfloat16 *row, int lane) {
+        u = __ldg(reinterpret_cast<const unsigned *>(row) + lane);
+    }
+    __device__ __forceinline__ void get(float (&f)[2]) const {
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u));
+        f[0] = a.x; f[1] = a.y;
+    }
+};
+template <int DPL>
+struct RowSlice<float, DPL> {
+    float v[DPL];
+    __device__ __forceinline__ void load(const float *row, int lane) {
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) v[e] = __ldg(row + lane * DPL + e);
+    }
+    __device__ __forceinline__ void get(float (&f)[DPL]) const {
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) f[e] = v[e];
+    }
+};
+
+// Split-K decode attention with the G query heads of a KV group packed into each warp: a warp step
+// takes KG = 32/G keys; every lane loads its DPL-element slice of those K and V rows (coalesced), forms
+// the 32 partial dot products (key, head), and a reduce-scatter across the warp leaves the full score
+// of pair (lane / G, lane % G) in each lane.  Online softmax per head (max and sum over the lanes of a
+// head), P V accumulated per head in each lane's slice, and the band statistics of the new token's
+// Self-Saliency Score ([i-w+1, i-1] plus the diagonal) from the same scores.  Scores are kept in log2
+// units; the partials are written in natural units (same format as decode_attn_kernel).
+template <int G>
+__device__ __forceinline__ float reduce_scatter32(float (&v)[32], int lane) {
+    // after the step with offset o the lane keeps the half of its values selected by bit o of its id
+#pragma unroll
+    for (int o = 16, n = 32; o >= 1; o >>= 1, n >>= 1) {
+        const bool upper = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < n / 2; ++i) {
+            const float send = upper ? v[i] : v[i + n / 2];
+            const float keep = upper ? v[i + n / 2] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+    }
+    return v[0];
+}
+
+template <typename T, int DPL, int G>
+__global__ void __launch_bounds__(256) decode_attn_packed_kernel(Dims s, DecodeLayout L, unsigned char *state,
+                                                                 StepGeom gm, const T *__restrict__ q_t) {
+    constexpr int KG = 32 / G, NW = 8, DD = 32 * DPL;
+    constexpr float kL2e = 1.4426950408889634f, kLn2f = 0.6931471805599453f;
+    __shared__ float sm_ml[NW][G][5];          // m, l, bm, bl, sdiag (log2 units)
+    __shared__ float sm_acc[NW][G][DD];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bg = blockIdx.x, split = blockIdx.y, b = bg / s.Hkv, g = bg % s.Hkv;
+    const int l0 = split * gm.per, l1 = min(gm.n, l0 + gm.per);
+    const int band_lo = max(0, gm.pos - s.w + 1);
+    const float sl2 = s.scale * kL2e;
+    float qv[G][DPL];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+        RowSlice<T, DPL> r;
+        r.load(q_t + ((size_t)b * s.H + g * G + h) * s.d, lane);
+        r.get(qv[h]);
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) qv[h][e] *= sl2;
+    }
+    float m = -INFINITY, l = 0.f, bm = -INFINITY, bl = 0.f, sd = -INFINITY;
+    float acc[G][DPL];
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) acc[h][e] = 0.f;
+    const int my_kk = lane / G;
+    for (int base = l0 + warp * KG; base < l1; base += NW * KG) {
+        RowSlice<T, DPL> kr[KG], vr[KG];
+#pragma unroll
+        for (int kk = 0; kk < KG; ++kk) {
+            // rows past the end re-read the last row of the range; their probabilities are zero
+            const int li = min(base + kk, l1 - 1);
+            kr[kk].load(list_row<T>(s, L, state, bg, gm, li, false), lane);
+            vr[kk].load(list_row<T>(s, L, state, bg, gm, li, true), lane);
+        }
+        float part[32];
+#pragma unroll
+        for (int kk = 0; kk < KG; ++kk) {
+            float kf[DPL];
+            kr[kk].get(kf);
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                float a = 0.f;
+#pragma unroll
+                for (int e = 0; e < DPL; ++e) a = fmaf(qv[h][e], kf[e], a);
+                part[kk * G + h] = a;
+            }
+        }
+        float sc = reduce_scatter32<G>(part, lane);
+        const int li = base + my_kk;
+        const bool valid = li < l1;
+        if (!valid) sc = -INFINITY;
+        if (valid && li >= gm.nk) {
+            const int j = gm.lo + (li - gm.nk);
+            if (j == gm.pos) {
+                sd = sc;
+            } else if (j >= band_lo) {
+                if (sc > bm) {
+                    bl = bl * exp2f(bm - sc) + 1.f;
+                    bm = sc;
+                } else {
+                    bl += exp2f(sc - bm);
+                }
+            }
+        }
+        float gmx = sc;
+#pragma unroll
+        for (int o = G; o < 32; o <<= 1) gmx = fmaxf(gmx, __shfl_xor_sync(0xffffffffu, gmx, o));
+        const float mn = fmaxf(m, gmx);
+        const float so = (m == -INFINITY) ? 0.f : exp2f(m - mn);
+        const float pr = valid ? exp2f(sc - mn) : 0.f;
+        float gs = pr;
+#pragma unroll
+        for (int o = G; o < 32; o <<= 1) gs += __shfl_xor_sync(0xffffffffu, gs, o);
+        l = l * so + gs;
+        m = mn;
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            const float a = __shfl_sync(0xffffffffu, so, h);
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) acc[h][e] *= a;
+        }
+#pragma unroll
+        for (int kk = 0; kk < KG; ++kk) {
+            float vf[DPL];
+            vr[kk].get(vf);
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                const float pk = __shfl_sync(0xffffffffu, pr, kk * G + h);
+#pragma unroll
+                for (int e = 0; e < DPL; ++e) acc[h][e] = fmaf(pk, vf[e], acc[h][e]);
+            }
+        }
+    }
+    // band statistics: combine the lanes of each head
+#pragma unroll
+    for (int o = G; o < 32; o <<= 1) {
+        const float obm = __shfl_xor_sync(0xffffffffu, bm, o);
+        const float obl = __shfl_xor_sync(0xffffffffu, bl, o);
+        const float nbm = fmaxf(bm, obm);
+        bl = (bm == -INFINITY ? 0.f : bl * exp2f(bm - nbm)) + (obm == -INFINITY ? 0.f : obl * exp2f(obm - nbm));
+        bm = nbm;
+        sd = fmaxf(sd, __shfl_xor_sync(0xffffffffu, sd, o));
+    }
+    if (lane < G) {
+        sm_ml[warp][lane][0] = m;
+        sm_ml[warp][lane][1] = l;
+        sm_ml[warp][lane][2] = bm;
+        sm_ml[warp][lane][3] = bl;
+        sm_ml[warp][lane][4] = sd;
+    }
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) sm_acc[warp][h][lane * DPL + e] = acc[h][e];
+    __syncthreads();
+    // combine the warps: per head and element
+    float *part_out = reinterpret_cast<float *>(state + L.part);
+    float *band_out = reinterpret_cast<float *>(state + L.band);
+    for (int t = threadIdx.x; t < G * DD; t += blockDim.x) {
+        const int h = t / DD, x = t % DD;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w_ = 0; w_ < NW; ++w_) M = fmaxf(M, sm_ml[w_][h][0]);
+        float A = 0.f, Ls = 0.f;
+#pragma unroll
+        for (int w_ = 0; w_ < NW; ++w_) {
+            const float mw = sm_ml[w_][h][0];
+            const float f = mw == -INFINITY ? 0.f : exp2f(mw - M);
+            A = fmaf(sm_acc[w_][h][x], f, A);
+            Ls = fmaf(sm_ml[w_][h][1], f, Ls);
+        }
+        const size_t pi = ((size_t)b * s.H + g * G + h) * kDecodeMaxSplits + split;
+        float *pp = part_out + pi * (s.d + 2);
+        pp[2 + x] = A;
+        if (x == 0) {
+            pp[0] = M == -INFINITY ? M : M * kLn2f;
+            pp[1] = Ls;
+            float BM = -INFINITY, SD = -INFINITY;
+#pragma unroll
+            for (int w_ = 0; w_ < NW; ++w_) {
+                BM = fmaxf(BM, sm_ml[w_][h][2]);
+                SD = fmaxf(SD, sm_ml[w_][h][4]);
+            }
+            float BL = 0.f;
+#pragma unroll
+            for (int w_ = 0; w_ < NW; ++w_) {
+                const float b_ = sm_ml[w_][h][2];
+                if (b_ != -INFINITY) BL = fmaf(sm_ml[w_][h][3], exp2f(b_ - BM), BL);
+            }
+            band_out[pi * 3 + 0] = BM == -INFINITY ? BM : BM * kLn2f;
+            band_out[pi * 3 + 1] = BL;
+            band_out[pi * 3 + 2] = SD == -INFINITY ? SD : SD * kLn2f;
+        }
+    }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(128) decode_combine_kernel(Dims s, DecodeLayout L, unsigned char *state, StepGeom gm,
                                                              const T *__restrict__ q_t, const T *__restrict__ Wq,
@@ -435,13 +656,26 @@ static cudaError_t decode_step_t(const Dims &s, unsigned char *state, const Deco
         gm.nk = 0;
         gm.n = 0;
     }
-    gm.nsplit = gm.n == 0 ? 0 : min(kDecodeMaxSplits, (gm.n + 255) / 256);
+    gm.nsplit = gm.n == 0 ? 0 : min(kDecodeMaxSplits, (gm.n + 511) / 512);
     gm.per = gm.nsplit ? (gm.n + gm.nsplit - 1) / gm.nsplit : 0;
     const int BK = s.B * s.Hkv;
     decode_append_kernel<T><<<BK, 128, 0, st>>>(s, L, state, pos, (const T *)k_t, (const T *)v_t, err);
     ++*launches;
     if (gm.nsplit) {
-        decode_attn_kernel<T><<<dim3(BK, gm.nsplit), 128, 0, st>>>(s, L, state, gm, (const T *)q_t);
+        const dim3 grid(BK, gm.nsplit);
+        const int G = s.G();
+#define STILL_DECODE_PACKED(DPL, GG) \
+    decode_attn_packed_kernel<T, DPL, GG><<<grid, 256, 0, st>>>(s, L, state, gm, (const T *)q_t)
+        if (s.d == 128 && G == 4) STILL_DECODE_PACKED(4, 4);
+        else if (s.d == 128 && G == 8) STILL_DECODE_PACKED(4, 8);
+        else if (s.d == 128 && G == 2) STILL_DECODE_PACKED(4, 2);
+        else if (s.d == 128 && G == 1 && sizeof(T) == 2) STILL_DECODE_PACKED(4, 1);
+        else if (s.d == 64 && G == 4) STILL_DECODE_PACKED(2, 4);
+        else if (s.d == 64 && G == 8) STILL_DECODE_PACKED(2, 8);
+        else if (s.d == 64 && G == 2) STILL_DECODE_PACKED(2, 2);
+        else if (s.d == 64 && G == 1) STILL_DECODE_PACKED(2, 1);
+        else decode_attn_kernel<T><<<grid, 128, 0, st>>>(s, L, state, gm, (const T *)q_t);
+#undef STILL_DECODE_PACKED
         ++*launches;
     }
     decode_combine_kernel<T><<<BK, 128, 0, st>>>(s, L, state, gm, (const T *)q_t, (const T *)Wq, (const T *)Wk,
