@@ -157,6 +157,31 @@ STILL_API still_status still_hybrid_prefill(const still_dims *dims, const void *
                                   size_t workspace_bytes, void *state, int state_capacity, void *stream);
 
 /*
+ * still_hybrid_prefill with its scratch in a fixed device array inside this
+ * library instead of a caller workspace (no counterpart in the method: the
+ * pages describe no memory management).  Same arguments, results and errors as
+ * still_hybrid_prefill, minus workspace and workspace_bytes.  It allocates
+ * nothing: no device, host or pinned memory, directly or through a library.
+ *   - Limit: shapes with still_prefill_workspace_bytes(dims) greater than
+ *     STILL_STATIC_WORKSPACE_BYTES (64 MiB) are rejected with
+ *     STILL_ERR_WORKSPACE before any work; use still_hybrid_prefill for them.
+ *   - Nothing in the array has to start at zero: each call writes every part of
+ *     the scratch it reads (its counter of recomputed rows is reset by the call
+ *     itself), so leftovers of earlier calls, of any shape, do no harm.
+ *   - One array per device: calls that overlap in time on one device (other
+ *     streams, other host threads) share it and race; serialise them.
+ *   - The array's address is looked up once per device, with that device
+ *     current, on the first call there (which may load the library's module for
+ *     it); make that first call before any stream capture.
+ * STILL_ERR_CUDA if the current device or the array's address cannot be had.
+ */
+#define STILL_STATIC_WORKSPACE_BYTES (64u << 20)
+STILL_API still_status still_hybrid_prefill_static(const still_dims *dims, const void *q, const void *k,
+                                                   const void *v, const void *Wq, const void *Wk, void *o,
+                                                   const int32_t *idx_in, void *state, int state_capacity,
+                                                   void *stream);
+
+/*
  * Chunk-granular delayed decode ([p1] "Chunk-Wise": during decoding the
  * selection is delayed at chunk granularity).  The state is one caller-owned
  * device buffer holding, per (b, g): the kept K/V cache, the linear state

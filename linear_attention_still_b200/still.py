@@ -21,7 +21,8 @@ STATUS = {0: "STILL_OK", 1: "STILL_ERR_INVALID_ARG", 2: "STILL_ERR_UNSUPPORTED",
 EXPORTS = ("still_status_string", "still_saliency", "still_select_topk", "still_npmap",
            "still_prefill_workspace_bytes", "still_prefill_workspace_layout", "still_hybrid_prefill",
            "still_decode_state_bytes", "still_decode_init", "still_decode_step", "still_get_device_status",
-           "still_launch_count", "still_timing_enable", "still_timing_read", "still_debug_set_trace")
+           "still_launch_count", "still_timing_enable", "still_timing_read", "still_debug_set_trace",
+           "still_hybrid_prefill_static")
 
 
 class StillError(RuntimeError):
@@ -53,6 +54,7 @@ _SIG = {
     "still_prefill_workspace_bytes": ([_D], ct.c_size_t),
     "still_prefill_workspace_layout": ([_D, ct.POINTER(still_ws_layout)], ct.c_int),
     "still_hybrid_prefill": ([_D, _P, _P, _P, _P, _P, _P, _P, _P, ct.c_size_t, _P, ct.c_int, _P], ct.c_int),
+    "still_hybrid_prefill_static": ([_D, _P, _P, _P, _P, _P, _P, _P, _P, ct.c_int, _P], ct.c_int),
     "still_decode_state_bytes": ([_D, ct.c_int], ct.c_size_t),
     "still_decode_init": ([_D, ct.c_int, _P, _P], ct.c_int),
     "still_decode_step": ([_D, _P, ct.c_int, ct.c_int, _P, _P, _P, _P, _P, _P, _P], ct.c_int),
@@ -141,6 +143,16 @@ def still_hybrid_prefill(dims, q, k, v, wq, wk, o, idx_in=None, workspace=None, 
         _lib.still_hybrid_prefill(ct.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(wq), _ptr(wk), _ptr(o),
                                   _ptr(idx_in), _ptr(workspace), int(workspace_bytes), _ptr(state),
                                   int(state_capacity), _stream(stream)))
+
+
+STATIC_WORKSPACE_BYTES = 64 << 20  # STILL_STATIC_WORKSPACE_BYTES
+
+
+def still_hybrid_prefill_static(dims, q, k, v, wq, wk, o, idx_in=None, state=None, state_capacity=0, stream=None):
+    """still_hybrid_prefill with the library's fixed device scratch (allocates nothing)."""
+    _ok("still_hybrid_prefill_static",
+        _lib.still_hybrid_prefill_static(ct.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(wq), _ptr(wk), _ptr(o),
+                                         _ptr(idx_in), _ptr(state), int(state_capacity), _stream(stream)))
 
 
 def still_decode_state_bytes(dims, capacity: int) -> int:
