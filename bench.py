@@ -111,6 +111,12 @@ class ClockSampler:
             return
         self.thread = threading.Thread(target=self._read, daemon=True)
         self.thread.start()
+        # nvidia-smi takes a moment to start: wait for its first sample, so that a short timed
+        # region still gets samples of its own, then keep only those
+        t_end = time.time() + 5.0
+        while not self.rows and time.time() < t_end and self.proc.poll() is None:
+            time.sleep(0.01)
+        self.rows.clear()
 
     def _read(self):
         for line in self.proc.stdout:

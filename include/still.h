@@ -12,8 +12,9 @@
  *
  * Conventions (all entry points):
  *  - Every tensor argument is a caller-owned DEVICE pointer in the row-major
- *    layout stated at the call, 16-byte aligned.  The library never allocates
- *    device memory; scratch space is passed in by the caller.
+ *    layout stated at the call, 16-byte aligned.  No call allocates memory;
+ *    scratch space is passed in by the caller (still_hybrid_prefill_static
+ *    uses a fixed array of the library instead).
  *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
  *    stream).  Every call is asynchronous on that stream.
  *  - Argument errors are detected on the host before anything is launched and
@@ -233,8 +234,12 @@ STILL_API uint64_t still_launch_count(void);
  * Diagnostics (no counterpart in the method): when `words` is non-NULL, the
  * tensor-core merge kernel records 16 progress words per CTA there (producer,
  * MMA issuer and each softmax warp: last step reached; 0xBAD.. on a bounded
- * wait that gave up; 0xD0E / 0xF1F at exit).  Pass host-mapped (pinned)
- * memory to read it while a kernel runs.  NULL (the default) disables it.
+ * wait that gave up; SM clock at CTA start, first score tile, epilogue and
+ * exit in words 10..13; 0xD0E / 0xF1F at exit).  The window-phase launch
+ * (G' = B*Hkv*G/2*ceil(N/128) CTAs) writes words [0, 16 G' + 2049); the
+ * kept-prefix launch writes from word 16 G' + 2080 on.  Pass host-mapped
+ * (pinned) memory to read it while a kernel runs.  NULL (the default)
+ * disables it.
  */
 STILL_API void still_debug_set_trace(unsigned *words);
 

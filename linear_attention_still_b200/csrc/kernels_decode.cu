@@ -15,6 +15,7 @@
 #include "common.cuh"
 #include "rowops.cuh"
 #include "still_internal.h"
+#include "tc_ptx.cuh"
 #include "topk.cuh"
 
 namespace still {
@@ -259,14 +260,28 @@ __global__ void __launch_bounds__(256) decode_attn_packed_kernel(Dims s, DecodeL
 #pragma unroll
         for (int e = 0; e < DPL; ++e) acc[h][e] = 0.f;
     const int my_kk = lane / G;
+    const size_t dv_kept = L.vhat - L.khat, dv_ring = L.ring_v - L.ring_k;
     for (int base = l0 + warp * KG; base < l1; base += NW * KG) {
+        // lane kk < KG works out where key base+kk lives (byte offset of its K row in the state; bit 0
+        // set for a window-ring row) and the warp shares it; keys past the end re-read the last key of
+        // the range, with probability zero
+        unsigned long long my_off = 0;
+        if (lane < KG) {
+            const int li = min(base + lane, l1 - 1);
+            if (li < gm.nk) {
+                my_off = L.khat + ((size_t)bg * L.cap_chunks * s.k + li) * s.d * sizeof(T);
+            } else {
+                const int j = gm.lo + (li - gm.nk);
+                my_off = (L.ring_k + ((size_t)bg * L.ring_rows + ring_row(s, j)) * s.d * sizeof(T)) | 1ull;
+            }
+        }
         RowSlice<T, DPL> kr[KG], vr[KG];
 #pragma unroll
         for (int kk = 0; kk < KG; ++kk) {
-            // rows past the end re-read the last row of the range; their probabilities are zero
-            const int li = min(base + kk, l1 - 1);
-            kr[kk].load(list_row<T>(s, L, state, bg, gm, li, false), lane);
-            vr[kk].load(list_row<T>(s, L, state, bg, gm, li, true), lane);
+            const unsigned long long off = __shfl_sync(0xffffffffu, my_off, kk);
+            const size_t ko = off & ~1ull, vo = ko + ((off & 1ull) ? dv_ring : dv_kept);
+            kr[kk].load(reinterpret_cast<const T *>(state + ko), lane);
+            vr[kk].load(reinterpret_cast<const T *>(state + vo), lane);
         }
         float part[32];
 #pragma unroll
@@ -367,6 +382,218 @@ __global__ void __launch_bounds__(256) decode_attn_packed_kernel(Dims s, DecodeL
         }
         const size_t pi = ((size_t)b * s.H + g * G + h) * kDecodeMaxSplits + split;
         float *pp = part_out + pi * (s.d + 2);
+        pp[2 + x] = A;
+        if (x == 0) {
+            pp[0] = M == -INFINITY ? M : M * kLn2f;
+            pp[1] = Ls;
+            float BM = -INFINITY, SD = -INFINITY;
+#pragma unroll
+            for (int w_ = 0; w_ < NW; ++w_) {
+                BM = fmaxf(BM, sm_ml[w_][h][2]);
+                SD = fmaxf(SD, sm_ml[w_][h][4]);
+            }
+            float BL = 0.f;
+#pragma unroll
+            for (int w_ = 0; w_ < NW; ++w_) {
+                const float b_ = sm_ml[w_][h][2];
+                if (b_ != -INFINITY) BL = fmaf(sm_ml[w_][h][3], exp2f(b_ - BM), BL);
+            }
+            band_out[pi * 3 + 0] = BM == -INFINITY ? BM : BM * kLn2f;
+            band_out[pi * 3 + 1] = BL;
+            band_out[pi * 3 + 2] = SD == -INFINITY ? SD : SD * kLn2f;
+        }
+    }
+}
+
+// bf16 decode attention on the warp-level tensor-core instruction (mma.sync m16n8k16, fp32
+// accumulate).  The step is bound by HBM (every kept and window row is read once); the SIMT form
+// of the same contraction spends more issue slots on shuffles and conversions than the memory
+// time allows, while one MMA does a 16-key x 16-dim slice for all heads of the group.  The G <= 8
+// query heads of the group are rows 0..G-1 of the 16-row A operand (the rest are zero).
+//   S^T tile: A = Q (heads x 16 dims), B = K^T (16 dims x 8 keys): a lane loads one 16-byte slice of
+//   a K row and uses it as the B fragments of two k-steps; Q's fragments follow the same
+//   permutation of the head dimension (a dot product does not depend on the order of its terms).
+//   O += P V: A = P (heads x 16 keys, straight from the score fragments), B = V (16 keys x 8 dims):
+//   a lane loads a contiguous DH/8-dim slice of four V rows and pairs rows with a byte permute;
+//   output column n of n-tile j is head dimension n*DH/8 + j.
+// Scores in log2 units; partials written in natural units (same format as decode_attn_kernel).
+__device__ __forceinline__ void mma16816(float (&c)[4], unsigned a0, unsigned a2, unsigned b0, unsigned b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+
+template <int DH, int G>
+__global__ void __launch_bounds__(128) decode_attn_mma_kernel(Dims s, DecodeLayout L, unsigned char *state,
+                                                              StepGeom gm, const __nv_bfloat16 *__restrict__ q_t) {
+    constexpr int NW = 4, NQ = DH / 32, NT = DH / 8, VW = DH / 64;
+    constexpr float kL2e = 1.4426950408889634f, kLn2f = 0.6931471805599453f;
+    static_assert(G >= 1 && G <= 8 && (DH == 64 || DH == 128), "decode mma shape");
+    __shared__ float sm_ml[NW][G][5];  // m, l, bm, bl, sdiag (log2 units)
+    __shared__ float sm_acc[NW][G][DH];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, c = lane & 3;
+    const int bg = blockIdx.x, split = blockIdx.y, b = bg / s.Hkv, g = bg % s.Hkv;
+    const int l0 = split * gm.per, l1 = min(gm.n, l0 + gm.per);
+    const int band_lo = max(0, gm.pos - s.w + 1);
+    const float sl2 = s.scale * kL2e;
+    const size_t dv_kept = L.vhat - L.khat, dv_ring = L.ring_v - L.ring_k;
+    constexpr size_t kRow = DH * sizeof(__nv_bfloat16);
+
+    unsigned qa0[2 * NQ], qa2[2 * NQ];
+#pragma unroll
+    for (int i = 0; i < NQ; ++i) {
+        uint4 u = make_uint4(0u, 0u, 0u, 0u);
+        if (gq < G) u = __ldg(reinterpret_cast<const uint4 *>(q_t + ((size_t)b * s.H + g * G + gq) * DH) + 4 * i + c);
+        qa0[2 * i] = u.x;
+        qa2[2 * i] = u.y;
+        qa0[2 * i + 1] = u.z;
+        qa2[2 * i + 1] = u.w;
+    }
+    float o[NT][4];
+#pragma unroll
+    for (int j = 0; j < NT; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+    float m = -INFINITY, l = 0.f, bm = -INFINITY, bl = 0.f, sd = -INFINITY;
+
+    for (int base = l0 + warp * 16; base < l1; base += NW * 16) {
+        // lane kk < 16 locates key base+kk (byte offset of its K row in the state, bit 0 set for a
+        // window-ring row); keys past the end re-read the last key of the range with probability zero
+        unsigned long long my_off = 0;
+        if (lane < 16) {
+            const int li = min(base + lane, l1 - 1);
+            if (li < gm.nk) {
+                my_off = L.khat + ((size_t)bg * L.cap_chunks * s.k + li) * kRow;
+            } else {
+                const int j = gm.lo + (li - gm.nk);
+                my_off = (L.ring_k + ((size_t)bg * L.ring_rows + ring_row(s, j)) * kRow) | 1ull;
+            }
+        }
+        uint4 kr[2][NQ], vr[4][VW];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const unsigned long long off = __shfl_sync(0xffffffffu, my_off, gq + 8 * h) & ~1ull;
+            const uint4 *row = reinterpret_cast<const uint4 *>(state + off);
+#pragma unroll
+            for (int i = 0; i < NQ; ++i) kr[h][i] = __ldg(row + 4 * i + c);
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const unsigned long long off = __shfl_sync(0xffffffffu, my_off, 2 * c + (r & 1) + 8 * (r >> 1));
+            const size_t vo = (off & ~1ull) + ((off & 1ull) ? dv_ring : dv_kept);
+            const uint4 *row = reinterpret_cast<const uint4 *>(state + vo);
+#pragma unroll
+            for (int i = 0; i < VW; ++i) vr[r][i] = __ldg(row + gq * VW + i);
+        }
+        // S^T for keys base+[0,8) and base+[8,16)
+        float st[2][4];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            st[h][0] = st[h][1] = st[h][2] = st[h][3] = 0.f;
+#pragma unroll
+            for (int i = 0; i < NQ; ++i) {
+                mma16816(st[h], qa0[2 * i], qa2[2 * i], kr[h][i].x, kr[h][i].y);
+                mma16816(st[h], qa0[2 * i + 1], qa2[2 * i + 1], kr[h][i].z, kr[h][i].w);
+            }
+        }
+        // this lane's scores: head gq, keys 2c, 2c+1, 8+2c, 9+2c
+        float sc[4];
+        float mx = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int li = base + 2 * c + (e & 1) + 8 * (e >> 1);
+            float x = st[e >> 1][e & 1] * sl2;
+            if (li >= l1) x = -INFINITY;
+            if (li < l1 && li >= gm.nk) {
+                const int j = gm.lo + (li - gm.nk);
+                if (j == gm.pos) {
+                    sd = x;
+                } else if (j >= band_lo) {
+                    if (x > bm) {
+                        bl = bl * tc::ex2(bm - x) + 1.f;
+                        bm = x;
+                    } else {
+                        bl += tc::ex2(x - bm);
+                    }
+                }
+            }
+            sc[e] = x;
+            mx = fmaxf(mx, x);
+        }
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        const float mn = fmaxf(m, mx);  // finite: key base+0 is always in range
+        const float so = tc::ex2(m - mn);  // m = -inf gives 0
+        float p[4], ps = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            p[e] = tc::ex2(sc[e] - mn);
+            ps += p[e];
+        }
+        ps += __shfl_xor_sync(0xffffffffu, ps, 1);
+        ps += __shfl_xor_sync(0xffffffffu, ps, 2);
+        l = l * so + ps;
+        m = mn;
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+            o[j][0] *= so;
+            o[j][1] *= so;
+        }
+        const unsigned pa0 = tc::pack_bf16x2(p[0], p[1]), pa2 = tc::pack_bf16x2(p[2], p[3]);
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+            const unsigned *w0 = reinterpret_cast<const unsigned *>(&vr[0][0]);
+            const unsigned *w1 = reinterpret_cast<const unsigned *>(&vr[1][0]);
+            const unsigned *w2 = reinterpret_cast<const unsigned *>(&vr[2][0]);
+            const unsigned *w3 = reinterpret_cast<const unsigned *>(&vr[3][0]);
+            const unsigned sel = (j & 1) ? 0x7632u : 0x5410u;
+            const unsigned b0 = __byte_perm(w0[j >> 1], w1[j >> 1], sel);
+            const unsigned b1 = __byte_perm(w2[j >> 1], w3[j >> 1], sel);
+            mma16816(o[j], pa0, pa2, b0, b1);
+        }
+    }
+    // band statistics of head gq: combine the four lanes of the row
+#pragma unroll
+    for (int x = 1; x <= 2; x <<= 1) {
+        const float obm = __shfl_xor_sync(0xffffffffu, bm, x);
+        const float obl = __shfl_xor_sync(0xffffffffu, bl, x);
+        const float nbm = fmaxf(bm, obm);
+        bl = (bm == -INFINITY ? 0.f : bl * tc::ex2(bm - nbm)) + (obm == -INFINITY ? 0.f : obl * tc::ex2(obm - nbm));
+        bm = nbm;
+        sd = fmaxf(sd, __shfl_xor_sync(0xffffffffu, sd, x));
+    }
+    if (gq < G) {
+        if (c == 0) {
+            sm_ml[warp][gq][0] = m;
+            sm_ml[warp][gq][1] = l;
+            sm_ml[warp][gq][2] = bm;
+            sm_ml[warp][gq][3] = bl;
+            sm_ml[warp][gq][4] = sd;
+        }
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+            sm_acc[warp][gq][(2 * c) * NT + j] = o[j][0];
+            sm_acc[warp][gq][(2 * c + 1) * NT + j] = o[j][1];
+        }
+    }
+    __syncthreads();
+    float *part_out = reinterpret_cast<float *>(state + L.part);
+    float *band_out = reinterpret_cast<float *>(state + L.band);
+    for (int t = threadIdx.x; t < G * DH; t += blockDim.x) {
+        const int h = t / DH, x = t % DH;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w_ = 0; w_ < NW; ++w_) M = fmaxf(M, sm_ml[w_][h][0]);
+        float A = 0.f, Ls = 0.f;
+#pragma unroll
+        for (int w_ = 0; w_ < NW; ++w_) {
+            const float mw = sm_ml[w_][h][0];
+            const float f = mw == -INFINITY ? 0.f : exp2f(mw - M);
+            A = fmaf(sm_acc[w_][h][x], f, A);
+            Ls = fmaf(sm_ml[w_][h][1], f, Ls);
+        }
+        const size_t pi = ((size_t)b * s.H + g * G + h) * kDecodeMaxSplits + split;
+        float *pp = part_out + pi * (DH + 2);
         pp[2 + x] = A;
         if (x == 0) {
             pp[0] = M == -INFINITY ? M : M * kLn2f;
@@ -498,6 +725,153 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(Dims s, DecodeLayou
         for (int hh = 0; hh < G; ++hh) acc += sig[hh];
         float *rr = reinterpret_cast<float *>(state + L.ring_r);
         rr[(size_t)bg * L.ring_rows + ring_row(s, gm.pos)] = s.w > 0 ? acc / (float)G : 0.f;
+        if (bg == 0) reinterpret_cast<DecodeHeader *>(state + L.header)->pos = gm.pos + 1;
+    }
+}
+
+// Combine for a window (w > 0) and G <= 8: one CTA of 256 threads per (b, g) does every head of the
+// group at once, with the work spread over all threads: split factors (a warp per head), the
+// softmax part (thread per (head, element)), Y = q Wq (thread per (head, feature), the d-long sums
+// unrolled so the Wq loads overlap), NP-Map per head, phi(q)^T S with S read once for the group
+// (thread per (element, slice of the features)), and the merge under the shared normaliser.
+constexpr int kCombineThreads = 256;
+
+size_t combine_wide_smem(const Dims &s) {
+    const int G = s.G(), P = kCombineThreads / s.d;
+    return (size_t)(G * 64 + G * 8 + 2 * G * s.d + G * s.D + P * G * s.d) * sizeof(float);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kCombineThreads) decode_combine_wide_kernel(Dims s, DecodeLayout L,
+                                                                              unsigned char *state, StepGeom gm,
+                                                                              const T *__restrict__ q_t,
+                                                                              const T *__restrict__ Wq,
+                                                                              T *__restrict__ o_t) {
+    extern __shared__ float cs[];
+    const int G = s.G(), d = s.d, D = s.D, ns = gm.nsplit, P = kCombineThreads / d;
+    float *sf = cs;           // [G][64] weight of each split
+    float *st = sf + G * 64;  // [G][8]: M, Ls, BM, BL, SD, lden, sigma
+    float *os = st + G * 8;   // [G][d] softmax numerator
+    float *qs = os + G * d;   // [G][d]
+    float *ph = qs + G * d;   // [G][D] Y, then phi(q)
+    float *lp = ph + G * D;   // [P][G][d] partial phi(q)^T S
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int bg = blockIdx.x, b = bg / s.Hkv, g = bg % s.Hkv;
+    const float *part = reinterpret_cast<const float *>(state + L.part);
+    const float *band = reinterpret_cast<const float *>(state + L.band);
+    const float *S = reinterpret_cast<const float *>(state + L.S) + (size_t)bg * D * d;
+    const float *z = reinterpret_cast<const float *>(state + L.z) + (size_t)bg * D;
+    const size_t pb0 = ((size_t)b * s.H + g * G) * kDecodeMaxSplits;
+
+    for (int hh = warp; hh < G; hh += kCombineThreads / 32) {
+        const size_t pb = pb0 + (size_t)hh * kDecodeMaxSplits;
+        float M = -INFINITY, BM = -INFINITY, SD = -INFINITY;
+        for (int sp = lane; sp < ns; sp += 32) {
+            M = fmaxf(M, part[(pb + sp) * (d + 2)]);
+            BM = fmaxf(BM, band[(pb + sp) * 3]);
+            SD = fmaxf(SD, band[(pb + sp) * 3 + 2]);
+        }
+        M = warp_max(M);
+        BM = warp_max(BM);
+        SD = warp_max(SD);
+        float Ls = 0.f, BL = 0.f;
+        for (int sp = lane; sp < ns; sp += 32) {
+            const float ms = part[(pb + sp) * (d + 2)];
+            const float f = ms == -INFINITY ? 0.f : expf(ms - M);
+            sf[hh * 64 + sp] = f;
+            Ls = fmaf(part[(pb + sp) * (d + 2) + 1], f, Ls);
+            const float bms = band[(pb + sp) * 3];
+            if (bms != -INFINITY) BL = fmaf(band[(pb + sp) * 3 + 1], expf(bms - BM), BL);
+        }
+        Ls = warp_sum(Ls);
+        BL = warp_sum(BL);
+        if (lane == 0) {
+            st[hh * 8 + 0] = M;
+            st[hh * 8 + 1] = Ls;
+            const int band_lo = max(0, gm.pos - s.w + 1);
+            st[hh * 8 + 6] = (band_lo == gm.pos) ? INFINITY : softplus_f(SD - (BM + logf(BL)));
+        }
+    }
+    for (int t = tid; t < G * d; t += kCombineThreads) qs[t] = to_f(q_t[((size_t)b * s.H + g * G) * d + t]);
+    __syncthreads();
+    for (int t = tid; t < G * d; t += kCombineThreads) {
+        const int hh = t / d, x = t % d;
+        const float *pp = part + (pb0 + (size_t)hh * kDecodeMaxSplits) * (d + 2) + 2 + x;
+        float a = 0.f;
+        for (int sp = 0; sp < ns; ++sp) a = fmaf(pp[(size_t)sp * (d + 2)], sf[hh * 64 + sp], a);
+        os[t] = a;
+    }
+    for (int t = tid; t < G * D; t += kCombineThreads) {
+        const int hh = t / D, a = t % D;
+        const T *w = Wq + (size_t)(g * G + hh) * d * D + a;
+        const float *qh = qs + hh * d;
+        float y[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int x = 0; x < d; x += 8) {  // d is a multiple of 8
+#pragma unroll
+            for (int e = 0; e < 8; ++e) y[e] = fmaf(qh[x + e], to_f(w[(size_t)(x + e) * D]), y[e]);
+        }
+        ph[t] = ((y[0] + y[1]) + (y[2] + y[3])) + ((y[4] + y[5]) + (y[6] + y[7]));
+    }
+    __syncthreads();
+    // NP-Map of each head's query ([p1] "Norm-Preserved Feature Map") and phi(q) . z
+    for (int hh = warp; hh < G; hh += kCombineThreads / 32) {
+        float *yh = ph + hh * D;
+        float mx = -INFINITY;
+        for (int a = lane; a < D; a += 32) mx = fmaxf(mx, yh[a]);
+        mx = warp_max(mx);
+        float ee = 0.f;
+        for (int a = lane; a < D; a += 32) {
+            const float e = expf(yh[a] - mx);
+            yh[a] = e;
+            ee = fmaf(e, e, ee);
+        }
+        ee = warp_sum(ee);
+        float nq = 0.f;
+        for (int x = lane; x < d; x += 32) nq = fmaf(qs[hh * d + x], qs[hh * d + x], nq);
+        nq = warp_sum(nq);
+        const float f = sqrtf(nq) / sqrtf(ee);
+        float ld = 0.f;
+        for (int a = lane; a < D; a += 32) {
+            const float v = yh[a] * f;
+            yh[a] = v;
+            ld = fmaf(v, z[a], ld);
+        }
+        ld = warp_sum(ld);
+        if (lane == 0) st[hh * 8 + 5] = ld;
+    }
+    __syncthreads();
+    if (tid < P * d) {
+        const int x = tid % d, pi = tid / d;
+        const int a0 = pi * D / P, a1 = (pi + 1) * D / P;
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int a = a0; a < a1; ++a) {
+            const float sv = S[(size_t)a * d + x];
+#pragma unroll
+            for (int hh = 0; hh < 8; ++hh)
+                if (hh < G) acc[hh] = fmaf(ph[hh * D + a], sv, acc[hh]);
+        }
+#pragma unroll
+        for (int hh = 0; hh < 8; ++hh)
+            if (hh < G) lp[(pi * G + hh) * d + x] = acc[hh];
+    }
+    __syncthreads();
+    for (int t = tid; t < G * d; t += kCombineThreads) {
+        const int hh = t / d, x = t % d;
+        float lin = 0.f;
+        for (int pi = 0; pi < P; ++pi) lin += lp[(pi * G + hh) * d + x];
+        const float M = st[hh * 8 + 0], Ls = st[hh * 8 + 1], ld = st[hh * 8 + 5];
+        const float Ms = ld > 0.f ? fmaxf(M, logf(ld)) : M;
+        const float a_soft = (M == -INFINITY) ? 0.f : expf(M - Ms);
+        const float a_lin = (Ms == -INFINITY) ? 0.f : expf(-Ms);
+        const float den = Ls * a_soft + ld * a_lin;
+        const float inv = den > 0.f ? 1.f / den : 0.f;
+        o_t[((size_t)b * s.H + g * G + hh) * d + x] = from_f<T>((os[t] * a_soft + lin * a_lin) * inv);
+    }
+    if (tid == 0) {
+        float acc = 0.f;
+        for (int hh = 0; hh < G; ++hh) acc += st[hh * 8 + 6];
+        float *rr = reinterpret_cast<float *>(state + L.ring_r);
+        rr[(size_t)bg * L.ring_rows + ring_row(s, gm.pos)] = acc / (float)G;
         if (bg == 0) reinterpret_cast<DecodeHeader *>(state + L.header)->pos = gm.pos + 1;
     }
 }
@@ -666,7 +1040,23 @@ static cudaError_t decode_step_t(const Dims &s, unsigned char *state, const Deco
         const int G = s.G();
 #define STILL_DECODE_PACKED(DPL, GG) \
     decode_attn_packed_kernel<T, DPL, GG><<<grid, 256, 0, st>>>(s, L, state, gm, (const T *)q_t)
-        if (s.d == 128 && G == 4) STILL_DECODE_PACKED(4, 4);
+#define STILL_DECODE_MMA(DH, GG) \
+    decode_attn_mma_kernel<DH, GG><<<grid, 128, 0, st>>>(s, L, state, gm, (const __nv_bfloat16 *)q_t)
+        const bool mma = sizeof(T) == 2 && (s.d == 64 || s.d == 128) && (G == 1 || G == 2 || G == 4 || G == 8);
+        if (mma) {
+            if (s.d == 128) {
+                if (G == 1) STILL_DECODE_MMA(128, 1);
+                else if (G == 2) STILL_DECODE_MMA(128, 2);
+                else if (G == 4) STILL_DECODE_MMA(128, 4);
+                else STILL_DECODE_MMA(128, 8);
+            } else {
+                if (G == 1) STILL_DECODE_MMA(64, 1);
+                else if (G == 2) STILL_DECODE_MMA(64, 2);
+                else if (G == 4) STILL_DECODE_MMA(64, 4);
+                else STILL_DECODE_MMA(64, 8);
+            }
+        }
+        else if (s.d == 128 && G == 4) STILL_DECODE_PACKED(4, 4);
         else if (s.d == 128 && G == 8) STILL_DECODE_PACKED(4, 8);
         else if (s.d == 128 && G == 2) STILL_DECODE_PACKED(4, 2);
         else if (s.d == 128 && G == 1 && sizeof(T) == 2) STILL_DECODE_PACKED(4, 1);
@@ -676,10 +1066,22 @@ static cudaError_t decode_step_t(const Dims &s, unsigned char *state, const Deco
         else if (s.d == 64 && G == 1) STILL_DECODE_PACKED(2, 1);
         else decode_attn_kernel<T><<<grid, 128, 0, st>>>(s, L, state, gm, (const T *)q_t);
 #undef STILL_DECODE_PACKED
+#undef STILL_DECODE_MMA
         ++*launches;
     }
-    decode_combine_kernel<T><<<BK, 128, 0, st>>>(s, L, state, gm, (const T *)q_t, (const T *)Wq, (const T *)Wk,
-                                                 (T *)o_t);
+    if (s.w > 0 && s.G() <= 8) {
+        const size_t smem = combine_wide_smem(s);
+        if (smem > 48 * 1024) {
+            cudaError_t e = cudaFuncSetAttribute(decode_combine_wide_kernel<T>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+        }
+        decode_combine_wide_kernel<T><<<BK, kCombineThreads, smem, st>>>(s, L, state, gm, (const T *)q_t,
+                                                                        (const T *)Wq, (T *)o_t);
+    } else {
+        decode_combine_kernel<T><<<BK, 128, 0, st>>>(s, L, state, gm, (const T *)q_t, (const T *)Wq, (const T *)Wk,
+                                                     (T *)o_t);
+    }
     ++*launches;
     if (pos % s.C == s.C - 1 && gm.t - m >= 0) {
         const int P = pow2_ceil(s.C), Pk = pow2_ceil(s.k > 0 ? s.k : 1);

@@ -190,6 +190,7 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(bar_area + Cfg::ABORT_OFF);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) trace_word(p.trace, 10, (unsigned)clock());
 
     // ---- CTA -> (b, g, head pair, query tile); heavier (later) query tiles first
     const int per_qt = p.B * p.Hkv * p.pairs;
@@ -527,6 +528,7 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
             if (lane == 0) trace_word(p.trace, 2 + warp, (ok ? 0x100u : 0xB00u) + 0x10u * j + 1);
             if (!ok) break;
             if (threadIdx.x % 128 == 0) trace_time(p.trace, x, j, 0);
+            if (threadIdx.x == 0 && j == 0) trace_word(p.trace, 11, (unsigned)clock());
             tc_fence_after();
             float sv[128];
 #pragma unroll
@@ -636,6 +638,7 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
             if (lane == 0) trace_word(p.trace, 2 + warp, 0x100u + 0x10u * j + 2);
         }
         // ---- epilogue: o = O / l
+        if (threadIdx.x == 0) trace_word(p.trace, 12, (unsigned)clock());
         ok = warp_all(ok && (n_tiles > 0 ? mbar_wait(BAR(B_O + x), (n_tiles - 1) & 1, abort_flag) : true));
         if (lane == 0) trace_word(p.trace, 2 + warp, ok ? 0xE00 : 0xBADE);
         if (ok) {
@@ -688,6 +691,7 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (threadIdx.x == 0) trace_word(p.trace, 13, (unsigned)clock());
     if (threadIdx.x == 0) trace_word(p.trace, 14, 0xD0E);
     if (warp == Cfg::MMA_WARP) tmem_dealloc(tmem, Cfg::TMEM_COLS);
     if (threadIdx.x == 0) trace_word(p.trace, 15, 0xF1F);
@@ -1306,6 +1310,8 @@ cudaError_t launch_merge_cfg(int mode, const Dims &s, const MergeOperands &a, un
     prm.qt_first = qt_first;
     prm.pairs = s.G() / HP;
     prm.trace = debug_trace_words();
+    if (prm.trace && mode != kMergeLocal)  // the prefix phase records after the window phase's words
+        prm.trace += 16u * (unsigned)n_qtiles * s.B * s.Hkv * prm.pairs + 2048u + 32u;
     auto kern = mode == kMergeLocal ? merge_tc_kernel<DH, DF, HP, kMergeExpVariant, kMergeLocal>
                                     : merge_tc_kernel<DH, DF, HP, kMergeExpVariant, kMergePrefix>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);

@@ -18,12 +18,15 @@ CASES = {
     "f32_no_window": (Shape(B=1, H=2, Hkv=1, N=100, d=64, D=32, w=0, C=64, k=0, dtype="f32"), 60),
     "bf16_keep_none": (Shape(B=1, H=4, Hkv=2, N=250, d=64, D=64, w=128, C=128, k=0), 20),
     "bf16_from_empty": (Shape(B=1, H=4, Hkv=2, N=0, d=64, D=64, w=128, C=128, k=16), 300),
-    # one case per head-packing of the split-K attention kernel, plus the general-group fallback
+    # one case per instantiation of the split-K attention kernels (tensor-core bf16, packed SIMT
+    # fp32), plus the general-group fallback
     "f32_d128_g8": (Shape(B=1, H=8, Hkv=1, N=300, d=128, D=64, w=128, C=64, k=8, dtype="f32"), 100),
     "bf16_d128_mha": (Shape(B=2, H=2, Hkv=2, N=260, d=128, D=128, w=128, C=128, k=16), 140),
     "bf16_d128_g2": (Shape(B=1, H=4, Hkv=2, N=200, d=128, D=128, w=128, C=64, k=12), 80),
     "f32_d64_mha": (Shape(B=1, H=2, Hkv=2, N=200, d=64, D=64, w=64, C=64, k=8, dtype="f32"), 80),
     "bf16_d64_g8": (Shape(B=1, H=16, Hkv=2, N=200, d=64, D=64, w=128, C=64, k=8), 80),
+    "bf16_d128_g8": (Shape(B=1, H=8, Hkv=1, N=300, d=128, D=64, w=128, C=64, k=8), 100),
+    "bf16_d64_mha": (Shape(B=2, H=2, Hkv=2, N=200, d=64, D=64, w=64, C=64, k=8), 80),
     "bf16_g16_fallback": (Shape(B=1, H=16, Hkv=1, N=200, d=64, D=64, w=64, C=64, k=8), 80),
     "f32_d96_fallback": (Shape(B=1, H=4, Hkv=2, N=150, d=96, D=64, w=64, C=64, k=8, dtype="f32"), 60),
 }
