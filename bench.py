@@ -90,6 +90,33 @@ def layer_flops(shape):
 
 # ----------------------------------------------------------------------------- clocks
 
+def profiled_traffic(workload: str):
+    """DRAM bytes per step of the merge launches from a committed ncu summary under profiles/, or
+    None when there is none for this workload or the kernel sources changed since the capture."""
+    import glob
+    import hashlib
+    for path in glob.glob(os.path.join(ROOT, "profiles", "merge_tc_*.md")):
+        kv = {}
+        with open(path) as f:
+            for line in f:
+                if ":" in line and line.startswith("    "):
+                    k_, _, v_ = line.strip().partition(": ")
+                    kv[k_] = v_
+        if kv.get("workload") != workload or "traffic_bytes_per_step" not in kv:
+            continue
+        for item in kv.get("source_sha256", "").split():
+            name, _, digest = item.partition("=")
+            src = os.path.join(ROOT, "linear_attention_still_b200", "csrc", name)
+            try:
+                with open(src, "rb") as f:
+                    if not hashlib.sha256(f.read()).hexdigest().startswith(digest):
+                        return None
+            except OSError:
+                return None
+        return int(kv["traffic_bytes_per_step"])
+    return None
+
+
 class ClockSampler:
     FIELDS = ["index", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
               "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
@@ -366,7 +393,8 @@ def run_ours(args):
         "kernel": "merge (window phase + kept-prefix phase)", "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
         "frac": (achieved / peak) if (achieved and peak) else None,
         "peak_source": "measured bf16_tflops" if "bf16_tflops" in peaks else "fallback 1.59 PFLOP/s",
-        "traffic": None, "flops_per_step": merge_flops(shape), "ms_per_step": merge_ms / merge_n if merge_n else None,
+        "traffic": profiled_traffic(args.workload), "traffic_unit": "DRAM bytes per step (both merge launches, ncu)",
+        "flops_per_step": merge_flops(shape), "ms_per_step": merge_ms / merge_n if merge_n else None,
     }
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -375,7 +403,7 @@ def run_ours(args):
         "roofline": roofline,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches, "clocks": clocks,
-        "kernel_ms_per_step": {k_: v_[0] / args.steps for k_, v_ in kern.items()},
+        "kernel_ms_per_step": {k_: v_[0] / args.steps for k_, v_ in kern.items() if v_[1]},
         "layer_tflops": layer_flops(shape) / (ms_per_step / 1e3) / 1e12, "device_status": status,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -497,10 +525,18 @@ def run_decode(args):
     e2e_ms = max_over_ranks(sum(s_.elapsed_time(e_) for s_, e_ in e_evs), world, "cuda")
     # untimed steps up to the timed region, which ends at the last position: it holds the step that
     # closes a chunk (position C-1 mod C) along with ordinary ones
+    # the last (up to 64) of them also give the per-kernel breakdown, with events around each launch
+    n_brk = min(64, cap - K - pos)
+    still.still_timing_read()
     while pos < cap - K:
+        if pos == cap - K - n_brk:
+            still.still_timing_enable(True)
         still.still_decode_step(dims, state, cap, pos, wq, wk, qdd[pos - N], kdd[pos - N], vdd[pos - N], o_t)
         pos += 1
     torch.cuda.synchronize()
+    still.still_timing_enable(False)
+    brk = still.still_timing_read()
+    kernel_ms = {k_: v_[0] / n_brk for k_, v_ in brk.items() if v_[1]} if n_brk > 0 else {}
     gpu_id = None
     try:
         gpu_id = f"GPU-{torch.cuda.get_device_properties(local).uuid}"
@@ -555,6 +591,7 @@ def run_decode(args):
                 "h2d_bytes_per_step": (qb.numel() + kb.numel() + vb.numel()) * qb.element_size(),
                 "d2h_bytes_per_step": o_host.numel() * o_host.element_size()},
         "gpu_launches": launches, "clocks": clocks,
+        "kernel_ms_per_step": kernel_ms, "kernel_ms_steps": n_brk,
         "step_ms": {"median": float(np.median(times)), "max": float(max(times)),
                     "chunk_close": [times[j] for j in close_steps],
                     # one chunk's worth of steps: C-1 ordinary steps and the one that closes the chunk

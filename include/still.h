@@ -220,15 +220,16 @@ STILL_API uint64_t still_launch_count(void);
 /*
  * Per-kernel timing for benchmarks (no counterpart in the method; host-side
  * instrumentation).  While enabled, every kernel launched by
- * still_hybrid_prefill is bracketed by a pair of CUDA events recorded on the
- * caller's stream (at most STILL_TIMING_MAX_LAUNCHES launches are kept; later
- * ones are not timed).  still_timing_read synchronises those events and, for
+ * still_hybrid_prefill and still_decode_step is bracketed by a pair of CUDA
+ * events recorded on the caller's stream (created on first use; at most
+ * STILL_TIMING_MAX_LAUNCHES launches are kept; later ones are not timed).  still_timing_read synchronises those events and, for
  * each kernel class c < n, writes the summed milliseconds to ms[c] and the
  * number of timed launches to launches[c], then forgets them.  Classes:
  * 0 saliency (group mean on the tensor-core path), 1 top-k + gather, 2 NP-Map,
  * 3 linear state, 4 softmax/linear merge (tensor-core path: window part with
  * the fused saliency), 5 decode-state export, 6 tensor-core merge of the kept
- * prefix and the linear branch.  Single-threaded use only.
+ * prefix and the linear branch, 7 decode append, 8 decode attention, 9 decode
+ * combine, 10 decode chunk close.  Single-threaded use only.
  */
 /*
  * Diagnostics (no counterpart in the method): when `words` is non-NULL, the
@@ -236,15 +237,18 @@ STILL_API uint64_t still_launch_count(void);
  * MMA issuer and each softmax warp: last step reached; 0xBAD.. on a bounded
  * wait that gave up; SM clock at CTA start, first score tile, epilogue and
  * exit in words 10..13; 0xD0E / 0xF1F at exit).  The window-phase launch
- * (G' = B*Hkv*G/2*ceil(N/128) CTAs) writes words [0, 16 G' + 2049); the
- * kept-prefix launch writes from word 16 G' + 2080 on.  Pass host-mapped
+ * (G1 = B*Hkv*(G/2)*ceil(N/128) CTAs) uses words [0, 16 G1 + 2049); the
+ * kept-prefix launch (G2 = B*Hkv*(G/2)*(ceil(N/128) - (m+1)C/128) CTAs) uses
+ * 16 G2 + 2049 words from word 16 G1 + 2080 on, so the buffer must hold
+ * 16 (G1 + G2) + 4129 words.  Word 2048 past each launch's per-CTA words
+ * selects the CTA whose per-tile clocks are recorded.  Pass host-mapped
  * (pinned) memory to read it while a kernel runs.  NULL (the default)
  * disables it.
  */
 STILL_API void still_debug_set_trace(unsigned *words);
 
 #define STILL_TIMING_MAX_LAUNCHES 4096
-#define STILL_TIMING_CLASSES 7
+#define STILL_TIMING_CLASSES 11
 STILL_API still_status still_timing_enable(int on);
 STILL_API still_status still_timing_read(double *ms, int *launches, int n);
 

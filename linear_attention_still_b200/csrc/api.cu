@@ -136,27 +136,35 @@ cudaEvent_t g_ev_pool[2 * STILL_TIMING_MAX_LAUNCHES];
 int g_ev_made = 0;
 
 struct TimingScope {
-    int slot = -1;
+    int slot;
     cudaStream_t st;
-    TimingScope(int cls, cudaStream_t s) : st(s) {
-        if (!g_timing || g_ntimed >= STILL_TIMING_MAX_LAUNCHES) return;
-        const int i = g_ntimed;
-        for (int e = 0; e < 2; ++e)
-            if (g_ev_made <= 2 * i + e) {
-                if (cudaEventCreate(&g_ev_pool[2 * i + e]) != cudaSuccess) return;
-                ++g_ev_made;
-            }
-        g_timed[i] = {g_ev_pool[2 * i], g_ev_pool[2 * i + 1], cls};
-        if (cudaEventRecord(g_timed[i].a, st) != cudaSuccess) return;
-        slot = i;
-        ++g_ntimed;
-    }
-    ~TimingScope() {
-        if (slot >= 0) cudaEventRecord(g_timed[slot].b, st);
-    }
+    TimingScope(int cls, cudaStream_t s) : slot(still::timing_begin(cls, s)), st(s) {}
+    ~TimingScope() { still::timing_end(slot, st); }
 };
 
 }  // namespace
+
+namespace still {
+
+int timing_begin(int cls, cudaStream_t st) {
+    if (!g_timing || g_ntimed >= STILL_TIMING_MAX_LAUNCHES) return -1;
+    const int i = g_ntimed;
+    for (int e = 0; e < 2; ++e)
+        if (g_ev_made <= 2 * i + e) {
+            if (cudaEventCreate(&g_ev_pool[2 * i + e]) != cudaSuccess) return -1;
+            ++g_ev_made;
+        }
+    g_timed[i] = {g_ev_pool[2 * i], g_ev_pool[2 * i + 1], cls};
+    if (cudaEventRecord(g_timed[i].a, st) != cudaSuccess) return -1;
+    ++g_ntimed;
+    return i;
+}
+
+void timing_end(int slot, cudaStream_t st) {
+    if (slot >= 0) cudaEventRecord(g_timed[slot].b, st);
+}
+
+}  // namespace still
 
 extern "C" {
 

@@ -406,29 +406,39 @@ __global__ void __launch_bounds__(256) decode_attn_packed_kernel(Dims s, DecodeL
 }
 
 // bf16 decode attention on the warp-level tensor-core instruction (mma.sync m16n8k16, fp32
-// accumulate).  The step is bound by HBM (every kept and window row is read once); the SIMT form
-// of the same contraction spends more issue slots on shuffles and conversions than the memory
-// time allows, while one MMA does a 16-key x 16-dim slice for all heads of the group.  The G <= 8
-// query heads of the group are rows 0..G-1 of the 16-row A operand (the rest are zero).
-//   S^T tile: A = Q (heads x 16 dims), B = K^T (16 dims x 8 keys): a lane loads one 16-byte slice of
-//   a K row and uses it as the B fragments of two k-steps; Q's fragments follow the same
-//   permutation of the head dimension (a dot product does not depend on the order of its terms).
-//   O += P V: A = P (heads x 16 keys, straight from the score fragments), B = V (16 keys x 8 dims):
-//   a lane loads a contiguous DH/8-dim slice of four V rows and pairs rows with a byte permute;
-//   output column n of n-tile j is head dimension n*DH/8 + j.
-// Scores in log2 units; partials written in natural units (same format as decode_attn_kernel).
-__device__ __forceinline__ void mma16816(float (&c)[4], unsigned a0, unsigned a2, unsigned b0, unsigned b1) {
+// accumulate).  The step is bound by HBM (every kept and window row is read once); the SIMT form of
+// the same contraction spends more issue slots on shuffles and conversions than the memory time
+// allows, while one MMA covers a 16 x 8 x 16 block.  Per warp step of 16 keys:
+//   S = Q K^T   (M = 16 rows: the G <= 8 query heads of the group, the rest zero; N = 8 keys; K = 16
+//               dims): a lane loads one 16-byte slice of a K row and uses it as the B fragments of two
+//               k-steps; Q's fragments follow the same permutation of the head dimension (a dot
+//               product does not depend on the order of its terms);
+//   O^T += V^T P^T  (M = 16 head dims, N = 8 heads, K = 16 keys): P^T is the score fragment as it
+//               stands (bf16), V^T pairs two V rows per register with a byte permute; a lane loads a
+//               contiguous DH/8-dim slice of four V rows, and row r of m-tile mt is head dim
+//               (DH/8) * (r % 8) + (DH/16) * (r / 8) + mt.
+// The next step's K/V rows are loaded before the current step is computed (two register buffers), so
+// every warp keeps two steps of loads in flight.  Scores in log2 units; partials are written in
+// natural units (same format as decode_attn_kernel).
+__device__ __forceinline__ void mma16816(float (&c)[4], unsigned a0, unsigned a1, unsigned a2, unsigned a3,
+                                         unsigned b0, unsigned b1) {
     asm volatile(
         "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
         "{%0,%1,%2,%3};\n"
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+template <int DH>
+struct DecodeKV {
+    uint4 k[2][DH / 32];  // K rows gq and gq+8: dims 32i + 8c .. +8
+    uint4 v[4][DH / 64];  // V rows 2c, 2c+1, 2c+8, 2c+9: dims (DH/8) gq .. +DH/8
+};
+
 template <int DH, int G>
-__global__ void __launch_bounds__(128) decode_attn_mma_kernel(Dims s, DecodeLayout L, unsigned char *state,
-                                                              StepGeom gm, const __nv_bfloat16 *__restrict__ q_t) {
-    constexpr int NW = 4, NQ = DH / 32, NT = DH / 8, VW = DH / 64;
+__global__ void __launch_bounds__(128, 2) decode_attn_mma_kernel(Dims s, DecodeLayout L, unsigned char *state,
+                                                                 StepGeom gm, const __nv_bfloat16 *__restrict__ q_t) {
+    constexpr int NW = 4, NQ = DH / 32, NM = DH / 16, VW = DH / 64;
     constexpr float kL2e = 1.4426950408889634f, kLn2f = 0.6931471805599453f;
     static_assert(G >= 1 && G <= 8 && (DH == 64 || DH == 128), "decode mma shape");
     __shared__ float sm_ml[NW][G][5];  // m, l, bm, bl, sdiag (log2 units)
@@ -451,14 +461,15 @@ __global__ void __launch_bounds__(128) decode_attn_mma_kernel(Dims s, DecodeLayo
         qa0[2 * i + 1] = u.z;
         qa2[2 * i + 1] = u.w;
     }
-    float o[NT][4];
+    float ot[NM][4];
 #pragma unroll
-    for (int j = 0; j < NT; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+    for (int mt = 0; mt < NM; ++mt) ot[mt][0] = ot[mt][1] = ot[mt][2] = ot[mt][3] = 0.f;
     float m = -INFINITY, l = 0.f, bm = -INFINITY, bl = 0.f, sd = -INFINITY;
 
-    for (int base = l0 + warp * 16; base < l1; base += NW * 16) {
-        // lane kk < 16 locates key base+kk (byte offset of its K row in the state, bit 0 set for a
-        // window-ring row); keys past the end re-read the last key of the range with probability zero
+    // lane kk < 16 locates key base+kk (byte offset of its K row in the state, bit 0 set for a
+    // window-ring row) and the warp shares it; keys past the end re-read the last key of the range
+    // with probability zero
+    auto load = [&](DecodeKV<DH> &t, int base) {
         unsigned long long my_off = 0;
         if (lane < 16) {
             const int li = min(base + lane, l1 - 1);
@@ -469,13 +480,12 @@ __global__ void __launch_bounds__(128) decode_attn_mma_kernel(Dims s, DecodeLayo
                 my_off = (L.ring_k + ((size_t)bg * L.ring_rows + ring_row(s, j)) * kRow) | 1ull;
             }
         }
-        uint4 kr[2][NQ], vr[4][VW];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const unsigned long long off = __shfl_sync(0xffffffffu, my_off, gq + 8 * h) & ~1ull;
             const uint4 *row = reinterpret_cast<const uint4 *>(state + off);
 #pragma unroll
-            for (int i = 0; i < NQ; ++i) kr[h][i] = __ldg(row + 4 * i + c);
+            for (int i = 0; i < NQ; ++i) t.k[h][i] = __ldg(row + 4 * i + c);
         }
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
@@ -483,17 +493,19 @@ __global__ void __launch_bounds__(128) decode_attn_mma_kernel(Dims s, DecodeLayo
             const size_t vo = (off & ~1ull) + ((off & 1ull) ? dv_ring : dv_kept);
             const uint4 *row = reinterpret_cast<const uint4 *>(state + vo);
 #pragma unroll
-            for (int i = 0; i < VW; ++i) vr[r][i] = __ldg(row + gq * VW + i);
+            for (int i = 0; i < VW; ++i) t.v[r][i] = __ldg(row + gq * VW + i);
         }
-        // S^T for keys base+[0,8) and base+[8,16)
+    };
+    auto process = [&](const DecodeKV<DH> &t, int base) {
+        // S for keys base+[0,8) and base+[8,16)
         float st[2][4];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             st[h][0] = st[h][1] = st[h][2] = st[h][3] = 0.f;
 #pragma unroll
             for (int i = 0; i < NQ; ++i) {
-                mma16816(st[h], qa0[2 * i], qa2[2 * i], kr[h][i].x, kr[h][i].y);
-                mma16816(st[h], qa0[2 * i + 1], qa2[2 * i + 1], kr[h][i].z, kr[h][i].w);
+                mma16816(st[h], qa0[2 * i], 0u, qa2[2 * i], 0u, t.k[h][i].x, t.k[h][i].y);
+                mma16816(st[h], qa0[2 * i + 1], 0u, qa2[2 * i + 1], 0u, t.k[h][i].z, t.k[h][i].w);
             }
         }
         // this lane's scores: head gq, keys 2c, 2c+1, 8+2c, 9+2c
@@ -522,7 +534,7 @@ __global__ void __launch_bounds__(128) decode_attn_mma_kernel(Dims s, DecodeLayo
         }
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-        const float mn = fmaxf(m, mx);  // finite: key base+0 is always in range
+        const float mn = fmaxf(m, mx);      // finite: key base+0 is always in range
         const float so = tc::ex2(m - mn);  // m = -inf gives 0
         float p[4], ps = 0.f;
 #pragma unroll
@@ -534,22 +546,45 @@ __global__ void __launch_bounds__(128) decode_attn_mma_kernel(Dims s, DecodeLayo
         ps += __shfl_xor_sync(0xffffffffu, ps, 2);
         l = l * so + ps;
         m = mn;
+        // O^T columns are heads 2c and 2c+1: their factors live in the lanes of rows 2c, 2c+1
+        const float so0 = __shfl_sync(0xffffffffu, so, 8 * c), so1 = __shfl_sync(0xffffffffu, so, 8 * c + 4);
 #pragma unroll
-        for (int j = 0; j < NT; ++j) {
-            o[j][0] *= so;
-            o[j][1] *= so;
+        for (int mt = 0; mt < NM; ++mt) {
+            ot[mt][0] *= so0;
+            ot[mt][1] *= so1;
+            ot[mt][2] *= so0;
+            ot[mt][3] *= so1;
         }
-        const unsigned pa0 = tc::pack_bf16x2(p[0], p[1]), pa2 = tc::pack_bf16x2(p[2], p[3]);
+        const unsigned pb0 = tc::pack_bf16x2(p[0], p[1]), pb1 = tc::pack_bf16x2(p[2], p[3]);
+        const unsigned *w0 = reinterpret_cast<const unsigned *>(&t.v[0][0]);
+        const unsigned *w1 = reinterpret_cast<const unsigned *>(&t.v[1][0]);
+        const unsigned *w2 = reinterpret_cast<const unsigned *>(&t.v[2][0]);
+        const unsigned *w3 = reinterpret_cast<const unsigned *>(&t.v[3][0]);
 #pragma unroll
-        for (int j = 0; j < NT; ++j) {
-            const unsigned *w0 = reinterpret_cast<const unsigned *>(&vr[0][0]);
-            const unsigned *w1 = reinterpret_cast<const unsigned *>(&vr[1][0]);
-            const unsigned *w2 = reinterpret_cast<const unsigned *>(&vr[2][0]);
-            const unsigned *w3 = reinterpret_cast<const unsigned *>(&vr[3][0]);
-            const unsigned sel = (j & 1) ? 0x7632u : 0x5410u;
-            const unsigned b0 = __byte_perm(w0[j >> 1], w1[j >> 1], sel);
-            const unsigned b1 = __byte_perm(w2[j >> 1], w3[j >> 1], sel);
-            mma16816(o[j], pa0, pa2, b0, b1);
+        for (int mt = 0; mt < NM; ++mt) {
+            const unsigned sel = (mt & 1) ? 0x7632u : 0x5410u;
+            const int lo_w = mt >> 1, hi_w = (NM + mt) >> 1;
+            const unsigned a0 = __byte_perm(w0[lo_w], w1[lo_w], sel);
+            const unsigned a1 = __byte_perm(w0[hi_w], w1[hi_w], sel);
+            const unsigned a2 = __byte_perm(w2[lo_w], w3[lo_w], sel);
+            const unsigned a3 = __byte_perm(w2[hi_w], w3[hi_w], sel);
+            mma16816(ot[mt], a0, a1, a2, a3, pb0, pb1);
+        }
+    };
+
+    {
+        DecodeKV<DH> ta, tb;
+        constexpr int kStep = NW * 16;
+        int base = l0 + warp * 16;
+        if (base < l1) load(ta, base);
+        while (base < l1) {
+            if (base + kStep < l1) load(tb, base + kStep);
+            process(ta, base);
+            base += kStep;
+            if (base >= l1) break;
+            if (base + kStep < l1) load(ta, base + kStep);
+            process(tb, base);
+            base += kStep;
         }
     }
     // band statistics of head gq: combine the four lanes of the row
@@ -570,10 +605,17 @@ __global__ void __launch_bounds__(128) decode_attn_mma_kernel(Dims s, DecodeLayo
             sm_ml[warp][gq][3] = bl;
             sm_ml[warp][gq][4] = sd;
         }
+    }
+    // O^T: columns heads 2c, 2c+1; rows gq (dims (DH/8) gq + mt) and gq+8 (dims (DH/8) gq + DH/16 + mt)
 #pragma unroll
-        for (int j = 0; j < NT; ++j) {
-            sm_acc[warp][gq][(2 * c) * NT + j] = o[j][0];
-            sm_acc[warp][gq][(2 * c + 1) * NT + j] = o[j][1];
+    for (int hc = 0; hc < 2; ++hc) {
+        const int hh = 2 * c + hc;
+        if (hh < G) {
+#pragma unroll
+            for (int mt = 0; mt < NM; ++mt) {
+                sm_acc[warp][hh][2 * NM * gq + mt] = ot[mt][hc];
+                sm_acc[warp][hh][2 * NM * gq + NM + mt] = ot[mt][2 + hc];
+            }
         }
     }
     __syncthreads();
@@ -1033,9 +1075,12 @@ static cudaError_t decode_step_t(const Dims &s, unsigned char *state, const Deco
     gm.nsplit = gm.n == 0 ? 0 : min(kDecodeMaxSplits, (gm.n + 511) / 512);
     gm.per = gm.nsplit ? (gm.n + gm.nsplit - 1) / gm.nsplit : 0;
     const int BK = s.B * s.Hkv;
+    int ts = timing_begin(kTimeDecodeAppend, st);
     decode_append_kernel<T><<<BK, 128, 0, st>>>(s, L, state, pos, (const T *)k_t, (const T *)v_t, err);
+    timing_end(ts, st);
     ++*launches;
     if (gm.nsplit) {
+        ts = timing_begin(kTimeDecodeAttn, st);
         const dim3 grid(BK, gm.nsplit);
         const int G = s.G();
 #define STILL_DECODE_PACKED(DPL, GG) \
@@ -1067,8 +1112,10 @@ static cudaError_t decode_step_t(const Dims &s, unsigned char *state, const Deco
         else decode_attn_kernel<T><<<grid, 128, 0, st>>>(s, L, state, gm, (const T *)q_t);
 #undef STILL_DECODE_PACKED
 #undef STILL_DECODE_MMA
+        timing_end(ts, st);
         ++*launches;
     }
+    ts = timing_begin(kTimeDecodeCombine, st);
     if (s.w > 0 && s.G() <= 8) {
         const size_t smem = combine_wide_smem(s);
         if (smem > 48 * 1024) {
@@ -1082,6 +1129,7 @@ static cudaError_t decode_step_t(const Dims &s, unsigned char *state, const Deco
         decode_combine_kernel<T><<<BK, 128, 0, st>>>(s, L, state, gm, (const T *)q_t, (const T *)Wq, (const T *)Wk,
                                                      (T *)o_t);
     }
+    timing_end(ts, st);
     ++*launches;
     if (pos % s.C == s.C - 1 && gm.t - m >= 0) {
         const int P = pow2_ceil(s.C), Pk = pow2_ceil(s.k > 0 ? s.k : 1);
@@ -1090,8 +1138,10 @@ static cudaError_t decode_step_t(const Dims &s, unsigned char *state, const Deco
             cudaFuncSetAttribute(decode_close_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         const int passes = (s.D * s.d + kFoldThreads * kFoldEnt - 1) / (kFoldThreads * kFoldEnt);
+        ts = timing_begin(kTimeDecodeClose, st);
         decode_close_kernel<T><<<dim3(BK, passes), kFoldThreads, smem, st>>>(s, L, state, gm.t - m, (const T *)Wk, P,
                                                                              Pk);
+        timing_end(ts, st);
         ++*launches;
     }
     return cudaGetLastError();

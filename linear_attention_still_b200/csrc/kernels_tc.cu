@@ -429,6 +429,7 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
             // ---- prologue: phi(q) from Y = Q Wq^T
             ok = warp_all(mbar_wait(BAR(B_QFULL), 0, abort_flag) && mbar_wait(BAR(B_Y + x), 0, abort_flag));
             if (lane == 0) trace_word(p.trace, 2 + warp, ok ? 1 : 0xBAD1);
+            if (threadIdx.x % 128 == 0) trace_time(p.trace, x, 63, 0);  // Y ready
             float y[DF];
             if (ok) {
                 tc_fence_after();
@@ -488,8 +489,10 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
             tc_fence_before();
             mbar_arrive(BAR(B_PHI + x));
             if (lane == 0) trace_word(p.trace, 2 + warp, 2);
+            if (threadIdx.x % 128 == 0) trace_time(p.trace, x, 63, 1);  // phi(q) written
             // ---- fold the window part (o_A, lse_A) into O = phi(q) S_t^T under one normaliser
             ok = warp_all(ok && mbar_wait(BAR(B_PRO), 0, abort_flag));
+            if (threadIdx.x % 128 == 0) trace_time(p.trace, x, 63, 2);  // phi(q) S_t^T done
             if (ok) {
                 tc_fence_after();
                 const bool valid = i < p.N;
@@ -518,6 +521,7 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
                 }
                 tmem_wait_st();
                 m_run = M;
+                if (threadIdx.x % 128 == 0) trace_time(p.trace, x, 63, 3);  // window part folded
                 l_run = wa + bden * wb;
             }
         }

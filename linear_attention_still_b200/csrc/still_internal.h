@@ -60,6 +60,11 @@ cudaError_t launch_merge_generic(const Dims &s, const void *q, const void *k, co
                                  const float *phik, void *o, cudaStream_t st);
 
 // ---- decode ----
+// Per-kernel event timing (still_timing_enable): returns a slot for timing_end, or -1 when off.
+int timing_begin(int cls, cudaStream_t st);
+void timing_end(int slot, cudaStream_t st);
+enum TimingClass { kTimeDecodeAppend = 7, kTimeDecodeAttn = 8, kTimeDecodeCombine = 9, kTimeDecodeClose = 10 };
+
 cudaError_t launch_decode_step(const Dims &s, unsigned char *state, const DecodeLayout &L, int pos, const void *Wq,
                                const void *Wk, const void *q_t, const void *k_t, const void *v_t, void *o_t,
                                unsigned *err, cudaStream_t st, int *launches);

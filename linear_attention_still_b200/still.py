@@ -183,7 +183,8 @@ def still_debug_set_trace(words=None):
     _lib.still_debug_set_trace(_ptr(words))
 
 
-TIMING_CLASSES = ("saliency", "topk_gather", "npmap", "linear_state", "merge", "state_export", "merge_prefix")
+TIMING_CLASSES = ("saliency", "topk_gather", "npmap", "linear_state", "merge", "state_export", "merge_prefix",
+                  "decode_append", "decode_attn", "decode_combine", "decode_close")
 
 
 def still_timing_enable(on: bool = True):

@@ -75,6 +75,9 @@ WORKLOADS = {
     "llama31_8b_layer_n64k": Shape(B=1, H=32, Hkv=8, N=65536, d=128, D=128, w=1024, C=1024, k=128),
     "llama31_8b_decode_b16_ctx64k": Shape(B=16, H=32, Hkv=8, N=65536, d=128, D=128, w=1024, C=1024,
                                           k=128, decode_steps=1024),
+    # the same decode at batch 4: small enough (about 5 GB on the device) for multi-pass profiling
+    "llama31_8b_decode_b4_ctx64k": Shape(B=4, H=32, Hkv=8, N=65536, d=128, D=128, w=1024, C=1024,
+                                         k=128, decode_steps=1024),
 }
 
 
