@@ -772,15 +772,58 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(Dims s, DecodeLayou
 }
 
 // Combine for a window (w > 0) and G <= 8: one CTA of 256 threads per (b, g) does every head of the
-// group at once, with the work spread over all threads: split factors (a warp per head), the
-// softmax part (thread per (head, element)), Y = q Wq (thread per (head, feature), the d-long sums
-// unrolled so the Wq loads overlap), NP-Map per head, phi(q)^T S with S read once for the group
-// (thread per (element, slice of the features)), and the merge under the shared normaliser.
+// group at once.  The kernel is latency bound (a few hundred KB per CTA, mostly from L2), so every
+// phase gives each thread many independent 8- or 16-byte loads:
+//   split weights per head (a warp per head);
+//   softmax numerator: thread per (head, element pair), the splits' partials as float2;
+//   Y = q Wq: thread per (head, 16-byte group of features, slice of the head dim), reduced in smem;
+//   NP-Map per head ([p1] "Norm-Preserved Feature Map") and phi(q) . z (a warp per head);
+//   phi(q)^T S: thread per (4 head-dim elements, slice of the features), S read once for the group
+//   as float4, reduced in smem;
+//   merge under the shared normaliser, group score of the new token into the ring.
 constexpr int kCombineThreads = 256;
 
+template <typename T>
+struct CombineGeom {
+    int G, d, D;
+    int nfv, xq, xlen;  // Y: feature vectors per head (16 bytes of Wq each), head-dim slices, slice length
+    int ar, alen;       // phi^T S: feature slices, slice length
+    __host__ __device__ explicit CombineGeom(const Dims &s) : G(s.G()), d(s.d), D(s.D) {
+        constexpr int V = 16 / (int)sizeof(T);
+        nfv = D / V;
+        const int combos = G * nfv;
+        xq = combos >= kCombineThreads ? 1 : kCombineThreads / combos;
+        xlen = (d + xq - 1) / xq;
+        ar = kCombineThreads / (d / 4) > 0 ? kCombineThreads / (d / 4) : 1;
+        alen = (D + ar - 1) / ar;
+    }
+    // floats of shared memory: weights, stats, numerator, q, phi, then one scratch area shared by the
+    // Y partials [xq][G][D] and the phi^T S partials [ar][G][d]
+    __host__ __device__ int smem_floats() const {
+        const int scratch = max(xq * G * D, ar * G * d);
+        return G * 64 + G * 8 + 2 * G * d + G * D + scratch;
+    }
+};
+
 size_t combine_wide_smem(const Dims &s) {
-    const int G = s.G(), P = kCombineThreads / s.d;
-    return (size_t)(G * 64 + G * 8 + 2 * G * s.d + G * s.D + P * G * s.d) * sizeof(float);
+    if (s.bf16) return (size_t)CombineGeom<__nv_bfloat16>(s).smem_floats() * sizeof(float);
+    return (size_t)CombineGeom<float>(s).smem_floats() * sizeof(float);
+}
+
+__device__ __forceinline__ void unpack16(const uint4 &u, const __nv_bfloat16 *, float (&f)[8]) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float2 t = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[e]));
+        f[2 * e] = t.x;
+        f[2 * e + 1] = t.y;
+    }
+}
+__device__ __forceinline__ void unpack16(const uint4 &u, const float *, float (&f)[4]) {
+    f[0] = __uint_as_float(u.x);
+    f[1] = __uint_as_float(u.y);
+    f[2] = __uint_as_float(u.z);
+    f[3] = __uint_as_float(u.w);
 }
 
 template <typename T>
@@ -789,14 +832,16 @@ __global__ void __launch_bounds__(kCombineThreads) decode_combine_wide_kernel(Di
                                                                               const T *__restrict__ q_t,
                                                                               const T *__restrict__ Wq,
                                                                               T *__restrict__ o_t) {
+    constexpr int V = 16 / (int)sizeof(T);
     extern __shared__ float cs[];
-    const int G = s.G(), d = s.d, D = s.D, ns = gm.nsplit, P = kCombineThreads / d;
+    const CombineGeom<T> cg(s);
+    const int G = cg.G, d = cg.d, D = cg.D, ns = gm.nsplit;
     float *sf = cs;           // [G][64] weight of each split
-    float *st = sf + G * 64;  // [G][8]: M, Ls, BM, BL, SD, lden, sigma
+    float *st = sf + G * 64;  // [G][8]: M, Ls, -, -, -, lden, sigma
     float *os = st + G * 8;   // [G][d] softmax numerator
     float *qs = os + G * d;   // [G][d]
     float *ph = qs + G * d;   // [G][D] Y, then phi(q)
-    float *lp = ph + G * D;   // [P][G][d] partial phi(q)^T S
+    float *scr = ph + G * D;  // Y partials [xq][G][D], then phi^T S partials [ar][G][d]
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int bg = blockIdx.x, b = bg / s.Hkv, g = bg % s.Hkv;
     const float *part = reinterpret_cast<const float *>(state + L.part);
@@ -836,26 +881,73 @@ __global__ void __launch_bounds__(kCombineThreads) decode_combine_wide_kernel(Di
     }
     for (int t = tid; t < G * d; t += kCombineThreads) qs[t] = to_f(q_t[((size_t)b * s.H + g * G) * d + t]);
     __syncthreads();
-    for (int t = tid; t < G * d; t += kCombineThreads) {
-        const int hh = t / d, x = t % d;
-        const float *pp = part + (pb0 + (size_t)hh * kDecodeMaxSplits) * (d + 2) + 2 + x;
-        float a = 0.f;
-        for (int sp = 0; sp < ns; ++sp) a = fmaf(pp[(size_t)sp * (d + 2)], sf[hh * 64 + sp], a);
-        os[t] = a;
-    }
-    for (int t = tid; t < G * D; t += kCombineThreads) {
-        const int hh = t / D, a = t % D;
-        const T *w = Wq + (size_t)(g * G + hh) * d * D + a;
-        const float *qh = qs + hh * d;
-        float y[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int x = 0; x < d; x += 8) {  // d is a multiple of 8
+    // softmax numerator: (head, element pair); partial rows are (d + 2) floats, so 8-byte aligned
+    for (int t = tid; t < G * d / 2; t += kCombineThreads) {
+        const int hh = t / (d / 2), x2 = t % (d / 2);
+        const float2 *pp = reinterpret_cast<const float2 *>(part + (pb0 + (size_t)hh * kDecodeMaxSplits) * (d + 2) + 2) + x2;
+        const size_t stride2 = (size_t)(d + 2) / 2;
+        float2 a = make_float2(0.f, 0.f);
+        int sp = 0;
+        for (; sp + 4 <= ns; sp += 4) {
+            float2 v[4];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) y[e] = fmaf(qh[x + e], to_f(w[(size_t)(x + e) * D]), y[e]);
+            for (int u = 0; u < 4; ++u) v[u] = pp[(size_t)(sp + u) * stride2];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float f = sf[hh * 64 + sp + u];
+                a.x = fmaf(v[u].x, f, a.x);
+                a.y = fmaf(v[u].y, f, a.y);
+            }
         }
-        ph[t] = ((y[0] + y[1]) + (y[2] + y[3])) + ((y[4] + y[5]) + (y[6] + y[7]));
+        for (; sp < ns; ++sp) {
+            const float2 v = pp[(size_t)sp * stride2];
+            const float f = sf[hh * 64 + sp];
+            a.x = fmaf(v.x, f, a.x);
+            a.y = fmaf(v.y, f, a.y);
+        }
+        os[hh * d + 2 * x2] = a.x;
+        os[hh * d + 2 * x2 + 1] = a.y;
+    }
+    // Y = q Wq: (head, feature vector, head-dim slice)
+    for (int t = tid; t < G * cg.nfv * cg.xq; t += kCombineThreads) {
+        const int xs = t % cg.xq, cv = t / cg.xq, hh = cv / cg.nfv, fv = cv % cg.nfv;
+        const int x0 = xs * cg.xlen, x1 = min(d, x0 + cg.xlen);
+        const uint4 *w = reinterpret_cast<const uint4 *>(Wq + (size_t)(g * G + hh) * d * D) + fv;
+        const int wstride = D / V;
+        float y[V];
+#pragma unroll
+        for (int e = 0; e < V; ++e) y[e] = 0.f;
+        int x = x0;
+        for (; x + 8 <= x1; x += 8) {
+            uint4 u[8];
+#pragma unroll
+            for (int r = 0; r < 8; ++r) u[r] = __ldg(w + (size_t)(x + r) * wstride);
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                float f[V];
+                unpack16(u[r], Wq, f);
+                const float qv = qs[hh * d + x + r];
+#pragma unroll
+                for (int e = 0; e < V; ++e) y[e] = fmaf(qv, f[e], y[e]);
+            }
+        }
+        for (; x < x1; ++x) {
+            float f[V];
+            unpack16(__ldg(w + (size_t)x * wstride), Wq, f);
+            const float qv = qs[hh * d + x];
+#pragma unroll
+            for (int e = 0; e < V; ++e) y[e] = fmaf(qv, f[e], y[e]);
+        }
+#pragma unroll
+        for (int e = 0; e < V; ++e) scr[(xs * G + hh) * D + fv * V + e] = y[e];
     }
     __syncthreads();
-    // NP-Map of each head's query ([p1] "Norm-Preserved Feature Map") and phi(q) . z
+    for (int t = tid; t < G * D; t += kCombineThreads) {
+        float y = 0.f;
+        for (int xs = 0; xs < cg.xq; ++xs) y += scr[xs * G * D + t];
+        ph[t] = y;
+    }
+    __syncthreads();
     for (int hh = warp; hh < G; hh += kCombineThreads / 32) {
         float *yh = ph + hh * D;
         float mx = -INFINITY;
@@ -882,25 +974,52 @@ __global__ void __launch_bounds__(kCombineThreads) decode_combine_wide_kernel(Di
         if (lane == 0) st[hh * 8 + 5] = ld;
     }
     __syncthreads();
-    if (tid < P * d) {
-        const int x = tid % d, pi = tid / d;
-        const int a0 = pi * D / P, a1 = (pi + 1) * D / P;
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int a = a0; a < a1; ++a) {
-            const float sv = S[(size_t)a * d + x];
+    // phi(q)^T S: (4 head-dim elements, feature slice); S rows are d floats, 16-byte aligned
+    if (tid < (d / 4) * cg.ar) {
+        const int x4 = tid % (d / 4), as = tid / (d / 4);
+        const int a0 = as * cg.alen, a1 = min(D, a0 + cg.alen);
+        float4 acc[8];
+#pragma unroll
+        for (int hh = 0; hh < 8; ++hh) acc[hh] = make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 *S4 = reinterpret_cast<const float4 *>(S) + x4;
+        int a = a0;
+        for (; a + 4 <= a1; a += 4) {
+            float4 sv[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) sv[u] = S4[(size_t)(a + u) * (d / 4)];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int hh = 0; hh < 8; ++hh)
+                    if (hh < G) {
+                        const float pv = ph[hh * D + a + u];
+                        acc[hh].x = fmaf(pv, sv[u].x, acc[hh].x);
+                        acc[hh].y = fmaf(pv, sv[u].y, acc[hh].y);
+                        acc[hh].z = fmaf(pv, sv[u].z, acc[hh].z);
+                        acc[hh].w = fmaf(pv, sv[u].w, acc[hh].w);
+                    }
+        }
+        for (; a < a1; ++a) {
+            const float4 sv = S4[(size_t)a * (d / 4)];
 #pragma unroll
             for (int hh = 0; hh < 8; ++hh)
-                if (hh < G) acc[hh] = fmaf(ph[hh * D + a], sv, acc[hh]);
+                if (hh < G) {
+                    const float pv = ph[hh * D + a];
+                    acc[hh].x = fmaf(pv, sv.x, acc[hh].x);
+                    acc[hh].y = fmaf(pv, sv.y, acc[hh].y);
+                    acc[hh].z = fmaf(pv, sv.z, acc[hh].z);
+                    acc[hh].w = fmaf(pv, sv.w, acc[hh].w);
+                }
         }
 #pragma unroll
         for (int hh = 0; hh < 8; ++hh)
-            if (hh < G) lp[(pi * G + hh) * d + x] = acc[hh];
+            if (hh < G) reinterpret_cast<float4 *>(scr + (as * G + hh) * d)[x4] = acc[hh];
     }
     __syncthreads();
     for (int t = tid; t < G * d; t += kCombineThreads) {
         const int hh = t / d, x = t % d;
         float lin = 0.f;
-        for (int pi = 0; pi < P; ++pi) lin += lp[(pi * G + hh) * d + x];
+        for (int as = 0; as < cg.ar; ++as) lin += scr[(as * G + hh) * d + x];
         const float M = st[hh * 8 + 0], Ls = st[hh * 8 + 1], ld = st[hh * 8 + 5];
         const float Ms = ld > 0.f ? fmaxf(M, logf(ld)) : M;
         const float a_soft = (M == -INFINITY) ? 0.f : expf(M - Ms);
@@ -1118,7 +1237,7 @@ static cudaError_t decode_step_t(const Dims &s, unsigned char *state, const Deco
     ts = timing_begin(kTimeDecodeCombine, st);
     if (s.w > 0 && s.G() <= 8) {
         const size_t smem = combine_wide_smem(s);
-        if (smem > 48 * 1024) {
+        if (smem > 48 * 1024) {  // at most ~66 KB (G = 8, d = D = 256)
             cudaError_t e = cudaFuncSetAttribute(decode_combine_wide_kernel<T>,
                                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             if (e != cudaSuccess) return e;
