@@ -122,7 +122,7 @@ __device__ __forceinline__ void exp_tile(const float (&sv)[128], float scale_log
             const int c0 = c * 32 + 2 * e;
             const float2 xx = ffma2(make_float2(sv[c0], sv[c0 + 1]), sc2, neg2);
             float2 pp;
-            if (EXPV == 2 && c == 3) {
+            if ((EXPV == 2 && c == 3) || (EXPV == 3 && (c & 1))) {
                 pp = exp2_poly2(xx);  // FMA pipe
             } else {
                 pp.x = ex2(xx.x);      // MUFU
@@ -151,9 +151,13 @@ __device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, int kk, uint32_t 
 }
 
 // EXPV selects the exponential phase: 0 scalar FFMA + MUFU, 1 packed FFMA2/FADD2 + MUFU,
-// 2 packed with the last 32-key chunk of each row on the FMA-pipe exp2.  Measured on B200 (1B 16K /
-// 8B B4 16K layers, merge ms): 0.502/3.276, 0.493/3.146, 0.497/3.209 -> variant 1 is built.
+// 2 packed with the last 32-key chunk of each row on the FMA-pipe exp2, 3 with every other 32-key
+// chunk there.  Measured on B200 with concurrent softmax warpgroups (1B 16K / 8B B4 16K layers, the
+// two merge phases, ms): variant 1 0.612/3.629, 2 0.608/3.646, 3 0.641/3.799 -> variant 1 is built.
 constexpr int kMergeExpVariant = 1;
+// Two heads per CTA: the softmax warpgroups take turns on the exponential phase (true) or run it
+// concurrently (false; measured 2-5 % faster: both warpgroups' exponentials keep the MUFU unit busy).
+constexpr bool kMergeTurns = false;
 // MODE kMergeLocal: keys = the window [max(0,(t-m)C), i]; also the Self-Saliency Score of every row
 //   ([p1] "Self-Saliency Score"): the band keys [i-w+1, i-1] are window keys, so the band's
 //   log-sum-exp is accumulated from the same exponentials (masked adds on the two partial tiles),
@@ -361,6 +365,8 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
                 tc_fence_after();
                 for (int x = 0; x < HP; ++x) issue_s(x, sStage);
             }
+            // In-order issue: per tile, head 0 then head 1 (next scores, then P V).  (An issuer driven by
+            // whichever barrier completes first measured 5-10 % slower on B200.)
             for (int j = 0; ok && j < n_tiles; ++j) {
                 const int s = j % Cfg::NS;
                 const uint64_t dv = sw128_desc(sStage + s * Cfg::STAGE_BYTES + Cfg::TILE_BYTES, Cfg::REG, 1024);
@@ -378,9 +384,7 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
                         }
                     }
                     if (x == 0) ok = mbar_wait(BAR(B_VFULL + s), (j / Cfg::NS) & 1, abort_flag);
-                    if (x == 0) trace_time(p.trace, 2, j, 4);
                     if (ok) ok = mbar_wait(BAR(B_P + x), j & 1, abort_flag);
-                    trace_time(p.trace, 2, j, 2 * x);
                     if (!ok) break;
                     tc_fence_after();
 #pragma unroll
@@ -395,7 +399,6 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
                         tc_fence_after();
                         issue_s(x, sK1);
                     }
-                    trace_time(p.trace, 2, j, 2 * x + 1);
                 }
                 if (ok) mma_commit(BAR(B_KVEMPTY + s));
             }
@@ -426,6 +429,12 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
         float bs = 0.f, sdiag = 0.f;  // LOCAL: band sum (same reference as l) and raw diagonal score
 
         if constexpr (!LOCAL) {
+            // the window part of this row (o_A, written by the window phase) is read in the fold below:
+            // start bringing it into L2 now
+            if (i < p.N) {
+#pragma unroll
+                for (int v = 0; v < DH * 2; v += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(p.o + row * DH + v / 2));
+            }
             // ---- prologue: phi(q) from Y = Q Wq^T
             ok = warp_all(mbar_wait(BAR(B_QFULL), 0, abort_flag) && mbar_wait(BAR(B_Y + x), 0, abort_flag));
             if (lane == 0) trace_word(p.trace, 2 + warp, ok ? 1 : 0xBAD1);
@@ -491,15 +500,21 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
             if (lane == 0) trace_word(p.trace, 2 + warp, 2);
             if (threadIdx.x % 128 == 0) trace_time(p.trace, x, 63, 1);  // phi(q) written
             // ---- fold the window part (o_A, lse_A) into O = phi(q) S_t^T under one normaliser
+            // the window part's row is loaded while phi(q) S_t^T runs
+            const bool valid = i < p.N;
+            const float lse_a = valid ? p.lse[row] : 0.f;
+            uint4 oa[DH / 8];
+            {
+                const uint4 *orow = reinterpret_cast<const uint4 *>(p.o + row * DH);
+#pragma unroll
+                for (int v = 0; v < DH / 8; ++v) oa[v] = valid ? orow[v] : make_uint4(0, 0, 0, 0);
+            }
             ok = warp_all(ok && mbar_wait(BAR(B_PRO), 0, abort_flag));
             if (threadIdx.x % 128 == 0) trace_time(p.trace, x, 63, 2);  // phi(q) S_t^T done
             if (ok) {
                 tc_fence_after();
-                const bool valid = i < p.N;
-                const float lse_a = valid ? p.lse[row] : 0.f;
                 const float M = bden > 0.f ? fmaxf(lse_a, __log2f(bden)) : lse_a;
                 const float wa = ex2(lse_a - M), wb = ex2(-M);
-                const uint4 *orow = reinterpret_cast<const uint4 *>(p.o + row * DH);
 #pragma unroll
                 for (int c = 0; c < DH / 32; ++c) {
                     uint32_t u[32];
@@ -507,7 +522,7 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
                     tmem_wait_ld();
 #pragma unroll
                     for (int v4 = 0; v4 < 4; ++v4) {
-                        const uint4 w = valid ? orow[c * 4 + v4] : make_uint4(0, 0, 0, 0);
+                        const uint4 w = oa[c * 4 + v4];
                         const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
@@ -562,15 +577,16 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
                 for (int c = 0; c < 128; ++c)
                     if (c >= limit) sv[c] = -INFINITY;
             }
-            float mx0 = sv[0], mx1 = sv[1], mx2 = sv[2], mx3 = sv[3];
+            // row max: four chains of 3-input max over 32 columns each (sv[32k .. 32k+31])
+            float mxc[4];
 #pragma unroll
-            for (int c = 4; c < 128; c += 4) {
-                mx0 = fmaxf(mx0, sv[c]);
-                mx1 = fmaxf(mx1, sv[c + 1]);
-                mx2 = fmaxf(mx2, sv[c + 2]);
-                mx3 = fmaxf(mx3, sv[c + 3]);
+            for (int k4 = 0; k4 < 4; ++k4) {
+                float mv = fmax3(sv[32 * k4], sv[32 * k4 + 1], sv[32 * k4 + 2]);
+#pragma unroll
+                for (int c = 32 * k4 + 3; c + 1 < 32 * k4 + 32; c += 2) mv = fmax3(mv, sv[c], sv[c + 1]);
+                mxc[k4] = fmaxf(mv, sv[32 * k4 + 31]);
             }
-            const float mnew = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * p.scale_log2;
+            const float mnew = fmax3(mxc[0], mxc[1], fmaxf(mxc[2], mxc[3])) * p.scale_log2;
             if (threadIdx.x % 128 == 0) trace_time(p.trace, x, j, 1);
             // Lazy rescale: a row moves its reference max only when the max grows by more than 2^8.
             // The O rescale uses warp-collective tcgen05.ld/st, so the warp takes it together when
@@ -608,7 +624,7 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
             }
             // Two heads per CTA: the warpgroups take turns on the exponential units, so one
             // warpgroup's exponentials overlap the other head's MMAs instead of contending with them.
-            if (HP == 2 && (x == 1 || j > 0)) {
+            if (HP == 2 && kMergeTurns && (x == 1 || j > 0)) {
                 ok = warp_all(mbar_wait(BAR(B_TURN + x), (x == 1 ? j : j - 1) & 1, abort_flag));
                 if (!ok) break;
             }
@@ -629,7 +645,7 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
             } else {
                 exp_tile<EXPV, false>(sv, p.scale_log2, m_run, tP, ls0, ls1, bsum, 0, 0);
             }
-            if (HP == 2) mbar_arrive(BAR(B_TURN + (x ^ 1)));
+            if (HP == 2 && kMergeTurns) mbar_arrive(BAR(B_TURN + (x ^ 1)));
             if (threadIdx.x % 128 == 0) trace_time(p.trace, x, j, 3);
             l_run += ls0 + ls1;
             if (btype == 1) bs += ls0 + ls1;
