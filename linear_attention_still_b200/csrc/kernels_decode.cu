@@ -659,6 +659,301 @@ __global__ void __launch_bounds__(128, 2) decode_attn_mma_kernel(Dims s, DecodeL
     }
 }
 
+// The tensor-core decode attention with the K/V rows staged in shared memory by 1-D bulk
+// copies (cp.async.bulk, no multicast): every warp owns a ring of NST stages of 16 keys (K and V
+// tiles, 16 rows each) and keeps NST tiles in flight without holding them in registers; lane 0
+// issues one copy per contiguous run of rows (kept cache rows of the group are contiguous, window
+// rows are contiguous within a chunk's ring slot).  Fragments are read from the stage with 16-byte
+// shared loads in the layout the register version used.
+// 1-D bulk copy from global memory into this CTA's shared memory (no multicast), completing on an
+// mbarrier.  Both addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
+// Orders this thread's earlier generic-proxy shared-memory accesses before later async-proxy ones
+// (a bulk copy into a buffer the thread has just read).
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+template <int DH>
+struct DecodeBulkCfg {
+    static constexpr int NW = 4, NST = 3, ROWS = 16;
+    static constexpr int TILE = ROWS * DH * 2;  // bytes of the K (or V) rows of one stage
+    static constexpr int STAGE = 2 * TILE;
+    static constexpr int RING = NST * STAGE;    // per warp
+    static constexpr int SMEM = NW * RING + NW * NST * 8;
+};
+
+__device__ __forceinline__ bool bar_wait_bounded(uint32_t bar, uint32_t parity) {
+    if (tc::mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = tc::globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (tc::mbar_try_wait(bar, parity)) return true;
+        if ((it & 63u) == 0 && tc::globaltimer_ns() - t0 > tc::kWaitLimitNs) return false;
+    }
+}
+
+template <int DH, int G>
+__global__ void __launch_bounds__(128, 2) decode_attn_bulk_kernel(Dims s, DecodeLayout L, unsigned char *state,
+                                                                  StepGeom gm, const __nv_bfloat16 *__restrict__ q_t,
+                                                                  unsigned *err) {
+    using Cfg = DecodeBulkCfg<DH>;
+    constexpr int NW = Cfg::NW, NST = Cfg::NST, NQ = DH / 32, NM = DH / 16, VW = DH / 64;
+    constexpr float kL2e = 1.4426950408889634f, kLn2f = 0.6931471805599453f;
+    static_assert(G >= 1 && G <= 8 && (DH == 64 || DH == 128), "decode mma shape");
+    static_assert(NW * G * (5 + DH) * 4 <= NW * Cfg::RING, "combine area fits in the rings");
+    extern __shared__ __align__(128) unsigned char dsm[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, c = lane & 3;
+    const int bg = blockIdx.x, split = blockIdx.y, b = bg / s.Hkv, g = bg % s.Hkv;
+    const int l0 = split * gm.per, l1 = min(gm.n, l0 + gm.per);
+    const int band_lo = max(0, gm.pos - s.w + 1);
+    const float sl2 = s.scale * kL2e;
+    unsigned char *ring = dsm + warp * Cfg::RING;
+    const uint32_t bar0 = tc::smem_u32(dsm + NW * Cfg::RING) + warp * NST * 8;
+    const __nv_bfloat16 *khat = reinterpret_cast<const __nv_bfloat16 *>(state + L.khat);
+    const __nv_bfloat16 *vhat = reinterpret_cast<const __nv_bfloat16 *>(state + L.vhat);
+    const __nv_bfloat16 *rk = reinterpret_cast<const __nv_bfloat16 *>(state + L.ring_k);
+    const __nv_bfloat16 *rv = reinterpret_cast<const __nv_bfloat16 *>(state + L.ring_v);
+
+    if (lane == 0) {
+        for (int st = 0; st < NST; ++st) tc::mbar_init(bar0 + st * 8, 1);
+        tc::mbar_fence_init();
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+
+    const int ntiles = (l1 - l0 + 15) / 16;
+    const int my_tiles = ntiles > warp ? (ntiles - warp + NW - 1) / NW : 0;
+    // lane 0: copies of this warp's tile number `it` into stage it % NST
+    auto issue = [&](int it) {
+        const int st = it % NST;
+        const int k0 = l0 + 16 * (warp + NW * it), k1 = min(l1, k0 + 16);
+        const uint32_t sK = tc::smem_u32(ring + st * Cfg::STAGE), sV = sK + Cfg::TILE, bar = bar0 + st * 8;
+        tc::mbar_arrive_expect_tx(bar, (uint32_t)(k1 - k0) * DH * 2 * 2);
+        for (int li = k0; li < k1;) {
+            int end;
+            size_t row;
+            const __nv_bfloat16 *kb, *vb;
+            if (li < gm.nk) {
+                end = min(k1, gm.nk);
+                row = (size_t)bg * L.cap_chunks * s.k + li;
+                kb = khat;
+                vb = vhat;
+            } else {
+                const int j = gm.lo + (li - gm.nk);
+                end = min(k1, li + (s.C - j % s.C));  // to the end of j's chunk slot
+                row = (size_t)bg * L.ring_rows + ring_row(s, j);
+                kb = rk;
+                vb = rv;
+            }
+            const uint32_t bytes = (uint32_t)(end - li) * DH * 2, off = (uint32_t)(li - k0) * DH * 2;
+            bulk_load(sK + off, kb + row * DH, bytes, bar);
+            bulk_load(sV + off, vb + row * DH, bytes, bar);
+            li = end;
+        }
+    };
+    if (lane == 0)
+        for (int it = 0; it < min(NST, my_tiles); ++it) issue(it);
+
+    unsigned qa0[2 * NQ], qa2[2 * NQ];
+#pragma unroll
+    for (int i = 0; i < NQ; ++i) {
+        uint4 u = make_uint4(0u, 0u, 0u, 0u);
+        if (gq < G) u = __ldg(reinterpret_cast<const uint4 *>(q_t + ((size_t)b * s.H + g * G + gq) * DH) + 4 * i + c);
+        qa0[2 * i] = u.x;
+        qa2[2 * i] = u.y;
+        qa0[2 * i + 1] = u.z;
+        qa2[2 * i + 1] = u.w;
+    }
+    float ot[NM][4];
+#pragma unroll
+    for (int mt = 0; mt < NM; ++mt) ot[mt][0] = ot[mt][1] = ot[mt][2] = ot[mt][3] = 0.f;
+    float m = -INFINITY, l = 0.f, bm = -INFINITY, bl = 0.f, sd = -INFINITY;
+
+    bool ok = true;
+    int it = 0;
+    for (; it < my_tiles; ++it) {
+        const int st = it % NST;
+        ok = bar_wait_bounded(bar0 + st * 8, (it / NST) & 1);
+        if (!__all_sync(0xffffffffu, ok)) {
+            ok = false;
+            break;
+        }
+        const int base = l0 + 16 * (warp + NW * it);
+        const uint4 *K4 = reinterpret_cast<const uint4 *>(ring + st * Cfg::STAGE);
+        const uint4 *V4 = reinterpret_cast<const uint4 *>(ring + st * Cfg::STAGE + Cfg::TILE);
+        // rows past the end of a partial tile were not copied (stale or never written): read as zeros
+        DecodeKV<DH> t;
+        const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const bool in = base + gq + 8 * h < l1;
+#pragma unroll
+            for (int i = 0; i < NQ; ++i) t.k[h][i] = in ? K4[(gq + 8 * h) * (DH / 8) + 4 * i + c] : z4;
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int key = 2 * c + (r & 1) + 8 * (r >> 1);
+            const bool in = base + key < l1;
+#pragma unroll
+            for (int i = 0; i < VW; ++i) t.v[r][i] = in ? V4[key * (DH / 8) + gq * VW + i] : z4;
+        }
+        // ---- S = Q K^T, online softmax, band statistics, O^T += V^T P^T (as decode_attn_mma_kernel)
+        float stt[2][4];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            stt[h][0] = stt[h][1] = stt[h][2] = stt[h][3] = 0.f;
+#pragma unroll
+            for (int i = 0; i < NQ; ++i) {
+                mma16816(stt[h], qa0[2 * i], 0u, qa2[2 * i], 0u, t.k[h][i].x, t.k[h][i].y);
+                mma16816(stt[h], qa0[2 * i + 1], 0u, qa2[2 * i + 1], 0u, t.k[h][i].z, t.k[h][i].w);
+            }
+        }
+        float sc[4];
+        float mx = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int li = base + 2 * c + (e & 1) + 8 * (e >> 1);
+            float x = stt[e >> 1][e & 1] * sl2;
+            if (li >= l1) x = -INFINITY;
+            if (li < l1 && li >= gm.nk) {
+                const int j = gm.lo + (li - gm.nk);
+                if (j == gm.pos) {
+                    sd = x;
+                } else if (j >= band_lo) {
+                    if (x > bm) {
+                        bl = bl * tc::ex2(bm - x) + 1.f;
+                        bm = x;
+                    } else {
+                        bl += tc::ex2(x - bm);
+                    }
+                }
+            }
+            sc[e] = x;
+            mx = fmaxf(mx, x);
+        }
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        const float mn = fmaxf(m, mx);      // finite: key base+0 is always in range
+        const float so = tc::ex2(m - mn);  // m = -inf gives 0
+        float pp[4], ps = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            pp[e] = tc::ex2(sc[e] - mn);
+            ps += pp[e];
+        }
+        ps += __shfl_xor_sync(0xffffffffu, ps, 1);
+        ps += __shfl_xor_sync(0xffffffffu, ps, 2);
+        l = l * so + ps;
+        m = mn;
+        const float so0 = __shfl_sync(0xffffffffu, so, 8 * c), so1 = __shfl_sync(0xffffffffu, so, 8 * c + 4);
+#pragma unroll
+        for (int mt = 0; mt < NM; ++mt) {
+            ot[mt][0] *= so0;
+            ot[mt][1] *= so1;
+            ot[mt][2] *= so0;
+            ot[mt][3] *= so1;
+        }
+        const unsigned pb0 = tc::pack_bf16x2(pp[0], pp[1]), pb1 = tc::pack_bf16x2(pp[2], pp[3]);
+        const unsigned *w0 = reinterpret_cast<const unsigned *>(&t.v[0][0]);
+        const unsigned *w1 = reinterpret_cast<const unsigned *>(&t.v[1][0]);
+        const unsigned *w2 = reinterpret_cast<const unsigned *>(&t.v[2][0]);
+        const unsigned *w3 = reinterpret_cast<const unsigned *>(&t.v[3][0]);
+#pragma unroll
+        for (int mt = 0; mt < NM; ++mt) {
+            const unsigned sel = (mt & 1) ? 0x7632u : 0x5410u;
+            const int lo_w = mt >> 1, hi_w = (NM + mt) >> 1;
+            mma16816(ot[mt], __byte_perm(w0[lo_w], w1[lo_w], sel), __byte_perm(w0[hi_w], w1[hi_w], sel),
+                     __byte_perm(w2[lo_w], w3[lo_w], sel), __byte_perm(w2[hi_w], w3[hi_w], sel), pb0, pb1);
+        }
+        // the stage's rows are in registers and used: hand it to the next copy
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && it + NST < my_tiles) issue(it + NST);
+    }
+    if (!ok) {
+        if (lane == 0) {
+            report(err, DEV_ERR_TIMEOUT);
+            // copies this warp issued and did not consume: wait for them (bounded) before exiting
+            for (int k = it; k < min(my_tiles, it + NST); ++k)
+                tc::mbar_wait_drain(bar0 + (k % NST) * 8, (k / NST) & 1, 100000000ull);
+        }
+        __syncwarp();
+    }
+    // band statistics of head gq: combine the four lanes of the row
+#pragma unroll
+    for (int x = 1; x <= 2; x <<= 1) {
+        const float obm = __shfl_xor_sync(0xffffffffu, bm, x);
+        const float obl = __shfl_xor_sync(0xffffffffu, bl, x);
+        const float nbm = fmaxf(bm, obm);
+        bl = (bm == -INFINITY ? 0.f : bl * tc::ex2(bm - nbm)) + (obm == -INFINITY ? 0.f : obl * tc::ex2(obm - nbm));
+        bm = nbm;
+        sd = fmaxf(sd, __shfl_xor_sync(0xffffffffu, sd, x));
+    }
+    __syncthreads();  // every warp is done with its ring: reuse it for the combine
+    auto sm_ml = reinterpret_cast<float (*)[G][5]>(dsm);
+    auto sm_acc = reinterpret_cast<float (*)[G][DH]>(dsm + NW * G * 5 * 4);
+    if (gq < G && c == 0) {
+        sm_ml[warp][gq][0] = m;
+        sm_ml[warp][gq][1] = l;
+        sm_ml[warp][gq][2] = bm;
+        sm_ml[warp][gq][3] = bl;
+        sm_ml[warp][gq][4] = sd;
+    }
+#pragma unroll
+    for (int hc = 0; hc < 2; ++hc) {
+        const int hh = 2 * c + hc;
+        if (hh < G) {
+#pragma unroll
+            for (int mt = 0; mt < NM; ++mt) {
+                sm_acc[warp][hh][2 * NM * gq + mt] = ot[mt][hc];
+                sm_acc[warp][hh][2 * NM * gq + NM + mt] = ot[mt][2 + hc];
+            }
+        }
+    }
+    __syncthreads();
+    float *part_out = reinterpret_cast<float *>(state + L.part);
+    float *band_out = reinterpret_cast<float *>(state + L.band);
+    for (int t2 = threadIdx.x; t2 < G * DH; t2 += blockDim.x) {
+        const int h = t2 / DH, x = t2 % DH;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w_ = 0; w_ < NW; ++w_) M = fmaxf(M, sm_ml[w_][h][0]);
+        float A = 0.f, Ls = 0.f;
+#pragma unroll
+        for (int w_ = 0; w_ < NW; ++w_) {
+            const float mw = sm_ml[w_][h][0];
+            const float f = mw == -INFINITY ? 0.f : exp2f(mw - M);
+            A = fmaf(sm_acc[w_][h][x], f, A);
+            Ls = fmaf(sm_ml[w_][h][1], f, Ls);
+        }
+        const size_t pi = ((size_t)b * s.H + g * G + h) * kDecodeMaxSplits + split;
+        float *pp2 = part_out + pi * (DH + 2);
+        pp2[2 + x] = A;
+        if (x == 0) {
+            pp2[0] = M == -INFINITY ? M : M * kLn2f;
+            pp2[1] = Ls;
+            float BM = -INFINITY, SD = -INFINITY;
+#pragma unroll
+            for (int w_ = 0; w_ < NW; ++w_) {
+                BM = fmaxf(BM, sm_ml[w_][h][2]);
+                SD = fmaxf(SD, sm_ml[w_][h][4]);
+            }
+            float BL = 0.f;
+#pragma unroll
+            for (int w_ = 0; w_ < NW; ++w_) {
+                const float b_ = sm_ml[w_][h][2];
+                if (b_ != -INFINITY) BL = fmaf(sm_ml[w_][h][3], exp2f(b_ - BM), BL);
+            }
+            band_out[pi * 3 + 0] = BM == -INFINITY ? BM : BM * kLn2f;
+            band_out[pi * 3 + 1] = BL;
+            band_out[pi * 3 + 2] = SD == -INFINITY ? SD : SD * kLn2f;
+        }
+    }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(128) decode_combine_kernel(Dims s, DecodeLayout L, unsigned char *state, StepGeom gm,
                                                              const T *__restrict__ q_t, const T *__restrict__ Wq,
@@ -849,6 +1144,9 @@ __global__ void __launch_bounds__(kCombineThreads) decode_combine_wide_kernel(Di
     const float *S = reinterpret_cast<const float *>(state + L.S) + (size_t)bg * D * d;
     const float *z = reinterpret_cast<const float *>(state + L.z) + (size_t)bg * D;
     const size_t pb0 = ((size_t)b * s.H + g * G) * kDecodeMaxSplits;
+    // the group's linear state is read late (phi^T S): start bringing it into L2 now
+    for (size_t off = (size_t)tid * 128; off < (size_t)D * d * 4; off += (size_t)kCombineThreads * 128)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const char *>(S) + off));
 
     for (int hh = warp; hh < G; hh += kCombineThreads / 32) {
         const size_t pb = pb0 + (size_t)hh * kDecodeMaxSplits;
@@ -983,12 +1281,12 @@ __global__ void __launch_bounds__(kCombineThreads) decode_combine_wide_kernel(Di
         for (int hh = 0; hh < 8; ++hh) acc[hh] = make_float4(0.f, 0.f, 0.f, 0.f);
         const float4 *S4 = reinterpret_cast<const float4 *>(S) + x4;
         int a = a0;
-        for (; a + 4 <= a1; a += 4) {
-            float4 sv[4];
+        for (; a + 8 <= a1; a += 8) {
+            float4 sv[8];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) sv[u] = S4[(size_t)(a + u) * (d / 4)];
+            for (int u = 0; u < 8; ++u) sv[u] = S4[(size_t)(a + u) * (d / 4)];
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
+            for (int u = 0; u < 8; ++u)
 #pragma unroll
                 for (int hh = 0; hh < 8; ++hh)
                     if (hh < G) {
@@ -1174,6 +1472,23 @@ cudaError_t launch_decode_init(const Dims &s, unsigned char *state, const Decode
     return cudaGetLastError();
 }
 
+// K/V rows of the tensor-core decode attention: staged in shared memory by bulk copies (true) or
+// loaded into registers (false).
+constexpr bool kDecodeBulk = true;
+
+// SMs of the current device (looked up once per device).
+int decode_sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
 template <typename T>
 static cudaError_t decode_step_t(const Dims &s, unsigned char *state, const DecodeLayout &L, int pos, const void *Wq,
                                  const void *Wk, const void *q_t, const void *k_t, const void *v_t, void *o_t,
@@ -1191,9 +1506,31 @@ static cudaError_t decode_step_t(const Dims &s, unsigned char *state, const Deco
         gm.nk = 0;
         gm.n = 0;
     }
-    gm.nsplit = gm.n == 0 ? 0 : min(kDecodeMaxSplits, (gm.n + 511) / 512);
-    gm.per = gm.nsplit ? (gm.n + gm.nsplit - 1) / gm.nsplit : 0;
     const int BK = s.B * s.Hkv;
+    gm.nsplit = gm.n == 0 ? 0 : min(kDecodeMaxSplits, (gm.n + 511) / 512);
+    const bool tc_path = sizeof(T) == 2 && (s.d == 64 || s.d == 128) && s.G() <= 8 && (8 % s.G()) == 0;
+    if (tc_path && kDecodeBulk && gm.n > 0) {
+        // splits of 512..2048 keys, as few as keep the last wave of CTAs nearly full (the
+        // bulk-copy kernel keeps 2 CTAs per SM at d = 128, 4 at d = 64)
+        const int slots = decode_sm_count() * (s.d == 128 ? 2 : 4);
+        const int lo_ns = max(1, (gm.n + 2047) / 2048), hi_ns = min(kDecodeMaxSplits, max(lo_ns, (gm.n + 511) / 512));
+        int best = hi_ns;
+        double best_eff = -1.0;
+        for (int ns = lo_ns; ns <= hi_ns; ++ns) {
+            const long long ctas = (long long)BK * ns, waves = (ctas + slots - 1) / slots;
+            const double eff = (double)ctas / (double)(waves * slots);
+            if (eff >= 0.95) {
+                best = ns;
+                break;
+            }
+            if (eff > best_eff) {
+                best_eff = eff;
+                best = ns;
+            }
+        }
+        gm.nsplit = best;
+    }
+    gm.per = gm.nsplit ? (gm.n + gm.nsplit - 1) / gm.nsplit : 0;
     int ts = timing_begin(kTimeDecodeAppend, st);
     decode_append_kernel<T><<<BK, 128, 0, st>>>(s, L, state, pos, (const T *)k_t, (const T *)v_t, err);
     timing_end(ts, st);
@@ -1204,8 +1541,19 @@ static cudaError_t decode_step_t(const Dims &s, unsigned char *state, const Deco
         const int G = s.G();
 #define STILL_DECODE_PACKED(DPL, GG) \
     decode_attn_packed_kernel<T, DPL, GG><<<grid, 256, 0, st>>>(s, L, state, gm, (const T *)q_t)
-#define STILL_DECODE_MMA(DH, GG) \
-    decode_attn_mma_kernel<DH, GG><<<grid, 128, 0, st>>>(s, L, state, gm, (const __nv_bfloat16 *)q_t)
+#define STILL_DECODE_MMA(DH, GG)                                                                          \
+    do {                                                                                                    \
+        if (kDecodeBulk) {                                                                                  \
+            const int smem_ = DecodeBulkCfg<DH>::SMEM;                                                      \
+            cudaError_t e_ = cudaFuncSetAttribute(decode_attn_bulk_kernel<DH, GG>,                          \
+                                                  cudaFuncAttributeMaxDynamicSharedMemorySize, smem_);      \
+            if (e_ != cudaSuccess) return e_;                                                               \
+            decode_attn_bulk_kernel<DH, GG><<<grid, 128, smem_, st>>>(s, L, state, gm,                      \
+                                                                      (const __nv_bfloat16 *)q_t, err);     \
+        } else {                                                                                            \
+            decode_attn_mma_kernel<DH, GG><<<grid, 128, 0, st>>>(s, L, state, gm, (const __nv_bfloat16 *)q_t); \
+        }                                                                                                   \
+    } while (0)
         const bool mma = sizeof(T) == 2 && (s.d == 64 || s.d == 128) && (G == 1 || G == 2 || G == 4 || G == 8);
         if (mma) {
             if (s.d == 128) {
