@@ -52,6 +52,9 @@ def parse():
     p.add_argument("--cpu-seconds", type=float, default=15.0, help="target oracle time of the CPU baseline")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--e2e-steps", type=int, default=10)
+    p.add_argument("--router", choices=["saliency", "diagonal"], default="saliency",
+                   help="prefill token router: the Self-Saliency Score, or the diagonal-only ablation "
+                        "(score -> per-chunk top-k -> prefill with that selection)")
     return p.parse_args()
 
 
@@ -174,7 +177,7 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- CPU baseline (oracle)
 
-def oracle_sample(shape, seconds: float, nthreads: int | None = None):
+def oracle_sample(shape, seconds: float, nthreads: int | None = None, router: str = "saliency"):
     """Time the fp64 oracle on whole (batch, KV group) slices -- saliency + top-k over all N tokens, then
     the outputs of every `stride`-th query row of the group's G heads -- slice after slice until about
     `seconds` have been spent (stride 1 when a slice is cheap enough), and scale to the whole layer.
@@ -200,7 +203,7 @@ def oracle_sample(shape, seconds: float, nthreads: int | None = None):
         t0 = time.perf_counter()
         idx = None
         if shape.w > 0 and shape.k > 0 and shape.T > 0:
-            _, r = oracle.saliency(d, q, k, nthreads=nth)
+            r = oracle.diagonal_score(d, q, k) if router == "diagonal" else oracle.saliency(d, q, k, nthreads=nth)[1]
             idx = oracle.topk(d, r)
         t_sel = time.perf_counter() - t0
         if stride is None:  # calibrate on a coarse sample of the first slice
@@ -223,7 +226,7 @@ def oracle_sample(shape, seconds: float, nthreads: int | None = None):
         if t_sel_sum >= seconds:
             break
     t_layer = t_total / done * len(slices)
-    desc = (f"oracle fp64, {done} of {len(slices)} (batch, KV group) slices of {shape.G} heads: saliency + top-k "
+    desc = (f"oracle fp64, {done} of {len(slices)} (batch, KV group) slices of {shape.G} heads: {router} score + top-k "
             f"over all {shape.N} tokens and every {stride}-th query row ({rows_done} rows); "
             f"{t_sel_sum:.1f} s measured, scaled to all rows and slices")
     return shape.B * shape.N / t_layer, t_sel_sum, desc, nth
@@ -250,7 +253,7 @@ def run_reference(args):
         if shape.decode_steps > 0:
             v, t, desc, nth = oracle_decode_sample(shape, per_step)
         else:
-            v, t, desc, nth = oracle_sample(shape, per_step)
+            v, t, desc, nth = oracle_sample(shape, per_step, router=getattr(args, "router", "saliency"))
         if i >= args.warmup:
             vals.append(v)
     value = statistics.median(vals) if vals else None
@@ -268,7 +271,8 @@ def run_reference(args):
 def config_of(shape, args):
     return {"workload": args.workload, "B": shape.B, "H": shape.H, "Hkv": shape.Hkv, "N": shape.N, "d": shape.d,
             "D": shape.D, "w": shape.w, "C": shape.C, "k": shape.k, "global_batch": shape.B * args.gpus,
-            "seq_len": shape.N, "parallelism": f"replicas{args.gpus}", "l2": "flushed before every step"}
+            "seq_len": shape.N, "parallelism": f"replicas{args.gpus}", "l2": "flushed before every step",
+            "router": getattr(args, "router", "saliency")}
 
 
 def max_over_ranks(value_ms: float, world: int, device=None) -> float:
@@ -315,15 +319,44 @@ def run_ours(args):
     flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
 
-    def step(t):
-        still.still_hybrid_prefill(dims, t["q"], t["k"], t["v"], t["wq"], t["wk"], o, workspace=ws)
+    diag = args.router == "diagonal" and shape.w > 0 and shape.k > 0 and shape.T > 0
+    if diag:
+        r_sel = torch.empty(shape.B, shape.Hkv, shape.N, dtype=torch.float32, device="cuda")
+        idx_sel = torch.empty(shape.B, shape.Hkv, shape.T, shape.k, dtype=torch.int32, device="cuda")
 
+    def step(t):
+        if diag:  # diagonal-only router: score, per-chunk top-k, then the layer on that selection
+            still.still_diagonal_score(dims, t["q"], t["k"], r_sel)
+            still.still_select_topk(dims, r_sel, idx_sel)
+            still.still_hybrid_prefill(dims, t["q"], t["k"], t["v"], t["wq"], t["wk"], o, idx_in=idx_sel,
+                                       workspace=ws)
+        else:
+            still.still_hybrid_prefill(dims, t["q"], t["k"], t["v"], t["wq"], t["wk"], o, workspace=ws)
+
+    torch.cuda.synchronize()
+    torch.cuda.reset_peak_memory_stats()
+    free0, total_mem = torch.cuda.mem_get_info()
     for _ in range(args.warmup):
         flush.zero_()
         step(devt)
     torch.cuda.synchronize()
     if still.still_get_device_status() != 0:
         raise RuntimeError("device-side check failed during warm-up")
+    # every byte the layer touches is a torch allocation made above (inputs, output, workspace; the
+    # library allocates nothing), so the allocator's high-water mark minus the L2-flush buffer is the
+    # layer's peak device memory
+    peak_layer = torch.cuda.max_memory_allocated() - flush.numel()
+    es = 2 if shape.dtype == "bf16" else 4
+    memory = {
+        "peak_device_bytes": int(peak_layer),
+        "workspace_bytes": int(ws.numel()),
+        "io_bytes": int(sum(t.numel() * t.element_size() for t in devt.values()) + o.numel() * o.element_size()),
+        # dense causal softmax attention of the same layer, for comparison (analytic):
+        "dense_flash_bytes": int((2 * shape.B * shape.H + 2 * shape.B * shape.Hkv) * shape.N * shape.d * es
+                                 + shape.B * shape.H * shape.N * 4),  # Q, K, V, O + row LSE
+        "dense_scores_bytes": int(shape.B * shape.H * shape.N * shape.N * es),  # materialised N x N scores
+        "free_before_bytes": int(free0), "total_bytes": int(total_mem),
+    }
 
     gpu_id = None
     try:
@@ -405,9 +438,10 @@ def run_ours(args):
         "gpu_launches": launches, "clocks": clocks,
         "kernel_ms_per_step": {k_: v_[0] / args.steps for k_, v_ in kern.items() if v_[1]},
         "layer_tflops": layer_flops(shape) / (ms_per_step / 1e3) / 1e12, "device_status": status,
+        "memory": memory,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, t, desc, nth = oracle_sample(shape, args.cpu_seconds)
+        v, t, desc, nth = oracle_sample(shape, args.cpu_seconds, router=args.router)
         line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": nth, "kind": "oracle", "sample": desc}
     if world > 1:
         torch.distributed.barrier()

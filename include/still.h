@@ -87,6 +87,18 @@ STILL_API still_status still_saliency(const still_dims *dims, const void *q, con
                             void *stream);
 
 /*
+ * Diagonal-only router score ([p4] "Surprising findings": an ablation routes on
+ * the diagonal attention alone): r_gi = mean over the G query heads of g of the
+ * raw diagonal logit tau <q_hi, k_gi> (read as the logit, not its band
+ * probability).  An alternative to still_saliency's r_kv: its per-chunk top-k
+ * (still_select_topk) passed as idx_in to still_hybrid_prefill runs the layer
+ * with this router.  w may be 0.
+ *   q [B,H,N,d], k [B,Hkv,N,d] dtype;  r_kv [B,Hkv,N] fp32 out
+ */
+STILL_API still_status still_diagonal_score(const still_dims *dims, const void *q, const void *k, float *r_kv,
+                                            void *stream);
+
+/*
  * Per-chunk top-k ([p1] "Chunk-Wise": scores per chunk, kept tokens chosen in
  * one batch; [p4] "Approach": top-scoring tokens go to softmax attention).
  * For every full chunk c < T = floor(N/C) of every (b, g): the k positions

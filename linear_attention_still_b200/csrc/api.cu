@@ -201,6 +201,16 @@ still_status still_saliency(const still_dims *dims, const void *q, const void *k
     return STILL_OK;
 }
 
+still_status still_diagonal_score(const still_dims *dims, const void *q, const void *k, float *r_kv, void *stream) {
+    Dims s;
+    still_status st = check_dims(dims, &s);
+    if (st) return st;
+    if ((long long)s.B * s.N == 0) return STILL_OK;
+    if (!q || !k || !r_kv || !aligned16(q) || !aligned16(k) || !aligned16(r_kv)) return STILL_ERR_INVALID_ARG;
+    STILL_LAUNCH(launch_diagonal_score(s, q, k, r_kv, static_cast<cudaStream_t>(stream)));
+    return STILL_OK;
+}
+
 still_status still_select_topk(const still_dims *dims, const float *r_kv, int32_t *idx, void *stream) {
     Dims s;
     still_status st = check_dims(dims, &s);

@@ -359,6 +359,50 @@ __global__ void __launch_bounds__(128) merge_generic_kernel(Dims s, const T *__r
 }  // namespace
 
 // ------------------------------------------------------------------ launchers
+// Diagonal-only router ([p4] "Surprising findings": routing on the diagonal attention alone):
+// r_{g,i} = mean over the G heads of g of tau <q_hi, k_gi>.  HBM-bound (reads Q and K once): a warp
+// per (b, g, row); each lane holds its d/32 slice of k_gi and dots it with each head's q_hi.
+template <typename T>
+__global__ void __launch_bounds__(256) diagonal_score_kernel(Dims s, const T *__restrict__ q,
+                                                             const T *__restrict__ k, float *__restrict__ r) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, G = s.G();
+    const long long row = (long long)blockIdx.x * 8 + warp;  // over B * Hkv * N
+    if (row >= (long long)s.B * s.Hkv * s.N) return;
+    const long long bg = row / s.N;
+    const int i = (int)(row % s.N), b = (int)(bg / s.Hkv), g = (int)(bg % s.Hkv);
+    const T *ki = k + (size_t)row * s.d;
+    float kv[kMaxD / 32];
+#pragma unroll
+    for (int u = 0; u < kMaxD / 32; ++u) {
+        const int x = lane + 32 * u;
+        kv[u] = x < s.d ? to_f(ki[x]) : 0.f;
+    }
+    float acc = 0.f;
+    for (int hh = 0; hh < G; ++hh) {
+        const T *qi = q + (((size_t)b * s.H + (size_t)g * G + hh) * s.N + i) * s.d;
+        float dot = 0.f;
+#pragma unroll
+        for (int u = 0; u < kMaxD / 32; ++u) {
+            const int x = lane + 32 * u;
+            if (x < s.d) dot = fmaf(to_f(qi[x]), kv[u], dot);
+        }
+        acc += warp_sum(dot);
+    }
+    if (lane == 0) r[row] = s.scale * acc / (float)G;
+}
+
+cudaError_t launch_diagonal_score(const Dims &s, const void *q, const void *k, float *r_kv, cudaStream_t st) {
+    const long long rows = (long long)s.B * s.Hkv * s.N;
+    if (rows == 0) return cudaSuccess;
+    const unsigned grid = (unsigned)((rows + 7) / 8);
+    if (s.bf16)
+        diagonal_score_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(s, (const __nv_bfloat16 *)q,
+                                                                   (const __nv_bfloat16 *)k, r_kv);
+    else
+        diagonal_score_kernel<float><<<grid, 256, 0, st>>>(s, (const float *)q, (const float *)k, r_kv);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_saliency_generic(const Dims &s, const void *q, const void *k, float *r_kv, float *r_q,
                                     cudaStream_t st) {
     dim3 grid((s.N + kSalRows - 1) / kSalRows, s.B * s.Hkv);

@@ -46,6 +46,7 @@ struct MergeOperands {
 };
 
 // ---- generic kernels (fp32 or bf16 storage, fp32 arithmetic) ----
+cudaError_t launch_diagonal_score(const Dims &s, const void *q, const void *k, float *r_kv, cudaStream_t st);
 cudaError_t launch_saliency_generic(const Dims &s, const void *q, const void *k, float *r_kv, float *r_q,
                                     cudaStream_t st);
 cudaError_t launch_topk_gather(const Dims &s, const float *r, int32_t *idx, const void *k, const void *v, void *khat,

@@ -22,7 +22,7 @@ EXPORTS = ("still_status_string", "still_saliency", "still_select_topk", "still_
            "still_prefill_workspace_bytes", "still_prefill_workspace_layout", "still_hybrid_prefill",
            "still_decode_state_bytes", "still_decode_init", "still_decode_step", "still_get_device_status",
            "still_launch_count", "still_timing_enable", "still_timing_read", "still_debug_set_trace",
-           "still_hybrid_prefill_static")
+           "still_hybrid_prefill_static", "still_diagonal_score")
 
 
 class StillError(RuntimeError):
@@ -50,6 +50,7 @@ _SIG = {
     "still_status_string": ([ct.c_int], ct.c_char_p),
     "still_saliency": ([_D, _P, _P, _P, _P, _P], ct.c_int),
     "still_select_topk": ([_D, _P, _P, _P], ct.c_int),
+    "still_diagonal_score": ([_D, _P, _P, _P, _P], ct.c_int),
     "still_npmap": ([ct.c_int, ct.c_int, ct.c_int, ct.c_int, ct.c_int, ct.c_int, _P, _P, _P, _P], ct.c_int),
     "still_prefill_workspace_bytes": ([_D], ct.c_size_t),
     "still_prefill_workspace_layout": ([_D, ct.POINTER(still_ws_layout)], ct.c_int),
@@ -118,6 +119,11 @@ def still_saliency(dims, q, k, r_kv, r_q=None, stream=None):
 
 def still_select_topk(dims, r_kv, idx, stream=None):
     _ok("still_select_topk", _lib.still_select_topk(ct.byref(dims), _ptr(r_kv), _ptr(idx), _stream(stream)))
+
+
+def still_diagonal_score(dims, q, k, r_kv, stream=None):
+    _ok("still_diagonal_score",
+        _lib.still_diagonal_score(ct.byref(dims), _ptr(q), _ptr(k), _ptr(r_kv), _stream(stream)))
 
 
 def still_npmap(B, Hx, N, d, D, dtype, x, W, phi, stream=None):

@@ -11,6 +11,7 @@ from .oracle import (  # noqa: F401
     Dims,
     build,
     saliency,
+    diagonal_score,
     topk,
     npmap,
     prefill,

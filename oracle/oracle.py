@@ -70,6 +70,7 @@ def _load():
         P = ct.c_void_p
         lib.od_saliency.argtypes = [ct.POINTER(_ODims), P, P, P, P, ct.c_int]
         lib.od_topk.argtypes = [ct.POINTER(_ODims), P, P]
+        lib.od_diagonal_score.argtypes = [ct.POINTER(_ODims), P, P, P]
         lib.od_npmap.argtypes = [ct.c_int, ct.c_int, ct.c_int, P, P, P]
         lib.od_prefill.argtypes = [ct.POINTER(_ODims), P, P, P, P, P, P, P, P, P, P, ct.c_long, ct.c_int]
         lib.od_linear_state.argtypes = [ct.POINTER(_ODims), P, P, P, P, ct.c_int, ct.c_int, ct.c_int, P, P]
@@ -116,6 +117,15 @@ def saliency(dims: Dims, q, k, nthreads: int | None = None):
     r = np.empty((dims.B, dims.Hkv, dims.N))
     _check(lib.od_saliency(ct.byref(dims.c()), _p(q), _p(k), _p(sigma), _p(r), _nthreads(nthreads)), "saliency")
     return sigma, r
+
+
+def diagonal_score(dims: Dims, q, k) -> np.ndarray:
+    """Diagonal-only router score r [B,Hkv,N] (float64): group mean of tau <q_hi, k_gi>."""
+    lib = _load()
+    q, k = _f64(q), _f64(k)
+    r = np.empty((dims.B, dims.Hkv, dims.N))
+    _check(lib.od_diagonal_score(ct.byref(dims.c()), _p(q), _p(k), _p(r)), "diagonal_score")
+    return r
 
 
 def topk(dims: Dims, r) -> np.ndarray:

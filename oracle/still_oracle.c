@@ -201,6 +201,35 @@ int od_saliency(const od_dims *s, const double *q, const double *k, double *sigm
     return OD_OK;
 }
 
+/*
+ * Diagonal-only router ([p4] "Surprising findings": an ablation that routes on
+ * the diagonal attention alone): r_{g,i} = mean over the G query heads of g of
+ * the raw diagonal logit s_ii = tau <q_hi, k_gi>.
+ * READING: "the diagonal attention alone" is taken as the raw logit s_ii, not
+ * its probability within the band (which would make it the saliency score's
+ * own ingredient p_ii); the GQA mean follows the saliency score's reading.
+ */
+int od_diagonal_score(const od_dims *s, const double *q, const double *k, double *r)
+{
+    int e = od_check(s);
+    if (e) return e;
+    int G = s->H / s->Hkv;
+    for (int b = 0; b < s->B; ++b)
+        for (int g = 0; g < s->Hkv; ++g)
+            for (int i = 0; i < s->N; ++i) {
+                const double *ki = k + (((size_t)b * s->Hkv + g) * s->N + i) * s->d;
+                double acc = 0.0;
+                for (int hh = 0; hh < G; ++hh) {
+                    const double *qi = q + (((size_t)b * s->H + g * G + hh) * s->N + i) * s->d;
+                    double dot = 0.0;
+                    for (int x = 0; x < s->d; ++x) dot += qi[x] * ki[x];
+                    acc += s->scale * dot;
+                }
+                r[((size_t)b * s->Hkv + g) * s->N + i] = acc / G;
+            }
+    return OD_OK;
+}
+
 /* ------------------------------------------------------------------------ */
 /* per-chunk top-k ([p1] "Chunk-Wise": scores are computed per chunk and the  */
 /* kept tokens are chosen in one batch; [p4] "Approach": the top-scoring      */

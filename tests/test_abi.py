@@ -91,6 +91,8 @@ def test_step_entry_points_reject(lib):
     d = _dims(lib)
     assert lib._lib.still_saliency(ct.byref(d), None, FAKE, FAKE, None, None) == 1
     assert lib._lib.still_select_topk(ct.byref(d), FAKE + 8, FAKE, None) == 1
+    assert lib._lib.still_diagonal_score(ct.byref(d), FAKE, None, FAKE, None) == 1
+    assert lib._lib.still_diagonal_score(ct.byref(d), FAKE, FAKE, FAKE + 4, None) == 1
     assert lib._lib.still_npmap(1, 2, 10, 12, 64, 1, FAKE, FAKE, FAKE, None) == 1
     assert lib._lib.still_npmap(1, 2, 10, 64, 512, 1, FAKE, FAKE, FAKE, None) == 2
 

@@ -158,3 +158,36 @@ def test_empty_inputs_are_noops(lib):
     lib.still_hybrid_prefill(d, x, x, x, x, x, x, workspace=torch.zeros(256, dtype=torch.uint8, device="cuda"))
     assert lib.still_launch_count() == n0
     assert lib.still_get_device_status() == 0
+
+
+@pytest.mark.parametrize("name", ["f32_b1_h2_n512", "bf16_gqa_ragged", "bf16_d128_g8", "bf16_no_window"])
+def test_diagonal_score_entry_point(lib, oracle_mod, name):
+    """Diagonal-only router score against the oracle's definition."""
+    shape = CASES[name]
+    inp = make_inputs(shape)
+    r = torch.empty(shape.B, shape.Hkv, shape.N, device="cuda")
+    lib.still_diagonal_score(lib.dims_of(shape), dev(inp.q, shape), dev(inp.k, shape), r)
+    assert lib.still_get_device_status() == 0
+    assert score_err(r.cpu().numpy(), oracle_mod.diagonal_score(odims(shape), inp.q, inp.k)) <= SCORE_TOL
+
+
+@pytest.mark.parametrize("name", ["bf16_gqa_ragged", "bf16_d128_two_chunk_window"])
+def test_diagonal_router_layer(lib, oracle_mod, name):
+    """The layer with the diagonal-only router: GPU score -> GPU per-chunk top-k -> prefill with that
+    selection, against the oracle's score, selection and layer output on the GPU's selection."""
+    shape = CASES[name]
+    inp = make_inputs(shape)
+    d = lib.dims_of(shape)
+    r = torch.empty(shape.B, shape.Hkv, shape.N, device="cuda")
+    lib.still_diagonal_score(d, dev(inp.q, shape), dev(inp.k, shape), r)
+    idx = torch.full((shape.B, shape.Hkv, shape.T, shape.k), -1, dtype=torch.int32, device="cuda")
+    lib.still_select_topk(d, r, idx)
+    od = odims(shape)
+    ora_r = oracle_mod.diagonal_score(od, inp.q, inp.k)
+    gr, gidx = r.cpu().numpy(), idx.cpu().numpy()
+    assert score_err(gr, ora_r) <= SCORE_TOL
+    check_selection(shape, shape.N, gidx, gr, ora_r, oracle_mod.topk(od, ora_r))
+    out = gpu_prefill(shape, inp, idx_in=gidx)
+    assert out["status"] == 0
+    ref = oracle_mod.prefill(od, inp.q, inp.k, inp.v, inp.wq, inp.wk, idx_in=gidx)["o"]
+    assert row_rel_err(out["o"], ref) <= OUT_TOL[shape.dtype]

@@ -96,6 +96,50 @@ def test_saliency_golden(oracle_mod):
 
 # ---------------------------------------------------------------- top-k
 
+# ---------------------------------------------------------------- diagonal-only router
+
+def test_diagonal_score_self_match_is_squared_norm(oracle_mod):
+    """q_hi = k_gi for every head of the group: r_gi = tau * ||k_gi||^2 (norm from numpy's routine)."""
+    rng = np.random.default_rng(21)
+    B, H, Hkv, N, d = 2, 6, 2, 33, 16
+    k = _rand(rng, B, Hkv, N, d)
+    q = np.repeat(k, H // Hkv, axis=1)
+    dims = oracle_mod.Dims(B=B, H=H, Hkv=Hkv, N=N, d=d, D=4, w=8, C=8, k=2)
+    r = oracle_mod.diagonal_score(dims, q, k)
+    np.testing.assert_allclose(r, np.linalg.norm(k, axis=-1) ** 2 / math.sqrt(d), rtol=1e-12)
+
+
+def test_diagonal_score_gqa_mean_cancels(oracle_mod):
+    """Heads of a group in pairs (q, -q): the group mean of the diagonal logits is 0."""
+    rng = np.random.default_rng(22)
+    q1 = _rand(rng, 1, 2, 20, 8)
+    q = np.concatenate([q1, -q1], axis=1)  # heads 0,1 | 2,3 = -(0,1); one group of 4
+    k = _rand(rng, 1, 1, 20, 8)
+    dims = oracle_mod.Dims(B=1, H=4, Hkv=1, N=20, d=8, D=4, w=4, C=4, k=1)
+    assert np.abs(oracle_mod.diagonal_score(dims, q, k)).max() < 1e-14
+
+
+def test_diagonal_router_selects_like_saliency_when_band_logits_vanish(oracle_mod):
+    """Keys orthogonal to every other token's query: each band logit s_ij (j != i) is 0, so
+    sigma = softplus(s_ii - ln(n-1)) is increasing in s_ii at a fixed band size n; the per-chunk
+    top-k of the diagonal router then equals that of the Self-Saliency Score."""
+    rng = np.random.default_rng(23)
+    N, C, w, kk = 64, 16, 16, 5
+    d = N
+    k = np.zeros((1, 1, N, d))
+    q = np.zeros((1, 1, N, d))
+    for i in range(N):  # token i lives on coordinate i only: <q_i, k_j> = 0 for j != i
+        k[0, 0, i, i] = rng.uniform(0.5, 3.0)
+        q[0, 0, i, i] = rng.uniform(0.5, 3.0)
+    dims = oracle_mod.Dims(B=1, H=1, Hkv=1, N=N, d=d, D=4, w=w, C=C, k=kk)
+    rd = oracle_mod.diagonal_score(dims, q, k)
+    _, rs = oracle_mod.saliency(dims, q, k)
+    # chunks past the first have full bands (n = w) for every row
+    sel_d = oracle_mod.topk(dims, rd)[:, :, 1:]
+    sel_s = oracle_mod.topk(dims, rs)[:, :, 1:]
+    np.testing.assert_array_equal(sel_d, sel_s)
+
+
 def test_topk_matches_sort(oracle_mod):
     """Top-k = first k of a sort by (score desc, index asc), reported ascending; ties and +inf."""
     rng = np.random.default_rng(4)
