@@ -52,6 +52,10 @@ def parse():
     p.add_argument("--cpu-seconds", type=float, default=15.0, help="target oracle time of the CPU baseline")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--e2e-steps", type=int, default=10)
+    p.add_argument("--keep", choices=["config", "all", "none"], default="config",
+                   help="tokens kept per chunk: the workload's k, all of them (k = C: exact causal softmax "
+                        "attention through the same kernels, a same-box dense comparator), or none (k = 0: "
+                        "window + linear branch only)")
     p.add_argument("--router", choices=["saliency", "diagonal"], default="saliency",
                    help="prefill token router: the Self-Saliency Score, or the diagonal-only ablation "
                         "(score -> per-chunk top-k -> prefill with that selection)")
@@ -245,7 +249,7 @@ def run_reference(args):
     rank, world, _ = dist_setup(args)
     if rank != 0:
         return
-    shape = WORKLOADS[args.workload]
+    shape = workload_shape(args)
     per_step = max(2.0, 150.0 / max(1, args.steps + args.warmup))
     vals = []
     desc, nth = "", 1
@@ -268,11 +272,22 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def workload_shape(args):
+    """The workload's shape with --keep applied (k = C keeps every token of a decided chunk)."""
+    shape = WORKLOADS[args.workload]
+    keep = getattr(args, "keep", "config")
+    if keep == "all" and shape.w > 0:
+        shape = shape.replace(k=shape.C)
+    elif keep == "none":
+        shape = shape.replace(k=0)
+    return shape
+
+
 def config_of(shape, args):
     return {"workload": args.workload, "B": shape.B, "H": shape.H, "Hkv": shape.Hkv, "N": shape.N, "d": shape.d,
             "D": shape.D, "w": shape.w, "C": shape.C, "k": shape.k, "global_batch": shape.B * args.gpus,
             "seq_len": shape.N, "parallelism": f"replicas{args.gpus}", "l2": "flushed before every step",
-            "router": getattr(args, "router", "saliency")}
+            "router": getattr(args, "router", "saliency"), "keep": getattr(args, "keep", "config")}
 
 
 def max_over_ranks(value_ms: float, world: int, device=None) -> float:
@@ -305,7 +320,7 @@ def run_ours(args):
                                 device_id=torch.device("cuda", local))
     from linear_attention_still_b200 import still
 
-    shape = WORKLOADS[args.workload]
+    shape = workload_shape(args)
     tdt = torch.bfloat16 if shape.dtype == "bf16" else torch.float32
     inp = make_inputs(shape.replace(seed=rank))
     host = {n: torch.from_numpy(np.ascontiguousarray(getattr(inp, n)[:, :, :shape.N] if n in "qkv" else
@@ -500,7 +515,7 @@ def run_decode(args):
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local))
     from linear_attention_still_b200 import still
-    shape = WORKLOADS[args.workload]
+    shape = workload_shape(args)
     N, steps, B = shape.N, shape.decode_steps, shape.B
     tdt = torch.bfloat16 if shape.dtype == "bf16" else torch.float32
     e2e_steps = min(args.e2e_steps, 20)

@@ -23,6 +23,9 @@ CASES = {
     "bf16_one_token": Shape(B=1, H=4, Hkv=1, N=1, d=64, D=64, w=128, C=128, k=8),
     "f32_gqa_d128_D64": Shape(B=1, H=4, Hkv=2, N=520, d=128, D=64, w=128, C=64, k=8, dtype="f32"),
     "bf16_d128_g8": Shape(B=1, H=16, Hkv=2, N=1100, d=128, D=128, w=256, C=256, k=40),
+    # largest head dim, feature width and group the library takes (SIMT path)
+    "f32_max_d_D_group": Shape(B=1, H=32, Hkv=1, N=200, d=256, D=256, w=64, C=64, k=8, dtype="f32"),
+    "bf16_max_d_D": Shape(B=1, H=4, Hkv=2, N=260, d=256, D=256, w=128, C=64, k=16),
 }
 
 
