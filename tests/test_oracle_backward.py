@@ -1,0 +1,76 @@
+"""Pins of the oracle's backward pass (oracle/backward.py) to central finite differences of the C
+forward oracle, with the per-chunk selection held fixed; plus the NP-Map backward alone."""
+import math
+
+import numpy as np
+import pytest
+
+from oracle import backward
+
+
+def _problem(rng, B, H, Hkv, N, d, D):
+    q = rng.standard_normal((B, H, N, d)) * np.exp(rng.normal(0, 0.4, (B, H, N, 1)))
+    k = rng.standard_normal((B, Hkv, N, d)) * np.exp(rng.normal(0, 0.4, (B, Hkv, N, 1)))
+    v = rng.standard_normal((B, Hkv, N, d))
+    wq = rng.standard_normal((H, d, D)) / math.sqrt(d)
+    wk = rng.standard_normal((Hkv, d, D)) / math.sqrt(d)
+    do = rng.standard_normal((B, H, N, d))
+    return q, k, v, wq, wk, do
+
+
+def _fd_check(oracle_mod, dims, args, idx, grads, eps=1e-5, tol=1e-6):
+    names = ("q", "k", "v", "wq", "wk")
+    q, k, v, wq, wk, do = args
+
+    def loss(q_, k_, v_, wq_, wk_):
+        o = oracle_mod.prefill(dims, q_, k_, v_, wq_, wk_, idx_in=idx, nthreads=1)["o"]
+        return float(np.sum(o * do))
+
+    base = [q, k, v, wq, wk]
+    for a, (name, g) in enumerate(zip(names, grads)):
+        x = base[a]
+        fd = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            ix = it.multi_index
+            plus = [t.copy() for t in base]
+            minus = [t.copy() for t in base]
+            plus[a][ix] += eps
+            minus[a][ix] -= eps
+            fd[ix] = (loss(*plus) - loss(*minus)) / (2 * eps)
+        err = np.abs(fd - g).max() / max(np.abs(fd).max(), 1e-12)
+        assert err < tol, (name, err)
+
+
+@pytest.mark.parametrize("w,C,kk,Hkv", [(4, 4, 2, 1), (8, 4, 1, 2), (0, 4, 0, 1), (4, 4, 4, 1)])
+def test_backward_matches_finite_differences(oracle_mod, w, C, kk, Hkv):
+    """Hybrid (window + kept + linear), a two-chunk window with GQA, pure linear (w = 0), and every
+    token kept (k = C: causal softmax)."""
+    rng = np.random.default_rng(31 + w + kk)
+    B, H, N, d, D = 1, 2, 14, 3, 3
+    args = _problem(rng, B, H, Hkv, N, d, D)
+    dims = oracle_mod.Dims(B=B, H=H, Hkv=Hkv, N=N, d=d, D=D, w=w, C=C, k=kk)
+    q, k, v, wq, wk, do = args
+    idx = oracle_mod.prefill(dims, q, k, v, wq, wk)["idx"] if (w > 0 and kk > 0) else None
+    grads = backward.layer_backward(q, k, v, wq, wk, do, idx, w, C)
+    _fd_check(oracle_mod, dims, args, idx, grads)
+
+
+def test_npmap_backward_matches_finite_differences():
+    rng = np.random.default_rng(5)
+    x, W, dphi = rng.standard_normal(5), rng.standard_normal((5, 4)), rng.standard_normal(4)
+    dx, dW = backward.npmap_backward(x, W, dphi)
+    eps = 1e-6
+    for a in range(5):
+        xp, xm = x.copy(), x.copy()
+        xp[a] += eps
+        xm[a] -= eps
+        fd = (backward.npmap_forward(xp, W) - backward.npmap_forward(xm, W)) @ dphi / (2 * eps)
+        assert abs(fd - dx[a]) < 1e-8 * max(1.0, abs(fd))
+    for a in range(5):
+        for c in range(4):
+            Wp, Wm = W.copy(), W.copy()
+            Wp[a, c] += eps
+            Wm[a, c] -= eps
+            fd = (backward.npmap_forward(x, Wp) - backward.npmap_forward(x, Wm)) @ dphi / (2 * eps)
+            assert abs(fd - dW[a, c]) < 1e-8 * max(1.0, abs(fd))
