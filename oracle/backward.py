@@ -100,17 +100,17 @@ def layer_backward(q, k, v, wq, wk, do, idx, w, C, scale=None):
                     o = o / Z
                     go = float(gi @ o)
                     dphiq = np.zeros_like(phiq)
-                    for n_, j in enumerate(soft):
-                        p = e[n_] / Z
-                        ds = p * (float(gi @ V[j]) - go)   # dL/ds_ij
-                        dq[b, h, i] += tau * ds * K[j]
-                        dk[b, g, j] += tau * ds * qi
-                        dv[b, g, j] += p * gi
-                    for n_, j in enumerate(lin):
-                        dw = (float(gi @ V[j]) - go) * math.exp(-M) / Z   # dL/dw_ij
-                        dv[b, g, j] += (wl[n_] / Z) * gi
-                        dphiq += dw * phik[j]
-                        dphik[j] += dw * phiq
+                    if len(soft):  # every index of a row's sets is distinct
+                        p = e / Z
+                        ds = p * (V[soft] @ gi - go)       # dL/ds_ij
+                        dq[b, h, i] += tau * (ds @ K[soft])
+                        dk[b, g, soft] += tau * np.outer(ds, qi)
+                        dv[b, g, soft] += np.outer(p, gi)
+                    if len(lin):
+                        dw = (V[lin] @ gi - go) * math.exp(-M) / Z   # dL/dw_ij
+                        dv[b, g, lin] += np.outer(wl / Z, gi)
+                        dphiq += dw @ phik[lin]
+                        dphik[lin] += np.outer(dw, phiq)
                     dx, dW = npmap_backward(qi, wq[h], dphiq)
                     dq[b, h, i] += dx
                     dwq[h] += dW
