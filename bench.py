@@ -56,6 +56,9 @@ def parse():
                    help="tokens kept per chunk: the workload's k, all of them (k = C: exact causal softmax "
                         "attention through the same kernels, a same-box dense comparator), or none (k = 0: "
                         "window + linear branch only)")
+    p.add_argument("--pass", dest="pass_", choices=["forward", "backward"], default="forward",
+                   help="prefill workloads: time the forward layer (default) or its backward pass "
+                        "(gradients of q, k, v, Wq, Wk with the selection held fixed)")
     p.add_argument("--router", choices=["saliency", "diagonal"], default="saliency",
                    help="prefill token router: the Self-Saliency Score, or the diagonal-only ablation "
                         "(score -> per-chunk top-k -> prefill with that selection)")
@@ -659,12 +662,136 @@ def run_decode(args):
         print(json.dumps(line), flush=True)
 
 
+def backward_flops(shape):
+    """Algorithmic FLOPs of the backward pass: per (query-head, softmax key) the forward recompute
+    (QK^T, PV: 4d) and the backward (QK^T again, dO.V, dq, dk, dv: 10d); per query-head the NP-Map
+    and linear-state products (about 12 d D); per unselected key of a decided chunk 8 d D."""
+    rows = shape.B * shape.H
+    return rows * (14 * shape.d * int(soft_sizes(shape).sum()) + shape.N * 12 * shape.d * shape.D) + \
+        shape.B * shape.Hkv * shape.N * 8 * shape.d * shape.D
+
+
+def run_backward(args):
+    import numpy as np
+    import torch
+
+    rank, world, local = dist_setup(args)
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    from linear_attention_still_b200 import still
+    shape = workload_shape(args)
+    tdt = torch.bfloat16 if shape.dtype == "bf16" else torch.float32
+    inp = make_inputs(shape.replace(seed=rank))
+    host = {n: torch.from_numpy(np.ascontiguousarray(getattr(inp, n))).to(tdt) for n in ("q", "k", "v", "wq", "wk")}
+    host["do"] = torch.from_numpy(np.random.default_rng(rank).standard_normal(inp.q.shape).astype(np.float32)).to(tdt)
+    del inp
+    devt = {n: t.cuda() for n, t in host.items()}
+    dims = still.dims_of(shape)
+    # the selection the forward makes, held fixed by the backward
+    ws_f = torch.empty(still.still_prefill_workspace_bytes(dims), dtype=torch.uint8, device="cuda")
+    o = torch.empty_like(devt["q"])
+    still.still_hybrid_prefill(dims, devt["q"], devt["k"], devt["v"], devt["wq"], devt["wk"], o, workspace=ws_f)
+    idx = None
+    if shape.k > 0 and shape.T > 0:
+        off = still.still_prefill_workspace_layout(dims)["idx"]
+        n_idx = shape.B * shape.Hkv * shape.T * shape.k
+        idx = ws_f[off:off + 4 * n_idx].view(torch.int32).clone()
+    del ws_f, o
+    f32 = dict(dtype=torch.float32, device="cuda")
+    grads = [torch.empty(shape.B, shape.H, shape.N, shape.d, **f32),
+             torch.empty(shape.B, shape.Hkv, shape.N, shape.d, **f32),
+             torch.empty(shape.B, shape.Hkv, shape.N, shape.d, **f32),
+             torch.empty(shape.H, shape.d, shape.D, **f32), torch.empty(shape.Hkv, shape.d, shape.D, **f32)]
+    ws = torch.empty(still.still_backward_workspace_bytes(dims), dtype=torch.uint8, device="cuda")
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(t):
+        still.still_hybrid_backward(dims, t["q"], t["k"], t["v"], t["wq"], t["wk"], idx, t["do"], *grads, workspace=ws)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step(devt)
+    torch.cuda.synchronize()
+    if still.still_get_device_status() != 0:
+        raise RuntimeError("device-side check failed during warm-up")
+    gpu_id = None
+    try:
+        gpu_id = f"GPU-{torch.cuda.get_device_properties(local).uuid}"
+    except Exception:
+        pass
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+    n0 = still.still_launch_count()
+    for s_, e_ in evs:
+        flush.zero_()
+        s_.record(stream)
+        step(devt)
+        e_.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop()
+    launches = still.still_launch_count() - n0
+    total_ms = max_over_ranks(sum(s_.elapsed_time(e_) for s_, e_ in evs), world, "cuda")
+    ms_per_step = total_ms / args.steps
+    tokens = shape.B * shape.N
+    # end to end: inputs and dO from pinned host memory, the five gradients back to the host
+    pinned = {n: t.pin_memory() for n, t in host.items()}
+    outs = [torch.empty(g_.shape, dtype=g_.dtype).pin_memory() for g_ in grads]
+    e_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+             for _ in range(args.e2e_steps)]
+    for s_, e_ in e_evs:
+        flush.zero_()
+        s_.record(stream)
+        for n in devt:
+            devt[n].copy_(pinned[n], non_blocking=True)
+        step(devt)
+        for h_, g_ in zip(outs, grads):
+            h_.copy_(g_, non_blocking=True)
+        e_.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(sum(s_.elapsed_time(e_) for s_, e_ in e_evs), world, "cuda")
+    # SIMT fp32 kernels: the ALU roofline is the FFMA rate, 148 SMs x 128 lanes x 2 FLOP x 1965 MHz
+    peak = 148 * 128 * 2 * 1.965e9 / 1e12
+    achieved = backward_flops(shape) / (ms_per_step / 1e3) / 1e12
+    line = {
+        "metric": "STILL hybrid-attn backward tokens/s per layer (gradients of q, k, v, Wq, Wk)",
+        "value": job_throughput(tokens, args.steps, world, total_ms), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": shape.dtype, "data": "synthetic",
+        "config": dict(config_of(shape, args), **{"pass": "backward"}),
+        "roofline": {"kernel": "backward pass (all kernels)", "bound": "alu", "achieved": achieved, "peak": peak,
+                     "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                     "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 FLOP x 1965 MHz (SIMT kernels)",
+                     "flops_per_step": backward_flops(shape)},
+        "e2e": {"value": job_throughput(tokens, args.e2e_steps, world, e2e_ms), "unit": "tokens/s",
+                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in pinned.values()),
+                "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in outs)},
+        "gpu_launches": launches, "clocks": clocks, "device_status": still.still_get_device_status(),
+    }
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
     elif WORKLOADS[args.workload].decode_steps > 0:
         run_decode(args)
+    elif args.pass_ == "backward":
+        run_backward(args)
     else:
         run_ours(args)
 

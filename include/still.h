@@ -195,6 +195,26 @@ STILL_API still_status still_hybrid_prefill_static(const still_dims *dims, const
                                                    void *stream);
 
 /*
+ * Backward pass of still_hybrid_prefill ([p1] introduction and "Chunk-Wise":
+ * one chunk-parallel implementation for training and inference): gradients of
+ * L = sum(dO * o) with respect to q, k, v, Wq and Wk, with the per-chunk
+ * selection idx held fixed (top-k is a discrete choice with no gradient).
+ * Requires a window (w >= 1; STILL_ERR_UNSUPPORTED for w = 0).
+ *   q, k, v, Wq, Wk  as for still_hybrid_prefill (dtype)
+ *   idx   [B,Hkv,T,k] int32, the selection the forward used (NULL when k = 0 or T = 0)
+ *   dO    [B,H,N,d] dtype, the gradient of the layer output
+ *   dq    [B,H,N,d], dk/dv [B,Hkv,N,d], dWq [H,d,D], dWk [Hkv,d,D]: fp32 out (overwritten)
+ *   workspace  device scratch of still_backward_workspace_bytes(dims) bytes, 256-byte aligned
+ * SIMT kernels with fp32 arithmetic (dk and dv accumulate with atomics, so
+ * their rounding depends on the schedule).
+ */
+STILL_API size_t still_backward_workspace_bytes(const still_dims *dims);
+STILL_API still_status still_hybrid_backward(const still_dims *dims, const void *q, const void *k, const void *v,
+                                             const void *Wq, const void *Wk, const int32_t *idx, const void *dO,
+                                             float *dq, float *dk, float *dv, float *dWq, float *dWk,
+                                             void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Chunk-granular delayed decode ([p1] "Chunk-Wise": during decoding the
  * selection is delayed at chunk granularity).  The state is one caller-owned
  * device buffer holding, per (b, g): the kept K/V cache, the linear state

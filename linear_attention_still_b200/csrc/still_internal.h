@@ -61,6 +61,21 @@ cudaError_t launch_merge_generic(const Dims &s, const void *q, const void *k, co
                                  const float *phik, void *o, cudaStream_t st);
 
 // ---- decode ----
+// Scratch of the backward pass (fp32, inside the caller's workspace).
+struct BackwardScratch {
+    float *phik;   // [B,Hkv,N,D]   NP-Map features of the keys
+    float *S, *z;  // [B,Hkv,T+1,D,d], [B,Hkv,T+1,D]  forward linear state per query chunk
+    float *A;      // [B,H,N,D]     a_i = exp(-Ms) / Z * phi(q_i)
+    float *Dv;     // [B,H,N]       D_i = <dO_i, o_i>
+    float *dYq;    // [B,H,N,D]     dL/d(q Wq)
+    float *R, *r;  // [B,Hkv,T+1,D,d], [B,Hkv,T+1,D]  suffix sums over query chunks
+    float *dYk;    // [B,Hkv,N,D]   dL/d(k Wk)
+};
+cudaError_t launch_backward(const Dims &s, const void *q, const void *k, const void *v, const void *Wq,
+                            const void *Wk, const int32_t *idx, const void *dO, float *dq, float *dk, float *dv,
+                            float *dWq, float *dWk, const BackwardScratch &w, unsigned *err, cudaStream_t st,
+                            int *launches);
+
 // Per-kernel event timing (still_timing_enable): returns a slot for timing_end, or -1 when off.
 int timing_begin(int cls, cudaStream_t st);
 void timing_end(int slot, cudaStream_t st);

@@ -22,7 +22,8 @@ EXPORTS = ("still_status_string", "still_saliency", "still_select_topk", "still_
            "still_prefill_workspace_bytes", "still_prefill_workspace_layout", "still_hybrid_prefill",
            "still_decode_state_bytes", "still_decode_init", "still_decode_step", "still_get_device_status",
            "still_launch_count", "still_timing_enable", "still_timing_read", "still_debug_set_trace",
-           "still_hybrid_prefill_static", "still_diagonal_score")
+           "still_hybrid_prefill_static", "still_diagonal_score", "still_backward_workspace_bytes",
+           "still_hybrid_backward")
 
 
 class StillError(RuntimeError):
@@ -56,6 +57,8 @@ _SIG = {
     "still_prefill_workspace_layout": ([_D, ct.POINTER(still_ws_layout)], ct.c_int),
     "still_hybrid_prefill": ([_D, _P, _P, _P, _P, _P, _P, _P, _P, ct.c_size_t, _P, ct.c_int, _P], ct.c_int),
     "still_hybrid_prefill_static": ([_D, _P, _P, _P, _P, _P, _P, _P, _P, ct.c_int, _P], ct.c_int),
+    "still_backward_workspace_bytes": ([_D], ct.c_size_t),
+    "still_hybrid_backward": ([_D] + [_P] * 13 + [ct.c_size_t, _P], ct.c_int),
     "still_decode_state_bytes": ([_D, ct.c_int], ct.c_size_t),
     "still_decode_init": ([_D, ct.c_int, _P, _P], ct.c_int),
     "still_decode_step": ([_D, _P, ct.c_int, ct.c_int, _P, _P, _P, _P, _P, _P, _P], ct.c_int),
@@ -159,6 +162,20 @@ def still_hybrid_prefill_static(dims, q, k, v, wq, wk, o, idx_in=None, state=Non
     _ok("still_hybrid_prefill_static",
         _lib.still_hybrid_prefill_static(ct.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(wq), _ptr(wk), _ptr(o),
                                          _ptr(idx_in), _ptr(state), int(state_capacity), _stream(stream)))
+
+
+def still_backward_workspace_bytes(dims) -> int:
+    return int(_lib.still_backward_workspace_bytes(ct.byref(dims)))
+
+
+def still_hybrid_backward(dims, q, k, v, wq, wk, idx, do, dq, dk, dv, dwq, dwk, workspace=None, workspace_bytes=None,
+                          stream=None):
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _ok("still_hybrid_backward",
+        _lib.still_hybrid_backward(ct.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(wq), _ptr(wk), _ptr(idx), _ptr(do),
+                                   _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dwq), _ptr(dwk), _ptr(workspace),
+                                   int(workspace_bytes), _stream(stream)))
 
 
 def still_decode_state_bytes(dims, capacity: int) -> int:

@@ -97,6 +97,22 @@ def test_step_entry_points_reject(lib):
     assert lib._lib.still_npmap(1, 2, 10, 64, 512, 1, FAKE, FAKE, FAKE, None) == 2
 
 
+def test_backward_rejects(lib):
+    f = lib._lib.still_hybrid_backward
+    d0 = _dims(lib, w=0, k=0)
+    assert f(ct.byref(d0), *([FAKE] * 13), 1 << 40, None) == 2          # no window: not covered
+    d = _dims(lib)
+    need = lib.still_backward_workspace_bytes(d)
+    assert need > 0
+    args = [FAKE] * 13
+    args[5] = None                                                       # selection missing (k > 0)
+    assert f(ct.byref(d), *args, need, None) == 1
+    assert f(ct.byref(d), *([FAKE] * 13), need - 1, None) == 3           # workspace too small
+    args = [FAKE] * 13
+    args[6] = FAKE + 4                                                   # misaligned dO
+    assert f(ct.byref(d), *args, need, None) == 1
+
+
 def test_decode_rejects(lib):
     d = _dims(lib)
     assert lib.still_decode_state_bytes(d, 4096) > 0
