@@ -121,7 +121,7 @@ __device__ void npmap_backward_warp(const float *xs, const T *__restrict__ W, in
 
 // One warp per query row (b, h, i): recomputes the row's forward, then dq_i (all of it), the
 // softmax branch's contributions to dk and dv (atomics), a_i, D_i and dL/d(q_i Wq).
-template <typename T>
+template <typename T, bool ATOMIC_KV>
 __global__ void __launch_bounds__(32 * kBwdWarps) bwd_row_kernel(Dims s, const T *__restrict__ q,
                                                                  const T *__restrict__ k, const T *__restrict__ v,
                                                                  const T *__restrict__ Wq,
@@ -131,6 +131,7 @@ __global__ void __launch_bounds__(32 * kBwdWarps) bwd_row_kernel(Dims s, const T
                                                                  const T *__restrict__ dO, float *__restrict__ dq,
                                                                  float *__restrict__ dk, float *__restrict__ dv,
                                                                  float *__restrict__ Abuf, float *__restrict__ Dbuf,
+                                                                 float *__restrict__ Msb, float *__restrict__ iZb,
                                                                  float *__restrict__ dYq, unsigned *err) {
     __shared__ __align__(16) float qs[kBwdWarps][kMaxD];
     __shared__ __align__(16) float gs[kBwdWarps][kMaxD];
@@ -211,7 +212,12 @@ __global__ void __launch_bounds__(32 * kBwdWarps) bwd_row_kernel(Dims s, const T
         if (x < d) Di = fmaf(gs[warp][x], (acc[u] * a_soft + lin[u] * a_lin) * invZ, Di);
     }
     Di = warp_sum(Di);
-    // ---- softmax branch backward
+    if (lane == 0) {
+        Msb[row] = Ms;
+        iZb[row] = invZ;
+    }
+    // ---- softmax branch backward: dq here; dk and dv by atomics (ATOMIC_KV) or, from the stored
+    //      Ms, 1/Z and D_i, in bwd_kv_block_kernel
     float dqa[kMaxD / 32];
 #pragma unroll
     for (int u = 0; u < kMaxD / 32; ++u) dqa[u] = 0.f;
@@ -237,8 +243,10 @@ __global__ void __launch_bounds__(32 * kBwdWarps) bwd_row_kernel(Dims s, const T
                 const int x = lane + 32 * u;
                 if (x < d) {
                     dqa[u] = fmaf(dSj, to_f(K[(size_t)jr * d + x]), dqa[u]);
-                    atomicAdd(dK + (size_t)jr * d + x, dSj * qs[warp][x]);
-                    atomicAdd(dV + (size_t)jr * d + x, Pj * gs[warp][x]);
+                    if (ATOMIC_KV) {
+                        atomicAdd(dK + (size_t)jr * d + x, dSj * qs[warp][x]);
+                        atomicAdd(dV + (size_t)jr * d + x, Pj * gs[warp][x]);
+                    }
                 }
             }
         }
@@ -262,6 +270,122 @@ __global__ void __launch_bounds__(32 * kBwdWarps) bwd_row_kernel(Dims s, const T
         const int x = lane + 32 * u;
         if (x < d) dq[(size_t)row * d + x] = dqa[u] + dxa[u];
     }
+}
+
+// Softmax branch, key side, by blocks of 32 keys of one (b, g) (d <= 128): the CTA streams the
+// query rows that attend to its keys through shared memory 32 at a time (q, dO and the row's Ms,
+// 1/Z, D_i), and thread (key kk, quarter sl of the head dim) accumulates its quarter of dk_j and
+// dv_j in registers:  P_ij = exp(tau <q_i, k_j> - Ms_i) / Z_i,  dS_ij = tau P_ij (<dO_i, v_j> - D_i),
+// dk_j += dS_ij q_i,  dv_j += P_ij dO_i  (dot products reduced over the 4 threads of a key).
+//   KEPT = false: keys j0..j0+31 of the sequence, queries from j0 to the end of the last key's window
+//   reach (chunks c .. c+m), each pair masked by i >= j and t(i) <= c(j) + m; writes dk, dv.
+//   KEPT = true: 32 kept keys of chunk c (entries of idx), queries of chunks t >= c+m+1 (every pair
+//   counts); adds to dk, dv.
+template <typename T, int DH, bool KEPT>
+__global__ void __launch_bounds__(128) bwd_kv_block_kernel(Dims s, const T *__restrict__ q,
+                                                           const T *__restrict__ k, const T *__restrict__ v,
+                                                           const int32_t *__restrict__ idx,
+                                                           const T *__restrict__ dO, const float *__restrict__ Msb,
+                                                           const float *__restrict__ iZb,
+                                                           const float *__restrict__ Dbuf, float *__restrict__ dk,
+                                                           float *__restrict__ dv) {
+    constexpr int QT = 32, SL = DH / 4;
+    __shared__ __align__(16) float qt[QT][DH];
+    __shared__ __align__(16) float gt[QT][DH];
+    __shared__ float st[QT][4];  // Ms, 1/Z, D, chunk of the row
+    const int tid = threadIdx.x, kk = tid >> 2, sl = tid & 3;
+    const int bg = blockIdx.y, b = bg / s.Hkv, g = bg % s.Hkv, G = s.G(), m = s.m(), T_ = s.T();
+    int j = -1, cj = 0;
+    int i0, i1;
+    if (!KEPT) {
+        const int j0 = blockIdx.x * QT;
+        if (j0 + kk < s.N) j = j0 + kk;
+        const int jl = min(s.N, j0 + QT) - 1;
+        i0 = j0;
+        i1 = min(s.N, (jl / s.C + m + 1) * s.C);
+        cj = j >= 0 ? j / s.C : 0;
+    } else {
+        const int c = blockIdx.x / ((s.k + QT - 1) / QT), n0 = (blockIdx.x % ((s.k + QT - 1) / QT)) * QT;
+        if (n0 + kk < s.k) j = idx[((size_t)bg * T_ + c) * s.k + n0 + kk];
+        if (j >= 0 && (j < c * s.C || j >= (c + 1) * s.C)) j = -1;  // outside its chunk: skipped
+        i0 = (c + m + 1) * s.C;
+        i1 = s.N;
+        cj = c;
+    }
+    float kr[SL], vr[SL], dka[SL], dva[SL];
+#pragma unroll
+    for (int e = 0; e < SL; ++e) {
+        kr[e] = j >= 0 ? to_f(k[((size_t)bg * s.N + j) * DH + sl * SL + e]) : 0.f;
+        vr[e] = j >= 0 ? to_f(v[((size_t)bg * s.N + j) * DH + sl * SL + e]) : 0.f;
+        dka[e] = dva[e] = 0.f;
+    }
+    for (int hh = 0; hh < G; ++hh) {
+        const size_t rb = ((size_t)b * s.H + (size_t)g * G + hh) * s.N;
+        for (int ib = i0; ib < i1; ib += QT) {
+            const int nq = min(QT, i1 - ib);
+            __syncthreads();  // the previous tile is consumed
+            for (int e = tid; e < QT * DH; e += 128) {
+                const int r = e / DH, x = e % DH;
+                qt[r][x] = r < nq ? to_f(q[(rb + ib + r) * DH + x]) : 0.f;
+                gt[r][x] = r < nq ? to_f(dO[(rb + ib + r) * DH + x]) : 0.f;
+            }
+            if (tid < QT) {
+                const int i = ib + tid;
+                st[tid][0] = tid < nq ? Msb[rb + i] : 0.f;
+                st[tid][1] = tid < nq ? iZb[rb + i] : 0.f;
+                st[tid][2] = tid < nq ? Dbuf[rb + i] : 0.f;
+                st[tid][3] = (float)(i / s.C);
+            }
+            __syncthreads();
+            for (int r = 0; r < nq; ++r) {
+                float sp = 0.f, gp = 0.f;
+#pragma unroll
+                for (int e = 0; e < SL; ++e) {
+                    sp = fmaf(qt[r][sl * SL + e], kr[e], sp);
+                    gp = fmaf(gt[r][sl * SL + e], vr[e], gp);
+                }
+                sp += __shfl_xor_sync(0xffffffffu, sp, 1);
+                sp += __shfl_xor_sync(0xffffffffu, sp, 2);
+                gp += __shfl_xor_sync(0xffffffffu, gp, 1);
+                gp += __shfl_xor_sync(0xffffffffu, gp, 2);
+                const int i = ib + r;
+                bool on = j >= 0;
+                if (!KEPT) on = on && i >= j && (int)st[r][3] <= cj + m;
+                const float P = on ? expf(s.scale * sp - st[r][0]) * st[r][1] : 0.f;
+                const float dS = s.scale * P * (gp - st[r][2]);
+#pragma unroll
+                for (int e = 0; e < SL; ++e) {
+                    dka[e] = fmaf(dS, qt[r][sl * SL + e], dka[e]);
+                    dva[e] = fmaf(P, gt[r][sl * SL + e], dva[e]);
+                }
+            }
+        }
+    }
+    if (j >= 0) {
+        float *dkr = dk + ((size_t)bg * s.N + j) * DH + sl * SL, *dvr = dv + ((size_t)bg * s.N + j) * DH + sl * SL;
+#pragma unroll
+        for (int e = 0; e < SL; ++e) {
+            if (KEPT) {
+                dkr[e] += dka[e];
+                dvr[e] += dva[e];
+            } else {
+                dkr[e] = dka[e];
+                dvr[e] = dva[e];
+            }
+        }
+    }
+}
+
+template <typename T, int DH>
+cudaError_t launch_kv_blocks(const Dims &s, const T *Q, const T *K, const T *V, const int32_t *idx, const T *GO,
+                             const BackwardScratch &w, float *dk, float *dv, cudaStream_t st) {
+    bwd_kv_block_kernel<T, DH, false><<<dim3((s.N + 31) / 32, s.B * s.Hkv), 128, 0, st>>>(
+        s, Q, K, V, idx, GO, w.Ms, w.iZ, w.Dv, dk, dv);
+    const int nc = s.T() - s.m() - 1 >= 0 ? s.T() - s.m() : 0;  // chunks c with c + m + 1 <= T
+    if (s.k > 0 && nc > 0)
+        bwd_kv_block_kernel<T, DH, true><<<dim3(nc * ((s.k + 31) / 32), s.B * s.Hkv), 128, 0, st>>>(
+            s, Q, K, V, idx, GO, w.Ms, w.iZ, w.Dv, dk, dv);
+    return cudaGetLastError();
 }
 
 // Per (b, g, query chunk t): R_t = sum over the chunk's rows of all G heads of a_i dO_i^T (D x d)
@@ -395,13 +519,24 @@ cudaError_t backward_t(const Dims &s, const void *q, const void *k, const void *
     e = launch_linear_state(s, w.phik, v, idx, w.S, w.z, nullptr, err, st);
     if (e != cudaSuccess) return e;
     *launches += 2;
-    if ((e = cudaMemsetAsync(dk, 0, sizeof(float) * (size_t)s.B * s.Hkv * s.N * s.d, st)) != cudaSuccess) return e;
-    if ((e = cudaMemsetAsync(dv, 0, sizeof(float) * (size_t)s.B * s.Hkv * s.N * s.d, st)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(w.dYk, 0, sizeof(float) * (size_t)s.B * s.Hkv * s.N * s.D, st)) != cudaSuccess) return e;
     const long long rows = (long long)s.B * s.H * s.N;
-    bwd_row_kernel<T><<<(unsigned)((rows + kBwdWarps - 1) / kBwdWarps), 32 * kBwdWarps, 0, st>>>(
-        s, Q, K, V, WQ, idx, w.S, w.z, GO, dq, dk, dv, w.A, w.Dv, w.dYq, err);
-    ++*launches;
+    const unsigned rgrid = (unsigned)((rows + kBwdWarps - 1) / kBwdWarps);
+    if (s.d == 64 || s.d == 128) {
+        // dk, dv by key blocks (written there; no atomics)
+        bwd_row_kernel<T, false><<<rgrid, 32 * kBwdWarps, 0, st>>>(s, Q, K, V, WQ, idx, w.S, w.z, GO, dq, dk, dv,
+                                                                    w.A, w.Dv, w.Ms, w.iZ, w.dYq, err);
+        e = s.d == 64 ? launch_kv_blocks<T, 64>(s, Q, K, V, idx, GO, w, dk, dv, st)
+                      : launch_kv_blocks<T, 128>(s, Q, K, V, idx, GO, w, dk, dv, st);
+        if (e != cudaSuccess) return e;
+        *launches += 3;
+    } else {
+        if ((e = cudaMemsetAsync(dk, 0, sizeof(float) * (size_t)s.B * s.Hkv * s.N * s.d, st)) != cudaSuccess) return e;
+        if ((e = cudaMemsetAsync(dv, 0, sizeof(float) * (size_t)s.B * s.Hkv * s.N * s.d, st)) != cudaSuccess) return e;
+        bwd_row_kernel<T, true><<<rgrid, 32 * kBwdWarps, 0, st>>>(s, Q, K, V, WQ, idx, w.S, w.z, GO, dq, dk, dv,
+                                                                   w.A, w.Dv, w.Ms, w.iZ, w.dYq, err);
+        ++*launches;
+    }
     bwd_chunk_kernel<T><<<dim3(T_ + 1, s.B * s.Hkv, (s.D * s.d + s.D + 255) / 256), 256, 0, st>>>(s, w.A, w.Dv, GO,
                                                                                                w.R, w.r);
     ++*launches;

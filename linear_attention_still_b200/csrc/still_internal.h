@@ -67,6 +67,7 @@ struct BackwardScratch {
     float *S, *z;  // [B,Hkv,T+1,D,d], [B,Hkv,T+1,D]  forward linear state per query chunk
     float *A;      // [B,H,N,D]     a_i = exp(-Ms) / Z * phi(q_i)
     float *Dv;     // [B,H,N]       D_i = <dO_i, o_i>
+    float *Ms, *iZ;  // [B,H,N]     each row's joint shift and 1 / shifted normaliser
     float *dYq;    // [B,H,N,D]     dL/d(q Wq)
     float *R, *r;  // [B,Hkv,T+1,D,d], [B,Hkv,T+1,D]  suffix sums over query chunks
     float *dYk;    // [B,Hkv,N,D]   dL/d(k Wk)

@@ -17,6 +17,9 @@ CASES = {
     "bf16_d128": Shape(B=1, H=4, Hkv=1, N=260, d=128, D=128, w=128, C=64, k=16),
     "f32_keep_all": Shape(B=1, H=2, Hkv=1, N=150, d=32, D=16, w=32, C=32, k=32, dtype="f32"),
     "f32_keep_none": Shape(B=1, H=2, Hkv=2, N=150, d=32, D=16, w=32, C=32, k=0, dtype="f32"),
+    # d in {64, 128} take dk, dv by key blocks (window pass + kept pass); the cases above with d = 32 by atomics
+    "bf16_keep_all_d64": Shape(B=1, H=2, Hkv=1, N=200, d=64, D=32, w=64, C=64, k=64),
+    "f32_two_chunk_window_d128": Shape(B=1, H=2, Hkv=1, N=230, d=128, D=64, w=64, C=32, k=8, dtype="f32"),
 }
 # fp32 arithmetic on the GPU (dk, dv accumulate with atomics in schedule order) against fp64
 GRAD_TOL = {"f32": 1e-4, "bf16": 1e-3}
