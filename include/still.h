@@ -88,7 +88,7 @@ STILL_API still_status still_saliency(const still_dims *dims, const void *q, con
 
 /*
  * Diagonal-only router score ([p4] "Surprising findings": an ablation routes on
- * the diagonal attention alone): r_gi = mean over the G query heads of g of the
+ * the diagonal term by itself): r_gi = mean over the G query heads of g of the
  * raw diagonal logit tau <q_hi, k_gi> (read as the logit, not its band
  * probability).  An alternative to still_saliency's r_kv: its per-chunk top-k
  * (still_select_topk) passed as idx_in to still_hybrid_prefill runs the layer

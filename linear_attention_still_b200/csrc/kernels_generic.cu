@@ -359,7 +359,7 @@ __global__ void __launch_bounds__(128) merge_generic_kernel(Dims s, const T *__r
 }  // namespace
 
 // ------------------------------------------------------------------ launchers
-// Diagonal-only router ([p4] "Surprising findings": routing on the diagonal attention alone):
+// Diagonal-only router ([p4] "Surprising findings": routing on the diagonal term by itself):
 // r_{g,i} = mean over the G heads of g of tau <q_hi, k_gi>.  HBM-bound (reads Q and K once): a warp
 // per (b, g, row); each lane holds its d/32 slice of k_gi and dots it with each head's q_hi.
 template <typename T>

@@ -101,8 +101,9 @@ static double od_logit(const od_dims *s, const double *qi, const double *kj)
 
 /*
  * Self-Saliency Score of one query row ([p1] "Self-Saliency Score"; [p4]
- * "Approach": a KL-style divergence between the sliding-window attention with
- * and without the diagonal term).
+ * "Approach": a divergence of the Kullback-Leibler kind that compares the
+ * window attention of the token with the same attention once its own key is
+ * left out).
  *
  * READINGS:
  *  - the band is B(i) = {j : max(0, i-w+1) <= j <= i}, i.e. w keys including
@@ -203,9 +204,9 @@ int od_saliency(const od_dims *s, const double *q, const double *k, double *sigm
 
 /*
  * Diagonal-only router ([p4] "Surprising findings": an ablation that routes on
- * the diagonal attention alone): r_{g,i} = mean over the G query heads of g of
+ * the diagonal term by itself): r_{g,i} = mean over the G query heads of g of
  * the raw diagonal logit s_ii = tau <q_hi, k_gi>.
- * READING: "the diagonal attention alone" is taken as the raw logit s_ii, not
+ * READING: "the diagonal term" is taken as the raw logit s_ii, not
  * its probability within the band (which would make it the saliency score's
  * own ingredient p_ii); the GQA mean follows the saliency score's reading.
  */
@@ -323,8 +324,8 @@ int od_npmap(int n, int d, int D, const double *x, const double *W, double *phi)
 /* ------------------------------------------------------------------------ */
 /* routing sets ([p1] intro: selected tokens -> softmax branch, the others    */
 /* -> linear branch, in the same layer; [p1] "Chunk-Wise": selection in       */
-/* batches per chunk, delayed; [p4] "Approach": routing is delayed and done   */
-/* per chunk).                                                                */
+/* batches per chunk, delayed; [p4] "Approach": the routing decision waits    */
+/* and is taken a chunk at a time).                                          */
 /*
  * READING (chunk-granular delay): for query i in chunk t = floor(i/C) with
  * m = w/C,
