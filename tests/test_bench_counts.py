@@ -1,0 +1,72 @@
+"""CPU checks of bench.py's measurement arithmetic: the softmax-set sizes behind the merge FLOP count
+and the decode bytes per step against the oracle's own routing sets, the --keep shapes, and the
+traffic lookup from a profile summary (used only while the kernel sources match its hashes)."""
+import hashlib
+import os
+import sys
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+from linear_attention_still_b200.synth import Shape  # noqa: E402
+from oracle import backward  # noqa: E402
+
+
+def _soft_sets(shape):
+    """|Soft(i)| from the oracle backward's routing sets (selection: the first k rows of each chunk)."""
+    def sel(c):
+        return list(range(c * shape.C, c * shape.C + shape.k))
+    return np.array([len(backward.routing_sets(i, shape.N, shape.w, shape.C, sel)[0]) for i in range(shape.N)])
+
+
+@pytest.mark.parametrize("shape", [Shape(B=1, H=4, Hkv=2, N=1000, d=64, D=64, w=128, C=128, k=16),
+                                   Shape(B=2, H=2, Hkv=1, N=777, d=32, D=16, w=256, C=64, k=8),
+                                   Shape(B=1, H=2, Hkv=1, N=300, d=32, D=16, w=0, C=64, k=0),
+                                   Shape(B=1, H=2, Hkv=1, N=50, d=32, D=16, w=64, C=64, k=8)])
+def test_soft_set_sizes_and_merge_flops(shape):
+    sizes = _soft_sets(shape)
+    np.testing.assert_array_equal(bench.soft_sizes(shape), sizes)
+    want = shape.B * shape.H * sum(4 * shape.d * n + 4 * shape.d * shape.D + 2 * shape.D for n in sizes)
+    assert bench.merge_flops(shape) == want
+
+
+def test_decode_bytes_count_the_softmax_rows():
+    shape = Shape(B=3, H=8, Hkv=2, N=0, d=64, D=32, w=128, C=64, k=8, decode_steps=1)
+    for pos in (0, 63, 64, 191, 192, 500, 1023):
+        full = shape.replace(N=pos + 1)
+        rows = len(backward.routing_sets(pos, pos + 1, shape.w, shape.C,
+                                         lambda c: list(range(c * shape.C, c * shape.C + shape.k)))[0])
+        want = shape.B * shape.Hkv * (rows * 2 * shape.d * 2 + shape.D * shape.d * 4 + shape.D * 4) + \
+            shape.B * shape.H * 2 * shape.d * 2
+        assert bench.decode_step_bytes(full, pos) == want, pos
+
+
+def test_keep_shapes():
+    class A:
+        workload = "llama32_1b_layer_n16k"
+        keep = "all"
+    s = bench.workload_shape(A)
+    assert s.k == s.C
+    A.keep = "none"
+    assert bench.workload_shape(A).k == 0
+    A.keep = "config"
+    assert bench.workload_shape(A).k == 64
+
+
+def test_traffic_lookup_follows_source_hashes(tmp_path, monkeypatch):
+    csrc = tmp_path / "linear_attention_still_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (tmp_path / "profiles").mkdir()
+    (csrc / "a.cu").write_bytes(b"kernel one")
+    digest = hashlib.sha256(b"kernel one").hexdigest()[:16]
+    (tmp_path / "profiles" / "merge_tc_x.md").write_text(
+        "# summary\n\n    workload: wl\n    traffic_bytes_per_step: 12345\n"
+        f"    source_sha256: a.cu={digest}\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.profiled_traffic("wl") == 12345
+    assert bench.profiled_traffic("other") is None
+    (csrc / "a.cu").write_bytes(b"kernel two")  # the kernel changed since the capture
+    assert bench.profiled_traffic("wl") is None
