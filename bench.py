@@ -40,6 +40,8 @@ from linear_attention_still_b200.synth import WORKLOADS, make_inputs  # noqa: E4
 
 DEFAULT_WORKLOAD = "llama32_1b_layer_n16k"
 METRIC = "STILL hybrid-attn prefill tokens/s per layer at 16K/64K; % of roofline"
+METRIC_DECODE = "STILL chunk-delayed decode tokens/s per layer (one token per sequence per step)"
+METRIC_BACKWARD = "STILL hybrid-attn backward tokens/s per layer (gradients of q, k, v, Wq, Wk)"
 
 
 def parse():
@@ -256,19 +258,26 @@ def run_reference(args):
     per_step = max(2.0, 150.0 / max(1, args.steps + args.warmup))
     vals = []
     desc, nth = "", 1
+    backward = shape.decode_steps == 0 and getattr(args, "pass_", "forward") == "backward"
     for i in range(args.warmup + args.steps):
         if shape.decode_steps > 0:
             v, t, desc, nth = oracle_decode_sample(shape, per_step)
+        elif backward:
+            v, t, desc, nth = oracle_backward_sample(shape, per_step)
         else:
             v, t, desc, nth = oracle_sample(shape, per_step, router=getattr(args, "router", "saliency"))
         if i >= args.warmup:
             vals.append(v)
     value = statistics.median(vals) if vals else None
+    metric = METRIC_DECODE if shape.decode_steps > 0 else (METRIC_BACKWARD if backward else METRIC)
+    config = config_of(shape, args)
+    if backward:
+        config["pass"] = "backward"
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "impl": "reference", "metric": metric, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_of(shape, args),
+        "config": config,
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": nth, "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -482,6 +491,50 @@ def decode_step_bytes(shape, pos: int) -> int:
     return shape.B * shape.Hkv * per_bg + shape.B * shape.H * 2 * shape.d * es
 
 
+def oracle_backward_sample(shape, seconds: float):
+    """fp64 oracle backward (oracle/backward.py, one process) on the first n tokens of one (batch,
+    KV group) slice, n grown until about `seconds` are spent, scaled to the layer by the ratio of
+    softmax (query, key) pairs, which dominate the work.  Returns (tokens/s, seconds, description,
+    threads)."""
+    import numpy as np
+
+    from oracle import backward
+    import oracle
+    oracle.build()
+    inp = make_inputs(shape.replace(decode_steps=0), batches=[0])
+    q = np.ascontiguousarray(inp.q[:, :shape.G])
+    k, v = inp.k[:, :1], inp.v[:, :1]
+    wq, wk = inp.wq[:shape.G], inp.wk[:1]
+    rng = np.random.default_rng(0)
+    n = min(shape.N, max(shape.C, 256))
+    spent, t_last = 0.0, 0.0
+    while True:
+        sl = shape.replace(B=1, H=shape.G, Hkv=1, N=n)
+        d = oracle.Dims.of(sl)
+        qs, ks, vs = q[:, :, :n], k[:, :, :n], v[:, :, :n]
+        do = rng.standard_normal(qs.shape)
+        idx = oracle.prefill(d, qs, ks, vs, wq, wk)["idx"] if (sl.k > 0 and sl.T > 0) else None
+        t0 = time.perf_counter()
+        backward.layer_backward(qs, ks, vs, wq, wk, do, idx, sl.w, sl.C)
+        t_last = time.perf_counter() - t0
+        spent += t_last
+        if n >= shape.N:
+            break
+        n2 = min(shape.N, n * 2)
+        # grow the sample only while the next one (work ~ softmax pairs) still fits the budget
+        t_next = t_last * float(soft_sizes(shape, n2).sum()) / max(float(soft_sizes(shape, n).sum()), 1.0)
+        if spent + t_next > seconds:
+            break
+        n = n2
+    pairs_sample = float(soft_sizes(shape, n).sum())
+    pairs_full = float(soft_sizes(shape).sum()) * shape.B * shape.Hkv
+    t_layer = t_last * pairs_full / max(pairs_sample, 1.0)
+    desc = (f"oracle backward fp64 (numpy, 1 process) on the first {n} tokens of one (batch, KV group) slice "
+            f"of {shape.G} heads ({t_last:.1f} s), scaled by softmax (query, key) pairs to the layer "
+            f"(x{pairs_full / max(pairs_sample, 1.0):.0f})")
+    return shape.B * shape.N / t_layer, spent, desc, 1
+
+
 def oracle_decode_sample(shape, seconds: float):
     """fp64 oracle cost of decode rows: one (batch 0, KV group 0) slice of N + steps tokens, the output
     rows of a sample of decode positions (the oracle evaluates the same definition as the prefill
@@ -628,7 +681,7 @@ def run_decode(args):
     close_steps = [j for j, p_ in enumerate(range(first, first + K)) if p_ % shape.C == shape.C - 1]
     status = still.still_get_device_status()
     line = {
-        "metric": "STILL chunk-delayed decode tokens/s per layer (one token per sequence per step)",
+        "metric": METRIC_DECODE,
         "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": shape.dtype, "data": "synthetic",
@@ -763,7 +816,7 @@ def run_backward(args):
     peak = 148 * 128 * 2 * 1.965e9 / 1e12
     achieved = backward_flops(shape) / (ms_per_step / 1e3) / 1e12
     line = {
-        "metric": "STILL hybrid-attn backward tokens/s per layer (gradients of q, k, v, Wq, Wk)",
+        "metric": METRIC_BACKWARD,
         "value": job_throughput(tokens, args.steps, world, total_ms), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": shape.dtype, "data": "synthetic",
