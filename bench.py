@@ -830,6 +830,9 @@ def run_backward(args):
                 "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in outs)},
         "gpu_launches": launches, "clocks": clocks, "device_status": still.still_get_device_status(),
     }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v_, t_, desc, nth = oracle_backward_sample(shape, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": v_, "unit": "tokens/s", "cores": nth, "kind": "oracle", "sample": desc}
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
