@@ -216,6 +216,27 @@ def test_no_window_is_linear_attention_closed_form(oracle_mod):
         np.testing.assert_allclose(out["o"][0, h], want, rtol=1e-12)
 
 
+@pytest.mark.parametrize("m", [1, 2])
+def test_window_plus_linear_closed_form(oracle_mod, m):
+    """k = 0, w = mC, W = 0: <phi(q_i), phi(k_j)> = ||q_i|| ||k_j||, so row i of query chunk t mixes the
+    window [(t-m)C, i] under exp(tau q.k) with every earlier token under ||q_i|| ||k_j|| weights, one
+    normaliser for both (chunk-SWA plus linear attention, written out with plain ranges)."""
+    rng = np.random.default_rng(12)
+    B, H, Hkv, N, d, D, C = 1, 2, 1, 70, 8, 5, 8
+    q, k, v, _, _ = _problem(rng, B, H, Hkv, N, d, D, spread=0.7)
+    out = oracle_mod.prefill(oracle_mod.Dims(B, H, Hkv, N, d, D, m * C, C, 0), q, k, v,
+                             np.zeros((H, d, D)), np.zeros((Hkv, d, D)))
+    tau = 1 / math.sqrt(d)
+    nk = np.linalg.norm(k[0, 0], axis=1)
+    for h in range(H):
+        for i in range(N):
+            lo = max(0, (i // C - m) * C)
+            e = np.exp(tau * (k[0, 0, lo:i + 1] @ q[0, h, i]))
+            wl = np.linalg.norm(q[0, h, i]) * nk[:lo]
+            want = (e @ v[0, 0, lo:i + 1] + wl @ v[0, 0, :lo]) / (e.sum() + wl.sum())
+            np.testing.assert_allclose(out["o"][0, h, i], want, rtol=1e-11, atol=1e-13)
+
+
 def test_no_window_equals_recurrence(oracle_mod):
     """w = 0, k = 0: the layer equals the token-by-token linear recurrence S_i = S_{i-1} + phi(k_i) v_i^T."""
     rng = np.random.default_rng(9)
