@@ -55,6 +55,16 @@ def test_saliency_equals_closed_form(oracle_mod, w):
     assert np.allclose(r[0, 0], sigma[0].mean(0))
 
 
+def test_saliency_window_beyond_sequence(oracle_mod):
+    """A window longer than the sequence clips to [0, i]: the scores equal those of w = N."""
+    rng = np.random.default_rng(14)
+    q, k, *_ = _problem(rng, H=2, Hkv=1, N=30, d=8)
+    base = dict(B=1, H=2, Hkv=1, N=30, d=8, D=4, k=1)
+    s_n, _ = oracle_mod.saliency(oracle_mod.Dims(w=30, C=30, **base), q, k)
+    s_big, _ = oracle_mod.saliency(oracle_mod.Dims(w=40, C=40, **base), q, k)
+    np.testing.assert_array_equal(s_n, s_big)
+
+
 def test_saliency_zero_query(oracle_mod):
     """q = 0: every logit is 0, so p_ii = 1/n and sigma = ln(n/(n-1)) with n the band size."""
     rng = np.random.default_rng(2)
@@ -138,6 +148,14 @@ def test_diagonal_router_selects_like_saliency_when_band_logits_vanish(oracle_mo
     sel_d = oracle_mod.topk(dims, rd)[:, :, 1:]
     sel_s = oracle_mod.topk(dims, rs)[:, :, 1:]
     np.testing.assert_array_equal(sel_d, sel_s)
+
+
+def test_npmap_single_feature_is_the_norm(oracle_mod):
+    """D = 1: f(xW) = [1], so phi(x) = ||x|| whatever W is."""
+    rng = np.random.default_rng(15)
+    for _ in range(5):
+        x, W = rng.standard_normal(7), rng.standard_normal((7, 1))
+        np.testing.assert_allclose(oracle_mod.npmap(x[None, :], W)[0], [np.linalg.norm(x)], rtol=1e-15)
 
 
 def test_topk_matches_sort(oracle_mod):
