@@ -142,3 +142,36 @@ def test_binding_fails_loudly_without_the_library(tmp_path):
     r = subprocess.run([sys.executable, "-c", "import linear_attention_still_b200.still"], cwd=tmp_path,
                        capture_output=True, text=True)
     assert r.returncode != 0 and "libstill.so is not built" in r.stderr
+
+
+@pytest.mark.parametrize("kw", [dict(), dict(dtype="f32"), dict(d=128, D=128, w=256, C=128, k=32, N=1300),
+                                dict(N=50), dict(w=0, k=0), dict(N=1)])
+def test_workspace_segments_hold_the_documented_tensors(lib, kw):
+    """Every segment of still_prefill_workspace_layout is 256-byte aligned, segments follow each
+    other without overlap, and each is at least as large as the tensor the header documents for
+    it (sizes restated here from the header's shapes)."""
+    d = _dims(lib, **kw)
+    L = lib.still_prefill_workspace_layout(d)
+    B, H, Hkv, N, hd, D, C, k = d.B, d.H, d.Hkv, d.N, d.d, d.D, d.C, d.k
+    T = N // C
+    es = 2 if d.dtype == 1 else 4
+    need = {"r": B * Hkv * N * 4, "idx": B * Hkv * T * k * 4, "khat": B * Hkv * T * k * hd * es,
+            "vhat": B * Hkv * T * k * hd * es, "S": B * Hkv * (T + 1) * D * hd * 4,
+            "z": B * Hkv * (T + 1) * D * 4}
+    order = ["r", "idx", "khat", "vhat", "S", "z", "phik", "sig", "lse", "fix", "wqt", "wkt", "st", "total"]
+    for a, b in zip(order, order[1:]):
+        assert L[a] % 256 == 0 and L[a] <= L[b], (a, b)
+        if a in need:
+            assert L[b] - L[a] >= need[a], a
+    if d.dtype == 1:  # bf16 path: per-head scores and the tensor-core operands
+        assert L["lse"] - L["sig"] >= B * H * N * 4
+        assert L["wqt"] - L["fix"] >= 256 + B * H * N * 4
+        assert L["wkt"] - L["wqt"] >= H * D * hd * 2
+        assert L["total"] - L["st"] >= B * Hkv * (T + 1) * hd * D * 2
+    assert L["total"] == lib.still_prefill_workspace_bytes(d)
+    bw = lib.still_backward_workspace_bytes(d)
+    if d.w > 0:
+        # phik, S, z, A, D, dYq, R, r, dYk, Ms, 1/Z (fp32)
+        floats = (B * Hkv * N * D + 2 * B * Hkv * (T + 1) * (D * hd + D) + B * H * N * (2 * D + 3)
+                  + B * Hkv * N * D)
+        assert bw >= floats * 4
