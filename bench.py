@@ -89,6 +89,30 @@ def merge_flops(shape):
     return rows * (4 * shape.d * int(soft_sizes(shape).sum()) + shape.N * (4 * shape.d * shape.D + 2 * shape.D))
 
 
+EX2_PER_CLOCK_PER_SM = 16  # ex2.approx: one warp instruction per 8 cycles on each of the 4 SMSPs (microbenchmarked)
+
+
+def merge_exps(shape):
+    """Exponentials of the merge kernel per step: one per (query-head, softmax key)."""
+    return shape.B * shape.H * int(soft_sizes(shape).sum())
+
+
+def exp_pipe_diag(shape, merge_ms_per_step, clocks=None, sms: int = 148):
+    """The merge's exponential rate against the MUFU ceiling (EX2_PER_CLOCK_PER_SM x SMs x the median
+    SM clock seen during the timed region, else the 1965 MHz maximum): a diagnostic beside the
+    tensor roofline, the tighter of the two at d = 64.  None without a merge time."""
+    if not merge_ms_per_step:
+        return None
+    mhz = (clocks or {}).get("sm_mhz") or 1965.0
+    peak = EX2_PER_CLOCK_PER_SM * sms * mhz * 1e6
+    exps = merge_exps(shape)
+    achieved = exps / (merge_ms_per_step / 1e3)
+    flop_s = merge_flops(shape) / (merge_ms_per_step / 1e3)
+    return {"exps_per_step": exps, "achieved": achieved, "peak": peak, "unit": "ex2/s", "frac": achieved / peak,
+            "sm_mhz": mhz, "sms": sms, "ms_at_exp_peak": exps / peak * 1e3,
+            "flops_per_exp": merge_flops(shape) / max(exps, 1), "achieved_tflops": flop_s / 1e12}
+
+
 def layer_flops(shape):
     """Algorithmic FLOPs of one whole step (all kernels)."""
     import numpy as np
@@ -500,6 +524,8 @@ def run_ours(args):
         "kernel_ms_per_step": {k_: v_[0] / args.steps for k_, v_ in kern.items() if v_[1]},
         "layer_tflops": layer_flops(shape) / (ms_per_step / 1e3) / 1e12, "device_status": status,
         "memory": memory,
+        "exp_pipe": exp_pipe_diag(shape, roofline["ms_per_step"], clocks,
+                                  torch.cuda.get_device_properties(local).multi_processor_count),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, t, desc, nth = oracle_sample(shape, args.cpu_seconds, router=args.router)

@@ -1,5 +1,5 @@
-"""CPU checks of bench.py's measurement arithmetic: the softmax-set sizes behind the merge FLOP count
-and the decode bytes per step against the oracle's own routing sets, the --keep shapes, and the
+"""CPU checks of bench.py's measurement arithmetic: the softmax-set sizes behind the merge FLOP and
+exponential counts and the decode bytes per step against the oracle's own routing sets, the --keep shapes, and the
 traffic lookup from a profile summary (used only while the kernel sources match its hashes)."""
 import hashlib
 import os
@@ -31,6 +31,22 @@ def test_soft_set_sizes_and_merge_flops(shape):
     np.testing.assert_array_equal(bench.soft_sizes(shape), sizes)
     want = shape.B * shape.H * sum(4 * shape.d * n + 4 * shape.d * shape.D + 2 * shape.D for n in sizes)
     assert bench.merge_flops(shape) == want
+    assert bench.merge_exps(shape) == shape.B * shape.H * int(sizes.sum())
+
+
+def test_exp_pipe_diagnostic():
+    shape = Shape(B=1, H=32, Hkv=8, N=16384, d=64, D=64, w=512, C=512, k=64)
+    assert bench.exp_pipe_diag(shape, None) is None
+    diag = bench.exp_pipe_diag(shape, 0.5, {"sm_mhz": 1000.0}, sms=100)
+    assert diag["peak"] == 16 * 100 * 1000.0 * 1e6
+    assert diag["achieved"] == pytest.approx(bench.merge_exps(shape) / 0.5e-3)
+    assert diag["frac"] == pytest.approx(diag["achieved"] / diag["peak"])
+    assert diag["flops_per_exp"] > 4 * shape.d  # 4d per pair plus the per-row linear-branch terms
+    # without a clock record the maximum clock is assumed; at d = 64 the exponentials take longer
+    # than the tensor work at the measured bf16 peak
+    d2 = bench.exp_pipe_diag(shape, 0.5, None)
+    assert d2["sm_mhz"] == 1965.0
+    assert d2["ms_at_exp_peak"] > bench.merge_flops(shape) / 1653.3e12 * 1e3
 
 
 def test_decode_bytes_count_the_softmax_rows():
