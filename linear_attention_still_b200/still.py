@@ -90,11 +90,34 @@ def dims_of(shape, N: int | None = None) -> still_dims:
 
 
 def _ptr(x):
+    """Address of a host-or-device operand (a tensor or a raw address)."""
     if x is None:
         return None
     if isinstance(x, int):
         return x
     return x.data_ptr()
+
+
+def _dptr(x, name: str = "operand"):
+    """Address of a device operand.  A raw int is passed as given; a tensor must be a contiguous CUDA
+    tensor on the current device -- the library takes no strides, and a host address or another
+    device's memory handed to a kernel would be read as if it were this device's."""
+    if x is None or isinstance(x, int):
+        return x
+    import torch
+    if not x.is_cuda:
+        raise ValueError(f"{name}: expected a CUDA tensor, got one on {x.device}")
+    if x.get_device() != torch.cuda.current_device():
+        raise ValueError(f"{name}: tensor on cuda:{x.get_device()}, current device is "
+                         f"cuda:{torch.cuda.current_device()}")
+    if not x.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous tensor (the library takes no strides)")
+    return x.data_ptr()
+
+
+def _dargs(**operands) -> list:
+    """_dptr of each keyword argument, in the order given."""
+    return [_dptr(x, name) for name, x in operands.items()]
 
 
 def _stream(stream):
@@ -116,22 +139,21 @@ def status_string(status: int) -> str:
 
 
 def still_saliency(dims, q, k, r_kv, r_q=None, stream=None):
-    _ok("still_saliency", _lib.still_saliency(ct.byref(dims), _ptr(q), _ptr(k), _ptr(r_kv), _ptr(r_q),
-                                              _stream(stream)))
+    _ok("still_saliency", _lib.still_saliency(ct.byref(dims), *_dargs(q=q, k=k, r_kv=r_kv, r_q=r_q), _stream(stream)))
 
 
 def still_select_topk(dims, r_kv, idx, stream=None):
-    _ok("still_select_topk", _lib.still_select_topk(ct.byref(dims), _ptr(r_kv), _ptr(idx), _stream(stream)))
+    _ok("still_select_topk", _lib.still_select_topk(ct.byref(dims), *_dargs(r_kv=r_kv, idx=idx), _stream(stream)))
 
 
 def still_diagonal_score(dims, q, k, r_kv, stream=None):
     _ok("still_diagonal_score",
-        _lib.still_diagonal_score(ct.byref(dims), _ptr(q), _ptr(k), _ptr(r_kv), _stream(stream)))
+        _lib.still_diagonal_score(ct.byref(dims), *_dargs(q=q, k=k, r_kv=r_kv), _stream(stream)))
 
 
 def still_npmap(B, Hx, N, d, D, dtype, x, W, phi, stream=None):
     dt = {"bf16": STILL_BF16, "f32": STILL_F32}[dtype] if isinstance(dtype, str) else int(dtype)
-    _ok("still_npmap", _lib.still_npmap(B, Hx, N, d, D, dt, _ptr(x), _ptr(W), _ptr(phi), _stream(stream)))
+    _ok("still_npmap", _lib.still_npmap(B, Hx, N, d, D, dt, *_dargs(x=x, W=W, phi=phi), _stream(stream)))
 
 
 def still_prefill_workspace_bytes(dims) -> int:
@@ -148,10 +170,10 @@ def still_hybrid_prefill(dims, q, k, v, wq, wk, o, idx_in=None, workspace=None, 
                          state_capacity=0, stream=None):
     if workspace_bytes is None:
         workspace_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    a = _dargs(q=q, k=k, v=v, wq=wq, wk=wk, o=o, idx_in=idx_in, workspace=workspace, state=state)
     _ok("still_hybrid_prefill",
-        _lib.still_hybrid_prefill(ct.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(wq), _ptr(wk), _ptr(o),
-                                  _ptr(idx_in), _ptr(workspace), int(workspace_bytes), _ptr(state),
-                                  int(state_capacity), _stream(stream)))
+        _lib.still_hybrid_prefill(ct.byref(dims), *a[:8], int(workspace_bytes), a[8], int(state_capacity),
+                                  _stream(stream)))
 
 
 STATIC_WORKSPACE_BYTES = 64 << 20  # STILL_STATIC_WORKSPACE_BYTES
@@ -159,9 +181,9 @@ STATIC_WORKSPACE_BYTES = 64 << 20  # STILL_STATIC_WORKSPACE_BYTES
 
 def still_hybrid_prefill_static(dims, q, k, v, wq, wk, o, idx_in=None, state=None, state_capacity=0, stream=None):
     """still_hybrid_prefill with the library's fixed device scratch (allocates nothing)."""
+    a = _dargs(q=q, k=k, v=v, wq=wq, wk=wk, o=o, idx_in=idx_in, state=state)
     _ok("still_hybrid_prefill_static",
-        _lib.still_hybrid_prefill_static(ct.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(wq), _ptr(wk), _ptr(o),
-                                         _ptr(idx_in), _ptr(state), int(state_capacity), _stream(stream)))
+        _lib.still_hybrid_prefill_static(ct.byref(dims), *a, int(state_capacity), _stream(stream)))
 
 
 def still_backward_workspace_bytes(dims) -> int:
@@ -172,10 +194,10 @@ def still_hybrid_backward(dims, q, k, v, wq, wk, idx, do, dq, dk, dv, dwq, dwk, 
                           stream=None):
     if workspace_bytes is None:
         workspace_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    a = _dargs(q=q, k=k, v=v, wq=wq, wk=wk, idx=idx, do=do, dq=dq, dk=dk, dv=dv, dwq=dwq, dwk=dwk,
+               workspace=workspace)
     _ok("still_hybrid_backward",
-        _lib.still_hybrid_backward(ct.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(wq), _ptr(wk), _ptr(idx), _ptr(do),
-                                   _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dwq), _ptr(dwk), _ptr(workspace),
-                                   int(workspace_bytes), _stream(stream)))
+        _lib.still_hybrid_backward(ct.byref(dims), *a, int(workspace_bytes), _stream(stream)))
 
 
 def still_decode_state_bytes(dims, capacity: int) -> int:
@@ -183,13 +205,15 @@ def still_decode_state_bytes(dims, capacity: int) -> int:
 
 
 def still_decode_init(dims, capacity, state, stream=None):
-    _ok("still_decode_init", _lib.still_decode_init(ct.byref(dims), int(capacity), _ptr(state), _stream(stream)))
+    _ok("still_decode_init", _lib.still_decode_init(ct.byref(dims), int(capacity), *_dargs(state=state),
+                                                    _stream(stream)))
 
 
 def still_decode_step(dims, state, capacity, pos, wq, wk, q_t, k_t, v_t, o_t, stream=None):
+    (st,) = _dargs(state=state)
     _ok("still_decode_step",
-        _lib.still_decode_step(ct.byref(dims), _ptr(state), int(capacity), int(pos), _ptr(wq), _ptr(wk), _ptr(q_t),
-                               _ptr(k_t), _ptr(v_t), _ptr(o_t), _stream(stream)))
+        _lib.still_decode_step(ct.byref(dims), st, int(capacity), int(pos),
+                               *_dargs(wq=wq, wk=wk, q_t=q_t, k_t=k_t, v_t=v_t, o_t=o_t), _stream(stream)))
 
 
 def still_get_device_status(stream=None) -> int:

@@ -175,3 +175,28 @@ def test_workspace_segments_hold_the_documented_tensors(lib, kw):
         floats = (B * Hkv * N * D + 2 * B * Hkv * (T + 1) * (D * hd + D) + B * H * N * (2 * D + 3)
                   + B * Hkv * N * D)
         assert bw >= floats * 4
+
+
+def test_binding_refuses_host_tensors_before_calling_the_library(lib):
+    """The binding hands the library bare addresses, so it refuses tensors that are not on the GPU
+    (a host address read by a kernel would fault) -- before any library call, so no GPU is needed."""
+    import torch
+    d = _dims(lib)
+    host = torch.zeros(1, 4, 300, 64, dtype=torch.bfloat16)
+    r = torch.zeros(1, 2, 300)
+    with pytest.raises(ValueError, match="q: expected a CUDA tensor"):
+        lib.still_saliency(d, host, FAKE, r)
+    with pytest.raises(ValueError, match="r_kv: expected a CUDA tensor"):
+        lib.still_diagonal_score(d, FAKE, FAKE, r)
+    with pytest.raises(ValueError, match="workspace: expected a CUDA tensor"):
+        lib.still_hybrid_prefill(d, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, workspace=torch.zeros(256, dtype=torch.uint8))
+    with pytest.raises(ValueError, match="state: expected a CUDA tensor"):
+        lib.still_decode_step(d, torch.zeros(16, dtype=torch.uint8), 64, 0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE)
+    with pytest.raises(ValueError, match="o_t: expected a CUDA tensor"):
+        lib.still_decode_step(d, FAKE, 64, 0, FAKE, FAKE, FAKE, FAKE, FAKE, torch.zeros(4, 64))
+    with pytest.raises(ValueError, match="dwk: expected a CUDA tensor"):
+        lib.still_hybrid_backward(d, *([FAKE] * 11), torch.zeros(2, 64, 64), workspace=FAKE, workspace_bytes=1 << 30)
+    # raw addresses (and a raw stream handle) pass through unchanged: the library's own validation answers
+    with pytest.raises(lib.StillError, match="INVALID_ARG"):
+        lib.still_saliency(lib.make_dims(B=1, H=4, Hkv=2, N=300, d=64, D=64, w=0, C=64, k=0), FAKE, FAKE, FAKE,
+                           stream=0)
