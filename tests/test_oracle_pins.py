@@ -104,6 +104,28 @@ def test_saliency_golden(oracle_mod):
             assert sigma[0, 0, i] == pytest.approx(want, rel=1e-9), (c["name"], i)
 
 
+def test_merge_golden(oracle_mod):
+    """Hand-derived outputs of a six-token layer (tests/golden/merge_hand.json): kept token, window,
+    linear branch over the unkept token of the one decided chunk, one normaliser; for both oracles."""
+    from oracle import brute
+    with open(os.path.join(GOLDEN, "merge_hand.json")) as f:
+        c = json.load(f)
+    dm, x = c["dims"], c["inputs"]
+    N, H = dm["N"], dm["H"]
+    q = np.array(x["q"], dtype=np.float64).reshape(1, H, N, 1)
+    k = np.array(x["k"], dtype=np.float64).reshape(1, 1, N, 1)
+    v = np.array(x["v"], dtype=np.float64).reshape(1, 1, N, 1)
+    wq = np.array(x["wq"], dtype=np.float64).reshape(H, 1, 1)
+    wk = np.array(x["wk"], dtype=np.float64).reshape(1, 1, 1)
+    idx = np.array(x["idx"], dtype=np.int32).reshape(1, 1, -1, 1)
+    dims = oracle_mod.Dims(1, H, 1, N, 1, 1, dm["w"], dm["C"], dm["k"], scale=dm["scale"])
+    o = oracle_mod.prefill(dims, q, k, v, wq, wk, idx_in=idx)["o"]
+    ob, _, _ = brute.layer(q, k, v, wq, wk, dm["w"], dm["C"], dm["k"], scale=dm["scale"], idx_in=idx)
+    for e in c["expected"]:
+        assert o[0, e["h"], e["i"], 0] == pytest.approx(e["o"], rel=1e-12), e
+        assert ob[0, e["h"], e["i"], 0] == pytest.approx(e["o"], rel=1e-12), e
+
+
 # ---------------------------------------------------------------- top-k
 
 # ---------------------------------------------------------------- diagonal-only router
