@@ -54,10 +54,12 @@ def parse():
     p.add_argument("--cpu-seconds", type=float, default=15.0, help="target oracle time of the CPU baseline")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--e2e-steps", type=int, default=10)
-    p.add_argument("--keep", choices=["config", "all", "none"], default="config",
+    p.add_argument("--keep", choices=["config", "all", "none", "window"], default="config",
                    help="tokens kept per chunk: the workload's k, all of them (k = C: exact causal softmax "
-                        "attention through the same kernels, a same-box dense comparator), or none (k = 0: "
-                        "window + linear branch only)")
+                        "attention through the same kernels, a same-box dense comparator), none (k = 0: "
+                        "window + linear branch only), or window (k = 0 with a window of the whole sequence: "
+                        "exact causal softmax attention in the window phase alone, flash-style, with no "
+                        "selection, kept cache or linear state)")
     p.add_argument("--pass", dest="pass_", choices=["forward", "backward"], default="forward",
                    help="prefill workloads: time the forward layer (default) or its backward pass "
                         "(gradients of q, k, v, Wq, Wk with the selection held fixed)")
@@ -350,6 +352,8 @@ def workload_shape(args):
         shape = shape.replace(k=shape.C)
     elif keep == "none":
         shape = shape.replace(k=0)
+    elif keep == "window":
+        shape = shape.replace(k=0, w=-(-shape.N // shape.C) * shape.C)
     return shape
 
 

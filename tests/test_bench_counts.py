@@ -70,6 +70,12 @@ def test_keep_shapes():
     assert bench.workload_shape(A).k == 0
     A.keep = "config"
     assert bench.workload_shape(A).k == 64
+    A.keep = "window"  # every query's window reaches token 0: exact causal softmax attention, no selection
+    s = bench.workload_shape(A)
+    assert s.k == 0 and s.w % s.C == 0 and s.w >= s.N
+    assert (bench.soft_sizes(s) == np.arange(s.N) + 1).all()
+    assert bench.merge_flops(s) == bench.merge_flops(bench.workload_shape(type("B", (), {"workload": A.workload,
+                                                                                           "keep": "all"})))
 
 
 def test_traffic_lookup_follows_source_hashes(tmp_path, monkeypatch):
