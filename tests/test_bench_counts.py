@@ -92,3 +92,25 @@ def test_traffic_lookup_follows_source_hashes(tmp_path, monkeypatch):
     assert bench.profiled_traffic("other") is None
     (csrc / "a.cu").write_bytes(b"kernel two")  # the kernel changed since the capture
     assert bench.profiled_traffic("wl") is None
+
+
+def test_reference_arm_line(tmp_path):
+    """`bench.py --impl reference` on the small fp32 workload: one JSON line with the contract's keys,
+    the oracle's own throughput as value, cpu_baseline and e2e carrying the same number."""
+    import json
+    import subprocess
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
+                        "still_f32_b1_h2_n512", "--steps", "3", "--warmup", "1"],
+                       capture_output=True, text=True, timeout=600, cwd=tmp_path)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "higher_is_better", "scaling", "vs_baseline",
+                "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["steps"] == 3 and line["warmup"] == 1
+    assert line["value"] > 0 and line["cpu_baseline"]["value"] == line["value"] == line["e2e"]["value"]
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+    assert line["config"]["workload"] == "still_f32_b1_h2_n512"
