@@ -105,25 +105,34 @@ def test_saliency_golden(oracle_mod):
 
 
 def test_merge_golden(oracle_mod):
-    """Hand-derived outputs of a six-token layer (tests/golden/merge_hand.json): kept token, window,
-    linear branch over the unkept token of the one decided chunk, one normaliser; for both oracles."""
+    """Hand-derived outputs of two six-token layers (tests/golden/merge_hand.json): kept token,
+    window, linear branch over the unkept token of the one decided chunk, one normaliser.  Checked
+    for the C oracle and the numpy brute force, and, where the case says so, for the decode state
+    machine run token by token (the chunk close at position 3 decides chunk 0 for positions 4, 5)."""
     from oracle import brute
     with open(os.path.join(GOLDEN, "merge_hand.json")) as f:
-        c = json.load(f)
-    dm, x = c["dims"], c["inputs"]
-    N, H = dm["N"], dm["H"]
-    q = np.array(x["q"], dtype=np.float64).reshape(1, H, N, 1)
-    k = np.array(x["k"], dtype=np.float64).reshape(1, 1, N, 1)
-    v = np.array(x["v"], dtype=np.float64).reshape(1, 1, N, 1)
-    wq = np.array(x["wq"], dtype=np.float64).reshape(H, 1, 1)
-    wk = np.array(x["wk"], dtype=np.float64).reshape(1, 1, 1)
-    idx = np.array(x["idx"], dtype=np.int32).reshape(1, 1, -1, 1)
-    dims = oracle_mod.Dims(1, H, 1, N, 1, 1, dm["w"], dm["C"], dm["k"], scale=dm["scale"])
-    o = oracle_mod.prefill(dims, q, k, v, wq, wk, idx_in=idx)["o"]
-    ob, _, _ = brute.layer(q, k, v, wq, wk, dm["w"], dm["C"], dm["k"], scale=dm["scale"], idx_in=idx)
-    for e in c["expected"]:
-        assert o[0, e["h"], e["i"], 0] == pytest.approx(e["o"], rel=1e-12), e
-        assert ob[0, e["h"], e["i"], 0] == pytest.approx(e["o"], rel=1e-12), e
+        cases = json.load(f)["cases"]
+    for c in cases:
+        dm, x = c["dims"], c["inputs"]
+        N, H = dm["N"], dm["H"]
+        q = np.array(x["q"], dtype=np.float64).reshape(1, H, N, 1)
+        k = np.array(x["k"], dtype=np.float64).reshape(1, 1, N, 1)
+        v = np.array(x["v"], dtype=np.float64).reshape(1, 1, N, 1)
+        wq = np.array(x["wq"], dtype=np.float64).reshape(H, 1, 1)
+        wk = np.array(x["wk"], dtype=np.float64).reshape(1, 1, 1)
+        idx = np.array(x["idx"], dtype=np.int32).reshape(1, 1, -1, 1) if "idx" in x else None
+        dims = oracle_mod.Dims(1, H, 1, N, 1, 1, dm["w"], dm["C"], dm["k"], scale=dm["scale"])
+        o = oracle_mod.prefill(dims, q, k, v, wq, wk, idx_in=idx)["o"]
+        ob, _, _ = brute.layer(q, k, v, wq, wk, dm["w"], dm["C"], dm["k"], scale=dm["scale"], idx_in=idx)
+        od = None
+        if c.get("decode"):
+            dec = oracle_mod.Decoder(dims, wq, wk)
+            od = np.stack([dec.step(q[:, :, t], k[:, :, t], v[:, :, t])[0] for t in range(N)], axis=2)
+        for e in c["expected"]:
+            assert o[0, e["h"], e["i"], 0] == pytest.approx(e["o"], rel=1e-12), (c["name"], e)
+            assert ob[0, e["h"], e["i"], 0] == pytest.approx(e["o"], rel=1e-12), (c["name"], e)
+            if od is not None:
+                assert od[0, e["h"], e["i"], 0] == pytest.approx(e["o"], rel=1e-12), (c["name"], e)
 
 
 # ---------------------------------------------------------------- top-k
