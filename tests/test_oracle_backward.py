@@ -74,3 +74,35 @@ def test_npmap_backward_matches_finite_differences():
             Wm[a, c] -= eps
             fd = (backward.npmap_forward(x, Wp) - backward.npmap_forward(x, Wm)) @ dphi / (2 * eps)
             assert abs(fd - dW[a, c]) < 1e-8 * max(1.0, abs(fd))
+
+
+def test_backward_golden():
+    """Hand-derived gradient of one output row (tests/golden/backward_hand.json) of the six-token
+    layer of tests/golden/merge_hand.json: dv = weight / Z, dk from e_j (v_j - o) / Z and the
+    linear token's |q| (v_0 - o) / Z, dq in closed form, and dWq = dWk = 0 because a one-feature
+    NP-Map is the norm."""
+    import json
+    import os
+    here = os.path.join(os.path.dirname(__file__), "golden")
+    with open(os.path.join(here, "backward_hand.json")) as f:
+        gold = json.load(f)
+    with open(os.path.join(here, "merge_hand.json")) as f:
+        case = next(c for c in json.load(f)["cases"] if c["name"] == gold["case"])
+    dm, x = case["dims"], case["inputs"]
+    N, H = dm["N"], dm["H"]
+    q = np.array(x["q"], dtype=np.float64).reshape(1, H, N, 1)
+    k = np.array(x["k"], dtype=np.float64).reshape(1, 1, N, 1)
+    v = np.array(x["v"], dtype=np.float64).reshape(1, 1, N, 1)
+    wq = np.array(x["wq"], dtype=np.float64).reshape(H, 1, 1)
+    wk = np.array(x["wk"], dtype=np.float64).reshape(1, 1, 1)
+    idx = np.array(x["idx"], dtype=np.int32).reshape(1, 1, -1, 1)
+    do = np.zeros_like(q)
+    up = gold["upstream"]
+    do[0, up["h"], up["i"], 0] = up["value"]
+    dq, dk, dv, dwq, dwk = backward.layer_backward(q, k, v, wq, wk, do, idx, dm["w"], dm["C"], scale=dm["scale"])
+    want_dq = np.zeros_like(q)
+    want_dq[0, gold["dq"]["h"], gold["dq"]["i"], 0] = gold["dq"]["value"]
+    np.testing.assert_allclose(dq, want_dq, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(dk[0, 0, :, 0], gold["dk"], rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(dv[0, 0, :, 0], gold["dv"], rtol=1e-12, atol=1e-14)
+    assert np.all(dwq == 0.0) and np.all(dwk == 0.0)
