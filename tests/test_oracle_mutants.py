@@ -1,9 +1,10 @@
 """The oracle's pins catch plausible mistakes: each mutant below is a copy of oracle/still_oracle.c
 with one such mistake planted (a dropped term, a wrong sign, index or direction, a transposed
 operand, an off-by-one chunk), built with gcc into a temporary library and run against the pins of
-tests/test_oracle_pins.py in a child process.  Every mutant must fail at least one pin, and the
+tests/test_oracle_pins.py in a child process; likewise copies of oracle/backward.py against the
+pins of tests/test_oracle_backward.py.  Every mutant must fail at least one pin, and the
 unmodified source, built and run the same way, must pass them all.  Nothing here touches the
-oracle's own build."""
+oracle's own files or build."""
 import os
 import subprocess
 import sys
@@ -94,3 +95,62 @@ def test_every_planted_mistake_fails_a_pin(tmp_path):
     assert rc == 0, "the unmodified oracle, built the same way, must pass every pin:\n" + out[-3000:]
     survivors = [name for name, (rc, _) in results.items() if rc != 1]
     assert not survivors, {name: (MUTANTS[name][0], results[name][1][-1500:]) for name in survivors}
+
+
+# name: (what the mistake is, text in oracle/backward.py, replacement)
+BACKWARD_MUTANTS = {
+    "ds_without_row_term": ("softmax logits: dL/ds without the - <g, o> term", "ds = p * (V[soft] @ gi - go)",
+                            "ds = p * (V[soft] @ gi)"),
+    "dk_without_scale": ("softmax keys: dk without the logit scale", "dk[b, g, soft] += tau * np.outer(ds, qi)",
+                         "dk[b, g, soft] += np.outer(ds, qi)"),
+    "dw_unshifted": ("linear weights: dL/dw without the shared shift", "dw = (V[lin] @ gi - go) * math.exp(-M) / Z",
+                     "dw = (V[lin] @ gi - go) / Z"),
+    "dv_linear_unnormalised": ("linear values: dv without 1/Z", "dv[b, g, lin] += np.outer(wl / Z, gi)",
+                               "dv[b, g, lin] += np.outer(wl, gi)"),
+    "linear_keys_dropped": ("linear keys: no gradient into phi(k)", "dphik[lin] += np.outer(dw, phiq)",
+                            "pass"),
+    "npmap_norm_term": ("NP-Map backward: the norm's own gradient dropped",
+                        "dx = W @ dy + (dn * x / n if n > 0 else 0.0)", "dx = W @ dy"),
+    # (Dropping the softmax Jacobian's mean term f.df would be no mistake here: the gradient that
+    # reaches f through u = f / ||f|| is orthogonal to f, so that term is zero.)
+    "npmap_projection": ("NP-Map backward: the normalisation's projection dropped",
+                         "df = (du - u * float(u @ du)) / nf", "df = du / nf"),
+    "npmap_dW_transposed": ("NP-Map backward: dW as the outer product the wrong way round", "dW = np.outer(x, dy)",
+                            "dW = np.outer(x, dy)[:, ::-1]"),
+}
+
+_BACKWARD_RUNNER = """
+import sys, types
+sys.path.insert(0, {root!r})
+import pytest
+import oracle
+mod = types.ModuleType("oracle.backward")
+mod.__file__ = {path!r}
+exec(compile(open({path!r}).read(), {path!r}, "exec"), mod.__dict__)
+sys.modules["oracle.backward"] = mod
+oracle.backward = mod
+sys.exit(pytest.main(["-q", "-x", "-p", "no:cacheprovider", {pins!r}]))
+"""
+
+
+def test_every_planted_backward_mistake_fails_a_pin(tmp_path):
+    src_path = os.path.join(ROOT, "oracle", "backward.py")
+    with open(src_path) as f:
+        original = f.read()
+    jobs = {"unmodified": original}
+    for name, (_, old, new) in BACKWARD_MUTANTS.items():
+        assert original.count(old) == 1, f"{name}: the mutated text must occur exactly once in backward.py"
+        jobs[name] = original.replace(old, new)
+    procs = {}
+    for name, source in jobs.items():
+        path = tmp_path / f"{name}.py"
+        path.write_text(source)
+        code = _BACKWARD_RUNNER.format(root=ROOT, path=str(path),
+                                       pins=os.path.join(ROOT, "tests", "test_oracle_backward.py"))
+        procs[name] = subprocess.Popen([sys.executable, "-c", code], cwd=str(tmp_path), stdout=subprocess.PIPE,
+                                       stderr=subprocess.STDOUT, text=True)
+    results = {name: (p.wait(timeout=900), p.stdout.read()) for name, p in procs.items()}
+    rc, out = results.pop("unmodified")
+    assert rc == 0, "the unmodified backward, loaded the same way, must pass every pin:\n" + out[-3000:]
+    survivors = [name for name, (rc, _) in results.items() if rc != 1]
+    assert not survivors, {name: (BACKWARD_MUTANTS[name][0], results[name][1][-1500:]) for name in survivors}
