@@ -555,11 +555,17 @@ def decode_step_bytes(shape, pos: int) -> int:
     return shape.B * shape.Hkv * per_bg + shape.B * shape.H * 2 * shape.d * es
 
 
+def _causal_pairs(n: int) -> float:
+    """(query, key) pairs of n causal rows, keys up to and including the row itself."""
+    return n * (n + 1) / 2.0
+
+
 def oracle_backward_sample(shape, seconds: float):
     """fp64 oracle backward (oracle/backward.py, one process) on the first n tokens of one (batch,
     KV group) slice, n grown once per process until about `seconds` are spent, scaled to the layer by
-    the ratio of softmax (query, key) pairs, which dominate the work.  Returns (tokens/s, seconds,
-    description, threads)."""
+    the ratio of causal (query, key) pairs n(n+1)/2: the numpy oracle visits every earlier token of
+    a row once, in its softmax or its linear set, at about the same cost either way.  Returns
+    (tokens/s, seconds, description, threads)."""
     import numpy as np
 
     from oracle import backward
@@ -594,19 +600,18 @@ def oracle_backward_sample(shape, seconds: float):
         spent = t_last
         while n < shape.N:
             n2 = min(shape.N, n * 2)
-            t_next = t_last * float(soft_sizes(shape, n2).sum()) / max(float(soft_sizes(shape, n).sum()), 1.0)
+            t_next = t_last * _causal_pairs(n2) / _causal_pairs(n)
             if spent + t_next > seconds:
                 break
             n = n2
             t_last = run(n)
             spent += t_last
         _ORACLE_CACHE[key] = n
-    pairs_sample = float(soft_sizes(shape, n).sum())
-    pairs_full = float(soft_sizes(shape).sum()) * shape.B * shape.Hkv
-    t_layer = t_last * pairs_full / max(pairs_sample, 1.0)
+    scale = _causal_pairs(shape.N) / _causal_pairs(n) * shape.B * shape.Hkv
+    t_layer = t_last * scale
     desc = (f"oracle backward fp64 (numpy, 1 process) on the first {n} tokens of one (batch, KV group) slice "
-            f"of {shape.G} heads ({t_last:.1f} s), scaled by softmax (query, key) pairs to the layer "
-            f"(x{pairs_full / max(pairs_sample, 1.0):.0f})")
+            f"of {shape.G} heads ({t_last:.1f} s), scaled to the layer by causal (query, key) pairs "
+            f"(x{scale:.0f})")
     return shape.B * shape.N / t_layer, t_last, desc, 1
 
 
