@@ -27,7 +27,12 @@
  *    width D, window w, chunk C, k tokens kept per full chunk.  The window is
  *    a whole number of chunks, w = m*C with m >= 1, or w = 0 (no window: pure
  *    linear attention, then k must be 0).  0 <= k <= C.  N is arbitrary; a
- *    trailing partial chunk is never selected from.
+ *    trailing partial chunk is never selected from.  d and D are multiples
+ *    of 8 (at least 8); scale is finite and >= 0; B, N >= 0; H, Hkv, C >= 1
+ *    (STILL_ERR_INVALID_ARG otherwise).  Limits of this implementation
+ *    (STILL_ERR_UNSUPPORTED beyond them): d, D <= 256; H/Hkv <= 32;
+ *    C <= 16384; B*H <= 65535; N <= 2^26.  The size queries return 0 for
+ *    dims that either check rejects.
  *  - dtype applies to q, k, v, o, Wq, Wk; scores, features and linear states
  *    are always fp32.
  */
