@@ -224,6 +224,19 @@ def _cached_inputs(shape, b: int):
     return _ORACLE_CACHE[key]
 
 
+def _row_runs(N: int, m: int):
+    """m positions of [0, N) (m a multiple of min(64, m), m <= N) in runs of up to 64 consecutive
+    ones whose centres are spread evenly: the oracle then walks them head-major with the position
+    fastest, as it walks a whole slice, so each thread keeps reusing the prefix it just read; the
+    mean position is (N - 1) / 2 up to rounding, so a cost linear in the position is estimated
+    without bias."""
+    import numpy as np
+    run = min(64, m)
+    nrun = m // run
+    starts = ((np.arange(nrun) + 0.5) * (N / nrun) - run / 2).astype(np.int64).clip(0, N - run)
+    return (starts[:, None] + np.arange(run)[None, :]).reshape(-1)
+
+
 def oracle_sample(shape, seconds: float, nthreads: int | None = None, router: str = "saliency"):
     """Time the fp64 oracle on one (batch, KV group) slice of G heads over the whole sequence: the
     score and per-chunk top-k of every token, the NP-Map of every key, and the output rows of m
@@ -253,17 +266,8 @@ def oracle_sample(shape, seconds: float, nthreads: int | None = None, router: st
         idx = oracle.topk(d, r)
         return idx, time.perf_counter() - t0
 
-    def positions(m):
-        """m positions in runs of up to 64 consecutive ones, the runs' centres spread evenly over
-        [0, N): the oracle then walks them head-major with the position fastest, as it walks the
-        whole slice, so each thread keeps reusing the prefix it just read."""
-        run = min(64, m)
-        nrun = m // run
-        starts = ((np.arange(nrun) + 0.5) * (N / nrun) - run / 2).astype(np.int64).clip(0, N - run)
-        return (starts[:, None] + np.arange(run)[None, :]).reshape(-1)
-
     def rows_call(idx, m):
-        pos = positions(m)
+        pos = _row_runs(N, m)
         rows = np.array([(0, h, int(p_)) for h in range(G) for p_ in pos], dtype=np.int32)
         t0 = time.perf_counter()
         oracle.prefill(d, q, k, v, wq, wk, idx_in=idx, rows=rows, nthreads=nth)

@@ -114,3 +114,21 @@ def test_reference_arm_line(tmp_path):
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
     assert line["config"]["workload"] == "still_f32_b1_h2_n512"
+
+
+@pytest.mark.parametrize("N,m", [(16384, 64), (16384, 704), (16384, 4352), (16384, 16384), (512, 512),
+                                 (65536, 128), (1000, 640)])
+def test_row_runs_are_an_unbiased_position_sample(N, m):
+    """The CPU baseline's row sample: m distinct positions of [0, N) in runs of 64 consecutive ones,
+    with mean position (N - 1)/2 up to one run's rounding, so a per-row cost linear in the position
+    sums to the whole slice's when scaled by N/m."""
+    pos = bench._row_runs(N, m)
+    assert len(pos) == m and len(set(pos.tolist())) == m
+    assert pos.min() >= 0 and pos.max() < N
+    run = min(64, m)
+    runs = pos.reshape(-1, run)
+    assert (np.diff(runs, axis=1) == 1).all()
+    assert abs(pos.mean() - (N - 1) / 2) <= max(1.0, 0.01 * N)
+    cost = lambda p: 3.0 + 0.5 * p  # noqa: E731  (constant plus a term linear in the position)
+    full = cost(np.arange(N)).sum()
+    assert cost(pos).sum() * N / m == pytest.approx(full, rel=0.01)
