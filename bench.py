@@ -242,10 +242,12 @@ def oracle_sample(shape, seconds: float, nthreads: int | None = None, router: st
     score and per-chunk top-k of every token, the NP-Map of every key, and the output rows of m
     positions spread evenly over [0, N) (all G heads each).  A row's cost in the oracle is a constant
     plus a term linear in its position (its linear branch and softmax set are built over its whole
-    prefix), so the evenly spread rows scaled by N/m estimate all N rows without a fitted model; m is
-    sized once per process and budget so that a step takes about `seconds`, and the selection is
-    re-timed every step unless it alone takes half the budget.  Returns (tokens/s, seconds measured,
-    description, threads)."""
+    prefix), so the evenly spread rows scaled by N/m estimate all N rows without a fitted model.  The
+    selection and the keys' NP-Map are each timed in full, every step unless one alone takes a
+    quarter of the budget (then once per process); the rows call gets the keys' features ready-made,
+    its fixed cost (routing masks, output buffer) and its cost per position are calibrated once per
+    process, and m is sized from them so that a step takes about `seconds`.  Returns (tokens/s,
+    seconds measured, description, threads)."""
     import numpy as np
 
     import oracle
@@ -266,43 +268,49 @@ def oracle_sample(shape, seconds: float, nthreads: int | None = None, router: st
         idx = oracle.topk(d, r)
         return idx, time.perf_counter() - t0
 
-    def rows_call(idx, m):
+    def features():
+        t0 = time.perf_counter()
+        phik = oracle.npmap(k[0, 0], wk[0])[None, None]
+        return phik, time.perf_counter() - t0
+
+    def timed(key, fn):
+        """fn() timed this step, or its result and time from an earlier step when it is costly."""
+        if key in _ORACLE_CACHE and _ORACLE_CACHE[key][1] > 0.25 * seconds:
+            return _ORACLE_CACHE[key][0], _ORACLE_CACHE[key][1], False
+        _ORACLE_CACHE[key] = fn()
+        return _ORACLE_CACHE[key][0], _ORACLE_CACHE[key][1], True
+
+    def rows_call(idx, phik, m):
         pos = _row_runs(N, m)
         rows = np.array([(0, h, int(p_)) for h in range(G) for p_ in pos], dtype=np.int32)
         t0 = time.perf_counter()
-        oracle.prefill(d, q, k, v, wq, wk, idx_in=idx, rows=rows, nthreads=nth)
+        oracle.prefill(d, q, k, v, wq, None, idx_in=idx, rows=rows, nthreads=nth, phik=phik)
         return time.perf_counter() - t0
 
-    sel_key = ("selection", shape, router, nth)
-    if not selects:
-        idx, t_sel = None, 0.0
-    elif sel_key in _ORACLE_CACHE and _ORACLE_CACHE[sel_key][1] > 0.5 * seconds:
-        idx, t_sel = _ORACLE_CACHE[sel_key]  # timed on an earlier step
-    else:
-        idx, t_sel = select()
-        _ORACLE_CACHE[sel_key] = (idx, t_sel)
+    idx, t_sel, sel_now = timed(("selection", shape, router, nth), select) if selects else (None, 0.0, False)
+    phik, t_phi, phi_now = timed(("features", shape), features)
     cal_key = ("rows", shape, router, nth)
     if cal_key not in _ORACLE_CACHE:  # once per process: the fixed cost of a call and the cost per position
-        t_setup = min(rows_call(idx, 1) for _ in range(3))  # the slice's NP-Map and routing, one position
+        t_call = min(rows_call(idx, phik, 1) for _ in range(3))
         m0 = min(N, 64)
         while True:  # grow the calibration sample until its rows outweigh the fixed cost
-            t = rows_call(idx, m0)
-            if m0 >= N or t - t_setup >= max(0.1, t_setup):
+            t = rows_call(idx, phik, m0)
+            if m0 >= N or t - t_call >= max(0.1, t_call):
                 break
             m0 = min(N, 2 * m0)
-        _ORACLE_CACHE[cal_key] = (t_setup, m0, max(t - t_setup, 1e-9) / m0)
-    t_setup, m0, per_pos = _ORACLE_CACHE[cal_key]
-    t_sel_step = t_sel if selects and _ORACLE_CACHE[sel_key][1] <= 0.5 * seconds else 0.0
-    m = int(min(N, max(m0, (seconds - t_sel_step - t_setup) / per_pos)))
+        _ORACLE_CACHE[cal_key] = (t_call, m0, max(t - t_call, 1e-9) / m0)
+    t_call, m0, per_pos = _ORACLE_CACHE[cal_key]
+    left = seconds - (t_sel if sel_now else 0.0) - (t_phi if phi_now else 0.0) - t_call
+    m = int(min(N, max(m0, left / per_pos)))
     m = N if m >= N else max(1, m // min(64, m)) * min(64, m)  # whole runs of 64
-    t_rows = rows_call(idx, m)
-    t_slice = t_sel + t_setup + max(t_rows - t_setup, 0.0) * N / m
+    t_rows = rows_call(idx, phik, m)
+    t_slice = t_sel + t_phi + t_call + max(t_rows - t_call, 0.0) * N / m
     t_layer = t_slice * shape.B * shape.Hkv
     desc = (f"oracle fp64 on one (batch, KV group) slice of {G} heads and {N} tokens: {router} score + "
-            f"top-k of every token ({t_sel:.2f} s), NP-Map of every key and routing ({t_setup:.2f} s, "
-            f"calibrated), output rows of {m} positions in evenly spread runs x {G} heads ({t_rows - t_setup:.2f} s, "
-            f"scaled x{N / m:.1f} to all positions); times {shape.B * shape.Hkv} slices")
-    return shape.B * N / t_layer, t_sel + t_setup + t_rows, desc, nth
+            f"top-k of every token ({t_sel:.2f} s), NP-Map of every key ({t_phi:.2f} s), output rows of {m} "
+            f"positions in evenly spread runs x {G} heads ({t_rows - t_call:.2f} s, scaled x{N / m:.1f} to all "
+            f"positions, plus the call's own {t_call:.2f} s); times {shape.B * shape.Hkv} slices")
+    return shape.B * N / t_layer, (t_sel if sel_now else 0.0) + (t_phi if phi_now else 0.0) + t_rows, desc, nth
 
 
 # ----------------------------------------------------------------------------- main arms
@@ -622,12 +630,12 @@ def oracle_backward_sample(shape, seconds: float):
 def oracle_decode_sample(shape, seconds: float):
     """fp64 oracle cost of decode rows: one (batch 0, KV group 0) slice of N + steps tokens, the output
     rows (G heads each) of m decode positions spread evenly over the decode steps, evaluated by the
-    same definition as a prefill row.  Every oracle call also maps every key of the slice through
-    the NP-Map, a fixed cost that a decode token does not carry: it is measured once per process
-    (the fastest of three one-position calls) and taken off.  The slice, its selection, that fixed
-    cost and the cost per position are set up once per process; m is sized to the budget (eight at
-    least).  Returns tokens/s of one sequence over all KV groups, seconds measured, description,
-    threads."""
+    same definition as a prefill row.  The slice, its selection and the NP-Map of its keys are set
+    up once per process and handed to every call (a decode token maps only its own key); the call's
+    remaining fixed cost (routing masks, output buffer) is measured once (the fastest of three
+    one-position calls) and taken off, and the cost per position calibrated with it; m is sized to
+    the budget (eight at least).  Returns tokens/s of one sequence over all KV groups, seconds
+    measured, description, threads."""
     import numpy as np
 
     import oracle
@@ -639,14 +647,15 @@ def oracle_decode_sample(shape, seconds: float):
         inp = make_inputs(shape.replace(B=1, H=shape.G, Hkv=1))
         d = oracle.Dims.of(full)
         _, r = oracle.saliency(d, inp.q, inp.k, nthreads=nth)
-        _ORACLE_CACHE[key] = [inp, d, oracle.topk(d, r), None]
-    inp, d, idx, cal = _ORACLE_CACHE[key]
+        phik = oracle.npmap(inp.k[0, 0], inp.wk[0])[None, None]
+        _ORACLE_CACHE[key] = [inp, d, oracle.topk(d, r), phik, None]
+    inp, d, idx, phik, cal = _ORACLE_CACHE[key]
 
     def run(m):
         pos = shape.N + (np.arange(m) + 0.5) * (shape.decode_steps / m)
         rows = np.array([(0, h, int(p_)) for h in range(shape.G) for p_ in pos], dtype=np.int32)
         t0 = time.perf_counter()
-        oracle.prefill(d, inp.q, inp.k, inp.v, inp.wq, inp.wk, idx_in=idx, rows=rows, nthreads=nth)
+        oracle.prefill(d, inp.q, inp.k, inp.v, inp.wq, None, idx_in=idx, rows=rows, nthreads=nth, phik=phik)
         return time.perf_counter() - t0
 
     if cal is None:
@@ -657,15 +666,15 @@ def oracle_decode_sample(shape, seconds: float):
             if m0 >= shape.decode_steps or t - t_fixed >= max(0.05, 0.5 * t_fixed):
                 break
             m0 = min(shape.decode_steps, 2 * m0)
-        cal = _ORACLE_CACHE[key][3] = (t_fixed, max(t - t_fixed, 1e-9) / m0)
+        cal = _ORACLE_CACHE[key][4] = (t_fixed, max(t - t_fixed, 1e-9) / m0)
     t_fixed, per_pos = cal
     m = int(min(shape.decode_steps, max(8, (seconds - t_fixed) / per_pos)))
     t_call = run(m)
     t_rows = max(t_call - t_fixed, 1e-9)
     per_token = t_rows / m * shape.Hkv  # one token of one sequence, every KV group
     desc = (f"oracle fp64: rows of {m} decode positions x {shape.G} heads of one KV group at context "
-            f"{shape.N} ({t_rows:.2f} s, after the call's fixed NP-Map cost of {t_fixed:.2f} s), scaled to "
-            f"all {shape.Hkv} KV groups")
+            f"{shape.N} ({t_rows:.2f} s, after the call's fixed {t_fixed:.2f} s; keys' NP-Map and selection "
+            f"prepared once), scaled to all {shape.Hkv} KV groups")
     return 1.0 / per_token, t_call, desc, nth
 
 

@@ -73,6 +73,8 @@ def _load():
         lib.od_diagonal_score.argtypes = [ct.POINTER(_ODims), P, P, P]
         lib.od_npmap.argtypes = [ct.c_int, ct.c_int, ct.c_int, P, P, P]
         lib.od_prefill.argtypes = [ct.POINTER(_ODims), P, P, P, P, P, P, P, P, P, P, ct.c_long, ct.c_int]
+        lib.od_prefill_given_phik.argtypes = [ct.POINTER(_ODims), P, P, P, P, P, P, P, P, P, P, ct.c_long,
+                                              ct.c_int]
         lib.od_linear_state.argtypes = [ct.POINTER(_ODims), P, P, P, P, ct.c_int, ct.c_int, ct.c_int, P, P]
         lib.od_decode_new.argtypes = [ct.POINTER(_ODims), P, P]
         lib.od_decode_new.restype = ct.c_void_p
@@ -148,21 +150,31 @@ def npmap(x, W) -> np.ndarray:
     return phi
 
 
-def prefill(dims: Dims, q, k, v, wq, wk, idx_in=None, rows=None, nthreads: int | None = None):
+def prefill(dims: Dims, q, k, v, wq, wk, idx_in=None, rows=None, nthreads: int | None = None, phik=None):
     """Full forward.  Returns dict(o=[B,H,N,d] (NaN where not computed), r, idx).
 
     idx_in [B,Hkv,T,k] injects the selection; rows [n,3] of (b,h,i) limits the
-    output rows computed."""
+    output rows computed; phik [B,Hkv,N,D] (as npmap computes it for every key
+    with its group's Wk) is used instead of computing phi(k) again (wk is then
+    not read)."""
     lib = _load()
-    q, k, v, wq, wk = map(_f64, (q, k, v, wq, wk))
+    q, k, v, wq = map(_f64, (q, k, v, wq))
     o = np.full((dims.B, dims.H, dims.N, dims.d), np.nan)
     r = np.full((dims.B, dims.Hkv, dims.N), np.nan)
     idx = np.zeros((dims.B, dims.Hkv, dims.T, dims.k), dtype=np.int32)
     ii = None if idx_in is None else _i32(idx_in)
     rr = None if rows is None else _i32(rows)
     nrows = 0 if rr is None else rr.shape[0]
-    rc = lib.od_prefill(ct.byref(dims.c()), _p(q), _p(k), _p(v), _p(wq), _p(wk), _p(ii), _p(o), _p(r), _p(idx),
-                        _p(rr), nrows, _nthreads(nthreads))
+    if phik is None:
+        wk = _f64(wk)
+        rc = lib.od_prefill(ct.byref(dims.c()), _p(q), _p(k), _p(v), _p(wq), _p(wk), _p(ii), _p(o), _p(r),
+                            _p(idx), _p(rr), nrows, _nthreads(nthreads))
+    else:
+        phik = _f64(phik)
+        if phik.shape != (dims.B, dims.Hkv, dims.N, dims.D):
+            raise ValueError(f"phik has shape {phik.shape}, expected {(dims.B, dims.Hkv, dims.N, dims.D)}")
+        rc = lib.od_prefill_given_phik(ct.byref(dims.c()), _p(q), _p(k), _p(v), _p(wq), _p(phik), _p(ii), _p(o),
+                                       _p(r), _p(idx), _p(rr), nrows, _nthreads(nthreads))
     _check(rc, "prefill")
     return {"o": o, "r": r, "idx": idx}
 

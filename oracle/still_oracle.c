@@ -497,33 +497,53 @@ static int od_selection(const od_dims *s, const double *q, const double *k, cons
  * Full layer forward.  idx_in (nullable) injects the per-chunk selection
  * instead of computing it; r_out / idx_out (nullable) return the scores and
  * the selection; rows (nullable) restricts the output to nrows (b,h,i)
- * triples.
+ * triples.  phik_in (nullable) supplies phi(k) [B,Hkv,N,D] of every key, as
+ * od_npmap computes it, instead of computing it from k and Wk here (callers
+ * that evaluate rows of the same keys many times pass it once computed).
  */
-int od_prefill(const od_dims *s, const double *q, const double *k, const double *v, const double *Wq,
-               const double *Wk, const int32_t *idx_in, double *o, double *r_out, int32_t *idx_out,
-               const int32_t *rows, long nrows, int nthreads)
+static int od_prefill_core(const od_dims *s, const double *q, const double *k, const double *v, const double *Wq,
+                           const double *Wk, const double *phik_in, const int32_t *idx_in, double *o,
+                           double *r_out, int32_t *idx_out, const int32_t *rows, long nrows, int nthreads)
 {
     int e = od_check(s);
     if (e) return e;
     size_t nkv = (size_t)s->B * s->Hkv * s->N;
     unsigned char *selmask = (unsigned char *)malloc(nkv + 1);
-    double *phik = (double *)malloc(sizeof(double) * nkv * s->D + 1);
-    if (!selmask || !phik) {
+    double *phik = phik_in ? NULL : (double *)malloc(sizeof(double) * nkv * s->D + 1);
+    if (!selmask || (!phik_in && !phik)) {
         free(selmask);
         free(phik);
         return OD_ENOMEM;
     }
     e = od_selection(s, q, k, idx_in, r_out, idx_out, selmask, nthreads);
     if (!e) {
-        od_phik_job PJ = {s, k, Wk, phik};
-        od_parallel_for((long)s->B * s->Hkv, nthreads, od_phik_task, &PJ);
-        od_out_job J = {s, q, k, v, Wq, phik, selmask, o, rows, rows ? nrows : (long)s->B * s->H * s->N, 0};
+        if (!phik_in) {
+            od_phik_job PJ = {s, k, Wk, phik};
+            od_parallel_for((long)s->B * s->Hkv, nthreads, od_phik_task, &PJ);
+        }
+        od_out_job J = {s, q, k, v, Wq, phik_in ? phik_in : phik, selmask, o, rows,
+                        rows ? nrows : (long)s->B * s->H * s->N, 0};
         od_parallel_for(J.nrows, nthreads, od_out_task, &J);
         if (J.bad) e = OD_ENONFINITE;
     }
     free(selmask);
     free(phik);
     return e;
+}
+
+int od_prefill(const od_dims *s, const double *q, const double *k, const double *v, const double *Wq,
+               const double *Wk, const int32_t *idx_in, double *o, double *r_out, int32_t *idx_out,
+               const int32_t *rows, long nrows, int nthreads)
+{
+    return od_prefill_core(s, q, k, v, Wq, Wk, NULL, idx_in, o, r_out, idx_out, rows, nrows, nthreads);
+}
+
+int od_prefill_given_phik(const od_dims *s, const double *q, const double *k, const double *v, const double *Wq,
+                          const double *phik, const int32_t *idx_in, double *o, double *r_out, int32_t *idx_out,
+                          const int32_t *rows, long nrows, int nthreads)
+{
+    if (!phik) return OD_EINVAL;
+    return od_prefill_core(s, q, k, v, Wq, NULL, phik, idx_in, o, r_out, idx_out, rows, nrows, nthreads);
 }
 
 /*

@@ -384,6 +384,25 @@ def test_rows_subset(oracle_mod):
         np.testing.assert_array_equal(part[b, h, i], full[b, h, i])
 
 
+def test_given_key_features_change_nothing(oracle_mod):
+    """prefill with phi(k) supplied (from the oracle's own npmap, per KV head with its Wk) gives the
+    same outputs, bit for bit, as prefill computing phi(k) itself -- whole layer and a row subset."""
+    rng = np.random.default_rng(16)
+    dims = oracle_mod.Dims(2, 4, 2, 40, 8, 5, 8, 8, 2)
+    q, k, v, wq, wk = _problem(rng, 2, 4, 2, 40, 8, 5)
+    phik = np.stack([np.stack([oracle_mod.npmap(k[b, g], wk[g]) for g in range(2)]) for b in range(2)])
+    ref = oracle_mod.prefill(dims, q, k, v, wq, wk)
+    got = oracle_mod.prefill(dims, q, k, v, wq, None, phik=phik)
+    np.testing.assert_array_equal(got["o"], ref["o"])
+    np.testing.assert_array_equal(got["idx"], ref["idx"])
+    rows = np.array([[0, 0, 0], [1, 3, 39], [0, 2, 17]])
+    part = oracle_mod.prefill(dims, q, k, v, wq, None, idx_in=ref["idx"], rows=rows, phik=phik)["o"]
+    for b, h, i in rows:
+        np.testing.assert_array_equal(part[b, h, i], ref["o"][b, h, i])
+    with pytest.raises(ValueError):
+        oracle_mod.prefill(dims, q, k, v, wq, None, phik=phik[:, :1])
+
+
 # ---------------------------------------------------------------- decode
 
 @pytest.mark.parametrize("w,C,kk,Hkv", [(8, 8, 2, 1), (16, 8, 3, 2), (0, 8, 0, 1), (8, 8, 8, 1), (8, 8, 0, 2)])
