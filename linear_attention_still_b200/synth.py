@@ -70,6 +70,9 @@ class Shape:
 WORKLOADS = {
     "still_f32_b1_h2_n512": Shape(B=1, H=2, Hkv=2, N=512, d=64, D=64, w=64, C=64, k=8,
                                   dtype="f32", heavy=4),
+    # the same layer decoding 128 tokens after its 512-token prefill (a chunk close every 64)
+    "still_f32_decode_b1_ctx512": Shape(B=1, H=2, Hkv=2, N=512, d=64, D=64, w=64, C=64, k=8,
+                                        dtype="f32", heavy=4, decode_steps=128),
     "llama32_1b_layer_n16k": Shape(B=1, H=32, Hkv=8, N=16384, d=64, D=64, w=512, C=512, k=64),
     "llama31_8b_layer_b4_n16k": Shape(B=4, H=32, Hkv=8, N=16384, d=128, D=128, w=1024, C=1024, k=128),
     "llama31_8b_layer_n64k": Shape(B=1, H=32, Hkv=8, N=65536, d=128, D=128, w=1024, C=1024, k=128),

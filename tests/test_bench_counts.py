@@ -94,13 +94,19 @@ def test_traffic_lookup_follows_source_hashes(tmp_path, monkeypatch):
     assert bench.profiled_traffic("wl") is None
 
 
-def test_reference_arm_line(tmp_path):
-    """`bench.py --impl reference` on the small fp32 workload: one JSON line with the contract's keys,
-    the oracle's own throughput as value, cpu_baseline and e2e carrying the same number."""
+@pytest.mark.parametrize("workload,extra,metric", [
+    ("still_f32_b1_h2_n512", [], bench.METRIC),
+    ("still_f32_b1_h2_n512", ["--pass", "backward"], bench.METRIC_BACKWARD),
+    ("still_f32_decode_b1_ctx512", [], bench.METRIC_DECODE),
+])
+def test_reference_arm_line(tmp_path, workload, extra, metric):
+    """`bench.py --impl reference` on the small fp32 workloads (prefill, its backward, decode): one
+    JSON line with the contract's keys and the pass's metric, the oracle's own throughput as value,
+    cpu_baseline and e2e carrying the same number."""
     import json
     import subprocess
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
-                        "still_f32_b1_h2_n512", "--steps", "3", "--warmup", "1"],
+                        workload, "--steps", "3", "--warmup", "1", *extra],
                        capture_output=True, text=True, timeout=600, cwd=tmp_path)
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
@@ -113,7 +119,7 @@ def test_reference_arm_line(tmp_path):
     assert line["value"] > 0 and line["cpu_baseline"]["value"] == line["value"] == line["e2e"]["value"]
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
-    assert line["config"]["workload"] == "still_f32_b1_h2_n512"
+    assert line["config"]["workload"] == workload and line["metric"] == metric
 
 
 @pytest.mark.parametrize("N,m", [(16384, 64), (16384, 704), (16384, 4352), (16384, 16384), (512, 512),
