@@ -23,7 +23,7 @@ def lib():
     return still
 
 
-def header_verdict(B, H, Hkv, N, d, D, w, C, k, scale, dtype):
+def header_status(B, H, Hkv, N, d, D, w, C, k, scale, dtype):
     """0 (valid), 1 (STILL_ERR_INVALID_ARG) or 2 (STILL_ERR_UNSUPPORTED) by the header's rules."""
     if B < 0 or N < 0 or H < 1 or Hkv < 1 or C < 1 or k < 0 or w < 0:
         return 1
@@ -83,7 +83,7 @@ def dims_st(draw):
 @given(dims_st())
 def test_validation_follows_the_header(lib, p):
     args = (p["B"], p["H"], p["Hkv"], p["N"], p["d"], p["D"], p["w"], p["C"], p["k"], p["scale"], p["dtype"])
-    want = header_verdict(*args)
+    want = header_status(*args)
     d = lib.still_dims(*args)
     ws = lib.still_prefill_workspace_bytes(d)
     if want:
