@@ -50,7 +50,7 @@ def parse():
     p.add_argument("--steps", type=int, default=300)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    p.add_argument("--workload", default=None, choices=sorted(WORKLOADS))
     p.add_argument("--cpu-seconds", type=float, default=15.0, help="target oracle time of the CPU baseline")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--e2e-steps", type=int, default=10)
@@ -63,10 +63,18 @@ def parse():
     p.add_argument("--pass", dest="pass_", choices=["forward", "backward"], default="forward",
                    help="prefill workloads: time the forward layer (default) or its backward pass "
                         "(gradients of q, k, v, Wq, Wk with the selection held fixed)")
+    p.add_argument("--workloads", choices=["auto", "none"], default="auto",
+                   help="auto: a default single-GPU run (no --workload, forward pass, default router and keep) "
+                        "also measures the other layer configurations (8B-shaped prefill at B4 x 16K and "
+                        "1 x 64K, the B16 x 64K decode) and reports each under `workloads`")
     p.add_argument("--router", choices=["saliency", "diagonal"], default="saliency",
                    help="prefill token router: the Self-Saliency Score, or the diagonal-only ablation "
                         "(score -> per-chunk top-k -> prefill with that selection)")
-    return p.parse_args()
+    a = p.parse_args()
+    a.workload_given = a.workload is not None
+    if a.workload is None:
+        a.workload = DEFAULT_WORKLOAD
+    return a
 
 
 # ----------------------------------------------------------------------------- algorithmic counts
@@ -156,16 +164,68 @@ def profiled_traffic(workload: str):
 
 
 class ClockSampler:
+    """SM clock, power and clock-event reasons sampled DURING a timed region (reads only).
+
+    In-process NVML queries every `period_s` (2 ms) from a thread, so that even a timed region of a
+    few tens of milliseconds gets samples of its own; falls back to an `nvidia-smi -lms 20` child
+    when NVML cannot be loaded."""
+
     FIELDS = ["index", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
               "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
               "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+    REASON_BITS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+                   "sw_power_cap": 0x4}
 
-    def __init__(self, gpu_id: str | None):
-        self.rows = []
+    def __init__(self, gpu_id: str | None, period_s: float = 0.002, nvml=None):
+        self.rows = []          # (sm_mhz, sm_max_mhz, power_w, set of reason names)
         self.proc = None
+        self.thread = None
         self.gpu_id = gpu_id
+        self.period_s = period_s
+        self.source = None
+        self._nvml = nvml
+        self._stop = threading.Event()
+
+    def _nvml_handle(self):
+        nv = self._nvml
+        if nv is None:
+            import pynvml as nv
+        nv.nvmlInit()
+        if self.gpu_id:
+            h = nv.nvmlDeviceGetHandleByUUID(self.gpu_id)
+        else:
+            h = nv.nvmlDeviceGetHandleByIndex(0)
+        return nv, h
+
+    def _nvml_sample(self, nv, h):
+        sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+        smax = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+        try:
+            pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+        except Exception:
+            pw = None
+        bits = int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))
+        self.rows.append((sm, smax, pw, {n for n, b in self.REASON_BITS.items() if bits & b}))
+
+    def _nvml_loop(self, nv, h):
+        while not self._stop.is_set():
+            try:
+                self._nvml_sample(nv, h)
+            except Exception:
+                return
+            self._stop.wait(self.period_s)
 
     def start(self):
+        try:
+            nv, h = self._nvml_handle()
+            self._nvml_sample(nv, h)  # fails here, not in the thread, when a query is unsupported
+            self.rows.clear()
+            self.source = f"nvml, every {self.period_s * 1e3:g} ms"
+            self.thread = threading.Thread(target=self._nvml_loop, args=(nv, h), daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            self.rows.clear()
         cmd = ["nvidia-smi", f"--query-gpu={','.join(self.FIELDS)}", "--format=csv,noheader,nounits", "-lms", "20"]
         if self.gpu_id:
             cmd += ["-i", self.gpu_id]
@@ -174,40 +234,47 @@ class ClockSampler:
         except OSError:
             self.proc = None
             return
-        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.source = "nvidia-smi -lms 20"
+        self.thread = threading.Thread(target=self._smi_read, daemon=True)
         self.thread.start()
-        # nvidia-smi takes a moment to start: wait for its first sample, so that a short timed
-        # region still gets samples of its own, then keep only those
+        # nvidia-smi takes a moment to start: wait for its first sample, then keep only later ones
         t_end = time.time() + 5.0
         while not self.rows and time.time() < t_end and self.proc.poll() is None:
             time.sleep(0.01)
         self.rows.clear()
 
-    def _read(self):
+    def _smi_read(self):
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+        def num(s):
+            try:
+                return float(s)
+            except ValueError:
+                return None
         for line in self.proc.stdout:
             parts = [x.strip() for x in line.split(",")]
-            if len(parts) == len(self.FIELDS):
-                self.rows.append(parts)
+            if len(parts) == len(self.FIELDS) and num(parts[1]) is not None:
+                self.rows.append((num(parts[1]), num(parts[2]), num(parts[3]),
+                                  {names[j] for j in range(4) if parts[5 + j].lower() == "active"}))
 
     def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.thread.join(timeout=5)
+        self._stop.set()
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
         if not self.rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
-        smax = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[j] for r in self.rows for j in range(4) if r[5 + j].lower() == "active"})
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "source": self.source}
+        sm = [r[0] for r in self.rows if r[0] is not None]
+        smax = [r[1] for r in self.rows if r[1] is not None]
+        pw = [r[2] for r in self.rows if r[2] is not None]
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "reasons": reasons, "samples": len(self.rows),
-                "power_w_max": max((float(r[3]) for r in self.rows if r[3].replace(".", "").isdigit()),
-                                   default=None)}
+                "reasons": sorted(set().union(*(r[3] for r in self.rows))), "samples": len(self.rows),
+                "power_w_max": max(pw) if pw else None, "source": self.source}
 
 
 # ----------------------------------------------------------------------------- CPU baseline (oracle)
@@ -356,9 +423,9 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
-def workload_shape(args):
+def workload_shape(args, name=None):
     """The workload's shape with --keep applied (k = C keeps every token of a decided chunk)."""
-    shape = WORKLOADS[args.workload]
+    shape = WORKLOADS[name or args.workload]
     keep = getattr(args, "keep", "config")
     if keep == "all" and shape.w > 0:
         shape = shape.replace(k=shape.C)
@@ -369,8 +436,8 @@ def workload_shape(args):
     return shape
 
 
-def config_of(shape, args):
-    return {"workload": args.workload, "B": shape.B, "H": shape.H, "Hkv": shape.Hkv, "N": shape.N, "d": shape.d,
+def config_of(shape, args, name=None):
+    return {"workload": name or args.workload, "B": shape.B, "H": shape.H, "Hkv": shape.Hkv, "N": shape.N, "d": shape.d,
             "D": shape.D, "w": shape.w, "C": shape.C, "k": shape.k, "global_batch": shape.B * args.gpus,
             "seq_len": shape.N, "parallelism": f"replicas{args.gpus}", "l2": "flushed before every step",
             "router": getattr(args, "router", "saliency"), "keep": getattr(args, "keep", "config")}
@@ -392,25 +459,18 @@ def job_throughput(tokens_per_rank: int, steps: int, world: int, max_ms: float) 
     return world * tokens_per_rank * steps / (max_ms / 1e3)
 
 
-def run_ours(args):
+def bench_prefill(args, name, rank, world, local, cpu_seconds):
+    """One prefill workload on this rank: the timed steps, the end-to-end steps, the roofline and (rank 0,
+    one GPU) the CPU baseline; returns the JSON line as a dict."""
     import numpy as np
     import torch
 
-    rank, world, local = dist_setup(args)
-    torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
     from linear_attention_still_b200 import still
 
-    shape = workload_shape(args)
+    shape = workload_shape(args, name)
     tdt = torch.bfloat16 if shape.dtype == "bf16" else torch.float32
-    inp = make_inputs(shape.replace(seed=rank))
-    host = {n: torch.from_numpy(np.ascontiguousarray(getattr(inp, n)[:, :, :shape.N] if n in "qkv" else
-                                                     getattr(inp, n))).to(tdt)
+    inp = make_inputs(shape.replace(seed=rank), threads=len(os.sched_getaffinity(0)))
+    host = {n: to_host_tensor(getattr(inp, n)[:, :, :shape.N] if n in "qkv" else getattr(inp, n), tdt)
             for n in ("q", "k", "v", "wq", "wk")}
     del inp
     devt = {n: t.cuda() for n, t in host.items()}
@@ -527,13 +587,13 @@ def run_ours(args):
         "kernel": "merge (window phase + kept-prefix phase)", "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
         "frac": (achieved / peak) if (achieved and peak) else None,
         "peak_source": "measured bf16_tflops" if "bf16_tflops" in peaks else "fallback 1.59 PFLOP/s",
-        "traffic": profiled_traffic(args.workload), "traffic_unit": "DRAM bytes per step (both merge launches, ncu)",
+        "traffic": profiled_traffic(name), "traffic_unit": "DRAM bytes per step (both merge launches, ncu)",
         "flops_per_step": merge_flops(shape), "ms_per_step": merge_ms / merge_n if merge_n else None,
     }
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": shape.dtype, "data": "synthetic", "config": config_of(shape, args),
+        "vs_baseline": None, "dtype": shape.dtype, "data": "synthetic", "config": config_of(shape, args, name),
         "roofline": roofline,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches, "clocks": clocks,
@@ -544,13 +604,10 @@ def run_ours(args):
                                   torch.cuda.get_device_properties(local).multi_processor_count),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, t, desc, nth = oracle_sample(shape, args.cpu_seconds, router=args.router)
+        v, t, desc, nth = oracle_sample(shape, cpu_seconds, router=args.router)
         line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": nth, "kind": "oracle", "sample": desc}
-    if world > 1:
-        torch.distributed.barrier()
-        torch.distributed.destroy_process_group()
-    if rank == 0:
-        print(json.dumps(line), flush=True)
+    del devt, o, ws, flush, host
+    return line
 
 
 # ----------------------------------------------------------------------------- decode workload
@@ -678,18 +735,14 @@ def oracle_decode_sample(shape, seconds: float):
     return 1.0 / per_token, t_call, desc, nth
 
 
-def run_decode(args):
+def bench_decode(args, name, rank, world, local, cpu_seconds):
+    """One decode workload on this rank (prefill of the context, then timed decode steps); returns the
+    JSON line as a dict."""
     import numpy as np
     import torch
 
-    rank, world, local = dist_setup(args)
-    torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=torch.device("cuda", local))
     from linear_attention_still_b200 import still
-    shape = workload_shape(args)
+    shape = workload_shape(args, name)
     N, steps, B = shape.N, shape.decode_steps, shape.B
     tdt = torch.bfloat16 if shape.dtype == "bf16" else torch.float32
     e2e_steps = min(args.e2e_steps, 20)
@@ -703,14 +756,18 @@ def run_decode(args):
     kd = torch.empty(steps, B, shape.Hkv, shape.d, dtype=tdt)
     vd = torch.empty_like(kd)
     wq = wk = None
-    for b in range(B):  # one batch item at a time keeps the host footprint bounded
-        inp = make_inputs(shape.replace(seed=shape.seed + rank), batches=[b])
-        q[b].copy_(torch.from_numpy(inp.q[0, :, :N]).to(tdt))
-        k[b].copy_(torch.from_numpy(inp.k[0, :, :N]).to(tdt))
-        v[b].copy_(torch.from_numpy(inp.v[0, :, :N]).to(tdt))
-        qd[:, b] = torch.from_numpy(np.ascontiguousarray(inp.q[0, :, N:].transpose(1, 0, 2))).to(tdt)
-        kd[:, b] = torch.from_numpy(np.ascontiguousarray(inp.k[0, :, N:].transpose(1, 0, 2))).to(tdt)
-        vd[:, b] = torch.from_numpy(np.ascontiguousarray(inp.v[0, :, N:].transpose(1, 0, 2))).to(tdt)
+    # a few batch items at a time (drawn concurrently) keeps the host footprint bounded; the prefix
+    # goes to the device in fp32 and is converted there
+    group = max(1, min(8, len(os.sched_getaffinity(0))))
+    for b0 in range(0, B, group):
+        bs = list(range(b0, min(B, b0 + group)))
+        inp = make_inputs(shape.replace(seed=shape.seed + rank), batches=bs, threads=len(bs))
+        for n, b in enumerate(bs):
+            for dst, src_ in ((q, inp.q), (k, inp.k), (v, inp.v)):
+                dst[b].copy_(torch.from_numpy(np.ascontiguousarray(src_[n, :, :N])).cuda().to(tdt))
+            qd[:, b] = torch.from_numpy(np.ascontiguousarray(inp.q[n, :, N:].transpose(1, 0, 2))).to(tdt)
+            kd[:, b] = torch.from_numpy(np.ascontiguousarray(inp.k[n, :, N:].transpose(1, 0, 2))).to(tdt)
+            vd[:, b] = torch.from_numpy(np.ascontiguousarray(inp.v[n, :, N:].transpose(1, 0, 2))).to(tdt)
         wq, wk = torch.from_numpy(inp.wq).to(tdt).cuda(), torch.from_numpy(inp.wk).to(tdt).cuda()
         del inp
     state = torch.empty(still.still_decode_state_bytes(dims, cap), dtype=torch.uint8, device="cuda")
@@ -803,7 +860,7 @@ def run_decode(args):
         "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": shape.dtype, "data": "synthetic",
-        "config": dict(config_of(shape, args), decode_steps_timed=K, first_position=first,
+        "config": dict(config_of(shape, args, name), decode_steps_timed=K, first_position=first,
                        chunk_close_steps_timed=len(close_steps),
                        l2="decode state (kept cache + window) larger than L2"),
         "roofline": {"kernel": "decode step (all kernels)", "bound": "hbm", "achieved": achieved, "peak": peak,
@@ -824,13 +881,10 @@ def run_decode(args):
         "device_status": status,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v_, t_, desc, nth = oracle_decode_sample(shape, args.cpu_seconds)
+        v_, t_, desc, nth = oracle_decode_sample(shape, cpu_seconds)
         line["cpu_baseline"] = {"value": v_, "unit": "tokens/s", "cores": nth, "kind": "oracle", "sample": desc}
-    if world > 1:
-        torch.distributed.barrier()
-        torch.distributed.destroy_process_group()
-    if rank == 0:
-        print(json.dumps(line), flush=True)
+    del state, qdd, kdd, vdd, o_t, qb, kb, vb, wq, wk
+    return line
 
 
 def backward_flops(shape):
@@ -842,18 +896,13 @@ def backward_flops(shape):
         shape.B * shape.Hkv * shape.N * 8 * shape.d * shape.D
 
 
-def run_backward(args):
+def bench_backward(args, name, rank, world, local, cpu_seconds):
+    """The backward pass of one prefill workload on this rank; returns the JSON line as a dict."""
     import numpy as np
     import torch
 
-    rank, world, local = dist_setup(args)
-    torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=torch.device("cuda", local))
     from linear_attention_still_b200 import still
-    shape = workload_shape(args)
+    shape = workload_shape(args, name)
     tdt = torch.bfloat16 if shape.dtype == "bf16" else torch.float32
     inp = make_inputs(shape.replace(seed=rank))
     host = {n: torch.from_numpy(np.ascontiguousarray(getattr(inp, n))).to(tdt) for n in ("q", "k", "v", "wq", "wk")}
@@ -938,7 +987,7 @@ def run_backward(args):
         "value": job_throughput(tokens, args.steps, world, total_ms), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": shape.dtype, "data": "synthetic",
-        "config": dict(config_of(shape, args), **{"pass": "backward"}),
+        "config": dict(config_of(shape, args, name), **{"pass": "backward"}),
         "roofline": {"kernel": "backward pass (all kernels)", "bound": "alu", "achieved": achieved, "peak": peak,
                      "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
                      "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 FLOP x 1965 MHz (SIMT kernels)",
@@ -949,8 +998,47 @@ def run_backward(args):
         "gpu_launches": launches, "clocks": clocks, "device_status": still.still_get_device_status(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v_, t_, desc, nth = oracle_backward_sample(shape, args.cpu_seconds)
+        v_, t_, desc, nth = oracle_backward_sample(shape, cpu_seconds)
         line["cpu_baseline"] = {"value": v_, "unit": "tokens/s", "cores": nth, "kind": "oracle", "sample": desc}
+    return line
+
+
+# the other layer configurations a default single-GPU run also reports (under `workloads`)
+EXTRA_WORKLOADS = ("llama31_8b_layer_b4_n16k", "llama31_8b_layer_n64k", "llama31_8b_decode_b16_ctx64k")
+EXTRA_CPU_SECONDS = 8.0
+
+
+def to_host_tensor(a, tdt):
+    import numpy as np
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a)).to(tdt)
+
+
+def bench_one(args, name, rank, world, local, cpu_seconds):
+    if WORKLOADS[name].decode_steps > 0:
+        return bench_decode(args, name, rank, world, local, cpu_seconds)
+    if args.pass_ == "backward":
+        return bench_backward(args, name, rank, world, local, cpu_seconds)
+    return bench_prefill(args, name, rank, world, local, cpu_seconds)
+
+
+def run_ours(args):
+    import torch
+
+    rank, world, local = dist_setup(args)
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    line = bench_one(args, args.workload, rank, world, local, args.cpu_seconds)
+    extras = args.workloads == "auto" and world == 1 and not args.workload_given and args.pass_ == "forward" \
+        and args.router == "saliency" and args.keep == "config"
+    if extras:
+        line["workloads"] = {}
+        for name in EXTRA_WORKLOADS:
+            torch.cuda.empty_cache()
+            line["workloads"][name] = bench_one(args, name, rank, world, local, EXTRA_CPU_SECONDS)
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
@@ -962,10 +1050,6 @@ def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
-    elif WORKLOADS[args.workload].decode_steps > 0:
-        run_decode(args)
-    elif args.pass_ == "backward":
-        run_backward(args)
     else:
         run_ours(args)
 

@@ -269,20 +269,20 @@ STILL_API uint64_t still_launch_count(void);
  * combine, 10 decode chunk close.  Single-threaded use only.
  */
 /*
- * Diagnostics (no counterpart in the method): when `words` is non-NULL, the
- * tensor-core merge kernel records 16 progress words per CTA there (producer,
- * MMA issuer and each softmax warp: last step reached; 0xBAD.. on a bounded
- * wait that gave up; SM clock at CTA start, first score tile, epilogue and
- * exit in words 10..13; 0xD0E / 0xF1F at exit).  The window-phase launch
- * (G1 = B*Hkv*(G/2)*ceil(N/128) CTAs) uses words [0, 16 G1 + 2049); the
- * kept-prefix launch (G2 = B*Hkv*(G/2)*(ceil(N/128) - (m+1)C/128) CTAs) uses
- * 16 G2 + 2049 words from word 16 G1 + 2080 on, so the buffer must hold
- * 16 (G1 + G2) + 4129 words.  Word 2048 past each launch's per-CTA words
- * selects the CTA whose per-tile clocks are recorded.  Pass host-mapped
- * (pinned) memory to read it while a kernel runs.  NULL (the default)
- * disables it.
+ * Test hooks of the head-dimension-64 tensor-core merge (no counterpart in the
+ * method; host state of the library, read when a merge is launched;
+ * single-threaded use only; (0, 0), the default, leaves the kernels alone).
+ *   stall != 0: the first CTA of every later launch loads its query tiles but
+ *     issues no key/value tile, so its MMA warp's bounded wait (2 s) runs out:
+ *     the CTA records STILL_ERR_TIMEOUT in the device status word (read it
+ *     with still_get_device_status), drains its own copies, frees its tensor
+ *     memory and returns, and every other CTA finishes normally.  The output
+ *     of that call is undefined; the context stays usable.
+ *   max_ctas > 0: the persistent merge grid holds at most max_ctas CTAs (one
+ *     per SM otherwise), so small problems also run many work items per CTA.
+ *     Results do not depend on it.
  */
-STILL_API void still_debug_set_trace(unsigned *words);
+STILL_API void still_debug_merge(int stall, int max_ctas);
 
 #define STILL_TIMING_MAX_LAUNCHES 4096
 #define STILL_TIMING_CLASSES 11

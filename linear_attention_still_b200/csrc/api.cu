@@ -21,7 +21,7 @@ cudaError_t launch_mean_heads(const Dims &s, const float *sigma, float *r, cudaS
 cudaError_t launch_saliency_fixup(const Dims &s, const void *q, const void *k, const int *list, const unsigned *count,
                                   float *sigma, cudaStream_t st);
 bool tc_saliency_supported(const Dims &s);
-void set_debug_trace_words(unsigned *p);
+void set_merge_debug(int stall, int max_ctas);
 cudaError_t launch_saliency_tc(const Dims &s, const void *q, const void *k, float *r_kv, float *r_q, unsigned *err,
                                cudaStream_t st);
 }  // namespace still
@@ -434,7 +434,7 @@ still_status still_decode_step(const still_dims *dims, void *state, int capacity
     return cuda_status(e);
 }
 
-void still_debug_set_trace(unsigned *words) { set_debug_trace_words(words); }
+void still_debug_merge(int stall, int max_ctas) { set_merge_debug(stall, max_ctas); }
 
 still_status still_timing_enable(int on) {
     g_timing = on != 0;

@@ -25,14 +25,13 @@
 #include "rowops.cuh"
 #include "still_internal.h"
 #include "tc_ptx.cuh"
+#include "tc_tile.cuh"
 
 namespace still {
 
 using namespace tc;
 
 namespace {
-
-constexpr float kLog2e = 1.4426950408889634f;
 
 template <int DH, int DF, int HP>
 struct MergeCfg {
@@ -46,7 +45,7 @@ struct MergeCfg {
     static constexpr int WQ_BYTES = DF * DH * 2;       // one Wq^T [DF rows x DH]
     static constexpr int ST_BYTES = DH * DF * 2;       // S_t^T [DH rows x DF]
     static_assert(HP * WQ_BYTES + ST_BYTES <= NS * STAGE_BYTES, "prologue tiles must fit the stage area");
-    static constexpr int NUM_BARS = 4 + 3 * NS + 6 * HP + 2;  // see the slot map in the kernel
+    static constexpr int NUM_BARS = 4 + 3 * NS + 5 * HP;  // see the slot map in the kernel
     static constexpr int TMEM_SLOT_OFF = 8 * NUM_BARS;          // u32 TMEM base address
     static constexpr int ABORT_OFF = TMEM_SLOT_OFF + 8;         // int abort flag
     static constexpr int BAR_BYTES = 256;
@@ -61,14 +60,12 @@ struct MergeCfg {
     static constexpr int REG_SOFTMAX = 208, REG_OTHER = 88;
     static_assert(HP != 2 || 2 * 128 * REG_SOFTMAX + 128 * REG_OTHER <= THREADS * 168, "register split");
     static constexpr int TMEM_COLS = 512;
-    // d = 64: P (bf16, 64 columns) gets its own TMEM columns, so the next tile's S = Q K^T can be
-    // issued as soon as the softmax has read S (it then overlaps the exponentials).  d = 128: the
-    // budget is full (2 x S + 2 x O = 512 columns) and P is written over S.
-    static constexpr bool PSEP = DH == 64;
+    // The budget is full at d = 128 (2 x S + 2 x O = 512 columns): P is written over S, and the next
+    // tile's scores wait for P V.  (Head dimension 64 runs the ring-scheduled kernel of merge_ring.cu.)
     __host__ __device__ static constexpr int s_col(int x) { return x * 128; }
-    __host__ __device__ static constexpr int p_col(int x) { return PSEP ? 128 * HP + x * 64 : x * 128; }
-    __host__ __device__ static constexpr int o_col(int x) { return 128 * HP + (PSEP ? 64 * HP : 0) + x * DH; }
-    static_assert(128 * HP + (PSEP ? 64 * HP : 0) + HP * DH <= TMEM_COLS, "TMEM budget");
+    __host__ __device__ static constexpr int p_col(int x) { return x * 128; }
+    __host__ __device__ static constexpr int o_col(int x) { return 128 * HP + x * DH; }
+    static_assert(128 * HP + HP * DH <= TMEM_COLS, "TMEM budget");
 };
 
 struct MergeParams {
@@ -84,80 +81,13 @@ struct MergeParams {
     int n_qtiles;          // ceil(N/128)
     int qt_first;          // first query tile of this launch (PREFIX: chunks t > m only)
     int pairs;             // G / HP
-    unsigned *trace;       // optional progress words (16 per CTA), see still_debug_set_trace
 };
-
-// Phase timeline of one CTA (diagnostics only): words [16*gridDim.x + (role*64 + j)*8 + phase] hold
-// the SM clock() when `role` (0/1 softmax warpgroup, 2 MMA issuer, 3 producer) reached `phase` of
-// key tile j, recorded for blockIdx.x == trace[16*gridDim.x + 2048] only.
-__device__ __forceinline__ void trace_time(unsigned *trace, int role, int j, int phase) {
-    if (trace && j < 64) {
-        const unsigned target = trace[16 * gridDim.x + 2048];
-        if (blockIdx.x == target)
-            trace[16 * gridDim.x + (role * 64 + j) * 8 + phase] = (unsigned)clock();
-    }
-}
-
-// Progress word of this CTA (diagnostics only; a no-op unless a trace buffer is set).
-__device__ __forceinline__ void trace_word(unsigned *trace, int slot, unsigned v) {
-    if (trace) *reinterpret_cast<volatile unsigned *>(trace + blockIdx.x * 16 + slot) = v;
-}
-
-constexpr float kLn2 = 0.6931471805599453f;
-
-// Exponentials of one 128-key row tile: p_c = 2^(s_c tau log2e - m), summed (ls0 + ls1) and written
-// as bf16 P to TMEM (four tcgen05.st of 16 columns).  BAND additionally sums p_c over the columns
-// [bc_lo, bc_hi) into bsum (the Self-Saliency band of this row inside the tile).
-template <int EXPV, bool BAND>
-__device__ __forceinline__ void exp_tile(const float (&sv)[128], float scale_log2, float m_run, uint32_t tP,
-                                         float &ls0, float &ls1, float &bsum, int bc_lo, int bc_hi) {
-    const float2 sc2 = make_float2(scale_log2, scale_log2);
-    const float2 neg2 = make_float2(-m_run, -m_run);
-    float2 ls = make_float2(0.f, 0.f);
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        uint32_t u[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-            const int c0 = c * 32 + 2 * e;
-            const float2 xx = ffma2(make_float2(sv[c0], sv[c0 + 1]), sc2, neg2);
-            float2 pp;
-            if ((EXPV == 2 && c == 3) || (EXPV == 3 && (c & 1))) {
-                pp = exp2_poly2(xx);  // FMA pipe
-            } else {
-                pp.x = ex2(xx.x);      // MUFU
-                pp.y = ex2(xx.y);
-            }
-            ls = fadd2(ls, pp);
-            if (BAND) {
-                if (c0 >= bc_lo && c0 < bc_hi) bsum += pp.x;
-                if (c0 + 1 >= bc_lo && c0 + 1 < bc_hi) bsum += pp.y;
-            }
-            u[e] = pack_bf16x2(pp.x, pp.y);
-        }
-        tmem_st16(tP + c * 16, u);
-    }
-    ls0 = ls.x;
-    ls1 = ls.y;
-}
-
-// tcgen05.ld/st are warp-collective: every decision that guards them is made warp-uniform.
-__device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
-
-// K-major SW128 descriptor of k-step kk (16 elements) of a tile whose rows are split into 64-col
-// regions of `region_bytes` each.
-__device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, int kk, uint32_t region_bytes) {
-    return sw128_desc(base + (kk >> 2) * region_bytes + (kk & 3) * 32, 16, 1024);
-}
 
 // EXPV selects the exponential phase: 0 scalar FFMA + MUFU, 1 packed FFMA2/FADD2 + MUFU,
 // 2 packed with the last 32-key chunk of each row on the FMA-pipe exp2, 3 with every other 32-key
 // chunk there.  Measured on B200 with concurrent softmax warpgroups (1B 16K / 8B B4 16K layers, the
 // two merge phases, ms): variant 1 0.612/3.629, 2 0.608/3.646, 3 0.641/3.799 -> variant 1 is built.
 constexpr int kMergeExpVariant = 1;
-// Two heads per CTA: the softmax warpgroups take turns on the exponential phase (true) or run it
-// concurrently (false; measured 2-5 % faster: both warpgroups' exponentials keep the MUFU unit busy).
-constexpr bool kMergeTurns = false;
 // MODE kMergeLocal: keys = the window [max(0,(t-m)C), i]; also the Self-Saliency Score of every row
 //   ([p1] "Self-Saliency Score"): the band keys [i-w+1, i-1] are window keys, so the band's
 //   log-sum-exp is accumulated from the same exponentials (masked adds on the two partial tiles),
@@ -187,14 +117,11 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
     const int B_QFULL = 0, B_WFULL = 1, B_PRO = 2, B_DRAIN = 3;
     const int B_KFULL = 4, B_VFULL = 4 + Cfg::NS, B_KVEMPTY = 4 + 2 * Cfg::NS;
     const int B_Y = 4 + 3 * Cfg::NS, B_PHI = B_Y + HP, B_S = B_PHI + HP, B_P = B_S + HP, B_O = B_P + HP;
-    const int B_TURN = B_O + HP;  // [2]: exponential-phase turn of softmax warpgroup 0 / 1
-    const int B_SFREE = B_TURN + 2;  // [HP]: the softmax has read S (separate-P schedule)
-    static_assert(Cfg::NUM_BARS == 4 + 3 * Cfg::NS + 6 * HP + 2, "slot map");
+    static_assert(Cfg::NUM_BARS == 4 + 3 * Cfg::NS + 5 * HP, "slot map");
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_area + Cfg::TMEM_SLOT_OFF);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(bar_area + Cfg::ABORT_OFF);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (threadIdx.x == 0) trace_word(p.trace, 10, (unsigned)clock());
 
     // ---- CTA -> (b, g, head pair, query tile); heavier (later) query tiles first
     const int per_qt = p.B * p.Hkv * p.pairs;
@@ -230,9 +157,6 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
             mbar_init(BAR(B_P + x), 128);
             mbar_init(BAR(B_O + x), 1);
         }
-        mbar_init(BAR(B_TURN + 0), 128);
-        mbar_init(BAR(B_TURN + 1), 128);
-        for (int x = 0; x < HP; ++x) mbar_init(BAR(B_SFREE + x), 128);
         *abort_flag = 0;
         mbar_fence_init();
     }
@@ -257,54 +181,51 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
     if (HP == 2) setmaxnreg_dec<Cfg::REG_OTHER>();
     if (warp == Cfg::PRODUCER_WARP) {
         // ================================================================ TMA producer
-        if (lane == 0) {
+        // (the whole warp runs the issue loop; one elected lane issues each copy)
+        {
             bool ok = true;
             int issued = 0;
-            mbar_arrive_expect_tx(BAR(B_QFULL), Cfg::Q_BYTES);
+            mbar_arrive_expect_tx_w(BAR(B_QFULL), Cfg::Q_BYTES);
             for (int x = 0; x < HP; ++x) {
                 const int h = g * p.G + pair * HP + x;
                 for (int rr = 0; rr < DH / 64; ++rr)
-                    tma_load_3d(sQ + x * Cfg::TILE_BYTES + rr * Cfg::REG, &map_q, BAR(B_QFULL), rr * 64, i0,
+                    tma_load_3d_w(sQ + x * Cfg::TILE_BYTES + rr * Cfg::REG, &map_q, BAR(B_QFULL), rr * 64, i0,
                                 b * p.H + h);
             }
             if (!LOCAL) {
-                mbar_arrive_expect_tx(BAR(B_WFULL), HP * Cfg::WQ_BYTES + Cfg::ST_BYTES);
+                mbar_arrive_expect_tx_w(BAR(B_WFULL), HP * Cfg::WQ_BYTES + Cfg::ST_BYTES);
                 for (int x = 0; x < HP; ++x) {
                     const int h = g * p.G + pair * HP + x;
                     for (int rr = 0; rr < DH / 64; ++rr)
-                        tma_load_3d(sStage + x * Cfg::WQ_BYTES + rr * (DF * 128), &map_wq, BAR(B_WFULL), rr * 64, 0,
+                        tma_load_3d_w(sStage + x * Cfg::WQ_BYTES + rr * (DF * 128), &map_wq, BAR(B_WFULL), rr * 64, 0,
                                     h);
                 }
                 for (int rr = 0; rr < DF / 64; ++rr)
-                    tma_load_3d(sStage + HP * Cfg::WQ_BYTES + rr * (DH * 128), &map_st, BAR(B_WFULL), rr * 64, 0,
+                    tma_load_3d_w(sStage + HP * Cfg::WQ_BYTES + rr * (DH * 128), &map_st, BAR(B_WFULL), rr * 64, 0,
                                 tslot);
-                trace_word(p.trace, 0, 1);
-                ok = mbar_wait(BAR(B_PRO), 0, abort_flag);  // prologue operands consumed
-                trace_word(p.trace, 0, ok ? 2 : 0xBAD2);
+                ok = mbar_wait_w(BAR(B_PRO), 0, abort_flag);  // prologue operands consumed
             }
             for (int j = 0; ok && j < n_tiles; ++j) {
                 const int s = j % Cfg::NS;
                 if (j >= Cfg::NS) {
-                    ok = mbar_wait(BAR(B_KVEMPTY + s), ((j / Cfg::NS) - 1) & 1, abort_flag);
+                    ok = mbar_wait_w(BAR(B_KVEMPTY + s), ((j / Cfg::NS) - 1) & 1, abort_flag);
                     if (!ok) break;
                 }
                 const uint32_t sK = sStage + s * Cfg::STAGE_BYTES, sV = sK + Cfg::TILE_BYTES;
                 const CUtensorMap *mk = LOCAL ? &map_k : &map_kh;
                 const CUtensorMap *mv = LOCAL ? &map_v : &map_vh;
                 const int row = LOCAL ? lo + j * Cfg::BN : j * Cfg::BN;
-                mbar_arrive_expect_tx(BAR(B_KFULL + s), Cfg::TILE_BYTES);
+                mbar_arrive_expect_tx_w(BAR(B_KFULL + s), Cfg::TILE_BYTES);
                 for (int rr = 0; rr < DH / 64; ++rr)
-                    tma_load_3d(sK + rr * Cfg::REG, mk, BAR(B_KFULL + s), rr * 64, row, bg);
-                mbar_arrive_expect_tx(BAR(B_VFULL + s), Cfg::TILE_BYTES);
+                    tma_load_3d_w(sK + rr * Cfg::REG, mk, BAR(B_KFULL + s), rr * 64, row, bg);
+                mbar_arrive_expect_tx_w(BAR(B_VFULL + s), Cfg::TILE_BYTES);
                 for (int rr = 0; rr < DH / 64; ++rr)
-                    tma_load_3d(sV + rr * Cfg::REG, mv, BAR(B_VFULL + s), rr * 64, row, bg);
+                    tma_load_3d_w(sV + rr * Cfg::REG, mv, BAR(B_VFULL + s), rr * 64, row, bg);
                 issued = j + 1;
-                trace_word(p.trace, 0, 0x100 + j);
-                trace_time(p.trace, 3, j, 0);
             }
             if (!ok) {
                 *abort_flag = 1;
-                report(p.err, DEV_ERR_TIMEOUT);
+                if (lane == 0) report(p.err, DEV_ERR_TIMEOUT);
                 // drain this CTA's copies still in flight
                 mbar_wait_drain(BAR(B_QFULL), 0, 100000000ull);
                 if (!LOCAL) mbar_wait_drain(BAR(B_WFULL), 0, 100000000ull);
@@ -316,34 +237,33 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
         }
     } else if (warp == Cfg::MMA_WARP) {
         // ================================================================ MMA issuer
-        if (lane == 0) {
+        // (the whole warp runs the issue loop; one elected lane issues each MMA and commit)
+        {
+            const uint32_t tmem_w = __shfl_sync(0xffffffffu, tmem, 0);
             constexpr uint32_t ID_Y = idesc_bf16(128, DF, 0, 0);
             constexpr uint32_t ID_LIN = idesc_bf16(128, DH, 0, 0);
             constexpr uint32_t ID_S = idesc_bf16(128, 128, 0, 0);
             constexpr uint32_t ID_PV = idesc_bf16(128, DH, 0, 1);
-            bool ok = mbar_wait(BAR(B_QFULL), 0, abort_flag) && (LOCAL || mbar_wait(BAR(B_WFULL), 0, abort_flag));
-            trace_word(p.trace, 1, ok ? 1 : 0xBAD1);
+            bool ok = mbar_wait_w(BAR(B_QFULL), 0, abort_flag) && (LOCAL || mbar_wait_w(BAR(B_WFULL), 0, abort_flag));
             if (ok && !LOCAL) {
                 tc_fence_after();
                 for (int x = 0; x < HP; ++x) {
                     const uint32_t aq = sQ + x * Cfg::TILE_BYTES, bw = sStage + x * Cfg::WQ_BYTES;
                     for (int kk = 0; kk < DH / 16; ++kk)
-                        mma_ss(tmem + Cfg::s_col(x), kmajor_desc(aq, kk, Cfg::REG), kmajor_desc(bw, kk, DF * 128),
+                        mma_ss_w(tmem_w + Cfg::s_col(x), kmajor_desc(aq, kk, Cfg::REG), kmajor_desc(bw, kk, DF * 128),
                                ID_Y, kk > 0);
-                    mma_commit(BAR(B_Y + x));
+                    mma_commit_w(BAR(B_Y + x));
                 }
                 for (int x = 0; x < HP && ok; ++x) {
-                    ok = mbar_wait(BAR(B_PHI + x), 0, abort_flag);
-                    trace_word(p.trace, 1, ok ? 3 + x : 0xBAD3);
+                    ok = mbar_wait_w(BAR(B_PHI + x), 0, abort_flag);
                     if (!ok) break;
                     tc_fence_after();
                     const uint32_t bs = sStage + HP * Cfg::WQ_BYTES;
                     for (int kk = 0; kk < DF / 16; ++kk)
-                        mma_ts(tmem + Cfg::o_col(x), tmem + Cfg::s_col(x) + kk * 8, kmajor_desc(bs, kk, DH * 128),
+                        mma_ts_w(tmem_w + Cfg::o_col(x), tmem_w + Cfg::s_col(x) + kk * 8, kmajor_desc(bs, kk, DH * 128),
                                ID_LIN, kk > 0);
                 }
-                if (ok) mma_commit(BAR(B_PRO));
-                trace_word(p.trace, 1, 5);
+                if (ok) mma_commit_w(BAR(B_PRO));
             }
             // Descriptors are built once per operand tile and advanced per 16-element k-step by a
             // constant added to the start-address field (addresses stay below 256 KB, so no carry).
@@ -356,11 +276,11 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
                 const uint64_t dk = sw128_desc(sK, 16, 1024);
 #pragma unroll
                 for (int kk = 0; kk < DH / 16; ++kk)
-                    mma_ss(tmem + Cfg::s_col(x), dq[x] + kstep(kk), dk + kstep(kk), ID_S, kk > 0);
-                mma_commit(BAR(B_S + x));
+                    mma_ss_w(tmem_w + Cfg::s_col(x), dq[x] + kstep(kk), dk + kstep(kk), ID_S, kk > 0);
+                mma_commit_w(BAR(B_S + x));
             };
             // first score tiles
-            if (ok && n_tiles > 0) ok = mbar_wait(BAR(B_KFULL + 0), 0, abort_flag);
+            if (ok && n_tiles > 0) ok = mbar_wait_w(BAR(B_KFULL + 0), 0, abort_flag);
             if (ok && n_tiles > 0) {
                 tc_fence_after();
                 for (int x = 0; x < HP; ++x) issue_s(x, sStage);
@@ -373,41 +293,31 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
                 const int s1 = (j + 1) % Cfg::NS;
                 const uint32_t sK1 = sStage + s1 * Cfg::STAGE_BYTES;
                 for (int x = 0; x < HP && ok; ++x) {
-                    if (Cfg::PSEP) {
-                        // next scores first: they only need the softmax to have read S_x(j)
-                        if (j + 1 < n_tiles) {
-                            if (x == 0) ok = mbar_wait(BAR(B_KFULL + s1), ((j + 1) / Cfg::NS) & 1, abort_flag);
-                            if (ok) ok = mbar_wait(BAR(B_SFREE + x), j & 1, abort_flag);
-                            if (!ok) break;
-                            tc_fence_after();
-                            issue_s(x, sK1);
-                        }
-                    }
-                    if (x == 0) ok = mbar_wait(BAR(B_VFULL + s), (j / Cfg::NS) & 1, abort_flag);
-                    if (ok) ok = mbar_wait(BAR(B_P + x), j & 1, abort_flag);
+                    if (x == 0) ok = mbar_wait_w(BAR(B_VFULL + s), (j / Cfg::NS) & 1, abort_flag);
+                    if (ok) ok = mbar_wait_w(BAR(B_P + x), j & 1, abort_flag);
                     if (!ok) break;
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)  // V k-step: 16 keys = 16 rows of 128 bytes
-                        mma_ts(tmem + Cfg::o_col(x), tmem + Cfg::p_col(x) + kk * 8, dv + (uint64_t)(kk * 128), ID_PV,
+                        mma_ts_w(tmem_w + Cfg::o_col(x), tmem_w + Cfg::p_col(x) + kk * 8, dv + (uint64_t)(kk * 128), ID_PV,
                                (LOCAL && j == 0 && kk == 0) ? 0u : 1u);  // LOCAL: the first PV starts O
-                    mma_commit(BAR(B_O + x));
-                    if (!Cfg::PSEP && j + 1 < n_tiles) {
+                    mma_commit_w(BAR(B_O + x));
+                    if (j + 1 < n_tiles) {
                         // P_x(j) lives over S_x: the next scores wait for PV_x(j) (in-order issue)
-                        if (x == 0) ok = mbar_wait(BAR(B_KFULL + s1), ((j + 1) / Cfg::NS) & 1, abort_flag);
+                        if (x == 0) ok = mbar_wait_w(BAR(B_KFULL + s1), ((j + 1) / Cfg::NS) & 1, abort_flag);
                         if (!ok) break;
                         tc_fence_after();
                         issue_s(x, sK1);
                     }
                 }
-                if (ok) mma_commit(BAR(B_KVEMPTY + s));
+                if (ok) mma_commit_w(BAR(B_KVEMPTY + s));
             }
             if (!ok) {
                 *abort_flag = 1;
-                report(p.err, DEV_ERR_TIMEOUT);
+                if (lane == 0) report(p.err, DEV_ERR_TIMEOUT);
             }
             // drain every MMA this thread issued before TMEM is released
-            mma_commit(BAR(B_DRAIN));
+            mma_commit_w(BAR(B_DRAIN));
             mbar_wait_drain(BAR(B_DRAIN), 0, 100000000ull);
         }
     }
@@ -437,8 +347,6 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
             }
             // ---- prologue: phi(q) from Y = Q Wq^T
             ok = warp_all(mbar_wait(BAR(B_QFULL), 0, abort_flag) && mbar_wait(BAR(B_Y + x), 0, abort_flag));
-            if (lane == 0) trace_word(p.trace, 2 + warp, ok ? 1 : 0xBAD1);
-            if (threadIdx.x % 128 == 0) trace_time(p.trace, x, 63, 0);  // Y ready
             float y[DF];
             if (ok) {
                 tc_fence_after();
@@ -497,8 +405,6 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
             }
             tc_fence_before();
             mbar_arrive(BAR(B_PHI + x));
-            if (lane == 0) trace_word(p.trace, 2 + warp, 2);
-            if (threadIdx.x % 128 == 0) trace_time(p.trace, x, 63, 1);  // phi(q) written
             // ---- fold the window part (o_A, lse_A) into O = phi(q) S_t^T under one normaliser
             // the window part's row is loaded while phi(q) S_t^T runs
             const bool valid = i < p.N;
@@ -510,7 +416,6 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
                 for (int v = 0; v < DH / 8; ++v) oa[v] = valid ? orow[v] : make_uint4(0, 0, 0, 0);
             }
             ok = warp_all(ok && mbar_wait(BAR(B_PRO), 0, abort_flag));
-            if (threadIdx.x % 128 == 0) trace_time(p.trace, x, 63, 2);  // phi(q) S_t^T done
             if (ok) {
                 tc_fence_after();
                 const float M = bden > 0.f ? fmaxf(lse_a, __log2f(bden)) : lse_a;
@@ -536,7 +441,6 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
                 }
                 tmem_wait_st();
                 m_run = M;
-                if (threadIdx.x % 128 == 0) trace_time(p.trace, x, 63, 3);  // window part folded
                 l_run = wa + bden * wb;
             }
         }
@@ -544,10 +448,7 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
         // ---- main loop over key tiles
         for (int j = 0; ok && j < n_tiles; ++j) {
             ok = warp_all(mbar_wait(BAR(B_S + x), j & 1, abort_flag));
-            if (lane == 0) trace_word(p.trace, 2 + warp, (ok ? 0x100u : 0xB00u) + 0x10u * j + 1);
             if (!ok) break;
-            if (threadIdx.x % 128 == 0) trace_time(p.trace, x, j, 0);
-            if (threadIdx.x == 0 && j == 0) trace_word(p.trace, 11, (unsigned)clock());
             tc_fence_after();
             float sv[128];
 #pragma unroll
@@ -558,10 +459,6 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
                 for (int e = 0; e < 32; ++e) sv[c * 32 + e] = __uint_as_float(u[e]);
             }
             tmem_wait_ld();
-            if (Cfg::PSEP) {
-                tc_fence_before();
-                mbar_arrive(BAR(B_SFREE + x));  // S_x may now take the next tile's scores
-            }
             // masks, only on the tiles that need them (warp-uniform test): LOCAL the causal diagonal
             // tile, PREFIX the ragged last tile of the kept rows
             const bool diag = LOCAL && j == n_tiles - 1;
@@ -577,29 +474,14 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
                 for (int c = 0; c < 128; ++c)
                     if (c >= limit) sv[c] = -INFINITY;
             }
-            // row max: four chains of 3-input max over 32 columns each (sv[32k .. 32k+31])
-            float mxc[4];
-#pragma unroll
-            for (int k4 = 0; k4 < 4; ++k4) {
-                float mv = fmax3(sv[32 * k4], sv[32 * k4 + 1], sv[32 * k4 + 2]);
-#pragma unroll
-                for (int c = 32 * k4 + 3; c + 1 < 32 * k4 + 32; c += 2) mv = fmax3(mv, sv[c], sv[c + 1]);
-                mxc[k4] = fmaxf(mv, sv[32 * k4 + 31]);
-            }
-            const float mnew = fmax3(mxc[0], mxc[1], fmaxf(mxc[2], mxc[3])) * p.scale_log2;
-            if (threadIdx.x % 128 == 0) trace_time(p.trace, x, j, 1);
-            // Lazy rescale: a row moves its reference max only when the max grows by more than 2^8.
+            const float mnew = row_max128(sv) * p.scale_log2;
+            // Lazy rescale: a row moves its reference max only when the max grows by more than
+            // kRescaleLog2 (see tc_tile.cuh).
             // The O rescale uses warp-collective tcgen05.ld/st, so the warp takes it together when
             // any of its rows needs it (rows that do not keep alpha = 1).
-            const bool need = mnew > m_run + 8.0f;
+            const bool need = mnew > m_run + kRescaleLog2;
             const float alpha = need ? ex2(m_run - mnew) : 1.f;
             const bool touch_o = need && m_run != -INFINITY;  // O holds nothing yet while m_run = -inf
-            if (Cfg::PSEP && j > 0) {
-                // PV_x(j-1) must be done: it still reads P_x, and O is about to be rescaled
-                ok = warp_all(mbar_wait(BAR(B_O + x), (j - 1) & 1, abort_flag));
-                if (!ok) break;
-                tc_fence_after();
-            }
             if (__any_sync(0xffffffffu, touch_o)) {
                 ok = warp_all(j == 0 ? (LOCAL || mbar_wait(BAR(B_PRO), 0, abort_flag))
                                      : mbar_wait(BAR(B_O + x), (j - 1) & 1, abort_flag));
@@ -622,13 +504,6 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
                 bs *= alpha;
                 m_run = mnew;
             }
-            // Two heads per CTA: the warpgroups take turns on the exponential units, so one
-            // warpgroup's exponentials overlap the other head's MMAs instead of contending with them.
-            if (HP == 2 && kMergeTurns && (x == 1 || j > 0)) {
-                ok = warp_all(mbar_wait(BAR(B_TURN + x), (x == 1 ? j : j - 1) & 1, abort_flag));
-                if (!ok) break;
-            }
-            if (threadIdx.x % 128 == 0) trace_time(p.trace, x, j, 2);
             // LOCAL band tiles: keys kstart + c; the band of row r is [i-w+1, i-1]
             int btype = 0;  // 0 none, 1 whole tile, 2 columns c > r, 3 columns c < r
             if (LOCAL) {
@@ -645,22 +520,15 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
             } else {
                 exp_tile<EXPV, false>(sv, p.scale_log2, m_run, tP, ls0, ls1, bsum, 0, 0);
             }
-            if (HP == 2 && kMergeTurns) mbar_arrive(BAR(B_TURN + (x ^ 1)));
-            if (threadIdx.x % 128 == 0) trace_time(p.trace, x, j, 3);
             l_run += ls0 + ls1;
             if (btype == 1) bs += ls0 + ls1;
             else if (btype >= 2) bs += bsum;
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(BAR(B_P + x));
-            if (threadIdx.x % 128 == 0) trace_time(p.trace, x, j, 4);
-            else if (lane == 0) trace_time(p.trace, x, j, 4 + (warp & 3));  // warps 1..3 of the group
-            if (lane == 0) trace_word(p.trace, 2 + warp, 0x100u + 0x10u * j + 2);
         }
         // ---- epilogue: o = O / l
-        if (threadIdx.x == 0) trace_word(p.trace, 12, (unsigned)clock());
         ok = warp_all(ok && (n_tiles > 0 ? mbar_wait(BAR(B_O + x), (n_tiles - 1) & 1, abort_flag) : true));
-        if (lane == 0) trace_word(p.trace, 2 + warp, ok ? 0xE00 : 0xBADE);
         if (ok) {
             tc_fence_after();
             const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
@@ -711,10 +579,7 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (threadIdx.x == 0) trace_word(p.trace, 13, (unsigned)clock());
-    if (threadIdx.x == 0) trace_word(p.trace, 14, 0xD0E);
     if (warp == Cfg::MMA_WARP) tmem_dealloc(tmem, Cfg::TMEM_COLS);
-    if (threadIdx.x == 0) trace_word(p.trace, 15, 0xF1F);
 }
 
 // ------------------------------------------------------------------ banded saliency
@@ -1256,7 +1121,11 @@ __global__ void transpose_wq_kernel(const __nv_bfloat16 *__restrict__ wq, __nv_b
     }
 }
 
+}  // namespace
+
 // ------------------------------------------------------------------ host side
+namespace tc {
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -1286,8 +1155,8 @@ bool make_map(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-}  // namespace
-unsigned *debug_trace_words();
+}  // namespace tc
+
 namespace {
 
 template <int DH, int DF, int HP>
@@ -1329,9 +1198,6 @@ cudaError_t launch_merge_cfg(int mode, const Dims &s, const MergeOperands &a, un
     prm.n_qtiles = n_qtiles;
     prm.qt_first = qt_first;
     prm.pairs = s.G() / HP;
-    prm.trace = debug_trace_words();
-    if (prm.trace && mode != kMergeLocal)  // the prefix phase records after the window phase's words
-        prm.trace += 16u * (unsigned)n_qtiles * s.B * s.Hkv * prm.pairs + 2048u + 32u;
     auto kern = mode == kMergeLocal ? merge_tc_kernel<DH, DF, HP, kMergeExpVariant, kMergeLocal>
                                     : merge_tc_kernel<DH, DF, HP, kMergeExpVariant, kMergePrefix>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
@@ -1343,9 +1209,6 @@ cudaError_t launch_merge_cfg(int mode, const Dims &s, const MergeOperands &a, un
 
 }  // namespace
 
-static unsigned *g_debug_trace = nullptr;
-unsigned *debug_trace_words() { return g_debug_trace; }
-void set_debug_trace_words(unsigned *p) { g_debug_trace = p; }
 
 bool tc_merge_supported(const Dims &s) {
     return s.bf16 && s.w > 0 && (s.d == 64 || s.d == 128) && (s.D == 64 || s.D == 128) && s.C % 128 == 0 &&
@@ -1408,18 +1271,18 @@ cudaError_t launch_linear_tc(const Dims &s, const void *k, const void *v, const 
     return cudaErrorNotSupported;
 }
 
+cudaError_t launch_merge_ring(int mode, const Dims &s, const MergeOperands &a, unsigned *err, cudaStream_t st);
+
 // mode 0: window part + Self-Saliency Score (writes o_A, lse_A, sigma); mode 1: kept prefix + linear
-// branch folded with the window part (writes o).
+// branch folded with the window part (writes o).  Head dimension 64 runs the persistent ring-scheduled
+// kernel (merge_ring.cu), 128 the kernel above.
 cudaError_t launch_merge_tc(int mode, const Dims &s, const MergeOperands &a, unsigned *err, cudaStream_t st) {
+    if (s.d == 64) return launch_merge_ring(mode, s, a, err, st);
     const bool pair = s.G() % 2 == 0;
-#define STILL_MERGE_CASE(DH, DF)                                                                     \
-    if (s.d == DH && s.D == DF)                                                                      \
-        return pair ? launch_merge_cfg<DH, DF, 2>(mode, s, a, err, st) : launch_merge_cfg<DH, DF, 1>(mode, s, a, err, st);
-    STILL_MERGE_CASE(64, 64)
-    STILL_MERGE_CASE(128, 128)
-    STILL_MERGE_CASE(64, 128)
-    STILL_MERGE_CASE(128, 64)
-#undef STILL_MERGE_CASE
+    if (s.d == 128 && s.D == 128)
+        return pair ? launch_merge_cfg<128, 128, 2>(mode, s, a, err, st) : launch_merge_cfg<128, 128, 1>(mode, s, a, err, st);
+    if (s.d == 128 && s.D == 64)
+        return pair ? launch_merge_cfg<128, 64, 2>(mode, s, a, err, st) : launch_merge_cfg<128, 64, 1>(mode, s, a, err, st);
     return cudaErrorNotSupported;
 }
 

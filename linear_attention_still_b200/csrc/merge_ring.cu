@@ -1,0 +1,703 @@
+// merge_ring.cu -- the hybrid merge of "STILL: Selecting Tokens for Intra-Layer Hybrid Attention to
+// Linearize LLMs" at head dimension 64 on sm_100a ([p1] jsqmd.com introduction: kept tokens go to
+// softmax attention and the rest to linear attention in the same layer, under one shared distribution;
+// [p4] atlas.scime.ai "Approach").  Same arithmetic and the same two phases as the head-dim-128 merge
+// in kernels_tc.cu; what differs is the schedule:
+//
+// * Persistent CTAs.  The grid holds one CTA per SM; each walks work items (b, g, head pair, 128
+//   queries of one chunk), heaviest query tiles first, CTA c taking items c, c + grid, ...  The producer
+//   loads the next item's query tiles (double-buffered) while the current item computes, and the MMA
+//   warp issues the next item's first score tile while the softmax warps run the current epilogue.
+// * A ring of TMEM slots per head.  Three slots of 64 columns: the scores of global tile J (128 keys,
+//   fp32) occupy slots J%3 and (J+1)%3, and its probabilities (bf16 pairs) are written over slot J%3.
+//   The next tile's scores go to slots (J+1)%3 and (J+2)%3: the first was freed when the softmax read
+//   tile J, the second held P(J-1), whose P V product the MMA warp issued earlier (tcgen05.mma from one
+//   thread executes in issue order).  So a softmax warpgroup never waits for a P V product before it
+//   writes P, only before the rare O rescale and the epilogue.  2 heads x (3 x 64) + 2 x 64 (O) = 512
+//   columns.
+//
+// Per row (TMEM lane = query row), as in the head-dim-128 kernel:
+//   window phase (kMergeLocal): keys [max(0,(t-m)C), i]; also the Self-Saliency Score of every row
+//     ([p1] "Self-Saliency Score") from the same exponentials; writes o_A, lse_A (log2) and sigma;
+//   prefix phase (kMergePrefix): prologue Y = Q Wq^T -> phi(q) = ||q|| e/||e||, O := phi(q) S_t^T,
+//     b := phi(q).z_t, folded with o_A under one normaliser ([p1] "NP-Map"); then the kept rows of the
+//     decided chunks ([p1] "Chunk-Wise parallel + delayed selection").
+// Every mbarrier wait is bounded; on a timeout the CTA records DEV_ERR_TIMEOUT, drains its own copies
+// and MMAs, frees TMEM and returns.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "still_internal.h"
+#include "tc_ptx.cuh"
+#include "tc_tile.cuh"
+
+namespace still {
+
+using namespace tc;
+
+namespace {
+
+template <int DF, int HP>
+struct RingCfg {
+    static constexpr int DH = 64;
+    static constexpr int BN = 128;                       // keys per tile
+    static constexpr int TILE_BYTES = 128 * 128;         // 128 rows x 64 bf16: one SW128 region
+    static constexpr int Q_BYTES = HP * TILE_BYTES;      // one item's query tiles
+    static constexpr int NQ = 2;                         // query buffers
+    static constexpr int NS = DF == 64 ? 4 : 3;          // K/V stages
+    static constexpr int STAGE_BYTES = 2 * TILE_BYTES;   // K + V
+    static constexpr int WQ_BYTES = DF * DH * 2;         // Wq^T of one head: DF rows x 64
+    static constexpr int ST_BYTES = DH * DF * 2;         // S_t^T: 64 rows x DF
+    static constexpr int W_BYTES = HP * WQ_BYTES + ST_BYTES;
+    static constexpr int BAR_BYTES = 512;
+    static constexpr int SMEM = NQ * Q_BYTES + NS * STAGE_BYTES + W_BYTES + BAR_BYTES + 1024;
+    static_assert(SMEM <= 232448, "shared memory");
+    static constexpr int THREADS = HP == 2 ? 384 : 192;
+    static constexpr int PRODUCER_WARP = 4 * HP, MMA_WARP = 4 * HP + 1;
+    // launch budget 384 x 168 = 64512 registers = 2 x 128 x 208 (softmax) + 128 x 88 (the rest)
+    static constexpr int REG_SOFTMAX = 208, REG_OTHER = 88;
+    static_assert(HP != 2 || 2 * 128 * REG_SOFTMAX + 128 * REG_OTHER <= THREADS * 168, "register split");
+    static constexpr int TMEM_COLS = HP == 2 ? 512 : 256;
+    __host__ __device__ static constexpr uint32_t ring(int x) { return 192u * x; }
+    __host__ __device__ static constexpr uint32_t o_col(int x) { return 192u * HP + 64u * x; }
+    static_assert(256 * HP <= TMEM_COLS, "TMEM budget");
+    // barrier slots
+    static constexpr int B_QFULL = 0, B_QEMPTY = 2, B_WFULL = 4, B_WEMPTY = 5, B_PRO = 6, B_DRAIN = 7;
+    static constexpr int B_KFULL = 8, B_VFULL = 8 + NS, B_KVEMPTY = 8 + 2 * NS;
+    static constexpr int B_Y = 8 + 3 * NS, B_PHI = B_Y + HP, B_S = B_PHI + HP, B_SFREE = B_S + HP,
+                         B_O = B_SFREE + HP, B_P = B_O + HP;  // B_P: [2 * HP], tile parity fastest
+    static constexpr int NUM_BARS = B_P + 2 * HP;
+    static constexpr int TMEM_SLOT_OFF = 8 * NUM_BARS;
+    static constexpr int ABORT_OFF = TMEM_SLOT_OFF + 8;
+    static_assert(ABORT_OFF + 8 <= BAR_BYTES, "barrier area overflow");
+};
+
+struct RingParams {
+    int B, H, Hkv, N, C, k, w, G, T;
+    float scale_log2;      // tau * log2(e)
+    const float *z;        // [B*Hkv*(T+1), DF] fp32
+    __nv_bfloat16 *o;      // [B,H,N,64]: window part (normalised) after LOCAL, final output after PREFIX
+    float *lse;            // [B,H,N]: log2-sum-exp of the window part (LOCAL writes, PREFIX reads)
+    float *sigma;          // [B,H,N]: Self-Saliency Score per query head (LOCAL writes)
+    int *fix_list;         // rows whose band sum underflowed against the window max (recomputed later)
+    unsigned *fix_count;
+    unsigned *err;
+    int n_qtiles;          // ceil(N/128)
+    int n_items;           // (n_qtiles - qt_first) x B x Hkv x pairs
+    int pairs;             // G / HP
+    int stall;             // test hook: CTA 0's producer issues no key/value tile (its consumers time out)
+};
+
+// Work item `it` (heaviest query tiles first).
+struct Item {
+    int b, bg, h0, i0, t, lo, nk, n_tiles, tslot;
+};
+
+template <int HP, bool LOCAL>
+__device__ __forceinline__ Item item_of(int it, const RingParams &p) {
+    Item I;
+    const int per_qt = p.B * p.Hkv * p.pairs;
+    const int qt = p.n_qtiles - 1 - it / per_qt;
+    const int rem = it % per_qt;
+    const int pair = rem % p.pairs;
+    I.bg = rem / p.pairs;
+    I.b = I.bg / p.Hkv;
+    const int g = I.bg % p.Hkv;
+    I.h0 = g * p.G + pair * HP;
+    I.i0 = qt * 128;
+    I.t = I.i0 / p.C;
+    const int m = p.w / p.C;
+    I.nk = p.k * max(0, I.t - m);                 // kept rows seen by this chunk
+    I.lo = max(0, (I.t - m) * p.C);               // window start
+    I.n_tiles = LOCAL ? (I.i0 - I.lo) / 128 + 1 : (I.nk + 127) / 128;
+    I.tslot = I.bg * (p.T + 1) + I.t;             // linear state slot
+    return I;
+}
+
+constexpr int kRingExpVariant = 1;  // see exp_tile: 1 = every exponential on the MUFU unit
+
+template <int DF, int HP, int EXPV, int MODE>
+__global__ void __launch_bounds__(RingCfg<DF, HP>::THREADS, 1)
+    merge_ring_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+                      const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_kh,
+                      const __grid_constant__ CUtensorMap map_vh, const __grid_constant__ CUtensorMap map_wq,
+                      const __grid_constant__ CUtensorMap map_st, const RingParams p) {
+    using Cfg = RingCfg<DF, HP>;
+    constexpr bool LOCAL = MODE == 0;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t sQ = sbase;                                      // NQ x HP query tiles
+    const uint32_t sStage = sQ + Cfg::NQ * Cfg::Q_BYTES;            // NS x (K tile, V tile)
+    const uint32_t sW = sStage + Cfg::NS * Cfg::STAGE_BYTES;        // HP x Wq^T, then S_t^T
+    uint8_t *bar_area = smem + Cfg::NQ * Cfg::Q_BYTES + Cfg::NS * Cfg::STAGE_BYTES + Cfg::W_BYTES;
+    const uint32_t sBar = smem_u32(bar_area);
+    auto BAR = [&](int i) { return sBar + 8u * i; };
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_area + Cfg::TMEM_SLOT_OFF);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bar_area + Cfg::ABORT_OFF);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int e = 0; e < 2; ++e) {
+            mbar_init(BAR(Cfg::B_QFULL + e), 1);
+            mbar_init(BAR(Cfg::B_QEMPTY + e), LOCAL ? 1 : 1 + 128 * HP);  // MMA commit (+ the softmax's ||q|| read)
+        }
+        mbar_init(BAR(Cfg::B_WFULL), 1);
+        mbar_init(BAR(Cfg::B_WEMPTY), 1);
+        mbar_init(BAR(Cfg::B_PRO), 1);
+        mbar_init(BAR(Cfg::B_DRAIN), 1);
+        for (int s = 0; s < Cfg::NS; ++s) {
+            mbar_init(BAR(Cfg::B_KFULL + s), 1);
+            mbar_init(BAR(Cfg::B_VFULL + s), 1);
+            mbar_init(BAR(Cfg::B_KVEMPTY + s), 1);
+        }
+        for (int x = 0; x < HP; ++x) {
+            mbar_init(BAR(Cfg::B_Y + x), 1);
+            mbar_init(BAR(Cfg::B_PHI + x), 128);
+            mbar_init(BAR(Cfg::B_S + x), 1);
+            mbar_init(BAR(Cfg::B_SFREE + x), 128);
+            mbar_init(BAR(Cfg::B_O + x), 1);
+            mbar_init(BAR(Cfg::B_P + 2 * x), 128);
+            mbar_init(BAR(Cfg::B_P + 2 * x + 1), 128);
+        }
+        *abort_flag = 0;
+        mbar_fence_init();
+    }
+    if (warp == Cfg::MMA_WARP) {
+        tmem_alloc(smem_u32(tmem_slot), Cfg::TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (warp == Cfg::PRODUCER_WARP && lane == 0) {
+        tma_prefetch_desc(&map_q);
+        tma_prefetch_desc(LOCAL ? &map_k : &map_kh);
+        tma_prefetch_desc(LOCAL ? &map_v : &map_vh);
+        if (!LOCAL) {
+            tma_prefetch_desc(&map_wq);
+            tma_prefetch_desc(&map_st);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp >= 4 * HP) {
+        if (HP == 2) setmaxnreg_dec<Cfg::REG_OTHER>();
+        if (warp == Cfg::PRODUCER_WARP) {
+            // (the whole warp runs the issue loop; one elected lane issues each copy)
+            // ================================================================ TMA producer
+            bool ok = true, stalled = false;
+            int G = 0, n = 0, nq = 0, nw = 0;  // K/V tiles, items, query loads, W loads issued
+            for (int it = blockIdx.x; ok && !stalled && it < p.n_items; it += gridDim.x, ++n) {
+                const Item I = item_of<HP, LOCAL>(it, p);
+                const int qb = n & 1;
+                if (n >= 2 && !(ok = mbar_wait_w(BAR(Cfg::B_QEMPTY + qb), ((n >> 1) - 1) & 1, abort_flag))) break;
+                mbar_arrive_expect_tx_w(BAR(Cfg::B_QFULL + qb), Cfg::Q_BYTES);
+                for (int x = 0; x < HP; ++x)
+                    tma_load_3d_w(sQ + qb * Cfg::Q_BYTES + x * Cfg::TILE_BYTES, &map_q, BAR(Cfg::B_QFULL + qb), 0, I.i0,
+                                I.b * p.H + I.h0 + x);
+                nq = n + 1;
+                if (!LOCAL) {
+                    if (n >= 1 && !(ok = mbar_wait_w(BAR(Cfg::B_WEMPTY), (n - 1) & 1, abort_flag))) break;
+                    mbar_arrive_expect_tx_w(BAR(Cfg::B_WFULL), Cfg::W_BYTES);
+                    for (int x = 0; x < HP; ++x)
+                        tma_load_3d_w(sW + x * Cfg::WQ_BYTES, &map_wq, BAR(Cfg::B_WFULL), 0, 0, I.h0 + x);
+                    for (int rr = 0; rr < DF / 64; ++rr)
+                        tma_load_3d_w(sW + HP * Cfg::WQ_BYTES + rr * (64 * 128), &map_st, BAR(Cfg::B_WFULL), rr * 64, 0,
+                                    I.tslot);
+                    nw = n + 1;
+                }
+                if (p.stall && blockIdx.x == 0) {
+                    stalled = true;  // no key/value tile: the MMA warp's bounded wait runs out
+                    break;
+                }
+                for (int jj = 0; jj < I.n_tiles; ++jj, ++G) {
+                    const int s = G % Cfg::NS;
+                    if (G >= Cfg::NS && !(ok = mbar_wait_w(BAR(Cfg::B_KVEMPTY + s), ((G / Cfg::NS) - 1) & 1, abort_flag)))
+                        break;
+                    const uint32_t sK = sStage + s * Cfg::STAGE_BYTES, sV = sK + Cfg::TILE_BYTES;
+                    const int row = LOCAL ? I.lo + jj * Cfg::BN : jj * Cfg::BN;
+                    mbar_arrive_expect_tx_w(BAR(Cfg::B_KFULL + s), Cfg::TILE_BYTES);
+                    tma_load_3d_w(sK, LOCAL ? &map_k : &map_kh, BAR(Cfg::B_KFULL + s), 0, row, I.bg);
+                    mbar_arrive_expect_tx_w(BAR(Cfg::B_VFULL + s), Cfg::TILE_BYTES);
+                    tma_load_3d_w(sV, LOCAL ? &map_v : &map_vh, BAR(Cfg::B_VFULL + s), 0, row, I.bg);
+                }
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                if (lane == 0) report(p.err, DEV_ERR_TIMEOUT);
+            }
+            if (!ok || stalled) {
+                // drain this CTA's copies still in flight
+                for (int u = max(0, nq - 2); u < nq; ++u)
+                    mbar_wait_drain(BAR(Cfg::B_QFULL + (u & 1)), (u >> 1) & 1, 100000000ull);
+                if (nw > 0) mbar_wait_drain(BAR(Cfg::B_WFULL), (nw - 1) & 1, 100000000ull);
+                for (int u = max(0, G - Cfg::NS); u < G; ++u) {
+                    mbar_wait_drain(BAR(Cfg::B_KFULL + u % Cfg::NS), (u / Cfg::NS) & 1, 100000000ull);
+                    mbar_wait_drain(BAR(Cfg::B_VFULL + u % Cfg::NS), (u / Cfg::NS) & 1, 100000000ull);
+                }
+            }
+        } else if (warp == Cfg::MMA_WARP) {
+            // (the whole warp runs the issue loop; one elected lane issues each MMA and commit)
+            const uint32_t tmem_w = __shfl_sync(0xffffffffu, tmem, 0);
+            // ================================================================ MMA issuer
+            constexpr uint32_t ID_N128 = idesc_bf16(128, 128, 0, 0);
+            constexpr uint32_t ID_N64 = idesc_bf16(128, 64, 0, 0);
+            constexpr uint32_t ID_PV = idesc_bf16(128, 64, 0, 1);
+            bool ok = true;
+            int J = 0, G = 0, n = 0;
+            // K-major k-step kk of a 64-column tile: 32 bytes per step inside the 128-byte row
+            auto kstep = [](int kk) -> uint64_t { return (uint64_t)((kk * 32) >> 4); };
+            // D[128 x nrows] = A[128 x 64] B[nrows x 64]^T into the ring slots of tile index Jt: columns
+            // 0..63 -> slot Jt%3, 64..127 -> slot (Jt+1)%3.  One N = 128 MMA per k-step where the two
+            // slots are adjacent and start on a 128-column boundary, else two N = 64 MMAs on the two
+            // halves of B's rows (each at a 64-column boundary).
+            auto issue_wide = [&](int x, int Jt, uint64_t da, uint32_t sB, int nrows) {
+                const int a = Jt % 3, bs = (Jt + 1) % 3;
+                const uint32_t col_a = Cfg::ring(x) + a * 64, col_b = Cfg::ring(x) + bs * 64;
+                const uint64_t db = sw128_desc(sB, 16, 1024);
+                if (nrows == 64) {
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) mma_ss_w(tmem_w + col_a, da + kstep(kk), db + kstep(kk), ID_N64, kk > 0);
+                } else if (col_b == col_a + 64 && (col_a & 127u) == 0) {
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) mma_ss_w(tmem_w + col_a, da + kstep(kk), db + kstep(kk), ID_N128, kk > 0);
+                } else {
+                    const uint64_t dbh = sw128_desc(sB + 64 * 128, 16, 1024);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        mma_ss_w(tmem_w + col_a, da + kstep(kk), db + kstep(kk), ID_N64, kk > 0);
+                        mma_ss_w(tmem_w + col_b, da + kstep(kk), dbh + kstep(kk), ID_N64, kk > 0);
+                    }
+                }
+            };
+            for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x, ++n) {
+                const Item I = item_of<HP, LOCAL>(it, p);
+                const int qb = n & 1;
+                uint64_t dq[HP];
+#pragma unroll
+                for (int x = 0; x < HP; ++x) dq[x] = sw128_desc(sQ + qb * Cfg::Q_BYTES + x * Cfg::TILE_BYTES, 16, 1024);
+                if (!(ok = mbar_wait_w(BAR(Cfg::B_QFULL + qb), (n >> 1) & 1, abort_flag))) break;
+                // the slots of tile J: the softmax has read tile J-1 (S or Y writes reuse its upper slot)
+                for (int x = 0; ok && x < HP && J > 0; ++x) ok = mbar_wait_w(BAR(Cfg::B_SFREE + x), (J - 1) & 1, abort_flag);
+                if (!ok) break;
+                if (!LOCAL) {
+                    // prologue: Y = Q Wq^T into the slots of tile J, phi(q) over its first slot, then
+                    // O := phi(q) S_t^T
+                    if (!(ok = mbar_wait_w(BAR(Cfg::B_WFULL), n & 1, abort_flag))) break;
+                    tc_fence_after();
+                    for (int x = 0; x < HP; ++x) {
+                        issue_wide(x, J, dq[x], sW + x * Cfg::WQ_BYTES, DF);
+                        mma_commit_w(BAR(Cfg::B_Y + x));
+                    }
+                    const uint32_t sST = sW + HP * Cfg::WQ_BYTES;
+                    for (int x = 0; ok && x < HP; ++x) {
+                        if (!(ok = mbar_wait_w(BAR(Cfg::B_PHI + x), n & 1, abort_flag))) break;
+                        tc_fence_after();
+#pragma unroll
+                        for (int kk = 0; kk < DF / 16; ++kk)
+                            mma_ts_w(tmem_w + Cfg::o_col(x), tmem_w + Cfg::ring(x) + (J % 3) * 64 + kk * 8,
+                                   kmajor_desc(sST, kk, 64 * 128), ID_N64, kk > 0);
+                    }
+                    if (!ok) break;
+                    mma_commit_w(BAR(Cfg::B_PRO));
+                    mma_commit_w(BAR(Cfg::B_WEMPTY));
+                }
+                if (I.n_tiles > 0) {
+                    if (!(ok = mbar_wait_w(BAR(Cfg::B_KFULL + G % Cfg::NS), (G / Cfg::NS) & 1, abort_flag))) break;
+                    tc_fence_after();
+                    for (int x = 0; x < HP; ++x) {
+                        issue_wide(x, J, dq[x], sStage + (G % Cfg::NS) * Cfg::STAGE_BYTES, 128);
+                        mma_commit_w(BAR(Cfg::B_S + x));
+                    }
+                }
+                for (int jj = 0; ok && jj < I.n_tiles; ++jj, ++G) {
+                    const int Jt = J + jj, s = G % Cfg::NS, s1 = (G + 1) % Cfg::NS;
+                    // next scores first: they need the softmax to have read S(Jt) (and P V(Jt-1), issued
+                    // before them, to have consumed P(Jt-1))
+                    if (jj + 1 < I.n_tiles) {
+                        for (int x = 0; x < HP; ++x) {
+                            if (x == 0 && !(ok = mbar_wait_w(BAR(Cfg::B_KFULL + s1), ((G + 1) / Cfg::NS) & 1, abort_flag)))
+                                break;
+                            if (!(ok = mbar_wait_w(BAR(Cfg::B_SFREE + x), Jt & 1, abort_flag))) break;
+                            tc_fence_after();
+                            issue_wide(x, Jt + 1, dq[x], sStage + s1 * Cfg::STAGE_BYTES, 128);
+                            mma_commit_w(BAR(Cfg::B_S + x));
+                        }
+                        if (!ok) break;
+                    }
+                    const uint64_t dv = sw128_desc(sStage + s * Cfg::STAGE_BYTES + Cfg::TILE_BYTES, Cfg::TILE_BYTES, 1024);
+                    for (int x = 0; x < HP; ++x) {
+                        if (x == 0 && !(ok = mbar_wait_w(BAR(Cfg::B_VFULL + s), (G / Cfg::NS) & 1, abort_flag))) break;
+                        if (!(ok = mbar_wait_w(BAR(Cfg::B_P + 2 * x + (Jt & 1)), (Jt >> 1) & 1, abort_flag))) break;
+                        tc_fence_after();
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk)  // 16 keys = 16 rows of V per k-step
+                            mma_ts_w(tmem_w + Cfg::o_col(x), tmem_w + Cfg::ring(x) + (Jt % 3) * 64 + kk * 8,
+                                   dv + (uint64_t)(kk * 128), ID_PV, (LOCAL && jj == 0 && kk == 0) ? 0u : 1u);
+                        mma_commit_w(BAR(Cfg::B_O + x));
+                    }
+                    if (!ok) break;
+                    mma_commit_w(BAR(Cfg::B_KVEMPTY + s));
+                }
+                if (!ok) break;
+                mma_commit_w(BAR(Cfg::B_QEMPTY + qb));
+                J += I.n_tiles;
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                if (lane == 0) report(p.err, DEV_ERR_TIMEOUT);
+            }
+            // drain every MMA this thread issued before TMEM is released
+            mma_commit_w(BAR(Cfg::B_DRAIN));
+            mbar_wait_drain(BAR(Cfg::B_DRAIN), 0, 100000000ull);
+        }
+    } else {
+        if (HP == 2) setmaxnreg_inc<Cfg::REG_SOFTMAX>();
+        // ================================================================ softmax warpgroups
+        const int x = warp >> 2;                       // head of the pair
+        const int r = (warp & 3) * 32 + lane;          // row in the tile = TMEM lane
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        const uint32_t tR = tmem + lane_off + Cfg::ring(x);
+        const uint32_t tO = tmem + lane_off + Cfg::o_col(x);
+        bool ok = true;
+        int J = 0, n = 0;
+        for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x, ++n) {
+            const Item I = item_of<HP, LOCAL>(it, p);
+            const int i = I.i0 + r;
+            const size_t row = ((size_t)I.b * p.H + I.h0 + x) * p.N + i;  // this thread's query row
+            const bool valid = i < p.N;
+            float m_run = -INFINITY, l_run = 0.f;
+            float bs = 0.f, sdiag = 0.f;  // LOCAL: band sum (same reference as l) and raw diagonal score
+
+            if constexpr (!LOCAL) {
+                // the window part of this row (o_A, written by the window phase) is read in the fold
+                if (valid) asm volatile("prefetch.global.L2 [%0];" ::"l"(p.o + row * 64));
+                const int qb = n & 1;
+                ok = warp_all(mbar_wait(BAR(Cfg::B_QFULL + qb), (n >> 1) & 1, abort_flag) &&
+                              mbar_wait(BAR(Cfg::B_Y + x), n & 1, abort_flag));
+                float y[DF];
+                const uint32_t ca = (J % 3) * 64, cb = ((J + 1) % 3) * 64;
+                if (ok) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int c = 0; c < DF / 32; ++c) {
+                        uint32_t u[32];
+                        tmem_ld32(tR + (c < 2 ? ca : cb) + (c & 1) * 32, u);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) y[c * 32 + e] = __uint_as_float(u[e]);
+                    }
+                }
+                // ||q||^2 from the swizzled query tile in shared memory
+                float qq = 0.f;
+                const uint8_t *qrow = smem + qb * Cfg::Q_BYTES + x * Cfg::TILE_BYTES + r * 128;
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    const uint4 u = *reinterpret_cast<const uint4 *>(qrow + ((ch ^ (r & 7)) << 4));
+                    const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = __bfloat1622float2(h2[e]);
+                        qq = fmaf(f.x, f.x, qq);
+                        qq = fmaf(f.y, f.y, qq);
+                    }
+                }
+                mbar_arrive(BAR(Cfg::B_QEMPTY + qb));  // this thread is done with the query tile
+                float ymax = -INFINITY;
+#pragma unroll
+                for (int c = 0; c < DF; ++c) ymax = fmaxf(ymax, y[c]);
+                float ee = 0.f;
+#pragma unroll
+                for (int c = 0; c < DF; ++c) {
+                    y[c] = ex2((y[c] - ymax) * kLog2e);
+                    ee = fmaf(y[c], y[c], ee);
+                }
+                const float f = sqrtf(qq) * rsqrtf(ee);
+                const float *zt = p.z + (size_t)I.tslot * DF;
+                float bden = 0.f;
+#pragma unroll
+                for (int c = 0; c < DF; ++c) {
+                    y[c] *= f;
+                    bden = fmaf(y[c], __ldg(zt + c), bden);
+                }
+                if (ok) {
+#pragma unroll
+                    for (int c = 0; c < DF / 64; ++c) {
+                        uint32_t u[32];
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) u[e] = pack_bf16x2(y[c * 64 + 2 * e], y[c * 64 + 2 * e + 1]);
+                        tmem_st32(tR + ca + c * 32, u);
+                    }
+                    tmem_wait_st();
+                }
+                tc_fence_before();
+                mbar_arrive(BAR(Cfg::B_PHI + x));
+                // fold the window part (o_A, lse_A) into O = phi(q) S_t^T under one normaliser; the
+                // window part's row is loaded while phi(q) S_t^T runs
+                const float lse_a = valid ? p.lse[row] : 0.f;
+                uint4 oa[8];
+                {
+                    const uint4 *orow = reinterpret_cast<const uint4 *>(p.o + row * 64);
+#pragma unroll
+                    for (int v = 0; v < 8; ++v) oa[v] = valid ? orow[v] : make_uint4(0, 0, 0, 0);
+                }
+                ok = warp_all(ok && mbar_wait(BAR(Cfg::B_PRO), n & 1, abort_flag));
+                if (ok) {
+                    tc_fence_after();
+                    const float M = bden > 0.f ? fmaxf(lse_a, __log2f(bden)) : lse_a;
+                    const float wa = ex2(lse_a - M), wb = ex2(-M);
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        uint32_t u[32];
+                        tmem_ld32(tO + c * 32, u);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int v4 = 0; v4 < 4; ++v4) {
+                            const uint4 w = oa[c * 4 + v4];
+                            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&ww[e]));
+                                const int q0 = 8 * v4 + 2 * e;
+                                u[q0] = __float_as_uint(fmaf(__uint_as_float(u[q0]), wb, a.x * wa));
+                                u[q0 + 1] = __float_as_uint(fmaf(__uint_as_float(u[q0 + 1]), wb, a.y * wa));
+                            }
+                        }
+                        tmem_st32(tO + c * 32, u);
+                    }
+                    tmem_wait_st();
+                    m_run = M;
+                    l_run = wa + bden * wb;
+                }
+            }
+
+            // ---- key tiles
+            for (int jj = 0; ok && jj < I.n_tiles; ++jj) {
+                const int Jt = J + jj;
+                ok = warp_all(mbar_wait(BAR(Cfg::B_S + x), Jt & 1, abort_flag));
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t ca = (Jt % 3) * 64, cb = ((Jt + 1) % 3) * 64;
+                float sv[128];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t u[32];
+                    tmem_ld32(tR + (c < 2 ? ca : cb) + (c & 1) * 32, u);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) sv[c * 32 + e] = __uint_as_float(u[e]);
+                }
+                tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(BAR(Cfg::B_SFREE + x));  // the slots may now take the next tile's scores
+                // masks, only on the tiles that need them (warp-uniform test): LOCAL the causal diagonal
+                // tile, PREFIX the ragged last tile of the kept rows
+                const bool diag = LOCAL && jj == I.n_tiles - 1;
+                const bool ragged = !LOCAL && I.nk - jj * Cfg::BN < Cfg::BN;
+                if (diag) {
+#pragma unroll
+                    for (int c = 0; c < 128; ++c)
+                        if (c == r) sdiag = sv[c];  // unrolled select keeps sv in registers
+                }
+                if (diag || ragged) {
+                    const int limit = diag ? r + 1 : I.nk - jj * Cfg::BN;
+#pragma unroll
+                    for (int c = 0; c < 128; ++c)
+                        if (c >= limit) sv[c] = -INFINITY;
+                }
+                const float mnew = row_max128(sv) * p.scale_log2;
+                // Lazy rescale: a row moves its reference max only when the max grows by more than
+                // kRescaleLog2 (see tc_tile.cuh).
+                // The O rescale uses warp-collective tcgen05.ld/st, so the warp takes it together when
+                // any of its rows needs it (rows that do not keep alpha = 1).
+                const bool need = mnew > m_run + kRescaleLog2;
+                const float alpha = need ? ex2(m_run - mnew) : 1.f;
+                const bool touch_o = need && m_run != -INFINITY;  // O holds nothing yet while m_run = -inf
+                if (__any_sync(0xffffffffu, touch_o)) {
+                    // P V(Jt-1) must be done before O is rescaled (the first tile of an item has no
+                    // P V in flight: the prologue's fold has completed)
+                    if (jj > 0) ok = warp_all(mbar_wait(BAR(Cfg::B_O + x), (Jt - 1) & 1, abort_flag));
+                    if (!ok) break;
+                    tc_fence_after();
+                    const float fa = touch_o ? alpha : 1.f;
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        uint32_t u[32];
+                        tmem_ld32(tO + c * 32, u);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * fa);
+                        tmem_st32(tO + c * 32, u);
+                    }
+                    tmem_wait_st();
+                }
+                if (need) {
+                    l_run *= alpha;
+                    bs *= alpha;
+                    m_run = mnew;
+                }
+                // LOCAL band tiles: keys kstart + c; the band of row r is [i-w+1, i-1]
+                int btype = 0;  // 0 none, 1 whole tile, 2 columns c > r, 3 columns c < r
+                if (LOCAL) {
+                    const int kstart = I.lo + jj * Cfg::BN;
+                    if (diag) btype = 3;
+                    else if (I.i0 >= p.w && kstart == I.i0 - p.w) btype = 2;
+                    else if (I.i0 >= p.w && kstart < I.i0 - p.w) btype = 0;
+                    else btype = 1;
+                }
+                float ls0, ls1, bsum = 0.f;
+                if (btype >= 2) {
+                    const int bc_lo = btype == 2 ? r + 1 : 0, bc_hi = btype == 2 ? 128 : r;
+                    exp_tile<EXPV, true>(sv, p.scale_log2, m_run, tR + ca, ls0, ls1, bsum, bc_lo, bc_hi);
+                } else {
+                    exp_tile<EXPV, false>(sv, p.scale_log2, m_run, tR + ca, ls0, ls1, bsum, 0, 0);
+                }
+                l_run += ls0 + ls1;
+                if (btype == 1) bs += ls0 + ls1;
+                else if (btype >= 2) bs += bsum;
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(BAR(Cfg::B_P + 2 * x + (Jt & 1)));
+            }
+            // ---- epilogue: o = O / l
+            ok = warp_all(ok && (I.n_tiles > 0 ? mbar_wait(BAR(Cfg::B_O + x), (J + I.n_tiles - 1) & 1, abort_flag)
+                                               : true));
+            if (ok) {
+                tc_fence_after();
+                const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+                __nv_bfloat16 *orow = p.o + row * 64;
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t u[32];
+                    tmem_ld32(tO + c * 32, u);
+                    tmem_wait_ld();
+                    if (valid) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
+#pragma unroll
+                        for (int v4 = 0; v4 < 4; ++v4) {
+                            uint4 w;
+                            w.x = pack_bf16x2(__uint_as_float(u[8 * v4 + 0]) * inv, __uint_as_float(u[8 * v4 + 1]) * inv);
+                            w.y = pack_bf16x2(__uint_as_float(u[8 * v4 + 2]) * inv, __uint_as_float(u[8 * v4 + 3]) * inv);
+                            w.z = pack_bf16x2(__uint_as_float(u[8 * v4 + 4]) * inv, __uint_as_float(u[8 * v4 + 5]) * inv);
+                            w.w = pack_bf16x2(__uint_as_float(u[8 * v4 + 6]) * inv, __uint_as_float(u[8 * v4 + 7]) * inv);
+                            dst[v4] = w;
+                        }
+                    }
+                }
+                if (LOCAL && valid) {
+                    p.lse[row] = m_run + __log2f(l_run);
+                    // sigma = softplus(s_ii - LSE_{band}) in natural units; +inf for an empty band (i = 0)
+                    float sig = INFINITY;
+                    if (i > 0) {
+                        if (bs > 0x1p-90f) {
+                            const float lse_band = (m_run + __log2f(bs)) * kLn2;
+                            sig = softplus_f(sdiag * (p.scale_log2 * kLn2) - lse_band);
+                        } else {
+                            // every band key sits > 90 binary orders below the window maximum: the
+                            // shared reference has underflowed the band sum; the row is rescored with
+                            // its own max
+                            p.fix_list[atomicAdd(p.fix_count, 1u)] = (int)row;
+                            sig = 0.f;
+                        }
+                    }
+                    p.sigma[row] = sig;
+                }
+            }
+            J += I.n_tiles;
+        }
+        if (!ok) {
+            *abort_flag = 1;
+            report(p.err, DEV_ERR_TIMEOUT);
+        }
+    }
+
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == Cfg::MMA_WARP) tmem_dealloc(tmem, Cfg::TMEM_COLS);
+}
+
+int sm_count() {
+    static int cached[128] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return 148;
+    if (!cached[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
+int g_stall = 0, g_max_ctas = 0;
+
+template <int DF, int HP>
+cudaError_t launch_ring_cfg(int mode, const Dims &s, const MergeOperands &a, unsigned *err, cudaStream_t st) {
+    using Cfg = RingCfg<DF, HP>;
+    const int T = s.T();
+    const int n_qtiles = (s.N + 127) / 128;
+    // PREFIX: only the query chunks t > m see a kept prefix or a linear state
+    const int qt_first = mode == 0 ? 0 : std::min(n_qtiles, (s.m() + 1) * s.C / 128);
+    if (qt_first >= n_qtiles) return cudaSuccess;
+    CUtensorMap mq, mk, mv, mkh, mvh, mw, ms;
+    const uint64_t khrows = (uint64_t)T * s.k > 0 ? (uint64_t)T * s.k : 1;
+    bool ok = make_map(&mq, a.q, 64, s.N, (uint64_t)s.B * s.H, 128) &&
+              make_map(&mk, a.k, 64, s.N, (uint64_t)s.B * s.Hkv, 128) &&
+              make_map(&mv, a.v, 64, s.N, (uint64_t)s.B * s.Hkv, 128) &&
+              make_map(&mkh, a.khat, 64, khrows, (uint64_t)s.B * s.Hkv, 128) &&
+              make_map(&mvh, a.vhat, 64, khrows, (uint64_t)s.B * s.Hkv, 128) &&
+              make_map(&mw, a.wqt, 64, DF, s.H, DF) &&
+              make_map(&ms, a.st_t, DF, 64, (uint64_t)s.B * s.Hkv * (T + 1), 64);
+    if (!ok) return cudaErrorInvalidValue;
+    RingParams prm;
+    prm.B = s.B;
+    prm.H = s.H;
+    prm.Hkv = s.Hkv;
+    prm.N = s.N;
+    prm.C = s.C;
+    prm.k = s.k;
+    prm.w = s.w;
+    prm.G = s.G();
+    prm.T = T;
+    prm.scale_log2 = s.scale * kLog2e;
+    prm.z = a.z;
+    prm.o = static_cast<__nv_bfloat16 *>(a.o);
+    prm.lse = a.lse;
+    prm.sigma = a.sigma;
+    prm.fix_list = a.fix_list;
+    prm.fix_count = a.fix_count;
+    prm.err = err;
+    prm.n_qtiles = n_qtiles;
+    prm.pairs = s.G() / HP;
+    prm.n_items = (n_qtiles - qt_first) * s.B * s.Hkv * prm.pairs;
+    prm.stall = g_stall;
+    auto kern = mode == 0 ? merge_ring_kernel<DF, HP, kRingExpVariant, 0> : merge_ring_kernel<DF, HP, kRingExpVariant, 1>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+    if (e != cudaSuccess) return e;
+    int ctas = std::min(prm.n_items, sm_count());
+    if (g_max_ctas > 0) ctas = std::min(ctas, g_max_ctas);
+    const unsigned grid = (unsigned)ctas;
+    kern<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(mq, mk, mv, mkh, mvh, mw, ms, prm);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+// Head dimension 64: mode 0 window part + Self-Saliency Score (writes o_A, lse_A, sigma); mode 1 kept
+// prefix + linear branch folded with the window part (writes o).
+cudaError_t launch_merge_ring(int mode, const Dims &s, const MergeOperands &a, unsigned *err, cudaStream_t st) {
+    if (s.d != 64) return cudaErrorNotSupported;
+    const bool pair = s.G() % 2 == 0;
+    if (s.D == 64) return pair ? launch_ring_cfg<64, 2>(mode, s, a, err, st) : launch_ring_cfg<64, 1>(mode, s, a, err, st);
+    if (s.D == 128)
+        return pair ? launch_ring_cfg<128, 2>(mode, s, a, err, st) : launch_ring_cfg<128, 1>(mode, s, a, err, st);
+    return cudaErrorNotSupported;
+}
+
+void set_merge_debug(int stall, int max_ctas) {
+    g_stall = stall;
+    g_max_ctas = max_ctas > 0 ? max_ctas : 0;
+}
+
+}  // namespace still

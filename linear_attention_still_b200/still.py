@@ -21,7 +21,7 @@ STATUS = {0: "STILL_OK", 1: "STILL_ERR_INVALID_ARG", 2: "STILL_ERR_UNSUPPORTED",
 EXPORTS = ("still_status_string", "still_saliency", "still_select_topk", "still_npmap",
            "still_prefill_workspace_bytes", "still_prefill_workspace_layout", "still_hybrid_prefill",
            "still_decode_state_bytes", "still_decode_init", "still_decode_step", "still_get_device_status",
-           "still_launch_count", "still_timing_enable", "still_timing_read", "still_debug_set_trace",
+           "still_launch_count", "still_timing_enable", "still_timing_read", "still_debug_merge",
            "still_hybrid_prefill_static", "still_diagonal_score", "still_backward_workspace_bytes",
            "still_hybrid_backward")
 
@@ -65,7 +65,7 @@ _SIG = {
     "still_get_device_status": ([_P], ct.c_int),
     "still_launch_count": ([], ct.c_uint64),
     "still_timing_enable": ([ct.c_int], ct.c_int),
-    "still_debug_set_trace": ([_P], None),
+    "still_debug_merge": ([ct.c_int, ct.c_int], None),
     "still_timing_read": ([ct.POINTER(ct.c_double), ct.POINTER(ct.c_int), ct.c_int], ct.c_int),
 }
 for _name, (_args, _res) in _SIG.items():
@@ -225,9 +225,11 @@ def still_launch_count() -> int:
     return int(_lib.still_launch_count())
 
 
-def still_debug_set_trace(words=None):
-    """Diagnostics: progress words of the tensor-core kernels go to `words` (pinned tensor or None)."""
-    _lib.still_debug_set_trace(_ptr(words))
+def still_debug_merge(stall: bool = False, max_ctas: int = 0):
+    """Test hooks of the head-dim-64 tensor-core merge: `stall` makes the first CTA of each later
+    launch load no key/value tile (its bounded wait runs out: STILL_ERR_TIMEOUT); `max_ctas` > 0 caps
+    the persistent grid.  Defaults restore normal operation."""
+    _lib.still_debug_merge(1 if stall else 0, int(max_ctas))
 
 
 TIMING_CLASSES = ("saliency", "topk_gather", "npmap", "linear_state", "merge", "state_export", "merge_prefix",

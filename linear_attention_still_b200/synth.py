@@ -125,11 +125,14 @@ class Inputs:
         return round_to_bf16(getattr(self, name))[1]
 
 
-def make_inputs(shape: Shape, seed: int | None = None, batches=None) -> Inputs:
+def make_inputs(shape: Shape, seed: int | None = None, batches=None, threads: int = 1) -> Inputs:
     """Draw the inputs for `shape` (Ntot = N + decode_steps tokens).
 
     batches: optional list of batch indices to draw (others are skipped); the
-    returned arrays then hold only those items, in the given order."""
+    returned arrays then hold only those items, in the given order.
+    threads: batch items drawn concurrently (each from its own stream, so the
+    values do not depend on it; numpy's generators release the GIL while they
+    fill an array)."""
     s = shape
     seed = s.seed if seed is None else seed
     ntot = s.N + s.decode_steps
@@ -145,7 +148,8 @@ def make_inputs(shape: Shape, seed: int | None = None, batches=None) -> Inputs:
     v = np.empty((nb, s.Hkv, ntot, s.d), dtype=f32)
     nh = min(s.n_heavy, max(ntot - 1, 0))
     heavy = np.zeros((nb, nh), dtype=np.int64)
-    for n, b in enumerate(bsel):
+
+    def draw(n: int, b: int) -> None:
         rng = np.random.Generator(np.random.PCG64(children[1 + b]))
         rng.standard_normal((s.H, ntot, s.d), dtype=f32, out=q[n])
         rng.standard_normal((s.Hkv, ntot, s.d), dtype=f32, out=k[n])
@@ -162,9 +166,20 @@ def make_inputs(shape: Shape, seed: int | None = None, batches=None) -> Inputs:
         q[n][:, pos, :] *= f32(4.0)
         k[n][:, pos, :] *= f32(4.0)
         v[n][:, pos, :] *= f32(4.0)
-    if s.dtype == "bf16":
-        for a in (q, k, v, wq, wk):
-            round_to_bf16_(a)
-    elif s.dtype != "f32":
+        if s.dtype == "bf16":
+            for a in (q[n], k[n], v[n]):
+                round_to_bf16_(a)
+
+    if s.dtype not in ("bf16", "f32"):
         raise ValueError(f"unknown dtype {s.dtype}")
+    if threads > 1 and nb > 1:
+        from concurrent.futures import ThreadPoolExecutor
+        with ThreadPoolExecutor(max_workers=min(threads, nb)) as ex:
+            list(ex.map(lambda nb_: draw(*nb_), enumerate(bsel)))
+    else:
+        for n, b in enumerate(bsel):
+            draw(n, b)
+    if s.dtype == "bf16":
+        for a in (wq, wk):
+            round_to_bf16_(a)
     return Inputs(s, q, k, v, wq, wk, heavy)
