@@ -735,9 +735,10 @@ def oracle_decode_sample(shape, seconds: float):
     return 1.0 / per_token, t_call, desc, nth
 
 
-def bench_decode(args, name, rank, world, local, cpu_seconds):
+def bench_decode(args, name, rank, world, local, cpu_seconds, all_steps=False):
     """One decode workload on this rank (prefill of the context, then timed decode steps); returns the
-    JSON line as a dict."""
+    JSON line as a dict.  all_steps: time every decode step left after the warm-up and end-to-end ones
+    (about one chunk cycle: C - 1 ordinary steps and the one that closes a chunk) instead of --steps."""
     import numpy as np
     import torch
 
@@ -746,7 +747,7 @@ def bench_decode(args, name, rank, world, local, cpu_seconds):
     N, steps, B = shape.N, shape.decode_steps, shape.B
     tdt = torch.bfloat16 if shape.dtype == "bf16" else torch.float32
     e2e_steps = min(args.e2e_steps, 20)
-    K = min(args.steps, steps - args.warmup - e2e_steps)
+    K = steps - args.warmup - e2e_steps if all_steps else min(args.steps, steps - args.warmup - e2e_steps)
     cap = N + steps
     dims = still.dims_of(shape)
     q = torch.empty(B, shape.H, N, shape.d, dtype=tdt, device="cuda")
@@ -1014,9 +1015,9 @@ def to_host_tensor(a, tdt):
     return torch.from_numpy(np.ascontiguousarray(a)).to(tdt)
 
 
-def bench_one(args, name, rank, world, local, cpu_seconds):
+def bench_one(args, name, rank, world, local, cpu_seconds, extra=False):
     if WORKLOADS[name].decode_steps > 0:
-        return bench_decode(args, name, rank, world, local, cpu_seconds)
+        return bench_decode(args, name, rank, world, local, cpu_seconds, all_steps=extra)
     if args.pass_ == "backward":
         return bench_backward(args, name, rank, world, local, cpu_seconds)
     return bench_prefill(args, name, rank, world, local, cpu_seconds)
@@ -1038,7 +1039,7 @@ def run_ours(args):
         line["workloads"] = {}
         for name in EXTRA_WORKLOADS:
             torch.cuda.empty_cache()
-            line["workloads"][name] = bench_one(args, name, rank, world, local, EXTRA_CPU_SECONDS)
+            line["workloads"][name] = bench_one(args, name, rank, world, local, EXTRA_CPU_SECONDS, extra=True)
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()

@@ -178,11 +178,20 @@ STILL_API still_status still_hybrid_prefill(const still_dims *dims, const void *
  * still_hybrid_prefill with its scratch in a fixed device array inside this
  * library instead of a caller workspace (no counterpart in the method: the
  * pages describe no memory management).  Same arguments, results and errors as
- * still_hybrid_prefill, minus workspace and workspace_bytes.  It allocates
- * nothing: no device, host or pinned memory, directly or through a library.
+ * still_hybrid_prefill, minus workspace and workspace_bytes: the same argument
+ * checks run first, in the same order, then the size limit below.  A call
+ * allocates nothing: no device, host or pinned memory, directly or through a
+ * library.
  *   - Limit: shapes with still_prefill_workspace_bytes(dims) greater than
  *     STILL_STATIC_WORKSPACE_BYTES (64 MiB) are rejected with
  *     STILL_ERR_WORKSPACE before any work; use still_hybrid_prefill for them.
+ *   - The 64 MiB array is reserved on a device when the library's module
+ *     holding it is loaded there: by default (lazy module loading) on the
+ *     first call of this entry point on that device, with
+ *     CUDA_MODULE_LOADING=EAGER when the process's context is created on it.
+ *     That reservation can fail for lack of device memory, which returns
+ *     STILL_ERR_CUDA; callers that must not allocate later should make one
+ *     warm-up call before entering their allocation-free loop.
  *   - Nothing in the array has to start at zero: each call writes every part of
  *     the scratch it reads (its counter of recomputed rows is reset by the call
  *     itself), so leftovers of earlier calls, of any shape, do no harm.
@@ -191,7 +200,8 @@ STILL_API still_status still_hybrid_prefill(const still_dims *dims, const void *
  *   - The array's address is looked up once per device, with that device
  *     current, on the first call there (which may load the library's module for
  *     it); make that first call before any stream capture.
- * STILL_ERR_CUDA if the current device or the array's address cannot be had.
+ * STILL_ERR_CUDA if the current device or the array's address cannot be had
+ * (device ordinals 128 and above are not supported).
  */
 #define STILL_STATIC_WORKSPACE_BYTES (64u << 20)
 STILL_API still_status still_hybrid_prefill_static(const still_dims *dims, const void *q, const void *k,
@@ -228,6 +238,24 @@ STILL_API still_status still_hybrid_backward(const still_dims *dims, const void 
  * tokens the state can hold.
  */
 STILL_API size_t still_decode_state_bytes(const still_dims *dims, int capacity);
+
+/*
+ * Byte offsets of the decode state's segments, for inspection (the kernels own
+ * the contents; a caller reads them only between calls on the stream).  Per
+ * (b, g), G = B*Hkv groups, cap_chunks = capacity / C:
+ *   khat, vhat  dtype [B,Hkv,cap_chunks*k,d]  kept rows of each closed chunk c at
+ *               rows [c*k, c*k+k), ascending positions
+ *   S, z        fp32 [B,Hkv,D,d], [B,Hkv,D]   linear state of the folded tokens
+ *   ring_k/v    dtype [B,Hkv,ring_rows,d]     rows of the last m+1 chunks
+ *   ring_r      fp32 [B,Hkv,ring_rows]        their group saliency scores
+ * Position j of the ring sits at row ((j / C) % (m+1)) * C + j % C
+ * (m = w / C; w = 0: row j % C); ring_rows = (m+1) * C (C when w = 0).
+ */
+typedef struct {
+    size_t header, khat, vhat, S, z, ring_k, ring_v, ring_r, total;
+    int ring_rows, cap_chunks;
+} still_state_layout;
+STILL_API still_status still_decode_state_layout(const still_dims *dims, int capacity, still_state_layout *out);
 
 /* Empty state at position 0. */
 STILL_API still_status still_decode_init(const still_dims *dims, int capacity, void *state, void *stream);

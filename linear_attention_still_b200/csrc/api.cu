@@ -305,6 +305,26 @@ size_t still_decode_state_bytes(const still_dims *dims, int capacity) {
     return decode_layout(s, capacity).total;
 }
 
+still_status still_decode_state_layout(const still_dims *dims, int capacity, still_state_layout *out) {
+    Dims s;
+    still_status st = check_dims(dims, &s, false);
+    if (st) return st;
+    if (capacity < 0 || capacity > (1 << 26) || !out) return STILL_ERR_INVALID_ARG;
+    const DecodeLayout L = decode_layout(s, capacity);
+    out->header = L.header;
+    out->khat = L.khat;
+    out->vhat = L.vhat;
+    out->S = L.S;
+    out->z = L.z;
+    out->ring_k = L.ring_k;
+    out->ring_v = L.ring_v;
+    out->ring_r = L.ring_r;
+    out->total = L.total;
+    out->ring_rows = L.ring_rows;
+    out->cap_chunks = L.cap_chunks;
+    return STILL_OK;
+}
+
 still_status still_decode_init(const still_dims *dims, int capacity, void *state, void *stream) {
     Dims s;
     still_status st = check_dims(dims, &s, false);
@@ -317,18 +337,39 @@ still_status still_decode_init(const still_dims *dims, int capacity, void *state
     return STILL_OK;
 }
 
-still_status still_hybrid_prefill(const still_dims *dims, const void *q, const void *k, const void *v, const void *Wq,
-                                  const void *Wk, void *o, const int32_t *idx_in, void *workspace,
-                                  size_t workspace_bytes, void *state, int state_capacity, void *stream) {
+}  // extern "C"
+
+namespace still {
+// Every check of still_hybrid_prefill except those of the workspace, in the order that call makes
+// them (dims, decode state, then the tensors); STILL_OK with *empty set when B * N == 0.
+still_status check_prefill_args(const still_dims *dims, const void *q, const void *k, const void *v, const void *Wq,
+                                const void *Wk, const void *o, const int32_t *idx_in, const void *state,
+                                int state_capacity, bool *empty) {
     Dims s;
     still_status st = check_dims(dims, &s);
     if (st) return st;
     if (state && (state_capacity < s.N || !aligned16(state))) return STILL_ERR_INVALID_ARG;
-    if ((long long)s.B * s.N == 0) return STILL_OK;
-    const void *ptrs[] = {q, k, v, Wq, Wk, o, workspace};
+    *empty = (long long)s.B * s.N == 0;
+    if (*empty) return STILL_OK;
+    const void *ptrs[] = {q, k, v, Wq, Wk, o};
     for (const void *p : ptrs)
         if (!p || !aligned16(p)) return STILL_ERR_INVALID_ARG;
     if (idx_in && !aligned16(idx_in)) return STILL_ERR_INVALID_ARG;
+    return STILL_OK;
+}
+}  // namespace still
+
+extern "C" {
+
+still_status still_hybrid_prefill(const still_dims *dims, const void *q, const void *k, const void *v, const void *Wq,
+                                  const void *Wk, void *o, const int32_t *idx_in, void *workspace,
+                                  size_t workspace_bytes, void *state, int state_capacity, void *stream) {
+    bool empty = false;
+    still_status st = check_prefill_args(dims, q, k, v, Wq, Wk, o, idx_in, state, state_capacity, &empty);
+    if (st || empty) return st;
+    if (!workspace || !aligned16(workspace)) return STILL_ERR_INVALID_ARG;
+    Dims s;
+    check_dims(dims, &s);
     const still_ws_layout W = ws_layout(s);
     if (workspace_bytes < W.total) return STILL_ERR_WORKSPACE;
     if (((uintptr_t)workspace & 255u) != 0) return STILL_ERR_INVALID_ARG;

@@ -8,13 +8,12 @@
 //   queries of one chunk), heaviest query tiles first, CTA c taking items c, c + grid, ...  The producer
 //   loads the next item's query tiles (double-buffered) while the current item computes, and the MMA
 //   warp issues the next item's first score tile while the softmax warps run the current epilogue.
-// * A ring of TMEM slots per head.  Three slots of 64 columns: the scores of global tile J (128 keys,
-//   fp32) occupy slots J%3 and (J+1)%3, and its probabilities (bf16 pairs) are written over slot J%3.
-//   The next tile's scores go to slots (J+1)%3 and (J+2)%3: the first was freed when the softmax read
-//   tile J, the second held P(J-1), whose P V product the MMA warp issued earlier (tcgen05.mma from one
-//   thread executes in issue order).  So a softmax warpgroup never waits for a P V product before it
-//   writes P, only before the rare O rescale and the epilogue.  2 heads x (3 x 64) + 2 x 64 (O) = 512
-//   columns.
+// * Scores, probabilities and output in separate TMEM columns per head: S (128 fp32 columns, one
+//   N = 128 MMA per k-step at a 128-column boundary), P (128 keys as bf16 pairs, 64 columns) and O (64):
+//   2 x (128 + 64 + 64) = 512 columns.  The next tile's scores are issued as soon as the softmax has
+//   read S; the softmax computes a tile's exponentials into registers and only then waits for the P V
+//   product that still reads the previous P (issued a whole exponential phase earlier, so normally
+//   done), rescales O if its max moved, and stores P.
 //
 // Per row (TMEM lane = query row), as in the head-dim-128 kernel:
 //   window phase (kMergeLocal): keys [max(0,(t-m)C), i]; also the Self-Saliency Score of every row
@@ -58,7 +57,8 @@ struct RingCfg {
     static constexpr int REG_SOFTMAX = 208, REG_OTHER = 88;
     static_assert(HP != 2 || 2 * 128 * REG_SOFTMAX + 128 * REG_OTHER <= THREADS * 168, "register split");
     static constexpr int TMEM_COLS = HP == 2 ? 512 : 256;
-    __host__ __device__ static constexpr uint32_t ring(int x) { return 192u * x; }
+    __host__ __device__ static constexpr uint32_t s_col(int x) { return 128u * x; }
+    __host__ __device__ static constexpr uint32_t p_col(int x) { return 128u * HP + 64u * x; }
     __host__ __device__ static constexpr uint32_t o_col(int x) { return 192u * HP + 64u * x; }
     static_assert(256 * HP <= TMEM_COLS, "TMEM budget");
     // barrier slots
@@ -66,7 +66,8 @@ struct RingCfg {
     static constexpr int B_KFULL = 8, B_VFULL = 8 + NS, B_KVEMPTY = 8 + 2 * NS;
     static constexpr int B_Y = 8 + 3 * NS, B_PHI = B_Y + HP, B_S = B_PHI + HP, B_SFREE = B_S + HP,
                          B_O = B_SFREE + HP, B_P = B_O + HP;  // B_P: [2 * HP], tile parity fastest
-    static constexpr int NUM_BARS = B_P + 2 * HP;
+    static constexpr int B_TURN = B_P + 2 * HP;                      // [2]: exponential-phase turns
+    static constexpr int NUM_BARS = B_TURN + 2;
     static constexpr int TMEM_SLOT_OFF = 8 * NUM_BARS;
     static constexpr int ABORT_OFF = TMEM_SLOT_OFF + 8;
     static_assert(ABORT_OFF + 8 <= BAR_BYTES, "barrier area overflow");
@@ -114,7 +115,14 @@ __device__ __forceinline__ Item item_of(int it, const RingParams &p) {
     return I;
 }
 
-constexpr int kRingExpVariant = 1;  // see exp_tile: 1 = every exponential on the MUFU unit
+constexpr int kRingExpVariant = 1;  // see exp_row: 1 = every exponential on the MUFU unit
+// Two heads per CTA: the softmax warpgroups take turns on the exponential phase of each tile (head 0,
+// head 1, head 0, ...), so one warpgroup's row bookkeeping (TMEM read of S, row max, P store) overlaps
+// the other's exponentials instead of both leaving the MUFU unit idle at the same time.
+#ifndef STILL_RING_TURNS
+#define STILL_RING_TURNS 1
+#endif
+constexpr bool kRingTurns = STILL_RING_TURNS != 0;
 
 template <int DF, int HP, int EXPV, int MODE>
 __global__ void __launch_bounds__(RingCfg<DF, HP>::THREADS, 1)
@@ -160,6 +168,8 @@ __global__ void __launch_bounds__(RingCfg<DF, HP>::THREADS, 1)
             mbar_init(BAR(Cfg::B_P + 2 * x), 128);
             mbar_init(BAR(Cfg::B_P + 2 * x + 1), 128);
         }
+        mbar_init(BAR(Cfg::B_TURN + 0), 128);
+        mbar_init(BAR(Cfg::B_TURN + 1), 128);
         *abort_flag = 0;
         mbar_fence_init();
     }
@@ -248,83 +258,90 @@ __global__ void __launch_bounds__(RingCfg<DF, HP>::THREADS, 1)
             int J = 0, G = 0, n = 0;
             // K-major k-step kk of a 64-column tile: 32 bytes per step inside the 128-byte row
             auto kstep = [](int kk) -> uint64_t { return (uint64_t)((kk * 32) >> 4); };
-            // D[128 x nrows] = A[128 x 64] B[nrows x 64]^T into the ring slots of tile index Jt: columns
-            // 0..63 -> slot Jt%3, 64..127 -> slot (Jt+1)%3.  One N = 128 MMA per k-step where the two
-            // slots are adjacent and start on a 128-column boundary, else two N = 64 MMAs on the two
-            // halves of B's rows (each at a 64-column boundary).
-            auto issue_wide = [&](int x, int Jt, uint64_t da, uint32_t sB, int nrows) {
-                const int a = Jt % 3, bs = (Jt + 1) % 3;
-                const uint32_t col_a = Cfg::ring(x) + a * 64, col_b = Cfg::ring(x) + bs * 64;
+            // D[128 x nrows] = A[128 x 64] B[nrows x 64]^T into the score columns of head x (nrows = 128:
+            // scores of a key tile; nrows = DF: Y = Q Wq^T of the prologue)
+            auto issue_qk = [&](int x, uint64_t da, uint32_t sB, int nrows) {
                 const uint64_t db = sw128_desc(sB, 16, 1024);
-                if (nrows == 64) {
+                const uint32_t id = nrows == 64 ? ID_N64 : ID_N128;
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) mma_ss_w(tmem_w + col_a, da + kstep(kk), db + kstep(kk), ID_N64, kk > 0);
-                } else if (col_b == col_a + 64 && (col_a & 127u) == 0) {
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) mma_ss_w(tmem_w + col_a, da + kstep(kk), db + kstep(kk), ID_N128, kk > 0);
-                } else {
-                    const uint64_t dbh = sw128_desc(sB + 64 * 128, 16, 1024);
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        mma_ss_w(tmem_w + col_a, da + kstep(kk), db + kstep(kk), ID_N64, kk > 0);
-                        mma_ss_w(tmem_w + col_b, da + kstep(kk), dbh + kstep(kk), ID_N64, kk > 0);
+                for (int kk = 0; kk < 4; ++kk) mma_ss_w(tmem_w + Cfg::s_col(x), da + kstep(kk), db + kstep(kk), id, kk > 0);
+            };
+            // The first MMA of an item that writes the score columns (LOCAL: the scores of its first key
+            // tile; PREFIX: Y = Q Wq^T) is issued during the previous item's last tile, right after the
+            // softmax has read that tile's scores, so it is ready when the softmax leaves the epilogue.
+            // `pre` marks an item whose first MMA was issued that way.
+            auto issue_head = [&](const Item &In, int nn, int Jn, int Gn) -> bool {
+                const int qbn = nn & 1;
+                if (!mbar_wait_w(BAR(Cfg::B_QFULL + qbn), (nn >> 1) & 1, abort_flag)) return false;
+                if (!LOCAL && !mbar_wait_w(BAR(Cfg::B_WFULL), nn & 1, abort_flag)) return false;
+                if (LOCAL && !mbar_wait_w(BAR(Cfg::B_KFULL + Gn % Cfg::NS), (Gn / Cfg::NS) & 1, abort_flag)) return false;
+                for (int x = 0; x < HP; ++x) {
+                    // the score columns: the softmax has read tile Jn-1
+                    if (Jn > 0 && !mbar_wait_w(BAR(Cfg::B_SFREE + x), (Jn - 1) & 1, abort_flag)) return false;
+                    tc_fence_after();
+                    const uint64_t dqn = sw128_desc(sQ + qbn * Cfg::Q_BYTES + x * Cfg::TILE_BYTES, 16, 1024);
+                    if (LOCAL) {
+                        issue_qk(x, dqn, sStage + (Gn % Cfg::NS) * Cfg::STAGE_BYTES, 128);
+                        mma_commit_w(BAR(Cfg::B_S + x));
+                    } else {
+                        issue_qk(x, dqn, sW + x * Cfg::WQ_BYTES, DF);
+                        mma_commit_w(BAR(Cfg::B_Y + x));
                     }
                 }
+                return true;
             };
+            bool pre = false;
             for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x, ++n) {
                 const Item I = item_of<HP, LOCAL>(it, p);
                 const int qb = n & 1;
                 uint64_t dq[HP];
 #pragma unroll
                 for (int x = 0; x < HP; ++x) dq[x] = sw128_desc(sQ + qb * Cfg::Q_BYTES + x * Cfg::TILE_BYTES, 16, 1024);
-                if (!(ok = mbar_wait_w(BAR(Cfg::B_QFULL + qb), (n >> 1) & 1, abort_flag))) break;
-                // the slots of tile J: the softmax has read tile J-1 (S or Y writes reuse its upper slot)
-                for (int x = 0; ok && x < HP && J > 0; ++x) ok = mbar_wait_w(BAR(Cfg::B_SFREE + x), (J - 1) & 1, abort_flag);
-                if (!ok) break;
+                if (!pre && (LOCAL ? I.n_tiles > 0 : true) && !(ok = issue_head(I, n, J, G))) break;
+                pre = false;
                 if (!LOCAL) {
-                    // prologue: Y = Q Wq^T into the slots of tile J, phi(q) over its first slot, then
-                    // O := phi(q) S_t^T
-                    if (!(ok = mbar_wait_w(BAR(Cfg::B_WFULL), n & 1, abort_flag))) break;
-                    tc_fence_after();
-                    for (int x = 0; x < HP; ++x) {
-                        issue_wide(x, J, dq[x], sW + x * Cfg::WQ_BYTES, DF);
-                        mma_commit_w(BAR(Cfg::B_Y + x));
-                    }
+                    // prologue: Y (issued above or ahead) -> phi(q) (bf16) over the score columns ->
+                    // O := phi(q) S_t^T -> the scores of the first kept tile
                     const uint32_t sST = sW + HP * Cfg::WQ_BYTES;
                     for (int x = 0; ok && x < HP; ++x) {
                         if (!(ok = mbar_wait_w(BAR(Cfg::B_PHI + x), n & 1, abort_flag))) break;
                         tc_fence_after();
 #pragma unroll
                         for (int kk = 0; kk < DF / 16; ++kk)
-                            mma_ts_w(tmem_w + Cfg::o_col(x), tmem_w + Cfg::ring(x) + (J % 3) * 64 + kk * 8,
+                            mma_ts_w(tmem_w + Cfg::o_col(x), tmem_w + Cfg::s_col(x) + kk * 8,
                                    kmajor_desc(sST, kk, 64 * 128), ID_N64, kk > 0);
                     }
                     if (!ok) break;
                     mma_commit_w(BAR(Cfg::B_PRO));
                     mma_commit_w(BAR(Cfg::B_WEMPTY));
-                }
-                if (I.n_tiles > 0) {
-                    if (!(ok = mbar_wait_w(BAR(Cfg::B_KFULL + G % Cfg::NS), (G / Cfg::NS) & 1, abort_flag))) break;
-                    tc_fence_after();
-                    for (int x = 0; x < HP; ++x) {
-                        issue_wide(x, J, dq[x], sStage + (G % Cfg::NS) * Cfg::STAGE_BYTES, 128);
-                        mma_commit_w(BAR(Cfg::B_S + x));
+                    if (I.n_tiles > 0) {
+                        if (!(ok = mbar_wait_w(BAR(Cfg::B_KFULL + G % Cfg::NS), (G / Cfg::NS) & 1, abort_flag))) break;
+                        tc_fence_after();
+                        for (int x = 0; x < HP; ++x) {
+                            issue_qk(x, dq[x], sStage + (G % Cfg::NS) * Cfg::STAGE_BYTES, 128);
+                            mma_commit_w(BAR(Cfg::B_S + x));
+                        }
                     }
                 }
+                const bool has_next = it + (int)gridDim.x < p.n_items;
                 for (int jj = 0; ok && jj < I.n_tiles; ++jj, ++G) {
                     const int Jt = J + jj, s = G % Cfg::NS, s1 = (G + 1) % Cfg::NS;
-                    // next scores first: they need the softmax to have read S(Jt) (and P V(Jt-1), issued
-                    // before them, to have consumed P(Jt-1))
+                    // next scores first: they only need the softmax to have read S(Jt)
                     if (jj + 1 < I.n_tiles) {
                         for (int x = 0; x < HP; ++x) {
                             if (x == 0 && !(ok = mbar_wait_w(BAR(Cfg::B_KFULL + s1), ((G + 1) / Cfg::NS) & 1, abort_flag)))
                                 break;
                             if (!(ok = mbar_wait_w(BAR(Cfg::B_SFREE + x), Jt & 1, abort_flag))) break;
                             tc_fence_after();
-                            issue_wide(x, Jt + 1, dq[x], sStage + s1 * Cfg::STAGE_BYTES, 128);
+                            issue_qk(x, dq[x], sStage + s1 * Cfg::STAGE_BYTES, 128);
                             mma_commit_w(BAR(Cfg::B_S + x));
                         }
                         if (!ok) break;
+                    } else if (has_next) {
+                        // last tile: the next item's first score-column MMA goes ahead of this P V
+                        const Item In = item_of<HP, LOCAL>(it + gridDim.x, p);
+                        if (!(ok = issue_head(In, n + 1, Jt + 1, G + 1))) break;
+                        pre = true;
                     }
                     const uint64_t dv = sw128_desc(sStage + s * Cfg::STAGE_BYTES + Cfg::TILE_BYTES, Cfg::TILE_BYTES, 1024);
                     for (int x = 0; x < HP; ++x) {
@@ -333,7 +350,7 @@ __global__ void __launch_bounds__(RingCfg<DF, HP>::THREADS, 1)
                         tc_fence_after();
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk)  // 16 keys = 16 rows of V per k-step
-                            mma_ts_w(tmem_w + Cfg::o_col(x), tmem_w + Cfg::ring(x) + (Jt % 3) * 64 + kk * 8,
+                            mma_ts_w(tmem_w + Cfg::o_col(x), tmem_w + Cfg::p_col(x) + kk * 8,
                                    dv + (uint64_t)(kk * 128), ID_PV, (LOCAL && jj == 0 && kk == 0) ? 0u : 1u);
                         mma_commit_w(BAR(Cfg::B_O + x));
                     }
@@ -358,7 +375,8 @@ __global__ void __launch_bounds__(RingCfg<DF, HP>::THREADS, 1)
         const int x = warp >> 2;                       // head of the pair
         const int r = (warp & 3) * 32 + lane;          // row in the tile = TMEM lane
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        const uint32_t tR = tmem + lane_off + Cfg::ring(x);
+        const uint32_t tS = tmem + lane_off + Cfg::s_col(x);
+        const uint32_t tP = tmem + lane_off + Cfg::p_col(x);
         const uint32_t tO = tmem + lane_off + Cfg::o_col(x);
         bool ok = true;
         int J = 0, n = 0;
@@ -377,13 +395,12 @@ __global__ void __launch_bounds__(RingCfg<DF, HP>::THREADS, 1)
                 ok = warp_all(mbar_wait(BAR(Cfg::B_QFULL + qb), (n >> 1) & 1, abort_flag) &&
                               mbar_wait(BAR(Cfg::B_Y + x), n & 1, abort_flag));
                 float y[DF];
-                const uint32_t ca = (J % 3) * 64, cb = ((J + 1) % 3) * 64;
                 if (ok) {
                     tc_fence_after();
 #pragma unroll
                     for (int c = 0; c < DF / 32; ++c) {
                         uint32_t u[32];
-                        tmem_ld32(tR + (c < 2 ? ca : cb) + (c & 1) * 32, u);
+                        tmem_ld32(tS + c * 32, u);
                         tmem_wait_ld();
 #pragma unroll
                         for (int e = 0; e < 32; ++e) y[c * 32 + e] = __uint_as_float(u[e]);
@@ -414,12 +431,19 @@ __global__ void __launch_bounds__(RingCfg<DF, HP>::THREADS, 1)
                     ee = fmaf(y[c], y[c], ee);
                 }
                 const float f = sqrtf(qq) * rsqrtf(ee);
-                const float *zt = p.z + (size_t)I.tslot * DF;
+                const float4 *zt = reinterpret_cast<const float4 *>(p.z + (size_t)I.tslot * DF);
                 float bden = 0.f;
 #pragma unroll
-                for (int c = 0; c < DF; ++c) {
-                    y[c] *= f;
-                    bden = fmaf(y[c], __ldg(zt + c), bden);
+                for (int c4 = 0; c4 < DF / 4; ++c4) {
+                    const float4 zz = __ldg(zt + c4);
+                    y[4 * c4] *= f;
+                    y[4 * c4 + 1] *= f;
+                    y[4 * c4 + 2] *= f;
+                    y[4 * c4 + 3] *= f;
+                    bden = fmaf(y[4 * c4], zz.x, bden);
+                    bden = fmaf(y[4 * c4 + 1], zz.y, bden);
+                    bden = fmaf(y[4 * c4 + 2], zz.z, bden);
+                    bden = fmaf(y[4 * c4 + 3], zz.w, bden);
                 }
                 if (ok) {
 #pragma unroll
@@ -427,7 +451,7 @@ __global__ void __launch_bounds__(RingCfg<DF, HP>::THREADS, 1)
                         uint32_t u[32];
 #pragma unroll
                         for (int e = 0; e < 32; ++e) u[e] = pack_bf16x2(y[c * 64 + 2 * e], y[c * 64 + 2 * e + 1]);
-                        tmem_st32(tR + ca + c * 32, u);
+                        tmem_st32(tS + c * 32, u);
                     }
                     tmem_wait_st();
                 }
@@ -478,18 +502,17 @@ __global__ void __launch_bounds__(RingCfg<DF, HP>::THREADS, 1)
                 ok = warp_all(mbar_wait(BAR(Cfg::B_S + x), Jt & 1, abort_flag));
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t ca = (Jt % 3) * 64, cb = ((Jt + 1) % 3) * 64;
                 float sv[128];
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     uint32_t u[32];
-                    tmem_ld32(tR + (c < 2 ? ca : cb) + (c & 1) * 32, u);
+                    tmem_ld32(tS + c * 32, u);
 #pragma unroll
                     for (int e = 0; e < 32; ++e) sv[c * 32 + e] = __uint_as_float(u[e]);
                 }
                 tmem_wait_ld();
                 tc_fence_before();
-                mbar_arrive(BAR(Cfg::B_SFREE + x));  // the slots may now take the next tile's scores
+                mbar_arrive(BAR(Cfg::B_SFREE + x));  // S may now take the next tile's scores
                 // masks, only on the tiles that need them (warp-uniform test): LOCAL the causal diagonal
                 // tile, PREFIX the ragged last tile of the kept rows
                 const bool diag = LOCAL && jj == I.n_tiles - 1;
@@ -513,24 +536,6 @@ __global__ void __launch_bounds__(RingCfg<DF, HP>::THREADS, 1)
                 const bool need = mnew > m_run + kRescaleLog2;
                 const float alpha = need ? ex2(m_run - mnew) : 1.f;
                 const bool touch_o = need && m_run != -INFINITY;  // O holds nothing yet while m_run = -inf
-                if (__any_sync(0xffffffffu, touch_o)) {
-                    // P V(Jt-1) must be done before O is rescaled (the first tile of an item has no
-                    // P V in flight: the prologue's fold has completed)
-                    if (jj > 0) ok = warp_all(mbar_wait(BAR(Cfg::B_O + x), (Jt - 1) & 1, abort_flag));
-                    if (!ok) break;
-                    tc_fence_after();
-                    const float fa = touch_o ? alpha : 1.f;
-#pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        uint32_t u[32];
-                        tmem_ld32(tO + c * 32, u);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * fa);
-                        tmem_st32(tO + c * 32, u);
-                    }
-                    tmem_wait_st();
-                }
                 if (need) {
                     l_run *= alpha;
                     bs *= alpha;
@@ -546,15 +551,47 @@ __global__ void __launch_bounds__(RingCfg<DF, HP>::THREADS, 1)
                     else btype = 1;
                 }
                 float ls0, ls1, bsum = 0.f;
+                uint32_t pu[64];
+                // head 1 takes its turn after head 0's exponentials of this tile, head 0 after head 1's
+                // of the previous one (barrier phase = global tile index)
+                if (HP == 2 && kRingTurns && (x == 1 || Jt > 0)) {
+                    ok = warp_all(mbar_wait(BAR(Cfg::B_TURN + x), (x == 1 ? Jt : Jt - 1) & 1, abort_flag));
+                    if (!ok) break;
+                }
                 if (btype >= 2) {
                     const int bc_lo = btype == 2 ? r + 1 : 0, bc_hi = btype == 2 ? 128 : r;
-                    exp_tile<EXPV, true>(sv, p.scale_log2, m_run, tR + ca, ls0, ls1, bsum, bc_lo, bc_hi);
+                    exp_row<EXPV, true>(sv, p.scale_log2, m_run, pu, ls0, ls1, bsum, bc_lo, bc_hi);
                 } else {
-                    exp_tile<EXPV, false>(sv, p.scale_log2, m_run, tR + ca, ls0, ls1, bsum, 0, 0);
+                    exp_row<EXPV, false>(sv, p.scale_log2, m_run, pu, ls0, ls1, bsum, 0, 0);
                 }
+                if (HP == 2 && kRingTurns) mbar_arrive(BAR(Cfg::B_TURN + (x ^ 1)));
                 l_run += ls0 + ls1;
                 if (btype == 1) bs += ls0 + ls1;
                 else if (btype >= 2) bs += bsum;
+                // P V(Jt-1) still reads P and adds into O: wait for it before P is rewritten or O rescaled.
+                // (It was issued a whole exponential phase ago.  The first tile of an item has none in
+                // flight: the previous item's epilogue waited for its last P V, and the prologue's fold
+                // waited for the only MMA that wrote O since.)  The wait is for phase Jt-1 of the O
+                // barrier, whose phase Jt-2 this warp already waited for at the previous tile, so the
+                // parity test cannot be fooled by a barrier two phases behind.
+                if (jj > 0) {
+                    ok = warp_all(mbar_wait(BAR(Cfg::B_O + x), (Jt - 1) & 1, abort_flag));
+                    if (!ok) break;
+                    tc_fence_after();
+                }
+                if (__any_sync(0xffffffffu, touch_o)) {
+                    const float fa = touch_o ? alpha : 1.f;
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        uint32_t u[32];
+                        tmem_ld32(tO + c * 32, u);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * fa);
+                        tmem_st32(tO + c * 32, u);
+                    }
+                }
+                store_p(tP, pu);
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(BAR(Cfg::B_P + 2 * x + (Jt & 1)));

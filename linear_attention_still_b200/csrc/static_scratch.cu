@@ -9,12 +9,13 @@
 #include <cstdint>
 
 #include "still.h"
+#include "still_internal.h"
 
 static __device__ __align__(256) unsigned char g_prefill_scratch[STILL_STATIC_WORKSPACE_BYTES];
 
 namespace {
 
-constexpr int kMaxDevices = 64;
+constexpr int kMaxDevices = 128;  // device ordinals 0..127, as for the device status word
 std::atomic<void *> g_scratch_addr[kMaxDevices];
 
 // Address of the current device's copy of the array, looked up once per device with that device
@@ -40,9 +41,11 @@ extern "C" STILL_API still_status still_hybrid_prefill_static(const still_dims *
                                                               const void *v, const void *Wq, const void *Wk, void *o,
                                                               const int32_t *idx_in, void *state, int state_capacity,
                                                               void *stream) {
+    // the regular entry point's checks first, in its order, so that both report the same error
+    bool empty = false;
+    still_status chk = still::check_prefill_args(dims, q, k, v, Wq, Wk, o, idx_in, state, state_capacity, &empty);
+    if (chk || empty) return chk;
     const size_t need = still_prefill_workspace_bytes(dims);
-    if (need == 0)  // invalid dims: the regular entry point reports which error
-        return still_hybrid_prefill(dims, q, k, v, Wq, Wk, o, idx_in, nullptr, 0, state, state_capacity, stream);
     if (need > (size_t)STILL_STATIC_WORKSPACE_BYTES) return STILL_ERR_WORKSPACE;
     void *scratch = nullptr;
     const still_status st = scratch_address(&scratch);

@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "still.h"
+
 namespace still {
 
 struct Dims {
@@ -76,6 +78,11 @@ cudaError_t launch_backward(const Dims &s, const void *q, const void *k, const v
                             const void *Wk, const int32_t *idx, const void *dO, float *dq, float *dk, float *dv,
                             float *dWq, float *dWk, const BackwardScratch &w, unsigned *err, cudaStream_t st,
                             int *launches);
+
+// Every argument check of still_hybrid_prefill except the workspace's (api.cu).
+still_status check_prefill_args(const still_dims *dims, const void *q, const void *k, const void *v, const void *Wq,
+                                const void *Wk, const void *o, const int32_t *idx_in, const void *state,
+                                int state_capacity, bool *empty);
 
 // Per-kernel event timing (still_timing_enable): returns a slot for timing_end, or -1 when off.
 int timing_begin(int cls, cudaStream_t st);

@@ -59,6 +59,47 @@ __device__ __forceinline__ void exp_tile(const float (&sv)[128], float scale_log
     ls1 = ls.y;
 }
 
+// The same exponentials into registers: u[e] = bf16 pair (p_{2e}, p_{2e+1}) of the row, to be stored
+// as P later (store_p).  Lets a softmax warp finish its exponentials before it waits for the MMA that
+// still reads the previous P.
+template <int EXPV, bool BAND>
+__device__ __forceinline__ void exp_row(const float (&sv)[128], float scale_log2, float m_run, uint32_t (&u)[64],
+                                        float &ls0, float &ls1, float &bsum, int bc_lo, int bc_hi) {
+    const float2 sc2 = make_float2(scale_log2, scale_log2);
+    const float2 neg2 = make_float2(-m_run, -m_run);
+    // four independent partial sums, so the adds do not serialise the exponentials
+    float2 ls[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+    float bs[2] = {0.f, 0.f};
+#pragma unroll
+    for (int e = 0; e < 64; ++e) {
+        const int c0 = 2 * e;
+        const float2 xx = ffma2(make_float2(sv[c0], sv[c0 + 1]), sc2, neg2);
+        float2 pp;
+        if ((EXPV == 2 && c0 >= 96) || (EXPV == 3 && ((c0 >> 5) & 1))) {
+            pp = exp2_poly2(xx);  // FMA pipe
+        } else {
+            pp.x = ex2(xx.x);      // MUFU
+            pp.y = ex2(xx.y);
+        }
+        ls[e & 3] = fadd2(ls[e & 3], pp);
+        if (BAND) {
+            if (c0 >= bc_lo && c0 < bc_hi) bs[e & 1] += pp.x;
+            if (c0 + 1 >= bc_lo && c0 + 1 < bc_hi) bs[e & 1] += pp.y;
+        }
+        u[e] = pack_bf16x2(pp.x, pp.y);
+    }
+    const float2 l01 = fadd2(ls[0], ls[1]), l23 = fadd2(ls[2], ls[3]);
+    ls0 = l01.x + l23.x;
+    ls1 = l01.y + l23.y;
+    if (BAND) bsum += bs[0] + bs[1];
+}
+
+// P row (64 packed bf16 pairs = 128 keys) into 64 TMEM columns.
+__device__ __forceinline__ void store_p(uint32_t tP, const uint32_t (&u)[64]) {
+    tmem_st32(tP, *reinterpret_cast<const uint32_t(*)[32]>(&u[0]));
+    tmem_st32(tP + 32, *reinterpret_cast<const uint32_t(*)[32]>(&u[32]));
+}
+
 // tcgen05.ld/st are warp-collective: every decision that guards them is made warp-uniform.
 __device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
 

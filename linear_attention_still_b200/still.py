@@ -23,7 +23,7 @@ EXPORTS = ("still_status_string", "still_saliency", "still_select_topk", "still_
            "still_decode_state_bytes", "still_decode_init", "still_decode_step", "still_get_device_status",
            "still_launch_count", "still_timing_enable", "still_timing_read", "still_debug_merge",
            "still_hybrid_prefill_static", "still_diagonal_score", "still_backward_workspace_bytes",
-           "still_hybrid_backward")
+           "still_hybrid_backward", "still_decode_state_layout")
 
 
 class StillError(RuntimeError):
@@ -35,6 +35,11 @@ class StillError(RuntimeError):
 class still_dims(ct.Structure):
     _fields_ = [(n, ct.c_int) for n in ("B", "H", "Hkv", "N", "d", "D", "w", "C", "k")] + \
                [("scale", ct.c_float), ("dtype", ct.c_int)]
+
+
+class still_state_layout(ct.Structure):
+    _fields_ = [(n, ct.c_size_t) for n in ("header", "khat", "vhat", "S", "z", "ring_k", "ring_v", "ring_r", "total")] + \
+               [("ring_rows", ct.c_int), ("cap_chunks", ct.c_int)]
 
 
 class still_ws_layout(ct.Structure):
@@ -61,6 +66,7 @@ _SIG = {
     "still_hybrid_backward": ([_D] + [_P] * 13 + [ct.c_size_t, _P], ct.c_int),
     "still_decode_state_bytes": ([_D, ct.c_int], ct.c_size_t),
     "still_decode_init": ([_D, ct.c_int, _P, _P], ct.c_int),
+    "still_decode_state_layout": ([_D, ct.c_int, ct.POINTER(still_state_layout)], ct.c_int),
     "still_decode_step": ([_D, _P, ct.c_int, ct.c_int, _P, _P, _P, _P, _P, _P, _P], ct.c_int),
     "still_get_device_status": ([_P], ct.c_int),
     "still_launch_count": ([], ct.c_uint64),
@@ -202,6 +208,12 @@ def still_hybrid_backward(dims, q, k, v, wq, wk, idx, do, dq, dk, dv, dwq, dwk, 
 
 def still_decode_state_bytes(dims, capacity: int) -> int:
     return int(_lib.still_decode_state_bytes(ct.byref(dims), int(capacity)))
+
+
+def still_decode_state_layout(dims, capacity) -> dict:
+    out = still_state_layout()
+    _ok("still_decode_state_layout", _lib.still_decode_state_layout(ct.byref(dims), int(capacity), ct.byref(out)))
+    return {n: int(getattr(out, n)) for n, _ in still_state_layout._fields_}
 
 
 def still_decode_init(dims, capacity, state, stream=None):

@@ -99,3 +99,64 @@ def test_decode_position_mismatch_is_reported(lib):
     o = torch.empty_like(x)
     lib.still_decode_step(d, state, cap, 3, w, w[:1], x, kv, kv, o)  # state is at 0
     assert lib.still_get_device_status() == 5
+
+
+def test_bf16_decode_scores_and_chunk_close_selection(lib, oracle_mod):
+    """bf16 decode on the tensor-core path, checked directly rather than through its outputs: the group
+    saliency score each decode step stores for its token (ring scores) against the oracle's
+    (<= 1e-3), and the rows kept by the chunk closes that happen during decode against the top-k of
+    the GPU's own scores (bit-exact) and the oracle's selection (differences only between oracle
+    near-ties)."""
+    from tests._gpu import SCORE_TOL, check_selection, score_err
+    shape, T = CASES["bf16_gqa"]
+    N0, C, k, m = shape.N, shape.C, shape.k, shape.w // shape.C
+    cap = N0 + T
+    full = shape.replace(N=cap)
+    inp = make_inputs(shape.replace(decode_steps=T))
+    d = lib.dims_of(shape, N=N0)
+    L = lib.still_decode_state_layout(d, cap)
+    state = torch.zeros(lib.still_decode_state_bytes(d, cap), dtype=torch.uint8, device="cuda")
+    lib.still_decode_init(d, cap, state)
+    out = gpu_prefill(shape, inp, N=N0, state=state, capacity=cap)
+    assert out["status"] == 0
+    BK = shape.B * shape.Hkv
+    ring_r = state[L["ring_r"]: L["ring_r"] + BK * L["ring_rows"] * 4].view(torch.float32).view(BK, L["ring_rows"])
+
+    def row(j):
+        return ((j // C) % (m + 1)) * C + j % C
+
+    r_gpu = np.full((shape.B, shape.Hkv, cap), np.nan)
+    r_gpu[:, :, :N0] = out["r"]
+    q, kk, v = (dev(getattr(inp, n), shape) for n in ("q", "k", "v"))
+    wq, wk = dev(inp.wq, shape), dev(inp.wk, shape)
+    o_t = torch.empty(shape.B, shape.H, shape.d, dtype=q.dtype, device="cuda")
+    closes = []
+    for p in range(N0, cap):
+        lib.still_decode_step(d, state, cap, p, wq, wk, q[:, :, p].contiguous(), kk[:, :, p].contiguous(),
+                              v[:, :, p].contiguous(), o_t)
+        r_gpu[:, :, p] = ring_r[:, row(p)].cpu().numpy().reshape(shape.B, shape.Hkv)
+        if p % C == C - 1 and p // C - m >= 0:
+            closes.append(p // C - m)  # this step closed chunk t - m
+    assert lib.still_get_device_status() == 0
+    assert closes, "the case must close a chunk during decode"
+    # scores of the decode tokens against the oracle's saliency of the whole sequence
+    _, r_ora = oracle_mod.saliency(odims(full), inp.q, inp.k)
+    assert score_err(r_gpu[:, :, N0:], r_ora[:, :, N0:]) <= SCORE_TOL
+    # kept rows of the chunks closed during decode, mapped back to positions by their keys
+    khat = state[L["khat"]: L["khat"] + BK * L["cap_chunks"] * k * shape.d * 2].view(torch.bfloat16)
+    khat = khat.view(shape.B, shape.Hkv, L["cap_chunks"] * k, shape.d).float().cpu().numpy()
+    kin = kk.float().cpu().numpy()
+    for c in closes:
+        lo = c * C
+        got = np.zeros((shape.B, shape.Hkv, 1, k), dtype=np.int32)
+        for b in range(shape.B):
+            for g in range(shape.Hkv):
+                for e in range(k):
+                    hit = np.nonzero((kin[b, g, lo:lo + C] == khat[b, g, c * k + e]).all(axis=-1))[0]
+                    assert hit.size == 1, (c, b, g, e)
+                    got[b, g, 0, e] = lo + hit[0]
+        sub = full.replace(N=C)  # one chunk: check_selection's top-k of this chunk's scores
+        gpu_r = r_gpu[:, :, lo:lo + C]
+        ora_r = r_ora[:, :, lo:lo + C]
+        ora_idx = oracle_mod.topk(odims(sub), ora_r)
+        check_selection(sub, C, got - lo, gpu_r, ora_r, ora_idx)
