@@ -137,29 +137,37 @@ def layer_flops(shape):
 # ----------------------------------------------------------------------------- clocks
 
 def profiled_traffic(workload: str):
-    """DRAM bytes per step of the merge launches from a committed ncu summary under profiles/, or
-    None when there is none for this workload or the kernel sources changed since the capture."""
+    """DRAM bytes per step of the merge launches from a committed ncu summary under profiles/ (a
+    block of `workload:`, `traffic_bytes_per_step:` and `source_sha256:` lines), or None when there
+    is none for this workload or the kernel sources changed since the capture."""
     import glob
     import hashlib
-    for path in glob.glob(os.path.join(ROOT, "profiles", "merge_tc_*.md")):
-        kv = {}
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "merge_*.md"))):
+        blocks, kv = [], {}
         with open(path) as f:
             for line in f:
-                if ":" in line and line.startswith("    "):
+                if ":" in line and line.startswith("    ") and not line.startswith("     "):
                     k_, _, v_ = line.strip().partition(": ")
+                    if k_ == "workload" and kv:
+                        blocks.append(kv)
+                        kv = {}
                     kv[k_] = v_
-        if kv.get("workload") != workload or "traffic_bytes_per_step" not in kv:
-            continue
-        for item in kv.get("source_sha256", "").split():
-            name, _, digest = item.partition("=")
-            src = os.path.join(ROOT, "linear_attention_still_b200", "csrc", name)
-            try:
-                with open(src, "rb") as f:
-                    if not hashlib.sha256(f.read()).hexdigest().startswith(digest):
-                        return None
-            except OSError:
-                return None
-        return int(kv["traffic_bytes_per_step"])
+        if kv:
+            blocks.append(kv)
+        for kv in blocks:
+            if kv.get("workload") != workload or "traffic_bytes_per_step" not in kv:
+                continue
+            fresh = True
+            for item in kv.get("source_sha256", "").split():
+                name, _, digest = item.partition("=")
+                src = os.path.join(ROOT, "linear_attention_still_b200", "csrc", name)
+                try:
+                    with open(src, "rb") as f:
+                        fresh = fresh and hashlib.sha256(f.read()).hexdigest().startswith(digest)
+                except OSError:
+                    fresh = False
+            if fresh:
+                return int(kv["traffic_bytes_per_step"])
     return None
 
 

@@ -216,6 +216,8 @@ __global__ void __launch_bounds__(256) linear_delta_kernel(Dims s, const float *
 
 // Inclusive prefix over slots 0..T: slots 0..m are zero (no chunk has been decided for them).
 // st_t (optional): a bf16 copy of every S_t, transposed to [d, D] (K-major operand of phi(q) S_t).
+// One thread per element of (S, z) of a (b, g); the slots are read eight at a time so that the loads
+// of a batch are in flight together (the sum over slots is sequential).
 __global__ void linear_prefix_kernel(Dims s, float *__restrict__ S, float *__restrict__ z,
                                      __nv_bfloat16 *__restrict__ st_t) {
     const int T_ = s.T(), m = s.m();
@@ -225,14 +227,22 @@ __global__ void linear_prefix_kernel(Dims s, float *__restrict__ S, float *__res
     if (gid >= total) return;
     const size_t bg = gid / per;
     const int e = (int)(gid % per);
+    const bool isS = e < Dd;
+    float *base = isS ? &S[bg * (T_ + 1) * Dd + e] : &z[bg * (T_ + 1) * s.D + (e - Dd)];
+    const size_t stride = isS ? (size_t)Dd : (size_t)s.D;
+    const int a = isS ? e / s.d : 0, x = isS ? e % s.d : 0;
     float run = 0.f;
-    for (int t = 0; t <= T_; ++t) {
-        float *p = e < Dd ? &S[(bg * (T_ + 1) + t) * Dd + e] : &z[(bg * (T_ + 1) + t) * s.D + (e - Dd)];
-        if (t >= m + 1) run += *p;
-        *p = run;
-        if (st_t && e < Dd) {
-            const int a = e / s.d, x = e % s.d;
-            st_t[((bg * (T_ + 1) + t) * s.d + x) * s.D + a] = __float2bfloat16_rn(run);
+    for (int t0 = 0; t0 <= T_; t0 += 8) {
+        float v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = (t0 + u <= T_) ? base[(size_t)(t0 + u) * stride] : 0.f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int t = t0 + u;
+            if (t > T_) break;
+            if (t >= m + 1) run += v[u];
+            base[(size_t)t * stride] = run;
+            if (st_t && isS) st_t[((bg * (T_ + 1) + t) * s.d + x) * s.D + a] = __float2bfloat16_rn(run);
         }
     }
 }

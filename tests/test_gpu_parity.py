@@ -26,6 +26,10 @@ CASES = {
     # largest head dim, feature width and group the library takes (SIMT path)
     "f32_max_d_D_group": Shape(B=1, H=32, Hkv=1, N=200, d=256, D=256, w=64, C=64, k=8, dtype="f32"),
     "bf16_max_d_D": Shape(B=1, H=4, Hkv=2, N=260, d=256, D=256, w=128, C=64, k=16),
+    # a window covering the whole sequence with k = 0: exact causal softmax attention in the window
+    # phase alone (the flash-style dense comparator `bench.py --keep window` times)
+    "bf16_window_covers_sequence": Shape(B=1, H=4, Hkv=2, N=700, d=64, D=64, w=768, C=128, k=0),
+    "bf16_d128_window_covers_sequence": Shape(B=1, H=4, Hkv=1, N=600, d=128, D=128, w=640, C=128, k=0),
 }
 
 
