@@ -123,6 +123,18 @@ def exp_pipe_diag(shape, merge_ms_per_step, clocks=None, sms: int = 148):
             "flops_per_exp": merge_flops(shape) / max(exps, 1), "achieved_tflops": flop_s / 1e12}
 
 
+def nowin_flops(shape):
+    """Algorithmic FLOPs of a w = 0 step (pure chunked linear attention): per (query-head, key of the
+    query's own chunk up to the query) 2D for <phi(q), phi(k)> and 2d for the weighted value; per
+    query-head 2dD for phi(q), 2dD + 2D for phi(q)^T S_t and phi(q)^T z_t; per key of a KV head 2dD
+    for phi(k) and 2dD for its outer product with v."""
+    import numpy as np
+    N, d, D, C = shape.N, shape.d, shape.D, shape.C
+    i = np.arange(N, dtype=np.int64)
+    intra = int((i - (i // C) * C + 1).sum())
+    return shape.B * shape.H * (2 * (D + d) * intra + N * (4 * d * D + 2 * D)) + shape.B * shape.Hkv * N * 4 * d * D
+
+
 def layer_flops(shape):
     """Algorithmic FLOPs of one whole step (all kernels)."""
     import numpy as np
@@ -131,6 +143,8 @@ def layer_flops(shape):
     sal = shape.B * shape.H * 2 * d * float(band.sum()) if shape.k > 0 else 0.0
     phik = shape.B * shape.Hkv * N * 2 * d * D
     lin = shape.B * shape.Hkv * N * 2 * D * d
+    if shape.w == 0:
+        return nowin_flops(shape)
     return merge_flops(shape) + sal + phik + lin
 
 
@@ -589,14 +603,17 @@ def bench_prefill(args, name, rank, world, local, cpu_seconds):
     # over the summed device time of its launches
     merge_ms = kern["merge"][0] + kern["merge_prefix"][0]
     merge_n = args.steps if merge_ms > 0 else 0
-    achieved = merge_flops(shape) / (merge_ms / merge_n / 1e3) / 1e12 if merge_n else None
+    mflops = nowin_flops(shape) if shape.w == 0 else merge_flops(shape)
+    achieved = mflops / (merge_ms / merge_n / 1e3) / 1e12 if merge_n else None
     peak = peaks.get("bf16_tflops", 1590.0) if shape.dtype == "bf16" else None
     roofline = {
-        "kernel": "merge (window phase + kept-prefix phase)", "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+        "kernel": "merge (window phase + kept-prefix phase)" if shape.w > 0 else
+                  "no-window merge (intra-chunk tile + phi(q)^T S_t, with the W^T transpose)",
+        "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
         "frac": (achieved / peak) if (achieved and peak) else None,
         "peak_source": "measured bf16_tflops" if "bf16_tflops" in peaks else "fallback 1.59 PFLOP/s",
         "traffic": profiled_traffic(name), "traffic_unit": "DRAM bytes per step (both merge launches, ncu)",
-        "flops_per_step": merge_flops(shape), "ms_per_step": merge_ms / merge_n if merge_n else None,
+        "flops_per_step": mflops, "ms_per_step": merge_ms / merge_n if merge_n else None,
     }
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -609,7 +626,8 @@ def bench_prefill(args, name, rank, world, local, cpu_seconds):
         "layer_tflops": layer_flops(shape) / (ms_per_step / 1e3) / 1e12, "device_status": status,
         "memory": memory,
         "exp_pipe": exp_pipe_diag(shape, roofline["ms_per_step"], clocks,
-                                  torch.cuda.get_device_properties(local).multi_processor_count),
+                                  torch.cuda.get_device_properties(local).multi_processor_count)
+        if shape.w > 0 else None,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, t, desc, nth = oracle_sample(shape, cpu_seconds, router=args.router)

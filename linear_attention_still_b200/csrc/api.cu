@@ -21,6 +21,10 @@ cudaError_t launch_mean_heads(const Dims &s, const float *sigma, float *r, cudaS
 cudaError_t launch_saliency_fixup(const Dims &s, const void *q, const void *k, const int *list, const unsigned *count,
                                   float *sigma, cudaStream_t st);
 bool tc_saliency_supported(const Dims &s);
+bool tc_nowin_supported(const Dims &s);
+cudaError_t launch_nowin_tc(const Dims &s, const void *q, const void *k, const void *v, const void *wqt,
+                            const void *wkt, const void *st_t, const float *z, void *o, unsigned *err,
+                            cudaStream_t st);
 void set_merge_debug(int stall, int max_ctas);
 cudaError_t launch_saliency_tc(const Dims &s, const void *q, const void *k, float *r_kv, float *r_q, unsigned *err,
                                cudaStream_t st);
@@ -96,7 +100,7 @@ still_ws_layout ws_layout(const Dims &s) {
     L.z = off;
     off = al256(off + BK * (T + 1) * s.D * 4);
     L.phik = off;  // phi(K) only on the SIMT path (the tensor-core linear state featurises in place)
-    const bool fused_lin = s.bf16 && tc_merge_supported(s) && tc_linear_supported(s);
+    const bool fused_lin = s.bf16 && ((tc_merge_supported(s) && tc_linear_supported(s)) || tc_nowin_supported(s));
     off = al256(off + (fused_lin ? 0 : BK * s.N * s.D * 4));
     const bool tc = s.bf16 != 0;  // per-head scores and transposed bf16 operands of the tensor-core path
     L.sig = off;
@@ -392,6 +396,28 @@ still_status still_hybrid_prefill(const still_dims *dims, const void *q, const v
     unsigned *fix_count = reinterpret_cast<unsigned *>(ws + W.fix);
     int *fix_list = reinterpret_cast<int *>(ws + W.fix + 256);
     MergeOperands mo{q, k, v, wqt, khat, vhat, st_t, z, o, lse, sig, fix_list, fix_count};
+    if (tc_nowin_supported(s)) {
+        // w = 0 (no softmax branch): the inter-chunk linear state on tensor cores (NP-Map of the keys
+        // fused), then every row's intra-chunk causal tile plus phi(q)^T S_t on tensor cores
+        {
+            TimingScope ts(3, cs);
+            STILL_LAUNCH(launch_w_transpose(s.Hkv, s.d, s.D, Wk, wkt, cs));
+            STILL_LAUNCH(launch_linear_tc(s, k, v, wkt, nullptr, S, z, err, cs));
+            STILL_LAUNCH(launch_linear_prefix(s, S, z, st_t, cs));
+        }
+        {
+            TimingScope ts(4, cs);
+            STILL_LAUNCH(launch_w_transpose(s.H, s.d, s.D, Wq, wqt, cs));
+            STILL_LAUNCH(launch_nowin_tc(s, q, k, v, wqt, wkt, st_t, z, o, err, cs));
+        }
+        if (state) {
+            DecodeLayout L = decode_layout(s, state_capacity);
+            TimingScope ts(5, cs);
+            STILL_LAUNCH(launch_state_export(s, static_cast<unsigned char *>(state), L, k, v, nullptr, khat, vhat, S,
+                                             z, cs));
+        }
+        return STILL_OK;
+    }
     if (use_tc) {
         // 1a. window part of the softmax branch and, from the same exponentials, the Self-Saliency
         //     Score of every query head (tensor cores)

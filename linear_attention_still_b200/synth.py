@@ -74,6 +74,8 @@ WORKLOADS = {
     "still_f32_decode_b1_ctx512": Shape(B=1, H=2, Hkv=2, N=512, d=64, D=64, w=64, C=64, k=8,
                                         dtype="f32", heavy=4, decode_steps=128),
     "llama32_1b_layer_n16k": Shape(B=1, H=32, Hkv=8, N=16384, d=64, D=64, w=512, C=512, k=64),
+    # the same layer with no softmax window (w = 0, k = 0): pure chunked linear attention with NP-Map
+    "llama32_1b_linear_n16k": Shape(B=1, H=32, Hkv=8, N=16384, d=64, D=64, w=0, C=512, k=0),
     "llama31_8b_layer_b4_n16k": Shape(B=4, H=32, Hkv=8, N=16384, d=128, D=128, w=1024, C=1024, k=128),
     "llama31_8b_layer_n64k": Shape(B=1, H=32, Hkv=8, N=65536, d=128, D=128, w=1024, C=1024, k=128),
     "llama31_8b_decode_b16_ctx64k": Shape(B=16, H=32, Hkv=8, N=65536, d=128, D=128, w=1024, C=1024,

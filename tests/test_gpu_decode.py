@@ -29,6 +29,8 @@ CASES = {
     "bf16_d64_mha": (Shape(B=2, H=2, Hkv=2, N=200, d=64, D=64, w=64, C=64, k=8), 80),
     "f32_g8_D256": (Shape(B=1, H=8, Hkv=1, N=150, d=64, D=256, w=64, C=64, k=8, dtype="f32"), 60),
     "bf16_no_window": (Shape(B=1, H=4, Hkv=2, N=100, d=64, D=64, w=0, C=64, k=0), 60),
+    # w = 0 prefill on the tensor-core path (C a multiple of 128), then decode across a chunk boundary
+    "bf16_no_window_tc": (Shape(B=1, H=4, Hkv=2, N=300, d=64, D=64, w=0, C=128, k=0), 100),
     "bf16_g16_fallback": (Shape(B=1, H=16, Hkv=1, N=200, d=64, D=64, w=64, C=64, k=8), 80),
     "f32_d96_fallback": (Shape(B=1, H=4, Hkv=2, N=150, d=96, D=64, w=64, C=64, k=8, dtype="f32"), 60),
 }

@@ -19,6 +19,8 @@ CASES = {
     "bf16_keep_none": Shape(B=1, H=4, Hkv=2, N=700, d=64, D=64, w=128, C=128, k=0),
     "f32_no_window": Shape(B=1, H=2, Hkv=1, N=300, d=64, D=32, w=0, C=64, k=0, dtype="f32"),
     "bf16_no_window": Shape(B=2, H=4, Hkv=2, N=333, d=64, D=64, w=0, C=128, k=0),
+    # w = 0 on the tensor-core path with chunks of four query tiles, D = 128, groups of 4, ragged tail
+    "bf16_no_window_c512_D128": Shape(B=1, H=8, Hkv=2, N=1300, d=64, D=128, w=0, C=512, k=0),
     "f32_shorter_than_chunk": Shape(B=1, H=2, Hkv=2, N=50, d=64, D=64, w=64, C=64, k=8, dtype="f32"),
     "bf16_one_token": Shape(B=1, H=4, Hkv=1, N=1, d=64, D=64, w=128, C=128, k=8),
     "f32_gqa_d128_D64": Shape(B=1, H=4, Hkv=2, N=520, d=128, D=64, w=128, C=64, k=8, dtype="f32"),
