@@ -115,7 +115,10 @@ __device__ __forceinline__ Item item_of(int it, const RingParams &p) {
     return I;
 }
 
-constexpr int kRingExpVariant = 1;  // see exp_row: 1 = every exponential on the MUFU unit
+// Where the exponentials run (see exp_row): the window phase keeps every exponential on the MUFU unit;
+// the kept-prefix phase sends the last 32 keys of each row to the FMA pipe.  Measured on B200 (1B 16K
+// layer, ms per phase, window / prefix): all on MUFU 0.232 / 0.291, a quarter on FMA 0.243 / 0.273.
+constexpr int kRingExpLocal = 1, kRingExpPrefix = 2;
 // Two heads per CTA: the softmax warpgroups take turns on the exponential phase of each tile (head 0,
 // head 1, head 0, ...), so one warpgroup's row bookkeeping (TMEM read of S, row max, P store) overlaps
 // the other's exponentials instead of both leaving the MUFU unit idle at the same time.
@@ -709,7 +712,7 @@ cudaError_t launch_ring_cfg(int mode, const Dims &s, const MergeOperands &a, uns
     prm.pairs = s.G() / HP;
     prm.n_items = (n_qtiles - qt_first) * s.B * s.Hkv * prm.pairs;
     prm.stall = g_stall;
-    auto kern = mode == 0 ? merge_ring_kernel<DF, HP, kRingExpVariant, 0> : merge_ring_kernel<DF, HP, kRingExpVariant, 1>;
+    auto kern = mode == 0 ? merge_ring_kernel<DF, HP, kRingExpLocal, 0> : merge_ring_kernel<DF, HP, kRingExpPrefix, 1>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
     if (e != cudaSuccess) return e;
     int ctas = std::min(prm.n_items, sm_count());
