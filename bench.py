@@ -476,6 +476,53 @@ def max_over_ranks(value_ms: float, world: int, device=None) -> float:
     return float(t.item())
 
 
+def pipelined_e2e(steps: int, h2d_fn, compute_fn, d2h_fn, nbuf: int = 2) -> float:
+    """Elapsed ms of `steps` end-to-end steps, each with its host->device input copy and its
+    device->host output copy inside the timed region, pipelined the way a caller would run it: the
+    inputs of step n+1 go up on one copy stream and the output of step n comes down on another while
+    step n+1 computes on the current stream, with `nbuf` device buffer sets and events ordering each
+    buffer's reuse.  h2d_fn(n, b), compute_fn(n, b) and d2h_fn(n, b) enqueue step n's work on the
+    current stream (the caller's callbacks run inside the right stream context); b = n % nbuf."""
+    import torch
+    main = torch.cuda.current_stream()
+    cs, os_ = torch.cuda.Stream(), torch.cuda.Stream()
+    h2d_ev = [torch.cuda.Event() for _ in range(nbuf)]
+    comp_ev = [torch.cuda.Event() for _ in range(nbuf)]
+    d2h_ev = [torch.cuda.Event() for _ in range(nbuf)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record(main)
+    cs.wait_event(start)
+    os_.wait_event(start)
+
+    def issue_h2d(n):
+        b = n % nbuf
+        with torch.cuda.stream(cs):
+            if n >= nbuf:
+                cs.wait_event(comp_ev[b])  # step n - nbuf has finished reading buffer set b
+            h2d_fn(n, b)
+            h2d_ev[b].record(cs)
+
+    issue_h2d(0)
+    for n in range(steps):
+        b = n % nbuf
+        if n + 1 < steps:
+            issue_h2d(n + 1)
+        main.wait_event(h2d_ev[b])
+        if n >= nbuf:
+            main.wait_event(d2h_ev[b])  # output buffer b has been copied out
+        compute_fn(n, b)
+        comp_ev[b].record(main)
+        with torch.cuda.stream(os_):
+            os_.wait_event(comp_ev[b])
+            d2h_fn(n, b)
+            d2h_ev[b].record(os_)
+    main.wait_stream(os_)
+    end.record(main)
+    torch.cuda.synchronize()
+    return start.elapsed_time(end)
+
+
 def job_throughput(tokens_per_rank: int, steps: int, world: int, max_ms: float) -> float:
     """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
     return world * tokens_per_rank * steps / (max_ms / 1e3)
@@ -507,14 +554,15 @@ def bench_prefill(args, name, rank, world, local, cpu_seconds):
         r_sel = torch.empty(shape.B, shape.Hkv, shape.N, dtype=torch.float32, device="cuda")
         idx_sel = torch.empty(shape.B, shape.Hkv, shape.T, shape.k, dtype=torch.int32, device="cuda")
 
-    def step(t):
+    def step(t, out=None):
+        out = o if out is None else out
         if diag:  # diagonal-only router: score, per-chunk top-k, then the layer on that selection
             still.still_diagonal_score(dims, t["q"], t["k"], r_sel)
             still.still_select_topk(dims, r_sel, idx_sel)
-            still.still_hybrid_prefill(dims, t["q"], t["k"], t["v"], t["wq"], t["wk"], o, idx_in=idx_sel,
+            still.still_hybrid_prefill(dims, t["q"], t["k"], t["v"], t["wq"], t["wk"], out, idx_in=idx_sel,
                                        workspace=ws)
         else:
-            still.still_hybrid_prefill(dims, t["q"], t["k"], t["v"], t["wq"], t["wk"], o, workspace=ws)
+            still.still_hybrid_prefill(dims, t["q"], t["k"], t["v"], t["wq"], t["wk"], out, workspace=ws)
 
     torch.cuda.synchronize()
     torch.cuda.reset_peak_memory_stats()
@@ -572,24 +620,29 @@ def bench_prefill(args, name, rank, world, local, cpu_seconds):
     tokens = shape.B * shape.N
     value = job_throughput(tokens, args.steps, world, total_ms)
 
-    # end to end through the same call with pinned host buffers
+    # end to end through the same call with pinned host buffers: every step copies its inputs up and
+    # its output down inside the timed region, pipelined across two buffer sets (pipelined_e2e)
     pinned = {n: t.pin_memory() for n, t in host.items()}
     o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in pinned.values())
     d2h = o_host.numel() * o_host.element_size()
-    e_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-             for _ in range(args.e2e_steps)]
-    for s_, e_ in e_evs:
+    dev_sets = [devt, {n: torch.empty_like(t) for n, t in devt.items()}]
+    o_sets = [o, torch.empty_like(o)]
+
+    def e2e_h2d(n, b):
+        for nm in dev_sets[b]:
+            dev_sets[b][nm].copy_(pinned[nm], non_blocking=True)
+
+    def e2e_compute(n, b):
         flush.zero_()
-        s_.record(stream)
-        for n in devt:
-            devt[n].copy_(pinned[n], non_blocking=True)
-        step(devt)
-        o_host.copy_(o, non_blocking=True)
-        e_.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(sum(s_.elapsed_time(e_) for s_, e_ in e_evs), world, "cuda")
+        step(dev_sets[b], o_sets[b])
+
+    def e2e_d2h(n, b):
+        o_host.copy_(o_sets[b], non_blocking=True)
+
+    e2e_ms = max_over_ranks(pipelined_e2e(args.e2e_steps, e2e_h2d, e2e_compute, e2e_d2h), world, "cuda")
     e2e_value = job_throughput(tokens, args.e2e_steps, world, e2e_ms)
+    del dev_sets, o_sets
     status = still.still_get_device_status()
 
     peaks = {}
@@ -620,7 +673,9 @@ def bench_prefill(args, name, rank, world, local, cpu_seconds):
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": shape.dtype, "data": "synthetic", "config": config_of(shape, args, name),
         "roofline": roofline,
-        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "pipelined": "inputs of step n+1 up and output of step n down on two copy streams, overlapping "
+                             "the compute of step n+1"},
         "gpu_launches": launches, "clocks": clocks,
         "kernel_ms_per_step": {k_: v_[0] / args.steps for k_, v_ in kern.items() if v_[1]},
         "layer_tflops": layer_flops(shape) / (ms_per_step / 1e3) / 1e12, "device_status": status,
@@ -814,22 +869,27 @@ def bench_decode(args, name, rank, world, local, cpu_seconds, all_steps=False):
     torch.cuda.synchronize()
     if still.still_get_device_status() != 0:
         raise RuntimeError("device-side check failed during warm-up")
-    # end to end: pinned host token -> device, step, o_t -> host
+    # end to end: each step's token goes up from pinned host memory and its output comes down inside
+    # the timed region, pipelined across two buffer sets (pipelined_e2e)
     pins = [t_.pin_memory() for t_ in (qd, kd, vd)]
     o_host = torch.empty(o_t.shape, dtype=tdt).pin_memory()
-    qb, kb, vb = (torch.empty_like(t_[0], device="cuda") for t_ in (qd, kd, vd))
-    e_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(e2e_steps)]
-    for s_, e_ in e_evs:
-        s_.record(stream)
-        qb.copy_(pins[0][pos - N], non_blocking=True)
-        kb.copy_(pins[1][pos - N], non_blocking=True)
-        vb.copy_(pins[2][pos - N], non_blocking=True)
-        still.still_decode_step(dims, state, cap, pos, wq, wk, qb, kb, vb, o_t)
-        o_host.copy_(o_t, non_blocking=True)
-        e_.record(stream)
-        pos += 1
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(sum(s_.elapsed_time(e_) for s_, e_ in e_evs), world, "cuda")
+    tok_sets = [[torch.empty_like(t_[0], device="cuda") for t_ in (qd, kd, vd)] for _ in range(2)]
+    ot_sets = [o_t, torch.empty_like(o_t)]
+    pos0 = pos
+
+    def e2e_h2d(n, b):
+        for x_, src_ in zip(tok_sets[b], pins):
+            x_.copy_(src_[pos0 + n - N], non_blocking=True)
+
+    def e2e_compute(n, b):
+        still.still_decode_step(dims, state, cap, pos0 + n, wq, wk, *tok_sets[b], ot_sets[b])
+
+    def e2e_d2h(n, b):
+        o_host.copy_(ot_sets[b], non_blocking=True)
+
+    e2e_ms = max_over_ranks(pipelined_e2e(e2e_steps, e2e_h2d, e2e_compute, e2e_d2h), world, "cuda")
+    pos += e2e_steps
+    qb, kb, vb = tok_sets[0]
     # untimed steps up to the timed region, which ends at the last position: it holds the step that
     # closes a chunk (position C-1 mod C) along with ordinary ones
     # the last (up to 64) of them also give the per-kernel breakdown, with events around each launch
@@ -896,7 +956,9 @@ def bench_decode(args, name, rank, world, local, cpu_seconds, all_steps=False):
                      "peak_source": "measured hbm_gbs" if "hbm_gbs" in peaks else "fallback 6.65 TB/s"},
         "e2e": {"value": job_throughput(B, e2e_steps, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": (qb.numel() + kb.numel() + vb.numel()) * qb.element_size(),
-                "d2h_bytes_per_step": o_host.numel() * o_host.element_size()},
+                "d2h_bytes_per_step": o_host.numel() * o_host.element_size(),
+                "pipelined": "token of step n+1 up and output of step n down on two copy streams, "
+                             "overlapping the compute of step n+1"},
         "gpu_launches": launches, "clocks": clocks,
         "kernel_ms_per_step": kernel_ms, "kernel_ms_steps": n_brk,
         "step_ms": {"median": float(np.median(times)), "max": float(max(times)),
