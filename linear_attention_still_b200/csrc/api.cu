@@ -217,13 +217,17 @@ still_status still_diagonal_score(const still_dims *dims, const void *q, const v
 
 namespace {
 // Backward scratch layout (256-byte aligned fp32 segments).
+constexpr int kBwdSegments = 14;
 size_t backward_layout(const Dims &s, size_t *off) {
     const size_t BH = (size_t)s.B * s.H, BK = (size_t)s.B * s.Hkv, T1 = (size_t)s.T() + 1;
-    const size_t sizes[11] = {BK * s.N * s.D, BK * T1 * s.D * s.d, BK * T1 * s.D, BH * s.N * s.D, BH * s.N,
-                              BH * s.N * s.D, BK * T1 * s.D * s.d, BK * T1 * s.D, BK * s.N * s.D, BH * s.N,
-                              BH * s.N};
+    // tensor-core path: the rows' log2 normalisers and the gathered kept rows (bf16, in fp32 units)
+    const bool tc = tc_backward_supported(s);
+    const size_t kept = tc ? (BK * s.T() * s.k * s.d * 2 + 3) / 4 : 0;
+    const size_t sizes[kBwdSegments] = {BK * s.N * s.D, BK * T1 * s.D * s.d, BK * T1 * s.D, BH * s.N * s.D, BH * s.N,
+                                        BH * s.N * s.D, BK * T1 * s.D * s.d, BK * T1 * s.D, BK * s.N * s.D, BH * s.N,
+                                        BH * s.N, tc ? BH * s.N : 0, kept, kept};
     size_t o = 0;
-    for (int i = 0; i < 11; ++i) {
+    for (int i = 0; i < kBwdSegments; ++i) {
         off[i] = o;
         o += (sizes[i] * 4 + 255) & ~(size_t)255;
     }
@@ -234,7 +238,7 @@ size_t backward_layout(const Dims &s, size_t *off) {
 size_t still_backward_workspace_bytes(const still_dims *dims) {
     Dims s;
     if (check_dims(dims, &s)) return 0;
-    size_t off[11];
+    size_t off[kBwdSegments];
     return backward_layout(s, off);
 }
 
@@ -252,12 +256,12 @@ still_status still_hybrid_backward(const still_dims *dims, const void *q, const 
         if (!p || !aligned16(p)) return STILL_ERR_INVALID_ARG;
     const bool select = s.k > 0 && s.T() > 0;
     if (select && (!idx || !aligned16(idx))) return STILL_ERR_INVALID_ARG;
-    size_t off[11];
+    size_t off[kBwdSegments];
     if (workspace_bytes < backward_layout(s, off)) return STILL_ERR_WORKSPACE;
     if (((uintptr_t)workspace & 255u) != 0) return STILL_ERR_INVALID_ARG;
     unsigned char *ws = static_cast<unsigned char *>(workspace);
     auto F = [&](int i) { return reinterpret_cast<float *>(ws + off[i]); };
-    BackwardScratch w{F(0), F(1), F(2), F(3), F(4), F(9), F(10), F(5), F(6), F(7), F(8)};
+    BackwardScratch w{F(0), F(1), F(2), F(3), F(4), F(9), F(10), F(5), F(6), F(7), F(8), F(11), F(12), F(13)};
     int launches = 0;
     cudaError_t e = launch_backward(s, q, k, v, Wq, Wk, select ? idx : nullptr, dO, dq, dk, dv, dWq, dWk, w,
                                     device_error_word(), static_cast<cudaStream_t>(stream), &launches);

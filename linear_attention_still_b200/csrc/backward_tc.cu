@@ -1,0 +1,701 @@
+// backward_tc.cu -- the softmax branch of the STILL layer's backward pass on sm_100a tensor cores
+// (bf16 storage, fp32 accumulation in TMEM).  "STILL: Selecting Tokens for Intra-Layer Hybrid
+// Attention to Linearize LLMs": [p1] jsqmd.com introduction and "Chunk-Wise" (one chunk-parallel
+// implementation serves training and inference); [p4] atlas.scime.ai "Approach".
+//
+// For query row i (head h of group g, chunk t) the softmax set is Soft(i) = the kept rows of chunks
+// 0..t-m-1 (the compact kept cache) ++ the window [max(0,(t-m)C), i]; the linear branch enters the
+// shared normaliser.  In log2 units (x_ij = tau log2(e) <q_i, k_j>):
+//   M = max_j x_ij,  l = sum_j 2^(x_ij - M),  u = sum_j 2^(x_ij - M) <dO_i, v_j>,
+//   Ms = max(M, log2 lden_i),  Z = l 2^(M - Ms) + lden_i 2^-Ms,  L_i = Ms + log2 Z,
+//   D_i = <dO_i, o_i> = (u 2^(M - Ms) + dl_i 2^-Ms) / Z,
+// with lden_i = phi(q_i).z_t and dl_i = <phi(q_i)^T S_t, dO_i> from the linear pre-pass.  Then
+//   P_ij = 2^(x_ij - L_i),  dS_ij = P_ij (<dO_i, v_j> - D_i),
+//   dq_i = tau sum_j dS_ij k_j,  dk_j = tau sum_i dS_ij q_i,  dv_j = sum_i P_ij dO_i.
+//
+// bwd_dq_tc_kernel: one CTA per (b, h, 128 query rows).  Two sweeps over the row tile's keys in tiles
+// of 64: sweep 1 forms S = Q K^T and dP = dO V^T (tcgen05, TMEM lane = row) and accumulates M, l, u in
+// registers; the row's L_i and D_i follow (written for the key pass); sweep 2 forms S and dP again,
+// dS (bf16) over dP's TMEM columns, and dQ += dS K with dS as the TMEM operand.
+// bwd_dkv_tc_kernel: one CTA per (b, g, 128 keys) [kept keys: per 128 kept-cache entries and one
+// segment of query rows].  For each head of the group and each 64-row query tile that sees the keys:
+// S^T = K Q^T and dP^T = V dO^T (TMEM lane = key), P^T and dS^T (bf16) over their own columns, then
+// dV += P^T dO and dK += dS^T Q with P^T / dS^T as TMEM operands; the accumulators stay in TMEM for
+// the whole CTA.  Window keys write dk, dv; kept keys add into the rows their entries name.
+//
+// Roles in both kernels: four row warps (TMEM lanes), one TMA producer warp, one MMA warp (which
+// also allocates TMEM).  Every mbarrier wait is bounded; on a timeout the CTA records
+// DEV_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "still_internal.h"
+#include "tc_ptx.cuh"
+#include "tc_tile.cuh"
+
+namespace still {
+
+using namespace tc;
+
+namespace {
+
+struct BwdParams {
+    int B, H, Hkv, N, C, k, w, G, T;
+    float scale, scale_log2;  // tau, tau log2(e)
+    const float *lden, *dl;   // [B,H,N] from the linear pre-pass (dq kernel)
+    float *L, *Dv;            // [B,H,N] log2 normaliser and D_i (dq kernel writes, key kernel reads)
+    float *dq, *dk, *dv;      // fp32 gradients
+    const int32_t *idx;       // [B,Hkv,T,k] (kept keys)
+    int n_qtiles;             // dq kernel: ceil(N / 128)
+    int n_ktiles;             // key kernel: 128-key tiles per (b, g)
+    int seg_rows;             // kept keys: query rows per segment
+    unsigned *err;
+};
+
+// ================================================================================ dq kernel
+template <int DH>
+struct BwdQCfg {
+    static constexpr int Q_REG = 128 * 128;          // 128 rows x 64 bf16 (one SW128 region)
+    static constexpr int K_REG = 64 * 128;           // 64 rows x 64 bf16
+    static constexpr int Q_BYTES = 128 * DH * 2;     // Q / dO tile (DH/64 regions)
+    static constexpr int K_BYTES = 64 * DH * 2;      // K / V tile of 64 keys
+    static constexpr int NS = DH == 64 ? 4 : 2;      // K/V stages
+    static constexpr int STAGE_BYTES = 2 * K_BYTES;
+    static constexpr int OFF_Q = 0, OFF_DO = Q_BYTES, OFF_STAGE = 2 * Q_BYTES,
+                         OFF_BAR = OFF_STAGE + NS * STAGE_BYTES;
+    static constexpr int B_QFULL = 0, B_S = 1, B_SDONE = 2, B_DQ = 3, B_DRAIN = 4, B_KFULL = 5,
+                         B_VFULL = 5 + NS, B_KVEMPTY = 5 + 2 * NS, NUM_BARS = 5 + 3 * NS;
+    static constexpr int TMEM_SLOT_OFF = 8 * NUM_BARS, ABORT_OFF = TMEM_SLOT_OFF + 8, BAR_BYTES = 256;
+    static_assert(ABORT_OFF + 8 <= BAR_BYTES, "barrier area overflow");
+    static constexpr int SMEM = OFF_BAR + BAR_BYTES + 1024;
+    static constexpr int THREADS = 192, PRODUCER_WARP = 4, MMA_WARP = 5;
+    // S (64 keys), dP (64 keys; dS in bf16 over its first 32 columns), dQ (DH)
+    static constexpr int S_COL = 0, DP_COL = 64, DQ_COL = 128, TMEM_COLS = 256;
+    static_assert(DQ_COL + DH <= TMEM_COLS, "TMEM budget");
+    static constexpr int MIN_BLOCKS = DH == 64 ? 2 : 1;  // two CTAs per SM overlap each other's phases
+    static_assert(MIN_BLOCKS * (SMEM + 1024) <= 233472, "shared memory per SM");
+};
+
+template <int DH>
+__global__ void __launch_bounds__(BwdQCfg<DH>::THREADS, BwdQCfg<DH>::MIN_BLOCKS)
+    bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_do,
+                     const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
+                     const __grid_constant__ CUtensorMap map_kh, const __grid_constant__ CUtensorMap map_vh,
+                     const BwdParams p) {
+    using Cfg = BwdQCfg<DH>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    uint8_t *bar_area = smem + Cfg::OFF_BAR;
+    const uint32_t sBar = smem_u32(bar_area);
+    auto BAR = [&](int i) { return sBar + 8u * i; };
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_area + Cfg::TMEM_SLOT_OFF);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bar_area + Cfg::ABORT_OFF);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // CTA -> (b, h, query tile); later query tiles (more kept keys) first
+    const int per_qt = p.B * p.H;
+    const int qt = p.n_qtiles - 1 - (int)(blockIdx.x / per_qt);
+    const int bh = blockIdx.x % per_qt;
+    const int b = bh / p.H, h = bh % p.H, g = h / p.G;
+    const int bg = b * p.Hkv + g;
+    const int i0 = qt * 128;
+    const int t = i0 / p.C, m = p.w / p.C;
+    const int nk = p.k * max(0, t - m);                 // kept rows seen by this chunk
+    const int lo = max(0, (t - m) * p.C);               // window start
+    const int nkt = (nk + 63) / 64;                     // kept tiles
+    const int nt = nkt + (i0 + 128 - lo) / 64;          // key tiles per sweep
+    const int ntot = 2 * nt;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < Cfg::NUM_BARS; ++i) mbar_init(BAR(i), i == Cfg::B_SDONE ? 128 : 1);
+        *abort_flag = 0;
+        mbar_fence_init();
+    }
+    if (warp == Cfg::MMA_WARP) {
+        tmem_alloc(smem_u32(tmem_slot), Cfg::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == Cfg::PRODUCER_WARP) {
+        // ================================================================ TMA producer (whole warp)
+        bool ok = true;
+        int issued = 0;
+        mbar_arrive_expect_tx_w(BAR(Cfg::B_QFULL), 2 * Cfg::Q_BYTES);
+        for (int rr = 0; rr < DH / 64; ++rr) {
+            tma_load_3d_w(sbase + Cfg::OFF_Q + rr * Cfg::Q_REG, &map_q, BAR(Cfg::B_QFULL), rr * 64, i0, bh);
+            tma_load_3d_w(sbase + Cfg::OFF_DO + rr * Cfg::Q_REG, &map_do, BAR(Cfg::B_QFULL), rr * 64, i0, bh);
+        }
+        for (int jj = 0; jj < ntot; ++jj) {
+            const int s = jj % Cfg::NS;
+            if (jj >= Cfg::NS && !(ok = mbar_wait_w(BAR(Cfg::B_KVEMPTY + s), ((jj / Cfg::NS) - 1) & 1, abort_flag)))
+                break;
+            const int j = jj < nt ? jj : jj - nt;
+            const bool kept = j < nkt;
+            const int row = kept ? 64 * j : lo + 64 * (j - nkt);
+            const CUtensorMap *mk = kept ? &map_kh : &map_k;
+            const CUtensorMap *mv = kept ? &map_vh : &map_v;
+            const uint32_t sK = sbase + Cfg::OFF_STAGE + s * Cfg::STAGE_BYTES, sV = sK + Cfg::K_BYTES;
+            mbar_arrive_expect_tx_w(BAR(Cfg::B_KFULL + s), Cfg::K_BYTES);
+            for (int rr = 0; rr < DH / 64; ++rr)
+                tma_load_3d_w(sK + rr * Cfg::K_REG, mk, BAR(Cfg::B_KFULL + s), rr * 64, row, bg);
+            mbar_arrive_expect_tx_w(BAR(Cfg::B_VFULL + s), Cfg::K_BYTES);
+            for (int rr = 0; rr < DH / 64; ++rr)
+                tma_load_3d_w(sV + rr * Cfg::K_REG, mv, BAR(Cfg::B_VFULL + s), rr * 64, row, bg);
+            issued = jj + 1;
+        }
+        if (!ok) {
+            *abort_flag = 1;
+            if (lane == 0) report(p.err, DEV_ERR_TIMEOUT);
+            mbar_wait_drain(BAR(Cfg::B_QFULL), 0, 100000000ull);
+            for (int jj = max(0, issued - Cfg::NS); jj < issued; ++jj) {
+                mbar_wait_drain(BAR(Cfg::B_KFULL + jj % Cfg::NS), (jj / Cfg::NS) & 1, 100000000ull);
+                mbar_wait_drain(BAR(Cfg::B_VFULL + jj % Cfg::NS), (jj / Cfg::NS) & 1, 100000000ull);
+            }
+        }
+    } else if (warp == Cfg::MMA_WARP) {
+        // ================================================================ MMA issuer (whole warp)
+        const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
+        constexpr uint32_t ID_S = idesc_bf16(128, 64, 0, 0);
+        constexpr uint32_t ID_DQ = idesc_bf16(128, DH, 0, 1);
+        const uint32_t sQ = sbase + Cfg::OFF_Q, sDO = sbase + Cfg::OFF_DO;
+        // dQ += dS K for tile jj (sweep 2): dS (bf16, 64 keys = 32 columns) from TMEM, K as the
+        // MN-major B operand (N = DH, K = 64 keys; 16 keys = 16 rows of 128 bytes per k-step)
+        auto issue_dq = [&](int jj) {
+            const uint64_t dk = sw128_desc(sbase + Cfg::OFF_STAGE + (jj % Cfg::NS) * Cfg::STAGE_BYTES, Cfg::K_REG, 1024);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                mma_ts_w(tm + Cfg::DQ_COL, tm + Cfg::DP_COL + kk * 8, dk + (uint64_t)(kk * 128), ID_DQ,
+                         (jj > nt || kk > 0) ? 1u : 0u);
+            mma_commit_w(BAR(Cfg::B_KVEMPTY + jj % Cfg::NS));
+        };
+        bool ok = mbar_wait_w(BAR(Cfg::B_QFULL), 0, abort_flag);
+        for (int jj = 0; ok && jj < ntot; ++jj) {
+            const int s = jj % Cfg::NS;
+            const uint32_t sK = sbase + Cfg::OFF_STAGE + s * Cfg::STAGE_BYTES, sV = sK + Cfg::K_BYTES;
+            if (!(ok = mbar_wait_w(BAR(Cfg::B_KFULL + s), (jj / Cfg::NS) & 1, abort_flag))) break;
+            if (!(ok = mbar_wait_w(BAR(Cfg::B_VFULL + s), (jj / Cfg::NS) & 1, abort_flag))) break;
+            if (jj > 0) {
+                // the row warps have read S, dP of tile jj-1 (and written its dS in sweep 2)
+                if (!(ok = mbar_wait_w(BAR(Cfg::B_SDONE), (jj - 1) & 1, abort_flag))) break;
+                tc_fence_after();
+                if (jj - 1 >= nt) issue_dq(jj - 1);  // in issue order before S, dP(jj) overwrite dS
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < DH / 16; ++kk)
+                mma_ss_w(tm + Cfg::S_COL, kmajor_desc(sQ, kk, Cfg::Q_REG), kmajor_desc(sK, kk, Cfg::K_REG), ID_S, kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < DH / 16; ++kk)
+                mma_ss_w(tm + Cfg::DP_COL, kmajor_desc(sDO, kk, Cfg::Q_REG), kmajor_desc(sV, kk, Cfg::K_REG), ID_S, kk > 0);
+            mma_commit_w(BAR(Cfg::B_S));
+            if (jj < nt) mma_commit_w(BAR(Cfg::B_KVEMPTY + s));  // sweep 1: the stage is done with
+        }
+        if (ok && (ok = mbar_wait_w(BAR(Cfg::B_SDONE), (ntot - 1) & 1, abort_flag))) {
+            tc_fence_after();
+            issue_dq(ntot - 1);
+            mma_commit_w(BAR(Cfg::B_DQ));
+        }
+        if (!ok) {
+            *abort_flag = 1;
+            if (lane == 0) report(p.err, DEV_ERR_TIMEOUT);
+        }
+        mma_commit_w(BAR(Cfg::B_DRAIN));
+        mbar_wait_drain(BAR(Cfg::B_DRAIN), 0, 100000000ull);
+    } else {
+        // ================================================================ row warps (TMEM lane = query row)
+        const int r = warp * 32 + lane;
+        const int i = i0 + r;
+        const bool live = i < p.N;
+        const size_t row = (size_t)bh * p.N + i;
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const uint32_t tS = tmem + lane_off + Cfg::S_COL, tDP = tmem + lane_off + Cfg::DP_COL,
+                       tDQ = tmem + lane_off + Cfg::DQ_COL;
+        const float lden = live ? p.lden[row] : 0.f, dl = live ? p.dl[row] : 0.f;
+        const float sl2 = p.scale_log2;
+        float M = -INFINITY, l = 0.f, u = 0.f, Lr = 0.f, Di = 0.f;
+        bool ok = true;
+        for (int jj = 0; jj < ntot; ++jj) {
+            if (!(ok = warp_all(mbar_wait(BAR(Cfg::B_S), jj & 1, abort_flag)))) break;
+            tc_fence_after();
+            const int j = jj < nt ? jj : jj - nt;
+            // columns c < lim are in Soft(i): kept entries below nk, window keys at or before i
+            const int lim = j < nkt ? nk - 64 * j : i - (lo + 64 * (j - nkt)) + 1;
+            if (jj < nt) {
+                // ---- sweep 1: running max, sum and sum of exp * <dO, v>
+                float sv[64];
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t w[32];
+                    tmem_ld32(tS + c * 32, w);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) sv[c * 32 + e] = c * 32 + e < lim ? __uint_as_float(w[e]) * sl2 : -INFINITY;
+                }
+                float mt = -INFINITY;
+#pragma unroll
+                for (int c = 0; c < 64; ++c) mt = fmaxf(mt, sv[c]);
+                const float mn = fmaxf(M, mt);
+                const float mref = mn == -INFINITY ? 0.f : mn;
+                const float sc = M == -INFINITY ? 0.f : ex2(M - mref);
+                float la = 0.f, lb = 0.f, ua = 0.f, ub = 0.f;
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t w[32];
+                    tmem_ld32(tDP + c * 32, w);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        const float p0 = ex2(sv[c * 32 + e] - mref), p1 = ex2(sv[c * 32 + e + 1] - mref);
+                        la += p0;
+                        lb += p1;
+                        ua = fmaf(p0, __uint_as_float(w[e]), ua);
+                        ub = fmaf(p1, __uint_as_float(w[e + 1]), ub);
+                    }
+                }
+                l = fmaf(l, sc, la + lb);
+                u = fmaf(u, sc, ua + ub);
+                M = mn;
+                tc_fence_before();
+                mbar_arrive(BAR(Cfg::B_SDONE));
+                if (jj == nt - 1) {
+                    // ---- the row's normaliser with the linear branch, and D_i
+                    const float Ms = lden > 0.f ? fmaxf(M, __log2f(lden)) : M;
+                    const float a_soft = ex2(M - Ms), a_lin = lden > 0.f ? ex2(-Ms) : 0.f;
+                    const float Z = fmaf(l, a_soft, lden * a_lin);
+                    Lr = Ms + __log2f(Z);
+                    Di = fmaf(u, a_soft, dl * a_lin) / Z;
+                    if (live) {
+                        p.L[row] = Lr;
+                        p.Dv[row] = Di;
+                    }
+                }
+            } else {
+                // ---- sweep 2: P = 2^(x - L), dS = P (dP - D) in bf16 over dP's first 32 columns
+                const float2 sc2 = make_float2(sl2, sl2), nl2 = make_float2(-Lr, -Lr);
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t ws[32], wd[32], pk[16];
+                    tmem_ld32(tS + c * 32, ws);
+                    tmem_ld32(tDP + c * 32, wd);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int c0 = c * 32 + 2 * e;
+                        const float2 x = ffma2(make_float2(__uint_as_float(ws[2 * e]), __uint_as_float(ws[2 * e + 1])),
+                                               sc2, nl2);
+                        const float d0 = c0 < lim ? ex2(x.x) * (__uint_as_float(wd[2 * e]) - Di) : 0.f;
+                        const float d1 = c0 + 1 < lim ? ex2(x.y) * (__uint_as_float(wd[2 * e + 1]) - Di) : 0.f;
+                        pk[e] = pack_bf16x2(d0, d1);
+                    }
+                    // columns [16c, 16c + 16) of dP were read above (chunk c loaded columns 32c..32c+31)
+                    tmem_st16(tDP + c * 16, pk);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(BAR(Cfg::B_SDONE));
+            }
+        }
+        // ---- epilogue: dq = tau dQ (fp32)
+        ok = warp_all(ok && mbar_wait(BAR(Cfg::B_DQ), 0, abort_flag));
+        if (ok) {
+            tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < DH / 32; ++c) {
+                uint32_t w[32];
+                tmem_ld32(tDQ + c * 32, w);
+                tmem_wait_ld();
+                if (live) {
+                    float4 *dst = reinterpret_cast<float4 *>(p.dq + row * DH + c * 32);
+#pragma unroll
+                    for (int v4 = 0; v4 < 8; ++v4)
+                        dst[v4] = make_float4(__uint_as_float(w[4 * v4]) * p.scale, __uint_as_float(w[4 * v4 + 1]) * p.scale,
+                                              __uint_as_float(w[4 * v4 + 2]) * p.scale,
+                                              __uint_as_float(w[4 * v4 + 3]) * p.scale);
+                }
+            }
+        }
+        if (!ok) {
+            *abort_flag = 1;
+            if (lane == 0) report(p.err, DEV_ERR_TIMEOUT);
+        }
+    }
+
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == Cfg::MMA_WARP) tmem_dealloc(tmem, Cfg::TMEM_COLS);
+}
+
+// ================================================================================ key kernel
+template <int DH>
+struct BwdKVCfg {
+    static constexpr int K_REG = 128 * 128;          // 128 rows x 64 bf16
+    static constexpr int Q_REG = 64 * 128;           // 64 rows x 64 bf16
+    static constexpr int K_BYTES = 128 * DH * 2;     // K / V tile of 128 keys
+    static constexpr int Q_BYTES = 64 * DH * 2;      // Q / dO tile of 64 query rows
+    static constexpr int NS = DH == 64 ? 4 : 2;      // query stages
+    static constexpr int STAGE_BYTES = 2 * Q_BYTES + 1024;  // Q, dO, then L and D of the 64 rows
+    static constexpr int OFF_K = 0, OFF_V = K_BYTES, OFF_STAGE = 2 * K_BYTES,
+                         OFF_BAR = OFF_STAGE + NS * STAGE_BYTES;
+    static constexpr int B_KVFULL = 0, B_S = 1, B_SDONE = 2, B_ACC = 3, B_DRAIN = 4, B_QFULL = 5,
+                         B_STFULL = 5 + NS, B_QEMPTY = 5 + 2 * NS, NUM_BARS = 5 + 3 * NS;
+    static constexpr int TMEM_SLOT_OFF = 8 * NUM_BARS, ABORT_OFF = TMEM_SLOT_OFF + 8, BAR_BYTES = 256;
+    static_assert(ABORT_OFF + 8 <= BAR_BYTES, "barrier area overflow");
+    static constexpr int SMEM = OFF_BAR + BAR_BYTES + 1024;
+    static constexpr int THREADS = 192, PRODUCER_WARP = 4, MMA_WARP = 5;
+    // S^T (64 queries; P^T in bf16 over its first 32 columns), dP^T (dS^T likewise), dV, dK
+    static constexpr int S_COL = 0, DP_COL = 64, DV_COL = 128, DK_COL = 128 + DH;
+    static constexpr int TMEM_COLS = DH == 64 ? 256 : 512;
+    static_assert(DK_COL + DH <= TMEM_COLS, "TMEM budget");
+    static constexpr int MIN_BLOCKS = DH == 64 ? 2 : 1;
+    static_assert(MIN_BLOCKS * (SMEM + 1024) <= 233472, "shared memory per SM");
+};
+
+template <int DH, bool KEPT>
+__global__ void __launch_bounds__(BwdKVCfg<DH>::THREADS, BwdKVCfg<DH>::MIN_BLOCKS)
+    bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
+                      const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_do,
+                      const BwdParams p) {
+    using Cfg = BwdKVCfg<DH>;
+    const int BK = p.B * p.Hkv;
+    const int bg = blockIdx.x % BK, b = bg / p.Hkv, g = bg % p.Hkv;
+    const int kt = (blockIdx.x / BK) % p.n_ktiles;
+    const int m = p.w / p.C;
+    const int j0 = kt * 128;  // first key (window) or kept-cache entry (kept) of the tile
+    int qbeg, qend;
+    if (!KEPT) {
+        qbeg = j0;
+        qend = min(p.N, (j0 / p.C + m + 1) * p.C);
+    } else {
+        const int seg = (int)(blockIdx.x / BK) / p.n_ktiles;
+        qbeg = (j0 / p.k + m + 1) * p.C + seg * p.seg_rows;  // queries that see the tile's first chunk
+        qend = min(p.N, qbeg + p.seg_rows);
+        if (qbeg >= p.N) return;  // (uniform over the CTA, before any barrier or TMEM use)
+    }
+    const int nqt = (qend - qbeg + 63) / 64;
+    const int tiles = p.G * nqt;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    uint8_t *bar_area = smem + Cfg::OFF_BAR;
+    const uint32_t sBar = smem_u32(bar_area);
+    auto BAR = [&](int i) { return sBar + 8u * i; };
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_area + Cfg::TMEM_SLOT_OFF);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bar_area + Cfg::ABORT_OFF);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < Cfg::NUM_BARS; ++i) {
+            const bool stats = i >= Cfg::B_STFULL && i < Cfg::B_STFULL + Cfg::NS;
+            mbar_init(BAR(i), i == Cfg::B_SDONE ? 128 : stats ? 32 : 1);
+        }
+        *abort_flag = 0;
+        mbar_fence_init();
+    }
+    if (warp == Cfg::MMA_WARP) {
+        tmem_alloc(smem_u32(tmem_slot), Cfg::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == Cfg::PRODUCER_WARP) {
+        // ================================================================ TMA producer (whole warp)
+        bool ok = true;
+        int issued = 0;
+        mbar_arrive_expect_tx_w(BAR(Cfg::B_KVFULL), 2 * Cfg::K_BYTES);
+        for (int rr = 0; rr < DH / 64; ++rr) {
+            tma_load_3d_w(sbase + Cfg::OFF_K + rr * Cfg::K_REG, &map_k, BAR(Cfg::B_KVFULL), rr * 64, j0, bg);
+            tma_load_3d_w(sbase + Cfg::OFF_V + rr * Cfg::K_REG, &map_v, BAR(Cfg::B_KVFULL), rr * 64, j0, bg);
+        }
+        for (int u = 0; u < tiles; ++u) {
+            const int s = u % Cfg::NS;
+            if (u >= Cfg::NS && !(ok = mbar_wait_w(BAR(Cfg::B_QEMPTY + s), ((u / Cfg::NS) - 1) & 1, abort_flag))) break;
+            const int hh = u / nqt, iq0 = qbeg + 64 * (u % nqt);
+            const int bh = b * p.H + g * p.G + hh;
+            const uint32_t sQ = sbase + Cfg::OFF_STAGE + s * Cfg::STAGE_BYTES, sDO = sQ + Cfg::Q_BYTES;
+            mbar_arrive_expect_tx_w(BAR(Cfg::B_QFULL + s), 2 * Cfg::Q_BYTES);
+            for (int rr = 0; rr < DH / 64; ++rr) {
+                tma_load_3d_w(sQ + rr * Cfg::Q_REG, &map_q, BAR(Cfg::B_QFULL + s), rr * 64, iq0, bh);
+                tma_load_3d_w(sDO + rr * Cfg::Q_REG, &map_do, BAR(Cfg::B_QFULL + s), rr * 64, iq0, bh);
+            }
+            // L and D of the 64 rows (zero past the sequence end; those columns are masked)
+            float *st = reinterpret_cast<float *>(smem + Cfg::OFF_STAGE + s * Cfg::STAGE_BYTES + 2 * Cfg::Q_BYTES);
+#pragma unroll
+            for (int e = lane; e < 64; e += 32) {
+                const int i = iq0 + e;
+                const size_t row = (size_t)bh * p.N + i;
+                st[e] = i < p.N ? p.L[row] : 0.f;
+                st[64 + e] = i < p.N ? p.Dv[row] : 0.f;
+            }
+            mbar_arrive(BAR(Cfg::B_STFULL + s));
+            issued = u + 1;
+        }
+        if (!ok) {
+            *abort_flag = 1;
+            if (lane == 0) report(p.err, DEV_ERR_TIMEOUT);
+            mbar_wait_drain(BAR(Cfg::B_KVFULL), 0, 100000000ull);
+            for (int u = max(0, issued - Cfg::NS); u < issued; ++u)
+                mbar_wait_drain(BAR(Cfg::B_QFULL + u % Cfg::NS), (u / Cfg::NS) & 1, 100000000ull);
+        }
+    } else if (warp == Cfg::MMA_WARP) {
+        // ================================================================ MMA issuer (whole warp)
+        const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
+        constexpr uint32_t ID_S = idesc_bf16(128, 64, 0, 0);
+        constexpr uint32_t ID_ACC = idesc_bf16(128, DH, 0, 1);
+        const uint32_t sK = sbase + Cfg::OFF_K, sV = sbase + Cfg::OFF_V;
+        // dV += P^T dO and dK += dS^T Q for tile u: P^T / dS^T (bf16, 64 queries = 32 columns) from
+        // TMEM, dO / Q as MN-major B operands (N = DH, K = 64 query rows; 16 rows per k-step)
+        auto issue_acc = [&](int u) {
+            const uint32_t sQ = sbase + Cfg::OFF_STAGE + (u % Cfg::NS) * Cfg::STAGE_BYTES, sDO = sQ + Cfg::Q_BYTES;
+            const uint64_t ddo = sw128_desc(sDO, Cfg::Q_REG, 1024), dqq = sw128_desc(sQ, Cfg::Q_REG, 1024);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                mma_ts_w(tm + Cfg::DV_COL, tm + Cfg::S_COL + kk * 8, ddo + (uint64_t)(kk * 128), ID_ACC,
+                         (u > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                mma_ts_w(tm + Cfg::DK_COL, tm + Cfg::DP_COL + kk * 8, dqq + (uint64_t)(kk * 128), ID_ACC,
+                         (u > 0 || kk > 0) ? 1u : 0u);
+            mma_commit_w(BAR(Cfg::B_QEMPTY + u % Cfg::NS));
+        };
+        bool ok = mbar_wait_w(BAR(Cfg::B_KVFULL), 0, abort_flag);
+        for (int u = 0; ok && u < tiles; ++u) {
+            const int s = u % Cfg::NS;
+            const uint32_t sQ = sbase + Cfg::OFF_STAGE + s * Cfg::STAGE_BYTES, sDO = sQ + Cfg::Q_BYTES;
+            if (!(ok = mbar_wait_w(BAR(Cfg::B_QFULL + s), (u / Cfg::NS) & 1, abort_flag))) break;
+            if (u > 0) {
+                if (!(ok = mbar_wait_w(BAR(Cfg::B_SDONE), (u - 1) & 1, abort_flag))) break;
+                tc_fence_after();
+                issue_acc(u - 1);  // in issue order before S^T, dP^T(u) overwrite P^T, dS^T
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < DH / 16; ++kk)
+                mma_ss_w(tm + Cfg::S_COL, kmajor_desc(sK, kk, Cfg::K_REG), kmajor_desc(sQ, kk, Cfg::Q_REG), ID_S, kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < DH / 16; ++kk)
+                mma_ss_w(tm + Cfg::DP_COL, kmajor_desc(sV, kk, Cfg::K_REG), kmajor_desc(sDO, kk, Cfg::Q_REG), ID_S, kk > 0);
+            mma_commit_w(BAR(Cfg::B_S));
+        }
+        if (ok && (ok = mbar_wait_w(BAR(Cfg::B_SDONE), (tiles - 1) & 1, abort_flag))) {
+            tc_fence_after();
+            issue_acc(tiles - 1);
+            mma_commit_w(BAR(Cfg::B_ACC));
+        }
+        if (!ok) {
+            *abort_flag = 1;
+            if (lane == 0) report(p.err, DEV_ERR_TIMEOUT);
+        }
+        mma_commit_w(BAR(Cfg::B_DRAIN));
+        mbar_wait_drain(BAR(Cfg::B_DRAIN), 0, 100000000ull);
+    } else {
+        // ================================================================ row warps (TMEM lane = key)
+        const int r = warp * 32 + lane;
+        const int TK = p.T * p.k;
+        // query rows i >= thr see this key: the key itself (window), or the chunk after the window
+        // that follows the entry's chunk (kept)
+        int thr;
+        if (!KEPT) thr = j0 + r;
+        else thr = j0 + r < TK ? ((j0 + r) / p.k + m + 1) * p.C : 0x7fffffff;
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const uint32_t tS = tmem + lane_off + Cfg::S_COL, tDP = tmem + lane_off + Cfg::DP_COL;
+        const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+        bool ok = true;
+        for (int u = 0; u < tiles; ++u) {
+            const int s = u % Cfg::NS;
+            if (!(ok = warp_all(mbar_wait(BAR(Cfg::B_S), u & 1, abort_flag) &&
+                                mbar_wait(BAR(Cfg::B_STFULL + s), (u / Cfg::NS) & 1, abort_flag))))
+                break;
+            tc_fence_after();
+            const int iq0 = qbeg + 64 * (u % nqt);
+            const int c_lo = thr - iq0, c_hi = p.N - iq0;  // columns c_lo <= c < c_hi count
+            const float *st = reinterpret_cast<const float *>(smem + Cfg::OFF_STAGE + s * Cfg::STAGE_BYTES + 2 * Cfg::Q_BYTES);
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                uint32_t ws[32], wd[32], pp[16], dd[16];
+                tmem_ld32(tS + c * 32, ws);
+                tmem_ld32(tDP + c * 32, wd);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const int c0 = c * 32 + 2 * e;
+                    const float2 Lc = *reinterpret_cast<const float2 *>(st + c0);
+                    const float2 Dc = *reinterpret_cast<const float2 *>(st + 64 + c0);
+                    const float2 x = ffma2(make_float2(__uint_as_float(ws[2 * e]), __uint_as_float(ws[2 * e + 1])), sc2,
+                                           make_float2(-Lc.x, -Lc.y));
+                    const bool v0 = c0 >= c_lo && c0 < c_hi, v1 = c0 + 1 >= c_lo && c0 + 1 < c_hi;
+                    const float p0 = v0 ? ex2(x.x) : 0.f, p1 = v1 ? ex2(x.y) : 0.f;
+                    const float d0 = v0 ? p0 * (__uint_as_float(wd[2 * e]) - Dc.x) : 0.f;
+                    const float d1 = v1 ? p1 * (__uint_as_float(wd[2 * e + 1]) - Dc.y) : 0.f;
+                    pp[e] = pack_bf16x2(p0, p1);
+                    dd[e] = pack_bf16x2(d0, d1);
+                }
+                // columns [16c, 16c + 16) were read above (chunk c loaded columns 32c..32c+31)
+                tmem_st16(tS + c * 16, pp);
+                tmem_st16(tDP + c * 16, dd);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(BAR(Cfg::B_SDONE));
+        }
+        // ---- epilogue: dv = dV, dk = tau dK (window: written; kept: added into the entry's row)
+        ok = warp_all(ok && mbar_wait(BAR(Cfg::B_ACC), 0, abort_flag));
+        if (ok) {
+            tc_fence_after();
+            int dst_row = -1;
+            if (!KEPT) {
+                if (j0 + r < p.N) dst_row = j0 + r;
+            } else if (j0 + r < TK && thr < p.N) {
+                const int e = j0 + r, c = e / p.k;
+                const int jr = p.idx[(size_t)bg * TK + e];
+                if (jr >= c * p.C && jr < (c + 1) * p.C) dst_row = jr;
+            }
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const uint32_t tA = tmem + lane_off + (half ? Cfg::DK_COL : Cfg::DV_COL);
+                float *out = half ? p.dk : p.dv;
+                const float f = half ? p.scale : 1.f;
+#pragma unroll
+                for (int c = 0; c < DH / 32; ++c) {
+                    uint32_t w[32];
+                    tmem_ld32(tA + c * 32, w);
+                    tmem_wait_ld();
+                    if (dst_row >= 0) {
+                        float4 *dst = reinterpret_cast<float4 *>(out + ((size_t)bg * p.N + dst_row) * DH + c * 32);
+#pragma unroll
+                        for (int v4 = 0; v4 < 8; ++v4) {
+                            const float4 val = make_float4(__uint_as_float(w[4 * v4]) * f, __uint_as_float(w[4 * v4 + 1]) * f,
+                                                           __uint_as_float(w[4 * v4 + 2]) * f,
+                                                           __uint_as_float(w[4 * v4 + 3]) * f);
+                            if (KEPT) atomicAdd(dst + v4, val);
+                            else dst[v4] = val;
+                        }
+                    }
+                }
+            }
+        }
+        if (!ok) {
+            *abort_flag = 1;
+            if (lane == 0) report(p.err, DEV_ERR_TIMEOUT);
+        }
+    }
+
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == Cfg::MMA_WARP) tmem_dealloc(tmem, Cfg::TMEM_COLS);
+}
+
+template <int DH>
+cudaError_t launch_bwd_cfg(const Dims &s, const void *q, const void *k, const void *v, const void *khat,
+                           const void *vhat, const void *dO, const BwdParams &prm_in, cudaStream_t st, int *launches) {
+    const int T = s.T();
+    const uint64_t BH = (uint64_t)s.B * s.H, BK = (uint64_t)s.B * s.Hkv;
+    const bool has_kept = s.k > 0 && T > 0;
+    BwdParams prm = prm_in;
+    // dq kernel: 128-row query / dO boxes, 64-row key boxes
+    CUtensorMap mq128, mdo128, mk64, mv64, mkh64, mvh64;
+    bool ok = make_map(&mq128, q, DH, s.N, BH, 128) && make_map(&mdo128, dO, DH, s.N, BH, 128) &&
+              make_map(&mk64, k, DH, s.N, BK, 64) && make_map(&mv64, v, DH, s.N, BK, 64);
+    if (has_kept)
+        ok = ok && make_map(&mkh64, khat, DH, (uint64_t)T * s.k, BK, 64) &&
+             make_map(&mvh64, vhat, DH, (uint64_t)T * s.k, BK, 64);
+    else
+        mkh64 = mk64, mvh64 = mv64;
+    if (!ok) return cudaErrorInvalidValue;
+    {
+        using Cfg = BwdQCfg<DH>;
+        prm.n_qtiles = (s.N + 127) / 128;
+        auto kern = bwd_dq_tc_kernel<DH>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+        if (e != cudaSuccess) return e;
+        kern<<<(unsigned)(prm.n_qtiles * BH), Cfg::THREADS, Cfg::SMEM, st>>>(mq128, mdo128, mk64, mv64, mkh64, mvh64,
+                                                                             prm);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        ++*launches;
+    }
+    // key kernels: 128-row key boxes, 64-row query / dO boxes
+    CUtensorMap mk128, mv128, mq64, mdo64, mkh128, mvh128;
+    ok = make_map(&mk128, k, DH, s.N, BK, 128) && make_map(&mv128, v, DH, s.N, BK, 128) &&
+         make_map(&mq64, q, DH, s.N, BH, 64) && make_map(&mdo64, dO, DH, s.N, BH, 64);
+    if (has_kept)
+        ok = ok && make_map(&mkh128, khat, DH, (uint64_t)T * s.k, BK, 128) &&
+             make_map(&mvh128, vhat, DH, (uint64_t)T * s.k, BK, 128);
+    if (!ok) return cudaErrorInvalidValue;
+    using Cfg = BwdKVCfg<DH>;
+    {
+        prm.n_ktiles = (s.N + 127) / 128;
+        auto kern = bwd_dkv_tc_kernel<DH, false>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+        if (e != cudaSuccess) return e;
+        kern<<<(unsigned)(prm.n_ktiles * BK), Cfg::THREADS, Cfg::SMEM, st>>>(mk128, mv128, mq64, mdo64, prm);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        ++*launches;
+    }
+    if (has_kept && (s.m() + 1) * s.C < s.N) {  // some query chunk decides chunk 0
+        // kept entries of chunks c with some deciding query chunk (c + m + 1 <= last chunk); the
+        // query rows of each 128-entry tile are split into segments so the long early tiles spread
+        prm.n_ktiles = (T * s.k + 127) / 128;
+        prm.seg_rows = 1024;
+        const int n_segs = (s.N + prm.seg_rows - 1) / prm.seg_rows;
+        auto kern = bwd_dkv_tc_kernel<DH, true>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+        if (e != cudaSuccess) return e;
+        kern<<<(unsigned)((uint64_t)n_segs * prm.n_ktiles * BK), Cfg::THREADS, Cfg::SMEM, st>>>(mkh128, mvh128, mq64,
+                                                                                                mdo64, prm);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        ++*launches;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace
+
+bool tc_backward_supported(const Dims &s) {
+    return s.bf16 && s.w > 0 && (s.d == 64 || s.d == 128) && s.C % 128 == 0 && s.N > 0;
+}
+
+// Softmax branch of the backward pass on tensor cores: dq (written), the rows' L and D, then dk, dv
+// (window keys written, kept keys added).  lden, dl come from the linear pre-pass.
+cudaError_t launch_backward_tc(const Dims &s, const void *q, const void *k, const void *v, const void *khat,
+                               const void *vhat, const int32_t *idx, const void *dO, const float *lden,
+                               const float *dl, float *L, float *Dv, float *dq, float *dk, float *dv, unsigned *err,
+                               cudaStream_t st, int *launches) {
+    BwdParams prm{};
+    prm.B = s.B;
+    prm.H = s.H;
+    prm.Hkv = s.Hkv;
+    prm.N = s.N;
+    prm.C = s.C;
+    prm.k = s.k;
+    prm.w = s.w;
+    prm.G = s.G();
+    prm.T = s.T();
+    prm.scale = s.scale;
+    prm.scale_log2 = s.scale * kLog2e;
+    prm.lden = lden;
+    prm.dl = dl;
+    prm.L = L;
+    prm.Dv = Dv;
+    prm.dq = dq;
+    prm.dk = dk;
+    prm.dv = dv;
+    prm.idx = idx;
+    prm.err = err;
+    if (s.d == 64) return launch_bwd_cfg<64>(s, q, k, v, khat, vhat, dO, prm, st, launches);
+    if (s.d == 128) return launch_bwd_cfg<128>(s, q, k, v, khat, vhat, dO, prm, st, launches);
+    return cudaErrorNotSupported;
+}
+
+}  // namespace still

@@ -504,6 +504,90 @@ __global__ void __launch_bounds__(256) bwd_weight_kernel(int B, int Hx, int N, i
     }
 }
 
+// Linear branch of one query row before the tensor-core softmax passes (one warp per row):
+// phi(q_i) -> Phi, sg_i = S_t dO_i -> SG, lden_i = phi(q_i).z_t and dl_i = <phi(q_i)^T S_t, dO_i> =
+// phi(q_i).sg_i (the two linear terms of the row's normaliser and of D_i).
+template <typename T>
+__global__ void __launch_bounds__(32 * kBwdWarps) bwd_lin_pre_kernel(Dims s, const T *__restrict__ q,
+                                                                     const T *__restrict__ Wq,
+                                                                     const float *__restrict__ S,
+                                                                     const float *__restrict__ z,
+                                                                     const T *__restrict__ dO, float *__restrict__ Phi,
+                                                                     float *__restrict__ SG, float *__restrict__ lden,
+                                                                     float *__restrict__ dl) {
+    __shared__ __align__(16) float qs[kBwdWarps][kMaxD];
+    __shared__ __align__(16) float gs[kBwdWarps][kMaxD];
+    __shared__ __align__(16) float ps[kBwdWarps][kMaxDf];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long row = (long long)blockIdx.x * kBwdWarps + warp;  // over B * H * N
+    if (row >= (long long)s.B * s.H * s.N) return;
+    const int d = s.d, D = s.D, G = s.G(), T_ = s.T();
+    const int i = (int)(row % s.N), h = (int)((row / s.N) % s.H), b = (int)(row / ((long long)s.N * s.H));
+    const int bg = b * s.Hkv + h / G, t = i / s.C;
+    for (int x = lane; x < d; x += 32) {
+        qs[warp][x] = to_f(q[(size_t)row * d + x]);
+        gs[warp][x] = to_f(dO[(size_t)row * d + x]);
+    }
+    __syncwarp();
+    npmap_row_warp<T>(qs[warp], Wq + (size_t)h * d * D, d, D, ps[warp], lane);
+    __syncwarp();
+    const size_t tslot = (size_t)bg * (T_ + 1) + t;
+    const float *St = S + tslot * D * d, *zt = z + tslot * D;
+    float ld = 0.f, dd = 0.f;
+    for (int a = lane; a < D; a += 32) {
+        const float sg = dot_row(gs[warp], St + (size_t)a * d, d);
+        const float ph = ps[warp][a];
+        ld = fmaf(ph, zt[a], ld);
+        dd = fmaf(ph, sg, dd);
+        Phi[(size_t)row * D + a] = ph;
+        SG[(size_t)row * D + a] = sg;
+    }
+    ld = warp_sum(ld);
+    dd = warp_sum(dd);
+    if (lane == 0) {
+        lden[row] = ld;
+        dl[row] = dd;
+    }
+}
+
+// Linear branch of one query row after the softmax passes (one warp per row), from the row's log2
+// normaliser L_i and D_i: c_i = 2^-L_i = exp(-Ms)/Z, dphi(q_i) = c_i (S_t dO_i - D_i z_t), then the
+// NP-Map backward (dq += dL/dq, dY -> dYq) and a_i = c_i phi(q_i) (in place of Phi) for the key side.
+template <typename T>
+__global__ void __launch_bounds__(32 * kBwdWarps) bwd_lin_post_kernel(Dims s, const T *__restrict__ q,
+                                                                      const T *__restrict__ Wq,
+                                                                      const float *__restrict__ z,
+                                                                      const float *__restrict__ L,
+                                                                      const float *__restrict__ Dv,
+                                                                      float *__restrict__ PhiA,
+                                                                      float *__restrict__ SGdY, float *__restrict__ dq) {
+    __shared__ __align__(16) float qs[kBwdWarps][kMaxD];
+    __shared__ __align__(16) float dps[kBwdWarps][kMaxDf];
+    __shared__ __align__(16) float dys[kBwdWarps][kMaxDf];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long row = (long long)blockIdx.x * kBwdWarps + warp;  // over B * H * N
+    if (row >= (long long)s.B * s.H * s.N) return;
+    const int d = s.d, D = s.D, G = s.G(), T_ = s.T();
+    const int i = (int)(row % s.N), h = (int)((row / s.N) % s.H), b = (int)(row / ((long long)s.N * s.H));
+    const int bg = b * s.Hkv + h / G, t = i / s.C;
+    for (int x = lane; x < d; x += 32) qs[warp][x] = to_f(q[(size_t)row * d + x]);
+    const float c = exp2f(-L[row]), Di = Dv[row];
+    const float *zt = z + ((size_t)bg * (T_ + 1) + t) * D;
+    for (int a = lane; a < D; a += 32) {
+        dps[warp][a] = c * (SGdY[(size_t)row * D + a] - Di * zt[a]);
+        PhiA[(size_t)row * D + a] *= c;
+    }
+    __syncwarp();
+    float dxa[kMaxD / 32];
+    npmap_backward_warp<T>(qs[warp], Wq + (size_t)h * d * D, d, D, dps[warp], dys[warp], dxa, lane);
+    for (int cc = lane; cc < D; cc += 32) SGdY[(size_t)row * D + cc] = dys[warp][cc];
+#pragma unroll
+    for (int u = 0; u < kMaxD / 32; ++u) {
+        const int x = lane + 32 * u;
+        if (x < d) dq[(size_t)row * d + x] += dxa[u];
+    }
+}
+
 template <typename T>
 cudaError_t backward_t(const Dims &s, const void *q, const void *k, const void *v, const void *Wq, const void *Wk,
                        const int32_t *idx, const void *dO, float *dq, float *dk, float *dv, float *dWq,
@@ -522,7 +606,34 @@ cudaError_t backward_t(const Dims &s, const void *q, const void *k, const void *
     if ((e = cudaMemsetAsync(w.dYk, 0, sizeof(float) * (size_t)s.B * s.Hkv * s.N * s.D, st)) != cudaSuccess) return e;
     const long long rows = (long long)s.B * s.H * s.N;
     const unsigned rgrid = (unsigned)((rows + kBwdWarps - 1) / kBwdWarps);
-    if (s.d == 64 || s.d == 128) {
+    if (tc_backward_supported(s)) {
+        // softmax branch on tensor cores: linear pre-pass (phi(q), S_t dO, lden, dl), then dq with
+        // the rows' normalisers, dk and dv by key tiles, then the linear branch's query and key sides
+        const bool tiled = tiled_linear_backward_supported(s);
+        if (s.k > 0 && T_ > 0) {
+            if ((e = launch_gather(s, idx, k, v, w.khat, w.vhat, err, st)) != cudaSuccess) return e;
+            ++*launches;
+        }
+        if (tiled) {
+            e = launch_linear_backward_tiled(0, s, q, k, v, Wq, Wk, dO, idx, w, dq, dk, dv, dWq, dWk, st);
+            if (e != cudaSuccess) return e;
+        } else {
+            bwd_lin_pre_kernel<T><<<rgrid, 32 * kBwdWarps, 0, st>>>(s, Q, WQ, w.S, w.z, GO, w.A, w.dYq, w.Ms, w.iZ);
+        }
+        ++*launches;
+        e = launch_backward_tc(s, q, k, v, w.khat, w.vhat, idx, dO, w.Ms, w.iZ, w.L, w.Dv, dq, dk, dv, err, st,
+                               launches);
+        if (e != cudaSuccess) return e;
+        if (tiled) {
+            // query side (dq, dWq), chunk sums, suffix, key side (dk, dv, dWk) of the linear branch
+            e = launch_linear_backward_tiled(1, s, q, k, v, Wq, Wk, dO, idx, w, dq, dk, dv, dWq, dWk, st);
+            if (e != cudaSuccess) return e;
+            *launches += T_ > 0 ? 4 : 3;
+            return cudaSuccess;
+        }
+        bwd_lin_post_kernel<T><<<rgrid, 32 * kBwdWarps, 0, st>>>(s, Q, WQ, w.z, w.L, w.Dv, w.A, w.dYq, dq);
+        ++*launches;
+    } else if (s.d == 64 || s.d == 128) {
         // dk, dv by key blocks (written there; no atomics)
         bwd_row_kernel<T, false><<<rgrid, 32 * kBwdWarps, 0, st>>>(s, Q, K, V, WQ, idx, w.S, w.z, GO, dq, dk, dv,
                                                                     w.A, w.Dv, w.Ms, w.iZ, w.dYq, err);
@@ -556,6 +667,13 @@ cudaError_t backward_t(const Dims &s, const void *q, const void *k, const void *
 }
 
 }  // namespace
+
+cudaError_t launch_bwd_suffix(const Dims &s, float *R, float *r, cudaStream_t st) {
+    const size_t ent = (size_t)s.B * s.Hkv * ((size_t)s.D * s.d + s.D);
+    if (ent == 0) return cudaSuccess;
+    bwd_suffix_kernel<<<(unsigned)((ent + 255) / 256), 256, 0, st>>>(s, R, r);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_backward(const Dims &s, const void *q, const void *k, const void *v, const void *Wq,
                             const void *Wk, const int32_t *idx, const void *dO, float *dq, float *dk, float *dv,

@@ -73,7 +73,22 @@ struct BackwardScratch {
     float *dYq;    // [B,H,N,D]     dL/d(q Wq)
     float *R, *r;  // [B,Hkv,T+1,D,d], [B,Hkv,T+1,D]  suffix sums over query chunks
     float *dYk;    // [B,Hkv,N,D]   dL/d(k Wk)
+    float *L;      // [B,H,N]       tensor-core path: each row's log2 normaliser Ms log2(e) + log2 Z
+    void *khat, *vhat;  // [B,Hkv,T*k,d] tensor-core path: the kept rows, gathered (bf16)
 };
+bool tc_backward_supported(const Dims &s);
+bool tiled_linear_backward_supported(const Dims &s);
+cudaError_t launch_linear_backward_tiled(int which, const Dims &s, const void *q, const void *k, const void *v,
+                                         const void *Wq, const void *Wk, const void *dO, const int32_t *idx,
+                                         const BackwardScratch &w, float *dq, float *dk, float *dv, float *dWq,
+                                         float *dWk, cudaStream_t st);
+cudaError_t launch_bwd_suffix(const Dims &s, float *R, float *r, cudaStream_t st);
+cudaError_t launch_gather(const Dims &s, const int32_t *idx, const void *k, const void *v, void *khat, void *vhat,
+                          unsigned *err, cudaStream_t st);
+cudaError_t launch_backward_tc(const Dims &s, const void *q, const void *k, const void *v, const void *khat,
+                               const void *vhat, const int32_t *idx, const void *dO, const float *lden,
+                               const float *dl, float *L, float *Dv, float *dq, float *dk, float *dv, unsigned *err,
+                               cudaStream_t st, int *launches);
 cudaError_t launch_backward(const Dims &s, const void *q, const void *k, const void *v, const void *Wq,
                             const void *Wk, const int32_t *idx, const void *dO, float *dq, float *dk, float *dv,
                             float *dWq, float *dWk, const BackwardScratch &w, unsigned *err, cudaStream_t st,

@@ -20,9 +20,19 @@ CASES = {
     # d in {64, 128} take dk, dv by key blocks (window pass + kept pass); the cases above with d = 32 by atomics
     "bf16_keep_all_d64": Shape(B=1, H=2, Hkv=1, N=200, d=64, D=32, w=64, C=64, k=64),
     "f32_two_chunk_window_d128": Shape(B=1, H=2, Hkv=1, N=230, d=128, D=64, w=64, C=32, k=8, dtype="f32"),
+    # bf16, d in {64, 128}, C a multiple of 128: the softmax branch on tensor cores (backward_tc.cu)
+    "tc_bf16_gqa_ragged": Shape(B=2, H=8, Hkv=2, N=700, d=64, D=64, w=128, C=128, k=16),
+    "tc_bf16_d128_two_chunk_window": Shape(B=1, H=4, Hkv=1, N=600, d=128, D=128, w=256, C=128, k=32),
+    "tc_bf16_kept_segments": Shape(B=1, H=4, Hkv=1, N=1400, d=64, D=64, w=128, C=128, k=32),
+    "tc_bf16_keep_all": Shape(B=1, H=2, Hkv=1, N=520, d=64, D=32, w=128, C=128, k=128),
+    "tc_bf16_keep_none_c256": Shape(B=1, H=2, Hkv=2, N=600, d=64, D=64, w=256, C=256, k=0),
 }
 # fp32 arithmetic on the GPU (dk, dv accumulate with atomics in schedule order) against fp64
 GRAD_TOL = {"f32": 1e-4, "bf16": 1e-3}
+# The tensor-core path rounds the MMA operands P and dS to bf16 (unit roundoff 2^-9 per product term,
+# independent between terms, so a sum's error is about 2^-9/sqrt(3) of its own rms); the bound on
+# max|err| / max|ref| keeps a margin of about 3.5 over that.
+TC_GRAD_TOL = 4e-3
 
 
 @pytest.fixture(scope="module")
@@ -62,7 +72,7 @@ def test_backward_matches_oracle(lib, oracle_mod, name):
     lib.still_hybrid_backward(d, dev(inp.q, shape), dev(inp.k, shape), dev(inp.v, shape), dev(inp.wq, shape),
                               dev(inp.wk, shape), idx_t, dev(do, shape), dq, dk, dv, dwq, dwk, workspace=ws)
     assert lib.still_get_device_status() == 0
-    tol = GRAD_TOL[shape.dtype]
+    tol = TC_GRAD_TOL if name.startswith("tc_") else GRAD_TOL[shape.dtype]
     for got, want, nm in zip((dq, dk, dv, dwq, dwk), ref, ("dq", "dk", "dv", "dWq", "dWk")):
         g = got.cpu().numpy()
         assert np.isfinite(g).all(), nm
