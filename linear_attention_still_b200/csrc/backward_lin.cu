@@ -9,13 +9,12 @@
 // with 4 x 4 register tiles (smem_mm), the per-row NP-Map steps on one warp per row.
 //   bwd_lin_pre_tile:  phi(q) (-> Phi), lden = phi(q).z_t, sg = S_t dO (-> SG), dl = phi(q).sg
 //   bwd_lin_post_tile: with L_i, D_i of the softmax pass: c = 2^-L, dphi = c (sg - D z_t),
-//                      a = c phi(q) (-> A, in place of Phi), the NP-Map backward dy, then
-//                      dq += dy Wq^T + (dn / ||q||) q and dWq += q^T dy (atomics)
-//   bwd_chunk_tile:    R_t = sum over the rows of query chunk t (all heads of the group) of a_i dO_i^T,
-//                      r_t = sum of a_i D_i
-//   bwd_key_tile:      unselected keys of a decided chunk c: with R, r the suffix sums from chunk
-//                      c + m + 1, dphi(k) = R v - r, dv += R^T phi(k), the NP-Map backward of k,
-//                      dk += dy Wk^T + (dn / ||k||) k and dWk += k^T dy (atomics)
+//                      a = c phi(q) (-> A, in place of Phi), the NP-Map backward dy (from phi alone),
+//                      then dq += dy Wq^T + (dn / ||q||) q, dWq += q^T dy, and the chunk sums of the
+//                      key side R_t += a^T dO, r_t += a^T D over the tile's rows (atomics)
+//   bwd_key_tile:      unselected keys of a decided chunk c: phi(k) from k Wk; with R, r the suffix
+//                      sums from chunk c + m + 1, dv += R^T phi(k), dphi(k) = R v - r, the NP-Map
+//                      backward of k, dk += dy Wk^T + (dn / ||k||) k and dWk += k^T dy (atomics)
 #include "common.cuh"
 #include "still_internal.h"
 
@@ -66,22 +65,65 @@ __device__ __forceinline__ void zero_acc(float (&acc)[MU][NU][4][4]) {
                 for (int j = 0; j < 4; ++j) acc[mu][nu][i][j] = 0.f;
 }
 
-// dst[r][c] (row stride ld) = src[r][c] for r < rows (zero for r >= valid), c < cols.
-template <typename T>
-__device__ __forceinline__ void load_rows(float *dst, int ld, const T *src, size_t sld, int rows, int cols, int valid) {
-    for (int e = threadIdx.x; e < rows * cols; e += kTileThreads) {
-        const int r = e / cols, c = e % cols;
-        dst[r * ld + c] = r < valid ? to_f(src[(size_t)r * sld + c]) : 0.f;
+// 16 bytes of a row: 8 bf16 or 4 fp32 values, widened to fp32.
+__device__ __forceinline__ void load16(const __nv_bfloat16 *p, float (&f)[8]) {
+    const uint4 u = *reinterpret_cast<const uint4 *>(p);
+    const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float2 t = __bfloat1622float2(h2[e]);
+        f[2 * e] = t.x;
+        f[2 * e + 1] = t.y;
+    }
+}
+__device__ __forceinline__ void load16(const float *p, float (&f)[4]) {
+    const float4 u = *reinterpret_cast<const float4 *>(p);
+    f[0] = u.x;
+    f[1] = u.y;
+    f[2] = u.z;
+    f[3] = u.w;
+}
+
+// dst[r][c] (row stride ld) = src[r][c] for r < ROWS (zero for r >= valid), c < COLS; rows of src
+// start on 16-byte boundaries (sld elements apart).  One 16-byte load per thread and step.
+template <int ROWS, int COLS, typename T>
+__device__ __forceinline__ void load_rows(float *dst, int ld, const T *src, size_t sld, int valid) {
+    constexpr int V = 16 / (int)sizeof(T), VPR = COLS / V;
+    static_assert(COLS % V == 0, "whole 16-byte vectors per row");
+#pragma unroll 2
+    for (int e = threadIdx.x; e < ROWS * VPR; e += kTileThreads) {
+        const int r = e / VPR, cv = e % VPR;
+        float f[V];
+        if (r < valid) {
+            load16(src + (size_t)r * sld + cv * V, f);
+        } else {
+#pragma unroll
+            for (int j = 0; j < V; ++j) f[j] = 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < V; j += 4)
+            *reinterpret_cast<float4 *>(dst + r * ld + cv * V + j) = make_float4(f[j], f[j + 1], f[j + 2], f[j + 3]);
     }
 }
 
-// dst[c][r] (row stride ld) = src[r][c], the transpose of the same block.
-template <typename T>
-__device__ __forceinline__ void load_rows_t(float *dst, int ld, const T *src, size_t sld, int rows, int cols,
-                                            int valid) {
-    for (int e = threadIdx.x; e < rows * cols; e += kTileThreads) {
-        const int r = e / cols, c = e % cols;
-        dst[c * ld + r] = r < valid ? to_f(src[(size_t)r * sld + c]) : 0.f;
+// dst[c][r] (row stride ld) = src[r][c], the transpose of the same block.  Consecutive threads take
+// consecutive rows, so the transposed shared-memory stores fall in consecutive banks.
+template <int ROWS, int COLS, typename T>
+__device__ __forceinline__ void load_rows_t(float *dst, int ld, const T *src, size_t sld, int valid) {
+    constexpr int V = 16 / (int)sizeof(T), VPR = COLS / V;
+    static_assert(COLS % V == 0 && ROWS % 32 == 0, "whole vectors, whole warps per column strip");
+#pragma unroll 2
+    for (int e = threadIdx.x; e < ROWS * VPR; e += kTileThreads) {
+        const int r = e % ROWS, cv = e / ROWS;
+        float f[V];
+        if (r < valid) {
+            load16(src + (size_t)r * sld + cv * V, f);
+        } else {
+#pragma unroll
+            for (int j = 0; j < V; ++j) f[j] = 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < V; ++j) dst[(cv * V + j) * ld + r] = f[j];
     }
 }
 
@@ -99,38 +141,30 @@ __device__ __forceinline__ void store_tile(float *dst, int ld, const float (&acc
                     make_float4(acc[mu][nu][i][0], acc[mu][nu][i][1], acc[mu][nu][i][2], acc[mu][nu][i][3]);
 }
 
-// NP-Map backward of one row (one warp; DF features, lane owns features lane + 32u): y = x W (fp32,
-// shared), ||x||^2, the upstream dphi -> dy = dL/dy written to dy_out (shared, stride-1), returns
-// dn / ||x|| (the coefficient of x in dL/dx; 0 when x = 0).
+// NP-Map backward of one row from phi itself (one warp; lane owns features lane + 32u): phi is a
+// positive multiple of f = softmax(y), so f = phi / sum(phi), ||x|| = ||phi|| and phi / ||x|| =
+// f / ||f||; x = 0 (phi = 0) has zero gradient.  Returns dn / ||x||, dy into dy.
 template <int DF>
-__device__ __forceinline__ float npmap_bwd_row(const float *y, float xx, const float (&dphi)[DF / 32], float *dy_out,
-                                               int lane) {
-    float f[DF / 32];
-    float mx = -INFINITY;
-#pragma unroll
-    for (int u = 0; u < DF / 32; ++u) mx = fmaxf(mx, y[lane + 32 * u]);
-    mx = warp_max(mx);
-    float se = 0.f;
+__device__ __forceinline__ float npmap_bwd_from_phi(const float (&ph)[DF / 32], const float (&dphi)[DF / 32],
+                                                    float (&dy)[DF / 32]) {
+    float sp = 0.f, pp = 0.f;
 #pragma unroll
     for (int u = 0; u < DF / 32; ++u) {
-        f[u] = expf(y[lane + 32 * u] - mx);
-        se += f[u];
+        sp += ph[u];
+        pp = fmaf(ph[u], ph[u], pp);
     }
-    se = warp_sum(se);
-    const float ise = 1.f / se;
-    float ff = 0.f;
+    sp = warp_sum(sp);
+    const float n = sqrtf(warp_sum(pp));
+    if (!(n > 0.f)) {
 #pragma unroll
-    for (int u = 0; u < DF / 32; ++u) {
-        f[u] *= ise;  // f = softmax(y)
-        ff = fmaf(f[u], f[u], ff);
+        for (int u = 0; u < DF / 32; ++u) dy[u] = 0.f;
+        return 0.f;
     }
-    const float nf = sqrtf(warp_sum(ff)), inf_ = 1.f / nf;
-    const float n = sqrtf(xx);
-    // phi = n u, u = f / ||f||
+    const float isp = 1.f / sp, in = 1.f / n, inf_ = sp * in;  // 1 / ||f|| = sum(phi) / ||phi||
     float dn = 0.f, udu = 0.f, du[DF / 32];
 #pragma unroll
     for (int u = 0; u < DF / 32; ++u) {
-        const float uu = f[u] * inf_;
+        const float uu = ph[u] * in;  // u = f / ||f|| = phi / ||phi||
         dn = fmaf(dphi[u], uu, dn);
         du[u] = n * dphi[u];
         udu = fmaf(uu, du[u], udu);
@@ -140,13 +174,13 @@ __device__ __forceinline__ float npmap_bwd_row(const float *y, float xx, const f
     float fdf = 0.f;
 #pragma unroll
     for (int u = 0; u < DF / 32; ++u) {
-        du[u] = (du[u] - f[u] * inf_ * udu) * inf_;  // df
-        fdf = fmaf(f[u], du[u], fdf);
+        du[u] = (du[u] - ph[u] * in * udu) * inf_;  // df
+        fdf = fmaf(ph[u] * isp, du[u], fdf);
     }
     fdf = warp_sum(fdf);
 #pragma unroll
-    for (int u = 0; u < DF / 32; ++u) dy_out[lane + 32 * u] = f[u] * (du[u] - fdf);  // dy = f (df - <f, df>)
-    return n > 0.f ? dn / n : 0.f;
+    for (int u = 0; u < DF / 32; ++u) dy[u] = ph[u] * isp * (du[u] - fdf);  // dy = f (df - <f, df>)
+    return dn * in;
 }
 
 // phi(x) of one row (one warp) from y = x W (shared, DF values) and ||x||^2: ||x|| e / ||e||,
@@ -187,11 +221,12 @@ struct LinTile {
     static constexpr int LDH = DH + 4, LDF = DF + 4;
     // pre:  XT/GT [DH][68], W/ST [DH][LDF], Y [64][LDF]
     static constexpr int PRE_FLOATS = DH * kLd64 + DH * LDF + 64 * LDF;
-    // post: XT [DH][68], W then W^T ([DH][LDF] / [DF][LDH]), Y then dY [64][LDF], dYT [DF][68], coef [64]
+    // post: q rows [64][LDH], Wq^T [DF][LDH] (then dO rows), dY^T [DF][68] (then A rows),
+    // dY [64][LDF], coef [64], D [64]
     static constexpr int WBUF = DH * LDF > DF * LDH ? DH * LDF : DF * LDH;
-    static constexpr int POST_FLOATS = DH * kLd64 + WBUF + 64 * LDF + DF * kLd64 + 64;
-    // key: KT [DH][68] (then VT), W / W^T / R^T / R, Y [64][LDF] (then dphi, dY), PT [DF][68]
-    // (phi(k)^T, then dY^T), coef [64], kept mask [64]
+    static constexpr int POST_FLOATS = 64 * LDH + WBUF + DF * kLd64 + 64 * LDF + 128;
+    // key: KT [DH][68] (K^T, V^T, K^T), Wk / R / R^T / Wk^T / K rows, Y [64][LDF] (Y_k, phi(k), dY),
+    // PT [DF][68] (phi(k)^T, dphi rows, dY^T), coef [64], kept mask [64]
     static constexpr int RBUF = WBUF;
     static constexpr int KEY_FLOATS = DH * kLd64 + RBUF + 64 * LDF + DF * kLd64 + 128;
 };
@@ -213,8 +248,8 @@ __global__ void __launch_bounds__(kTileThreads) bwd_lin_pre_tile(Dims s, const T
     const int valid = min(64, s.N - i0);
     const size_t row0 = (size_t)bh * s.N + i0;
     const size_t tslot = (size_t)bg * (s.T() + 1) + t;
-    load_rows_t(XT, kLd64, q + row0 * DH, DH, 64, DH, valid);
-    load_rows(W, Cfg::LDF, Wq + (size_t)h * DH * DF, DF, DH, DF, DH);
+    load_rows_t<64, DH>(XT, kLd64, q + row0 * DH, DH, valid);
+    load_rows<DH, DF>(W, Cfg::LDF, Wq + (size_t)h * DH * DF, DF, DH);
     __syncthreads();
     {
         float acc[1][DF / 64][4][4];
@@ -240,8 +275,8 @@ __global__ void __launch_bounds__(kTileThreads) bwd_lin_pre_tile(Dims s, const T
     }
     __syncthreads();
     // sg = dO S_t^T: dO^T over the q tile, S_t^T over Wq
-    load_rows_t(XT, kLd64, dO + row0 * DH, DH, 64, DH, valid);
-    load_rows_t(W, Cfg::LDF, S + tslot * DF * DH, DH, DF, DH, DF);  // W[x][a] = S[a][x]
+    load_rows_t<64, DH>(XT, kLd64, dO + row0 * DH, DH, valid);
+    load_rows_t<DF, DH>(W, Cfg::LDF, S + tslot * DF * DH, DH, DF);  // W[x][a] = S[a][x]
     __syncthreads();
     float acc[1][DF / 64][4][4];
     zero_acc(acc);
@@ -269,14 +304,17 @@ __global__ void __launch_bounds__(kTileThreads) bwd_lin_pre_tile(Dims s, const T
 
 template <typename T, int DH, int DF>
 __global__ void __launch_bounds__(kTileThreads) bwd_lin_post_tile(Dims s, const T *__restrict__ q,
-                                                                  const T *__restrict__ Wq, const float *__restrict__ z,
+                                                                  const T *__restrict__ Wq, const T *__restrict__ dO,
+                                                                  const float *__restrict__ z,
                                                                   const float *__restrict__ L,
                                                                   const float *__restrict__ Dv, float *__restrict__ PhiA,
                                                                   const float *__restrict__ SG, float *__restrict__ dq,
-                                                                  float *__restrict__ dWq) {
+                                                                  float *__restrict__ dWq, float *__restrict__ R,
+                                                                  float *__restrict__ rr) {
     using Cfg = LinTile<DH, DF>;
     extern __shared__ __align__(16) float sm[];
-    float *XT = sm, *W = XT + DH * kLd64, *Y = W + Cfg::WBUF, *dYT = Y + 64 * Cfg::LDF, *coef = dYT + DF * kLd64;
+    float *Xr = sm, *WT = Xr + 64 * Cfg::LDH, *dYT = WT + Cfg::WBUF, *dY = dYT + DF * kLd64, *coef = dY + 64 * Cfg::LDF,
+          *Ds = coef + 64;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int ntile = (s.N + 63) / 64;
     const int bh = blockIdx.x / ntile, i0 = (blockIdx.x % ntile) * 64;
@@ -284,37 +322,35 @@ __global__ void __launch_bounds__(kTileThreads) bwd_lin_post_tile(Dims s, const 
     const int t = i0 / s.C;
     const int valid = min(64, s.N - i0);
     const size_t row0 = (size_t)bh * s.N + i0;
+    const size_t tslot = (size_t)bg * (s.T() + 1) + t;
     const T *Wh = Wq + (size_t)h * DH * DF;
-    load_rows_t(XT, kLd64, q + row0 * DH, DH, 64, DH, valid);
-    load_rows(W, Cfg::LDF, Wh, DF, DH, DF, DH);
-    __syncthreads();
-    {
-        float acc[1][DF / 64][4][4];
-        zero_acc(acc);
-        smem_mm<1, DF / 64>(XT, kLd64, W, Cfg::LDF, DH, acc);  // Y = X Wq
-        store_tile(Y, Cfg::LDF, acc);
-    }
-    __syncthreads();
-    load_rows_t(W, Cfg::LDH, Wh, DF, DH, DF, DH);  // W^T [DF][DH] for dX = dY Wq^T
-    const float *zt = z + ((size_t)bg * (s.T() + 1) + t) * DF;
+    load_rows<64, DH>(Xr, Cfg::LDH, q + row0 * DH, DH, valid);
+    load_rows_t<DH, DF>(WT, Cfg::LDH, Wh, DF, DH);  // Wq^T [DF][DH]
+    // per row: c = 2^-L, dphi = c (sg - D z_t), a = c phi (global, read back below), NP-Map backward
+    // from phi itself (f = phi / sum(phi), ||q|| = ||phi||)
+    const float *zt = z + tslot * DF;
     for (int r = warp; r < 64; r += 8) {
-        float dphi[DF / 32];
         const size_t row = row0 + r;
         const bool live = r < valid;
         const float c = live ? exp2f(-L[row]) : 0.f, Di = live ? Dv[row] : 0.f;
+        float ph[DF / 32], dphi[DF / 32], dy[DF / 32];
 #pragma unroll
         for (int u = 0; u < DF / 32; ++u) {
             const int a = lane + 32 * u;
+            ph[u] = live ? PhiA[row * DF + a] : 0.f;
             dphi[u] = live ? c * (SG[row * DF + a] - Di * zt[a]) : 0.f;
-            if (live) PhiA[row * DF + a] *= c;
+            if (live) PhiA[row * DF + a] = c * ph[u];
         }
-        // dy over y (row r of Y), then into dYT[c][r]
-        float *yr = Y + r * Cfg::LDF;
-        const float cf = npmap_bwd_row<DF>(yr, col_sqnorm<DH>(XT, kLd64, r, lane), dphi, yr, lane);
-        __syncwarp();
+        const float cf = npmap_bwd_from_phi<DF>(ph, dphi, dy);
 #pragma unroll
-        for (int u = 0; u < DF / 32; ++u) dYT[(lane + 32 * u) * kLd64 + r] = yr[lane + 32 * u];
-        if (lane == 0) coef[r] = cf;
+        for (int u = 0; u < DF / 32; ++u) {
+            dY[r * Cfg::LDF + lane + 32 * u] = dy[u];
+            dYT[(lane + 32 * u) * kLd64 + r] = dy[u];
+        }
+        if (lane == 0) {
+            coef[r] = cf;
+            Ds[r] = Di;
+        }
     }
     __syncthreads();
     const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
@@ -322,7 +358,7 @@ __global__ void __launch_bounds__(kTileThreads) bwd_lin_post_tile(Dims s, const 
         // dq += dY Wq^T + coef q
         float acc[1][DH / 64][4][4];
         zero_acc(acc);
-        smem_mm<1, DH / 64>(dYT, kLd64, W, Cfg::LDH, DF, acc);
+        smem_mm<1, DH / 64>(dYT, kLd64, WT, Cfg::LDH, DF, acc);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int r = ty * 4 + i;
@@ -330,25 +366,22 @@ __global__ void __launch_bounds__(kTileThreads) bwd_lin_post_tile(Dims s, const 
 #pragma unroll
             for (int nu = 0; nu < DH / 64; ++nu) {
                 const int x = tx * 4 + 64 * nu;
+                const float4 xq = *reinterpret_cast<const float4 *>(Xr + r * Cfg::LDH + x);
                 float4 *dst = reinterpret_cast<float4 *>(dq + (row0 + r) * DH + x);
                 float4 v = *dst;
-                v.x += acc[0][nu][i][0] + coef[r] * XT[(x + 0) * kLd64 + r];
-                v.y += acc[0][nu][i][1] + coef[r] * XT[(x + 1) * kLd64 + r];
-                v.z += acc[0][nu][i][2] + coef[r] * XT[(x + 2) * kLd64 + r];
-                v.w += acc[0][nu][i][3] + coef[r] * XT[(x + 3) * kLd64 + r];
+                v.x += acc[0][nu][i][0] + coef[r] * xq.x;
+                v.y += acc[0][nu][i][1] + coef[r] * xq.y;
+                v.z += acc[0][nu][i][2] + coef[r] * xq.z;
+                v.w += acc[0][nu][i][3] + coef[r] * xq.w;
                 *dst = v;
             }
         }
     }
-    __syncthreads();
     {
-        // dWq += X^T dY: AT[k = row][x] = q rows (re-read into W's buffer), B = dY [row][c] (in Y)
-        float *Xr = W;
-        load_rows(Xr, Cfg::LDH, q + row0 * DH, DH, 64, DH, valid);
-        __syncthreads();
+        // dWq += X^T dY (the q rows, the dY rows)
         float acc[DH / 64][DF / 64][4][4];
         zero_acc(acc);
-        smem_mm<DH / 64, DF / 64>(Xr, Cfg::LDH, Y, Cfg::LDF, 64, acc);
+        smem_mm<DH / 64, DF / 64>(Xr, Cfg::LDH, dY, Cfg::LDF, 64, acc);
         float *dW = dWq + (size_t)h * DH * DF;
 #pragma unroll
         for (int mu = 0; mu < DH / 64; ++mu)
@@ -359,56 +392,40 @@ __global__ void __launch_bounds__(kTileThreads) bwd_lin_post_tile(Dims s, const 
                     atomicAdd(reinterpret_cast<float4 *>(dW + (size_t)(ty * 4 + 64 * mu + i) * DF + tx * 4 + 64 * nu),
                               make_float4(acc[mu][nu][i][0], acc[mu][nu][i][1], acc[mu][nu][i][2], acc[mu][nu][i][3]));
     }
-}
-
-// R_t (D x d) and r_t (D) of query chunk t for (b, g): sum over the chunk's rows of all G heads.
-template <typename T, int DH, int DF>
-__global__ void __launch_bounds__(kTileThreads) bwd_chunk_tile(Dims s, const float *__restrict__ A,
-                                                               const float *__restrict__ Dv, const T *__restrict__ dO,
-                                                               float *__restrict__ R, float *__restrict__ rr) {
-    extern __shared__ __align__(16) float sm[];
-    // R_t[a][x] = sum_i A[i][a] dO[i][x]: the reduction runs over the rows, so both tiles stay row-major
-    float *Ar = sm, *Gt = Ar + 64 * (DF + 4), *Ds = Gt + 64 * (DH + 4);
-    const int T_ = s.T(), G = s.G();
-    const int bg = blockIdx.x / (T_ + 1), t = blockIdx.x % (T_ + 1);
-    const int b = bg / s.Hkv, g = bg % s.Hkv;
-    const int i_lo = t * s.C, i_hi = min(s.N, i_lo + s.C);
-    float acc[DF / 64][DH / 64][4][4];
-    zero_acc(acc);
-    float racc = 0.f;
-    for (int hh = 0; hh < G; ++hh) {
-        const size_t rb = ((size_t)b * s.H + g * G + hh) * s.N;
-        for (int i0 = i_lo; i0 < i_hi; i0 += 64) {
-            const int valid = min(64, i_hi - i0);
-            __syncthreads();
-            load_rows(Ar, DF + 4, A + (rb + i0) * DF, DF, 64, DF, valid);
-            load_rows(Gt, DH + 4, dO + (rb + i0) * DH, DH, 64, DH, valid);
-            if (threadIdx.x < 64) Ds[threadIdx.x] = (int)threadIdx.x < valid ? Dv[rb + i0 + threadIdx.x] : 0.f;
-            __syncthreads();
-            smem_mm<DF / 64, DH / 64>(Ar, DF + 4, Gt, DH + 4, 64, acc);
-            if (threadIdx.x < DF)
-                for (int r = 0; r < 64; ++r) racc = fmaf(Ar[r * (DF + 4) + threadIdx.x], Ds[r], racc);
+    __syncthreads();
+    {
+        // the chunk sums of the key side: R_t += A^T dO, r_t += A^T D over the tile's rows (a = c phi
+        // rows over dYT's buffer, dO rows over Wq^T's)
+        float *Ar = dYT, *Go = WT;
+        static_assert(64 * (DF + 4) <= DF * kLd64, "A rows fit the dY^T buffer");
+        load_rows<64, DF>(Ar, Cfg::LDF, PhiA + row0 * DF, DF, valid);
+        load_rows<64, DH>(Go, Cfg::LDH, dO + row0 * DH, DH, valid);
+        __syncthreads();
+        float acc[DF / 64][DH / 64][4][4];
+        zero_acc(acc);
+        smem_mm<DF / 64, DH / 64>(Ar, Cfg::LDF, Go, Cfg::LDH, 64, acc);
+        float *Rt = R + tslot * DF * DH;
+#pragma unroll
+        for (int mu = 0; mu < DF / 64; ++mu)
+#pragma unroll
+            for (int nu = 0; nu < DH / 64; ++nu)
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    atomicAdd(reinterpret_cast<float4 *>(Rt + (size_t)(ty * 4 + 64 * mu + i) * DH + tx * 4 + 64 * nu),
+                              make_float4(acc[mu][nu][i][0], acc[mu][nu][i][1], acc[mu][nu][i][2], acc[mu][nu][i][3]));
+        if (threadIdx.x < DF) {
+            float racc = 0.f;
+            for (int r = 0; r < 64; ++r) racc = fmaf(Ar[r * Cfg::LDF + threadIdx.x], Ds[r], racc);
+            atomicAdd(rr + tslot * DF + threadIdx.x, racc);
         }
     }
-    const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
-    const size_t slot = (size_t)bg * (T_ + 1) + t;
-#pragma unroll
-    for (int mu = 0; mu < DF / 64; ++mu)
-#pragma unroll
-        for (int nu = 0; nu < DH / 64; ++nu)
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                *reinterpret_cast<float4 *>(R + (slot * DF + ty * 4 + 64 * mu + i) * DH + tx * 4 + 64 * nu) =
-                    make_float4(acc[mu][nu][i][0], acc[mu][nu][i][1], acc[mu][nu][i][2], acc[mu][nu][i][3]);
-    if (threadIdx.x < DF) rr[slot * DF + threadIdx.x] = racc;
 }
 
-// Unselected keys of 64-key tiles of decided chunks: dphi(k) = R v - r, dv += R^T phi(k),
-// NP-Map backward of k: dk += dy Wk^T + coef k, dWk += k^T dy.
+// Unselected keys of 64-key tiles of decided chunks: phi(k) from K Wk, dv += phi(k) R,
+// dphi(k) = V R^T - r, the NP-Map backward from phi(k): dk += dy Wk^T + coef k, dWk += k^T dy.
 template <typename T, int DH, int DF>
 __global__ void __launch_bounds__(kTileThreads) bwd_key_tile(Dims s, const T *__restrict__ k, const T *__restrict__ v,
                                                              const T *__restrict__ Wk, const int32_t *__restrict__ idx,
-                                                             const float *__restrict__ phik,
                                                              const float *__restrict__ R, const float *__restrict__ rr,
                                                              float *__restrict__ dk, float *__restrict__ dv,
                                                              float *__restrict__ dWk) {
@@ -435,20 +452,29 @@ __global__ void __launch_bounds__(kTileThreads) bwd_key_tile(Dims s, const T *__
             const int j = idx[((size_t)bg * T_ + c) * s.k + n] - j0;
             if (j >= 0 && j < 64) keep[j] = 1;
         }
-    // dphi = V R^T - r: V^T over KT, R^T [x][a] over Wb
-    load_rows_t(KT, kLd64, v + row0 * DH, DH, 64, DH, 64);
-    load_rows_t(Wb, Cfg::LDF, Rs, DH, DF, DH, DF);
+    // Y_k = K Wk, then phi(k) per row (row-major over Y, transposed into PT)
+    load_rows_t<64, DH>(KT, kLd64, k + row0 * DH, DH, 64);
+    load_rows<DH, DF>(Wb, Cfg::LDF, Wg, DF, DH);
     __syncthreads();
     {
         float acc[1][DF / 64][4][4];
         zero_acc(acc);
         smem_mm<1, DF / 64>(KT, kLd64, Wb, Cfg::LDF, DH, acc);
-        store_tile(Y, Cfg::LDF, acc);  // Y <- V R^T (r subtracted below)
+        store_tile(Y, Cfg::LDF, acc);
     }
     __syncthreads();
-    // dv += phi(k) R: phi(k)^T over PT, R [a][x] over Wb
-    load_rows_t(PT, kLd64, phik + row0 * DF, DF, 64, DF, 64);
-    load_rows(Wb, Cfg::LDH, Rs, DH, DF, DH, DF);
+    for (int r = warp; r < 64; r += 8) {
+        float ph[DF / 32];
+        npmap_fwd_row<DF>(Y + r * Cfg::LDF, col_sqnorm<DH>(KT, kLd64, r, lane), ph, lane);
+        __syncwarp();
+#pragma unroll
+        for (int u = 0; u < DF / 32; ++u) {
+            Y[r * Cfg::LDF + lane + 32 * u] = ph[u];
+            PT[(lane + 32 * u) * kLd64 + r] = ph[u];
+        }
+    }
+    // dv += phi(k) R (R [a][x] over Wb)
+    load_rows<DF, DH>(Wb, Cfg::LDH, Rs, DH, DF);
     __syncthreads();
     const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
     {
@@ -472,37 +498,39 @@ __global__ void __launch_bounds__(kTileThreads) bwd_key_tile(Dims s, const T *__
         }
     }
     __syncthreads();
-    // Y_k = K Wk (into PT's buffer, row-major [64][LDF]; PT is free) with K^T over KT, Wk over Wb
-    float *Yk = PT;
-    static_assert(64 * (DF + 4) <= DF * kLd64, "Yk fits PT");
-    load_rows_t(KT, kLd64, k + row0 * DH, DH, 64, DH, 64);
-    load_rows(Wb, Cfg::LDF, Wg, DF, DH, DF, DH);
+    // dphi = V R^T (row-major over PT; r subtracted per row below): V^T over KT, R^T [x][a] over Wb
+    float *dP = PT;
+    static_assert(64 * (DF + 4) <= DF * kLd64, "dphi rows fit PT");
+    load_rows_t<64, DH>(KT, kLd64, v + row0 * DH, DH, 64);
+    load_rows_t<DF, DH>(Wb, Cfg::LDF, Rs, DH, DF);
     __syncthreads();
     {
         float acc[1][DF / 64][4][4];
         zero_acc(acc);
         smem_mm<1, DF / 64>(KT, kLd64, Wb, Cfg::LDF, DH, acc);
-        store_tile(Yk, Cfg::LDF, acc);
+        store_tile(dP, Cfg::LDF, acc);
     }
     __syncthreads();
-    // per key row: dy of the NP-Map (over Y's row: dphi there is consumed first), coef
+    // per key row: the NP-Map backward from phi(k) (row of Y), dy over the same row of Y
     for (int r = warp; r < 64; r += 8) {
-        float dphi[DF / 32];
+        float ph[DF / 32], dphi[DF / 32], dy[DF / 32];
         const bool on = !keep[r];
 #pragma unroll
         for (int u = 0; u < DF / 32; ++u) {
             const int a = lane + 32 * u;
-            dphi[u] = on ? Y[r * Cfg::LDF + a] - rs[a] : 0.f;
+            ph[u] = Y[r * Cfg::LDF + a];
+            dphi[u] = on ? dP[r * Cfg::LDF + a] - rs[a] : 0.f;
         }
-        __syncwarp();
-        const float cf = npmap_bwd_row<DF>(Yk + r * Cfg::LDF, col_sqnorm<DH>(KT, kLd64, r, lane), dphi,
-                                           Y + r * Cfg::LDF, lane);
+        const float cf = npmap_bwd_from_phi<DF>(ph, dphi, dy);
+#pragma unroll
+        for (int u = 0; u < DF / 32; ++u) Y[r * Cfg::LDF + lane + 32 * u] = dy[u];
         if (lane == 0) coef[r] = on ? cf : 0.f;
     }
     __syncthreads();
-    // dk += dY Wk^T + coef k: dY^T over PT (Yk no longer needed), Wk^T over Wb
-    load_rows_t(PT, kLd64, Y, Cfg::LDF, 64, DF, 64);
-    load_rows_t(Wb, Cfg::LDH, Wg, DF, DH, DF, DH);
+    // dk += dY Wk^T + coef k: dY^T over PT, Wk^T over Wb, K^T (for coef k) back over KT
+    load_rows_t<64, DF>(PT, kLd64, Y, Cfg::LDF, 64);
+    load_rows_t<DH, DF>(Wb, Cfg::LDH, Wg, DF, DH);
+    load_rows_t<64, DH>(KT, kLd64, k + row0 * DH, DH, 64);
     __syncthreads();
     {
         float acc[1][DH / 64][4][4];
@@ -528,7 +556,7 @@ __global__ void __launch_bounds__(kTileThreads) bwd_key_tile(Dims s, const T *__
     __syncthreads();
     {
         // dWk += K^T dY: K rows over Wb, dY [row][a] in Y (kept rows are zero there: dphi = 0)
-        load_rows(Wb, Cfg::LDH, k + row0 * DH, DH, 64, DH, 64);
+        load_rows<64, DH>(Wb, Cfg::LDH, k + row0 * DH, DH, 64);
         __syncthreads();
         float acc[DH / 64][DF / 64][4][4];
         zero_acc(acc);
@@ -562,25 +590,22 @@ cudaError_t launch_lin_cfg(int which, const Dims &s, const void *q, const void *
             s, (const T *)q, (const T *)Wq, w.S, w.z, (const T *)dO, w.A, w.dYq, w.Ms, w.iZ);
         return cudaGetLastError();
     }
-    // which == 1: query side after the softmax pass, the chunk sums, their suffix, the key side
+    // which == 1: query side after the softmax pass (with the chunk sums), their suffix, the key side
+    const int T_ = s.T();
+    const size_t BK = (size_t)s.B * s.Hkv;
     if ((e = cudaMemsetAsync(dWq, 0, sizeof(float) * (size_t)s.H * DH * DF, st)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(dWk, 0, sizeof(float) * (size_t)s.Hkv * DH * DF, st)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(w.R, 0, sizeof(float) * BK * (T_ + 1) * DF * DH, st)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(w.r, 0, sizeof(float) * BK * (T_ + 1) * DF, st)) != cudaSuccess) return e;
     if ((e = prep((const void *)bwd_lin_post_tile<T, DH, DF>, Cfg::POST_FLOATS)) != cudaSuccess) return e;
     bwd_lin_post_tile<T, DH, DF><<<qgrid, kTileThreads, Cfg::POST_FLOATS * 4, st>>>(
-        s, (const T *)q, (const T *)Wq, w.z, w.L, w.Dv, w.A, w.dYq, dq, dWq);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    const int T_ = s.T();
-    const int chunk_floats = 64 * (DF + 4) + 64 * (DH + 4) + 64;
-    if ((e = prep((const void *)bwd_chunk_tile<T, DH, DF>, chunk_floats)) != cudaSuccess) return e;
-    bwd_chunk_tile<T, DH, DF><<<(unsigned)((size_t)s.B * s.Hkv * (T_ + 1)), kTileThreads, chunk_floats * 4, st>>>(
-        s, w.A, w.Dv, (const T *)dO, w.R, w.r);
+        s, (const T *)q, (const T *)Wq, (const T *)dO, w.z, w.L, w.Dv, w.A, w.dYq, dq, dWq, w.R, w.r);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = launch_bwd_suffix(s, w.R, w.r, st)) != cudaSuccess) return e;
     if (T_ > 0) {
         if ((e = prep((const void *)bwd_key_tile<T, DH, DF>, Cfg::KEY_FLOATS)) != cudaSuccess) return e;
-        bwd_key_tile<T, DH, DF><<<(unsigned)((size_t)s.B * s.Hkv * (T_ * s.C / 64)), kTileThreads,
-                                  Cfg::KEY_FLOATS * 4, st>>>(s, (const T *)k, (const T *)v, (const T *)Wk, idx, w.phik,
-                                                             w.R, w.r, dk, dv, dWk);
+        bwd_key_tile<T, DH, DF><<<(unsigned)(BK * (T_ * s.C / 64)), kTileThreads, Cfg::KEY_FLOATS * 4, st>>>(
+            s, (const T *)k, (const T *)v, (const T *)Wk, idx, w.R, w.r, dk, dv, dWk);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     return cudaSuccess;

@@ -596,13 +596,22 @@ cudaError_t backward_t(const Dims &s, const void *q, const void *k, const void *
     const T *GO = (const T *)dO;
     const int T_ = s.T();
     cudaError_t e;
-    // linear state of the forward (S_t, z_t per query chunk)
-    e = launch_npmap(s.B * s.Hkv * s.N, s.Hkv, s.N, s.d, s.D, s.bf16, k, Wk, w.phik, st);
-    if (e != cudaSuccess) return e;
-    ++*launches;
-    e = launch_linear_state(s, w.phik, v, idx, w.S, w.z, nullptr, err, st);
-    if (e != cudaSuccess) return e;
-    *launches += 2;
+    // linear state of the forward (S_t, z_t per query chunk): on tensor cores where the tiled linear
+    // backward runs (it forms phi(k) itself), else from phi(k) of every key
+    const bool tiled_state = tc_backward_supported(s) && tiled_linear_backward_supported(s) && tc_linear_supported(s);
+    if (tiled_state) {
+        if ((e = launch_w_transpose(s.Hkv, s.d, s.D, Wk, w.wkt, st)) != cudaSuccess) return e;
+        if ((e = launch_linear_tc(s, k, v, w.wkt, idx, w.S, w.z, err, st)) != cudaSuccess) return e;
+        if ((e = launch_linear_prefix(s, w.S, w.z, nullptr, st)) != cudaSuccess) return e;
+        *launches += 3;
+    } else {
+        e = launch_npmap(s.B * s.Hkv * s.N, s.Hkv, s.N, s.d, s.D, s.bf16, k, Wk, w.phik, st);
+        if (e != cudaSuccess) return e;
+        ++*launches;
+        e = launch_linear_state(s, w.phik, v, idx, w.S, w.z, nullptr, err, st);
+        if (e != cudaSuccess) return e;
+        *launches += 2;
+    }
     if ((e = cudaMemsetAsync(w.dYk, 0, sizeof(float) * (size_t)s.B * s.Hkv * s.N * s.D, st)) != cudaSuccess) return e;
     const long long rows = (long long)s.B * s.H * s.N;
     const unsigned rgrid = (unsigned)((rows + kBwdWarps - 1) / kBwdWarps);
@@ -628,7 +637,7 @@ cudaError_t backward_t(const Dims &s, const void *q, const void *k, const void *
             // query side (dq, dWq), chunk sums, suffix, key side (dk, dv, dWk) of the linear branch
             e = launch_linear_backward_tiled(1, s, q, k, v, Wq, Wk, dO, idx, w, dq, dk, dv, dWq, dWk, st);
             if (e != cudaSuccess) return e;
-            *launches += T_ > 0 ? 4 : 3;
+            *launches += T_ > 0 ? 3 : 2;
             return cudaSuccess;
         }
         bwd_lin_post_kernel<T><<<rgrid, 32 * kBwdWarps, 0, st>>>(s, Q, WQ, w.z, w.L, w.Dv, w.A, w.dYq, dq);

@@ -75,7 +75,12 @@ struct BackwardScratch {
     float *dYk;    // [B,Hkv,N,D]   dL/d(k Wk)
     float *L;      // [B,H,N]       tensor-core path: each row's log2 normaliser Ms log2(e) + log2 Z
     void *khat, *vhat;  // [B,Hkv,T*k,d] tensor-core path: the kept rows, gathered (bf16)
+    void *wkt;     // [Hkv,D,d] tensor-core path: Wk^T (bf16), operand of the linear-state kernel
 };
+bool tc_linear_supported(const Dims &s);
+cudaError_t launch_w_transpose(int Hx, int d, int D, const void *w, void *wt, cudaStream_t st);
+cudaError_t launch_linear_tc(const Dims &s, const void *k, const void *v, const void *wkt, const int32_t *idx,
+                             float *S, float *z, unsigned *err, cudaStream_t st);
 bool tc_backward_supported(const Dims &s);
 bool tiled_linear_backward_supported(const Dims &s);
 cudaError_t launch_linear_backward_tiled(int which, const Dims &s, const void *q, const void *k, const void *v,
