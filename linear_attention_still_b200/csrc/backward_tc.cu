@@ -23,8 +23,8 @@
 // dV += P^T dO and dK += dS^T Q with P^T / dS^T as TMEM operands; the accumulators stay in TMEM for
 // the whole CTA.  Window keys write dk, dv; kept keys add into the rows their entries name.
 //
-// Roles in both kernels: four row warps (TMEM lanes), one TMA producer warp, one MMA warp (which
-// also allocates TMEM).  Every mbarrier wait is bounded; on a timeout the CTA records
+// Roles in both kernels: two warpgroups of row warps (TMEM lane = row; each warpgroup takes half of a
+// tile's 64 columns), one TMA producer warp, one MMA warp (which also allocates TMEM).  Every mbarrier wait is bounded; on a timeout the CTA records
 // DEV_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
 
@@ -63,15 +63,19 @@ struct BwdQCfg {
     static constexpr int STAGE_BYTES = 2 * K_BYTES;
     static constexpr int OFF_Q = 0, OFF_DO = Q_BYTES, OFF_STAGE = 2 * Q_BYTES,
                          OFF_BAR = OFF_STAGE + NS * STAGE_BYTES;
-    static constexpr int B_QFULL = 0, B_S = 1, B_SDONE = 2, B_DQ = 3, B_DRAIN = 4, B_KFULL = 5,
-                         B_VFULL = 5 + NS, B_KVEMPTY = 5 + 2 * NS, NUM_BARS = 5 + 3 * NS;
+    // B_SDONE: the row warps hold S, dP of a tile in registers; B_DSFULL + (n & 1): they wrote the dS
+    // of sweep-2 tile n (two barriers taking turns, so neither runs two phases ahead of its waiter)
+    static constexpr int B_QFULL = 0, B_S = 1, B_SDONE = 2, B_DQ = 3, B_DRAIN = 4, B_WG = 5, B_DSFULL = 6,
+                         B_KFULL = 8, B_VFULL = 8 + NS, B_KVEMPTY = 8 + 2 * NS, NUM_BARS = 8 + 3 * NS;
     static constexpr int TMEM_SLOT_OFF = 8 * NUM_BARS, ABORT_OFF = TMEM_SLOT_OFF + 8, BAR_BYTES = 256;
     static_assert(ABORT_OFF + 8 <= BAR_BYTES, "barrier area overflow");
-    static constexpr int SMEM = OFF_BAR + BAR_BYTES + 1024;
-    static constexpr int THREADS = 192, PRODUCER_WARP = 4, MMA_WARP = 5;
-    // S (64 keys), dP (64 keys; dS in bf16 over its first 32 columns), dQ (DH)
-    static constexpr int S_COL = 0, DP_COL = 64, DQ_COL = 128, TMEM_COLS = 256;
-    static_assert(DQ_COL + DH <= TMEM_COLS, "TMEM budget");
+    static constexpr int OFF_XCH = OFF_BAR + BAR_BYTES;   // [2][128][3] row statistics of each half
+    static constexpr int SMEM = OFF_XCH + 2 * 128 * 3 * 4 + 1024;
+    // Two warpgroups of row warps: warpgroup x takes key columns [32x, 32x + 32) of every tile.
+    static constexpr int THREADS = 320, PRODUCER_WARP = 8, MMA_WARP = 9, ROW_THREADS = 256;
+    // S (64 keys), dP (64 keys), dQ (DH), dS of alternate tiles (bf16, 64 keys = 32 columns each)
+    static constexpr int S_COL = 0, DP_COL = 64, DQ_COL = 128, DS_COL = 128 + DH, TMEM_COLS = DH == 64 ? 256 : 512;
+    static_assert(DS_COL + 64 <= TMEM_COLS, "TMEM budget");
     static constexpr int MIN_BLOCKS = DH == 64 ? 2 : 1;  // two CTAs per SM overlap each other's phases
     static_assert(MIN_BLOCKS * (SMEM + 1024) <= 233472, "shared memory per SM");
 };
@@ -108,7 +112,10 @@ __global__ void __launch_bounds__(BwdQCfg<DH>::THREADS, BwdQCfg<DH>::MIN_BLOCKS)
     const int ntot = 2 * nt;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < Cfg::NUM_BARS; ++i) mbar_init(BAR(i), i == Cfg::B_SDONE ? 128 : 1);
+        for (int i = 0; i < Cfg::NUM_BARS; ++i)
+            mbar_init(BAR(i), i == Cfg::B_SDONE || i == Cfg::B_WG || i == Cfg::B_DSFULL || i == Cfg::B_DSFULL + 1
+                                  ? Cfg::ROW_THREADS
+                                  : 1);
         *abort_flag = 0;
         mbar_fence_init();
     }
@@ -163,13 +170,15 @@ __global__ void __launch_bounds__(BwdQCfg<DH>::THREADS, BwdQCfg<DH>::MIN_BLOCKS)
         constexpr uint32_t ID_S = idesc_bf16(128, 64, 0, 0);
         constexpr uint32_t ID_DQ = idesc_bf16(128, DH, 0, 1);
         const uint32_t sQ = sbase + Cfg::OFF_Q, sDO = sbase + Cfg::OFF_DO;
-        // dQ += dS K for tile jj (sweep 2): dS (bf16, 64 keys = 32 columns) from TMEM, K as the
-        // MN-major B operand (N = DH, K = 64 keys; 16 keys = 16 rows of 128 bytes per k-step)
+        // dQ += dS K for tile jj (sweep 2): dS (bf16, 64 keys = 32 columns, buffer jj & 1) from TMEM, K
+        // as the MN-major B operand (N = DH, K = 64 keys; 16 keys = 16 rows of 128 bytes per k-step).
+        // The row warps reuse a dS buffer only after B_S of the tile two later, whose commit covers
+        // this MMA.
         auto issue_dq = [&](int jj) {
             const uint64_t dk = sw128_desc(sbase + Cfg::OFF_STAGE + (jj % Cfg::NS) * Cfg::STAGE_BYTES, Cfg::K_REG, 1024);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                mma_ts_w(tm + Cfg::DQ_COL, tm + Cfg::DP_COL + kk * 8, dk + (uint64_t)(kk * 128), ID_DQ,
+                mma_ts_w(tm + Cfg::DQ_COL, tm + Cfg::DS_COL + 32 * (jj & 1) + kk * 8, dk + (uint64_t)(kk * 128), ID_DQ,
                          (jj > nt || kk > 0) ? 1u : 0u);
             mma_commit_w(BAR(Cfg::B_KVEMPTY + jj % Cfg::NS));
         };
@@ -179,12 +188,8 @@ __global__ void __launch_bounds__(BwdQCfg<DH>::THREADS, BwdQCfg<DH>::MIN_BLOCKS)
             const uint32_t sK = sbase + Cfg::OFF_STAGE + s * Cfg::STAGE_BYTES, sV = sK + Cfg::K_BYTES;
             if (!(ok = mbar_wait_w(BAR(Cfg::B_KFULL + s), (jj / Cfg::NS) & 1, abort_flag))) break;
             if (!(ok = mbar_wait_w(BAR(Cfg::B_VFULL + s), (jj / Cfg::NS) & 1, abort_flag))) break;
-            if (jj > 0) {
-                // the row warps have read S, dP of tile jj-1 (and written its dS in sweep 2)
-                if (!(ok = mbar_wait_w(BAR(Cfg::B_SDONE), (jj - 1) & 1, abort_flag))) break;
-                tc_fence_after();
-                if (jj - 1 >= nt) issue_dq(jj - 1);  // in issue order before S, dP(jj) overwrite dS
-            }
+            // the row warps hold S, dP of tile jj-1 in registers: the columns are free
+            if (jj > 0 && !(ok = mbar_wait_w(BAR(Cfg::B_SDONE), (jj - 1) & 1, abort_flag))) break;
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < DH / 16; ++kk)
@@ -194,8 +199,15 @@ __global__ void __launch_bounds__(BwdQCfg<DH>::THREADS, BwdQCfg<DH>::MIN_BLOCKS)
                 mma_ss_w(tm + Cfg::DP_COL, kmajor_desc(sDO, kk, Cfg::Q_REG), kmajor_desc(sV, kk, Cfg::K_REG), ID_S, kk > 0);
             mma_commit_w(BAR(Cfg::B_S));
             if (jj < nt) mma_commit_w(BAR(Cfg::B_KVEMPTY + s));  // sweep 1: the stage is done with
+            if (jj - 1 >= nt) {
+                // dS of tile jj-1 written: dQ += dS K (overlaps the row warps' work on tile jj)
+                const int n = jj - 1 - nt;
+                if (!(ok = mbar_wait_w(BAR(Cfg::B_DSFULL + (n & 1)), (n >> 1) & 1, abort_flag))) break;
+                tc_fence_after();
+                issue_dq(jj - 1);
+            }
         }
-        if (ok && (ok = mbar_wait_w(BAR(Cfg::B_SDONE), (ntot - 1) & 1, abort_flag))) {
+        if (ok && (ok = mbar_wait_w(BAR(Cfg::B_DSFULL + ((nt - 1) & 1)), ((nt - 1) >> 1) & 1, abort_flag))) {
             tc_fence_after();
             issue_dq(ntot - 1);
             mma_commit_w(BAR(Cfg::B_DQ));
@@ -208,13 +220,16 @@ __global__ void __launch_bounds__(BwdQCfg<DH>::THREADS, BwdQCfg<DH>::MIN_BLOCKS)
         mbar_wait_drain(BAR(Cfg::B_DRAIN), 0, 100000000ull);
     } else {
         // ================================================================ row warps (TMEM lane = query row)
-        const int r = warp * 32 + lane;
+        // warpgroup x takes key columns [32x, 32x + 32) of each tile; the two halves of a row combine
+        // their running statistics once, after sweep 1
+        const int x = warp >> 2, quarter = warp & 3;
+        const int r = quarter * 32 + lane;
         const int i = i0 + r;
         const bool live = i < p.N;
         const size_t row = (size_t)bh * p.N + i;
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-        const uint32_t tS = tmem + lane_off + Cfg::S_COL, tDP = tmem + lane_off + Cfg::DP_COL,
-                       tDQ = tmem + lane_off + Cfg::DQ_COL;
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        const uint32_t tS = tmem + lane_off + Cfg::S_COL + 32 * x, tDP = tmem + lane_off + Cfg::DP_COL + 32 * x,
+                       tDS = tmem + lane_off + Cfg::DS_COL + 16 * x;
         const float lden = live ? p.lden[row] : 0.f, dl = live ? p.dl[row] : 0.f;
         const float sl2 = p.scale_log2;
         float M = -INFINITY, l = 0.f, u = 0.f, Lr = 0.f, Di = 0.f;
@@ -224,33 +239,33 @@ __global__ void __launch_bounds__(BwdQCfg<DH>::THREADS, BwdQCfg<DH>::MIN_BLOCKS)
             tc_fence_after();
             const int j = jj < nt ? jj : jj - nt;
             // columns c < lim are in Soft(i): kept entries below nk, window keys at or before i
-            const int lim = j < nkt ? nk - 64 * j : i - (lo + 64 * (j - nkt)) + 1;
+            const int lim = (j < nkt ? nk - 64 * j : i - (lo + 64 * (j - nkt)) + 1) - 32 * x;
             if (jj < nt) {
-                // ---- sweep 1: running max, sum and sum of exp * <dO, v>
-                float sv[64];
-#pragma unroll
-                for (int c = 0; c < 2; ++c) {
+                // ---- sweep 1: running max, sum and sum of exp * <dO, v> over this half's columns
+                float sv[32];
+                {
                     uint32_t w[32];
-                    tmem_ld32(tS + c * 32, w);
+                    tmem_ld32(tS, w);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) sv[c * 32 + e] = c * 32 + e < lim ? __uint_as_float(w[e]) * sl2 : -INFINITY;
+                    for (int e = 0; e < 32; ++e) sv[e] = e < lim ? __uint_as_float(w[e]) * sl2 : -INFINITY;
                 }
                 float mt = -INFINITY;
 #pragma unroll
-                for (int c = 0; c < 64; ++c) mt = fmaxf(mt, sv[c]);
+                for (int e = 0; e < 32; ++e) mt = fmaxf(mt, sv[e]);
                 const float mn = fmaxf(M, mt);
                 const float mref = mn == -INFINITY ? 0.f : mn;
                 const float sc = M == -INFINITY ? 0.f : ex2(M - mref);
                 float la = 0.f, lb = 0.f, ua = 0.f, ub = 0.f;
-#pragma unroll
-                for (int c = 0; c < 2; ++c) {
+                {
                     uint32_t w[32];
-                    tmem_ld32(tDP + c * 32, w);
+                    tmem_ld32(tDP, w);
                     tmem_wait_ld();
+                    tc_fence_before();
+                    mbar_arrive(BAR(Cfg::B_SDONE));  // S and dP of this tile are in registers
 #pragma unroll
                     for (int e = 0; e < 32; e += 2) {
-                        const float p0 = ex2(sv[c * 32 + e] - mref), p1 = ex2(sv[c * 32 + e + 1] - mref);
+                        const float p0 = ex2(sv[e] - mref), p1 = ex2(sv[e + 1] - mref);
                         la += p0;
                         lb += p1;
                         ua = fmaf(p0, __uint_as_float(w[e]), ua);
@@ -260,57 +275,66 @@ __global__ void __launch_bounds__(BwdQCfg<DH>::THREADS, BwdQCfg<DH>::MIN_BLOCKS)
                 l = fmaf(l, sc, la + lb);
                 u = fmaf(u, sc, ua + ub);
                 M = mn;
-                tc_fence_before();
-                mbar_arrive(BAR(Cfg::B_SDONE));
                 if (jj == nt - 1) {
-                    // ---- the row's normaliser with the linear branch, and D_i
+                    // ---- combine the two halves, then the row's normaliser with the linear branch and D_i
+                    float *xch = reinterpret_cast<float *>(smem + Cfg::OFF_XCH);
+                    xch[(x * 128 + r) * 3 + 0] = M;
+                    xch[(x * 128 + r) * 3 + 1] = l;
+                    xch[(x * 128 + r) * 3 + 2] = u;
+                    mbar_arrive(BAR(Cfg::B_WG));
+                    if (!(ok = warp_all(mbar_wait(BAR(Cfg::B_WG), 0, abort_flag)))) break;
+                    const float Mo = xch[((x ^ 1) * 128 + r) * 3 + 0], lo_ = xch[((x ^ 1) * 128 + r) * 3 + 1],
+                                uo = xch[((x ^ 1) * 128 + r) * 3 + 2];
+                    const float Mc = fmaxf(M, Mo);
+                    const float f0 = M == -INFINITY ? 0.f : ex2(M - Mc), f1 = Mo == -INFINITY ? 0.f : ex2(Mo - Mc);
+                    l = l * f0 + lo_ * f1;
+                    u = u * f0 + uo * f1;
+                    M = Mc;
                     const float Ms = lden > 0.f ? fmaxf(M, __log2f(lden)) : M;
                     const float a_soft = ex2(M - Ms), a_lin = lden > 0.f ? ex2(-Ms) : 0.f;
                     const float Z = fmaf(l, a_soft, lden * a_lin);
                     Lr = Ms + __log2f(Z);
                     Di = fmaf(u, a_soft, dl * a_lin) / Z;
-                    if (live) {
+                    if (live && x == 0) {
                         p.L[row] = Lr;
                         p.Dv[row] = Di;
                     }
                 }
             } else {
-                // ---- sweep 2: P = 2^(x - L), dS = P (dP - D) in bf16 over dP's first 32 columns
+                // ---- sweep 2: P = 2^(x - L), dS = P (dP - D) in bf16 into this half of the dS columns
                 const float2 sc2 = make_float2(sl2, sl2), nl2 = make_float2(-Lr, -Lr);
+                uint32_t ws[32], wd[32], pk[16];
+                tmem_ld32(tS, ws);
+                tmem_ld32(tDP, wd);
+                tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(BAR(Cfg::B_SDONE));  // S and dP of this tile are in registers
 #pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    uint32_t ws[32], wd[32], pk[16];
-                    tmem_ld32(tS + c * 32, ws);
-                    tmem_ld32(tDP + c * 32, wd);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int c0 = c * 32 + 2 * e;
-                        const float2 x = ffma2(make_float2(__uint_as_float(ws[2 * e]), __uint_as_float(ws[2 * e + 1])),
-                                               sc2, nl2);
-                        const float d0 = c0 < lim ? ex2(x.x) * (__uint_as_float(wd[2 * e]) - Di) : 0.f;
-                        const float d1 = c0 + 1 < lim ? ex2(x.y) * (__uint_as_float(wd[2 * e + 1]) - Di) : 0.f;
-                        pk[e] = pack_bf16x2(d0, d1);
-                    }
-                    // columns [16c, 16c + 16) of dP were read above (chunk c loaded columns 32c..32c+31)
-                    tmem_st16(tDP + c * 16, pk);
+                for (int e = 0; e < 16; ++e) {
+                    const float2 xx = ffma2(make_float2(__uint_as_float(ws[2 * e]), __uint_as_float(ws[2 * e + 1])),
+                                            sc2, nl2);
+                    const float d0 = 2 * e < lim ? ex2(xx.x) * (__uint_as_float(wd[2 * e]) - Di) : 0.f;
+                    const float d1 = 2 * e + 1 < lim ? ex2(xx.y) * (__uint_as_float(wd[2 * e + 1]) - Di) : 0.f;
+                    pk[e] = pack_bf16x2(d0, d1);
                 }
+                tmem_st16(tDS + 32 * (jj & 1), pk);
                 tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(BAR(Cfg::B_SDONE));
+                mbar_arrive(BAR(Cfg::B_DSFULL + ((jj - nt) & 1)));
             }
         }
-        // ---- epilogue: dq = tau dQ (fp32)
+        // ---- epilogue: dq = tau dQ (fp32); warpgroup x writes columns [x DH/2, (x + 1) DH/2)
         ok = warp_all(ok && mbar_wait(BAR(Cfg::B_DQ), 0, abort_flag));
         if (ok) {
             tc_fence_after();
 #pragma unroll
-            for (int c = 0; c < DH / 32; ++c) {
+            for (int c = 0; c < DH / 64; ++c) {
+                const int col = x * (DH / 2) + c * 32;
                 uint32_t w[32];
-                tmem_ld32(tDQ + c * 32, w);
+                tmem_ld32(tmem + lane_off + Cfg::DQ_COL + col, w);
                 tmem_wait_ld();
                 if (live) {
-                    float4 *dst = reinterpret_cast<float4 *>(p.dq + row * DH + c * 32);
+                    float4 *dst = reinterpret_cast<float4 *>(p.dq + row * DH + col);
 #pragma unroll
                     for (int v4 = 0; v4 < 8; ++v4)
                         dst[v4] = make_float4(__uint_as_float(w[4 * v4]) * p.scale, __uint_as_float(w[4 * v4 + 1]) * p.scale,
@@ -339,26 +363,30 @@ struct BwdKVCfg {
     static constexpr int Q_REG = 64 * 128;           // 64 rows x 64 bf16
     static constexpr int K_BYTES = 128 * DH * 2;     // K / V tile of 128 keys
     static constexpr int Q_BYTES = 64 * DH * 2;      // Q / dO tile of 64 query rows
-    static constexpr int NS = DH == 64 ? 4 : 2;      // query stages
+    static constexpr int NS = DH == 64 ? 8 : 4;      // query stages
     static constexpr int STAGE_BYTES = 2 * Q_BYTES + 1024;  // Q, dO, then L and D of the 64 rows
     static constexpr int OFF_K = 0, OFF_V = K_BYTES, OFF_STAGE = 2 * K_BYTES,
                          OFF_BAR = OFF_STAGE + NS * STAGE_BYTES;
-    static constexpr int B_KVFULL = 0, B_S = 1, B_SDONE = 2, B_ACC = 3, B_DRAIN = 4, B_QFULL = 5,
-                         B_STFULL = 5 + NS, B_QEMPTY = 5 + 2 * NS, NUM_BARS = 5 + 3 * NS;
-    static constexpr int TMEM_SLOT_OFF = 8 * NUM_BARS, ABORT_OFF = TMEM_SLOT_OFF + 8, BAR_BYTES = 256;
+    // Two S^T / dP^T buffers: tile u uses buffer u & 1 and warpgroup u & 1 of the row warps, so the
+    // MMAs of tile u + 1 run while the other warpgroup works on tile u.  B_S + b: S^T, dP^T of a tile
+    // in buffer b are ready; B_PDONE + b: P^T, dS^T of that tile are written.
+    static constexpr int B_KVFULL = 0, B_ACC = 1, B_DRAIN = 2, B_S = 3, B_PDONE = 5, B_QFULL = 7,
+                         B_STFULL = 7 + NS, B_QEMPTY = 7 + 2 * NS, NUM_BARS = 7 + 3 * NS;
+    static constexpr int TMEM_SLOT_OFF = 8 * NUM_BARS, ABORT_OFF = TMEM_SLOT_OFF + 8, BAR_BYTES = 512;
     static_assert(ABORT_OFF + 8 <= BAR_BYTES, "barrier area overflow");
     static constexpr int SMEM = OFF_BAR + BAR_BYTES + 1024;
-    static constexpr int THREADS = 192, PRODUCER_WARP = 4, MMA_WARP = 5;
-    // S^T (64 queries; P^T in bf16 over its first 32 columns), dP^T (dS^T likewise), dV, dK
-    static constexpr int S_COL = 0, DP_COL = 64, DV_COL = 128, DK_COL = 128 + DH;
-    static constexpr int TMEM_COLS = DH == 64 ? 256 : 512;
+    static_assert(SMEM <= 232448, "shared memory");
+    static constexpr int THREADS = 320, PRODUCER_WARP = 8, MMA_WARP = 9;
+    // per buffer b: S^T (64 queries; P^T in bf16 over its first 32 columns), dP^T (dS^T likewise);
+    // then dV, dK
+    __host__ __device__ static constexpr int s_col(int b) { return 128 * b; }
+    __host__ __device__ static constexpr int dp_col(int b) { return 128 * b + 64; }
+    static constexpr int DV_COL = 256, DK_COL = 256 + DH, TMEM_COLS = 512;
     static_assert(DK_COL + DH <= TMEM_COLS, "TMEM budget");
-    static constexpr int MIN_BLOCKS = DH == 64 ? 2 : 1;
-    static_assert(MIN_BLOCKS * (SMEM + 1024) <= 233472, "shared memory per SM");
 };
 
 template <int DH, bool KEPT>
-__global__ void __launch_bounds__(BwdKVCfg<DH>::THREADS, BwdKVCfg<DH>::MIN_BLOCKS)
+__global__ void __launch_bounds__(BwdKVCfg<DH>::THREADS, 1)
     bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
                       const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_do,
                       const BwdParams p) {
@@ -394,7 +422,7 @@ __global__ void __launch_bounds__(BwdKVCfg<DH>::THREADS, BwdKVCfg<DH>::MIN_BLOCK
     if (threadIdx.x == 0) {
         for (int i = 0; i < Cfg::NUM_BARS; ++i) {
             const bool stats = i >= Cfg::B_STFULL && i < Cfg::B_STFULL + Cfg::NS;
-            mbar_init(BAR(i), i == Cfg::B_SDONE ? 128 : stats ? 32 : 1);
+            mbar_init(BAR(i), i == Cfg::B_PDONE || i == Cfg::B_PDONE + 1 ? 128 : stats ? 32 : 1);
         }
         *abort_flag = 0;
         mbar_fence_init();
@@ -417,6 +445,22 @@ __global__ void __launch_bounds__(BwdKVCfg<DH>::THREADS, BwdKVCfg<DH>::MIN_BLOCK
             tma_load_3d_w(sbase + Cfg::OFF_K + rr * Cfg::K_REG, &map_k, BAR(Cfg::B_KVFULL), rr * 64, j0, bg);
             tma_load_3d_w(sbase + Cfg::OFF_V + rr * Cfg::K_REG, &map_v, BAR(Cfg::B_KVFULL), rr * 64, j0, bg);
         }
+        // L and D of a tile's 64 rows (zero past the sequence end; those columns are masked), two per
+        // lane, loaded into registers one tile ahead of their stores so the loads' latency overlaps
+        const float *__restrict__ gL = p.L;
+        const float *__restrict__ gD = p.Dv;
+        float nL[2], nD[2];
+        auto load_stats = [&](int u) {
+            const int hh = u / nqt, iq0 = qbeg + 64 * (u % nqt);
+            const size_t rb = (size_t)(b * p.H + g * p.G + hh) * p.N;
+#pragma unroll
+            for (int k2 = 0; k2 < 2; ++k2) {
+                const int i = iq0 + lane + 32 * k2;
+                nL[k2] = i < p.N ? __ldg(gL + rb + i) : 0.f;
+                nD[k2] = i < p.N ? __ldg(gD + rb + i) : 0.f;
+            }
+        };
+        if (tiles > 0) load_stats(0);
         for (int u = 0; u < tiles; ++u) {
             const int s = u % Cfg::NS;
             if (u >= Cfg::NS && !(ok = mbar_wait_w(BAR(Cfg::B_QEMPTY + s), ((u / Cfg::NS) - 1) & 1, abort_flag))) break;
@@ -428,15 +472,13 @@ __global__ void __launch_bounds__(BwdKVCfg<DH>::THREADS, BwdKVCfg<DH>::MIN_BLOCK
                 tma_load_3d_w(sQ + rr * Cfg::Q_REG, &map_q, BAR(Cfg::B_QFULL + s), rr * 64, iq0, bh);
                 tma_load_3d_w(sDO + rr * Cfg::Q_REG, &map_do, BAR(Cfg::B_QFULL + s), rr * 64, iq0, bh);
             }
-            // L and D of the 64 rows (zero past the sequence end; those columns are masked)
+            const float cL0 = nL[0], cL1 = nL[1], cD0 = nD[0], cD1 = nD[1];
+            if (u + 1 < tiles) load_stats(u + 1);
             float *st = reinterpret_cast<float *>(smem + Cfg::OFF_STAGE + s * Cfg::STAGE_BYTES + 2 * Cfg::Q_BYTES);
-#pragma unroll
-            for (int e = lane; e < 64; e += 32) {
-                const int i = iq0 + e;
-                const size_t row = (size_t)bh * p.N + i;
-                st[e] = i < p.N ? p.L[row] : 0.f;
-                st[64 + e] = i < p.N ? p.Dv[row] : 0.f;
-            }
+            st[lane] = cL0;
+            st[lane + 32] = cL1;
+            st[64 + lane] = cD0;
+            st[96 + lane] = cD1;
             mbar_arrive(BAR(Cfg::B_STFULL + s));
             issued = u + 1;
         }
@@ -454,40 +496,46 @@ __global__ void __launch_bounds__(BwdKVCfg<DH>::THREADS, BwdKVCfg<DH>::MIN_BLOCK
         constexpr uint32_t ID_ACC = idesc_bf16(128, DH, 0, 1);
         const uint32_t sK = sbase + Cfg::OFF_K, sV = sbase + Cfg::OFF_V;
         // dV += P^T dO and dK += dS^T Q for tile u: P^T / dS^T (bf16, 64 queries = 32 columns) from
-        // TMEM, dO / Q as MN-major B operands (N = DH, K = 64 query rows; 16 rows per k-step)
+        // buffer u & 1 of TMEM, dO / Q as MN-major B operands (N = DH, K = 64 query rows; 16 rows per
+        // k-step).  Issued before the scores of tile u + 2, which overwrite that buffer.
         auto issue_acc = [&](int u) {
+            const int b = u & 1;
             const uint32_t sQ = sbase + Cfg::OFF_STAGE + (u % Cfg::NS) * Cfg::STAGE_BYTES, sDO = sQ + Cfg::Q_BYTES;
             const uint64_t ddo = sw128_desc(sDO, Cfg::Q_REG, 1024), dqq = sw128_desc(sQ, Cfg::Q_REG, 1024);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                mma_ts_w(tm + Cfg::DV_COL, tm + Cfg::S_COL + kk * 8, ddo + (uint64_t)(kk * 128), ID_ACC,
+                mma_ts_w(tm + Cfg::DV_COL, tm + Cfg::s_col(b) + kk * 8, ddo + (uint64_t)(kk * 128), ID_ACC,
                          (u > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                mma_ts_w(tm + Cfg::DK_COL, tm + Cfg::DP_COL + kk * 8, dqq + (uint64_t)(kk * 128), ID_ACC,
+                mma_ts_w(tm + Cfg::DK_COL, tm + Cfg::dp_col(b) + kk * 8, dqq + (uint64_t)(kk * 128), ID_ACC,
                          (u > 0 || kk > 0) ? 1u : 0u);
             mma_commit_w(BAR(Cfg::B_QEMPTY + u % Cfg::NS));
         };
         bool ok = mbar_wait_w(BAR(Cfg::B_KVFULL), 0, abort_flag);
         for (int u = 0; ok && u < tiles; ++u) {
-            const int s = u % Cfg::NS;
+            const int s = u % Cfg::NS, b = u & 1;
             const uint32_t sQ = sbase + Cfg::OFF_STAGE + s * Cfg::STAGE_BYTES, sDO = sQ + Cfg::Q_BYTES;
             if (!(ok = mbar_wait_w(BAR(Cfg::B_QFULL + s), (u / Cfg::NS) & 1, abort_flag))) break;
-            if (u > 0) {
-                if (!(ok = mbar_wait_w(BAR(Cfg::B_SDONE), (u - 1) & 1, abort_flag))) break;
-                tc_fence_after();
-                issue_acc(u - 1);  // in issue order before S^T, dP^T(u) overwrite P^T, dS^T
-            }
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < DH / 16; ++kk)
-                mma_ss_w(tm + Cfg::S_COL, kmajor_desc(sK, kk, Cfg::K_REG), kmajor_desc(sQ, kk, Cfg::Q_REG), ID_S, kk > 0);
+                mma_ss_w(tm + Cfg::s_col(b), kmajor_desc(sK, kk, Cfg::K_REG), kmajor_desc(sQ, kk, Cfg::Q_REG), ID_S,
+                         kk > 0);
 #pragma unroll
             for (int kk = 0; kk < DH / 16; ++kk)
-                mma_ss_w(tm + Cfg::DP_COL, kmajor_desc(sV, kk, Cfg::K_REG), kmajor_desc(sDO, kk, Cfg::Q_REG), ID_S, kk > 0);
-            mma_commit_w(BAR(Cfg::B_S));
+                mma_ss_w(tm + Cfg::dp_col(b), kmajor_desc(sV, kk, Cfg::K_REG), kmajor_desc(sDO, kk, Cfg::Q_REG), ID_S,
+                         kk > 0);
+            mma_commit_w(BAR(Cfg::B_S + b));
+            if (u > 0) {
+                // P^T, dS^T of tile u-1 written by the other warpgroup (overlaps S^T, dP^T of tile u)
+                const int v = u - 1;
+                if (!(ok = mbar_wait_w(BAR(Cfg::B_PDONE + (v & 1)), (v >> 1) & 1, abort_flag))) break;
+                tc_fence_after();
+                issue_acc(v);
+            }
         }
-        if (ok && (ok = mbar_wait_w(BAR(Cfg::B_SDONE), (tiles - 1) & 1, abort_flag))) {
+        if (ok && (ok = mbar_wait_w(BAR(Cfg::B_PDONE + ((tiles - 1) & 1)), ((tiles - 1) >> 1) & 1, abort_flag))) {
             tc_fence_after();
             issue_acc(tiles - 1);
             mma_commit_w(BAR(Cfg::B_ACC));
@@ -500,55 +548,59 @@ __global__ void __launch_bounds__(BwdKVCfg<DH>::THREADS, BwdKVCfg<DH>::MIN_BLOCK
         mbar_wait_drain(BAR(Cfg::B_DRAIN), 0, 100000000ull);
     } else {
         // ================================================================ row warps (TMEM lane = key)
-        const int r = warp * 32 + lane;
+        // warpgroup x takes the tiles u = x, x + 2, ... (TMEM buffer x)
+        const int x = warp >> 2, quarter = warp & 3;
+        const int r = quarter * 32 + lane;
         const int TK = p.T * p.k;
         // query rows i >= thr see this key: the key itself (window), or the chunk after the window
         // that follows the entry's chunk (kept)
         int thr;
         if (!KEPT) thr = j0 + r;
         else thr = j0 + r < TK ? ((j0 + r) / p.k + m + 1) * p.C : 0x7fffffff;
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-        const uint32_t tS = tmem + lane_off + Cfg::S_COL, tDP = tmem + lane_off + Cfg::DP_COL;
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        const uint32_t tS = tmem + lane_off + Cfg::s_col(x), tDP = tmem + lane_off + Cfg::dp_col(x);
         const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
         bool ok = true;
-        for (int u = 0; u < tiles; ++u) {
+        for (int u = x; u < tiles; u += 2) {
             const int s = u % Cfg::NS;
-            if (!(ok = warp_all(mbar_wait(BAR(Cfg::B_S), u & 1, abort_flag) &&
+            if (!(ok = warp_all(mbar_wait(BAR(Cfg::B_S + x), (u >> 1) & 1, abort_flag) &&
                                 mbar_wait(BAR(Cfg::B_STFULL + s), (u / Cfg::NS) & 1, abort_flag))))
                 break;
             tc_fence_after();
             const int iq0 = qbeg + 64 * (u % nqt);
             const int c_lo = thr - iq0, c_hi = p.N - iq0;  // columns c_lo <= c < c_hi count
-            const float *st = reinterpret_cast<const float *>(smem + Cfg::OFF_STAGE + s * Cfg::STAGE_BYTES + 2 * Cfg::Q_BYTES);
+            const float *st = reinterpret_cast<const float *>(smem + Cfg::OFF_STAGE + s * Cfg::STAGE_BYTES +
+                                                              2 * Cfg::Q_BYTES);
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
                 uint32_t ws[32], wd[32], pp[16], dd[16];
-                tmem_ld32(tS + c * 32, ws);
-                tmem_ld32(tDP + c * 32, wd);
+                tmem_ld32(tS + 32 * c, ws);
+                tmem_ld32(tDP + 32 * c, wd);
                 tmem_wait_ld();
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    const int c0 = c * 32 + 2 * e;
+                    const int c0 = 32 * c + 2 * e;
                     const float2 Lc = *reinterpret_cast<const float2 *>(st + c0);
                     const float2 Dc = *reinterpret_cast<const float2 *>(st + 64 + c0);
-                    const float2 x = ffma2(make_float2(__uint_as_float(ws[2 * e]), __uint_as_float(ws[2 * e + 1])), sc2,
-                                           make_float2(-Lc.x, -Lc.y));
+                    const float2 xx = ffma2(make_float2(__uint_as_float(ws[2 * e]), __uint_as_float(ws[2 * e + 1])), sc2,
+                                            make_float2(-Lc.x, -Lc.y));
                     const bool v0 = c0 >= c_lo && c0 < c_hi, v1 = c0 + 1 >= c_lo && c0 + 1 < c_hi;
-                    const float p0 = v0 ? ex2(x.x) : 0.f, p1 = v1 ? ex2(x.y) : 0.f;
+                    const float p0 = v0 ? ex2(xx.x) : 0.f, p1 = v1 ? ex2(xx.y) : 0.f;
                     const float d0 = v0 ? p0 * (__uint_as_float(wd[2 * e]) - Dc.x) : 0.f;
                     const float d1 = v1 ? p1 * (__uint_as_float(wd[2 * e + 1]) - Dc.y) : 0.f;
                     pp[e] = pack_bf16x2(p0, p1);
                     dd[e] = pack_bf16x2(d0, d1);
                 }
                 // columns [16c, 16c + 16) were read above (chunk c loaded columns 32c..32c+31)
-                tmem_st16(tS + c * 16, pp);
-                tmem_st16(tDP + c * 16, dd);
+                tmem_st16(tS + 16 * c, pp);
+                tmem_st16(tDP + 16 * c, dd);
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(BAR(Cfg::B_SDONE));
+            mbar_arrive(BAR(Cfg::B_PDONE + x));
         }
-        // ---- epilogue: dv = dV, dk = tau dK (window: written; kept: added into the entry's row)
+        // ---- epilogue: warpgroup 0 writes dv = dV, warpgroup 1 dk = tau dK (window: written; kept:
+        //      added into the entry's row)
         ok = warp_all(ok && mbar_wait(BAR(Cfg::B_ACC), 0, abort_flag));
         if (ok) {
             tc_fence_after();
@@ -560,26 +612,23 @@ __global__ void __launch_bounds__(BwdKVCfg<DH>::THREADS, BwdKVCfg<DH>::MIN_BLOCK
                 const int jr = p.idx[(size_t)bg * TK + e];
                 if (jr >= c * p.C && jr < (c + 1) * p.C) dst_row = jr;
             }
+            const uint32_t tA = tmem + lane_off + (x ? Cfg::DK_COL : Cfg::DV_COL);
+            float *out = x ? p.dk : p.dv;
+            const float f = x ? p.scale : 1.f;
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                const uint32_t tA = tmem + lane_off + (half ? Cfg::DK_COL : Cfg::DV_COL);
-                float *out = half ? p.dk : p.dv;
-                const float f = half ? p.scale : 1.f;
+            for (int c = 0; c < DH / 32; ++c) {
+                uint32_t w[32];
+                tmem_ld32(tA + c * 32, w);
+                tmem_wait_ld();
+                if (dst_row >= 0) {
+                    float4 *dst = reinterpret_cast<float4 *>(out + ((size_t)bg * p.N + dst_row) * DH + c * 32);
 #pragma unroll
-                for (int c = 0; c < DH / 32; ++c) {
-                    uint32_t w[32];
-                    tmem_ld32(tA + c * 32, w);
-                    tmem_wait_ld();
-                    if (dst_row >= 0) {
-                        float4 *dst = reinterpret_cast<float4 *>(out + ((size_t)bg * p.N + dst_row) * DH + c * 32);
-#pragma unroll
-                        for (int v4 = 0; v4 < 8; ++v4) {
-                            const float4 val = make_float4(__uint_as_float(w[4 * v4]) * f, __uint_as_float(w[4 * v4 + 1]) * f,
-                                                           __uint_as_float(w[4 * v4 + 2]) * f,
-                                                           __uint_as_float(w[4 * v4 + 3]) * f);
-                            if (KEPT) atomicAdd(dst + v4, val);
-                            else dst[v4] = val;
-                        }
+                    for (int v4 = 0; v4 < 8; ++v4) {
+                        const float4 val = make_float4(__uint_as_float(w[4 * v4]) * f, __uint_as_float(w[4 * v4 + 1]) * f,
+                                                       __uint_as_float(w[4 * v4 + 2]) * f,
+                                                       __uint_as_float(w[4 * v4 + 3]) * f);
+                        if (KEPT) atomicAdd(dst + v4, val);
+                        else dst[v4] = val;
                     }
                 }
             }
