@@ -150,13 +150,14 @@ def layer_flops(shape):
 
 # ----------------------------------------------------------------------------- clocks
 
-def profiled_traffic(workload: str):
-    """DRAM bytes per step of the merge launches from a committed ncu summary under profiles/ (a
-    block of `workload:`, `traffic_bytes_per_step:` and `source_sha256:` lines), or None when there
-    is none for this workload or the kernel sources changed since the capture."""
+def profiled_traffic(workload: str, prefix: str = "merge_"):
+    """DRAM bytes per step of the profiled launches (the merge pair; with prefix "bwd_", the
+    backward's dq kernel) from a committed ncu summary under profiles/<prefix>*.md (a block of
+    `workload:`, `traffic_bytes_per_step:` and `source_sha256:` lines), or None when there is none
+    for this workload or the kernel sources changed since the capture."""
     import glob
     import hashlib
-    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "merge_*.md"))):
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", prefix + "*.md"))):
         blocks, kv = [], {}
         with open(path) as f:
             for line in f:
@@ -1068,19 +1069,56 @@ def bench_backward(args, name, rank, world, local, cpu_seconds):
         e_.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(sum(s_.elapsed_time(e_) for s_, e_ in e_evs), world, "cuda")
-    # SIMT fp32 kernels: the ALU roofline is the FFMA rate, 148 SMs x 128 lanes x 2 FLOP x 1965 MHz
-    peak = 148 * 128 * 2 * 1.965e9 / 1e12
-    achieved = backward_flops(shape) / (ms_per_step / 1e3) / 1e12
+    # per-kernel breakdown: two more steps with events around the launches (outside the timed region)
+    still.still_timing_read()
+    still.still_timing_enable(True)
+    for _ in range(2):
+        flush.zero_()
+        step(devt)
+    torch.cuda.synchronize()
+    still.still_timing_enable(False)
+    kernel_ms = {k_: v_[0] / 2 for k_, v_ in still.still_timing_read().items() if v_[1]}
+    peaks = {}
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peaks = json.load(f)
+    except OSError:
+        pass
+    pairs = int(soft_sizes(shape).sum()) * shape.B * shape.H
+    if "bwd_dq" in kernel_ms:
+        # tensor-core path: the dominant kernel is the dq kernel; its algorithmic work is S = Q K^T,
+        # dP = dO V^T and dQ += dS K (6 d FLOP per query-head and softmax key; the statistics sweep
+        # that forms S and dP a first time is not counted)
+        peak = peaks.get("bf16_tflops", 1590.0)
+        dq_flops = 6 * shape.d * pairs
+        roof = {"kernel": "bwd_dq_tc_kernel (dq of the softmax branch)", "bound": "tensor",
+                "achieved": dq_flops / (kernel_ms["bwd_dq"] / 1e3) / 1e12, "peak": peak, "unit": "TFLOP/s",
+                "traffic": profiled_traffic(name, prefix="bwd_"),
+                "flops_per_launch": dq_flops,
+                "peak_source": "measured bf16_tflops (burst)" if "bf16_tflops" in peaks else "fallback 1.59 PFLOP/s",
+                "key_kernel": {"kernel": "bwd_dkv_tc_kernel (window and kept keys)", "ms": kernel_ms.get("bwd_dkv"),
+                               "flops": 8 * shape.d * pairs,
+                               "achieved": 8 * shape.d * pairs / (kernel_ms["bwd_dkv"] / 1e3) / 1e12
+                               if kernel_ms.get("bwd_dkv") else None},
+                "whole_pass": {"flops_per_step": backward_flops(shape),
+                               "achieved": backward_flops(shape) / (ms_per_step / 1e3) / 1e12}}
+        roof["frac"] = roof["achieved"] / peak
+    else:
+        # SIMT fp32 kernels: the ALU roofline is the FFMA rate, 148 SMs x 128 lanes x 2 FLOP x 1965 MHz
+        peak = 148 * 128 * 2 * 1.965e9 / 1e12
+        achieved = backward_flops(shape) / (ms_per_step / 1e3) / 1e12
+        roof = {"kernel": "backward pass (all kernels)", "bound": "alu", "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 FLOP x 1965 MHz (SIMT kernels)",
+                "flops_per_step": backward_flops(shape)}
     line = {
         "metric": METRIC_BACKWARD,
         "value": job_throughput(tokens, args.steps, world, total_ms), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": shape.dtype, "data": "synthetic",
         "config": dict(config_of(shape, args, name), **{"pass": "backward"}),
-        "roofline": {"kernel": "backward pass (all kernels)", "bound": "alu", "achieved": achieved, "peak": peak,
-                     "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
-                     "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 FLOP x 1965 MHz (SIMT kernels)",
-                     "flops_per_step": backward_flops(shape)},
+        "roofline": roof,
+        "kernel_ms_per_step": kernel_ms,
         "e2e": {"value": job_throughput(tokens, args.e2e_steps, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in pinned.values()),
                 "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in outs)},

@@ -285,7 +285,7 @@ STILL_API uint64_t still_launch_count(void);
 /*
  * Per-kernel timing for benchmarks (no counterpart in the method; host-side
  * instrumentation).  While enabled, every kernel launched by
- * still_hybrid_prefill and still_decode_step is bracketed by a pair of CUDA
+ * still_hybrid_prefill, still_decode_step and still_hybrid_backward is bracketed by a pair of CUDA
  * events recorded on the caller's stream (created on first use; at most
  * STILL_TIMING_MAX_LAUNCHES launches are kept; later ones are not timed).  still_timing_read synchronises those events and, for
  * each kernel class c < n, writes the summed milliseconds to ms[c] and the
@@ -294,7 +294,9 @@ STILL_API uint64_t still_launch_count(void);
  * 3 linear state, 4 softmax/linear merge (tensor-core path: window part with
  * the fused saliency), 5 decode-state export, 6 tensor-core merge of the kept
  * prefix and the linear branch, 7 decode append, 8 decode attention, 9 decode
- * combine, 10 decode chunk close.  Single-threaded use only.
+ * combine, 10 decode chunk close, 11 backward dq (tensor cores), 12 backward dk/dv
+ * (tensor cores, window and kept keys), 13 backward linear branch (linear state,
+ * NP-Map backward, chunk sums, key side; the tiled path).  Single-threaded use only.
  */
 /*
  * Test hooks of the head-dimension-64 tensor-core merge (no counterpart in the
@@ -313,7 +315,7 @@ STILL_API uint64_t still_launch_count(void);
 STILL_API void still_debug_merge(int stall, int max_ctas);
 
 #define STILL_TIMING_MAX_LAUNCHES 4096
-#define STILL_TIMING_CLASSES 11
+#define STILL_TIMING_CLASSES 14
 STILL_API still_status still_timing_enable(int on);
 STILL_API still_status still_timing_read(double *ms, int *launches, int n);
 

@@ -229,10 +229,12 @@ struct LinTile {
     // PT [DF][68] (phi(k)^T, dphi rows, dY^T), coef [64], kept mask [64]
     static constexpr int RBUF = WBUF;
     static constexpr int KEY_FLOATS = DH * kLd64 + RBUF + 64 * LDF + DF * kLd64 + 128;
+    // three CTAs per SM where the shared memory allows it (d = D = 64: at most 70 KB each)
+    static constexpr int MIN_BLOCKS = DH == 64 && DF == 64 ? 3 : 1;
 };
 
 template <typename T, int DH, int DF>
-__global__ void __launch_bounds__(kTileThreads) bwd_lin_pre_tile(Dims s, const T *__restrict__ q,
+__global__ void __launch_bounds__(kTileThreads, LinTile<DH, DF>::MIN_BLOCKS) bwd_lin_pre_tile(Dims s, const T *__restrict__ q,
                                                                  const T *__restrict__ Wq, const float *__restrict__ S,
                                                                  const float *__restrict__ z, const T *__restrict__ dO,
                                                                  float *__restrict__ Phi, float *__restrict__ SG,
@@ -303,7 +305,7 @@ __global__ void __launch_bounds__(kTileThreads) bwd_lin_pre_tile(Dims s, const T
 }
 
 template <typename T, int DH, int DF>
-__global__ void __launch_bounds__(kTileThreads) bwd_lin_post_tile(Dims s, const T *__restrict__ q,
+__global__ void __launch_bounds__(kTileThreads, LinTile<DH, DF>::MIN_BLOCKS) bwd_lin_post_tile(Dims s, const T *__restrict__ q,
                                                                   const T *__restrict__ Wq, const T *__restrict__ dO,
                                                                   const float *__restrict__ z,
                                                                   const float *__restrict__ L,
@@ -424,7 +426,7 @@ __global__ void __launch_bounds__(kTileThreads) bwd_lin_post_tile(Dims s, const 
 // Unselected keys of 64-key tiles of decided chunks: phi(k) from K Wk, dv += phi(k) R,
 // dphi(k) = V R^T - r, the NP-Map backward from phi(k): dk += dy Wk^T + coef k, dWk += k^T dy.
 template <typename T, int DH, int DF>
-__global__ void __launch_bounds__(kTileThreads) bwd_key_tile(Dims s, const T *__restrict__ k, const T *__restrict__ v,
+__global__ void __launch_bounds__(kTileThreads, LinTile<DH, DF>::MIN_BLOCKS) bwd_key_tile(Dims s, const T *__restrict__ k, const T *__restrict__ v,
                                                              const T *__restrict__ Wk, const int32_t *__restrict__ idx,
                                                              const float *__restrict__ R, const float *__restrict__ rr,
                                                              float *__restrict__ dk, float *__restrict__ dv,

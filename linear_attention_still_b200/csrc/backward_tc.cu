@@ -669,8 +669,10 @@ cudaError_t launch_bwd_cfg(const Dims &s, const void *q, const void *k, const vo
         auto kern = bwd_dq_tc_kernel<DH>;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
         if (e != cudaSuccess) return e;
+        const int ts = timing_begin(kTimeBwdDq, st);
         kern<<<(unsigned)(prm.n_qtiles * BH), Cfg::THREADS, Cfg::SMEM, st>>>(mq128, mdo128, mk64, mv64, mkh64, mvh64,
                                                                              prm);
+        timing_end(ts, st);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         ++*launches;
     }
@@ -688,7 +690,9 @@ cudaError_t launch_bwd_cfg(const Dims &s, const void *q, const void *k, const vo
         auto kern = bwd_dkv_tc_kernel<DH, false>;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
         if (e != cudaSuccess) return e;
+        const int ts = timing_begin(kTimeBwdDkv, st);
         kern<<<(unsigned)(prm.n_ktiles * BK), Cfg::THREADS, Cfg::SMEM, st>>>(mk128, mv128, mq64, mdo64, prm);
+        timing_end(ts, st);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         ++*launches;
     }
@@ -701,8 +705,10 @@ cudaError_t launch_bwd_cfg(const Dims &s, const void *q, const void *k, const vo
         auto kern = bwd_dkv_tc_kernel<DH, true>;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
         if (e != cudaSuccess) return e;
+        const int ts = timing_begin(kTimeBwdDkv, st);
         kern<<<(unsigned)((uint64_t)n_segs * prm.n_ktiles * BK), Cfg::THREADS, Cfg::SMEM, st>>>(mkh128, mvh128, mq64,
                                                                                                 mdo64, prm);
+        timing_end(ts, st);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         ++*launches;
     }

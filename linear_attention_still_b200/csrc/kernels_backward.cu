@@ -600,9 +600,11 @@ cudaError_t backward_t(const Dims &s, const void *q, const void *k, const void *
     // backward runs (it forms phi(k) itself), else from phi(k) of every key
     const bool tiled_state = tc_backward_supported(s) && tiled_linear_backward_supported(s) && tc_linear_supported(s);
     if (tiled_state) {
+        const int ts = timing_begin(kTimeBwdLinear, st);
         if ((e = launch_w_transpose(s.Hkv, s.d, s.D, Wk, w.wkt, st)) != cudaSuccess) return e;
         if ((e = launch_linear_tc(s, k, v, w.wkt, idx, w.S, w.z, err, st)) != cudaSuccess) return e;
         if ((e = launch_linear_prefix(s, w.S, w.z, nullptr, st)) != cudaSuccess) return e;
+        timing_end(ts, st);
         *launches += 3;
     } else {
         e = launch_npmap(s.B * s.Hkv * s.N, s.Hkv, s.N, s.d, s.D, s.bf16, k, Wk, w.phik, st);
@@ -624,7 +626,9 @@ cudaError_t backward_t(const Dims &s, const void *q, const void *k, const void *
             ++*launches;
         }
         if (tiled) {
+            const int ts = timing_begin(kTimeBwdLinear, st);
             e = launch_linear_backward_tiled(0, s, q, k, v, Wq, Wk, dO, idx, w, dq, dk, dv, dWq, dWk, st);
+            timing_end(ts, st);
             if (e != cudaSuccess) return e;
         } else {
             bwd_lin_pre_kernel<T><<<rgrid, 32 * kBwdWarps, 0, st>>>(s, Q, WQ, w.S, w.z, GO, w.A, w.dYq, w.Ms, w.iZ);
@@ -635,7 +639,9 @@ cudaError_t backward_t(const Dims &s, const void *q, const void *k, const void *
         if (e != cudaSuccess) return e;
         if (tiled) {
             // query side (dq, dWq), chunk sums, suffix, key side (dk, dv, dWk) of the linear branch
+            const int ts = timing_begin(kTimeBwdLinear, st);
             e = launch_linear_backward_tiled(1, s, q, k, v, Wq, Wk, dO, idx, w, dq, dk, dv, dWq, dWk, st);
+            timing_end(ts, st);
             if (e != cudaSuccess) return e;
             *launches += T_ > 0 ? 3 : 2;
             return cudaSuccess;

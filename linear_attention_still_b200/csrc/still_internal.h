@@ -107,7 +107,15 @@ still_status check_prefill_args(const still_dims *dims, const void *q, const voi
 // Per-kernel event timing (still_timing_enable): returns a slot for timing_end, or -1 when off.
 int timing_begin(int cls, cudaStream_t st);
 void timing_end(int slot, cudaStream_t st);
-enum TimingClass { kTimeDecodeAppend = 7, kTimeDecodeAttn = 8, kTimeDecodeCombine = 9, kTimeDecodeClose = 10 };
+enum TimingClass {
+    kTimeDecodeAppend = 7,
+    kTimeDecodeAttn = 8,
+    kTimeDecodeCombine = 9,
+    kTimeDecodeClose = 10,
+    kTimeBwdDq = 11,
+    kTimeBwdDkv = 12,
+    kTimeBwdLinear = 13
+};
 
 cudaError_t launch_decode_step(const Dims &s, unsigned char *state, const DecodeLayout &L, int pos, const void *Wq,
                                const void *Wk, const void *q_t, const void *k_t, const void *v_t, void *o_t,

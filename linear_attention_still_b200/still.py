@@ -245,7 +245,8 @@ def still_debug_merge(stall: bool = False, max_ctas: int = 0):
 
 
 TIMING_CLASSES = ("saliency", "topk_gather", "npmap", "linear_state", "merge", "state_export", "merge_prefix",
-                  "decode_append", "decode_attn", "decode_combine", "decode_close")
+                  "decode_append", "decode_attn", "decode_combine", "decode_close", "bwd_dq", "bwd_dkv",
+                  "bwd_linear")
 
 
 def still_timing_enable(on: bool = True):
