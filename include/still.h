@@ -214,14 +214,17 @@ STILL_API still_status still_hybrid_prefill_static(const still_dims *dims, const
  * one chunk-parallel implementation for training and inference): gradients of
  * L = sum(dO * o) with respect to q, k, v, Wq and Wk, with the per-chunk
  * selection idx held fixed (top-k is a discrete choice with no gradient).
- * Requires a window (w >= 1; STILL_ERR_UNSUPPORTED for w = 0).
+ * w = 0 (no window, k = 0: every earlier token in the linear set) is covered.
  *   q, k, v, Wq, Wk  as for still_hybrid_prefill (dtype)
  *   idx   [B,Hkv,T,k] int32, the selection the forward used (NULL when k = 0 or T = 0)
  *   dO    [B,H,N,d] dtype, the gradient of the layer output
  *   dq    [B,H,N,d], dk/dv [B,Hkv,N,d], dWq [H,d,D], dWk [Hkv,d,D]: fp32 out (overwritten)
  *   workspace  device scratch of still_backward_workspace_bytes(dims) bytes, 256-byte aligned
- * SIMT kernels with fp32 arithmetic (dk and dv accumulate with atomics, so
- * their rounding depends on the schedule).
+ * bf16 with d in {64, 128}, C a multiple of 128 and w >= 1: the softmax branch
+ * runs on tensor cores (P and dS enter the MMAs in bf16) and, for D in {64, 128},
+ * the linear branch in tiled fp32 kernels whose weight and chunk sums add with
+ * atomics; otherwise SIMT kernels with fp32 arithmetic (w = 0 among them).
+ * Sums that use atomics round in schedule order.
  */
 STILL_API size_t still_backward_workspace_bytes(const still_dims *dims);
 STILL_API still_status still_hybrid_backward(const still_dims *dims, const void *q, const void *k, const void *v,

@@ -250,7 +250,6 @@ still_status still_hybrid_backward(const still_dims *dims, const void *q, const 
     Dims s;
     still_status st = check_dims(dims, &s);
     if (st) return st;
-    if (s.w == 0) return STILL_ERR_UNSUPPORTED;  // token-granular linear set: not covered by this pass
     if ((long long)s.B * s.N == 0) return STILL_OK;
     const void *ptrs[] = {q, k, v, Wq, Wk, dO, dq, dk, dv, dWq, dWk, workspace};
     for (const void *p : ptrs)

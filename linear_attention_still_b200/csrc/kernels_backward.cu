@@ -588,6 +588,222 @@ __global__ void __launch_bounds__(32 * kBwdWarps) bwd_lin_post_kernel(Dims s, co
     }
 }
 
+// ------------------------------------------------------------------ w = 0 (no softmax window)
+// Every key j <= i is in the linear set of row i (pure causal linear attention with the NP-Map):
+// with w_ij = <phi(q_i), phi(k_j)>, Z_i = sum_{j<=i} w_ij, o_i = sum_{j<=i} w_ij v_j / Z_i,
+// D_i = <dO_i, o_i> and a_i = phi(q_i) / Z_i,
+//   dphi(q_i) = (sum_{j<=i} phi(k_j) (<v_j, dO_i> - D_i)) / Z_i,
+//   dphi(k_j) = sum_{i>=j} a_i (<dO_i, v_j> - D_i),   dv_j = sum_{i>=j} <a_i, phi(k_j)> dO_i.
+// The sums over earlier chunks come from the chunk states S_t, z_t (prefix) and R_t, r_t (suffix);
+// the rows of a key's own chunk are summed explicitly.  SIMT, fp32, correct-first.
+
+// One warp per query row: o_i, D_i, a_i, the NP-Map backward of q (dq written, dYq).
+template <typename T>
+__global__ void __launch_bounds__(32 * kBwdWarps) bwd_nowin_row_kernel(Dims s, const T *__restrict__ q,
+                                                                       const T *__restrict__ v,
+                                                                       const T *__restrict__ Wq,
+                                                                       const float *__restrict__ phik,
+                                                                       const float *__restrict__ S,
+                                                                       const float *__restrict__ z,
+                                                                       const T *__restrict__ dO, float *__restrict__ dq,
+                                                                       float *__restrict__ Abuf, float *__restrict__ Dbuf,
+                                                                       float *__restrict__ dYq) {
+    __shared__ __align__(16) float qs[kBwdWarps][kMaxD];
+    __shared__ __align__(16) float gs[kBwdWarps][kMaxD];
+    __shared__ __align__(16) float ps[kBwdWarps][kMaxDf];
+    __shared__ __align__(16) float dps[kBwdWarps][kMaxDf];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long row = (long long)blockIdx.x * kBwdWarps + warp;  // over B * H * N
+    if (row >= (long long)s.B * s.H * s.N) return;
+    const int d = s.d, D = s.D, G = s.G(), T_ = s.T();
+    const int i = (int)(row % s.N), h = (int)((row / s.N) % s.H), b = (int)(row / ((long long)s.N * s.H));
+    const int bg = b * s.Hkv + h / G, t = i / s.C, c0 = t * s.C;
+    for (int x = lane; x < d; x += 32) {
+        qs[warp][x] = to_f(q[(size_t)row * d + x]);
+        gs[warp][x] = to_f(dO[(size_t)row * d + x]);
+    }
+    __syncwarp();
+    npmap_row_warp<T>(qs[warp], Wq + (size_t)h * d * D, d, D, ps[warp], lane);
+    __syncwarp();
+    const size_t tslot = (size_t)bg * (T_ + 1) + t;
+    const float *St = S + tslot * D * d, *zt = z + tslot * D;
+    const T *Vb = v + (size_t)bg * s.N * d;
+    const float *Pk = phik + (size_t)bg * s.N * D;
+    // pass 1: Z and the numerator (lane holds elements x = lane + 32u)
+    float Z = 0.f;
+    for (int a = lane; a < D; a += 32) Z = fmaf(ps[warp][a], zt[a], Z);
+    Z = warp_sum(Z);
+    float num[kMaxD / 32];
+#pragma unroll
+    for (int u = 0; u < kMaxD / 32; ++u) {
+        const int x = lane + 32 * u;
+        float acc = 0.f;
+        if (x < d)
+            for (int a = 0; a < D; ++a) acc = fmaf(ps[warp][a], St[(size_t)a * d + x], acc);
+        num[u] = acc;
+    }
+    for (int j = c0; j <= i; ++j) {
+        float wj = 0.f;
+        for (int a = lane; a < D; a += 32) wj = fmaf(ps[warp][a], Pk[(size_t)j * D + a], wj);
+        wj = warp_sum(wj);
+        Z += wj;
+#pragma unroll
+        for (int u = 0; u < kMaxD / 32; ++u) {
+            const int x = lane + 32 * u;
+            if (x < d) num[u] = fmaf(wj, to_f(Vb[(size_t)j * d + x]), num[u]);
+        }
+    }
+    const float iZ = Z > 0.f ? 1.f / Z : 0.f;
+    float Di = 0.f;
+#pragma unroll
+    for (int u = 0; u < kMaxD / 32; ++u) {
+        const int x = lane + 32 * u;
+        if (x < d) Di = fmaf(gs[warp][x], num[u] * iZ, Di);
+    }
+    Di = warp_sum(Di);
+    // pass 2: dphi(q) = (S_t dO - D z_t + sum_j phi(k_j) (<v_j, dO> - D)) / Z
+    for (int a = lane; a < D; a += 32) {
+        const float *sr = St + (size_t)a * d;
+        float sg = 0.f;
+        for (int x = 0; x < d; ++x) sg = fmaf(sr[x], gs[warp][x], sg);
+        dps[warp][a] = sg - Di * zt[a];
+    }
+    __syncwarp();
+    for (int j = c0; j <= i; ++j) {
+        float vg = 0.f;
+        for (int x = lane; x < d; x += 32) vg = fmaf(to_f(Vb[(size_t)j * d + x]), gs[warp][x], vg);
+        const float cf = warp_sum(vg) - Di;
+        for (int a = lane; a < D; a += 32) dps[warp][a] = fmaf(cf, Pk[(size_t)j * D + a], dps[warp][a]);
+    }
+    for (int a = lane; a < D; a += 32) {
+        dps[warp][a] *= iZ;
+        Abuf[(size_t)row * D + a] = ps[warp][a] * iZ;
+    }
+    if (lane == 0) Dbuf[row] = Di;
+    __syncwarp();
+    float dxa[kMaxD / 32];
+    npmap_backward_warp<T>(qs[warp], Wq + (size_t)h * d * D, d, D, dps[warp], ps[warp], dxa, lane);
+    for (int c = lane; c < D; c += 32) dYq[(size_t)row * D + c] = ps[warp][c];
+#pragma unroll
+    for (int u = 0; u < kMaxD / 32; ++u) {
+        const int x = lane + 32 * u;
+        if (x < d) dq[(size_t)row * d + x] = dxa[u];
+    }
+}
+
+// One warp per key row j (chunk c): dphi(k_j), dv_j from the later chunks (R, r of slot c + 1 after
+// the suffix sums) and from the rows i >= j of chunk c (all heads of the group); then the NP-Map
+// backward of k (dk written, dYk).
+template <typename T>
+__global__ void __launch_bounds__(32 * kBwdWarps) bwd_nowin_key_kernel(Dims s, const T *__restrict__ k,
+                                                                       const T *__restrict__ v,
+                                                                       const T *__restrict__ Wk,
+                                                                       const float *__restrict__ phik,
+                                                                       const float *__restrict__ Abuf,
+                                                                       const float *__restrict__ Dbuf,
+                                                                       const T *__restrict__ dO,
+                                                                       const float *__restrict__ R,
+                                                                       const float *__restrict__ r, float *__restrict__ dk,
+                                                                       float *__restrict__ dv, float *__restrict__ dYk) {
+    __shared__ __align__(16) float ks[kBwdWarps][kMaxD];
+    __shared__ __align__(16) float vs[kBwdWarps][kMaxD];
+    __shared__ __align__(16) float dps[kBwdWarps][kMaxDf];
+    __shared__ __align__(16) float dys[kBwdWarps][kMaxDf];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long krow = (long long)blockIdx.x * kBwdWarps + warp;  // over B * Hkv * N
+    if (krow >= (long long)s.B * s.Hkv * s.N) return;
+    const int d = s.d, D = s.D, G = s.G(), T_ = s.T();
+    const int j = (int)(krow % s.N), bg = (int)(krow / s.N), b = bg / s.Hkv, g = bg % s.Hkv;
+    const int c = j / s.C, c1 = min(s.N, (c + 1) * s.C);
+    for (int x = lane; x < d; x += 32) {
+        ks[warp][x] = to_f(k[(size_t)krow * d + x]);
+        vs[warp][x] = to_f(v[(size_t)krow * d + x]);
+    }
+    __syncwarp();
+    const float *ph = phik + (size_t)krow * D;
+    const bool later = c + 1 <= T_;  // slot c + 1 exists (it is empty when no row lies past chunk c)
+    const size_t slot = (size_t)bg * (T_ + 1) + c + 1;
+    for (int a = lane; a < D; a += 32) {
+        float acc = 0.f;
+        if (later) {
+            const float *rr = R + slot * D * d + (size_t)a * d;
+            for (int x = 0; x < d; ++x) acc = fmaf(rr[x], vs[warp][x], acc);
+            acc -= r[slot * D + a];
+        }
+        dps[warp][a] = acc;
+    }
+    float dva[kMaxD / 32];
+#pragma unroll
+    for (int u = 0; u < kMaxD / 32; ++u) {
+        const int x = lane + 32 * u;
+        float acc = 0.f;
+        if (x < d && later)
+            for (int a = 0; a < D; ++a) acc = fmaf(R[slot * D * d + (size_t)a * d + x], ph[a], acc);
+        dva[u] = acc;
+    }
+    __syncwarp();
+    for (int hh = 0; hh < G; ++hh) {
+        const size_t rb = ((size_t)b * s.H + g * G + hh) * s.N;
+        for (int i = j; i < c1; ++i) {
+            const T *gi = dO + (rb + i) * d;
+            const float *ai = Abuf + (rb + i) * D;
+            float gv = 0.f, aw = 0.f;
+            for (int x = lane; x < d; x += 32) gv = fmaf(to_f(gi[x]), vs[warp][x], gv);
+            for (int a = lane; a < D; a += 32) aw = fmaf(ai[a], ph[a], aw);
+            const float cf = warp_sum(gv) - Dbuf[rb + i];
+            aw = warp_sum(aw);
+            for (int a = lane; a < D; a += 32) dps[warp][a] = fmaf(cf, ai[a], dps[warp][a]);
+#pragma unroll
+            for (int u = 0; u < kMaxD / 32; ++u) {
+                const int x = lane + 32 * u;
+                if (x < d) dva[u] = fmaf(aw, to_f(gi[x]), dva[u]);
+            }
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < kMaxD / 32; ++u) {
+        const int x = lane + 32 * u;
+        if (x < d) dv[(size_t)krow * d + x] = dva[u];
+    }
+    __syncwarp();
+    float dxa[kMaxD / 32];
+    npmap_backward_warp<T>(ks[warp], Wk + (size_t)g * d * D, d, D, dps[warp], dys[warp], dxa, lane);
+    for (int cc = lane; cc < D; cc += 32) dYk[(size_t)krow * D + cc] = dys[warp][cc];
+#pragma unroll
+    for (int u = 0; u < kMaxD / 32; ++u) {
+        const int x = lane + 32 * u;
+        if (x < d) dk[(size_t)krow * d + x] = dxa[u];
+    }
+}
+
+template <typename T>
+cudaError_t backward_nowin_t(const Dims &s, const void *q, const void *k, const void *v, const void *Wq,
+                             const void *Wk, const void *dO, float *dq, float *dk, float *dv, float *dWq, float *dWk,
+                             const BackwardScratch &w, unsigned *err, cudaStream_t st, int *launches) {
+    const T *Q = (const T *)q, *K = (const T *)k, *V = (const T *)v, *WQ = (const T *)Wq, *WK = (const T *)Wk;
+    const T *GO = (const T *)dO;
+    const int T_ = s.T();
+    Dims s0 = s;
+    s0.k = 0;  // w = 0: nothing is kept; every earlier chunk enters the linear state whole
+    cudaError_t e = launch_npmap(s.B * s.Hkv * s.N, s.Hkv, s.N, s.d, s.D, s.bf16, k, Wk, w.phik, st);
+    if (e != cudaSuccess) return e;
+    if ((e = launch_linear_state(s0, w.phik, v, nullptr, w.S, w.z, nullptr, err, st)) != cudaSuccess) return e;
+    *launches += 3;
+    const long long rows = (long long)s.B * s.H * s.N;
+    bwd_nowin_row_kernel<T><<<(unsigned)((rows + kBwdWarps - 1) / kBwdWarps), 32 * kBwdWarps, 0, st>>>(
+        s, Q, V, WQ, w.phik, w.S, w.z, GO, dq, w.A, w.Dv, w.dYq);
+    bwd_chunk_kernel<T><<<dim3(T_ + 1, s.B * s.Hkv, (s.D * s.d + s.D + 255) / 256), 256, 0, st>>>(s, w.A, w.Dv, GO,
+                                                                                               w.R, w.r);
+    if ((e = launch_bwd_suffix(s, w.R, w.r, st)) != cudaSuccess) return e;
+    const long long krows = (long long)s.B * s.Hkv * s.N;
+    bwd_nowin_key_kernel<T><<<(unsigned)((krows + kBwdWarps - 1) / kBwdWarps), 32 * kBwdWarps, 0, st>>>(
+        s, K, V, WK, w.phik, w.A, w.Dv, GO, w.R, w.r, dk, dv, w.dYk);
+    bwd_weight_kernel<T><<<dim3(s.d, s.H), 256, 0, st>>>(s.B, s.H, s.N, s.d, s.D, Q, w.dYq, dWq);
+    bwd_weight_kernel<T><<<dim3(s.d, s.Hkv), 256, 0, st>>>(s.B, s.Hkv, s.N, s.d, s.D, K, w.dYk, dWk);
+    *launches += 6;
+    return cudaGetLastError();
+}
+
 template <typename T>
 cudaError_t backward_t(const Dims &s, const void *q, const void *k, const void *v, const void *Wq, const void *Wk,
                        const int32_t *idx, const void *dO, float *dq, float *dk, float *dv, float *dWq,
@@ -694,6 +910,11 @@ cudaError_t launch_backward(const Dims &s, const void *q, const void *k, const v
                             const void *Wk, const int32_t *idx, const void *dO, float *dq, float *dk, float *dv,
                             float *dWq, float *dWk, const BackwardScratch &w, unsigned *err, cudaStream_t st,
                             int *launches) {
+    if (s.w == 0) {
+        if (s.bf16)
+            return backward_nowin_t<__nv_bfloat16>(s, q, k, v, Wq, Wk, dO, dq, dk, dv, dWq, dWk, w, err, st, launches);
+        return backward_nowin_t<float>(s, q, k, v, Wq, Wk, dO, dq, dk, dv, dWq, dWk, w, err, st, launches);
+    }
     if (s.bf16)
         return backward_t<__nv_bfloat16>(s, q, k, v, Wq, Wk, idx, dO, dq, dk, dv, dWq, dWk, w, err, st, launches);
     return backward_t<float>(s, q, k, v, Wq, Wk, idx, dO, dq, dk, dv, dWq, dWk, w, err, st, launches);

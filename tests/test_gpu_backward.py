@@ -20,6 +20,10 @@ CASES = {
     # d in {64, 128} take dk, dv by key blocks (window pass + kept pass); the cases above with d = 32 by atomics
     "bf16_keep_all_d64": Shape(B=1, H=2, Hkv=1, N=200, d=64, D=32, w=64, C=64, k=64),
     "f32_two_chunk_window_d128": Shape(B=1, H=2, Hkv=1, N=230, d=128, D=64, w=64, C=32, k=8, dtype="f32"),
+    # w = 0: no window, every earlier token in the linear set (pure causal linear attention)
+    "f32_no_window": Shape(B=1, H=4, Hkv=2, N=150, d=32, D=16, w=0, C=32, k=0, dtype="f32"),
+    "bf16_no_window_gqa": Shape(B=2, H=4, Hkv=1, N=200, d=64, D=32, w=0, C=64, k=0),
+    "bf16_no_window_d128_ragged": Shape(B=1, H=2, Hkv=2, N=300, d=128, D=64, w=0, C=128, k=0),
     # bf16, d in {64, 128}, C a multiple of 128: the softmax branch on tensor cores (backward_tc.cu)
     "tc_bf16_gqa_ragged": Shape(B=2, H=8, Hkv=2, N=700, d=64, D=64, w=128, C=128, k=16),
     "tc_bf16_d128_two_chunk_window": Shape(B=1, H=4, Hkv=1, N=600, d=128, D=128, w=256, C=128, k=32),
