@@ -217,7 +217,7 @@ still_status still_diagonal_score(const still_dims *dims, const void *q, const v
 
 namespace {
 // Backward scratch layout (256-byte aligned fp32 segments).
-constexpr int kBwdSegments = 15;
+constexpr int kBwdSegments = 17;
 size_t backward_layout(const Dims &s, size_t *off) {
     const size_t BH = (size_t)s.B * s.H, BK = (size_t)s.B * s.Hkv, T1 = (size_t)s.T() + 1;
     // tensor-core path: the rows' log2 normalisers and the gathered kept rows (bf16, in fp32 units)
@@ -226,7 +226,9 @@ size_t backward_layout(const Dims &s, size_t *off) {
     const size_t sizes[kBwdSegments] = {BK * s.N * s.D, BK * T1 * s.D * s.d, BK * T1 * s.D, BH * s.N * s.D, BH * s.N,
                                         BH * s.N * s.D, BK * T1 * s.D * s.d, BK * T1 * s.D, BK * s.N * s.D, BH * s.N,
                                         BH * s.N, tc ? BH * s.N : 0, kept, kept,
-                                        tc ? ((size_t)s.Hkv * s.d * s.D * 2 + 3) / 4 : 0};
+                                        tc ? ((size_t)s.Hkv * s.d * s.D * 2 + 3) / 4 : 0,
+                                        tc ? ((size_t)s.H * s.d * s.D * 2 + 3) / 4 : 0,
+                                        tc ? (BK * T1 * s.d * s.D * 2 + 3) / 4 : 0};
     size_t o = 0;
     for (int i = 0; i < kBwdSegments; ++i) {
         off[i] = o;
@@ -261,7 +263,7 @@ still_status still_hybrid_backward(const still_dims *dims, const void *q, const 
     if (((uintptr_t)workspace & 255u) != 0) return STILL_ERR_INVALID_ARG;
     unsigned char *ws = static_cast<unsigned char *>(workspace);
     auto F = [&](int i) { return reinterpret_cast<float *>(ws + off[i]); };
-    BackwardScratch w{F(0), F(1), F(2), F(3), F(4), F(9), F(10), F(5), F(6), F(7), F(8), F(11), F(12), F(13), F(14)};
+    BackwardScratch w{F(0), F(1), F(2), F(3), F(4), F(9), F(10), F(5), F(6), F(7), F(8), F(11), F(12), F(13), F(14), F(15), F(16)};
     int launches = 0;
     cudaError_t e = launch_backward(s, q, k, v, Wq, Wk, select ? idx : nullptr, dO, dq, dk, dv, dWq, dWk, w,
                                     device_error_word(), static_cast<cudaStream_t>(stream), &launches);

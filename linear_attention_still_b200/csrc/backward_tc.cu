@@ -42,7 +42,9 @@ namespace {
 struct BwdParams {
     int B, H, Hkv, N, C, k, w, G, T;
     float scale, scale_log2;  // tau, tau log2(e)
-    const float *lden, *dl;   // [B,H,N] from the linear pre-pass (dq kernel)
+    const float *lden, *dl;   // [B,H,N] from the linear pre-pass (dq kernel without its own prologue)
+    const float *z;           // [B*Hkv*(T+1), D] z_t (dq kernel prologue)
+    float *Phi, *SG;          // [B,H,N,D] phi(q) and S_t dO (fp32), written by the dq kernel prologue
     float *L, *Dv;            // [B,H,N] log2 normaliser and D_i (dq kernel writes, key kernel reads)
     float *dq, *dk, *dv;      // fp32 gradients
     const int32_t *idx;       // [B,Hkv,T,k] (kept keys)
@@ -53,40 +55,56 @@ struct BwdParams {
 };
 
 // ================================================================================ dq kernel
-template <int DH>
+// DF = 0: the rows' linear terms (phi(q).z_t, <phi(q)^T S_t, dO>) come from the pre-pass in global
+// memory.  DF in {64, 128}: the kernel forms them itself in a prologue on the tensor cores:
+// Y = Q Wq^T, phi(q) per row (stored fp32 for the linear branch's later kernels and in bf16 over
+// Y's TMEM columns), lin = phi(q) S_t^T and sg = dO S_t (bf16 S_t^T; sg stored fp32), as the forward
+// merge's prologue does.
+template <int DH, int DF>
 struct BwdQCfg {
+    static constexpr bool PRO = DF > 0;
     static constexpr int Q_REG = 128 * 128;          // 128 rows x 64 bf16 (one SW128 region)
     static constexpr int K_REG = 64 * 128;           // 64 rows x 64 bf16
     static constexpr int Q_BYTES = 128 * DH * 2;     // Q / dO tile (DH/64 regions)
     static constexpr int K_BYTES = 64 * DH * 2;      // K / V tile of 64 keys
-    static constexpr int NS = DH == 64 ? 4 : 2;      // K/V stages
+    static constexpr int WQ_BYTES = PRO ? DF * DH * 2 : 0;  // Wq^T [DF rows x DH] (DH/64 regions of DF rows)
+    static constexpr int ST_BYTES = PRO ? DH * DF * 2 : 0;  // S_t^T [DH rows x DF] (DF/64 regions of DH rows)
+    static constexpr int NS = DH == 64 ? (DF == 128 ? 2 : PRO ? 3 : 4) : 2;  // K/V stages
     static constexpr int STAGE_BYTES = 2 * K_BYTES;
-    static constexpr int OFF_Q = 0, OFF_DO = Q_BYTES, OFF_STAGE = 2 * Q_BYTES,
-                         OFF_BAR = OFF_STAGE + NS * STAGE_BYTES;
+    static constexpr int OFF_Q = 0, OFF_DO = Q_BYTES, OFF_WQ = 2 * Q_BYTES, OFF_ST = OFF_WQ + WQ_BYTES,
+                         OFF_STAGE = OFF_ST + ST_BYTES, OFF_BAR = OFF_STAGE + NS * STAGE_BYTES;
     // B_SDONE: the row warps hold S, dP of a tile in registers; B_DSFULL + (n & 1): they wrote the dS
     // of sweep-2 tile n (two barriers taking turns, so neither runs two phases ahead of its waiter)
+    // prologue: B_WFULL (Wq^T, S_t^T tiles), B_Y (Y done), B_PHI (phi(q) written, warpgroup 0),
+    // B_LIN (lin and sg done), B_PRO (warpgroup 0 has read them)
     static constexpr int B_QFULL = 0, B_S = 1, B_SDONE = 2, B_DQ = 3, B_DRAIN = 4, B_WG = 5, B_DSFULL = 6,
-                         B_KFULL = 8, B_VFULL = 8 + NS, B_KVEMPTY = 8 + 2 * NS, NUM_BARS = 8 + 3 * NS;
+                         B_WFULL = 8, B_Y = 9, B_PHI = 10, B_LIN = 11, B_PRO = 12, B_KFULL = 13, B_VFULL = 13 + NS,
+                         B_KVEMPTY = 13 + 2 * NS, NUM_BARS = 13 + 3 * NS;
     static constexpr int TMEM_SLOT_OFF = 8 * NUM_BARS, ABORT_OFF = TMEM_SLOT_OFF + 8, BAR_BYTES = 256;
     static_assert(ABORT_OFF + 8 <= BAR_BYTES, "barrier area overflow");
     static constexpr int OFF_XCH = OFF_BAR + BAR_BYTES;   // [2][128][3] row statistics of each half
-    static constexpr int SMEM = OFF_XCH + 2 * 128 * 3 * 4 + 1024;
+    static constexpr int OFF_LXC = OFF_XCH + 2 * 128 * 3 * 4;  // [128][2] lden, dl (prologue, for warpgroup 1)
+    static constexpr int SMEM = OFF_LXC + 128 * 2 * 4 + 1024;
     // Two warpgroups of row warps: warpgroup x takes key columns [32x, 32x + 32) of every tile.
     static constexpr int THREADS = 320, PRODUCER_WARP = 8, MMA_WARP = 9, ROW_THREADS = 256;
-    // S (64 keys), dP (64 keys), dQ (DH), dS of alternate tiles (bf16, 64 keys = 32 columns each)
+    // S (64 keys), dP (64 keys), dQ (DH), dS of alternate tiles (bf16, 64 keys = 32 columns each);
+    // prologue: Y then phi (bf16) at column 0, lin at DQ_COL, then sg at column 0
     static constexpr int S_COL = 0, DP_COL = 64, DQ_COL = 128, DS_COL = 128 + DH, TMEM_COLS = DH == 64 ? 256 : 512;
-    static_assert(DS_COL + 64 <= TMEM_COLS, "TMEM budget");
+    static constexpr int Y_COL = 0, LIN_COL = DQ_COL;
+    static_assert(DS_COL + 64 <= TMEM_COLS && DF <= 128, "TMEM budget");
     static constexpr int MIN_BLOCKS = DH == 64 ? 2 : 1;  // two CTAs per SM overlap each other's phases
     static_assert(MIN_BLOCKS * (SMEM + 1024) <= 233472, "shared memory per SM");
 };
 
-template <int DH>
-__global__ void __launch_bounds__(BwdQCfg<DH>::THREADS, BwdQCfg<DH>::MIN_BLOCKS)
+template <int DH, int DF>
+__global__ void __launch_bounds__(BwdQCfg<DH, DF>::THREADS, BwdQCfg<DH, DF>::MIN_BLOCKS)
     bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_do,
                      const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
                      const __grid_constant__ CUtensorMap map_kh, const __grid_constant__ CUtensorMap map_vh,
+                     const __grid_constant__ CUtensorMap map_wq, const __grid_constant__ CUtensorMap map_st,
                      const BwdParams p) {
-    using Cfg = BwdQCfg<DH>;
+    using Cfg = BwdQCfg<DH, DF>;
+    constexpr bool PRO = Cfg::PRO;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
@@ -110,12 +128,13 @@ __global__ void __launch_bounds__(BwdQCfg<DH>::THREADS, BwdQCfg<DH>::MIN_BLOCKS)
     const int nkt = (nk + 63) / 64;                     // kept tiles
     const int nt = nkt + (i0 + 128 - lo) / 64;          // key tiles per sweep
     const int ntot = 2 * nt;
+    const int tslot = bg * (p.T + 1) + t;               // linear state slot of the chunk
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < Cfg::NUM_BARS; ++i)
             mbar_init(BAR(i), i == Cfg::B_SDONE || i == Cfg::B_WG || i == Cfg::B_DSFULL || i == Cfg::B_DSFULL + 1
                                   ? Cfg::ROW_THREADS
-                                  : 1);
+                                  : (i == Cfg::B_PHI || i == Cfg::B_PRO) ? 128 : 1);
         *abort_flag = 0;
         mbar_fence_init();
     }
@@ -136,6 +155,13 @@ __global__ void __launch_bounds__(BwdQCfg<DH>::THREADS, BwdQCfg<DH>::MIN_BLOCKS)
         for (int rr = 0; rr < DH / 64; ++rr) {
             tma_load_3d_w(sbase + Cfg::OFF_Q + rr * Cfg::Q_REG, &map_q, BAR(Cfg::B_QFULL), rr * 64, i0, bh);
             tma_load_3d_w(sbase + Cfg::OFF_DO + rr * Cfg::Q_REG, &map_do, BAR(Cfg::B_QFULL), rr * 64, i0, bh);
+        }
+        if constexpr (PRO) {
+            mbar_arrive_expect_tx_w(BAR(Cfg::B_WFULL), Cfg::WQ_BYTES + Cfg::ST_BYTES);
+            for (int rr = 0; rr < DH / 64; ++rr)
+                tma_load_3d_w(sbase + Cfg::OFF_WQ + rr * (DF * 128), &map_wq, BAR(Cfg::B_WFULL), rr * 64, 0, h);
+            for (int rr = 0; rr < DF / 64; ++rr)
+                tma_load_3d_w(sbase + Cfg::OFF_ST + rr * (DH * 128), &map_st, BAR(Cfg::B_WFULL), rr * 64, 0, tslot);
         }
         for (int jj = 0; jj < ntot; ++jj) {
             const int s = jj % Cfg::NS;
@@ -159,6 +185,7 @@ __global__ void __launch_bounds__(BwdQCfg<DH>::THREADS, BwdQCfg<DH>::MIN_BLOCKS)
             *abort_flag = 1;
             if (lane == 0) report(p.err, DEV_ERR_TIMEOUT);
             mbar_wait_drain(BAR(Cfg::B_QFULL), 0, 100000000ull);
+            if (PRO) mbar_wait_drain(BAR(Cfg::B_WFULL), 0, 100000000ull);
             for (int jj = max(0, issued - Cfg::NS); jj < issued; ++jj) {
                 mbar_wait_drain(BAR(Cfg::B_KFULL + jj % Cfg::NS), (jj / Cfg::NS) & 1, 100000000ull);
                 mbar_wait_drain(BAR(Cfg::B_VFULL + jj % Cfg::NS), (jj / Cfg::NS) & 1, 100000000ull);
@@ -183,6 +210,34 @@ __global__ void __launch_bounds__(BwdQCfg<DH>::THREADS, BwdQCfg<DH>::MIN_BLOCKS)
             mma_commit_w(BAR(Cfg::B_KVEMPTY + jj % Cfg::NS));
         };
         bool ok = mbar_wait_w(BAR(Cfg::B_QFULL), 0, abort_flag);
+        if (PRO && ok && (ok = mbar_wait_w(BAR(Cfg::B_WFULL), 0, abort_flag))) {
+            // Y = Q Wq^T (K-major Wq^T rows of DH)
+            constexpr uint32_t ID_Y = idesc_bf16(128, PRO ? DF : 64, 0, 0);
+            constexpr uint32_t ID_LIN = idesc_bf16(128, DH, 0, 0);
+            constexpr uint32_t ID_SG = idesc_bf16(128, PRO ? DF : 64, 0, 1);
+            const uint32_t sWQ = sbase + Cfg::OFF_WQ, sST = sbase + Cfg::OFF_ST;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < DH / 16; ++kk)
+                mma_ss_w(tm + Cfg::Y_COL, kmajor_desc(sQ, kk, Cfg::Q_REG), kmajor_desc(sWQ, kk, DF * 128), ID_Y, kk > 0);
+            mma_commit_w(BAR(Cfg::B_Y));
+            if ((ok = mbar_wait_w(BAR(Cfg::B_PHI), 0, abort_flag))) {
+                tc_fence_after();
+                // lin = phi(q) S_t^T: phi (bf16) from TMEM, S_t^T rows of DF (K-major)
+#pragma unroll
+                for (int kk = 0; kk < DF / 16; ++kk)
+                    mma_ts_w(tm + Cfg::LIN_COL, tm + Cfg::Y_COL + kk * 8, kmajor_desc(sST, kk, DH * 128), ID_LIN, kk > 0);
+                // sg = dO S_t: the S_t^T tile as an MN-major operand (N = DF features, K = DH rows), over
+                // Y's columns (the MMA above, issued first, has read phi)
+                const uint64_t dst = sw128_desc(sST, DH * 128, 1024);
+#pragma unroll
+                for (int kk = 0; kk < DH / 16; ++kk)
+                    mma_ss_w(tm + Cfg::Y_COL, kmajor_desc(sDO, kk, Cfg::Q_REG), dst + (uint64_t)(kk * 128), ID_SG,
+                             kk > 0);
+                mma_commit_w(BAR(Cfg::B_LIN));
+                ok = mbar_wait_w(BAR(Cfg::B_PRO), 0, abort_flag);  // warpgroup 0 has read lin and sg
+            }
+        }
         for (int jj = 0; ok && jj < ntot; ++jj) {
             const int s = jj % Cfg::NS;
             const uint32_t sK = sbase + Cfg::OFF_STAGE + s * Cfg::STAGE_BYTES, sV = sK + Cfg::K_BYTES;
@@ -230,11 +285,132 @@ __global__ void __launch_bounds__(BwdQCfg<DH>::THREADS, BwdQCfg<DH>::MIN_BLOCKS)
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const uint32_t tS = tmem + lane_off + Cfg::S_COL + 32 * x, tDP = tmem + lane_off + Cfg::DP_COL + 32 * x,
                        tDS = tmem + lane_off + Cfg::DS_COL + 16 * x;
-        const float lden = live ? p.lden[row] : 0.f, dl = live ? p.dl[row] : 0.f;
+        float lden = 0.f, dl = 0.f;
+        bool ok = true;
+        if constexpr (!PRO) {
+            lden = live ? p.lden[row] : 0.f;
+            dl = live ? p.dl[row] : 0.f;
+        } else if (x == 0) {
+            // ---- prologue (warpgroup 0, row r): phi(q) from Y, lden = phi.z_t, dl = <lin, dO>, sg
+            const uint32_t tY = tmem + lane_off + Cfg::Y_COL;
+            ok = warp_all(mbar_wait(BAR(Cfg::B_QFULL), 0, abort_flag) && mbar_wait(BAR(Cfg::B_Y), 0, abort_flag));
+            if (ok) {
+                tc_fence_after();
+                // ||q||^2 from the swizzled Q tile
+                float qq = 0.f;
+#pragma unroll
+                for (int rr = 0; rr < DH / 64; ++rr)
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) {
+                        const uint4 w4 = *reinterpret_cast<const uint4 *>(smem + Cfg::OFF_Q + rr * Cfg::Q_REG + r * 128 +
+                                                                          ((ch ^ (r & 7)) << 4));
+                        const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&w4);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 f2 = __bfloat1622float2(h2[e]);
+                            qq = fmaf(f2.x, f2.x, fmaf(f2.y, f2.y, qq));
+                        }
+                    }
+                // three passes over Y in TMEM (32 columns at a time): max, sum of e^2, then phi
+                float ymax = -INFINITY;
+#pragma unroll
+                for (int c = 0; c < DF / 32; ++c) {
+                    uint32_t w[32];
+                    tmem_ld32(tY + 32 * c, w);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) ymax = fmaxf(ymax, __uint_as_float(w[e]));
+                }
+                float ee = 0.f;
+#pragma unroll
+                for (int c = 0; c < DF / 32; ++c) {
+                    uint32_t w[32];
+                    tmem_ld32(tY + 32 * c, w);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const float ex = ex2((__uint_as_float(w[e]) - ymax) * kLog2e);
+                        ee = fmaf(ex, ex, ee);
+                    }
+                }
+                const float fscale = sqrtf(qq) * rsqrtf(ee);
+                const float *zt = p.z + (size_t)tslot * DF;
+                float *phig = p.Phi + row * DF;
+#pragma unroll
+                for (int c = 0; c < DF / 32; ++c) {
+                    uint32_t w[32], pk[16];
+                    tmem_ld32(tY + 32 * c, w);
+                    tmem_wait_ld();
+                    float ph[32];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        ph[e] = ex2((__uint_as_float(w[e]) - ymax) * kLog2e) * fscale;
+                        lden = fmaf(ph[e], __ldg(zt + 32 * c + e), lden);
+                    }
+                    if (live) {
+#pragma unroll
+                        for (int v4 = 0; v4 < 8; ++v4)
+                            reinterpret_cast<float4 *>(phig + 32 * c)[v4] =
+                                make_float4(ph[4 * v4], ph[4 * v4 + 1], ph[4 * v4 + 2], ph[4 * v4 + 3]);
+                    }
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(ph[2 * e], ph[2 * e + 1]);
+                    // phi (bf16) of columns 32c.. lands on columns [16c, 16c + 16), already read
+                    tmem_st16(tY + 16 * c, pk);
+                }
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            mbar_arrive(BAR(Cfg::B_PHI));
+            ok = warp_all(ok && mbar_wait(BAR(Cfg::B_LIN), 0, abort_flag));
+            if (ok) {
+                tc_fence_after();
+                // dl = <phi(q)^T S_t, dO> with dO from the swizzled dO tile
+#pragma unroll
+                for (int c = 0; c < DH / 32; ++c) {
+                    uint32_t w[32];
+                    tmem_ld32(tmem + lane_off + Cfg::LIN_COL + 32 * c, w);
+                    tmem_wait_ld();
+                    const int rr = c >> 1;
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch) {
+                        const int chunk = (c & 1) * 4 + ch;  // 16-byte chunk of the 128-byte row
+                        const uint4 w4 = *reinterpret_cast<const uint4 *>(smem + Cfg::OFF_DO + rr * Cfg::Q_REG + r * 128 +
+                                                                          ((chunk ^ (r & 7)) << 4));
+                        const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&w4);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 f2 = __bfloat1622float2(h2[e]);
+                            dl = fmaf(__uint_as_float(w[ch * 8 + 2 * e]), f2.x, dl);
+                            dl = fmaf(__uint_as_float(w[ch * 8 + 2 * e + 1]), f2.y, dl);
+                        }
+                    }
+                }
+                // sg = dO S_t (fp32) for the linear branch's query side
+                float *sgg = p.SG + row * DF;
+#pragma unroll
+                for (int c = 0; c < DF / 32; ++c) {
+                    uint32_t w[32];
+                    tmem_ld32(tY + 32 * c, w);
+                    tmem_wait_ld();
+                    if (live) {
+#pragma unroll
+                        for (int v4 = 0; v4 < 8; ++v4)
+                            reinterpret_cast<float4 *>(sgg + 32 * c)[v4] =
+                                make_float4(__uint_as_float(w[4 * v4]), __uint_as_float(w[4 * v4 + 1]),
+                                            __uint_as_float(w[4 * v4 + 2]), __uint_as_float(w[4 * v4 + 3]));
+                    }
+                }
+            }
+            float *lx = reinterpret_cast<float *>(smem + Cfg::OFF_LXC);
+            lx[2 * r] = lden;
+            lx[2 * r + 1] = dl;
+            tc_fence_before();
+            mbar_arrive(BAR(Cfg::B_PRO));
+        }
         const float sl2 = p.scale_log2;
         float M = -INFINITY, l = 0.f, u = 0.f, Lr = 0.f, Di = 0.f;
-        bool ok = true;
-        for (int jj = 0; jj < ntot; ++jj) {
+        for (int jj = 0; ok && jj < ntot; ++jj) {
             if (!(ok = warp_all(mbar_wait(BAR(Cfg::B_S), jj & 1, abort_flag)))) break;
             tc_fence_after();
             const int j = jj < nt ? jj : jj - nt;
@@ -285,6 +461,11 @@ __global__ void __launch_bounds__(BwdQCfg<DH>::THREADS, BwdQCfg<DH>::MIN_BLOCKS)
                     if (!(ok = warp_all(mbar_wait(BAR(Cfg::B_WG), 0, abort_flag)))) break;
                     const float Mo = xch[((x ^ 1) * 128 + r) * 3 + 0], lo_ = xch[((x ^ 1) * 128 + r) * 3 + 1],
                                 uo = xch[((x ^ 1) * 128 + r) * 3 + 2];
+                    if (PRO && x == 1) {  // the prologue's linear terms of this row (warpgroup 0)
+                        const float *lx = reinterpret_cast<const float *>(smem + Cfg::OFF_LXC);
+                        lden = lx[2 * r];
+                        dl = lx[2 * r + 1];
+                    }
                     const float Mc = fmaxf(M, Mo);
                     const float f0 = M == -INFINITY ? 0.f : ex2(M - Mc), f1 = Mo == -INFINITY ? 0.f : ex2(Mo - Mc);
                     l = l * f0 + lo_ * f1;
@@ -646,9 +827,27 @@ __global__ void __launch_bounds__(BwdKVCfg<DH>::THREADS, 1)
     if (warp == Cfg::MMA_WARP) tmem_dealloc(tmem, Cfg::TMEM_COLS);
 }
 
+// The dq kernel with its own linear prologue (DF = D) or with the pre-pass's terms (DF = 0).
+template <int DH, int DF>
+cudaError_t launch_dq(const Dims &s, const CUtensorMap *maps, const void *wqt, const void *st_t, const BwdParams &prm,
+                      cudaStream_t st) {
+    using Cfg = BwdQCfg<DH, DF>;
+    CUtensorMap mwq = maps[0], mst = maps[0];
+    if (DF > 0 && (!make_map(&mwq, wqt, DH, DF, s.H, DF) ||
+                   !make_map(&mst, st_t, DF, DH, (uint64_t)s.B * s.Hkv * (s.T() + 1), DH)))
+        return cudaErrorInvalidValue;
+    auto kern = bwd_dq_tc_kernel<DH, DF>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+    if (e != cudaSuccess) return e;
+    kern<<<(unsigned)(prm.n_qtiles * (uint64_t)s.B * s.H), Cfg::THREADS, Cfg::SMEM, st>>>(
+        maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], mwq, mst, prm);
+    return cudaGetLastError();
+}
+
 template <int DH>
 cudaError_t launch_bwd_cfg(const Dims &s, const void *q, const void *k, const void *v, const void *khat,
-                           const void *vhat, const void *dO, const BwdParams &prm_in, cudaStream_t st, int *launches) {
+                           const void *vhat, const void *dO, const void *wqt, const void *st_t,
+                           const BwdParams &prm_in, cudaStream_t st, int *launches) {
     const int T = s.T();
     const uint64_t BH = (uint64_t)s.B * s.H, BK = (uint64_t)s.B * s.Hkv;
     const bool has_kept = s.k > 0 && T > 0;
@@ -664,16 +863,16 @@ cudaError_t launch_bwd_cfg(const Dims &s, const void *q, const void *k, const vo
         mkh64 = mk64, mvh64 = mv64;
     if (!ok) return cudaErrorInvalidValue;
     {
-        using Cfg = BwdQCfg<DH>;
         prm.n_qtiles = (s.N + 127) / 128;
-        auto kern = bwd_dq_tc_kernel<DH>;
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
-        if (e != cudaSuccess) return e;
+        const CUtensorMap maps[6] = {mq128, mdo128, mk64, mv64, mkh64, mvh64};
         const int ts = timing_begin(kTimeBwdDq, st);
-        kern<<<(unsigned)(prm.n_qtiles * BH), Cfg::THREADS, Cfg::SMEM, st>>>(mq128, mdo128, mk64, mv64, mkh64, mvh64,
-                                                                             prm);
+        cudaError_t e;
+        if (!wqt) e = launch_dq<DH, 0>(s, maps, nullptr, nullptr, prm, st);
+        else if (s.D == 64) e = launch_dq<DH, 64>(s, maps, wqt, st_t, prm, st);
+        else if (s.D == 128) e = launch_dq<DH, 128>(s, maps, wqt, st_t, prm, st);
+        else e = cudaErrorNotSupported;
         timing_end(ts, st);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if (e != cudaSuccess) return e;
         ++*launches;
     }
     // key kernels: 128-row key boxes, 64-row query / dO boxes
@@ -722,11 +921,13 @@ bool tc_backward_supported(const Dims &s) {
 }
 
 // Softmax branch of the backward pass on tensor cores: dq (written), the rows' L and D, then dk, dv
-// (window keys written, kept keys added).  lden, dl come from the linear pre-pass.
+// (window keys written, kept keys added).  The rows' linear terms come from the pre-pass (lden, dl)
+// or, with pro.wqt set (D in {64, 128}), from the dq kernel's own prologue, which also writes
+// phi(q) and S_t dO (pro.Phi, pro.SG) for the linear branch.
 cudaError_t launch_backward_tc(const Dims &s, const void *q, const void *k, const void *v, const void *khat,
                                const void *vhat, const int32_t *idx, const void *dO, const float *lden,
-                               const float *dl, float *L, float *Dv, float *dq, float *dk, float *dv, unsigned *err,
-                               cudaStream_t st, int *launches) {
+                               const float *dl, const BwdPrologue &pro, float *L, float *Dv, float *dq, float *dk,
+                               float *dv, unsigned *err, cudaStream_t st, int *launches) {
     BwdParams prm{};
     prm.B = s.B;
     prm.H = s.H;
@@ -741,6 +942,9 @@ cudaError_t launch_backward_tc(const Dims &s, const void *q, const void *k, cons
     prm.scale_log2 = s.scale * kLog2e;
     prm.lden = lden;
     prm.dl = dl;
+    prm.z = pro.z;
+    prm.Phi = pro.Phi;
+    prm.SG = pro.SG;
     prm.L = L;
     prm.Dv = Dv;
     prm.dq = dq;
@@ -748,8 +952,8 @@ cudaError_t launch_backward_tc(const Dims &s, const void *q, const void *k, cons
     prm.dv = dv;
     prm.idx = idx;
     prm.err = err;
-    if (s.d == 64) return launch_bwd_cfg<64>(s, q, k, v, khat, vhat, dO, prm, st, launches);
-    if (s.d == 128) return launch_bwd_cfg<128>(s, q, k, v, khat, vhat, dO, prm, st, launches);
+    if (s.d == 64) return launch_bwd_cfg<64>(s, q, k, v, khat, vhat, dO, pro.wqt, pro.st_t, prm, st, launches);
+    if (s.d == 128) return launch_bwd_cfg<128>(s, q, k, v, khat, vhat, dO, pro.wqt, pro.st_t, prm, st, launches);
     return cudaErrorNotSupported;
 }
 

@@ -819,9 +819,10 @@ cudaError_t backward_t(const Dims &s, const void *q, const void *k, const void *
         const int ts = timing_begin(kTimeBwdLinear, st);
         if ((e = launch_w_transpose(s.Hkv, s.d, s.D, Wk, w.wkt, st)) != cudaSuccess) return e;
         if ((e = launch_linear_tc(s, k, v, w.wkt, idx, w.S, w.z, err, st)) != cudaSuccess) return e;
-        if ((e = launch_linear_prefix(s, w.S, w.z, nullptr, st)) != cudaSuccess) return e;
+        if ((e = launch_linear_prefix(s, w.S, w.z, w.st_t, st)) != cudaSuccess) return e;  // + S_t^T (bf16)
+        if ((e = launch_w_transpose(s.H, s.d, s.D, Wq, w.wqt, st)) != cudaSuccess) return e;
         timing_end(ts, st);
-        *launches += 3;
+        *launches += 4;
     } else {
         e = launch_npmap(s.B * s.Hkv * s.N, s.Hkv, s.N, s.d, s.D, s.bf16, k, Wk, w.phik, st);
         if (e != cudaSuccess) return e;
@@ -841,16 +842,23 @@ cudaError_t backward_t(const Dims &s, const void *q, const void *k, const void *
             if ((e = launch_gather(s, idx, k, v, w.khat, w.vhat, err, st)) != cudaSuccess) return e;
             ++*launches;
         }
-        if (tiled) {
+        // tiled linear branch with the tensor-core linear state: the dq kernel forms the rows' linear
+        // terms itself (its prologue writes phi(q) and S_t dO for the later linear kernels)
+        BwdPrologue pro{nullptr, nullptr, w.z, w.A, w.dYq};
+        if (tiled && tiled_state) {
+            pro.wqt = w.wqt;
+            pro.st_t = w.st_t;
+        } else if (tiled) {
             const int ts = timing_begin(kTimeBwdLinear, st);
             e = launch_linear_backward_tiled(0, s, q, k, v, Wq, Wk, dO, idx, w, dq, dk, dv, dWq, dWk, st);
             timing_end(ts, st);
             if (e != cudaSuccess) return e;
+            ++*launches;
         } else {
             bwd_lin_pre_kernel<T><<<rgrid, 32 * kBwdWarps, 0, st>>>(s, Q, WQ, w.S, w.z, GO, w.A, w.dYq, w.Ms, w.iZ);
+            ++*launches;
         }
-        ++*launches;
-        e = launch_backward_tc(s, q, k, v, w.khat, w.vhat, idx, dO, w.Ms, w.iZ, w.L, w.Dv, dq, dk, dv, err, st,
+        e = launch_backward_tc(s, q, k, v, w.khat, w.vhat, idx, dO, w.Ms, w.iZ, pro, w.L, w.Dv, dq, dk, dv, err, st,
                                launches);
         if (e != cudaSuccess) return e;
         if (tiled) {

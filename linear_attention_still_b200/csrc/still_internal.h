@@ -76,6 +76,8 @@ struct BackwardScratch {
     float *L;      // [B,H,N]       tensor-core path: each row's log2 normaliser Ms log2(e) + log2 Z
     void *khat, *vhat;  // [B,Hkv,T*k,d] tensor-core path: the kept rows, gathered (bf16)
     void *wkt;     // [Hkv,D,d] tensor-core path: Wk^T (bf16), operand of the linear-state kernel
+    void *wqt;     // [H,D,d] tensor-core path: Wq^T (bf16), operand of the dq kernel's prologue
+    void *st_t;    // [B,Hkv,T+1,d,D] tensor-core path: S_t^T (bf16), operand of the dq kernel's prologue
 };
 bool tc_linear_supported(const Dims &s);
 cudaError_t launch_w_transpose(int Hx, int d, int D, const void *w, void *wt, cudaStream_t st);
@@ -90,10 +92,17 @@ cudaError_t launch_linear_backward_tiled(int which, const Dims &s, const void *q
 cudaError_t launch_bwd_suffix(const Dims &s, float *R, float *r, cudaStream_t st);
 cudaError_t launch_gather(const Dims &s, const int32_t *idx, const void *k, const void *v, void *khat, void *vhat,
                           unsigned *err, cudaStream_t st);
+// Inputs of the dq kernel's own linear prologue (wqt = nullptr: none; lden, dl are read instead).
+struct BwdPrologue {
+    const void *wqt;    // [H,D,d] Wq^T (bf16)
+    const void *st_t;   // [B,Hkv,T+1,d,D] S_t^T (bf16)
+    const float *z;     // [B,Hkv,T+1,D]
+    float *Phi, *SG;    // [B,H,N,D] out: phi(q), S_t dO
+};
 cudaError_t launch_backward_tc(const Dims &s, const void *q, const void *k, const void *v, const void *khat,
                                const void *vhat, const int32_t *idx, const void *dO, const float *lden,
-                               const float *dl, float *L, float *Dv, float *dq, float *dk, float *dv, unsigned *err,
-                               cudaStream_t st, int *launches);
+                               const float *dl, const BwdPrologue &pro, float *L, float *Dv, float *dq, float *dk,
+                               float *dv, unsigned *err, cudaStream_t st, int *launches);
 cudaError_t launch_backward(const Dims &s, const void *q, const void *k, const void *v, const void *Wq,
                             const void *Wk, const int32_t *idx, const void *dO, float *dq, float *dk, float *dv,
                             float *dWq, float *dWk, const BackwardScratch &w, unsigned *err, cudaStream_t st,
