@@ -39,6 +39,8 @@ using namespace tc;
 
 namespace {
 
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+
 struct BwdParams {
     int B, H, Hkv, N, C, k, w, G, T;
     float scale, scale_log2;  // tau, tau log2(e)
@@ -418,21 +420,33 @@ __global__ void __launch_bounds__(BwdQCfg<DH, DF>::THREADS, BwdQCfg<DH, DF>::MIN
             const int lim = (j < nkt ? nk - 64 * j : i - (lo + 64 * (j - nkt)) + 1) - 32 * x;
             if (jj < nt) {
                 // ---- sweep 1: running max, sum and sum of exp * <dO, v> over this half's columns
+                // (raw scores; tau log2(e) > 0 is applied to the max and inside the exponent's FFMA)
                 float sv[32];
                 {
                     uint32_t w[32];
                     tmem_ld32(tS, w);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) sv[e] = e < lim ? __uint_as_float(w[e]) * sl2 : -INFINITY;
+                    for (int e = 0; e < 32; ++e) sv[e] = __uint_as_float(w[e]);
                 }
-                float mt = -INFINITY;
+                if (!warp_all(lim >= 32)) {  // a ragged or diagonal tile: masked columns never win
 #pragma unroll
-                for (int e = 0; e < 32; ++e) mt = fmaxf(mt, sv[e]);
+                    for (int e = 0; e < 32; ++e) sv[e] = e < lim ? sv[e] : -INFINITY;
+                }
+                float m3[3] = {sv[0], sv[1], sv[2]};
+#pragma unroll
+                for (int e = 3; e + 2 < 32; e += 3) {
+                    m3[0] = fmaxf(m3[0], sv[e]);
+                    m3[1] = fmaxf(m3[1], sv[e + 1]);
+                    m3[2] = fmaxf(m3[2], sv[e + 2]);
+                }
+                const float mt = fmax3(fmax3(m3[0], m3[1], m3[2]), sv[30], sv[31]) * sl2;
                 const float mn = fmaxf(M, mt);
                 const float mref = mn == -INFINITY ? 0.f : mn;
                 const float sc = M == -INFINITY ? 0.f : ex2(M - mref);
-                float la = 0.f, lb = 0.f, ua = 0.f, ub = 0.f;
+                const float2 sl2v = make_float2(sl2, sl2), nm = make_float2(-mref, -mref);
+                float2 l2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+                float2 u2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
                 {
                     uint32_t w[32];
                     tmem_ld32(tDP, w);
@@ -441,15 +455,16 @@ __global__ void __launch_bounds__(BwdQCfg<DH, DF>::THREADS, BwdQCfg<DH, DF>::MIN
                     mbar_arrive(BAR(Cfg::B_SDONE));  // S and dP of this tile are in registers
 #pragma unroll
                     for (int e = 0; e < 32; e += 2) {
-                        const float p0 = ex2(sv[e] - mref), p1 = ex2(sv[e + 1] - mref);
-                        la += p0;
-                        lb += p1;
-                        ua = fmaf(p0, __uint_as_float(w[e]), ua);
-                        ub = fmaf(p1, __uint_as_float(w[e + 1]), ub);
+                        const float2 xx = ffma2(make_float2(sv[e], sv[e + 1]), sl2v, nm);
+                        const float2 pp = make_float2(ex2(xx.x), ex2(xx.y));
+                        l2[(e >> 1) & 1] = fadd2(l2[(e >> 1) & 1], pp);
+                        u2[(e >> 1) & 1] = ffma2(pp, make_float2(__uint_as_float(w[e]), __uint_as_float(w[e + 1])),
+                                                 u2[(e >> 1) & 1]);
                     }
                 }
-                l = fmaf(l, sc, la + lb);
-                u = fmaf(u, sc, ua + ub);
+                const float2 ls = fadd2(l2[0], l2[1]), us = fadd2(u2[0], u2[1]);
+                l = fmaf(l, sc, ls.x + ls.y);
+                u = fmaf(u, sc, us.x + us.y);
                 M = mn;
                 if (jj == nt - 1) {
                     // ---- combine the two halves, then the row's normaliser with the linear branch and D_i
@@ -483,20 +498,26 @@ __global__ void __launch_bounds__(BwdQCfg<DH, DF>::THREADS, BwdQCfg<DH, DF>::MIN
                 }
             } else {
                 // ---- sweep 2: P = 2^(x - L), dS = P (dP - D) in bf16 into this half of the dS columns
-                const float2 sc2 = make_float2(sl2, sl2), nl2 = make_float2(-Lr, -Lr);
+                const float2 sc2 = make_float2(sl2, sl2), nl2 = make_float2(-Lr, -Lr), nd2 = make_float2(-Di, -Di);
                 uint32_t ws[32], wd[32], pk[16];
                 tmem_ld32(tS, ws);
                 tmem_ld32(tDP, wd);
                 tmem_wait_ld();
                 tc_fence_before();
                 mbar_arrive(BAR(Cfg::B_SDONE));  // S and dP of this tile are in registers
+                const bool full = warp_all(lim >= 32);
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
                     const float2 xx = ffma2(make_float2(__uint_as_float(ws[2 * e]), __uint_as_float(ws[2 * e + 1])),
                                             sc2, nl2);
-                    const float d0 = 2 * e < lim ? ex2(xx.x) * (__uint_as_float(wd[2 * e]) - Di) : 0.f;
-                    const float d1 = 2 * e + 1 < lim ? ex2(xx.y) * (__uint_as_float(wd[2 * e + 1]) - Di) : 0.f;
-                    pk[e] = pack_bf16x2(d0, d1);
+                    float2 pp = make_float2(ex2(xx.x), ex2(xx.y));
+                    if (!full) {
+                        pp.x = 2 * e < lim ? pp.x : 0.f;
+                        pp.y = 2 * e + 1 < lim ? pp.y : 0.f;
+                    }
+                    const float2 dd = fmul2(pp, fadd2(make_float2(__uint_as_float(wd[2 * e]), __uint_as_float(wd[2 * e + 1])),
+                                                      nd2));
+                    pk[e] = pack_bf16x2(dd.x, dd.y);
                 }
                 tmem_st16(tDS + 32 * (jj & 1), pk);
                 tmem_wait_st();
@@ -750,6 +771,7 @@ __global__ void __launch_bounds__(BwdKVCfg<DH>::THREADS, 1)
             tc_fence_after();
             const int iq0 = qbeg + 64 * (u % nqt);
             const int c_lo = thr - iq0, c_hi = p.N - iq0;  // columns c_lo <= c < c_hi count
+            const bool full = warp_all(c_lo <= 0 && c_hi >= 64);
             const float *st = reinterpret_cast<const float *>(smem + Cfg::OFF_STAGE + s * Cfg::STAGE_BYTES +
                                                               2 * Cfg::Q_BYTES);
 #pragma unroll
@@ -765,12 +787,19 @@ __global__ void __launch_bounds__(BwdKVCfg<DH>::THREADS, 1)
                     const float2 Dc = *reinterpret_cast<const float2 *>(st + 64 + c0);
                     const float2 xx = ffma2(make_float2(__uint_as_float(ws[2 * e]), __uint_as_float(ws[2 * e + 1])), sc2,
                                             make_float2(-Lc.x, -Lc.y));
-                    const bool v0 = c0 >= c_lo && c0 < c_hi, v1 = c0 + 1 >= c_lo && c0 + 1 < c_hi;
-                    const float p0 = v0 ? ex2(xx.x) : 0.f, p1 = v1 ? ex2(xx.y) : 0.f;
-                    const float d0 = v0 ? p0 * (__uint_as_float(wd[2 * e]) - Dc.x) : 0.f;
-                    const float d1 = v1 ? p1 * (__uint_as_float(wd[2 * e + 1]) - Dc.y) : 0.f;
-                    pp[e] = pack_bf16x2(p0, p1);
-                    dd[e] = pack_bf16x2(d0, d1);
+                    float2 pv = make_float2(ex2(xx.x), ex2(xx.y));
+                    if (!full) {  // (the stats of masked columns may be garbage: select, never multiply)
+                        pv.x = c0 >= c_lo && c0 < c_hi ? pv.x : 0.f;
+                        pv.y = c0 + 1 >= c_lo && c0 + 1 < c_hi ? pv.y : 0.f;
+                    }
+                    float2 dv2 = fmul2(pv, fadd2(make_float2(__uint_as_float(wd[2 * e]), __uint_as_float(wd[2 * e + 1])),
+                                                 make_float2(-Dc.x, -Dc.y)));
+                    if (!full) {
+                        dv2.x = pv.x != 0.f ? dv2.x : 0.f;
+                        dv2.y = pv.y != 0.f ? dv2.y : 0.f;
+                    }
+                    pp[e] = pack_bf16x2(pv.x, pv.y);
+                    dd[e] = pack_bf16x2(dv2.x, dv2.y);
                 }
                 // columns [16c, 16c + 16) were read above (chunk c loaded columns 32c..32c+31)
                 tmem_st16(tS + 16 * c, pp);
