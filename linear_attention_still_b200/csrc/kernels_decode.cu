@@ -695,9 +695,14 @@ __device__ __forceinline__ bool bar_wait_bounded(uint32_t bar, uint32_t parity) 
     }
 }
 
+// k_t, v_t (optional): the step's new key and value, appended here instead of by a kernel of their
+// own: the CTA whose key range ends the list (it holds the diagonal, position pos) writes them into
+// the window ring before any of its copies start.
 template <int DH, int G>
 __global__ void __launch_bounds__(128, 2) decode_attn_bulk_kernel(Dims s, DecodeLayout L, unsigned char *state,
                                                                   StepGeom gm, const __nv_bfloat16 *__restrict__ q_t,
+                                                                  const __nv_bfloat16 *__restrict__ k_t,
+                                                                  const __nv_bfloat16 *__restrict__ v_t,
                                                                   unsigned *err) {
     using Cfg = DecodeBulkCfg<DH>;
     constexpr int NW = Cfg::NW, NST = Cfg::NST, NQ = DH / 32, NM = DH / 16, VW = DH / 64;
@@ -723,6 +728,22 @@ __global__ void __launch_bounds__(128, 2) decode_attn_bulk_kernel(Dims s, Decode
     }
     fence_proxy_async_smem();
     __syncwarp();
+    if (k_t) {
+        if (bg == 0 && split == 0 && threadIdx.x == 0 &&
+            reinterpret_cast<const DecodeHeader *>(state + L.header)->pos != gm.pos)
+            report(err, DEV_ERR_POSITION);
+        if (l1 == gm.n) {
+            const size_t row = (size_t)bg * L.ring_rows + ring_row(s, gm.pos);
+            for (int x = threadIdx.x; x < DH / 8; x += blockDim.x) {
+                reinterpret_cast<uint4 *>(const_cast<__nv_bfloat16 *>(rk) + row * DH)[x] =
+                    __ldg(reinterpret_cast<const uint4 *>(k_t + (size_t)bg * DH) + x);
+                reinterpret_cast<uint4 *>(const_cast<__nv_bfloat16 *>(rv) + row * DH)[x] =
+                    __ldg(reinterpret_cast<const uint4 *>(v_t + (size_t)bg * DH) + x);
+            }
+            asm volatile("fence.proxy.async.global;" ::: "memory");  // the row, before the bulk copies read it
+        }
+        __syncthreads();
+    }
 
     const int ntiles = (l1 - l0 + 15) / 16;
     const int my_tiles = ntiles > warp ? (ntiles - warp + NW - 1) / NW : 0;
@@ -1531,10 +1552,17 @@ static cudaError_t decode_step_t(const Dims &s, unsigned char *state, const Deco
         gm.nsplit = best;
     }
     gm.per = gm.nsplit ? (gm.n + gm.nsplit - 1) / gm.nsplit : 0;
-    int ts = timing_begin(kTimeDecodeAppend, st);
-    decode_append_kernel<T><<<BK, 128, 0, st>>>(s, L, state, pos, (const T *)k_t, (const T *)v_t, err);
-    timing_end(ts, st);
-    ++*launches;
+    // the bulk-copy attention kernel appends the step's key and value itself
+    const int Gs = s.G();
+    const bool fold_append = kDecodeBulk && gm.nsplit > 0 && sizeof(T) == 2 && (s.d == 64 || s.d == 128) &&
+                             (Gs == 1 || Gs == 2 || Gs == 4 || Gs == 8);
+    int ts = -1;
+    if (!fold_append) {
+        ts = timing_begin(kTimeDecodeAppend, st);
+        decode_append_kernel<T><<<BK, 128, 0, st>>>(s, L, state, pos, (const T *)k_t, (const T *)v_t, err);
+        timing_end(ts, st);
+        ++*launches;
+    }
     if (gm.nsplit) {
         ts = timing_begin(kTimeDecodeAttn, st);
         const dim3 grid(BK, gm.nsplit);
@@ -1548,8 +1576,9 @@ static cudaError_t decode_step_t(const Dims &s, unsigned char *state, const Deco
             cudaError_t e_ = cudaFuncSetAttribute(decode_attn_bulk_kernel<DH, GG>,                          \
                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smem_);      \
             if (e_ != cudaSuccess) return e_;                                                               \
-            decode_attn_bulk_kernel<DH, GG><<<grid, 128, smem_, st>>>(s, L, state, gm,                      \
-                                                                      (const __nv_bfloat16 *)q_t, err);     \
+            decode_attn_bulk_kernel<DH, GG><<<grid, 128, smem_, st>>>(                                      \
+                s, L, state, gm, (const __nv_bfloat16 *)q_t, (const __nv_bfloat16 *)k_t,                    \
+                (const __nv_bfloat16 *)v_t, err);                                                           \
         } else {                                                                                            \
             decode_attn_mma_kernel<DH, GG><<<grid, 128, 0, st>>>(s, L, state, gm, (const __nv_bfloat16 *)q_t); \
         }                                                                                                   \
