@@ -225,6 +225,8 @@ struct LinTile {
     // dY [64][LDF], coef [64], D [64]
     static constexpr int WBUF = DH * LDF > DF * LDH ? DH * LDF : DF * LDH;
     static constexpr int POST_FLOATS = 64 * LDH + WBUF + DF * kLd64 + 64 * LDF + 128;
+    // sums: q rows [64][LDH], dY rows [64][LDF], dO rows [64][LDH], a rows [64][LDF], D [64]
+    static constexpr int SUMS_FLOATS = 2 * 64 * LDH + 2 * 64 * LDF + 64;
     // key: KT [DH][68] (K^T, V^T, K^T), Wk / R / R^T / Wk^T / K rows, Y [64][LDF] (Y_k, phi(k), dY),
     // PT [DF][68] (phi(k)^T, dphi rows, dY^T), coef [64], kept mask [64]
     static constexpr int RBUF = WBUF;
@@ -423,6 +425,66 @@ __global__ void __launch_bounds__(kTileThreads, LinTile<DH, DF>::MIN_BLOCKS) bwd
     }
 }
 
+// The query side's sums once the dq kernel has formed dY and a (its epilogue): dWq += q^T dY and the
+// key side's chunk sums R_t += a^T dO, r_t += a^T D over the tile's 64 rows (atomics).
+template <typename T, int DH, int DF>
+__global__ void __launch_bounds__(kTileThreads, LinTile<DH, DF>::MIN_BLOCKS) bwd_lin_sums_tile(
+    Dims s, const T *__restrict__ q, const T *__restrict__ dO, const float *__restrict__ Dv,
+    const float *__restrict__ A, const float *__restrict__ dY, float *__restrict__ dWq, float *__restrict__ R,
+    float *__restrict__ rr) {
+    using Cfg = LinTile<DH, DF>;
+    extern __shared__ __align__(16) float sm[];
+    float *Xr = sm, *Yr = Xr + 64 * Cfg::LDH, *Go = Yr + 64 * Cfg::LDF, *Ar = Go + 64 * Cfg::LDH,
+          *Ds = Ar + 64 * Cfg::LDF;
+    const int ntile = (s.N + 63) / 64;
+    const int bh = blockIdx.x / ntile, i0 = (blockIdx.x % ntile) * 64;
+    const int h = bh % s.H, b = bh / s.H, bg = b * s.Hkv + h / s.G();
+    const int t = i0 / s.C;
+    const int valid = min(64, s.N - i0);
+    const size_t row0 = (size_t)bh * s.N + i0;
+    const size_t tslot = (size_t)bg * (s.T() + 1) + t;
+    load_rows<64, DH>(Xr, Cfg::LDH, q + row0 * DH, DH, valid);
+    load_rows<64, DF>(Yr, Cfg::LDF, dY + row0 * DF, DF, valid);
+    load_rows<64, DH>(Go, Cfg::LDH, dO + row0 * DH, DH, valid);
+    load_rows<64, DF>(Ar, Cfg::LDF, A + row0 * DF, DF, valid);
+    if (threadIdx.x < 64) Ds[threadIdx.x] = (int)threadIdx.x < valid ? Dv[row0 + threadIdx.x] : 0.f;
+    __syncthreads();
+    const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
+    {
+        float acc[DH / 64][DF / 64][4][4];
+        zero_acc(acc);
+        smem_mm<DH / 64, DF / 64>(Xr, Cfg::LDH, Yr, Cfg::LDF, 64, acc);
+        float *dW = dWq + (size_t)h * DH * DF;
+#pragma unroll
+        for (int mu = 0; mu < DH / 64; ++mu)
+#pragma unroll
+            for (int nu = 0; nu < DF / 64; ++nu)
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    atomicAdd(reinterpret_cast<float4 *>(dW + (size_t)(ty * 4 + 64 * mu + i) * DF + tx * 4 + 64 * nu),
+                              make_float4(acc[mu][nu][i][0], acc[mu][nu][i][1], acc[mu][nu][i][2], acc[mu][nu][i][3]));
+    }
+    {
+        float acc[DF / 64][DH / 64][4][4];
+        zero_acc(acc);
+        smem_mm<DF / 64, DH / 64>(Ar, Cfg::LDF, Go, Cfg::LDH, 64, acc);
+        float *Rt = R + tslot * DF * DH;
+#pragma unroll
+        for (int mu = 0; mu < DF / 64; ++mu)
+#pragma unroll
+            for (int nu = 0; nu < DH / 64; ++nu)
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    atomicAdd(reinterpret_cast<float4 *>(Rt + (size_t)(ty * 4 + 64 * mu + i) * DH + tx * 4 + 64 * nu),
+                              make_float4(acc[mu][nu][i][0], acc[mu][nu][i][1], acc[mu][nu][i][2], acc[mu][nu][i][3]));
+        if (threadIdx.x < DF) {
+            float racc = 0.f;
+            for (int r = 0; r < 64; ++r) racc = fmaf(Ar[r * Cfg::LDF + threadIdx.x], Ds[r], racc);
+            atomicAdd(rr + tslot * DF + threadIdx.x, racc);
+        }
+    }
+}
+
 // Unselected keys of 64-key tiles of decided chunks: phi(k) from K Wk, dv += phi(k) R,
 // dphi(k) = V R^T - r, the NP-Map backward from phi(k): dk += dy Wk^T + coef k, dWk += k^T dy.
 template <typename T, int DH, int DF>
@@ -592,16 +654,24 @@ cudaError_t launch_lin_cfg(int which, const Dims &s, const void *q, const void *
             s, (const T *)q, (const T *)Wq, w.S, w.z, (const T *)dO, w.A, w.dYq, w.Ms, w.iZ);
         return cudaGetLastError();
     }
-    // which == 1: query side after the softmax pass (with the chunk sums), their suffix, the key side
+    // which == 1: query side after the softmax pass (with the chunk sums), their suffix, the key side;
+    // which == 2: the same when the dq kernel has already formed dq, dY and a
     const int T_ = s.T();
     const size_t BK = (size_t)s.B * s.Hkv;
     if ((e = cudaMemsetAsync(dWq, 0, sizeof(float) * (size_t)s.H * DH * DF, st)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(dWk, 0, sizeof(float) * (size_t)s.Hkv * DH * DF, st)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(w.R, 0, sizeof(float) * BK * (T_ + 1) * DF * DH, st)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(w.r, 0, sizeof(float) * BK * (T_ + 1) * DF, st)) != cudaSuccess) return e;
-    if ((e = prep((const void *)bwd_lin_post_tile<T, DH, DF>, Cfg::POST_FLOATS)) != cudaSuccess) return e;
-    bwd_lin_post_tile<T, DH, DF><<<qgrid, kTileThreads, Cfg::POST_FLOATS * 4, st>>>(
-        s, (const T *)q, (const T *)Wq, (const T *)dO, w.z, w.L, w.Dv, w.A, w.dYq, dq, dWq, w.R, w.r);
+    if (which == 2) {
+        // the dq kernel has formed dY and a (and dq): only the sums remain on the query side
+        if ((e = prep((const void *)bwd_lin_sums_tile<T, DH, DF>, Cfg::SUMS_FLOATS)) != cudaSuccess) return e;
+        bwd_lin_sums_tile<T, DH, DF><<<qgrid, kTileThreads, Cfg::SUMS_FLOATS * 4, st>>>(
+            s, (const T *)q, (const T *)dO, w.Dv, w.A, w.dYq, dWq, w.R, w.r);
+    } else {
+        if ((e = prep((const void *)bwd_lin_post_tile<T, DH, DF>, Cfg::POST_FLOATS)) != cudaSuccess) return e;
+        bwd_lin_post_tile<T, DH, DF><<<qgrid, kTileThreads, Cfg::POST_FLOATS * 4, st>>>(
+            s, (const T *)q, (const T *)Wq, (const T *)dO, w.z, w.L, w.Dv, w.A, w.dYq, dq, dWq, w.R, w.r);
+    }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = launch_bwd_suffix(s, w.R, w.r, st)) != cudaSuccess) return e;
     if (T_ > 0) {
@@ -635,7 +705,8 @@ bool tiled_linear_backward_supported(const Dims &s) {
 }
 
 // which = 0: the linear pre-pass (Phi, SG, lden, dl); which = 1: everything of the linear branch that
-// follows the softmax pass (dq, dWq, R_t, r_t, their suffix sums, dk, dv, dWk of the unselected keys).
+// follows the softmax pass (dq, dWq, R_t, r_t, their suffix sums, dk, dv, dWk of the unselected keys);
+// which = 2: as 1 after a dq kernel with the linear prologue and epilogue (dq, dY and a formed there).
 cudaError_t launch_linear_backward_tiled(int which, const Dims &s, const void *q, const void *k, const void *v,
                                          const void *Wq, const void *Wk, const void *dO, const int32_t *idx,
                                          const BackwardScratch &w, float *dq, float *dk, float *dv, float *dWq,

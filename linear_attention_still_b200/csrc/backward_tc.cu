@@ -46,7 +46,8 @@ struct BwdParams {
     float scale, scale_log2;  // tau, tau log2(e)
     const float *lden, *dl;   // [B,H,N] from the linear pre-pass (dq kernel without its own prologue)
     const float *z;           // [B*Hkv*(T+1), D] z_t (dq kernel prologue)
-    float *Phi, *SG;          // [B,H,N,D] phi(q) and S_t dO (fp32), written by the dq kernel prologue
+    float *Phi, *SG;          // [B,H,N,D] phi(q) and S_t dO (fp32), written by the dq kernel prologue; its
+                              // epilogue then replaces them with a = 2^-L phi(q) and dY = dL/d(q Wq)
     float *L, *Dv;            // [B,H,N] log2 normaliser and D_i (dq kernel writes, key kernel reads)
     float *dq, *dk, *dv;      // fp32 gradients
     const int32_t *idx;       // [B,Hkv,T,k] (kept keys)
@@ -79,14 +80,15 @@ struct BwdQCfg {
     // of sweep-2 tile n (two barriers taking turns, so neither runs two phases ahead of its waiter)
     // prologue: B_WFULL (Wq^T, S_t^T tiles), B_Y (Y done), B_PHI (phi(q) written, warpgroup 0),
     // B_LIN (lin and sg done), B_PRO (warpgroup 0 has read them)
+    // epilogue (with the prologue): B_W2FULL (the Wq tile), B_DY (dY / tau written, both warpgroups)
     static constexpr int B_QFULL = 0, B_S = 1, B_SDONE = 2, B_DQ = 3, B_DRAIN = 4, B_WG = 5, B_DSFULL = 6,
-                         B_WFULL = 8, B_Y = 9, B_PHI = 10, B_LIN = 11, B_PRO = 12, B_KFULL = 13, B_VFULL = 13 + NS,
-                         B_KVEMPTY = 13 + 2 * NS, NUM_BARS = 13 + 3 * NS;
+                         B_WFULL = 8, B_Y = 9, B_PHI = 10, B_LIN = 11, B_PRO = 12, B_W2FULL = 13, B_DY = 14,
+                         B_KFULL = 15, B_VFULL = 15 + NS, B_KVEMPTY = 15 + 2 * NS, NUM_BARS = 15 + 3 * NS;
     static constexpr int TMEM_SLOT_OFF = 8 * NUM_BARS, ABORT_OFF = TMEM_SLOT_OFF + 8, BAR_BYTES = 256;
     static_assert(ABORT_OFF + 8 <= BAR_BYTES, "barrier area overflow");
     static constexpr int OFF_XCH = OFF_BAR + BAR_BYTES;   // [2][128][3] row statistics of each half
-    static constexpr int OFF_LXC = OFF_XCH + 2 * 128 * 3 * 4;  // [128][2] lden, dl (prologue, for warpgroup 1)
-    static constexpr int SMEM = OFF_LXC + 128 * 2 * 4 + 1024;
+    static constexpr int OFF_LXC = OFF_XCH + 2 * 128 * 3 * 4;  // [128][3] lden, dl, ||q||^2 (prologue, for warpgroup 1)
+    static constexpr int SMEM = OFF_LXC + 128 * 3 * 4 + 1024;
     // Two warpgroups of row warps: warpgroup x takes key columns [32x, 32x + 32) of every tile.
     static constexpr int THREADS = 320, PRODUCER_WARP = 8, MMA_WARP = 9, ROW_THREADS = 256;
     // S (64 keys), dP (64 keys), dQ (DH), dS of alternate tiles (bf16, 64 keys = 32 columns each);
@@ -104,7 +106,7 @@ __global__ void __launch_bounds__(BwdQCfg<DH, DF>::THREADS, BwdQCfg<DH, DF>::MIN
                      const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
                      const __grid_constant__ CUtensorMap map_kh, const __grid_constant__ CUtensorMap map_vh,
                      const __grid_constant__ CUtensorMap map_wq, const __grid_constant__ CUtensorMap map_st,
-                     const BwdParams p) {
+                     const __grid_constant__ CUtensorMap map_w, const BwdParams p) {
     using Cfg = BwdQCfg<DH, DF>;
     constexpr bool PRO = Cfg::PRO;
     extern __shared__ uint8_t smem_raw[];
@@ -134,7 +136,8 @@ __global__ void __launch_bounds__(BwdQCfg<DH, DF>::THREADS, BwdQCfg<DH, DF>::MIN
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < Cfg::NUM_BARS; ++i)
-            mbar_init(BAR(i), i == Cfg::B_SDONE || i == Cfg::B_WG || i == Cfg::B_DSFULL || i == Cfg::B_DSFULL + 1
+            mbar_init(BAR(i), i == Cfg::B_SDONE || i == Cfg::B_WG || i == Cfg::B_DSFULL || i == Cfg::B_DSFULL + 1 ||
+                                      i == Cfg::B_DY
                                   ? Cfg::ROW_THREADS
                                   : (i == Cfg::B_PHI || i == Cfg::B_PRO) ? 128 : 1);
         *abort_flag = 0;
@@ -183,11 +186,20 @@ __global__ void __launch_bounds__(BwdQCfg<DH, DF>::THREADS, BwdQCfg<DH, DF>::MIN
                 tma_load_3d_w(sV + rr * Cfg::K_REG, mv, BAR(Cfg::B_VFULL + s), rr * 64, row, bg);
             issued = jj + 1;
         }
+        bool w2 = false;
+        if (PRO && ok && (ok = mbar_wait_w(BAR(Cfg::B_PRO), 0, abort_flag))) {
+            // Wq [DH rows x DF] for dq += dY Wq^T, over the Wq^T tile the prologue has finished with
+            mbar_arrive_expect_tx_w(BAR(Cfg::B_W2FULL), Cfg::WQ_BYTES);
+            for (int rr = 0; rr < DF / 64; ++rr)
+                tma_load_3d_w(sbase + Cfg::OFF_WQ + rr * (DH * 128), &map_w, BAR(Cfg::B_W2FULL), rr * 64, 0, h);
+            w2 = true;
+        }
         if (!ok) {
             *abort_flag = 1;
             if (lane == 0) report(p.err, DEV_ERR_TIMEOUT);
             mbar_wait_drain(BAR(Cfg::B_QFULL), 0, 100000000ull);
             if (PRO) mbar_wait_drain(BAR(Cfg::B_WFULL), 0, 100000000ull);
+            if (w2) mbar_wait_drain(BAR(Cfg::B_W2FULL), 0, 100000000ull);
             for (int jj = max(0, issued - Cfg::NS); jj < issued; ++jj) {
                 mbar_wait_drain(BAR(Cfg::B_KFULL + jj % Cfg::NS), (jj / Cfg::NS) & 1, 100000000ull);
                 mbar_wait_drain(BAR(Cfg::B_VFULL + jj % Cfg::NS), (jj / Cfg::NS) & 1, 100000000ull);
@@ -267,7 +279,16 @@ __global__ void __launch_bounds__(BwdQCfg<DH, DF>::THREADS, BwdQCfg<DH, DF>::MIN
         if (ok && (ok = mbar_wait_w(BAR(Cfg::B_DSFULL + ((nt - 1) & 1)), ((nt - 1) >> 1) & 1, abort_flag))) {
             tc_fence_after();
             issue_dq(ntot - 1);
-            mma_commit_w(BAR(Cfg::B_DQ));
+            if (PRO && (ok = mbar_wait_w(BAR(Cfg::B_W2FULL), 0, abort_flag) && mbar_wait_w(BAR(Cfg::B_DY), 0, abort_flag))) {
+                // dQ += (dY / tau) Wq^T: dY (bf16, DF features = DF/2 columns) from TMEM over S, Wq rows of DF
+                constexpr uint32_t ID_W = idesc_bf16(128, DH, 0, 0);
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < DF / 16; ++kk)
+                    mma_ts_w(tm + Cfg::DQ_COL, tm + Cfg::S_COL + kk * 8, kmajor_desc(sbase + Cfg::OFF_WQ, kk, DH * 128), ID_W,
+                             1u);
+            }
+            if (ok) mma_commit_w(BAR(Cfg::B_DQ));
         }
         if (!ok) {
             *abort_flag = 1;
@@ -287,7 +308,7 @@ __global__ void __launch_bounds__(BwdQCfg<DH, DF>::THREADS, BwdQCfg<DH, DF>::MIN
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const uint32_t tS = tmem + lane_off + Cfg::S_COL + 32 * x, tDP = tmem + lane_off + Cfg::DP_COL + 32 * x,
                        tDS = tmem + lane_off + Cfg::DS_COL + 16 * x;
-        float lden = 0.f, dl = 0.f;
+        float lden = 0.f, dl = 0.f, qn2 = 0.f;  // qn2 = ||q||^2 = ||phi(q)||^2 (prologue)
         bool ok = true;
         if constexpr (!PRO) {
             lden = live ? p.lden[row] : 0.f;
@@ -336,6 +357,7 @@ __global__ void __launch_bounds__(BwdQCfg<DH, DF>::THREADS, BwdQCfg<DH, DF>::MIN
                     }
                 }
                 const float fscale = sqrtf(qq) * rsqrtf(ee);
+                qn2 = qq;
                 const float *zt = p.z + (size_t)tslot * DF;
                 float *phig = p.Phi + row * DF;
 #pragma unroll
@@ -405,8 +427,9 @@ __global__ void __launch_bounds__(BwdQCfg<DH, DF>::THREADS, BwdQCfg<DH, DF>::MIN
                 }
             }
             float *lx = reinterpret_cast<float *>(smem + Cfg::OFF_LXC);
-            lx[2 * r] = lden;
-            lx[2 * r + 1] = dl;
+            lx[3 * r] = lden;
+            lx[3 * r + 1] = dl;
+            lx[3 * r + 2] = qn2;
             tc_fence_before();
             mbar_arrive(BAR(Cfg::B_PRO));
         }
@@ -478,8 +501,9 @@ __global__ void __launch_bounds__(BwdQCfg<DH, DF>::THREADS, BwdQCfg<DH, DF>::MIN
                                 uo = xch[((x ^ 1) * 128 + r) * 3 + 2];
                     if (PRO && x == 1) {  // the prologue's linear terms of this row (warpgroup 0)
                         const float *lx = reinterpret_cast<const float *>(smem + Cfg::OFF_LXC);
-                        lden = lx[2 * r];
-                        dl = lx[2 * r + 1];
+                        lden = lx[3 * r];
+                        dl = lx[3 * r + 1];
+                        qn2 = lx[3 * r + 2];
                     }
                     const float Mc = fmaxf(M, Mo);
                     const float f0 = M == -INFINITY ? 0.f : ex2(M - Mc), f1 = Mo == -INFINITY ? 0.f : ex2(Mo - Mc);
@@ -525,7 +549,49 @@ __global__ void __launch_bounds__(BwdQCfg<DH, DF>::THREADS, BwdQCfg<DH, DF>::MIN
                 mbar_arrive(BAR(Cfg::B_DSFULL + ((jj - nt) & 1)));
             }
         }
-        // ---- epilogue: dq = tau dQ (fp32); warpgroup x writes columns [x DH/2, (x + 1) DH/2)
+        float kappa = 0.f;  // with the prologue: the x-coefficient of the NP-Map backward, dL/dq += kappa q
+        if constexpr (PRO) {
+            // ---- the linear branch's query side (warpgroup x: features [x DF/2, (x + 1) DF/2) of the row):
+            // dphi = 2^-L (S_t dO - D z_t); NP-Map backward from phi itself: with kappa = <phi, dphi> / |phi|^2,
+            // dY = phi (dphi - kappa phi) and dL/dq = dY Wq^T + kappa q (the f.df term vanishes: df is
+            // orthogonal to f).  Both sums are known: |phi|^2 = |q|^2 and <phi, dphi> = 2^-L (<phi, S_t dO>
+            // - D <phi, z_t>) = 2^-L (dl - D lden).  a = 2^-L phi and dY replace phi and S_t dO in memory.
+            constexpr int HF = DF / 2;
+            const float cl = ex2(-Lr);
+            const float *zt = p.z + (size_t)tslot * DF + x * HF;
+            float *phg = p.Phi + row * DF + x * HF, *sgg = p.SG + row * DF + x * HF;
+            kappa = qn2 > 0.f ? cl * (dl - Di * lden) / qn2 : 0.f;
+            const float itau = 1.f / p.scale;
+            const uint32_t tDY = tmem + lane_off + Cfg::S_COL + x * (HF / 2);
+#pragma unroll
+            for (int c = 0; c < HF / 32; ++c) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int a4 = 0; a4 < 8; ++a4) {
+                    float4 ph = make_float4(0.f, 0.f, 0.f, 0.f), dy = ph;
+                    if (ok && live) {
+                        ph = reinterpret_cast<const float4 *>(phg)[8 * c + a4];
+                        const float4 sg = reinterpret_cast<const float4 *>(sgg)[8 * c + a4];
+                        const float4 zz = __ldg(reinterpret_cast<const float4 *>(zt) + 8 * c + a4);
+                        dy.x = ph.x * (cl * (sg.x - Di * zz.x) - kappa * ph.x);
+                        dy.y = ph.y * (cl * (sg.y - Di * zz.y) - kappa * ph.y);
+                        dy.z = ph.z * (cl * (sg.z - Di * zz.z) - kappa * ph.z);
+                        dy.w = ph.w * (cl * (sg.w - Di * zz.w) - kappa * ph.w);
+                        reinterpret_cast<float4 *>(phg)[8 * c + a4] = make_float4(cl * ph.x, cl * ph.y, cl * ph.z, cl * ph.w);
+                        reinterpret_cast<float4 *>(sgg)[8 * c + a4] = dy;
+                    }
+                    pk[2 * a4] = pack_bf16x2(dy.x * itau, dy.y * itau);
+                    pk[2 * a4 + 1] = pack_bf16x2(dy.z * itau, dy.w * itau);
+                }
+                // dY / tau (bf16) of features x HF + 32c.. into columns [x HF/2 + 16c, +16) over S (free:
+                // every tile's S has been read)
+                tmem_st16(tDY + 16 * c, pk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(BAR(Cfg::B_DY));
+        }
+        // ---- epilogue: dq = tau dQ (+ kappa q) (fp32); warpgroup x writes columns [x DH/2, (x + 1) DH/2)
         ok = warp_all(ok && mbar_wait(BAR(Cfg::B_DQ), 0, abort_flag));
         if (ok) {
             tc_fence_after();
@@ -536,12 +602,31 @@ __global__ void __launch_bounds__(BwdQCfg<DH, DF>::THREADS, BwdQCfg<DH, DF>::MIN
                 tmem_ld32(tmem + lane_off + Cfg::DQ_COL + col, w);
                 tmem_wait_ld();
                 if (live) {
+                    float qv[32];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) qv[e] = 0.f;
+                    if (PRO) {  // q of columns col.. from the swizzled Q tile
+#pragma unroll
+                        for (int ch = 0; ch < 4; ++ch) {
+                            const int chunk = ((col & 63) >> 3) + ch;
+                            const uint4 w4 = *reinterpret_cast<const uint4 *>(smem + Cfg::OFF_Q + (col >> 6) * Cfg::Q_REG +
+                                                                              r * 128 + ((chunk ^ (r & 7)) << 4));
+                            const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&w4);
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 f2 = __bfloat1622float2(h2[e]);
+                                qv[ch * 8 + 2 * e] = f2.x;
+                                qv[ch * 8 + 2 * e + 1] = f2.y;
+                            }
+                        }
+                    }
                     float4 *dst = reinterpret_cast<float4 *>(p.dq + row * DH + col);
 #pragma unroll
                     for (int v4 = 0; v4 < 8; ++v4)
-                        dst[v4] = make_float4(__uint_as_float(w[4 * v4]) * p.scale, __uint_as_float(w[4 * v4 + 1]) * p.scale,
-                                              __uint_as_float(w[4 * v4 + 2]) * p.scale,
-                                              __uint_as_float(w[4 * v4 + 3]) * p.scale);
+                        dst[v4] = make_float4(fmaf(__uint_as_float(w[4 * v4]), p.scale, kappa * qv[4 * v4]),
+                                              fmaf(__uint_as_float(w[4 * v4 + 1]), p.scale, kappa * qv[4 * v4 + 1]),
+                                              fmaf(__uint_as_float(w[4 * v4 + 2]), p.scale, kappa * qv[4 * v4 + 2]),
+                                              fmaf(__uint_as_float(w[4 * v4 + 3]), p.scale, kappa * qv[4 * v4 + 3]));
                 }
             }
         }
@@ -858,24 +943,25 @@ __global__ void __launch_bounds__(BwdKVCfg<DH>::THREADS, 1)
 
 // The dq kernel with its own linear prologue (DF = D) or with the pre-pass's terms (DF = 0).
 template <int DH, int DF>
-cudaError_t launch_dq(const Dims &s, const CUtensorMap *maps, const void *wqt, const void *st_t, const BwdParams &prm,
-                      cudaStream_t st) {
+cudaError_t launch_dq(const Dims &s, const CUtensorMap *maps, const void *wqt, const void *st_t, const void *Wq,
+                      const BwdParams &prm, cudaStream_t st) {
     using Cfg = BwdQCfg<DH, DF>;
-    CUtensorMap mwq = maps[0], mst = maps[0];
+    CUtensorMap mwq = maps[0], mst = maps[0], mw = maps[0];
     if (DF > 0 && (!make_map(&mwq, wqt, DH, DF, s.H, DF) ||
-                   !make_map(&mst, st_t, DF, DH, (uint64_t)s.B * s.Hkv * (s.T() + 1), DH)))
+                   !make_map(&mst, st_t, DF, DH, (uint64_t)s.B * s.Hkv * (s.T() + 1), DH) ||
+                   !make_map(&mw, Wq, DF, DH, s.H, DH)))
         return cudaErrorInvalidValue;
     auto kern = bwd_dq_tc_kernel<DH, DF>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
     if (e != cudaSuccess) return e;
     kern<<<(unsigned)(prm.n_qtiles * (uint64_t)s.B * s.H), Cfg::THREADS, Cfg::SMEM, st>>>(
-        maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], mwq, mst, prm);
+        maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], mwq, mst, mw, prm);
     return cudaGetLastError();
 }
 
 template <int DH>
 cudaError_t launch_bwd_cfg(const Dims &s, const void *q, const void *k, const void *v, const void *khat,
-                           const void *vhat, const void *dO, const void *wqt, const void *st_t,
+                           const void *vhat, const void *dO, const void *wqt, const void *st_t, const void *Wq,
                            const BwdParams &prm_in, cudaStream_t st, int *launches) {
     const int T = s.T();
     const uint64_t BH = (uint64_t)s.B * s.H, BK = (uint64_t)s.B * s.Hkv;
@@ -896,9 +982,9 @@ cudaError_t launch_bwd_cfg(const Dims &s, const void *q, const void *k, const vo
         const CUtensorMap maps[6] = {mq128, mdo128, mk64, mv64, mkh64, mvh64};
         const int ts = timing_begin(kTimeBwdDq, st);
         cudaError_t e;
-        if (!wqt) e = launch_dq<DH, 0>(s, maps, nullptr, nullptr, prm, st);
-        else if (s.D == 64) e = launch_dq<DH, 64>(s, maps, wqt, st_t, prm, st);
-        else if (s.D == 128) e = launch_dq<DH, 128>(s, maps, wqt, st_t, prm, st);
+        if (!wqt) e = launch_dq<DH, 0>(s, maps, nullptr, nullptr, nullptr, prm, st);
+        else if (s.D == 64) e = launch_dq<DH, 64>(s, maps, wqt, st_t, Wq, prm, st);
+        else if (s.D == 128) e = launch_dq<DH, 128>(s, maps, wqt, st_t, Wq, prm, st);
         else e = cudaErrorNotSupported;
         timing_end(ts, st);
         if (e != cudaSuccess) return e;
@@ -981,8 +1067,9 @@ cudaError_t launch_backward_tc(const Dims &s, const void *q, const void *k, cons
     prm.dv = dv;
     prm.idx = idx;
     prm.err = err;
-    if (s.d == 64) return launch_bwd_cfg<64>(s, q, k, v, khat, vhat, dO, pro.wqt, pro.st_t, prm, st, launches);
-    if (s.d == 128) return launch_bwd_cfg<128>(s, q, k, v, khat, vhat, dO, pro.wqt, pro.st_t, prm, st, launches);
+    if (s.d == 64) return launch_bwd_cfg<64>(s, q, k, v, khat, vhat, dO, pro.wqt, pro.st_t, pro.Wq, prm, st, launches);
+    if (s.d == 128)
+        return launch_bwd_cfg<128>(s, q, k, v, khat, vhat, dO, pro.wqt, pro.st_t, pro.Wq, prm, st, launches);
     return cudaErrorNotSupported;
 }
 

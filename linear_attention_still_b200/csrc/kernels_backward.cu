@@ -844,7 +844,7 @@ cudaError_t backward_t(const Dims &s, const void *q, const void *k, const void *
         }
         // tiled linear branch with the tensor-core linear state: the dq kernel forms the rows' linear
         // terms itself (its prologue writes phi(q) and S_t dO for the later linear kernels)
-        BwdPrologue pro{nullptr, nullptr, w.z, w.A, w.dYq};
+        BwdPrologue pro{nullptr, Wq, nullptr, w.z, w.A, w.dYq};
         if (tiled && tiled_state) {
             pro.wqt = w.wqt;
             pro.st_t = w.st_t;
@@ -862,9 +862,10 @@ cudaError_t backward_t(const Dims &s, const void *q, const void *k, const void *
                                launches);
         if (e != cudaSuccess) return e;
         if (tiled) {
-            // query side (dq, dWq), chunk sums, suffix, key side (dk, dv, dWk) of the linear branch
+            // query side (dq, dWq), chunk sums, suffix, key side (dk, dv, dWk) of the linear branch (the
+            // dq kernel with the prologue has formed dq, dY and a itself)
             const int ts = timing_begin(kTimeBwdLinear, st);
-            e = launch_linear_backward_tiled(1, s, q, k, v, Wq, Wk, dO, idx, w, dq, dk, dv, dWq, dWk, st);
+            e = launch_linear_backward_tiled(pro.wqt ? 2 : 1, s, q, k, v, Wq, Wk, dO, idx, w, dq, dk, dv, dWq, dWk, st);
             timing_end(ts, st);
             if (e != cudaSuccess) return e;
             *launches += T_ > 0 ? 3 : 2;

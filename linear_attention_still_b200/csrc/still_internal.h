@@ -95,9 +95,10 @@ cudaError_t launch_gather(const Dims &s, const int32_t *idx, const void *k, cons
 // Inputs of the dq kernel's own linear prologue (wqt = nullptr: none; lden, dl are read instead).
 struct BwdPrologue {
     const void *wqt;    // [H,D,d] Wq^T (bf16)
+    const void *Wq;     // [H,d,D] Wq (bf16): its epilogue adds dY Wq^T to dq
     const void *st_t;   // [B,Hkv,T+1,d,D] S_t^T (bf16)
     const float *z;     // [B,Hkv,T+1,D]
-    float *Phi, *SG;    // [B,H,N,D] out: phi(q), S_t dO
+    float *Phi, *SG;    // [B,H,N,D] out: a = 2^-L phi(q) and dY = dL/d(q Wq) (phi(q), S_t dO on the way)
 };
 cudaError_t launch_backward_tc(const Dims &s, const void *q, const void *k, const void *v, const void *khat,
                                const void *vhat, const int32_t *idx, const void *dO, const float *lden,
