@@ -100,7 +100,7 @@ def test_step_entry_points_reject(lib):
 def test_backward_rejects(lib):
     f = lib._lib.still_hybrid_backward
     d0 = _dims(lib, w=0, k=0)
-    assert f(ct.byref(d0), *([FAKE] * 13), 1 << 40, None) == 2          # no window: not covered
+    assert lib.still_backward_workspace_bytes(d0) > 0                    # no window: covered (sized, no call)
     d = _dims(lib)
     need = lib.still_backward_workspace_bytes(d)
     assert need > 0
