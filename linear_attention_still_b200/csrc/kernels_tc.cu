@@ -87,7 +87,14 @@ struct MergeParams {
 // 2 packed with the last 32-key chunk of each row on the FMA-pipe exp2, 3 with every other 32-key
 // chunk there.  Measured on B200 with concurrent softmax warpgroups (1B 16K / 8B B4 16K layers, the
 // two merge phases, ms): variant 1 0.612/3.629, 2 0.608/3.646, 3 0.641/3.799 -> variant 1 is built.
-constexpr int kMergeExpVariant = 1;
+#ifndef STILL_MERGE_EXP
+#define STILL_MERGE_EXP 1
+#endif
+constexpr int kMergeExpVariant = STILL_MERGE_EXP;
+// Every wait of this kernel sleeps in mbarrier.try_wait instead of spinning (fewer issue slots and
+// shared-memory tests taken from the softmax warps).  Measured on B200 (8B B4 16K layer, both phases):
+// 3.24 -> 3.13 ms per step; the head-dim-64 ring kernel measured 0.489 -> 0.496 ms and keeps spinning.
+constexpr bool kMergeSuspend = true;
 // MODE kMergeLocal: keys = the window [max(0,(t-m)C), i]; also the Self-Saliency Score of every row
 //   ([p1] "Self-Saliency Score"): the band keys [i-w+1, i-1] are window keys, so the band's
 //   log-sum-exp is accumulated from the same exponentials (masked adds on the two partial tiles),
@@ -203,12 +210,12 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
                 for (int rr = 0; rr < DF / 64; ++rr)
                     tma_load_3d_w(sStage + HP * Cfg::WQ_BYTES + rr * (DH * 128), &map_st, BAR(B_WFULL), rr * 64, 0,
                                 tslot);
-                ok = mbar_wait_w(BAR(B_PRO), 0, abort_flag);  // prologue operands consumed
+                ok = mbar_wait_wt<kMergeSuspend>(BAR(B_PRO), 0, abort_flag);  // prologue operands consumed
             }
             for (int j = 0; ok && j < n_tiles; ++j) {
                 const int s = j % Cfg::NS;
                 if (j >= Cfg::NS) {
-                    ok = mbar_wait_w(BAR(B_KVEMPTY + s), ((j / Cfg::NS) - 1) & 1, abort_flag);
+                    ok = mbar_wait_wt<kMergeSuspend>(BAR(B_KVEMPTY + s), ((j / Cfg::NS) - 1) & 1, abort_flag);
                     if (!ok) break;
                 }
                 const uint32_t sK = sStage + s * Cfg::STAGE_BYTES, sV = sK + Cfg::TILE_BYTES;
@@ -244,7 +251,7 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
             constexpr uint32_t ID_LIN = idesc_bf16(128, DH, 0, 0);
             constexpr uint32_t ID_S = idesc_bf16(128, 128, 0, 0);
             constexpr uint32_t ID_PV = idesc_bf16(128, DH, 0, 1);
-            bool ok = mbar_wait_w(BAR(B_QFULL), 0, abort_flag) && (LOCAL || mbar_wait_w(BAR(B_WFULL), 0, abort_flag));
+            bool ok = mbar_wait_wt<kMergeSuspend>(BAR(B_QFULL), 0, abort_flag) && (LOCAL || mbar_wait_wt<kMergeSuspend>(BAR(B_WFULL), 0, abort_flag));
             if (ok && !LOCAL) {
                 tc_fence_after();
                 for (int x = 0; x < HP; ++x) {
@@ -255,7 +262,7 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
                     mma_commit_w(BAR(B_Y + x));
                 }
                 for (int x = 0; x < HP && ok; ++x) {
-                    ok = mbar_wait_w(BAR(B_PHI + x), 0, abort_flag);
+                    ok = mbar_wait_wt<kMergeSuspend>(BAR(B_PHI + x), 0, abort_flag);
                     if (!ok) break;
                     tc_fence_after();
                     const uint32_t bs = sStage + HP * Cfg::WQ_BYTES;
@@ -280,7 +287,7 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
                 mma_commit_w(BAR(B_S + x));
             };
             // first score tiles
-            if (ok && n_tiles > 0) ok = mbar_wait_w(BAR(B_KFULL + 0), 0, abort_flag);
+            if (ok && n_tiles > 0) ok = mbar_wait_wt<kMergeSuspend>(BAR(B_KFULL + 0), 0, abort_flag);
             if (ok && n_tiles > 0) {
                 tc_fence_after();
                 for (int x = 0; x < HP; ++x) issue_s(x, sStage);
@@ -293,8 +300,8 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
                 const int s1 = (j + 1) % Cfg::NS;
                 const uint32_t sK1 = sStage + s1 * Cfg::STAGE_BYTES;
                 for (int x = 0; x < HP && ok; ++x) {
-                    if (x == 0) ok = mbar_wait_w(BAR(B_VFULL + s), (j / Cfg::NS) & 1, abort_flag);
-                    if (ok) ok = mbar_wait_w(BAR(B_P + x), j & 1, abort_flag);
+                    if (x == 0) ok = mbar_wait_wt<kMergeSuspend>(BAR(B_VFULL + s), (j / Cfg::NS) & 1, abort_flag);
+                    if (ok) ok = mbar_wait_wt<kMergeSuspend>(BAR(B_P + x), j & 1, abort_flag);
                     if (!ok) break;
                     tc_fence_after();
 #pragma unroll
@@ -304,7 +311,7 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
                     mma_commit_w(BAR(B_O + x));
                     if (j + 1 < n_tiles) {
                         // P_x(j) lives over S_x: the next scores wait for PV_x(j) (in-order issue)
-                        if (x == 0) ok = mbar_wait_w(BAR(B_KFULL + s1), ((j + 1) / Cfg::NS) & 1, abort_flag);
+                        if (x == 0) ok = mbar_wait_wt<kMergeSuspend>(BAR(B_KFULL + s1), ((j + 1) / Cfg::NS) & 1, abort_flag);
                         if (!ok) break;
                         tc_fence_after();
                         issue_s(x, sK1);
@@ -346,7 +353,7 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
                 for (int v = 0; v < DH * 2; v += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(p.o + row * DH + v / 2));
             }
             // ---- prologue: phi(q) from Y = Q Wq^T
-            ok = warp_all(mbar_wait(BAR(B_QFULL), 0, abort_flag) && mbar_wait(BAR(B_Y + x), 0, abort_flag));
+            ok = warp_all(mbar_wait_t<kMergeSuspend>(BAR(B_QFULL), 0, abort_flag) && mbar_wait_t<kMergeSuspend>(BAR(B_Y + x), 0, abort_flag));
             float y[DF];
             if (ok) {
                 tc_fence_after();
@@ -415,7 +422,7 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
 #pragma unroll
                 for (int v = 0; v < DH / 8; ++v) oa[v] = valid ? orow[v] : make_uint4(0, 0, 0, 0);
             }
-            ok = warp_all(ok && mbar_wait(BAR(B_PRO), 0, abort_flag));
+            ok = warp_all(ok && mbar_wait_t<kMergeSuspend>(BAR(B_PRO), 0, abort_flag));
             if (ok) {
                 tc_fence_after();
                 const float M = bden > 0.f ? fmaxf(lse_a, __log2f(bden)) : lse_a;
@@ -447,47 +454,24 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
 
         // ---- main loop over key tiles
         for (int j = 0; ok && j < n_tiles; ++j) {
-            ok = warp_all(mbar_wait(BAR(B_S + x), j & 1, abort_flag));
+            ok = warp_all(mbar_wait_t<kMergeSuspend>(BAR(B_S + x), j & 1, abort_flag));
             if (!ok) break;
             tc_fence_after();
-            float sv[128];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t u[32];
-                tmem_ld32(tS + c * 32, u);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) sv[c * 32 + e] = __uint_as_float(u[e]);
-            }
-            tmem_wait_ld();
-            // masks, only on the tiles that need them (warp-uniform test): LOCAL the causal diagonal
-            // tile, PREFIX the ragged last tile of the kept rows
             const bool diag = LOCAL && j == n_tiles - 1;
             const bool ragged = !LOCAL && nk - j * Cfg::BN < Cfg::BN;
-            if (diag) {
-#pragma unroll
-                for (int c = 0; c < 128; ++c)
-                    if (c == r) sdiag = sv[c];  // unrolled select keeps sv in registers
-            }
-            if (diag || ragged) {
-                const int limit = diag ? r + 1 : nk - j * Cfg::BN;
-#pragma unroll
-                for (int c = 0; c < 128; ++c)
-                    if (c >= limit) sv[c] = -INFINITY;
-            }
-            const float mnew = row_max128(sv) * p.scale_log2;
-            // Lazy rescale: a row moves its reference max only when the max grows by more than
-            // kRescaleLog2 (see tc_tile.cuh).
-            // The O rescale uses warp-collective tcgen05.ld/st, so the warp takes it together when
-            // any of its rows needs it (rows that do not keep alpha = 1).
-            const bool need = mnew > m_run + kRescaleLog2;
-            const float alpha = need ? ex2(m_run - mnew) : 1.f;
-            const bool touch_o = need && m_run != -INFINITY;  // O holds nothing yet while m_run = -inf
-            if (__any_sync(0xffffffffu, touch_o)) {
-                ok = warp_all(j == 0 ? (LOCAL || mbar_wait(BAR(B_PRO), 0, abort_flag))
-                                     : mbar_wait(BAR(B_O + x), (j - 1) & 1, abort_flag));
-                if (!ok) break;
+            const int limit = diag ? r + 1 : nk - j * Cfg::BN;
+            float sv[128];
+            load_s_row(tS, sv, diag, ragged, limit, r, sdiag);
+            // O *= a on the rows that move their reference (warp-collective: the warp takes it together
+            // when any of its rows needs it).  P V(j-1) has completed: the scores of tile j were issued
+            // after it (PREFIX j = 0: the prologue's phi(q) S_t^T).
+            auto rescale_o = [&](bool touch, float a) -> bool {
+                if (!__any_sync(0xffffffffu, touch)) return true;
+                if (!warp_all(j == 0 ? (LOCAL || mbar_wait_t<kMergeSuspend>(BAR(B_PRO), 0, abort_flag))
+                                     : mbar_wait_t<kMergeSuspend>(BAR(B_O + x), (j - 1) & 1, abort_flag)))
+                    return false;
                 tc_fence_after();
-                const float f = touch_o ? alpha : 1.f;
+                const float f = touch ? a : 1.f;
 #pragma unroll
                 for (int c = 0; c < DH / 32; ++c) {
                     uint32_t u[32];
@@ -498,7 +482,15 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
                     tmem_st32(tO + c * 32, u);
                 }
                 tmem_wait_st();
-            }
+                return true;
+            };
+            // Lazy rescale: a row moves its reference max only when the max grows by more than
+            // kRescaleLog2 (see tc_tile.cuh).
+            const float mnew = row_max128(sv) * p.scale_log2;
+            const bool need = mnew > m_run + kRescaleLog2;
+            const float alpha = need ? ex2(m_run - mnew) : 1.f;
+            // O holds nothing yet while m_run = -inf
+            if (!(ok = rescale_o(need && m_run != -INFINITY, alpha))) break;
             if (need) {
                 l_run *= alpha;
                 bs *= alpha;
@@ -513,6 +505,7 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
                 else if (i0 >= p.w && kstart < i0 - p.w) btype = 0;
                 else btype = 1;
             }
+            // exponentials stored to P (over S) as they are formed
             float ls0, ls1, bsum = 0.f;
             if (btype >= 2) {
                 const int bc_lo = btype == 2 ? r + 1 : 0, bc_hi = btype == 2 ? 128 : r;
@@ -528,7 +521,7 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
             mbar_arrive(BAR(B_P + x));
         }
         // ---- epilogue: o = O / l
-        ok = warp_all(ok && (n_tiles > 0 ? mbar_wait(BAR(B_O + x), (n_tiles - 1) & 1, abort_flag) : true));
+        ok = warp_all(ok && (n_tiles > 0 ? mbar_wait_t<kMergeSuspend>(BAR(B_O + x), (n_tiles - 1) & 1, abort_flag) : true));
         if (ok) {
             tc_fence_after();
             const float inv = l_run > 0.f ? 1.f / l_run : 0.f;

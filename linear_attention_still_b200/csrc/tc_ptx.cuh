@@ -38,9 +38,8 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
 }
 
-// Non-suspending test of a phase.  (A thread suspended in mbarrier.try_wait was measured to notice a
-// completed phase only at a coarse periodic wake-up, ~14K SM clocks apart, with or without a suspend
-// hint; spinning on test_wait reacts at once.)
+// Non-suspending test of a phase (spinning on it reacts at once; see mbar_wait_susp for the sleeping
+// form).
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -67,6 +66,42 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
             if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
         }
     }
+}
+
+// Potentially suspending test of a phase: the thread may sleep in hardware until the phase completes
+// or a system-dependent time limit passes, without taking issue slots while it sleeps.  (Measured on
+// B200: a merge whose waits all sleep here ran as fast as or faster than with spinning waits, so the
+// wake-up follows the phase closely.)
+__device__ __forceinline__ bool mbar_try_wait_susp(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait built on the suspending test (same limit and abort rule as mbar_wait).
+__device__ __forceinline__ bool mbar_wait_susp(uint32_t bar, uint32_t parity, volatile int *abort) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        if (mbar_try_wait_susp(bar, parity)) return true;
+        if (*abort) return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    }
+}
+
+// Named CTA barriers (ids 1..15; id 0 is __syncthreads): `count` threads in whole warps take part;
+// arriving warps do not wait, syncing warps sleep in hardware until the count is reached.
+__device__ __forceinline__ void nbar_sync(uint32_t id, uint32_t count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+__device__ __forceinline__ void nbar_arrive(uint32_t id, uint32_t count) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 // Wait that ignores the abort flag (used to drain this CTA's own copies and MMAs before exit).

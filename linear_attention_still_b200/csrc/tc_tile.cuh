@@ -100,12 +100,48 @@ __device__ __forceinline__ void store_p(uint32_t tP, const uint32_t (&u)[64]) {
     tmem_st32(tP + 32, *reinterpret_cast<const uint32_t(*)[32]>(&u[32]));
 }
 
+// S row of one key tile from TMEM into registers, masked on the tiles that need it (warp-uniform test):
+// LOCAL the causal diagonal tile (columns past the row), PREFIX the ragged last tile of the kept rows.
+// On the diagonal tile the row's own raw score is kept in sdiag.
+__device__ __forceinline__ void load_s_row(uint32_t tS, float (&sv)[128], bool diag, bool ragged, int limit, int r,
+                                           float &sdiag) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        uint32_t u[32];
+        tmem_ld32(tS + c * 32, u);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) sv[c * 32 + e] = __uint_as_float(u[e]);
+    }
+    tmem_wait_ld();
+    if (diag) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+            if (c == r) sdiag = sv[c];  // unrolled select keeps sv in registers
+    }
+    if (diag || ragged) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+            if (c >= limit) sv[c] = -INFINITY;
+    }
+}
+
 // tcgen05.ld/st are warp-collective: every decision that guards them is made warp-uniform.
 __device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
 
 // Bounded mbarrier wait taken by a whole warp, with one result for all its lanes.
 __device__ __forceinline__ bool mbar_wait_w(uint32_t bar, uint32_t parity, volatile int *abort) {
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
+}
+
+// The same two waits with the form chosen per kernel: SUSP = true sleeps in mbarrier.try_wait between
+// tests (no issue slots taken while waiting), false spins on the non-suspending test.
+template <bool SUSP>
+__device__ __forceinline__ bool mbar_wait_t(uint32_t bar, uint32_t parity, volatile int *abort) {
+    return SUSP ? mbar_wait_susp(bar, parity, abort) : mbar_wait(bar, parity, abort);
+}
+template <bool SUSP>
+__device__ __forceinline__ bool mbar_wait_wt(uint32_t bar, uint32_t parity, volatile int *abort) {
+    return __all_sync(0xffffffffu, mbar_wait_t<SUSP>(bar, parity, abort));
 }
 
 // K-major SW128 descriptor of k-step kk (16 elements) of a tile whose rows are split into 64-col

@@ -200,3 +200,37 @@ def test_diagonal_router_layer(lib, oracle_mod, name):
     assert out["status"] == 0
     ref = oracle_mod.prefill(od, inp.q, inp.k, inp.v, inp.wq, inp.wk, idx_in=gidx)["o"]
     assert row_rel_err(out["o"], ref) <= OUT_TOL[shape.dtype]
+
+
+# Logits that grow (or shrink) by tens of binary orders along the keys: later window tiles (ramp up) or
+# the kept prefix after the window part (ramp down) exceed each row's reference maximum by far more than
+# the lazy-rescale threshold, so the online softmax moves its reference in mid-row, O and the sums are
+# rescaled, and tiles whose probabilities overflow the threshold are recomputed.
+LARGE_LOGIT_CASES = {
+    "bf16_d64_ramp_up": (Shape(B=1, H=4, Hkv=2, N=1500, d=64, D=64, w=256, C=256, k=128), "up"),
+    "bf16_d64_ramp_down": (Shape(B=1, H=4, Hkv=2, N=1500, d=64, D=64, w=256, C=256, k=128), "down"),
+    "bf16_d128_ramp_up": (Shape(B=1, H=4, Hkv=1, N=1500, d=128, D=128, w=256, C=256, k=128), "up"),
+    "bf16_d128_ramp_down": (Shape(B=1, H=4, Hkv=1, N=1500, d=128, D=128, w=256, C=256, k=128), "down"),
+}
+
+
+@pytest.mark.parametrize("name", list(LARGE_LOGIT_CASES))
+def test_prefill_parity_large_logits(lib, oracle_mod, name):
+    from linear_attention_still_b200.synth import round_to_bf16_
+    shape, ramp = LARGE_LOGIT_CASES[name]
+    inp = make_inputs(shape)
+    pos = np.arange(shape.N, dtype=np.float32) / shape.N
+    f = 1.0 + 5.0 * pos if ramp == "up" else 6.0 - 5.0 * pos
+    inp.k *= f[None, None, :, None]
+    inp.q *= np.float32(3.0)
+    round_to_bf16_(inp.k)
+    round_to_bf16_(inp.q)
+    out = gpu_prefill(shape, inp)
+    assert out["status"] == 0
+    d = odims(shape)
+    _, ora_r = oracle_mod.saliency(d, inp.q, inp.k)
+    assert score_err(out["r"], ora_r) <= SCORE_TOL
+    check_selection(shape, shape.N, out["idx"], out["r"], ora_r, oracle_mod.topk(d, ora_r))
+    ref = oracle_mod.prefill(d, inp.q, inp.k, inp.v, inp.wq, inp.wk, idx_in=out["idx"])["o"]
+    err = row_rel_err(out["o"], ref)
+    assert err <= OUT_TOL[shape.dtype], err
