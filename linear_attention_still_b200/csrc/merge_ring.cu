@@ -41,31 +41,39 @@ using namespace tc;
 
 namespace {
 
-template <int DF, int HP>
+template <int DF, int HP, int NH>
 struct RingCfg {
+    // NH = 2: two independent single-head pipelines (halves) in one CTA, each with its own item stream,
+    // query / key / value buffers, barriers and 256 TMEM columns (see the file comment)
+    static_assert(NH == 1 || (NH == 2 && HP == 1 && DF == 64), "two halves run one head each, D = 64");
     static constexpr int DH = 64;
     static constexpr int BN = 128;                       // keys per tile
     static constexpr int TILE_BYTES = 128 * 128;         // 128 rows x 64 bf16: one SW128 region
     static constexpr int Q_BYTES = HP * TILE_BYTES;      // one item's query tiles
     static constexpr int NQ = 2;                         // query buffers
-    static constexpr int NS = DF == 64 ? 4 : 3;          // K/V stages
+    static constexpr int NS = NH == 2 ? 2 : (DF == 64 ? 4 : 3);  // K/V stages
     static constexpr int STAGE_BYTES = 2 * TILE_BYTES;   // K + V
     static constexpr int WQ_BYTES = DF * DH * 2;         // Wq^T of one head: DF rows x 64
     static constexpr int ST_BYTES = DH * DF * 2;         // S_t^T: 64 rows x DF
     static constexpr int W_BYTES = HP * WQ_BYTES + ST_BYTES;
-    static constexpr int BAR_BYTES = 512;
-    static constexpr int SMEM = NQ * Q_BYTES + NS * STAGE_BYTES + W_BYTES + BAR_BYTES + 1024;
+    static constexpr int BAR_BYTES = NH == 2 ? 256 : 512;  // per half
+    static constexpr int HALF_BYTES = NQ * Q_BYTES + NS * STAGE_BYTES + W_BYTES;  // one half's operands
+    static_assert(HALF_BYTES % 1024 == 0, "tiles stay on 1024-byte boundaries");
+    static constexpr int SMEM = NH * HALF_BYTES + NH * BAR_BYTES + 1024;
     static_assert(SMEM <= 232448, "shared memory");
-    static constexpr int THREADS = HP == 2 ? 384 : 192;
-    static constexpr int PRODUCER_WARP = 4 * HP, MMA_WARP = 4 * HP + 1;
+    static constexpr int SOFTMAX_WARPS = 4 * HP * NH;
+    static constexpr int THREADS = SOFTMAX_WARPS == 8 ? 384 : 192;
+    // warps after the softmax warps: per half a TMA producer warp and an MMA warp (half 0's below)
+    static constexpr int PRODUCER_WARP = SOFTMAX_WARPS, MMA_WARP = SOFTMAX_WARPS + 1;
     // launch budget 384 x 168 = 64512 registers = 2 x 128 x 208 (softmax) + 128 x 88 (the rest)
     static constexpr int REG_SOFTMAX = 208, REG_OTHER = 88;
-    static_assert(HP != 2 || 2 * 128 * REG_SOFTMAX + 128 * REG_OTHER <= THREADS * 168, "register split");
-    static constexpr int TMEM_COLS = HP == 2 ? 512 : 256;
+    static_assert(THREADS != 384 || 2 * 128 * REG_SOFTMAX + 128 * REG_OTHER <= THREADS * 168, "register split");
+    static constexpr int TMEM_COLS = THREADS == 384 ? 512 : 256;
+    static constexpr uint32_t HALF_COLS = 256u * HP;  // TMEM columns of one half
     __host__ __device__ static constexpr uint32_t s_col(int x) { return 128u * x; }
     __host__ __device__ static constexpr uint32_t p_col(int x) { return 128u * HP + 64u * x; }
     __host__ __device__ static constexpr uint32_t o_col(int x) { return 192u * HP + 64u * x; }
-    static_assert(256 * HP <= TMEM_COLS, "TMEM budget");
+    static_assert(NH * 256 * HP <= TMEM_COLS, "TMEM budget");
     // barrier slots
     static constexpr int B_QFULL = 0, B_QEMPTY = 2, B_WFULL = 4, B_WEMPTY = 5, B_PRO = 6, B_DRAIN = 7;
     static constexpr int B_KFULL = 8, B_VFULL = 8 + NS, B_KVEMPTY = 8 + 2 * NS;
@@ -140,55 +148,69 @@ constexpr int kRingExpLocal = STILL_RING_EXP_LOCAL, kRingExpPrefix = STILL_RING_
 #define STILL_RING_TURNS 3
 #endif
 constexpr int kRingTurns = STILL_RING_TURNS;
+// D = 64: two independent single-head halves per CTA (1) or one two-head pipeline (0).
+#ifndef STILL_RING_HALVES
+#define STILL_RING_HALVES 0
+#endif
+constexpr bool kRingHalves = STILL_RING_HALVES != 0;
 static_assert(kRingTurns == 0 || kRingTurns == 1 || kRingTurns == 3, "hand-over form");
 
 
-template <int DF, int HP, int EXPV, int MODE>
-__global__ void __launch_bounds__(RingCfg<DF, HP>::THREADS, 1)
+template <int DF, int HP, int NH, int EXPV, int MODE>
+__global__ void __launch_bounds__(RingCfg<DF, HP, NH>::THREADS, 1)
     merge_ring_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                       const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_kh,
                       const __grid_constant__ CUtensorMap map_vh, const __grid_constant__ CUtensorMap map_wq,
                       const __grid_constant__ CUtensorMap map_st, const RingParams p) {
-    using Cfg = RingCfg<DF, HP>;
+    using Cfg = RingCfg<DF, HP, NH>;
     constexpr bool LOCAL = MODE == 0;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *smem0 = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // the half this warp serves: softmax warps by warpgroup, then (producer, MMA) pairs per half
+    const int half = warp < Cfg::SOFTMAX_WARPS ? warp / (4 * HP) : min((warp - Cfg::SOFTMAX_WARPS) >> 1, NH - 1);
+    uint8_t *smem = smem0 + half * Cfg::HALF_BYTES;
     const uint32_t sbase = smem_u32(smem);
     const uint32_t sQ = sbase;                                      // NQ x HP query tiles
     const uint32_t sStage = sQ + Cfg::NQ * Cfg::Q_BYTES;            // NS x (K tile, V tile)
     const uint32_t sW = sStage + Cfg::NS * Cfg::STAGE_BYTES;        // HP x Wq^T, then S_t^T
-    uint8_t *bar_area = smem + Cfg::NQ * Cfg::Q_BYTES + Cfg::NS * Cfg::STAGE_BYTES + Cfg::W_BYTES;
-    const uint32_t sBar = smem_u32(bar_area);
+    uint8_t *bar_area0 = smem0 + NH * Cfg::HALF_BYTES;  // half 0's barriers, the TMEM slot and abort flag
+    const uint32_t sBar = smem_u32(bar_area0 + half * Cfg::BAR_BYTES);
     auto BAR = [&](int i) { return sBar + 8u * i; };
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_area + Cfg::TMEM_SLOT_OFF);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(bar_area + Cfg::ABORT_OFF);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_area0 + Cfg::TMEM_SLOT_OFF);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bar_area0 + Cfg::ABORT_OFF);
+    // work items of this half: ifirst, ifirst + istep, ...
+    const int ifirst = (int)blockIdx.x * NH + half, istep = (int)gridDim.x * NH;
 
     if (threadIdx.x == 0) {
-        for (int e = 0; e < 2; ++e) {
-            mbar_init(BAR(Cfg::B_QFULL + e), 1);
-            mbar_init(BAR(Cfg::B_QEMPTY + e), LOCAL ? 1 : 1 + 128 * HP);  // MMA commit (+ the softmax's ||q|| read)
+        for (int hh = 0; hh < NH; ++hh) {
+            const uint32_t hb = smem_u32(bar_area0 + hh * Cfg::BAR_BYTES);
+            auto BAR = [&](int i) { return hb + 8u * i; };
+            for (int e = 0; e < 2; ++e) {
+                mbar_init(BAR(Cfg::B_QFULL + e), 1);
+                mbar_init(BAR(Cfg::B_QEMPTY + e), LOCAL ? 1 : 1 + 128 * HP);  // MMA commit (+ the softmax's ||q|| read)
+            }
+            mbar_init(BAR(Cfg::B_WFULL), 1);
+            mbar_init(BAR(Cfg::B_WEMPTY), 1);
+            mbar_init(BAR(Cfg::B_PRO), 1);
+            mbar_init(BAR(Cfg::B_DRAIN), 1);
+            for (int s = 0; s < Cfg::NS; ++s) {
+                mbar_init(BAR(Cfg::B_KFULL + s), 1);
+                mbar_init(BAR(Cfg::B_VFULL + s), 1);
+                mbar_init(BAR(Cfg::B_KVEMPTY + s), 1);
+            }
+            for (int x = 0; x < HP; ++x) {
+                mbar_init(BAR(Cfg::B_Y + x), 1);
+                mbar_init(BAR(Cfg::B_PHI + x), 128);
+                mbar_init(BAR(Cfg::B_S + x), 1);
+                mbar_init(BAR(Cfg::B_SFREE + x), 128);
+                mbar_init(BAR(Cfg::B_O + x), 1);
+                mbar_init(BAR(Cfg::B_P + 2 * x), 128);
+                mbar_init(BAR(Cfg::B_P + 2 * x + 1), 128);
+            }
+            mbar_init(BAR(Cfg::B_TURN + 0), 128);
+            mbar_init(BAR(Cfg::B_TURN + 1), 128);
         }
-        mbar_init(BAR(Cfg::B_WFULL), 1);
-        mbar_init(BAR(Cfg::B_WEMPTY), 1);
-        mbar_init(BAR(Cfg::B_PRO), 1);
-        mbar_init(BAR(Cfg::B_DRAIN), 1);
-        for (int s = 0; s < Cfg::NS; ++s) {
-            mbar_init(BAR(Cfg::B_KFULL + s), 1);
-            mbar_init(BAR(Cfg::B_VFULL + s), 1);
-            mbar_init(BAR(Cfg::B_KVEMPTY + s), 1);
-        }
-        for (int x = 0; x < HP; ++x) {
-            mbar_init(BAR(Cfg::B_Y + x), 1);
-            mbar_init(BAR(Cfg::B_PHI + x), 128);
-            mbar_init(BAR(Cfg::B_S + x), 1);
-            mbar_init(BAR(Cfg::B_SFREE + x), 128);
-            mbar_init(BAR(Cfg::B_O + x), 1);
-            mbar_init(BAR(Cfg::B_P + 2 * x), 128);
-            mbar_init(BAR(Cfg::B_P + 2 * x + 1), 128);
-        }
-        mbar_init(BAR(Cfg::B_TURN + 0), 128);
-        mbar_init(BAR(Cfg::B_TURN + 1), 128);
         *abort_flag = 0;
         mbar_fence_init();
     }
@@ -208,16 +230,18 @@ __global__ void __launch_bounds__(RingCfg<DF, HP>::THREADS, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
+    const uint32_t tmem0 = *tmem_slot;
+    const uint32_t tmem = tmem0 + half * Cfg::HALF_COLS;  // this half's columns
 
-    if (warp >= 4 * HP) {
-        if (HP == 2) setmaxnreg_dec<Cfg::REG_OTHER>();
-        if (warp == Cfg::PRODUCER_WARP) {
+    if (warp >= Cfg::SOFTMAX_WARPS) {
+        if (Cfg::THREADS == 384) setmaxnreg_dec<Cfg::REG_OTHER>();
+        const int role = warp - Cfg::SOFTMAX_WARPS - 2 * half;  // 0 producer, 1 MMA issuer, else idle
+        if (role == 0) {
             // (the whole warp runs the issue loop; one elected lane issues each copy)
             // ================================================================ TMA producer
             bool ok = true, stalled = false;
             int G = 0, n = 0, nq = 0, nw = 0;  // K/V tiles, items, query loads, W loads issued
-            for (int it = blockIdx.x; ok && !stalled && it < p.n_items; it += gridDim.x, ++n) {
+            for (int it = ifirst; ok && !stalled && it < p.n_items; it += istep, ++n) {
                 const Item I = item_of<HP, LOCAL>(it, p);
                 const int qb = n & 1;
                 if (n >= 2 && !(ok = mbar_wait_w(BAR(Cfg::B_QEMPTY + qb), ((n >> 1) - 1) & 1, abort_flag))) break;
@@ -266,7 +290,7 @@ __global__ void __launch_bounds__(RingCfg<DF, HP>::THREADS, 1)
                     mbar_wait_drain(BAR(Cfg::B_VFULL + u % Cfg::NS), (u / Cfg::NS) & 1, 100000000ull);
                 }
             }
-        } else if (warp == Cfg::MMA_WARP) {
+        } else if (role == 1) {
             // (the whole warp runs the issue loop; one elected lane issues each MMA and commit)
             const uint32_t tmem_w = __shfl_sync(0xffffffffu, tmem, 0);
             // ================================================================ MMA issuer
@@ -310,7 +334,7 @@ __global__ void __launch_bounds__(RingCfg<DF, HP>::THREADS, 1)
                 return true;
             };
             bool pre = false;
-            for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x, ++n) {
+            for (int it = ifirst; ok && it < p.n_items; it += istep, ++n) {
                 const Item I = item_of<HP, LOCAL>(it, p);
                 const int qb = n & 1;
                 uint64_t dq[HP];
@@ -342,7 +366,7 @@ __global__ void __launch_bounds__(RingCfg<DF, HP>::THREADS, 1)
                         }
                     }
                 }
-                const bool has_next = it + (int)gridDim.x < p.n_items;
+                const bool has_next = it + istep < p.n_items;
                 for (int jj = 0; ok && jj < I.n_tiles; ++jj, ++G) {
                     const int Jt = J + jj, s = G % Cfg::NS, s1 = (G + 1) % Cfg::NS;
                     // next scores first: they only need the softmax to have read S(Jt)
@@ -358,7 +382,7 @@ __global__ void __launch_bounds__(RingCfg<DF, HP>::THREADS, 1)
                         if (!ok) break;
                     } else if (has_next) {
                         // last tile: the next item's first score-column MMA goes ahead of this P V
-                        const Item In = item_of<HP, LOCAL>(it + gridDim.x, p);
+                        const Item In = item_of<HP, LOCAL>(it + istep, p);
                         if (!(ok = issue_head(In, n + 1, Jt + 1, G + 1))) break;
                         pre = true;
                     }
@@ -389,9 +413,9 @@ __global__ void __launch_bounds__(RingCfg<DF, HP>::THREADS, 1)
             mbar_wait_drain(BAR(Cfg::B_DRAIN), 0, 100000000ull);
         }
     } else {
-        if (HP == 2) setmaxnreg_inc<Cfg::REG_SOFTMAX>();
+        if (Cfg::THREADS == 384) setmaxnreg_inc<Cfg::REG_SOFTMAX>();
         // ================================================================ softmax warpgroups
-        const int x = warp >> 2;                       // head of the pair
+        const int x = (warp >> 2) - half * HP;         // head of the pair
         const int r = (warp & 3) * 32 + lane;          // row in the tile = TMEM lane
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t tS = tmem + lane_off + Cfg::s_col(x);
@@ -399,7 +423,7 @@ __global__ void __launch_bounds__(RingCfg<DF, HP>::THREADS, 1)
         const uint32_t tO = tmem + lane_off + Cfg::o_col(x);
         bool ok = true;
         int J = 0, n = 0;
-        for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x, ++n) {
+        for (int it = ifirst; ok && it < p.n_items; it += istep, ++n) {
             const Item I = item_of<HP, LOCAL>(it, p);
             const int i = I.i0 + r;
             const size_t row = ((size_t)I.b * p.H + I.h0 + x) * p.N + i;  // this thread's query row
@@ -667,7 +691,7 @@ __global__ void __launch_bounds__(RingCfg<DF, HP>::THREADS, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == Cfg::MMA_WARP) tmem_dealloc(tmem, Cfg::TMEM_COLS);
+    if (warp == Cfg::MMA_WARP) tmem_dealloc(tmem0, Cfg::TMEM_COLS);
 }
 
 int sm_count() {
@@ -684,9 +708,9 @@ int sm_count() {
 
 int g_stall = 0, g_max_ctas = 0;
 
-template <int DF, int HP>
+template <int DF, int HP, int NH>
 cudaError_t launch_ring_cfg(int mode, const Dims &s, const MergeOperands &a, unsigned *err, cudaStream_t st) {
-    using Cfg = RingCfg<DF, HP>;
+    using Cfg = RingCfg<DF, HP, NH>;
     const int T = s.T();
     const int n_qtiles = (s.N + 127) / 128;
     // PREFIX: only the query chunks t > m see a kept prefix or a linear state
@@ -724,10 +748,11 @@ cudaError_t launch_ring_cfg(int mode, const Dims &s, const MergeOperands &a, uns
     prm.pairs = s.G() / HP;
     prm.n_items = (n_qtiles - qt_first) * s.B * s.Hkv * prm.pairs;
     prm.stall = g_stall;
-    auto kern = mode == 0 ? merge_ring_kernel<DF, HP, kRingExpLocal, 0> : merge_ring_kernel<DF, HP, kRingExpPrefix, 1>;
+    auto kern = mode == 0 ? merge_ring_kernel<DF, HP, NH, kRingExpLocal, 0>
+                          : merge_ring_kernel<DF, HP, NH, kRingExpPrefix, 1>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
     if (e != cudaSuccess) return e;
-    int ctas = std::min(prm.n_items, sm_count());
+    int ctas = std::min((prm.n_items + NH - 1) / NH, sm_count());
     if (g_max_ctas > 0) ctas = std::min(ctas, g_max_ctas);
     const unsigned grid = (unsigned)ctas;
     kern<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(mq, mk, mv, mkh, mvh, mw, ms, prm);
@@ -741,9 +766,12 @@ cudaError_t launch_ring_cfg(int mode, const Dims &s, const MergeOperands &a, uns
 cudaError_t launch_merge_ring(int mode, const Dims &s, const MergeOperands &a, unsigned *err, cudaStream_t st) {
     if (s.d != 64) return cudaErrorNotSupported;
     const bool pair = s.G() % 2 == 0;
-    if (s.D == 64) return pair ? launch_ring_cfg<64, 2>(mode, s, a, err, st) : launch_ring_cfg<64, 1>(mode, s, a, err, st);
+    if (s.D == 64) {
+        if (kRingHalves) return launch_ring_cfg<64, 1, 2>(mode, s, a, err, st);
+        return pair ? launch_ring_cfg<64, 2, 1>(mode, s, a, err, st) : launch_ring_cfg<64, 1, 1>(mode, s, a, err, st);
+    }
     if (s.D == 128)
-        return pair ? launch_ring_cfg<128, 2>(mode, s, a, err, st) : launch_ring_cfg<128, 1>(mode, s, a, err, st);
+        return pair ? launch_ring_cfg<128, 2, 1>(mode, s, a, err, st) : launch_ring_cfg<128, 1, 1>(mode, s, a, err, st);
     return cudaErrorNotSupported;
 }
 
