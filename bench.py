@@ -63,6 +63,9 @@ def parse():
     p.add_argument("--pass", dest="pass_", choices=["forward", "backward"], default="forward",
                    help="prefill workloads: time the forward layer (default) or its backward pass "
                         "(gradients of q, k, v, Wq, Wk with the selection held fixed)")
+    p.add_argument("--bwd-stats", choices=["saved", "recompute"], default="saved",
+                   help="backward pass: take each row's normaliser and D_i from the forward's output and "
+                        "normaliser (saved, what a training step has at hand) or form them again (recompute)")
     p.add_argument("--workloads", choices=["auto", "none"], default="auto",
                    help="auto: a default single-GPU run (no --workload, forward pass, default router and keep) "
                         "also measures the other layer configurations (8B-shaped prefill at B4 x 16K and "
@@ -1005,10 +1008,18 @@ def bench_backward(args, name, rank, world, local, cpu_seconds):
     o = torch.empty_like(devt["q"])
     still.still_hybrid_prefill(dims, devt["q"], devt["k"], devt["v"], devt["wq"], devt["wk"], o, workspace=ws_f)
     idx = None
+    lay = still.still_prefill_workspace_layout(dims)
     if shape.k > 0 and shape.T > 0:
-        off = still.still_prefill_workspace_layout(dims)["idx"]
+        off = lay["idx"]
         n_idx = shape.B * shape.Hkv * shape.T * shape.k
         idx = ws_f[off:off + 4 * n_idx].view(torch.int32).clone()
+    saved = args.bwd_stats == "saved"
+    if saved:
+        # what a training step's forward leaves for the backward: its output and every row's normaliser
+        n_rows = shape.B * shape.H * shape.N
+        host["o"] = o.cpu()
+        host["lse"] = ws_f[lay["lse"]:lay["lse"] + 4 * n_rows].view(torch.float32).cpu().clone()
+        devt["o"], devt["lse"] = o, host["lse"].cuda()
     del ws_f, o
     f32 = dict(dtype=torch.float32, device="cuda")
     grads = [torch.empty(shape.B, shape.H, shape.N, shape.d, **f32),
@@ -1020,7 +1031,12 @@ def bench_backward(args, name, rank, world, local, cpu_seconds):
     stream = torch.cuda.current_stream()
 
     def step(t):
-        still.still_hybrid_backward(dims, t["q"], t["k"], t["v"], t["wq"], t["wk"], idx, t["do"], *grads, workspace=ws)
+        if saved:
+            still.still_hybrid_backward_saved(dims, t["q"], t["k"], t["v"], t["wq"], t["wk"], idx, t["do"], t["o"],
+                                              t["lse"], *grads, workspace=ws)
+        else:
+            still.still_hybrid_backward(dims, t["q"], t["k"], t["v"], t["wq"], t["wk"], idx, t["do"], *grads,
+                                        workspace=ws)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -1087,8 +1103,8 @@ def bench_backward(args, name, rank, world, local, cpu_seconds):
     pairs = int(soft_sizes(shape).sum()) * shape.B * shape.H
     if "bwd_dq" in kernel_ms:
         # tensor-core path: the dominant kernel is the dq kernel; its algorithmic work is S = Q K^T,
-        # dP = dO V^T and dQ += dS K (6 d FLOP per query-head and softmax key; the statistics sweep
-        # that forms S and dP a first time is not counted)
+        # dP = dO V^T and dQ += dS K (6 d FLOP per query-head and softmax key; with --bwd-stats recompute
+        # the statistics sweep that forms S and dP a first time is not counted)
         peak = peaks.get("bf16_tflops", 1590.0)
         dq_flops = 6 * shape.d * pairs
         roof = {"kernel": "bwd_dq_tc_kernel (dq of the softmax branch)", "bound": "tensor",
@@ -1116,7 +1132,7 @@ def bench_backward(args, name, rank, world, local, cpu_seconds):
         "value": job_throughput(tokens, args.steps, world, total_ms), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": shape.dtype, "data": "synthetic",
-        "config": dict(config_of(shape, args, name), **{"pass": "backward"}),
+        "config": dict(config_of(shape, args, name), **{"pass": "backward", "stats": args.bwd_stats}),
         "roofline": roof,
         "kernel_ms_per_step": kernel_ms,
         "e2e": {"value": job_throughput(tokens, args.e2e_steps, world, e2e_ms), "unit": "tokens/s",

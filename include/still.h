@@ -233,6 +233,32 @@ STILL_API still_status still_hybrid_backward(const still_dims *dims, const void 
                                              void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * The same backward pass given what the forward left behind ([p1] "Chunk-Wise":
+ * one implementation for training and inference, where a training step runs
+ * the forward first).  Every row's gradient needs its normaliser L_i (both
+ * branches) and D_i = <dO_i, o_i>; still_hybrid_backward forms them with a
+ * first sweep over the row's keys, this call takes them from the forward:
+ *   o     [B,H,N,d] dtype, the output of still_hybrid_prefill on the same inputs
+ *         (and the same selection idx)
+ *   lse   [B,H,N] fp32, the forward's per-row log2 normaliser: the region "lse" of
+ *         the workspace of that still_hybrid_prefill call (offset in
+ *         still_prefill_workspace_layout), read after the call completed and
+ *         before the workspace is used again
+ * Other arguments, errors and workspace as for still_hybrid_backward; o and lse
+ * must be non-NULL and 16-byte aligned.  They are used where the forward ran its
+ * tensor-core merge and the backward its tensor-core softmax branch (bf16,
+ * d and D in {64, 128}, C a multiple of 128, w >= 1); elsewhere the call forms the
+ * statistics itself, as still_hybrid_backward does.  D_i comes from the rounded
+ * o (dtype), so the gradients differ from still_hybrid_backward's by rounding.
+ */
+STILL_API still_status still_hybrid_backward_saved(const still_dims *dims, const void *q, const void *k,
+                                                   const void *v, const void *Wq, const void *Wk,
+                                                   const int32_t *idx, const void *dO, const void *o,
+                                                   const float *lse, float *dq, float *dk, float *dv, float *dWq,
+                                                   float *dWk, void *workspace, size_t workspace_bytes,
+                                                   void *stream);
+
+/*
  * Chunk-granular delayed decode ([p1] "Chunk-Wise": during decoding the
  * selection is delayed at chunk granularity).  The state is one caller-owned
  * device buffer holding, per (b, g): the kept K/V cache, the linear state

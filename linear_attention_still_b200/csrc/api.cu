@@ -271,6 +271,37 @@ still_status still_hybrid_backward(const still_dims *dims, const void *q, const 
     return e == cudaSuccess ? STILL_OK : STILL_ERR_CUDA;
 }
 
+still_status still_hybrid_backward_saved(const still_dims *dims, const void *q, const void *k, const void *v,
+                                         const void *Wq, const void *Wk, const int32_t *idx, const void *dO,
+                                         const void *o, const float *lse, float *dq, float *dk, float *dv,
+                                         float *dWq, float *dWk, void *workspace, size_t workspace_bytes,
+                                         void *stream) {
+    Dims s;
+    still_status st = check_dims(dims, &s);
+    if (st) return st;
+    if ((long long)s.B * s.N == 0) return STILL_OK;
+    const void *ptrs[] = {q, k, v, Wq, Wk, dO, o, lse, dq, dk, dv, dWq, dWk, workspace};
+    for (const void *p : ptrs)
+        if (!p || !aligned16(p)) return STILL_ERR_INVALID_ARG;
+    const bool select = s.k > 0 && s.T() > 0;
+    if (select && (!idx || !aligned16(idx))) return STILL_ERR_INVALID_ARG;
+    size_t off[kBwdSegments];
+    if (workspace_bytes < backward_layout(s, off)) return STILL_ERR_WORKSPACE;
+    if (((uintptr_t)workspace & 255u) != 0) return STILL_ERR_INVALID_ARG;
+    unsigned char *ws = static_cast<unsigned char *>(workspace);
+    auto F = [&](int i) { return reinterpret_cast<float *>(ws + off[i]); };
+    BackwardScratch w{F(0), F(1), F(2), F(3), F(4), F(9), F(10), F(5), F(6), F(7), F(8), F(11), F(12), F(13), F(14), F(15), F(16)};
+    // the forward leaves every row's whole normaliser in its workspace on the tensor-core merge path only;
+    // elsewhere the statistics are formed again as in still_hybrid_backward
+    const bool saved = tc_merge_supported(s);
+    int launches = 0;
+    cudaError_t e = launch_backward(s, q, k, v, Wq, Wk, select ? idx : nullptr, dO, dq, dk, dv, dWq, dWk, w,
+                                    device_error_word(), static_cast<cudaStream_t>(stream), &launches,
+                                    saved ? o : nullptr, saved ? lse : nullptr);
+    g_launches.fetch_add((uint64_t)launches, std::memory_order_relaxed);
+    return e == cudaSuccess ? STILL_OK : STILL_ERR_CUDA;
+}
+
 still_status still_select_topk(const still_dims *dims, const float *r_kv, int32_t *idx, void *stream) {
     Dims s;
     still_status st = check_dims(dims, &s);

@@ -49,6 +49,8 @@ struct BwdParams {
     float *Phi, *SG;          // [B,H,N,D] phi(q) and S_t dO (fp32), written by the dq kernel prologue; its
                               // epilogue then replaces them with a = 2^-L phi(q) and dY = dL/d(q Wq)
     float *L, *Dv;            // [B,H,N] log2 normaliser and D_i (dq kernel writes, key kernel reads)
+    const float *lse_in;      // [B,H,N] the forward's log2 normaliser, or null (the dq kernel forms it)
+    const __nv_bfloat16 *o_in;  // [B,H,N,d] the forward's output (with lse_in: D_i = <dO_i, o_i>)
     float *dq, *dk, *dv;      // fp32 gradients
     const int32_t *idx;       // [B,Hkv,T,k] (kept keys)
     int n_qtiles;             // dq kernel: ceil(N / 128)
@@ -133,6 +135,9 @@ __global__ void __launch_bounds__(BwdQCfg<DH, DF>::THREADS, BwdQCfg<DH, DF>::MIN
     const int nt = nkt + (i0 + 128 - lo) / 64;          // key tiles per sweep
     const int ntot = 2 * nt;
     const int tslot = bg * (p.T + 1) + t;               // linear state slot of the chunk
+    // with the forward's normaliser and output the statistics sweep is skipped: tiles first .. ntot - 1
+    // (pipeline slot and barrier phase of tile jj: jj - first)
+    const int first = p.lse_in ? nt : 0;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < Cfg::NUM_BARS; ++i)
@@ -168,9 +173,9 @@ __global__ void __launch_bounds__(BwdQCfg<DH, DF>::THREADS, BwdQCfg<DH, DF>::MIN
             for (int rr = 0; rr < DF / 64; ++rr)
                 tma_load_3d_w(sbase + Cfg::OFF_ST + rr * (DH * 128), &map_st, BAR(Cfg::B_WFULL), rr * 64, 0, tslot);
         }
-        for (int jj = 0; jj < ntot; ++jj) {
-            const int s = jj % Cfg::NS;
-            if (jj >= Cfg::NS && !(ok = mbar_wait_w(BAR(Cfg::B_KVEMPTY + s), ((jj / Cfg::NS) - 1) & 1, abort_flag)))
+        for (int pj = 0; pj < ntot - first; ++pj) {
+            const int jj = pj + first, s = pj % Cfg::NS;
+            if (pj >= Cfg::NS && !(ok = mbar_wait_w(BAR(Cfg::B_KVEMPTY + s), ((pj / Cfg::NS) - 1) & 1, abort_flag)))
                 break;
             const int j = jj < nt ? jj : jj - nt;
             const bool kept = j < nkt;
@@ -184,7 +189,7 @@ __global__ void __launch_bounds__(BwdQCfg<DH, DF>::THREADS, BwdQCfg<DH, DF>::MIN
             mbar_arrive_expect_tx_w(BAR(Cfg::B_VFULL + s), Cfg::K_BYTES);
             for (int rr = 0; rr < DH / 64; ++rr)
                 tma_load_3d_w(sV + rr * Cfg::K_REG, mv, BAR(Cfg::B_VFULL + s), rr * 64, row, bg);
-            issued = jj + 1;
+            issued = pj + 1;
         }
         bool w2 = false;
         if (PRO && ok && (ok = mbar_wait_w(BAR(Cfg::B_PRO), 0, abort_flag))) {
@@ -200,9 +205,9 @@ __global__ void __launch_bounds__(BwdQCfg<DH, DF>::THREADS, BwdQCfg<DH, DF>::MIN
             mbar_wait_drain(BAR(Cfg::B_QFULL), 0, 100000000ull);
             if (PRO) mbar_wait_drain(BAR(Cfg::B_WFULL), 0, 100000000ull);
             if (w2) mbar_wait_drain(BAR(Cfg::B_W2FULL), 0, 100000000ull);
-            for (int jj = max(0, issued - Cfg::NS); jj < issued; ++jj) {
-                mbar_wait_drain(BAR(Cfg::B_KFULL + jj % Cfg::NS), (jj / Cfg::NS) & 1, 100000000ull);
-                mbar_wait_drain(BAR(Cfg::B_VFULL + jj % Cfg::NS), (jj / Cfg::NS) & 1, 100000000ull);
+            for (int pj = max(0, issued - Cfg::NS); pj < issued; ++pj) {
+                mbar_wait_drain(BAR(Cfg::B_KFULL + pj % Cfg::NS), (pj / Cfg::NS) & 1, 100000000ull);
+                mbar_wait_drain(BAR(Cfg::B_VFULL + pj % Cfg::NS), (pj / Cfg::NS) & 1, 100000000ull);
             }
         }
     } else if (warp == Cfg::MMA_WARP) {
@@ -216,12 +221,13 @@ __global__ void __launch_bounds__(BwdQCfg<DH, DF>::THREADS, BwdQCfg<DH, DF>::MIN
         // The row warps reuse a dS buffer only after B_S of the tile two later, whose commit covers
         // this MMA.
         auto issue_dq = [&](int jj) {
-            const uint64_t dk = sw128_desc(sbase + Cfg::OFF_STAGE + (jj % Cfg::NS) * Cfg::STAGE_BYTES, Cfg::K_REG, 1024);
+            const int st = (jj - first) % Cfg::NS;
+            const uint64_t dk = sw128_desc(sbase + Cfg::OFF_STAGE + st * Cfg::STAGE_BYTES, Cfg::K_REG, 1024);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
                 mma_ts_w(tm + Cfg::DQ_COL, tm + Cfg::DS_COL + 32 * (jj & 1) + kk * 8, dk + (uint64_t)(kk * 128), ID_DQ,
                          (jj > nt || kk > 0) ? 1u : 0u);
-            mma_commit_w(BAR(Cfg::B_KVEMPTY + jj % Cfg::NS));
+            mma_commit_w(BAR(Cfg::B_KVEMPTY + st));
         };
         bool ok = mbar_wait_w(BAR(Cfg::B_QFULL), 0, abort_flag);
         if (PRO && ok && (ok = mbar_wait_w(BAR(Cfg::B_WFULL), 0, abort_flag))) {
@@ -252,13 +258,13 @@ __global__ void __launch_bounds__(BwdQCfg<DH, DF>::THREADS, BwdQCfg<DH, DF>::MIN
                 ok = mbar_wait_w(BAR(Cfg::B_PRO), 0, abort_flag);  // warpgroup 0 has read lin and sg
             }
         }
-        for (int jj = 0; ok && jj < ntot; ++jj) {
-            const int s = jj % Cfg::NS;
+        for (int jj = first; ok && jj < ntot; ++jj) {
+            const int pj = jj - first, s = pj % Cfg::NS;
             const uint32_t sK = sbase + Cfg::OFF_STAGE + s * Cfg::STAGE_BYTES, sV = sK + Cfg::K_BYTES;
-            if (!(ok = mbar_wait_w(BAR(Cfg::B_KFULL + s), (jj / Cfg::NS) & 1, abort_flag))) break;
-            if (!(ok = mbar_wait_w(BAR(Cfg::B_VFULL + s), (jj / Cfg::NS) & 1, abort_flag))) break;
+            if (!(ok = mbar_wait_w(BAR(Cfg::B_KFULL + s), (pj / Cfg::NS) & 1, abort_flag))) break;
+            if (!(ok = mbar_wait_w(BAR(Cfg::B_VFULL + s), (pj / Cfg::NS) & 1, abort_flag))) break;
             // the row warps hold S, dP of tile jj-1 in registers: the columns are free
-            if (jj > 0 && !(ok = mbar_wait_w(BAR(Cfg::B_SDONE), (jj - 1) & 1, abort_flag))) break;
+            if (pj > 0 && !(ok = mbar_wait_w(BAR(Cfg::B_SDONE), (pj - 1) & 1, abort_flag))) break;
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < DH / 16; ++kk)
@@ -435,8 +441,42 @@ __global__ void __launch_bounds__(BwdQCfg<DH, DF>::THREADS, BwdQCfg<DH, DF>::MIN
         }
         const float sl2 = p.scale_log2;
         float M = -INFINITY, l = 0.f, u = 0.f, Lr = 0.f, Di = 0.f;
-        for (int jj = 0; ok && jj < ntot; ++jj) {
-            if (!(ok = warp_all(mbar_wait(BAR(Cfg::B_S), jj & 1, abort_flag)))) break;
+        if (p.lse_in) {
+            // the forward's normaliser of the row and D_i = <dO_i, o_i> (dO from the swizzled tile)
+            ok = warp_all(ok && mbar_wait(BAR(Cfg::B_QFULL), 0, abort_flag));
+            if (ok && live) {
+                Lr = p.lse_in[row];
+                const uint4 *orow = reinterpret_cast<const uint4 *>(p.o_in + row * DH);
+#pragma unroll
+                for (int c = 0; c < DH / 8; ++c) {
+                    const uint4 ov = orow[c];
+                    const uint4 gv = *reinterpret_cast<const uint4 *>(smem + Cfg::OFF_DO + (c >> 3) * Cfg::Q_REG + r * 128 +
+                                                                      (((c & 7) ^ (r & 7)) << 4));
+                    const __nv_bfloat162 *oh = reinterpret_cast<const __nv_bfloat162 *>(&ov);
+                    const __nv_bfloat162 *gh = reinterpret_cast<const __nv_bfloat162 *>(&gv);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 of = __bfloat1622float2(oh[e]), gf = __bfloat1622float2(gh[e]);
+                        Di = fmaf(of.x, gf.x, fmaf(of.y, gf.y, Di));
+                    }
+                }
+                if (x == 0) {
+                    p.L[row] = Lr;
+                    p.Dv[row] = Di;
+                }
+            }
+            if (PRO && x == 1) {  // the prologue's linear terms of this row (warpgroup 0)
+                ok = warp_all(ok && mbar_wait(BAR(Cfg::B_PRO), 0, abort_flag));
+                if (ok) {
+                    const float *lx = reinterpret_cast<const float *>(smem + Cfg::OFF_LXC);
+                    lden = lx[3 * r];
+                    dl = lx[3 * r + 1];
+                    qn2 = lx[3 * r + 2];
+                }
+            }
+        }
+        for (int jj = first; ok && jj < ntot; ++jj) {
+            if (!(ok = warp_all(mbar_wait(BAR(Cfg::B_S), (jj - first) & 1, abort_flag)))) break;
             tc_fence_after();
             const int j = jj < nt ? jj : jj - nt;
             // columns c < lim are in Soft(i): kept entries below nk, window keys at or before i
@@ -1062,6 +1102,8 @@ cudaError_t launch_backward_tc(const Dims &s, const void *q, const void *k, cons
     prm.SG = pro.SG;
     prm.L = L;
     prm.Dv = Dv;
+    prm.lse_in = pro.lse_fwd;
+    prm.o_in = static_cast<const __nv_bfloat16 *>(pro.o_fwd);
     prm.dq = dq;
     prm.dk = dk;
     prm.dv = dv;

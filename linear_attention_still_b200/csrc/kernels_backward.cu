@@ -807,7 +807,8 @@ cudaError_t backward_nowin_t(const Dims &s, const void *q, const void *k, const 
 template <typename T>
 cudaError_t backward_t(const Dims &s, const void *q, const void *k, const void *v, const void *Wq, const void *Wk,
                        const int32_t *idx, const void *dO, float *dq, float *dk, float *dv, float *dWq,
-                       float *dWk, const BackwardScratch &w, unsigned *err, cudaStream_t st, int *launches) {
+                       float *dWk, const BackwardScratch &w, unsigned *err, cudaStream_t st, int *launches,
+                       const void *o_fwd, const float *lse_fwd) {
     const T *Q = (const T *)q, *K = (const T *)k, *V = (const T *)v, *WQ = (const T *)Wq, *WK = (const T *)Wk;
     const T *GO = (const T *)dO;
     const int T_ = s.T();
@@ -845,6 +846,8 @@ cudaError_t backward_t(const Dims &s, const void *q, const void *k, const void *
         // tiled linear branch with the tensor-core linear state: the dq kernel forms the rows' linear
         // terms itself (its prologue writes phi(q) and S_t dO for the later linear kernels)
         BwdPrologue pro{nullptr, Wq, nullptr, w.z, w.A, w.dYq};
+        pro.o_fwd = o_fwd;      // the forward's output and normaliser (null: the dq kernel forms L, D)
+        pro.lse_fwd = lse_fwd;
         if (tiled && tiled_state) {
             pro.wqt = w.wqt;
             pro.st_t = w.st_t;
@@ -918,15 +921,16 @@ cudaError_t launch_bwd_suffix(const Dims &s, float *R, float *r, cudaStream_t st
 cudaError_t launch_backward(const Dims &s, const void *q, const void *k, const void *v, const void *Wq,
                             const void *Wk, const int32_t *idx, const void *dO, float *dq, float *dk, float *dv,
                             float *dWq, float *dWk, const BackwardScratch &w, unsigned *err, cudaStream_t st,
-                            int *launches) {
+                            int *launches, const void *o_fwd, const float *lse_fwd) {
     if (s.w == 0) {
         if (s.bf16)
             return backward_nowin_t<__nv_bfloat16>(s, q, k, v, Wq, Wk, dO, dq, dk, dv, dWq, dWk, w, err, st, launches);
         return backward_nowin_t<float>(s, q, k, v, Wq, Wk, dO, dq, dk, dv, dWq, dWk, w, err, st, launches);
     }
     if (s.bf16)
-        return backward_t<__nv_bfloat16>(s, q, k, v, Wq, Wk, idx, dO, dq, dk, dv, dWq, dWk, w, err, st, launches);
-    return backward_t<float>(s, q, k, v, Wq, Wk, idx, dO, dq, dk, dv, dWq, dWk, w, err, st, launches);
+        return backward_t<__nv_bfloat16>(s, q, k, v, Wq, Wk, idx, dO, dq, dk, dv, dWq, dWk, w, err, st, launches, o_fwd,
+                                         lse_fwd);
+    return backward_t<float>(s, q, k, v, Wq, Wk, idx, dO, dq, dk, dv, dWq, dWk, w, err, st, launches, nullptr, nullptr);
 }
 
 }  // namespace still

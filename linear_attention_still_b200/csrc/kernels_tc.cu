@@ -73,7 +73,8 @@ struct MergeParams {
     float scale_log2;      // tau * log2(e)
     const float *z;        // [B*Hkv*(T+1), DF] fp32
     __nv_bfloat16 *o;      // [B,H,N,DH]: window part (normalised) after LOCAL, final output after PREFIX
-    float *lse;            // [B,H,N]: log2-sum-exp of the window part (LOCAL writes, PREFIX reads)
+    float *lse;            // [B,H,N]: log2-sum-exp of the window part (LOCAL writes, PREFIX reads and
+                           // replaces it with the row's whole log2 normaliser)
     float *sigma;          // [B,H,N]: Self-Saliency Score per query head (LOCAL writes)
     int *fix_list;         // rows whose band sum underflowed against the window max (recomputed later)
     unsigned *fix_count;
@@ -544,6 +545,9 @@ __global__ void __launch_bounds__(MergeCfg<DH, DF, HP>::THREADS, 1)
                     }
                 }
             }
+            // lse: LOCAL the window part's log2-sum-exp (read back by the prefix phase); PREFIX the
+            // row's whole normaliser (both branches), left for the backward pass
+            if (!LOCAL && i < p.N) p.lse[row] = m_run + __log2f(l_run);
             if (LOCAL && i < p.N) {
                 p.lse[row] = m_run + __log2f(l_run);
                 // sigma = softplus(s_ii - LSE_{band}) in natural units; +inf for an empty band (i = 0)

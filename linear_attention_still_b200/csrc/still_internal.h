@@ -99,6 +99,10 @@ struct BwdPrologue {
     const void *st_t;   // [B,Hkv,T+1,d,D] S_t^T (bf16)
     const float *z;     // [B,Hkv,T+1,D]
     float *Phi, *SG;    // [B,H,N,D] out: a = 2^-L phi(q) and dY = dL/d(q Wq) (phi(q), S_t dO on the way)
+    // the forward's output [B,H,N,d] and per-row log2 normaliser [B,H,N], or null: with them the dq
+    // kernel takes L_i and D_i = <dO_i, o_i> as given and skips its statistics sweep
+    const void *o_fwd = nullptr;
+    const float *lse_fwd = nullptr;
 };
 cudaError_t launch_backward_tc(const Dims &s, const void *q, const void *k, const void *v, const void *khat,
                                const void *vhat, const int32_t *idx, const void *dO, const float *lden,
@@ -107,7 +111,7 @@ cudaError_t launch_backward_tc(const Dims &s, const void *q, const void *k, cons
 cudaError_t launch_backward(const Dims &s, const void *q, const void *k, const void *v, const void *Wq,
                             const void *Wk, const int32_t *idx, const void *dO, float *dq, float *dk, float *dv,
                             float *dWq, float *dWk, const BackwardScratch &w, unsigned *err, cudaStream_t st,
-                            int *launches);
+                            int *launches, const void *o_fwd = nullptr, const float *lse_fwd = nullptr);
 
 // Every argument check of still_hybrid_prefill except the workspace's (api.cu).
 still_status check_prefill_args(const still_dims *dims, const void *q, const void *k, const void *v, const void *Wq,

@@ -23,7 +23,7 @@ EXPORTS = ("still_status_string", "still_saliency", "still_select_topk", "still_
            "still_decode_state_bytes", "still_decode_init", "still_decode_step", "still_get_device_status",
            "still_launch_count", "still_timing_enable", "still_timing_read", "still_debug_merge",
            "still_hybrid_prefill_static", "still_diagonal_score", "still_backward_workspace_bytes",
-           "still_hybrid_backward", "still_decode_state_layout")
+           "still_hybrid_backward", "still_hybrid_backward_saved", "still_decode_state_layout")
 
 
 class StillError(RuntimeError):
@@ -64,6 +64,7 @@ _SIG = {
     "still_hybrid_prefill_static": ([_D, _P, _P, _P, _P, _P, _P, _P, _P, ct.c_int, _P], ct.c_int),
     "still_backward_workspace_bytes": ([_D], ct.c_size_t),
     "still_hybrid_backward": ([_D] + [_P] * 13 + [ct.c_size_t, _P], ct.c_int),
+    "still_hybrid_backward_saved": ([_D] + [_P] * 15 + [ct.c_size_t, _P], ct.c_int),
     "still_decode_state_bytes": ([_D, ct.c_int], ct.c_size_t),
     "still_decode_init": ([_D, ct.c_int, _P, _P], ct.c_int),
     "still_decode_state_layout": ([_D, ct.c_int, ct.POINTER(still_state_layout)], ct.c_int),
@@ -204,6 +205,16 @@ def still_hybrid_backward(dims, q, k, v, wq, wk, idx, do, dq, dk, dv, dwq, dwk, 
                workspace=workspace)
     _ok("still_hybrid_backward",
         _lib.still_hybrid_backward(ct.byref(dims), *a, int(workspace_bytes), _stream(stream)))
+
+
+def still_hybrid_backward_saved(dims, q, k, v, wq, wk, idx, do, o, lse, dq, dk, dv, dwq, dwk, workspace=None,
+                                workspace_bytes=None, stream=None):
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    a = _dargs(q=q, k=k, v=v, wq=wq, wk=wk, idx=idx, do=do, o=o, lse=lse, dq=dq, dk=dk, dv=dv, dwq=dwq, dwk=dwk,
+               workspace=workspace)
+    _ok("still_hybrid_backward_saved",
+        _lib.still_hybrid_backward_saved(ct.byref(dims), *a, int(workspace_bytes), _stream(stream)))
 
 
 def still_decode_state_bytes(dims, capacity: int) -> int:

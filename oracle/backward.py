@@ -64,9 +64,23 @@ def routing_sets(i, N, w, C, sel_of_chunk):
     return soft + local, lin
 
 
-def layer_backward(q, k, v, wq, wk, do, idx, w, C, scale=None):
+def _round_bf16(x):
+    """x rounded to the nearest bf16 (ties to even), returned in fp64."""
+    x = np.array(x, dtype=np.float32)
+    u = x.view(np.uint32)
+    u += ((u >> 16) & 1) + np.uint32(0x7FFF)
+    u &= np.uint32(0xFFFF0000)
+    return x.astype(np.float64)
+
+
+def layer_backward(q, k, v, wq, wk, do, idx, w, C, scale=None, d_from_output=None):
     """Gradients (dq, dk, dv, dwq, dwk) of L = sum(do * o) with the selection idx [B,Hkv,T,k] held
-    fixed (idx may be None when no chunk is ever decided, or k = 0)."""
+    fixed (idx may be None when no chunk is ever decided, or k = 0).
+
+    d_from_output="bf16": the row term D_i = <do_i, o_i> is formed from the row's output rounded to
+    bf16, as a backward that takes the forward's stored (bf16) output does; every other step is exact.
+    (D_i enters dL/ds_ij and dL/dw_ij through the difference do.v_j - D_i, so the rounding of o reaches
+    dq, dk, dWq and dWk but not dv.)"""
     q, k, v, wq, wk, do = (np.asarray(a, np.float64) for a in (q, k, v, wq, wk, do))
     B, H, N, d = q.shape
     Hkv = k.shape[1]
@@ -98,7 +112,7 @@ def layer_backward(q, k, v, wq, wk, do, idx, w, C, scale=None):
                         continue
                     o = (e @ V[soft] if len(soft) else 0.0) + (wl @ V[lin] if len(lin) else 0.0)
                     o = o / Z
-                    go = float(gi @ o)
+                    go = float(gi @ (_round_bf16(o) if d_from_output == "bf16" else o))
                     dphiq = np.zeros_like(phiq)
                     if len(soft):  # every index of a row's sets is distinct
                         p = e / Z

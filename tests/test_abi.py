@@ -111,6 +111,13 @@ def test_backward_rejects(lib):
     args = [FAKE] * 13
     args[6] = FAKE + 4                                                   # misaligned dO
     assert f(ct.byref(d), *args, need, None) == 1
+    # the form that takes the forward's output and normaliser refuses before any launch as well
+    fs = lib._lib.still_hybrid_backward_saved
+    for i, bad in ((7, None), (8, None), (8, FAKE + 4), (5, None)):       # o, lse, misaligned lse, idx
+        args = [FAKE] * 15
+        args[i] = bad
+        assert fs(ct.byref(d), *args, need, None) == 1, i
+    assert fs(ct.byref(d), *([FAKE] * 15), need - 1, None) == 3
 
 
 def test_decode_rejects(lib):

@@ -106,3 +106,23 @@ def test_backward_golden():
     np.testing.assert_allclose(dk[0, 0, :, 0], gold["dk"], rtol=1e-12, atol=1e-14)
     np.testing.assert_allclose(dv[0, 0, :, 0], gold["dv"], rtol=1e-12, atol=1e-14)
     assert np.all(dwq == 0.0) and np.all(dwk == 0.0)
+
+
+def test_output_rounded_in_d_reaches_every_gradient_but_dv():
+    """The backward form that takes D_i = <do_i, o_i> from the forward's stored bf16 output: on the
+    seeded inputs of the GPU case tc_bf16_gqa_ragged, rounding o alone moves dq and dk by under 1e-2 of
+    their largest entry and leaves dv exactly as it is (dv = P^T do does not involve D_i).  The GPU
+    parity test of still_hybrid_backward_saved allows 2e-2 for the gradients D_i reaches."""
+    import oracle
+    from linear_attention_still_b200.synth import Shape, make_inputs, round_to_bf16
+    shape = Shape(B=2, H=8, Hkv=2, N=700, d=64, D=64, w=128, C=128, k=16)
+    inp = make_inputs(shape)
+    do = round_to_bf16(np.random.default_rng(77).standard_normal(inp.q.shape).astype(np.float32))[0]
+    idx = oracle.prefill(oracle.Dims.of(shape), inp.q, inp.k, inp.v, inp.wq, inp.wk)["idx"]
+    exact = backward.layer_backward(inp.q, inp.k, inp.v, inp.wq, inp.wk, do, idx, shape.w, shape.C)
+    rounded = backward.layer_backward(inp.q, inp.k, inp.v, inp.wq, inp.wk, do, idx, shape.w, shape.C,
+                                      d_from_output="bf16")
+    rel = [float(np.abs(a - b).max() / np.abs(b).max()) for a, b in zip(rounded, exact)]
+    assert rel[2] == 0.0                                   # dv
+    assert 0.0 < rel[0] < 1e-2 and 0.0 < rel[1] < 1e-2     # dq, dk
+    assert rel[3] < 1e-2 and rel[4] < 1e-2                 # dWq, dWk
