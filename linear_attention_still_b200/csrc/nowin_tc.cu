@@ -30,15 +30,25 @@ using namespace tc;
 
 namespace {
 
+// D = 64: two CTAs per SM (256 TMEM columns and one key/value stage each), so one CTA's serial
+// chain (Y_K -> phi(k) -> A -> P -> P V) overlaps the other's (1), or one CTA per SM (0).  Measured on
+// B200 (1B-shaped layer, w = 0, 16K tokens): 0.290 -> 0.212 ms for this kernel, 168 registers with a
+// few spilled instead of 184.
+#ifndef STILL_NOWIN_PAIR
+#define STILL_NOWIN_PAIR 1
+#endif
+
 template <int DF>
 struct NowinCfg {
+    static constexpr bool PAIR = STILL_NOWIN_PAIR != 0 && DF == 64;
+    static constexpr int MINB = PAIR ? 2 : 1;
     static constexpr int DH = 64;
     static constexpr int REG = 128 * 128;                // 128 rows x 64 bf16 (one SW128 region)
     static constexpr int Q_BYTES = REG;                  // 128 queries x 64
     static constexpr int W_BYTES = DF * 128;             // Wq^T / Wk^T: DF rows x 64
     static constexpr int ST_BYTES = 64 * DF * 2;         // S_t^T: 64 rows x DF (DF/64 regions of 64 rows)
     static constexpr int PHI_BYTES = 128 * DF * 2;       // 128 rows x DF (DF/64 regions)
-    static constexpr int NS = 2;
+    static constexpr int NS = PAIR ? 1 : 2;
     static constexpr int STAGE_BYTES = 2 * REG;          // K + V
     static constexpr int OFF_Q = 0, OFF_WQ = OFF_Q + Q_BYTES, OFF_WK = OFF_WQ + W_BYTES, OFF_ST = OFF_WK + W_BYTES,
                          OFF_PQ = OFF_ST + ST_BYTES, OFF_PK = OFF_PQ + PHI_BYTES, OFF_STAGE = OFF_PK + PHI_BYTES,
@@ -46,9 +56,11 @@ struct NowinCfg {
     static constexpr int BAR_BYTES = 512;
     static constexpr int SMEM = OFF_BAR + BAR_BYTES + 1024;
     static_assert(SMEM <= 232448, "shared memory");
+    static_assert(MINB * (SMEM + 1024) <= 233472, "shared memory per SM");
     static constexpr int THREADS = 192;
     static constexpr int PRODUCER_WARP = 4, MMA_WARP = 5;
-    static constexpr int A_COL = 0, YK_COL = 128, O_COL = 256, TMEM_COLS = 512;
+    static constexpr int A_COL = 0, YK_COL = 128, O_COL = PAIR ? 192 : 256, TMEM_COLS = PAIR ? 256 : 512;
+    static_assert(O_COL + 64 <= TMEM_COLS && YK_COL + DF <= O_COL, "TMEM columns");
     // barrier slots
     static constexpr int B_QFULL = 0, B_WFULL = 1, B_YQ = 2, B_PHIQ = 3, B_PRO = 4, B_DRAIN = 5, B_YK = 6,
                          B_PHIK = 7, B_A = 8, B_P = 9, B_O = 10, B_KFULL = 11, B_VFULL = 11 + NS,
@@ -120,7 +132,7 @@ __device__ __forceinline__ float row_sqnorm_sw128(const uint8_t *tile, int row) 
 }
 
 template <int DF>
-__global__ void __launch_bounds__(NowinCfg<DF>::THREADS, 1)
+__global__ void __launch_bounds__(NowinCfg<DF>::THREADS, NowinCfg<DF>::MINB)
     nowin_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_wq,
                     const __grid_constant__ CUtensorMap map_wk, const __grid_constant__ CUtensorMap map_st,
