@@ -1318,12 +1318,13 @@ static cudaError_t launch_saliency_cfg(const Dims &s, const void *q, const void 
 // Self-Saliency Score of the rows listed by the window kernel, recomputed with the band's own maximum
 // (one warp per row, lanes split the band keys; same definition as the window kernel:
 // sigma = softplus(s_ii - LSE_{j in [i-w+1, i-1]} s_ij)).
+template <int DH>
 __global__ void __launch_bounds__(128) saliency_fixup_kernel(const __nv_bfloat16 *__restrict__ q,
                                                              const __nv_bfloat16 *__restrict__ k,
                                                              const int *__restrict__ list,
                                                              const unsigned *__restrict__ count, float *sigma, int H,
-                                                             int Hkv, int N, int d, int w, float scale) {
-    __shared__ __align__(16) float qs[4][256];
+                                                             int Hkv, int N, int w, float scale) {
+    __shared__ __align__(16) float qs[4][DH];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const unsigned n = *count;
     for (unsigned e = blockIdx.x * 4 + warp; e < n; e += gridDim.x * 4) {
@@ -1331,13 +1332,30 @@ __global__ void __launch_bounds__(128) saliency_fixup_kernel(const __nv_bfloat16
         const int i = (int)(row % N);
         const size_t bh = row / N;
         const int h = (int)(bh % H), b = (int)(bh / H), g = h / (H / Hkv);
-        const __nv_bfloat16 *kg = k + ((size_t)b * Hkv + g) * N * d;
-        for (int x = lane; x < d; x += 32) qs[warp][x] = __bfloat162float(q[row * d + x]);
+        const __nv_bfloat16 *kg = k + ((size_t)b * Hkv + g) * N * DH;
+        for (int x = lane; x < DH; x += 32) qs[warp][x] = __bfloat162float(q[row * DH + x]);
         __syncwarp();
         const int lo = max(0, i - w + 1);
         float mx = -INFINITY, sm = 0.f;
+        // one band key per lane and step; the key row's DH/8 loads are all issued before its dot product
+#pragma unroll 2
         for (int j = lo + lane; j < i; j += 32) {
-            const float l = scale * dot_row(qs[warp], kg + (size_t)j * d, d);
+            const uint4 *kr = reinterpret_cast<const uint4 *>(kg + (size_t)j * DH);
+            uint4 u[DH / 8];
+#pragma unroll
+            for (int x8 = 0; x8 < DH / 8; ++x8) u[x8] = __ldg(kr + x8);
+            float acc = 0.f;
+#pragma unroll
+            for (int x8 = 0; x8 < DH / 8; ++x8) {
+                const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&u[x8]);
+#pragma unroll
+                for (int e2 = 0; e2 < 4; ++e2) {
+                    const float2 f = __bfloat1622float2(h2[e2]);
+                    acc = fmaf(qs[warp][8 * x8 + 2 * e2], f.x, acc);
+                    acc = fmaf(qs[warp][8 * x8 + 2 * e2 + 1], f.y, acc);
+                }
+            }
+            const float l = scale * acc;
             if (l > mx) {
                 sm = sm * expf(mx - l) + 1.f;
                 mx = l;
@@ -1348,7 +1366,7 @@ __global__ void __launch_bounds__(128) saliency_fixup_kernel(const __nv_bfloat16
         const float M = warp_max(mx);
         const float Z = warp_sum(mx == -INFINITY ? 0.f : sm * expf(mx - M));
         float dp = 0.f;
-        for (int x = lane; x < d; x += 32) dp = fmaf(qs[warp][x], __bfloat162float(kg[(size_t)i * d + x]), dp);
+        for (int x = lane; x < DH; x += 32) dp = fmaf(qs[warp][x], __bfloat162float(kg[(size_t)i * DH + x]), dp);
         const float sii = scale * warp_sum(dp);
         if (lane == 0) sigma[row] = (i == lo) ? INFINITY : softplus_f(sii - (M + logf(Z)));
         __syncwarp();
@@ -1357,9 +1375,13 @@ __global__ void __launch_bounds__(128) saliency_fixup_kernel(const __nv_bfloat16
 
 cudaError_t launch_saliency_fixup(const Dims &s, const void *q, const void *k, const int *list, const unsigned *count,
                                   float *sigma, cudaStream_t st) {
-    saliency_fixup_kernel<<<148, 128, 0, st>>>(static_cast<const __nv_bfloat16 *>(q),
-                                                static_cast<const __nv_bfloat16 *>(k), list, count, sigma, s.H,
-                                                s.Hkv, s.N, s.d, s.w, s.scale);
+    const __nv_bfloat16 *qb = static_cast<const __nv_bfloat16 *>(q), *kb = static_cast<const __nv_bfloat16 *>(k);
+    if (s.d == 64)
+        saliency_fixup_kernel<64><<<148, 128, 0, st>>>(qb, kb, list, count, sigma, s.H, s.Hkv, s.N, s.w, s.scale);
+    else if (s.d == 128)
+        saliency_fixup_kernel<128><<<148, 128, 0, st>>>(qb, kb, list, count, sigma, s.H, s.Hkv, s.N, s.w, s.scale);
+    else
+        return cudaErrorNotSupported;
     return cudaGetLastError();
 }
 
