@@ -837,6 +837,11 @@ __global__ void mean_heads_kernel(const float *__restrict__ sigma, float *__rest
 // memory in the 128-byte-swizzled layout -> Delta S += Phi^T V and Delta z += Phi^T 1 (tcgen05,
 // Phi^T and V as MN-major operands, fp32 accumulators in TMEM).  The feature dimension is padded
 // to 128 rows of the MMA (D = 64 leaves the upper half zero).
+#ifndef STILL_LIN_PAIR
+#define STILL_LIN_PAIR 1
+#endif
+constexpr bool kLinPair = STILL_LIN_PAIR != 0;
+
 template <int DH, int DF>
 struct LinCfg {
     static constexpr int REG = 128 * 128;                 // 128 rows x 64 bf16
@@ -854,7 +859,15 @@ struct LinCfg {
     static constexpr int SMEM = WK_BYTES + NS * STAGE_BYTES + PHI_BYTES + ONES_BYTES + BAR_BYTES + 1024;
     static constexpr int THREADS = 128 + 64;
     static constexpr int PRODUCER_WARP = 4, MMA_WARP = 5;
-    static constexpr int Y_COL = 0, S_COL = 256, Z_COL = 384, TMEM_COLS = 512;
+    // d = D = 64: two CTAs per SM (the two Y buffers, S and z fit in 256 TMEM columns), so the chunk
+    // CTAs of a layer run in one wave instead of two
+    static constexpr bool PAIR = kLinPair && DH == 64 && DF == 64;
+    static constexpr int MINB = PAIR ? 2 : 1;
+    static constexpr int YB = PAIR ? DF : 128;  // columns between the two Y buffers
+    static constexpr int Y_COL = 0, S_COL = PAIR ? 2 * DF : 256, Z_COL = S_COL + (PAIR ? DH : 128),
+                         TMEM_COLS = PAIR ? 256 : 512;
+    static_assert(Z_COL + 16 <= TMEM_COLS && Y_COL + YB + DF <= S_COL, "TMEM columns");
+    static_assert(MINB * (SMEM + 1024) <= 233472, "shared memory per SM");
 };
 
 struct LinParams {
@@ -866,7 +879,7 @@ struct LinParams {
 };
 
 template <int DH, int DF>
-__global__ void __launch_bounds__(LinCfg<DH, DF>::THREADS, 1)
+__global__ void __launch_bounds__(LinCfg<DH, DF>::THREADS, LinCfg<DH, DF>::MINB)
     linear_state_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
                            const __grid_constant__ CUtensorMap map_wk, const LinParams p) {
     using Cfg = LinCfg<DH, DF>;
@@ -968,7 +981,7 @@ __global__ void __launch_bounds__(LinCfg<DH, DF>::THREADS, 1)
                 const uint32_t sK = sStage + s * Cfg::STAGE_BYTES;
                 #pragma unroll 1
                 for (int kk = 0; kk < DH / 16; ++kk)
-                    mma_ss(tmem + Cfg::Y_COL + yb * 128, kmajor_desc(sK, kk, Cfg::REG), kmajor_desc(sWk, kk, DF * 128),
+                    mma_ss(tmem + Cfg::Y_COL + yb * Cfg::YB, kmajor_desc(sK, kk, Cfg::REG), kmajor_desc(sWk, kk, DF * 128),
                            ID_Y, kk > 0);
                 mma_commit(BAR(B_YFULL + yb));
                 return true;
@@ -1014,7 +1027,7 @@ __global__ void __launch_bounds__(LinCfg<DH, DF>::THREADS, 1)
 #pragma unroll
             for (int cc = 0; cc < DF / 32; ++cc) {
                 uint32_t uu[32];
-                tmem_ld32(tmem + lane_off + Cfg::Y_COL + yb * 128 + cc * 32, uu);
+                tmem_ld32(tmem + lane_off + Cfg::Y_COL + yb * Cfg::YB + cc * 32, uu);
 #pragma unroll
                 for (int e = 0; e < 32; ++e) y[cc * 32 + e] = __uint_as_float(uu[e]);
             }
