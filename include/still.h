@@ -177,7 +177,11 @@ STILL_API still_status still_hybrid_prefill(const still_dims *dims, const void *
 /*
  * still_hybrid_prefill with its scratch in a fixed device array inside this
  * library instead of a caller workspace (no counterpart in the method: the
- * pages describe no memory management).  Same arguments, results and errors as
+ * pages describe no memory management).  It is for callers that cannot
+ * allocate device memory around the call: a serving loop that must keep its
+ * footprint fixed once it has started, code running under a memory budget that
+ * another owner enforces, or a host thread that must not call cudaMalloc (which
+ * can synchronise the device) while other work is in flight.  Same arguments, results and errors as
  * still_hybrid_prefill, minus workspace and workspace_bytes: the same argument
  * checks run first, in the same order, then the size limit below.  A call
  * allocates nothing: no device, host or pinned memory, directly or through a
