@@ -136,7 +136,8 @@ typedef struct {
     size_t vhat;   /* dtype [B,Hkv,T*k,d]      kept values                     */
     size_t S;      /* fp32  [B,Hkv,T+1,D,d]    linear state seen by chunk t    */
     size_t z;      /* fp32  [B,Hkv,T+1,D]      linear normaliser seen by chunk t */
-    size_t phik;   /* fp32  [B,Hkv,N,D]        NP-Map features of the keys     */
+    size_t phik;   /* fp32  [B,Hkv,N,D]        NP-Map features of the keys (SIMT path; bf16 on the
+                      tensor-core w = 0 path; empty on the tensor-core hybrid path) */
     size_t sig;    /* fp32  [B,H,N]            per-query-head saliency (bf16 tensor-core path) */
     size_t lse;    /* fp32  [B,H,N]            log2-sum-exp of each row's window part (same path) */
     size_t fix;    /* u32 count + int32 [B*H*N] rows whose band score is recomputed (same path) */

@@ -22,9 +22,10 @@ cudaError_t launch_saliency_fixup(const Dims &s, const void *q, const void *k, c
                                   float *sigma, cudaStream_t st);
 bool tc_saliency_supported(const Dims &s);
 bool tc_nowin_supported(const Dims &s);
-cudaError_t launch_nowin_tc(const Dims &s, const void *q, const void *k, const void *v, const void *wqt,
-                            const void *wkt, const void *st_t, const float *z, void *o, unsigned *err,
-                            cudaStream_t st);
+cudaError_t launch_nowin_phik(const Dims &s, const void *k, const void *wkt, void *phik, unsigned *err,
+                              cudaStream_t st);
+cudaError_t launch_nowin_tc(const Dims &s, const void *q, const void *v, const void *wqt, const void *st_t,
+                            const float *z, const void *phik, void *o, unsigned *err, cudaStream_t st);
 void set_merge_debug(int stall, int max_ctas);
 cudaError_t launch_saliency_tc(const Dims &s, const void *q, const void *k, float *r_kv, float *r_q, unsigned *err,
                                cudaStream_t st);
@@ -99,9 +100,12 @@ still_ws_layout ws_layout(const Dims &s) {
     off = al256(off + BK * (T + 1) * s.D * s.d * 4);
     L.z = off;
     off = al256(off + BK * (T + 1) * s.D * 4);
-    L.phik = off;  // phi(K) only on the SIMT path (the tensor-core linear state featurises in place)
-    const bool fused_lin = s.bf16 && ((tc_merge_supported(s) && tc_linear_supported(s)) || tc_nowin_supported(s));
-    off = al256(off + (fused_lin ? 0 : BK * s.N * s.D * 4));
+    // phi(K): fp32 on the SIMT path; bf16 for the intra-chunk tiles of the tensor-core w = 0 path; none
+    // on the tensor-core hybrid path (its linear state featurises the keys in place)
+    L.phik = off;
+    const bool nowin = tc_nowin_supported(s);
+    const bool fused_lin = s.bf16 && tc_merge_supported(s) && tc_linear_supported(s);
+    off = al256(off + (nowin ? BK * s.N * s.D * 2 : fused_lin ? 0 : BK * s.N * s.D * 4));
     const bool tc = s.bf16 != 0;  // per-head scores and transposed bf16 operands of the tensor-core path
     L.sig = off;
     off = al256(off + (tc ? (size_t)s.B * s.H * s.N * 4 : 0));
@@ -435,7 +439,8 @@ still_status still_hybrid_prefill(const still_dims *dims, const void *q, const v
     MergeOperands mo{q, k, v, wqt, khat, vhat, st_t, z, o, lse, sig, fix_list, fix_count};
     if (tc_nowin_supported(s)) {
         // w = 0 (no softmax branch): the inter-chunk linear state on tensor cores (NP-Map of the keys
-        // fused), then every row's intra-chunk causal tile plus phi(q)^T S_t on tensor cores
+        // fused), then phi(k) of every key once (bf16, for the intra-chunk tiles) and every row's
+        // intra-chunk causal tile plus phi(q)^T S_t on tensor cores
         {
             TimingScope ts(3, cs);
             STILL_LAUNCH(launch_w_transpose(s.Hkv, s.d, s.D, Wk, wkt, cs));
@@ -445,7 +450,8 @@ still_status still_hybrid_prefill(const still_dims *dims, const void *q, const v
         {
             TimingScope ts(4, cs);
             STILL_LAUNCH(launch_w_transpose(s.H, s.d, s.D, Wq, wqt, cs));
-            STILL_LAUNCH(launch_nowin_tc(s, q, k, v, wqt, wkt, st_t, z, o, err, cs));
+            STILL_LAUNCH(launch_nowin_phik(s, k, wkt, ws + W.phik, err, cs));
+            STILL_LAUNCH(launch_nowin_tc(s, q, v, wqt, st_t, z, ws + W.phik, o, err, cs));
         }
         if (state) {
             DecodeLayout L = decode_layout(s, state_capacity);

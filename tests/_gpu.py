@@ -70,7 +70,8 @@ def score_err(r, ref) -> float:
     r = np.asarray(r, np.float64)
     ref = np.asarray(ref, np.float64)
     both_inf = np.isinf(r) & np.isinf(ref) & (np.sign(r) == np.sign(ref))
-    err = np.where(both_inf, 0.0, np.abs(r - ref) / np.maximum(np.abs(ref), 1.0))
+    with np.errstate(invalid="ignore"):   # inf - inf on the both_inf entries, masked below
+        err = np.where(both_inf, 0.0, np.abs(r - ref) / np.maximum(np.abs(ref), 1.0))
     err = np.where(np.isnan(err), np.inf, err)
     return float(err.max()) if err.size else 0.0
 
