@@ -216,33 +216,73 @@ __global__ void __launch_bounds__(256) linear_delta_kernel(Dims s, const float *
 
 // Inclusive prefix over slots 0..T: slots 0..m are zero (no chunk has been decided for them).
 // st_t (optional): a bf16 copy of every S_t, transposed to [d, D] (K-major operand of phi(q) S_t).
-// One thread per element of (S, z) of a (b, g); the slots are read eight at a time so that the loads
-// of a batch are in flight together (the sum over slots is sequential).
-__global__ void linear_prefix_kernel(Dims s, float *__restrict__ S, float *__restrict__ z,
-                                     __nv_bfloat16 *__restrict__ st_t) {
-    const int T_ = s.T(), m = s.m();
-    const int Dd = s.D * s.d, per = Dd + s.D;
-    const size_t gid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const size_t total = (size_t)s.B * s.Hkv * per;
-    if (gid >= total) return;
-    const size_t bg = gid / per;
-    const int e = (int)(gid % per);
-    const bool isS = e < Dd;
-    float *base = isS ? &S[bg * (T_ + 1) * Dd + e] : &z[bg * (T_ + 1) * s.D + (e - Dd)];
-    const size_t stride = isS ? (size_t)Dd : (size_t)s.D;
-    const int a = isS ? e / s.d : 0, x = isS ? e % s.d : 0;
-    float run = 0.f;
-    for (int t0 = 0; t0 <= T_; t0 += 8) {
-        float v[8];
+// One CTA per (b, g) and tile of kPfxRows rows (a) x 32 columns (x) of S's [D, d] elements, two per
+// thread; z goes with the tiles of column 0.  Slots are read eight at a time (the loads of a batch in
+// flight together; the sum over slots is sequential, in slot order).  The transposed copy passes
+// through shared memory, so that its stores, like the loads, cover whole 32-byte sectors: written
+// straight from the [D, d] order, each of them was a lone 2-byte store.
+constexpr int kPfxRows = 16, kPfxSlots = 8, kPfxThreads = 256;
+constexpr int kPfxPer = kPfxRows * 32 / kPfxThreads;  // elements per thread
+static_assert(kPfxPer * kPfxThreads == kPfxRows * 32 && kPfxThreads % kPfxRows == 0, "prefix tile");
+
+__global__ void __launch_bounds__(kPfxThreads) linear_prefix_kernel(Dims s, float *__restrict__ S,
+                                                                   float *__restrict__ z,
+                                                                   __nv_bfloat16 *__restrict__ st_t) {
+    __shared__ float tile[kPfxRows][33];
+    const int T_ = s.T(), m = s.m(), D = s.D, d = s.d;
+    const size_t Dd = (size_t)D * d;
+    const int bg = blockIdx.z, a0 = blockIdx.y * kPfxRows, x0 = blockIdx.x * 32;
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+    float *Sb = S + (size_t)bg * (T_ + 1) * Dd;
+    float *zb = z + (size_t)bg * (T_ + 1) * D;
+    bool live[kPfxPer];
+    size_t off[kPfxPer];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) v[u] = (t0 + u <= T_) ? base[(size_t)(t0 + u) * stride] : 0.f;
+    for (int u = 0; u < kPfxPer; ++u) {
+        const int a = a0 + ty + 8 * u;
+        live[u] = a < D && x0 + tx < d;
+        off[u] = live[u] ? (size_t)a * d + x0 + tx : 0;
+    }
+    const bool has_z = blockIdx.x == 0 && ty == 0 && tx < kPfxRows && a0 + tx < D;
+    // transposed store of this thread: row x0 + xo (+ 32 / kPfxPer per element), column a0 + ao
+    const int ao = threadIdx.x % kPfxRows, xo = threadIdx.x / kPfxRows;
+    float run[kPfxPer], zrun = 0.f;
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int t = t0 + u;
-            if (t > T_) break;
-            if (t >= m + 1) run += v[u];
-            base[(size_t)t * stride] = run;
-            if (st_t && isS) st_t[((bg * (T_ + 1) + t) * s.d + x) * s.D + a] = __float2bfloat16_rn(run);
+    for (int u = 0; u < kPfxPer; ++u) run[u] = 0.f;
+    for (int t0 = 0; t0 <= T_; t0 += kPfxSlots) {
+        float v[kPfxSlots][kPfxPer], vz[kPfxSlots];
+#pragma unroll
+        for (int q = 0; q < kPfxSlots; ++q) {
+            const int t = t0 + q;
+            const bool add = t <= T_ && t >= m + 1;
+#pragma unroll
+            for (int u = 0; u < kPfxPer; ++u) v[q][u] = add && live[u] ? Sb[(size_t)t * Dd + off[u]] : 0.f;
+            vz[q] = add && has_z ? zb[(size_t)t * D + a0 + tx] : 0.f;
+        }
+#pragma unroll
+        for (int q = 0; q < kPfxSlots; ++q) {
+            const int t = t0 + q;
+            if (t > T_) break;  // the same for every thread of the CTA
+#pragma unroll
+            for (int u = 0; u < kPfxPer; ++u) {
+                run[u] += v[q][u];
+                if (live[u]) Sb[(size_t)t * Dd + off[u]] = run[u];
+            }
+            zrun += vz[q];
+            if (has_z) zb[(size_t)t * D + a0 + tx] = zrun;
+            if (st_t) {
+#pragma unroll
+                for (int u = 0; u < kPfxPer; ++u) tile[ty + 8 * u][tx] = run[u];
+                __syncthreads();
+#pragma unroll
+                for (int u = 0; u < kPfxPer; ++u) {
+                    const int xr = xo + u * (kPfxThreads / kPfxRows);
+                    const int x = x0 + xr, a = a0 + ao;
+                    if (x < d && a < D)
+                        st_t[((size_t)(bg * (T_ + 1) + t) * d + x) * D + a] = __float2bfloat16_rn(tile[ao][xr]);
+                }
+                __syncthreads();
+            }
         }
     }
 }
@@ -504,10 +544,9 @@ cudaError_t launch_linear_state(const Dims &s, const float *phik, const void *v,
 }
 
 cudaError_t launch_linear_prefix(const Dims &s, float *S, float *z, void *st_t, cudaStream_t st) {
-    const size_t total = (size_t)s.B * s.Hkv * ((size_t)s.D * s.d + s.D);
-    if (total == 0) return cudaSuccess;
-    linear_prefix_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(s, S, z,
-                                                                         static_cast<__nv_bfloat16 *>(st_t));
+    if ((size_t)s.B * s.Hkv * s.D * s.d == 0) return cudaSuccess;
+    const dim3 grid((unsigned)((s.d + 31) / 32), (unsigned)((s.D + kPfxRows - 1) / kPfxRows), (unsigned)(s.B * s.Hkv));
+    linear_prefix_kernel<<<grid, kPfxThreads, 0, st>>>(s, S, z, static_cast<__nv_bfloat16 *>(st_t));
     return cudaGetLastError();
 }
 
