@@ -665,11 +665,13 @@ def bench_prefill(args, name, rank, world, local, cpu_seconds):
     peak = peaks.get("bf16_tflops", 1590.0) if shape.dtype == "bf16" else None
     roofline = {
         "kernel": "merge (window phase + kept-prefix phase)" if shape.w > 0 else
-                  "no-window merge (intra-chunk tile + phi(q)^T S_t, with the W^T transpose)",
+                  "no-window merge (phi(K) once, intra-chunk tile + phi(q)^T S_t, with the W^T transpose)",
         "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
         "frac": (achieved / peak) if (achieved and peak) else None,
         "peak_source": "measured bf16_tflops" if "bf16_tflops" in peaks else "fallback 1.59 PFLOP/s",
-        "traffic": profiled_traffic(name), "traffic_unit": "DRAM bytes per step (both merge launches, ncu)",
+        "traffic": profiled_traffic(name),
+        "traffic_unit": "DRAM bytes per step (both merge launches, ncu)" if shape.w > 0 else
+                        "DRAM bytes per step (the three no-window launches, ncu)",
         "flops_per_step": mflops, "ms_per_step": merge_ms / merge_n if merge_n else None,
     }
     line = {
