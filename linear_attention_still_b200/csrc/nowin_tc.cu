@@ -156,7 +156,8 @@ __device__ __forceinline__ float row_sqnorm_sw128(const uint8_t *tile, int row) 
     return acc;
 }
 
-// Row `row` of a 128-row tile in Y's TMEM columns (this warp's lane quarter) as DF floats.
+// This thread's TMEM lane of DF fp32 columns starting at t (t carries the warp's lane quarter), as
+// floats; warp-collective.
 template <int DF>
 __device__ __forceinline__ void load_y_row(uint32_t t, float (&y)[DF]) {
 #pragma unroll
