@@ -470,7 +470,7 @@ cudaError_t launch_topk_gather(const Dims &s, const float *r, int32_t *idx, cons
     if (T_ == 0 || s.k == 0 || s.B * s.Hkv == 0) return cudaSuccess;
     const int P = pow2_ceil(s.C), Pk = pow2_ceil(s.k);
     const size_t smem = (size_t)P * 8 + (size_t)Pk * 4;
-    const int threads = 1024;
+    const int threads = P / 2 < 64 ? 64 : P / 2 > 1024 ? 1024 : P / 2;  // one compare-exchange per thread and stage
     dim3 grid(s.B * s.Hkv * T_);
     cudaError_t e;
     if (s.bf16) {

@@ -5,11 +5,22 @@
 
 namespace still {
 
+// Barrier after a bitonic compare-exchange stage of `stride` within sorts of `size` (of n entries).
+// Work item t pairs entry lo = 2t - (t & (stride-1)) with lo + stride, and a warp's items are always
+// the same aligned runs of 32 consecutive t (blockDim.x a multiple of 32), so a stage of stride <= 32
+// touches only the warp's own runs of 64 entries: between two such stages a warp barrier suffices.
+// A full barrier follows every other stage and the last one.
+__device__ __forceinline__ void bitonic_stage_sync(int size, int stride, int n) {
+    const int next = stride > 1 ? stride >> 1 : size;  // stride of the next stage
+    if (stride <= 32 && next <= 32 && !(stride == 1 && size == n)) __syncwarp();
+    else __syncthreads();
+}
+
 // Sort the n (<= P, P a power of two) scores sc[0..n) by (score desc, position asc) and leave the
 // first k positions, ascending, in pos[0..k).  keys: P u64 of shared memory; pos: Pk u32 (Pk a power
-// of two >= k).  Every thread of the block must call this.  The key packs the order-preserving score
-// bits over the complemented position, so all keys are distinct and a plain descending sort
-// realises the tie-break.
+// of two >= k).  Every thread of the block must call this, with blockDim.x a multiple of 32.  The key
+// packs the order-preserving score bits over the complemented position, so all keys are distinct and
+// a plain descending sort realises the tie-break.
 __device__ __forceinline__ void block_topk(const float *sc, int n, int k, unsigned long long *keys, uint32_t *pos,
                                            int P, int Pk) {
     for (int j = threadIdx.x; j < P; j += blockDim.x)
@@ -26,7 +37,7 @@ __device__ __forceinline__ void block_topk(const float *sc, int n, int k, unsign
                     keys[hi] = a;
                 }
             }
-            __syncthreads();
+            bitonic_stage_sync(size, stride, P);
         }
     }
     for (int t = threadIdx.x; t < Pk; t += blockDim.x)
@@ -43,7 +54,7 @@ __device__ __forceinline__ void block_topk(const float *sc, int n, int k, unsign
                     pos[hi] = a;
                 }
             }
-            __syncthreads();
+            bitonic_stage_sync(size, stride, Pk);
         }
     }
 }
