@@ -1,6 +1,7 @@
 """CPU checks of bench.py's measurement arithmetic: the softmax-set sizes behind the merge FLOP and
-exponential counts and the decode bytes per step against the oracle's own routing sets, the --keep shapes, and the
-traffic lookup from a profile summary (used only while the kernel sources match its hashes)."""
+exponential counts and the decode bytes per step against the oracle's own routing sets, the w = 0 FLOP count
+against an enumeration of its pairs, the --keep shapes, and the traffic lookup from a profile summary (used
+only while the kernel sources match its hashes) with the committed summaries' blocks."""
 import hashlib
 import os
 import sys
@@ -76,6 +77,42 @@ def test_keep_shapes():
     assert (bench.soft_sizes(s) == np.arange(s.N) + 1).all()
     assert bench.merge_flops(s) == bench.merge_flops(bench.workload_shape(type("B", (), {"workload": A.workload,
                                                                                            "keep": "all"})))
+
+
+@pytest.mark.parametrize("shape", [Shape(B=1, H=4, Hkv=2, N=300, d=64, D=64, w=0, C=128, k=0),
+                                   Shape(B=2, H=2, Hkv=1, N=77, d=32, D=16, w=0, C=32, k=0)])
+def test_nowin_flops_by_counting(shape):
+    """The w = 0 FLOP count against an explicit enumeration of the (query, key) pairs of the
+    intra-chunk causal tiles (query i sees the keys of its own chunk up to itself)."""
+    pairs = sum(1 for i in range(shape.N) for j in range(shape.N) if j // shape.C == i // shape.C and j <= i)
+    d, D = shape.d, shape.D
+    want = (shape.B * shape.H * (pairs * 2 * (D + d) + shape.N * (4 * d * D + 2 * D))
+            + shape.B * shape.Hkv * shape.N * 4 * d * D)
+    assert bench.nowin_flops(shape) == want
+
+
+def test_committed_profiles_name_known_workloads_and_sources():
+    """Every machine-readable block under profiles/ names a workload of the synthetic set, a positive
+    byte count and digests of source files that exist (whether they still match is the bench's call)."""
+    import glob
+    from linear_attention_still_b200.synth import WORKLOADS
+    seen = 0
+    for path in glob.glob(os.path.join(ROOT, "profiles", "*.md")):
+        for line in open(path):
+            if not line.startswith("    ") or line.startswith("     "):
+                continue
+            key, _, val = line.strip().partition(": ")
+            if key == "workload":
+                assert val in WORKLOADS, (path, val)
+                seen += 1
+            elif key == "traffic_bytes_per_step":
+                assert int(val) > 0, path
+            elif key == "source_sha256":
+                for item in val.split():
+                    name, _, digest = item.partition("=")
+                    assert len(digest) == 16, (path, item)
+                    assert os.path.exists(os.path.join(ROOT, "linear_attention_still_b200", "csrc", name)), (path, name)
+    assert seen >= 4
 
 
 def test_traffic_lookup_follows_source_hashes(tmp_path, monkeypatch):
